@@ -1,0 +1,351 @@
+"""Pins of the CPU oracle against facts other than itself.
+
+Each test ties an oracle function to something its own code cannot fake: a
+value the pages print, a closed form, a textbook/library routine on a
+special case, an invariant of the definition, or brute force on tiny inputs.
+Citations name the page title and section.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen import counter_hash as ch
+from gen import recipes
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _bf16(x):
+    return ch.f32_to_bf16_bits(np.asarray(x, dtype=np.float64))
+
+
+# --------------------------------------------------------------- accounting
+
+def test_kv_cache_size_worked_example():
+    """Page "长上下文：稀疏注意力 / DSA / IndexShare", "动手：算清两堵墙": the
+    printed output 0.2 / 7.0 / 53.4 GiB."""
+    rows = []
+    with open(os.path.join(GOLDEN, "kv_cache_size.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].split()
+            if not line:
+                continue
+            if line[0] == "per_token_kib":
+                per_tok = int(line[1])
+                continue
+            rows.append([int(v) for v in line[:5]] + [line[5]])
+    assert len(rows) == 3
+    for n_layers, kv_heads, head_dim, bytes_per, n_tok, expect in rows:
+        got = oracle.kv_cache_gib(n_layers, kv_heads, head_dim, n_tok, bytes_per)
+        assert f"{got:.1f}" == expect
+    one_tok = oracle.kv_cache_gib(28, 4, 128, 1, 2) * 1024 ** 3
+    assert one_tok == per_tok * 1024
+
+
+def test_pair_counts_at_1m():
+    """Same page and section: 1e12 full pairs, 82 亿 with a 8192 window
+    (1/122), 20.5 亿 with top-k 2048 (1/488), each as rounded on the page."""
+    vals = {}
+    with open(os.path.join(GOLDEN, "pair_counts.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].split()
+            if line:
+                vals[line[0]] = line[1:]
+    n = int(vals["n"][0])
+    pc = oracle.pair_counts(n, 8192, 2048)
+    for key, name in (("full", "full"), ("window", "window8192"), ("topk", "topk2048")):
+        printed, unit, sig, ratio = vals[name]
+        # the page rounds to the significant digits it prints
+        assert float(f"{pc[key] / float(unit):.{int(sig)}g}") == float(printed)
+        assert round(pc["full"] / pc[key]) == int(ratio)
+
+
+# ------------------------------------------------------------------ scores
+
+def test_index_scores_one_hot_query_reads_a_key_column():
+    """A one-hot indexer query e_c scores each key by its c-th entry; a
+    transposed operand or wrong axis fails this."""
+    rng = _rng(1)
+    k = rng.integers(-4, 5, size=(37, 16))
+    for c in (0, 5, 15):
+        q = np.zeros((1, 16))
+        q[0, c] = 1.0
+        s = oracle.index_scores(_bf16(q), _bf16(k))
+        np.testing.assert_array_equal(s[0], k[:, c])
+    q2 = np.zeros((2, 16))
+    q2[0, 3] = 2.0
+    q2[1, 7] = -1.0
+    s = oracle.index_scores(_bf16(q2), _bf16(k))
+    np.testing.assert_array_equal(s[0], 2 * k[:, 3])
+    np.testing.assert_array_equal(s[1], -k[:, 7])
+
+
+def test_index_scores_integer_inputs_are_exact():
+    rng = _rng(2)
+    q = rng.integers(-4, 5, size=(5, 128))
+    k = rng.integers(-4, 5, size=(50, 128))
+    s = oracle.index_scores(_bf16(q), _bf16(k))
+    exact = np.array([[sum(int(a) * int(b) for a, b in zip(qr, kr)) for kr in k] for qr in q])
+    np.testing.assert_array_equal(s, exact)
+    assert np.abs(s).max() <= 16 * 128
+
+
+# --------------------------------------------------------------- selection
+
+def _brute_topk(scores, k):
+    """Brute force over all k-subsets: largest total score, then the
+    lexicographically smallest sorted position tuple (the lower-position
+    tie-break).  Independent of any sort of the scores."""
+    n = len(scores)
+    kk = min(k, n)
+    best = None
+    for sub in itertools.combinations(range(n), kk):
+        key = (sum(scores[i] for i in sub), tuple(-i for i in sub))
+        if best is None or key > best[0]:
+            best = (key, sub)
+    return np.array(best[1], dtype=np.int64)
+
+
+def test_topk_matches_brute_force_on_tiny_rows():
+    rng = _rng(3)
+    for trial in range(300):
+        n = int(rng.integers(1, 10))
+        k = int(rng.integers(1, 11))
+        scores = [int(v) for v in rng.integers(-3, 4, size=n)]  # many ties
+        got = oracle.topk_select(np.array(scores, dtype=np.float64), k)
+        np.testing.assert_array_equal(got, _brute_topk(scores, k))
+
+
+def test_topk_set_dominates_its_complement():
+    """Every chosen element beats every unchosen one under (score desc,
+    position asc); the result is ascending and of size min(k, n)."""
+    rng = _rng(4)
+    for trial in range(50):
+        n = int(rng.integers(1, 3000))
+        k = int(rng.integers(1, 600))
+        s = rng.integers(-40, 41, size=n).astype(np.float64)
+        sel = oracle.topk_select(s, k)
+        assert sel.size == min(k, n)
+        assert np.all(np.diff(sel) > 0)
+        mask = np.zeros(n, bool)
+        mask[sel] = True
+        if mask.all():
+            continue
+        worst_in = min(zip(-s[mask], np.nonzero(mask)[0]), key=lambda t: (-t[0], -t[1]))
+        rest = np.nonzero(~mask)[0]
+        for u in rest[:200]:
+            # chosen (worst) must rank before u
+            assert (-worst_in[0] > s[u]) or (-worst_in[0] == s[u] and worst_in[1] < u)
+
+
+def test_topk_special_cases():
+    # all-equal scores -> the first k positions
+    np.testing.assert_array_equal(oracle.topk_select(np.zeros(100), 7), np.arange(7))
+    # fewer candidates than k -> all of them
+    np.testing.assert_array_equal(oracle.topk_select(np.array([3.0, -1.0, 2.0]), 10), [0, 1, 2])
+    # -0.0 and +0.0 compare equal (position decides)
+    np.testing.assert_array_equal(oracle.topk_select(np.array([-0.0, 0.0, -1.0]), 1), [0])
+    np.testing.assert_array_equal(oracle.topk_select(np.array([-1.0, -0.0, 0.0]), 1), [1])
+    with pytest.raises(ValueError):
+        oracle.topk_select(np.array([1.0, np.nan]), 1)
+
+
+def test_index_topk_causal_rows_take_everything_below_k():
+    """Config-1 shape on a small scale: query t has t+1 causal candidates,
+    so rows with t+1 <= k keep every earlier position."""
+    rng = _rng(5)
+    L, d, k = 300, 16, 64
+    q = _bf16(rng.integers(-4, 5, size=(1, L, d)))
+    kk = _bf16(rng.integers(-4, 5, size=(1, L, d)))
+    idx, count = oracle.index_topk(q, kk, L, 0, k)
+    for t in range(L):
+        assert count[0, t] == min(k, t + 1)
+        if t + 1 <= k:
+            np.testing.assert_array_equal(idx[0, t, : t + 1], np.arange(t + 1))
+            assert np.all(idx[0, t, t + 1:] == -1)
+        assert idx[0, t, : count[0, t]].max() <= t
+
+
+def test_index_topk_decode_lengths_per_sequence():
+    rng = _rng(6)
+    B, T, d, k = 3, 50, 8, 10
+    q = _bf16(rng.integers(-4, 5, size=(B, 1, d)))
+    kk = _bf16(rng.integers(-4, 5, size=(B, T, d)))
+    lens = np.array([50, 7, 0])
+    idx, count = oracle.index_topk(q, kk, lens, 10 ** 9, k)
+    assert list(count[:, 0]) == [10, 7, 0]
+    assert np.all(idx[2, 0] == -1)
+    np.testing.assert_array_equal(idx[1, 0, :7], np.arange(7))
+
+
+def test_planted_needles_are_retrieved():
+    """Planted needle (p, t): k_idx[p] = 8 q_idx[t].  For integer q != 0 with
+    entries in [-4, 4], 8|q|^2 >= 8|q|_1 > 4|q|_1 >= any unplanted score, so
+    only the other planted rows can outrank p, and p is in the top-k."""
+    cfg = recipes.Prefill("needle_small", seed=11, B=1, L=4096, d=64, Hq=4, Hkv=1, D=128,
+                          k=64, n_layers=1, share_every=1, n_needles=32)
+    inp = recipes.prefill_host_inputs(cfg, with_attention=False)
+    q, kk = inp["q_idx"][0], inp["k_idx"][0]
+    pairs = recipes.needle_pairs(cfg)
+    for p, t in pairs:
+        qv = oracle.bf16_bits_to_f64(q[0, t])
+        s = oracle.index_scores(q[0, t:t + 1], kk[0, : t + 1])[0]
+        assert s[p] == 8 * float(qv @ qv)
+        sel = oracle.topk_select(s, cfg.k)
+        assert p in set(sel.tolist())
+
+
+# --------------------------------------------------------------- attention
+
+def _sdpa_dense_causal(q, K, V):
+    """torch's scaled_dot_product_attention (float64, causal) with each kv
+    head repeated for its query heads: the textbook dense attention."""
+    Tq, Hq, D = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    qt = torch.from_numpy(q).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(np.repeat(K, G, axis=1)).permute(1, 0, 2)[None]
+    vt = torch.from_numpy(np.repeat(V, G, axis=1)).permute(1, 0, 2)[None]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    return o[0].permute(1, 0, 2).numpy()
+
+
+def test_sparse_attention_with_k_at_least_context_is_dense_causal():
+    """[YOIO] §1.1: with every causal key selected, sparse attention is
+    softmax(QK^T/sqrt(d))V with a causal mask."""
+    rng = _rng(7)
+    L, Hq, Hkv, D, d = 40, 4, 2, 32, 8
+    qi = _bf16(rng.integers(-4, 5, size=(1, L, d)))
+    ki = _bf16(rng.integers(-4, 5, size=(1, L, d)))
+    idx, count = oracle.index_topk(qi, ki, L, 0, L)
+    q = rng.standard_normal((1, L, Hq, D))
+    K = rng.standard_normal((1, L, Hkv, D))
+    V = rng.standard_normal((1, L, Hkv, D))
+    out, _ = oracle.sparse_attention(q, K, V, idx, count)
+    ref = _sdpa_dense_causal(q[0], K[0], V[0])
+    np.testing.assert_allclose(out[0], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_output_is_convex_combination_of_selected_rows():
+    rng = _rng(8)
+    Hq, Hkv, D, n = 8, 2, 16, 33
+    q = rng.standard_normal((Hq, D)) * 3
+    K = rng.standard_normal((n, Hkv, D))
+    V = rng.standard_normal((n, Hkv, D))
+    o, lse = oracle.attention_over_rows(q, K, V)
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        assert np.all(o[h] <= V[:, g].max(axis=0) + 1e-12)
+        assert np.all(o[h] >= V[:, g].min(axis=0) - 1e-12)
+    # weights sum to one: V = 1 everywhere gives 1
+    o1, _ = oracle.attention_over_rows(q, K, np.ones_like(V))
+    np.testing.assert_allclose(o1, 1.0, rtol=0, atol=1e-12)
+    # one constant V row repeated gives that row
+    row = rng.standard_normal((Hkv, D))
+    oc, _ = oracle.attention_over_rows(q, K, np.broadcast_to(row, V.shape).copy())
+    for h in range(Hq):
+        np.testing.assert_allclose(oc[h], row[h // G], atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = _rng(9)
+    D = 8
+    K = rng.standard_normal((5, 1, D))
+    V = rng.standard_normal((5, 1, D))
+    # q = 0: uniform weights -> mean of the selected V rows; lse = log n
+    o, lse = oracle.attention_over_rows(np.zeros((2, D)), K, V)
+    np.testing.assert_allclose(o, np.broadcast_to(V[:, 0].mean(axis=0), (2, D)), atol=1e-12)
+    np.testing.assert_allclose(lse, math.log(5), atol=1e-12)
+    # two rows whose scaled scores differ by delta: weight = logistic(delta)
+    q = np.zeros((1, D))
+    q[0, 0] = 1.0
+    K2 = np.zeros((2, 1, D))
+    K2[0, 0, 0] = 2.0
+    V2 = np.zeros((2, 1, D))
+    V2[0, 0, :] = 1.0
+    o2, _ = oracle.attention_over_rows(q, K2, V2, scale=1.5)
+    w = 1.0 / (1.0 + math.exp(-3.0))
+    np.testing.assert_allclose(o2[0], w, atol=1e-12)
+    # empty selection
+    o3, l3 = oracle.attention_over_rows(np.ones((3, D)), np.zeros((0, 1, D)), np.zeros((0, 1, D)))
+    assert np.all(o3 == 0) and np.all(np.isneginf(l3))
+
+
+def test_attention_is_invariant_to_the_order_of_selected_rows():
+    rng = _rng(10)
+    q = rng.standard_normal((4, 16))
+    K = rng.standard_normal((20, 2, 16))
+    V = rng.standard_normal((20, 2, 16))
+    perm = rng.permutation(20)
+    o1, l1 = oracle.attention_over_rows(q, K, V)
+    o2, l2 = oracle.attention_over_rows(q, K[perm], V[perm])
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+def test_lse_is_log_sum_exp_of_scaled_scores():
+    from scipy.special import logsumexp
+    rng = _rng(12)
+    q = rng.standard_normal((2, 32))
+    K = rng.standard_normal((9, 1, 32))
+    V = rng.standard_normal((9, 1, 32))
+    _, lse = oracle.attention_over_rows(q, K, V, scale=0.3)
+    for h in range(2):
+        np.testing.assert_allclose(lse[h], logsumexp(0.3 * K[:, 0] @ q[h]), atol=1e-12)
+
+
+# -------------------------------------------------------------------- gist
+
+def test_gist_equal_scores_take_the_first_chunks():
+    n_chunks, cl, kc = 50, 16, 8
+    gk = np.zeros((n_chunks, 4))
+    for p in (0, 5, 16):
+        rows, chunks = oracle.gist_route_unfold(np.ones(4), gk, cl, kc, p)
+        np.testing.assert_array_equal(chunks, np.arange(kc))
+        assert rows.size == kc * (cl + 1) + p
+        np.testing.assert_array_equal(rows[: kc * 17], np.arange(kc * 17))
+        np.testing.assert_array_equal(rows[kc * 17:], n_chunks * 17 + np.arange(p))
+
+
+def test_gist_hand_worked_example():
+    """4 chunks of 2 raw tokens + 1 gist (stride 3); gist scores
+    [1, 5, -2, 5] with k = 2 keep chunks 1 and 3; rows are written out by
+    hand from the interleaved layout, then the 2-token partial chunk."""
+    gk = np.array([[1.0], [5.0], [-2.0], [5.0]])
+    rows, chunks = oracle.gist_route_unfold(np.array([1.0]), gk, chunk_len=2, k_chunks=2, partial_len=2)
+    assert chunks.tolist() == [1, 3]
+    assert rows.tolist() == [3, 4, 5, 9, 10, 11, 12, 13]
+    # more chunks requested than exist -> all chunks
+    rows, chunks = oracle.gist_route_unfold(np.array([1.0]), gk, chunk_len=2, k_chunks=9, partial_len=0)
+    assert chunks.tolist() == [0, 1, 2, 3]
+    assert rows.tolist() == list(range(12))
+
+
+# ----------------------------------------------------------------- sharing
+
+def test_layer_owners_every_four_layers():
+    """[LC] "DSA 与 IndexShare": every 4 layers share one indexer result;
+    [IC] §五: 75% of indexer computation removed -> 1 full layer in 4."""
+    owners = oracle.layer_owners(28, share_every=4)
+    assert owners == [4 * (l // 4) for l in range(28)]
+    full = sum(1 for l, o in enumerate(owners) if o == l)
+    assert full == 7 and 1 - full / 28 == 0.75
+
+
+def test_layer_owners_pattern():
+    """[IC] §二: a shared layer reuses the nearest full layer before it."""
+    assert oracle.layer_owners(6, pattern="FSSFSF") == [0, 0, 0, 3, 3, 5]
+    assert oracle.layer_owners(1, pattern="F") == [0]
+    for bad in ("SFF", "FX", "FF"):
+        with pytest.raises(ValueError):
+            oracle.layer_owners(3, pattern=bad)
