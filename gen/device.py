@@ -53,3 +53,17 @@ def fill_normal(t, seed: int, tid: int, start: int = 0):
     if rc != 0:
         raise RuntimeError(f"sagen_fill_normal_bf16 failed: cuda error {rc}")
     return t
+
+
+def build(verbose: bool = False) -> str:
+    """Compile gen/device.cu into gen/libsagen.so (nvcc, sm_100a)."""
+    import subprocess
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
+           "-Xcompiler", "-fPIC", "-shared", os.path.join(_HERE, "device.cu"), "-o", LIB_PATH]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed for gen/device.cu:\n{r.stdout}\n{r.stderr}")
+    return LIB_PATH

@@ -1,0 +1,234 @@
+/*
+ * sa.h -- C ABI of libsa.so: indexer-routed token-sparse attention with one
+ * routing index shared by a group of layers, plus gist-chunk routing.
+ *
+ * Sources (page title, section):
+ *   [YOIO] "你只索引一次：当AI学会'过目不忘'的遗忘艺术", a write-up of
+ *          "You Only Index Once: Cross-Layer Sparse Attention with Shared Routing".
+ *   [LC]   "长上下文：稀疏注意力 / DSA / IndexShare".
+ *   [SSA]  "斯坦福大学研究团队如何让AI'聪明地遗忘'" (Simplified Sparse Attention).
+ *   [IC]   "清华提出IndexCache技术：让AI大模型处理长文本时速度提升80%".
+ *   [GSA]  "Forget, Then Recall: Learnable Compression and Selective Unfolding
+ *          via Gist Sparse Attention".
+ *
+ * Conventions shared by every call
+ *   - Tensors are caller-owned DEVICE pointers, contiguous, row-major.
+ *     bf16 tensors are passed as void* and hold bfloat16 bit patterns.
+ *   - Every call validates its arguments on the host first and returns an
+ *     error WITHOUT launching anything if they are bad.  Valid calls enqueue
+ *     their kernels on `stream` and return at once: no host synchronisation,
+ *     no device allocation, no host allocation on the hot path.
+ *   - Kernel launch failures return SA_ERR_CUDA; sa_last_error() gives the
+ *     detail.  Faults inside a kernel surface later, on the stream, as for
+ *     any CUDA kernel.
+ *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
+ *   - No kernel of this library waits on another CTA, kernel or device.
+ *   - Calls are not thread-safe with respect to one shared workspace;
+ *     calls on different streams need different workspaces.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* sa_stream_t;
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size   */
+  SA_ERR_UNSUPPORTED = 2,   /* valid but outside this build's shape support  */
+  SA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned    */
+  SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed          */
+  SA_ERR_TIMEOUT = 5,       /* reserved: no kernel in this library waits     */
+  SA_ERR_STALE_INDEX = 6    /* shared layer read before its full layer ran   */
+} sa_status;
+
+/* Limits of this build. */
+#define SA_MAX_K 4096           /* largest top-k                                */
+#define SA_HEAD_DIM 128         /* attention head_dim supported                 */
+#define SA_WS_ALIGN 256         /* workspace pointers must be 256-byte aligned  */
+
+/* Static, never-null description of a status code. */
+const char* sa_status_string(sa_status s);
+/* Detail of the last failing call made by this host thread ("" if none). */
+const char* sa_last_error(void);
+/* Library ABI version (major * 100 + minor). */
+int sa_version(void);
+
+/* ------------------------------------------------------------------------
+ * Indexer scoring + per-query top-k.
+ *
+ * [LC] "DSA 与 IndexShare": a light indexer scores every history token and
+ * each query keeps only its top-k tokens; [YOIO] §1.3 (token-level top-k)
+ * and §2.3 (the indexer's output is each query's top-k token indices).
+ *
+ * Score of query t against cached token j: s = q_idx[b,t,:] . k_idx[b,j,:],
+ * one indexer head, accumulated in fp32 (exact for integer-valued bf16
+ * inputs with |s| < 2^24).  Candidates of query t are the positions
+ *     0 <= j <= q_pos0 + t   and   j < len_b,
+ * where len_b = kv_len[b] if kv_len is given, else Tk.  (Causality is
+ * inclusive: a token may select itself.  For decode pass Tq = 1 and
+ * q_pos0 = len - 1, or any q_pos0 >= len - 1.)
+ *
+ * Selection keeps k_eff = min(k, n_candidates) positions: the largest
+ * scores, equal scores ordered by LOWER position first.  Row (b,t) of
+ * idx_out holds them in ASCENDING position order followed by -1 padding;
+ * count_out[b,t] = k_eff.  score_out, if given, holds each kept position's
+ * fp32 score in the same slots (NaN-free padding value: -inf).
+ *
+ *   q_idx      [B, Tq, d]      bf16
+ *   k_idx      [B, Tk_max, d]  bf16   (rows >= len_b are never read)
+ *   kv_len     [B] int32 or NULL      (each 0 <= kv_len[b] <= Tk; values
+ *                                      outside are clamped on the device)
+ *   idx_out    [B, Tq, k] int32;  count_out [B, Tq] int32
+ *   score_out  [B, Tq, k] fp32 or NULL
+ *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes,
+ *              SA_WS_ALIGN-aligned; contents need no initialisation and are
+ *              clobbered.
+ * Supported: d in {64, 128}; 1 <= k <= SA_MAX_K; Tq >= 1; 0 <= Tk <= Tk_max.
+ * Scores must be free of NaN (NaN inputs give an unspecified selection).
+ * ---------------------------------------------------------------------- */
+size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k);
+sa_status sa_index_score_topk(const void* q_idx, const void* k_idx,
+                              int B, int Tq, int Tk, int Tk_max, int d, int k,
+                              int q_pos0, const int32_t* kv_len,
+                              int32_t* idx_out, int32_t* count_out, float* score_out,
+                              void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Gathered sparse attention, prefill (one call per layer).
+ *
+ * [YOIO] §1.1: Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V; §2.3: each
+ * layer's selector fetches from its KV cache only the rows named by the
+ * shared index and attends over them.  [LC] "DSA 与 IndexShare": core
+ * attention drops from O(L^2) to O(Lk).
+ *
+ * For token t of sequence b and query head h (kv head g = h / (Hq/Hkv)):
+ *   z_i = scale * q[b,t,h,:] . k_cache[b, j_i, g, :],  j_i = idx[b,t,i], i < count[b,t]
+ *   out[b,t,h,:] = sum_i softmax(z)_i v_cache[b, j_i, g, :]
+ *   lse[b,t,h]   = ln sum_i exp(z_i)          (natural log; -inf if count = 0)
+ * An empty row (count = 0) gives out = 0.  scale <= 0 selects 1/sqrt(D).
+ * bf16 inputs, fp32 accumulation and softmax, bf16 output.
+ *
+ *   q        [B, T, Hq, D] bf16
+ *   k_cache  [B, Tk_max, Hkv, D] bf16;  v_cache same shape
+ *   idx      [B, T, k] int32 (each used entry in [0, Tk_max); entries past
+ *            count are ignored); count [B, T] int32 (clamped to [0, k])
+ *   out      [B, T, Hq, D] bf16;  lse [B, T, Hq] fp32 or NULL
+ * Supported: D = 128; Hq % Hkv == 0; 1 <= Hq/Hkv <= 16; k <= SA_MAX_K.
+ * Out-of-range used indices are a caller error (the kernel does not check).
+ * ---------------------------------------------------------------------- */
+sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* idx, const int32_t* count,
+                                 int B, int T, int Tk_max, int Hq, int Hkv, int D, int k,
+                                 float scale, void* out, float* lse, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Gathered sparse attention, decode (one query token per sequence).
+ *
+ * Same arithmetic as the prefill call.  The selected rows are split across
+ * CTAs; each CTA loads every selected K/V row of its kv head once for all
+ * Hq/Hkv query heads of that group, and the partial results are merged with
+ * the log-sum-exp rule ([SSA] §六: split-K partial attention over a compact
+ * index list, KV shared by a GQA group loaded once, then a log-sum-exp merge).
+ *
+ *   q        [B, Hq, D] bf16
+ *   idx      [B, k] int32 (row stride k); count [B] int32 (clamped to [0, k])
+ *   out      [B, Hq, D] bf16;  lse [B, Hq] fp32 or NULL
+ *   ws       >= sa_sparse_attn_decode_workspace(...) bytes, SA_WS_ALIGN-aligned
+ * Supported: as for prefill.
+ * ---------------------------------------------------------------------- */
+size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k);
+sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* idx, const int32_t* count,
+                                int B, int Tk_max, int Hq, int Hkv, int D, int k,
+                                float scale, void* out, float* lse,
+                                void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Gist-chunk routing with selective unfolding (decode).
+ *
+ * [SSA] §二/§三 and [GSA] 2.1-2.2: the sequence is cut into chunks of
+ * chunk_len raw tokens, each followed by one gist token; the query is
+ * scored by dot product against every chunk's gist key, the top k_chunks
+ * chunks are kept, and each kept chunk is unfolded into its raw tokens plus
+ * its own gist.  Unkept gists are left out ([SSA] §八 and [GSA] 4 find this
+ * "selected gists + selected raw" context best).  The current, incomplete
+ * chunk (partial_len[b] tokens) is always appended.
+ *
+ * Cache layout assumed for the row ids: chunk c occupies rows
+ * (chunk_len+1)*c .. (chunk_len+1)*c + chunk_len - 1 (raw) and
+ * (chunk_len+1)*c + chunk_len (gist); the partial chunk starts at
+ * (chunk_len+1)*n_chunks.
+ *
+ * Chunk selection follows the top-k rule above (equal scores: lower chunk).
+ * rows_out row b: for each kept chunk in ascending order its chunk_len+1
+ * rows, then the partial rows, then -1 padding; count_out[b] = number of
+ * rows.  chunks_out (optional) holds the kept chunk ids, ascending, -1 padded.
+ *
+ *   q_route     [B, d] bf16;   gist_key [B, n_chunks, d] bf16
+ *   partial_len [B] int32 (clamped on the device to [0, chunk_len])
+ *   rows_out    [B, k_chunks*(chunk_len+1) + chunk_len] int32
+ *   count_out   [B] int32;    chunks_out [B, k_chunks] int32 or NULL
+ * Supported: d in {64, 128}; 1 <= k_chunks <= SA_MAX_K; 1 <= chunk_len <= 256.
+ * ---------------------------------------------------------------------- */
+size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks);
+sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key,
+                               int B, int n_chunks, int chunk_len, int d, int k_chunks,
+                               const int32_t* partial_len,
+                               int32_t* rows_out, int32_t* count_out, int32_t* chunks_out,
+                               void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Shared index cache (host object; its device buffers are caller-owned).
+ *
+ * [IC] §二 and §六: layers are "full" (run their own indexer and store the
+ * result) or "shared" (reuse the index of the nearest full layer before
+ * them); one temporary buffer holds the current index and is overwritten at
+ * the next full layer, so sharing adds no memory.  [LC] "DSA 与 IndexShare"
+ * and [YOIO] §2.2: the expensive top-k is done once and reused by every layer
+ * of the group.
+ *
+ * create: pattern is a string of 'F'/'S' of length n_layers starting with
+ *   'F', or NULL to use share_every (layer l is full iff l % share_every == 0).
+ *   idx_buf [B, Tq, k] int32 and count_buf [B, Tq] int32 are device buffers
+ *   that must outlive the cache.
+ * begin_step: starts a new forward step; every shared layer becomes stale
+ *   until its full layer writes again.
+ * update: full layers only; runs sa_index_score_topk into the buffers.
+ * mark_written: records that the caller itself filled the buffers for full
+ *   layer `layer` (e.g. with sa_index_score_topk on its own stream).
+ * get: returns the buffers for `layer` and the version of the write it reads.
+ *   SA_ERR_STALE_INDEX if, in this step, the layer's full layer has not
+ *   written or a later full layer has overwritten the buffer.
+ * The object is not thread-safe.
+ * ---------------------------------------------------------------------- */
+typedef struct sa_index_cache sa_index_cache;
+sa_status sa_index_cache_create(int n_layers, const char* pattern, int share_every,
+                                int B, int Tq, int k, int32_t* idx_buf, int32_t* count_buf,
+                                sa_index_cache** out);
+void sa_index_cache_destroy(sa_index_cache* cache);
+/* 1 if `layer` is a full layer, 0 if shared, -1 if out of range or cache NULL. */
+int sa_index_cache_is_full(const sa_index_cache* cache, int layer);
+/* The full layer whose index `layer` reads, or -1 if out of range. */
+int sa_index_cache_owner(const sa_index_cache* cache, int layer);
+sa_status sa_index_cache_begin_step(sa_index_cache* cache);
+sa_status sa_index_cache_update(sa_index_cache* cache, int layer, const void* q_idx,
+                                const void* k_idx, int Tk, int Tk_max, int d, int q_pos0,
+                                const int32_t* kv_len, void* ws, size_t ws_bytes,
+                                sa_stream_t stream);
+sa_status sa_index_cache_mark_written(sa_index_cache* cache, int layer);
+sa_status sa_index_cache_get(sa_index_cache* cache, int layer, const int32_t** idx,
+                             const int32_t** count, uint64_t* version);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SA_H_ */

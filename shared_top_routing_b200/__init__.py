@@ -1,0 +1,25 @@
+"""B200-native indexer-routed token-sparse attention with a cross-layer shared index.
+
+The product is the C ABI ``libsa.so`` (declared in ``include/sa.h``, sources
+in ``csrc/``).  ``shared_top_routing_b200.sa`` is its Python binding; it only
+marshals arguments.  Build with ``python -m shared_top_routing_b200.build``.
+"""
+from .sa import (  # noqa: F401
+    IndexCache,
+    SAError,
+    lib,
+    sa_gist_route_unfold,
+    sa_index_score_topk,
+    sa_sparse_attn_decode,
+    sa_sparse_attn_prefill,
+)
+
+__all__ = [
+    "IndexCache",
+    "SAError",
+    "lib",
+    "sa_gist_route_unfold",
+    "sa_index_score_topk",
+    "sa_sparse_attn_decode",
+    "sa_sparse_attn_prefill",
+]

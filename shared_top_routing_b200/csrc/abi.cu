@@ -1,0 +1,403 @@
+// C ABI of libsa.so: host-side validation, workspace sizing, dispatch and
+// the shared index cache.  Declarations and contracts are in include/sa.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/sa.h"
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sa_status fail(sa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+sa_status ok() {
+  g_last_error.clear();
+  return SA_OK;
+}
+
+sa_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(SA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sa_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return SA_OK;
+  if (ws == nullptr) return fail(SA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
+  if (!aligned(ws, SA_WS_ALIGN)) return fail(SA_ERR_WORKSPACE, "workspace is not %d-byte aligned", SA_WS_ALIGN);
+  if (ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace has %zu bytes, %zu are needed", ws_bytes, need);
+  return SA_OK;
+}
+
+cudaStream_t as_cuda(sa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+sa_status validate_index(const void* q_idx, const void* k_idx, int B, int Tq, int Tk, int Tk_max,
+                         int d, int k, const int32_t* idx_out, const int32_t* count_out) {
+  if (B < 0 || Tq < 1 || Tk < 0 || Tk_max < 0 || Tk > Tk_max)
+    return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d Tq=%d Tk=%d Tk_max=%d (need B>=0, Tq>=1, 0<=Tk<=Tk_max)",
+                B, Tq, Tk, Tk_max);
+  if (k < 1) return fail(SA_ERR_INVALID_ARG, "k=%d must be >= 1", k);
+  if (k > SA_MAX_K) return fail(SA_ERR_UNSUPPORTED, "k=%d exceeds SA_MAX_K=%d", k, SA_MAX_K);
+  if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "d=%d unsupported (64 or 128)", d);
+  if ((long long)Tk_max * d > (1ll << 40))
+    return fail(SA_ERR_UNSUPPORTED, "Tk_max=%d too large", Tk_max);
+  if (B == 0) return SA_OK;
+  if (!q_idx || !k_idx || !idx_out || !count_out)
+    return fail(SA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16))
+    return fail(SA_ERR_INVALID_ARG, "q_idx and k_idx must be 16-byte aligned");
+  if (!aligned(idx_out, 4) || !aligned(count_out, 4))
+    return fail(SA_ERR_INVALID_ARG, "idx_out and count_out must be 4-byte aligned");
+  return SA_OK;
+}
+
+bool use_candidates(int Tk_max) { return Tk_max > sa::kDirectMaxCand; }
+
+sa_status validate_attn(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                        const int32_t* count, int B, int T, int Tk_max, int Hq, int Hkv, int D,
+                        int k, const void* out) {
+  if (B < 0 || T < 0 || Tk_max < 1 || Hq < 1 || Hkv < 1 || k < 1)
+    return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d T=%d Tk_max=%d Hq=%d Hkv=%d k=%d", B, T,
+                Tk_max, Hq, Hkv, k);
+  if (D != SA_HEAD_DIM) return fail(SA_ERR_UNSUPPORTED, "D=%d unsupported (only %d)", D, SA_HEAD_DIM);
+  if (Hq % Hkv != 0) return fail(SA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (Hq / Hkv > 16) return fail(SA_ERR_UNSUPPORTED, "Hq/Hkv=%d > 16 unsupported", Hq / Hkv);
+  if (k > (1 << 20)) return fail(SA_ERR_UNSUPPORTED, "k=%d too large", k);
+  if (B == 0 || T == 0) return SA_OK;
+  if (!q || !kc || !vc || !idx || !count || !out) return fail(SA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(out, 16))
+    return fail(SA_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
+  if (!aligned(idx, 4) || !aligned(count, 4)) return fail(SA_ERR_INVALID_ARG, "idx/count misaligned");
+  return SA_OK;
+}
+
+}  // namespace
+
+namespace sa {
+
+cudaError_t ensure_dynamic_smem(const void* func, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(func, dev);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
+}
+
+}  // namespace sa
+
+// =============================================================== C ABI
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG: invalid argument";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED: shape not supported by this build";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA: CUDA runtime or launch failure";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT: reserved";
+    case SA_ERR_STALE_INDEX: return "SA_ERR_STALE_INDEX: shared layer read before its full layer wrote";
+  }
+  return "unknown sa_status";
+}
+
+const char* sa_last_error(void) { return g_last_error.c_str(); }
+
+int sa_version(void) { return 100; }
+
+// ------------------------------------------------------------- indexer
+
+size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
+  (void)d;
+  (void)k;
+  if (B <= 0 || Tq <= 0 || Tk_max < 0) return 0;
+  if (Tq == 1) return sa::row_workspace_bytes(B, Tk_max, use_candidates(Tk_max));
+  int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
+  return sa::row_workspace_bytes(B * rows, Tk_max, false);
+}
+
+sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int Tq, int Tk,
+                              int Tk_max, int d, int k, int q_pos0, const int32_t* kv_len,
+                              int32_t* idx_out, int32_t* count_out, float* score_out, void* ws,
+                              size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = validate_index(q_idx, k_idx, B, Tq, Tk, Tk_max, d, k, idx_out, count_out);
+  if (st != SA_OK) return st;
+  if (B == 0) return ok();
+  const size_t need = sa_index_score_topk_workspace(B, Tq, Tk_max, d, k);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
+  cudaStream_t cs = as_cuda(stream);
+  const uint16_t* q = static_cast<const uint16_t*>(q_idx);
+  const uint16_t* km = static_cast<const uint16_t*>(k_idx);
+  sa::FinishOut out;
+  out.idx = idx_out;
+  out.count = count_out;
+  out.score = score_out;
+  cudaError_t e;
+  if (Tq == 1) {
+    const bool cand = use_candidates(Tk_max);
+    sa::RowWorkspace w;
+    sa::carve_row_workspace(ws, B, Tk_max, cand, &w);
+    if (cand) {
+      // histogram and candidate counters start at zero (adjacent in the workspace)
+      size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
+      if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
+    }
+    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, cand, cs)) != cudaSuccess)
+      return cuda_fail(e, "score_decode launch");
+    if (cand && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
+      return cuda_fail(e, "collect launch");
+    if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, cand, out, cs)) != cudaSuccess)
+      return cuda_fail(e, "finish launch");
+    return ok();
+  }
+  const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
+  sa::RowWorkspace w;
+  sa::carve_row_workspace(ws, B * rows, Tk_max, false, &w);
+  for (int t0 = 0; t0 < Tq; t0 += rows) {
+    const int nr = (Tq - t0 < rows) ? Tq - t0 : rows;
+    if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, w, cs)) != cudaSuccess)
+      return cuda_fail(e, "score_prefill launch");
+    if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, false, out, cs)) != cudaSuccess)
+      return cuda_fail(e, "finish launch");
+  }
+  return ok();
+}
+
+// ----------------------------------------------------------- attention
+
+sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* idx, const int32_t* count, int B, int T, int Tk_max,
+                                 int Hq, int Hkv, int D, int k, float scale, void* out, float* lse,
+                                 sa_stream_t stream) {
+  sa_status st = validate_attn(q, k_cache, v_cache, idx, count, B, T, Tk_max, Hq, Hkv, D, k, out);
+  if (st != SA_OK) return st;
+  if (B == 0 || T == 0) return ok();
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaError_t e = sa::launch_attn_prefill(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k_cache),
+      static_cast<const uint16_t*>(v_cache), idx, count, B, T, Tk_max, Hq, Hkv, k, sc,
+      static_cast<uint16_t*>(out), lse, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
+  return ok();
+}
+
+size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || k <= 0) return 0;
+  return sa::decode_attn_workspace_bytes(B, Hq, Hkv, D, k);
+}
+
+sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,
+                                int Hkv, int D, int k, float scale, void* out, float* lse, void* ws,
+                                size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = validate_attn(q, k_cache, v_cache, idx, count, B, 1, Tk_max, Hq, Hkv, D, k, out);
+  if (st != SA_OK) return st;
+  if (B == 0) return ok();
+  if ((st = check_ws(ws, ws_bytes, sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k))) != SA_OK)
+    return st;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaError_t e = sa::launch_attn_decode(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k_cache),
+      static_cast<const uint16_t*>(v_cache), idx, count, B, Tk_max, Hq, Hkv, k, sc,
+      static_cast<uint16_t*>(out), lse, ws, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode launch");
+  return ok();
+}
+
+// ---------------------------------------------------------------- gist
+
+size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) {
+  (void)d;
+  (void)k_chunks;
+  if (B <= 0 || n_chunks < 0) return 0;
+  return sa::row_workspace_bytes(B, n_chunks, use_candidates(n_chunks));
+}
+
+sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B, int n_chunks,
+                               int chunk_len, int d, int k_chunks, const int32_t* partial_len,
+                               int32_t* rows_out, int32_t* count_out, int32_t* chunks_out, void* ws,
+                               size_t ws_bytes, sa_stream_t stream) {
+  if (B < 0 || n_chunks < 0) return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d n_chunks=%d", B, n_chunks);
+  if (chunk_len < 1 || chunk_len > 256)
+    return fail(SA_ERR_UNSUPPORTED, "chunk_len=%d unsupported (1..256)", chunk_len);
+  if (k_chunks < 1) return fail(SA_ERR_INVALID_ARG, "k_chunks=%d must be >= 1", k_chunks);
+  if (k_chunks > SA_MAX_K) return fail(SA_ERR_UNSUPPORTED, "k_chunks=%d exceeds SA_MAX_K", k_chunks);
+  if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "d=%d unsupported (64 or 128)", d);
+  if ((long long)(n_chunks + 1) * (chunk_len + 1) > 0x7FFFFFFFll)
+    return fail(SA_ERR_UNSUPPORTED, "row ids overflow int32");
+  if (B == 0) return ok();
+  if (!q_route || !gist_key || !rows_out || !count_out) return fail(SA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned(q_route, 16) || !aligned(gist_key, 16))
+    return fail(SA_ERR_INVALID_ARG, "q_route and gist_key must be 16-byte aligned");
+  sa_status st = check_ws(ws, ws_bytes, sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks));
+  if (st != SA_OK) return st;
+  cudaStream_t cs = as_cuda(stream);
+  const bool cand = use_candidates(n_chunks);
+  sa::RowWorkspace w;
+  sa::carve_row_workspace(ws, B, n_chunks, cand, &w);
+  cudaError_t e;
+  if (cand) {
+    size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
+    if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
+  }
+  const int q_pos0 = n_chunks - 1;  // every complete chunk is a candidate
+  if ((e = sa::launch_score_decode(static_cast<const uint16_t*>(q_route),
+                                   static_cast<const uint16_t*>(gist_key), B, d, n_chunks, n_chunks,
+                                   q_pos0, nullptr, w, cand, cs)) != cudaSuccess)
+    return cuda_fail(e, "gist score launch");
+  if (cand && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
+    return cuda_fail(e, "gist collect launch");
+  sa::FinishOut out;
+  out.count = count_out;
+  out.rows = rows_out;
+  out.rows_stride = k_chunks * (chunk_len + 1) + chunk_len;
+  out.chunk_len = chunk_len;
+  out.n_chunks = n_chunks;
+  out.partial_len = partial_len;
+  out.chunks = chunks_out;
+  if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, cand, out, cs)) != cudaSuccess)
+    return cuda_fail(e, "gist finish launch");
+  return ok();
+}
+
+}  // extern "C"
+
+// ========================================================= index cache
+
+struct sa_index_cache {
+  int n_layers = 0;
+  std::vector<int> owner;
+  int B = 0, Tq = 0, k = 0;
+  int32_t* idx_buf = nullptr;
+  int32_t* count_buf = nullptr;
+  uint64_t version = 0;      // bumped at every write
+  int last_writer = -1;      // full layer whose index the buffer holds in this step
+  uint64_t last_version = 0;
+};
+
+extern "C" {
+
+sa_status sa_index_cache_create(int n_layers, const char* pattern, int share_every, int B, int Tq,
+                                int k, int32_t* idx_buf, int32_t* count_buf, sa_index_cache** out) {
+  if (out == nullptr) return fail(SA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (n_layers < 1) return fail(SA_ERR_INVALID_ARG, "n_layers=%d must be >= 1", n_layers);
+  if (B < 0 || Tq < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "bad sizes B=%d Tq=%d k=%d", B, Tq, k);
+  if (k > SA_MAX_K) return fail(SA_ERR_UNSUPPORTED, "k=%d exceeds SA_MAX_K", k);
+  if (B > 0 && (!idx_buf || !count_buf)) return fail(SA_ERR_INVALID_ARG, "NULL index buffer");
+  std::string pat;
+  if (pattern != nullptr) {
+    pat = pattern;
+    if ((int)pat.size() != n_layers)
+      return fail(SA_ERR_INVALID_ARG, "pattern length %zu != n_layers %d", pat.size(), n_layers);
+  } else {
+    if (share_every < 1) return fail(SA_ERR_INVALID_ARG, "share_every=%d must be >= 1", share_every);
+    for (int l = 0; l < n_layers; ++l) pat.push_back(l % share_every == 0 ? 'F' : 'S');
+  }
+  if (pat[0] != 'F') return fail(SA_ERR_INVALID_ARG, "layer 0 must be a full layer ('F')");
+  auto* c = new sa_index_cache();
+  c->n_layers = n_layers;
+  int cur = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (pat[l] == 'F') cur = l;
+    else if (pat[l] != 'S') {
+      delete c;
+      return fail(SA_ERR_INVALID_ARG, "pattern character %d is '%c' (need 'F' or 'S')", l, pat[l]);
+    }
+    c->owner.push_back(cur);
+  }
+  c->B = B;
+  c->Tq = Tq;
+  c->k = k;
+  c->idx_buf = idx_buf;
+  c->count_buf = count_buf;
+  *out = c;
+  return ok();
+}
+
+void sa_index_cache_destroy(sa_index_cache* cache) { delete cache; }
+
+int sa_index_cache_is_full(const sa_index_cache* c, int layer) {
+  if (!c || layer < 0 || layer >= c->n_layers) return -1;
+  return c->owner[layer] == layer ? 1 : 0;
+}
+
+int sa_index_cache_owner(const sa_index_cache* c, int layer) {
+  if (!c || layer < 0 || layer >= c->n_layers) return -1;
+  return c->owner[layer];
+}
+
+sa_status sa_index_cache_begin_step(sa_index_cache* c) {
+  if (!c) return fail(SA_ERR_INVALID_ARG, "cache is NULL");
+  c->last_writer = -1;
+  return ok();
+}
+
+sa_status sa_index_cache_mark_written(sa_index_cache* c, int layer) {
+  if (!c) return fail(SA_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(SA_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (c->owner[layer] != layer) return fail(SA_ERR_INVALID_ARG, "layer %d is a shared layer", layer);
+  c->version += 1;
+  c->last_writer = layer;
+  c->last_version = c->version;
+  return ok();
+}
+
+sa_status sa_index_cache_update(sa_index_cache* c, int layer, const void* q_idx, const void* k_idx,
+                                int Tk, int Tk_max, int d, int q_pos0, const int32_t* kv_len,
+                                void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!c) return fail(SA_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(SA_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (c->owner[layer] != layer)
+    return fail(SA_ERR_INVALID_ARG, "layer %d is a shared layer; it reuses layer %d's index", layer,
+                c->owner[layer]);
+  sa_status st = sa_index_score_topk(q_idx, k_idx, c->B, c->Tq, Tk, Tk_max, d, c->k, q_pos0, kv_len,
+                                     c->idx_buf, c->count_buf, nullptr, ws, ws_bytes, stream);
+  if (st != SA_OK) return st;
+  return sa_index_cache_mark_written(c, layer);
+}
+
+sa_status sa_index_cache_get(sa_index_cache* c, int layer, const int32_t** idx,
+                             const int32_t** count, uint64_t* version) {
+  if (!c) return fail(SA_ERR_INVALID_ARG, "cache is NULL");
+  if (layer < 0 || layer >= c->n_layers) return fail(SA_ERR_INVALID_ARG, "layer %d out of range", layer);
+  const int o = c->owner[layer];
+  if (c->last_writer != o)
+    return fail(SA_ERR_STALE_INDEX, "layer %d reads full layer %d's index, but the buffer holds %s", layer,
+                o, c->last_writer < 0 ? "no index of this step" : "a later full layer's index");
+  if (idx) *idx = c->idx_buf;
+  if (count) *count = c->count_buf;
+  if (version) *version = c->last_version;
+  return ok();
+}
+
+}  // extern "C"

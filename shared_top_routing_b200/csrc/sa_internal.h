@@ -1,0 +1,72 @@
+// Internal launchers of libsa.so (host side).  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sa {
+
+// Rows of at most this many candidates are selected by one CTA reading the
+// whole row ("direct" mode); longer rows go through histogram + collect.
+constexpr int kDirectMaxCand = 16384;
+
+struct RowWorkspace {
+  uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys
+  long long ld = 0;
+  uint32_t* hist = nullptr;      // [rows][kHistBins]
+  uint32_t* cand_cnt = nullptr;  // [rows]
+  uint32_t* cand_key = nullptr;  // [rows][kCandCap]
+  uint32_t* cand_pos = nullptr;  // [rows][kCandCap]
+};
+
+// Finish-kernel output description.
+struct FinishOut {
+  int32_t* idx = nullptr;        // [B, Tq, k]
+  int32_t* count = nullptr;      // [B, Tq]
+  float* score = nullptr;        // [B, Tq, k] or null
+  // gist unfolding (when rows != null)
+  int32_t* rows = nullptr;       // [B, rows_stride]
+  int rows_stride = 0;
+  int chunk_len = 0;
+  int n_chunks = 0;
+  const int32_t* partial_len = nullptr;
+  int32_t* chunks = nullptr;     // [B, k] or null
+};
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_dynamic_smem(const void* func, size_t bytes);
+
+size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates);
+void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, RowWorkspace* out);
+
+// One query per batch row (decode / gist): keys[b][j] = key(q[b].k[b][j]) for
+// j < n_b = clamp(min(q_pos0+1, len_b), 0), plus the first-digit histogram.
+cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, int d, int Tk_max,
+                                int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
+                                bool with_hist, cudaStream_t st);
+cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
+                           const RowWorkspace& w, cudaStream_t st);
+// Exact selection per row.  rows = B * rows_per_batch; row r is query
+// t0 + r % rows_per_batch of batch r / rows_per_batch.
+cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+                          const int32_t* kv_len, int k, const RowWorkspace& w, bool candidates,
+                          const FinishOut& out, cudaStream_t st);
+// Prefill scoring of queries [t0, t0+rows) into the key slab.
+cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,
+                                 int Tk_max, int Tk, int q_pos0, const int32_t* kv_len, int t0,
+                                 int rows, const RowWorkspace& w, cudaStream_t st);
+int prefill_rows_per_launch(int B, int Tq, int Tk_max);
+
+// Attention.
+size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
+cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                               const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,
+                               int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,
+                               cudaStream_t st);
+cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                                const int32_t* idx, const int32_t* count, int B, int T, int Tk_max,
+                                int Hq, int Hkv, int k, float scale, uint16_t* out, float* lse,
+                                cudaStream_t st);
+
+}  // namespace sa

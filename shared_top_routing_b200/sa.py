@@ -1,0 +1,325 @@
+"""Python binding of libsa.so: argument marshalling only.
+
+Every function here passes raw device pointers, sizes and the current CUDA
+stream to the C ABI declared in ``include/sa.h``; every step of the path runs
+in the library's CUDA kernels.  torch is used for device memory (outputs and
+workspaces) and streams.  If ``libsa.so`` is missing the import of a compute
+function fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+SA_OK = 0
+SA_ERR_INVALID_ARG = 1
+SA_ERR_UNSUPPORTED = 2
+SA_ERR_WORKSPACE = 3
+SA_ERR_CUDA = 4
+SA_ERR_TIMEOUT = 5
+SA_ERR_STALE_INDEX = 6
+SA_MAX_K = 4096
+SA_WS_ALIGN = 256
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/sa.h
+SIGNATURES = {
+    "sa_status_string": (ctypes.c_char_p, [_I]),
+    "sa_last_error": (ctypes.c_char_p, []),
+    "sa_version": (_I, []),
+    "sa_index_score_topk_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "sa_index_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "sa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
+    "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
+    "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
+    "sa_index_cache_destroy": (None, [_P]),
+    "sa_index_cache_is_full": (_I, [_P, _I]),
+    "sa_index_cache_owner": (_I, [_P, _I]),
+    "sa_index_cache_begin_step": (_I, [_P]),
+    "sa_index_cache_update": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "sa_index_cache_mark_written": (_I, [_P, _I]),
+    "sa_index_cache_get": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                ctypes.POINTER(ctypes.c_uint64)]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, func: str, detail: str):
+        super().__init__(f"{func} -> {status_string(status)}: {detail}")
+        self.status = status
+
+
+def lib():
+    """The loaded libsa.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"libsa.so not found at {LIB_PATH}; build it with "
+                        "`python -m shared_top_routing_b200.build` (no fallback exists)")
+                L = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().sa_status_string(s).decode()
+
+
+def last_error() -> str:
+    return lib().sa_last_error().decode()
+
+
+def _check(status: int, func: str):
+    if status != SA_OK:
+        raise SAError(status, func, last_error())
+
+
+# ------------------------------------------------------------ torch plumbing
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype_size, device=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.element_size() != dtype_size:
+        raise ValueError(f"{name} must have {dtype_size}-byte elements")
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device, key: str = "", stream=None):
+    """A cached device workspace of at least ``nbytes`` (256-byte aligned)."""
+    torch = _torch()
+    if nbytes <= 0:
+        return None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    k = (str(device), s.cuda_stream, key)
+    buf = _ws_cache.get(k)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[k] = buf
+    return buf
+
+
+# --------------------------------------------------------------- the calls
+
+def sa_index_score_topk(q_idx, k_idx, k: int, Tk: int | None = None, q_pos0: int | None = None,
+                        kv_len=None, idx_out=None, count_out=None, with_scores: bool = False,
+                        ws=None, stream=None):
+    """Indexer scores + per-query top-k (see sa.h).
+
+    q_idx [B, Tq, d] or [B, d] (decode) bf16; k_idx [B, Tk_max, d] bf16.
+    Tk defaults to Tk_max; q_pos0 defaults to Tk - Tq (prefill whose queries
+    are the last Tq cached tokens; for decode Tk - 1).
+    Returns (idx [B, Tq, k] int32, count [B, Tq] int32[, score [B, Tq, k] fp32]).
+    """
+    torch = _torch()
+    decode_shape = q_idx.dim() == 2
+    q3 = q_idx.unsqueeze(1) if decode_shape else q_idx
+    B, Tq, d = q3.shape
+    Tk_max = k_idx.shape[1]
+    Tk = Tk_max if Tk is None else Tk
+    q_pos0 = Tk - Tq if q_pos0 is None else q_pos0
+    _need(q3, "q_idx", 2)
+    _need(k_idx, "k_idx", 2)
+    dev = q3.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Tq, k), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((B, Tq), dtype=torch.int32, device=dev)
+    score = torch.empty((B, Tq, k), dtype=torch.float32, device=dev) if with_scores else None
+    need = lib().sa_index_score_topk_workspace(B, Tq, Tk_max, d, k)
+    if ws is None:
+        ws = workspace(need, dev, "index", stream)
+    st = lib().sa_index_score_topk(_ptr(q3), _ptr(k_idx), B, Tq, Tk, Tk_max, d, k, q_pos0,
+                                   _ptr(kv_len), _ptr(idx_out), _ptr(count_out), _ptr(score),
+                                   _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "sa_index_score_topk")
+    if decode_shape:
+        idx_v, cnt_v = idx_out.view(B, k), count_out.view(B)
+        return (idx_v, cnt_v, score.view(B, k)) if with_scores else (idx_v, cnt_v)
+    return (idx_out, count_out, score) if with_scores else (idx_out, count_out)
+
+
+def sa_sparse_attn_prefill(q, k_cache, v_cache, idx, count, scale: float = 0.0, out=None,
+                           with_lse: bool = False, stream=None):
+    """q [B, T, Hq, D]; k_cache/v_cache [B, Tk_max, Hkv, D]; idx [B, T, k]; count [B, T]."""
+    torch = _torch()
+    B, T, Hq, D = q.shape
+    _, Tk_max, Hkv, _ = k_cache.shape
+    k = idx.shape[-1]
+    for t, n, sz in ((q, "q", 2), (k_cache, "k_cache", 2), (v_cache, "v_cache", 2),
+                     (idx, "idx", 4), (count, "count", 4)):
+        _need(t, n, sz)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    st = lib().sa_sparse_attn_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx), _ptr(count),
+                                      B, T, Tk_max, Hq, Hkv, D, k, scale, _ptr(out), _ptr(lse),
+                                      _stream(stream))
+    _check(st, "sa_sparse_attn_prefill")
+    return (out, lse) if with_lse else out
+
+
+def sa_sparse_attn_decode(q, k_cache, v_cache, idx, count, scale: float = 0.0, out=None,
+                          with_lse: bool = False, ws=None, stream=None):
+    """q [B, Hq, D]; k_cache/v_cache [B, Tk_max, Hkv, D]; idx [B, k]; count [B]."""
+    torch = _torch()
+    B, Hq, D = q.shape
+    _, Tk_max, Hkv, _ = k_cache.shape
+    k = idx.shape[-1]
+    for t, n, sz in ((q, "q", 2), (k_cache, "k_cache", 2), (v_cache, "v_cache", 2),
+                     (idx, "idx", 4), (count, "count", 4)):
+        _need(t, n, sz)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    need = lib().sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k)
+    if ws is None:
+        ws = workspace(need, q.device, "attn_decode", stream)
+    st = lib().sa_sparse_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx), _ptr(count),
+                                     B, Tk_max, Hq, Hkv, D, k, scale, _ptr(out), _ptr(lse),
+                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "sa_sparse_attn_decode")
+    return (out, lse) if with_lse else out
+
+
+def sa_gist_route_unfold(q_route, gist_key, chunk_len: int, k_chunks: int, partial_len,
+                         rows_out=None, count_out=None, with_chunks: bool = False, ws=None,
+                         stream=None):
+    """q_route [B, d]; gist_key [B, n_chunks, d]; partial_len [B] int32 (device).
+    Returns (rows [B, k_chunks*(chunk_len+1)+chunk_len], count [B][, chunks [B, k_chunks]])."""
+    torch = _torch()
+    B, d = q_route.shape
+    n_chunks = gist_key.shape[1]
+    _need(q_route, "q_route", 2)
+    _need(gist_key, "gist_key", 2)
+    _need(partial_len, "partial_len", 4)
+    dev = q_route.device
+    stride = k_chunks * (chunk_len + 1) + chunk_len
+    if rows_out is None:
+        rows_out = torch.empty((B, stride), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    chunks = torch.empty((B, k_chunks), dtype=torch.int32, device=dev) if with_chunks else None
+    need = lib().sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks)
+    if ws is None:
+        ws = workspace(need, dev, "gist", stream)
+    st = lib().sa_gist_route_unfold(_ptr(q_route), _ptr(gist_key), B, n_chunks, chunk_len, d,
+                                    k_chunks, _ptr(partial_len), _ptr(rows_out), _ptr(count_out),
+                                    _ptr(chunks), _ptr(ws), 0 if ws is None else ws.numel(),
+                                    _stream(stream))
+    _check(st, "sa_gist_route_unfold")
+    return (rows_out, count_out, chunks) if with_chunks else (rows_out, count_out)
+
+
+class IndexCache:
+    """Shared index cache: full layers run the indexer into one buffer, shared
+    layers read it (see sa_index_cache_* in sa.h).  The buffers are device
+    tensors owned by this object (or passed in)."""
+
+    def __init__(self, n_layers: int, B: int, Tq: int, k: int, pattern: str | None = None,
+                 share_every: int = 4, device=None, idx_buf=None, count_buf=None):
+        self._h = None
+        self.idx_buf = idx_buf
+        self.count_buf = count_buf
+        if B > 0 and (idx_buf is None or count_buf is None):
+            torch = _torch()
+            self.idx_buf = torch.empty((B, Tq, k), dtype=torch.int32, device=device)
+            self.count_buf = torch.empty((B, Tq), dtype=torch.int32, device=device)
+        h = ctypes.c_void_p()
+        pat = pattern.encode() if pattern is not None else None
+        st = lib().sa_index_cache_create(n_layers, pat, share_every, B, Tq, k,
+                                         _ptr(self.idx_buf), _ptr(self.count_buf), ctypes.byref(h))
+        _check(st, "sa_index_cache_create")
+        self._h = h
+        self.n_layers, self.B, self.Tq, self.k = n_layers, B, Tq, k
+
+    def close(self):
+        if self._h is not None and self._h.value:
+            lib().sa_index_cache_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def is_full(self, layer: int) -> int:
+        return lib().sa_index_cache_is_full(self._h, layer)
+
+    def owner(self, layer: int) -> int:
+        return lib().sa_index_cache_owner(self._h, layer)
+
+    def begin_step(self):
+        _check(lib().sa_index_cache_begin_step(self._h), "sa_index_cache_begin_step")
+
+    def mark_written(self, layer: int):
+        _check(lib().sa_index_cache_mark_written(self._h, layer), "sa_index_cache_mark_written")
+
+    def update(self, layer: int, q_idx, k_idx, Tk: int | None = None, q_pos0: int | None = None,
+               kv_len=None, ws=None, stream=None):
+        q3 = q_idx.unsqueeze(1) if q_idx.dim() == 2 else q_idx
+        B, Tq, d = q3.shape
+        Tk_max = k_idx.shape[1]
+        Tk = Tk_max if Tk is None else Tk
+        q_pos0 = Tk - Tq if q_pos0 is None else q_pos0
+        need = lib().sa_index_score_topk_workspace(B, Tq, Tk_max, d, self.k)
+        if ws is None:
+            ws = workspace(need, q3.device, "index", stream)
+        st = lib().sa_index_cache_update(self._h, layer, _ptr(q3), _ptr(k_idx), Tk, Tk_max, d, q_pos0,
+                                         _ptr(kv_len), _ptr(ws), 0 if ws is None else ws.numel(),
+                                         _stream(stream))
+        _check(st, "sa_index_cache_update")
+
+    def get(self, layer: int):
+        """(idx_ptr, count_ptr, version) for `layer`; raises SAError on a stale read."""
+        ip, cp, ver = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_uint64()
+        st = lib().sa_index_cache_get(self._h, layer, ctypes.byref(ip), ctypes.byref(cp),
+                                      ctypes.byref(ver))
+        _check(st, "sa_index_cache_get")
+        return ip.value, cp.value, ver.value
+
+    def get_tensors(self, layer: int):
+        """The index buffers for `layer` (checked against the C object)."""
+        ip, cp, ver = self.get(layer)
+        assert ip == self.idx_buf.data_ptr() and cp == self.count_buf.data_ptr()
+        return self.idx_buf, self.count_buf, ver

@@ -1,0 +1,189 @@
+"""C ABI checks that need no GPU: the library loads and exports every symbol
+include/sa.h declares, host-side validation rejects bad arguments before
+any CUDA call, and the shared index cache follows its full/shared rules.
+
+Only calls that fail validation, size queries and the host-only index cache
+are made here; nothing computes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from shared_top_routing_b200 import sa as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sa.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("sa_index_score_topk", "sa_sparse_attn_prefill", "sa_sparse_attn_decode",
+                 "sa_gist_route_unfold", "sa_index_cache_create", "sa_index_cache_get",
+                 "sa_index_cache_update"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(S.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding knows every declared entry point
+    assert set(_declared()) <= set(S.SIGNATURES)
+
+
+def test_status_strings_and_version():
+    assert S.lib().sa_version() == 100
+    for code in range(7):
+        assert S.status_string(code)
+    assert "unknown" in S.status_string(99)
+
+
+FAKE = ctypes.c_void_p(0x100000)   # never dereferenced: every call below fails validation
+
+
+def _topk(**kw):
+    a = dict(q=FAKE, k=FAKE, B=1, Tq=1, Tk=10, Tk_max=10, d=64, kk=8, q_pos0=9, kv_len=None,
+             idx=FAKE, cnt=FAKE, score=None, ws=None, ws_bytes=0)
+    a.update(kw)
+    return S.lib().sa_index_score_topk(a["q"], a["k"], a["B"], a["Tq"], a["Tk"], a["Tk_max"], a["d"],
+                                       a["kk"], a["q_pos0"], a["kv_len"], a["idx"], a["cnt"],
+                                       a["score"], a["ws"], a["ws_bytes"], None)
+
+
+def test_index_topk_validation():
+    assert _topk(Tk=11) == S.SA_ERR_INVALID_ARG                 # Tk > Tk_max
+    assert _topk(B=-1) == S.SA_ERR_INVALID_ARG
+    assert _topk(Tq=0) == S.SA_ERR_INVALID_ARG
+    assert _topk(kk=0) == S.SA_ERR_INVALID_ARG
+    assert _topk(kk=S.SA_MAX_K + 1) == S.SA_ERR_UNSUPPORTED
+    assert _topk(d=96) == S.SA_ERR_UNSUPPORTED
+    assert _topk(q=None) == S.SA_ERR_INVALID_ARG
+    assert _topk(k=ctypes.c_void_p(0x100008)) == S.SA_ERR_INVALID_ARG  # misaligned
+    assert "aligned" in S.last_error()
+    assert _topk(ws=None, ws_bytes=0) == S.SA_ERR_WORKSPACE
+    assert _topk(ws=ctypes.c_void_p(0x100010), ws_bytes=1 << 30) == S.SA_ERR_WORKSPACE
+    assert _topk(ws=FAKE, ws_bytes=16) == S.SA_ERR_WORKSPACE
+    assert "bytes" in S.last_error()
+    assert _topk(B=0) == S.SA_OK                                # nothing to do, no launch
+
+
+def test_workspace_sizes():
+    L = S.lib()
+    small = L.sa_index_score_topk_workspace(8, 1, 4096, 128, 2048)
+    big = L.sa_index_score_topk_workspace(8, 1, 32832, 128, 2048)
+    assert 0 < small < big
+    assert big % 256 == 0
+    assert L.sa_index_score_topk_workspace(0, 1, 100, 64, 8) == 0
+    # prefill slab of at most 512 MiB
+    assert L.sa_index_score_topk_workspace(1, 65536, 65536, 64, 2048) <= (512 << 20) + (1 << 20)
+    assert L.sa_sparse_attn_decode_workspace(8, 32, 8, 128, 2048) > 0
+    assert L.sa_gist_route_unfold_workspace(4, 8192, 128, 64) > 0
+
+
+def test_attention_validation():
+    L = S.lib()
+
+    def pre(**kw):
+        a = dict(B=1, T=4, Tk_max=16, Hq=8, Hkv=2, D=128, k=8, q=FAKE, out=FAKE)
+        a.update(kw)
+        return L.sa_sparse_attn_prefill(a["q"], FAKE, FAKE, FAKE, FAKE, a["B"], a["T"], a["Tk_max"],
+                                        a["Hq"], a["Hkv"], a["D"], a["k"], 0.0, a["out"], None, None)
+
+    assert pre(D=64) == S.SA_ERR_UNSUPPORTED
+    assert pre(Hq=6, Hkv=4) == S.SA_ERR_INVALID_ARG
+    assert pre(Hq=64, Hkv=2) == S.SA_ERR_UNSUPPORTED           # G = 32 > 16
+    assert pre(q=None) == S.SA_ERR_INVALID_ARG
+    assert pre(out=ctypes.c_void_p(0x100002)) == S.SA_ERR_INVALID_ARG
+    assert pre(T=0) == S.SA_OK
+    st = L.sa_sparse_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 8, 2, 128, 8, 0.0, FAKE, None,
+                                 None, 0, None)
+    assert st == S.SA_ERR_WORKSPACE
+
+
+def test_gist_validation():
+    L = S.lib()
+
+    def gist(**kw):
+        a = dict(B=1, n=64, cl=16, d=128, kc=4, ws=None, wsb=0)
+        a.update(kw)
+        return L.sa_gist_route_unfold(FAKE, FAKE, a["B"], a["n"], a["cl"], a["d"], a["kc"], FAKE, FAKE,
+                                      FAKE, None, a["ws"], a["wsb"], None)
+
+    assert gist(cl=0) == S.SA_ERR_UNSUPPORTED
+    assert gist(kc=0) == S.SA_ERR_INVALID_ARG
+    assert gist(d=32) == S.SA_ERR_UNSUPPORTED
+    assert gist(n=-1) == S.SA_ERR_INVALID_ARG
+    assert gist() == S.SA_ERR_WORKSPACE
+    assert gist(B=0) == S.SA_OK
+
+
+def _cache(n_layers, pattern=None, share_every=4):
+    h = ctypes.c_void_p()
+    pat = pattern.encode() if pattern else None
+    st = S.lib().sa_index_cache_create(n_layers, pat, share_every, 2, 1, 16, FAKE, FAKE, ctypes.byref(h))
+    return st, h
+
+
+def test_index_cache_schedule_and_staleness():
+    """Page "清华提出IndexCache技术…", §二 and §六: full layers write one
+    buffer, shared layers read the nearest preceding full layer's index."""
+    L = S.lib()
+    st, h = _cache(8, share_every=4)
+    assert st == S.SA_OK
+    try:
+        assert [L.sa_index_cache_is_full(h, l) for l in range(8)] == [1, 0, 0, 0, 1, 0, 0, 0]
+        assert [L.sa_index_cache_owner(h, l) for l in range(8)] == [0, 0, 0, 0, 4, 4, 4, 4]
+        assert L.sa_index_cache_is_full(h, 8) == -1
+        ip, cp, ver = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_uint64()
+        get = lambda l: L.sa_index_cache_get(h, l, ctypes.byref(ip), ctypes.byref(cp), ctypes.byref(ver))
+        assert L.sa_index_cache_begin_step(h) == S.SA_OK
+        assert get(1) == S.SA_ERR_STALE_INDEX                   # layer 0 has not run yet
+        assert L.sa_index_cache_mark_written(h, 1) == S.SA_ERR_INVALID_ARG  # shared layer
+        assert L.sa_index_cache_mark_written(h, 0) == S.SA_OK
+        versions = []
+        for l in range(4):
+            assert get(l) == S.SA_OK
+            assert ip.value == FAKE.value and cp.value == FAKE.value
+            versions.append(ver.value)
+        assert len(set(versions)) == 1                           # one index for the group
+        assert get(4) == S.SA_ERR_STALE_INDEX
+        assert L.sa_index_cache_mark_written(h, 4) == S.SA_OK
+        assert get(5) == S.SA_OK and ver.value == versions[0] + 1
+        assert get(2) == S.SA_ERR_STALE_INDEX                   # overwritten by layer 4
+        assert L.sa_index_cache_begin_step(h) == S.SA_OK
+        assert get(4) == S.SA_ERR_STALE_INDEX                   # new step
+        # update on a shared layer is refused before any launch
+        st = L.sa_index_cache_update(h, 3, FAKE, FAKE, 10, 10, 64, 9, None, None, 0, None)
+        assert st == S.SA_ERR_INVALID_ARG
+    finally:
+        L.sa_index_cache_destroy(h)
+
+
+def test_index_cache_pattern_rules():
+    L = S.lib()
+    st, h = _cache(6, pattern="FSSFSF")
+    assert st == S.SA_OK
+    assert [L.sa_index_cache_owner(h, l) for l in range(6)] == [0, 0, 0, 3, 3, 5]
+    L.sa_index_cache_destroy(h)
+    for bad in ("SFFFFF", "FSXFFF", "FSSFSFF"):   # starts shared, bad letter, wrong length
+        st, h = _cache(6, pattern=bad)
+        assert st == S.SA_ERR_INVALID_ARG
+    st, h = _cache(4, pattern=None, share_every=0)
+    assert st == S.SA_ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    assert S.lib().sa_index_cache_create(4, None, 4, 1, 1, S.SA_MAX_K + 1, FAKE, FAKE,
+                                         ctypes.byref(h)) == S.SA_ERR_UNSUPPORTED
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(S, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(S, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        S.lib()

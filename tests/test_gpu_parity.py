@@ -1,0 +1,320 @@
+"""GPU parity against the CPU oracle at sizes the oracle finishes in seconds.
+
+Indices and counts must match bit for bit (integer-valued indexer inputs make
+every fp32 score exact); attention outputs must be within max-abs 2e-2 and
+mean-abs 2e-3 of the fp64 oracle.  Sizes span several tiles and ragged
+tails; edge cases cover empty rows, k >= candidates, all-equal and signed-zero
+scores, heavy ties and the candidate-overflow fallback."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import shared_top_routing_b200 as sa
+from gen import counter_hash as ch
+from tests.gpu_util import assert_close_attn, assert_lse_close, dev, i32, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _ints(seed, tid, shape, lo=-4, hi=4):
+    return ch.int_bf16(seed, tid, count=int(np.prod(shape)), lo=lo, hi=hi).reshape(shape)
+
+
+def _normals(seed, tid, shape):
+    return ch.normal_bf16(seed, tid, count=int(np.prod(shape))).reshape(shape)
+
+
+# ---------------------------------------------------------------- decode top-k
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("k,lens,Tk_max", [
+    (256, [3000, 1, 0, 257], 3000),            # direct mode, ragged, empty row, n = k + 1
+    (7, [9999, 5000, 7, 6], 10007),            # n <= k rows
+    (2048, [16385, 30000, 2047, 40000], 40000),  # candidate mode, several collect CTAs
+    (4096, [50000, 4096, 4097, 100], 50000),   # largest k
+    (1, [12345, 1, 20000], 20000),
+])
+def test_decode_topk_matches_oracle(d, k, lens, Tk_max):
+    B = len(lens)
+    seed = 1000 + d + k
+    q = _ints(seed, 1, (B, d))
+    kk = _ints(seed, 2, (B, Tk_max, d))
+    idx, cnt, sc = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=max(lens), q_pos0=10 ** 9,
+                                          kv_len=i32(lens), with_scores=True)
+    ridx, rcnt = oracle.index_topk(q[:, None, :], kk, np.array(lens), 10 ** 9, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0])
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
+    # scores of the chosen positions
+    sc = sc.cpu().numpy()
+    for b in range(B):
+        n = rcnt[b, 0]
+        if n:
+            full = oracle.index_scores(q[b:b + 1], kk[b, ridx[b, 0, :n]])[0]
+            np.testing.assert_array_equal(sc[b, :n], full)
+        assert np.all(np.isneginf(sc[b, n:]))
+
+
+@pytest.mark.parametrize("n", [5000, 60000])
+def test_decode_topk_all_equal_and_signed_zero_scores(n):
+    """q = 0 makes every score +0 or -0 (the sign of each key's entries):
+    all compare equal, so the first k positions win.  n = 60000 overflows the
+    candidate list and takes the full-row path."""
+    d, k = 128, 2048
+    q = np.zeros((1, d), np.uint16)
+    kk = _ints(77, 3, (1, n, d), lo=-4, hi=0)      # many all-negative rows -> -0 scores
+    kk[0, ::3] = ch.f32_to_bf16_bits(-np.ones(d))  # certainly -0
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k)
+    torch.cuda.synchronize()
+    assert cnt.item() == k
+    np.testing.assert_array_equal(idx.cpu().numpy()[0], np.arange(k))
+
+
+def test_decode_topk_heavy_ties():
+    """A one-hot query gives only 9 distinct scores: huge tie groups at the
+    threshold, decided by position."""
+    d, n, k = 64, 40000, 3000
+    q = np.zeros((2, d))
+    q[0, 5] = 1.0
+    q[1, 0] = -2.0
+    qb = ch.f32_to_bf16_bits(q)
+    kk = _ints(78, 4, (2, n, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(qb), to_dev(kk), k)
+    ridx, rcnt = oracle.index_topk(qb[:, None, :], kk, n, n - 1, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0])
+
+
+def test_decode_topk_q_pos0_limits_candidates():
+    d, n, k = 64, 1000, 100
+    q = _ints(79, 1, (1, d))
+    kk = _ints(79, 2, (1, n, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=n, q_pos0=49)
+    torch.cuda.synchronize()
+    assert cnt.item() == 50
+    np.testing.assert_array_equal(idx.cpu().numpy()[0, :50], np.arange(50))
+    assert np.all(idx.cpu().numpy()[0, 50:] == -1)
+
+
+# --------------------------------------------------------------- prefill top-k
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,L,k,Tk,q_pos0", [
+    (1, 1, 16, 1, 0),
+    (2, 77, 16, 77, 0),
+    (1, 300, 64, 300, 0),
+    (1, 1000, 256, 1000, 0),
+    (2, 130, 40, 530, 400),     # chunked prefill: queries are the last 130 of 530 tokens
+])
+def test_prefill_topk_matches_oracle(d, B, L, k, Tk, q_pos0):
+    seed = 2000 + L + d
+    q = _ints(seed, 1, (B, L, d))
+    kk = _ints(seed, 2, (B, Tk, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0)
+    ridx, rcnt = oracle.index_topk(q, kk, Tk, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
+def test_prefill_topk_real_valued_scores():
+    """Non-integer bf16 inputs: the GPU's fp32 tile sums may differ from the
+    fp64 oracle in the last bits, so compare sets via the oracle's scores:
+    every chosen position must be valid and the chosen score sum must equal
+    the oracle's within fp32 rounding."""
+    B, L, d, k = 1, 400, 64, 50
+    q = _normals(81, 1, (B, L, d))
+    kk = _normals(81, 2, (B, L, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k)
+    ridx, rcnt = oracle.index_topk(q, kk, L, 0, k)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    s = oracle.index_scores(q[0], kk[0])
+    for t in range(L):
+        n = rcnt[0, t]
+        got = idx[0, t, :n]
+        assert np.all(np.diff(got) > 0) and got.max() <= t
+        np.testing.assert_allclose(s[t, got].sum(), s[t, ridx[0, t, :n]].sum(), rtol=1e-5, atol=1e-3)
+
+
+# ----------------------------------------------------------------- attention
+
+def _random_index(rng, B, Tk_max, k, counts):
+    idx = np.full((B, k), -1, np.int32)
+    for b, c in enumerate(counts):
+        idx[b, :c] = np.sort(rng.choice(Tk_max, size=c, replace=False))
+    return idx
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (28, 4), (8, 1), (16, 16)])
+@pytest.mark.parametrize("k,counts", [(2048, [2048, 1000, 0, 1]), (100, [100, 33, 64, 7]),
+                                      (1104, [1104, 1090, 1, 1089])])
+def test_decode_attention_matches_oracle(Hq, Hkv, k, counts):
+    rng = np.random.default_rng(Hq * 1000 + k)
+    B, Tk_max, D = len(counts), 3000, 128
+    q = _normals(3000 + Hq, 1, (B, Hq, D))
+    K = _normals(3000 + Hq, 2, (B, Tk_max, Hkv, D))
+    V = _normals(3000 + Hq, 3, (B, Tk_max, Hkv, D))
+    idx = _random_index(rng, B, Tk_max, k, counts)
+    out, lse = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), i32(idx), i32(counts),
+                                        with_lse=True)
+    Kr = [K[b, idx[b, :c]] for b, c in enumerate(counts)]
+    Vr = [V[b, idx[b, :c]] for b, c in enumerate(counts)]
+    ref, rlse = oracle.sparse_attention_decode(q, Kr, Vr)
+    torch.cuda.synchronize()
+    assert_close_attn(out.float().cpu().numpy(), ref, "decode attention")
+    assert_lse_close(lse.cpu().numpy(), rlse, "decode lse")
+
+
+def test_decode_attention_scale_and_repeat_calls():
+    """Explicit scale; two calls in a row reuse the workspace (tickets reset)."""
+    B, Hq, Hkv, D, Tk_max, k = 2, 8, 2, 128, 500, 300
+    q = _normals(31, 1, (B, Hq, D))
+    K = _normals(31, 2, (B, Tk_max, Hkv, D))
+    V = _normals(31, 3, (B, Tk_max, Hkv, D))
+    idx = _random_index(np.random.default_rng(5), B, Tk_max, k, [300, 250])
+    ref, _ = oracle.sparse_attention_decode(q, [K[0, idx[0]], K[1, idx[1, :250]]],
+                                            [V[0, idx[0]], V[1, idx[1, :250]]], scale=0.05)
+    for _ in range(2):
+        out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), i32(idx), i32([300, 250]),
+                                       scale=0.05)
+        torch.cuda.synchronize()
+        assert_close_attn(out.float().cpu().numpy(), ref, "decode attention, scale 0.05")
+
+
+@pytest.mark.parametrize("Hq,Hkv,k", [(8, 1, 256), (16, 4, 64), (12, 4, 100)])
+def test_prefill_attention_matches_oracle(Hq, Hkv, k):
+    B, L, d, D = 2, 300, 64, 128
+    seed = 4000 + Hq + k
+    qi = _ints(seed, 1, (B, L, d))
+    ki = _ints(seed, 2, (B, L, d))
+    q = _normals(seed, 3, (B, L, Hq, D))
+    K = _normals(seed, 4, (B, L, Hkv, D))
+    V = _normals(seed, 5, (B, L, Hkv, D))
+    idx, cnt = sa.sa_index_score_topk(to_dev(qi), to_dev(ki), k)
+    out, lse = sa.sa_sparse_attn_prefill(to_dev(q), to_dev(K), to_dev(V), idx, cnt, with_lse=True)
+    ridx, rcnt = oracle.index_topk(qi, ki, L, 0, k)
+    ref, rlse = oracle.sparse_attention(q, K, V, ridx, rcnt)
+    torch.cuda.synchronize()
+    assert_close_attn(out.float().cpu().numpy(), ref, "prefill attention")
+    assert_lse_close(lse.cpu().numpy(), rlse, "prefill lse")
+
+
+def test_prefill_attention_with_k_at_least_context_is_dense_causal():
+    """k >= L selects every causal key: the output is dense causal attention
+    (checked against torch's SDPA on the CPU in fp64)."""
+    B, L, Hq, Hkv, D, d = 1, 200, 8, 2, 128, 64
+    qi = _ints(55, 1, (B, L, d))
+    ki = _ints(55, 2, (B, L, d))
+    q = _normals(55, 3, (B, L, Hq, D))
+    K = _normals(55, 4, (B, L, Hkv, D))
+    V = _normals(55, 5, (B, L, Hkv, D))
+    idx, cnt = sa.sa_index_score_topk(to_dev(qi), to_dev(ki), 256)
+    out = sa.sa_sparse_attn_prefill(to_dev(q), to_dev(K), to_dev(V), idx, cnt)
+    f = lambda x: torch.from_numpy(oracle.bf16_bits_to_f64(x))
+    G = Hq // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        f(q)[0].permute(1, 0, 2), f(K)[0].repeat_interleave(G, 1).permute(1, 0, 2),
+        f(V)[0].repeat_interleave(G, 1).permute(1, 0, 2), is_causal=True).permute(1, 0, 2)
+    torch.cuda.synchronize()
+    assert_close_attn(out[0].float().cpu().numpy(), ref.numpy(), "dense-equivalent prefill")
+
+
+def test_attention_constant_values_and_clamped_indices():
+    """V rows all equal to one row -> output equals that row for any weights;
+    out-of-range indices inside count read a clamped row, never fault."""
+    B, Hq, Hkv, D, Tk_max, k = 1, 4, 1, 128, 64, 16
+    q = _normals(9, 1, (B, Hq, D))
+    K = _normals(9, 2, (B, Tk_max, Hkv, D))
+    row = _normals(9, 3, (1, 1, 1, D))
+    V = np.broadcast_to(row, (B, Tk_max, Hkv, D)).copy()
+    idx = np.arange(k, dtype=np.int32)[None] * 4
+    idx[0, 3] = 10 ** 6
+    idx[0, 4] = -5
+    out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), i32(idx), i32([k]))
+    torch.cuda.synchronize()
+    expect = np.broadcast_to(oracle.bf16_bits_to_f64(row[0, 0, 0]), (Hq, D))
+    assert_close_attn(out[0].float().cpu().numpy(), expect, "constant V")
+
+
+# ---------------------------------------------------------------------- gist
+
+@pytest.mark.parametrize("n_chunks,k_chunks,chunk_len,partial", [
+    (500, 64, 16, [1, 7, 16]),
+    (40, 64, 16, [0, 3, 16]),          # fewer chunks than k
+    (20000, 64, 16, [16, 5, 1]),       # candidate mode
+    (3000, 100, 4, [2, 0, 4]),
+])
+def test_gist_route_unfold_matches_oracle(n_chunks, k_chunks, chunk_len, partial):
+    B, d = len(partial), 128
+    qr = _ints(5000 + n_chunks, 1, (B, d))
+    gk = _ints(5000 + n_chunks, 2, (B, n_chunks, d))
+    rows, cnt, chunks = sa.sa_gist_route_unfold(to_dev(qr), to_dev(gk), chunk_len, k_chunks,
+                                                i32(partial), with_chunks=True)
+    torch.cuda.synchronize()
+    rows, cnt, chunks = rows.cpu().numpy(), cnt.cpu().numpy(), chunks.cpu().numpy()
+    stride = k_chunks * (chunk_len + 1) + chunk_len
+    for b in range(B):
+        rr, rc = oracle.gist_route_unfold(qr[b], gk[b], chunk_len, k_chunks, partial[b])
+        assert cnt[b] == rr.size
+        np.testing.assert_array_equal(rows[b, : rr.size], rr)
+        assert np.all(rows[b, rr.size:stride] == -1)
+        np.testing.assert_array_equal(chunks[b, : rc.size], rc)
+        assert np.all(chunks[b, rc.size:] == -1)
+
+
+def test_gist_equal_scores_take_first_chunks():
+    B, n_chunks, d = 2, 300, 64
+    qr = np.zeros((B, d), np.uint16)
+    gk = _ints(6, 1, (B, n_chunks, d))
+    rows, cnt = sa.sa_gist_route_unfold(to_dev(qr), to_dev(gk), 16, 64, i32([3, 0]))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(rows.cpu().numpy()[0, : 64 * 17], np.arange(64 * 17))
+    assert list(cnt.cpu().numpy()) == [64 * 17 + 3, 64 * 17]
+
+
+# --------------------------------------------------------------- index cache
+
+def test_index_cache_layers_share_one_index():
+    """[IC] §二/§六 and [LC] "DSA 与 IndexShare": the group's full layer runs
+    the indexer once; each layer of the group attends over exactly that index."""
+    B, T, d, k, Hq, Hkv, D, n_layers = 2, 5000, 128, 512, 16, 4, 128, 4
+    q_idx = _ints(7, 1, (B, d))
+    k_idx = _ints(7, 2, (B, T, d))
+    cache = sa.IndexCache(n_layers, B, 1, k, share_every=4, device=dev())
+    cache.begin_step()
+    with pytest.raises(sa.SAError):
+        cache.get(2)
+    cache.update(0, to_dev(q_idx), to_dev(k_idx), Tk=T, q_pos0=T - 1)
+    ridx, rcnt = oracle.index_topk(q_idx[:, None, :], k_idx, T, T - 1, k)
+    versions = set()
+    for layer in range(n_layers):
+        idx, cnt, ver = cache.get_tensors(layer)
+        versions.add(ver)
+        q = _normals(70 + layer, 1, (B, Hq, D))
+        K = _normals(70 + layer, 2, (B, T, Hkv, D))
+        V = _normals(70 + layer, 3, (B, T, Hkv, D))
+        out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), idx.view(B, k), cnt.view(B))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+        ref, _ = oracle.sparse_attention_decode(q, [K[b, ridx[b, 0]] for b in range(B)],
+                                                [V[b, ridx[b, 0]] for b in range(B)])
+        assert_close_attn(out.float().cpu().numpy(), ref, f"layer {layer}")
+    assert len(versions) == 1
+    cache.close()
+
+
+# ------------------------------------------------------------- device inputs
+
+def test_device_generator_matches_host_generator():
+    from gen import device as gd
+    t = torch.empty(100003, dtype=torch.bfloat16, device=dev())
+    gd.fill_normal(t, 12, 34, start=777)
+    np.testing.assert_array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  ch.normal_bf16(12, 34, start=777, count=100003))
+    gd.fill_int(t, 12, 35, start=5)
+    np.testing.assert_array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  ch.int_bf16(12, 35, start=5, count=100003))
