@@ -1,0 +1,586 @@
+"""Benchmark of the sparse-attention hot path on B200.
+
+Default workload (the headline): decode, batch 8 sequences of 32768 cached
+tokens, 4 layers sharing one routing index (the group's first layer runs the
+indexer once per step), indexer d = 128, attention 32 query heads over 8 kv
+heads, head_dim 128, top-k 2048.  One step = the indexer top-k for the group
+plus the gathered sparse attention of all 4 layers for one new token of every
+sequence.  Metric: decode steps/s (whole job; weak scaling over GPUs, each
+rank runs its own 8 sequences).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--config decode_32k|decode_1m|gist|prefill_2k|prefill_64k]
+
+Prints one JSON line (rank 0).  Inputs are synthetic and seeded (gen/); they
+are generated on the device before timing.  The per-step working set
+(320 MiB) and the caches (4.3 GB) are larger than the 126 MB L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gen import recipes as R  # noqa: E402
+
+CONFIGS = {
+    "decode_32k": R.DECODE_32K,
+    "decode_1m": R.DECODE_1M,
+    "gist": R.GIST_128K,
+    "prefill_2k": R.PREFILL_2K,
+    "prefill_64k": R.PREFILL_64K,
+}
+MIB = 1 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------- clock sampler
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons (read-only)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        # samples under load: within 20% of the busiest clock seen, else all
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+# ------------------------------------------------------------------ decode
+
+class DecodeBench:
+    """Decode step of a group-shared index: full layers run the indexer into
+    the shared index buffer, every layer attends over it."""
+
+    def __init__(self, cfg: R.Decode, device, rank: int):
+        import torch
+        import shared_top_routing_b200 as sa
+        from gen import torch_inputs as TI
+        self.torch, self.sa, self.cfg, self.dev = torch, sa, cfg, device
+        seed_cfg = R.Decode(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+        self.inp = TI.decode_inputs(seed_cfg, device)
+        c = cfg
+        self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
+        L = sa.lib()
+        self.ws_idx = torch.empty(L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k),
+                                  dtype=torch.uint8, device=device)
+        self.ws_attn = torch.empty(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
+                                   dtype=torch.uint8, device=device)
+        self.out = [torch.empty((c.B, c.Hq, c.D), dtype=torch.bfloat16, device=device)
+                    for _ in range(c.n_layers)]
+        self.graphs = {}
+        self.events = {}
+        self.launches_per_step = c.n_groups * 3 + c.n_layers  # score, collect, finish per group; attention per layer
+
+    def step(self, s: int, ev=None):
+        c, sa = self.cfg, self.sa
+        Tk = c.N + s + 1
+        self.cache.begin_step()
+        for layer in range(c.n_layers):
+            if self.cache.is_full(layer) == 1:
+                g = layer // c.share_every
+                if ev is not None:
+                    ev[("idx", layer, 0)].record()
+                self.cache.update(layer, self.inp["q_idx"][g][s], self.inp["k_idx"][g], Tk=Tk,
+                                  q_pos0=Tk - 1, ws=self.ws_idx)
+                if ev is not None:
+                    ev[("idx", layer, 1)].record()
+            idx, cnt, _ = self.cache.get_tensors(layer)
+            if ev is not None:
+                ev[("attn", layer, 0)].record()
+            sa.sa_sparse_attn_decode(self.inp["q"][layer][s], self.inp["K"][layer], self.inp["V"][layer],
+                                     idx.view(c.B, c.k), cnt.view(c.B), out=self.out[layer],
+                                     ws=self.ws_attn)
+            if ev is not None:
+                ev[("attn", layer, 1)].record()
+
+    def _new_events(self):
+        torch, c = self.torch, self.cfg
+        ev = {}
+        for layer in range(c.n_layers):
+            for e in (0, 1):
+                if layer % c.share_every == 0:
+                    ev[("idx", layer, e)] = torch.cuda.Event(enable_timing=True, external=True)
+                ev[("attn", layer, e)] = torch.cuda.Event(enable_timing=True, external=True)
+        return ev
+
+    def capture(self, steps):
+        torch = self.torch
+        stream = torch.cuda.Stream(device=self.dev)
+        for s in steps:
+            ev = self._new_events()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                self.step(s, ev)
+            self.graphs[s] = g
+            self.events[s] = ev
+
+    def kernel_times(self, steps):
+        """Average per-launch device time (ms) of the index and attention
+        parts, from the events captured inside the graphs."""
+        idx_t, attn_t = [], []
+        for s in set(steps):
+            ev = self.events[s]
+            for (kind, layer, e), a in ev.items():
+                if e != 0:
+                    continue
+                dt = a.elapsed_time(ev[(kind, layer, 1)])
+                (idx_t if kind == "idx" else attn_t).append(dt)
+        return (statistics.mean(idx_t) if idx_t else None, statistics.mean(attn_t) if attn_t else None)
+
+    def algorithmic_bytes(self):
+        """Bytes the method must move per step (gathered K/V of the kept rows,
+        the indexer-key stream, queries, indices and outputs)."""
+        c = self.cfg
+        Tk = c.N + 1
+        score = c.n_groups * c.B * Tk * c.d * 2
+        attn_one = c.B * c.k * c.Hkv * c.D * 2 * 2 + c.B * c.Hq * c.D * 2 * 2 + c.B * c.k * 4
+        return score, attn_one
+
+
+def run_native(args, cfg, rank, world):
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    if not isinstance(cfg, R.Decode):
+        return run_native_other(args, cfg, rank, world, dev, peaks)
+    b = DecodeBench(cfg, dev, rank)
+    n_steps = cfg.steps
+    torch.cuda.synchronize()
+    # eager warm-up (kernel attributes, first-touch), then graph capture
+    for i in range(max(1, args.warmup)):
+        b.step(i % n_steps)
+    torch.cuda.synchronize()
+    b.capture(range(n_steps))
+    for i in range(args.warmup):
+        b.graphs[i % n_steps].replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_uuid(torch, dev)) if rank == 0 else None
+    # keep the GPU busy ~1 s before the timed region so clocks are sampled under load
+    t_end = time.time() + (args.soak_seconds if sampler else 0.0)
+    i = 0
+    while time.time() < t_end:
+        b.graphs[i % n_steps].replay()
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    order = [(args.warmup + i) % n_steps for i in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for s in order:
+        b.graphs[s].replay()
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(stop)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    idx_ms, attn_ms = b.kernel_times(order)
+    ms_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # end to end: per step H2D of the new token's rows and queries from pinned
+    # host memory, the step, D2H of all layers' outputs; through the same API
+    e2e = None if args.no_e2e else run_e2e(b, args, dev, world)
+
+    score_bytes, attn_bytes = b.algorithmic_bytes()
+    attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms else None
+    roof = {"kernel": "attn_decode_kernel", "bound": "hbm", "achieved": round(attn_gbs, 1) if attn_gbs else None,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(attn_gbs / peaks["hbm_gbs"], 4) if attn_gbs else None,
+            "traffic": args.traffic, "peak_source": peaks["source"],
+            "algorithmic_bytes_per_launch": attn_bytes}
+    idx_gbs = score_bytes / cfg.n_groups / (idx_ms * 1e-3) / 1e9 if idx_ms else None
+    step_bytes = score_bytes + cfg.n_layers * attn_bytes
+    line = {
+        "metric": "decode steps/s", "value": round(value, 2), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter-hash generator; integer indexer inputs, Irwin-Hall normal K/V/q)",
+        "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.N, "layers": cfg.n_layers,
+                   "share_every": cfg.share_every, "d_idx": cfg.d, "q_heads": cfg.Hq,
+                   "kv_heads": cfg.Hkv, "head_dim": cfg.D, "top_k": cfg.k,
+                   "parallelism": f"replicas{world}",
+                   "l2": "no flush; per-step working set 320 MiB and caches 4.3 GB exceed the 126 MB L2",
+                   "timing": "CUDA graphs per step, CUDA events on the launch stream, max over ranks"},
+        "roofline": roof,
+        "kernels": {"index_topk_ms": round(idx_ms, 5) if idx_ms else None,
+                    "index_topk_scoring_GBps": round(idx_gbs, 1) if idx_gbs else None,
+                    "attn_decode_ms": round(attn_ms, 5) if attn_ms else None,
+                    "step_algorithmic_MiB": round(step_bytes / MIB, 2),
+                    "step_hbm_frac": round(step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "e2e": e2e,
+        "gpu_launches": b.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(cfg, budget_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(b, args, dev, world):
+    import torch
+    c = b.cfg
+    n_steps = c.steps
+    pin = lambda t: t.cpu().pin_memory()
+    host = {}
+    for s in range(n_steps):
+        pos = c.N + s
+        h = {"q_idx": {g: pin(b.inp["q_idx"][g][s]) for g in b.inp["q_idx"]},
+             "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
+             "q": {l: pin(b.inp["q"][l][s]) for l in b.inp["q"]},
+             "K_row": {l: pin(b.inp["K"][l][:, pos]) for l in b.inp["K"]},
+             "V_row": {l: pin(b.inp["V"][l][:, pos]) for l in b.inp["V"]}}
+        host[s] = h
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in b.out]
+    h2d = 0
+    for v in host[0].values():
+        for t in v.values():
+            h2d += t.numel() * t.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+    qi_dev = {g: torch.empty_like(b.inp["q_idx"][g][0]) for g in b.inp["q_idx"]}
+    q_dev = {l: torch.empty_like(b.inp["q"][l][0]) for l in b.inp["q"]}
+
+    def e2e_step(s):
+        h = host[s]
+        pos = c.N + s
+        for g in h["q_idx"]:
+            qi_dev[g].copy_(h["q_idx"][g], non_blocking=True)
+            b.inp["k_idx"][g][:, pos].copy_(h["k_row"][g], non_blocking=True)
+        for l in h["q"]:
+            q_dev[l].copy_(h["q"][l], non_blocking=True)
+            b.inp["K"][l][:, pos].copy_(h["K_row"][l], non_blocking=True)
+            b.inp["V"][l][:, pos].copy_(h["V_row"][l], non_blocking=True)
+        Tk = pos + 1
+        b.cache.begin_step()
+        for layer in range(c.n_layers):
+            if b.cache.is_full(layer) == 1:
+                g = layer // c.share_every
+                b.cache.update(layer, qi_dev[g], b.inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=b.ws_idx)
+            idx, cnt, _ = b.cache.get_tensors(layer)
+            b.sa.sa_sparse_attn_decode(q_dev[layer], b.inp["K"][layer], b.inp["V"][layer],
+                                       idx.view(c.B, c.k), cnt.view(c.B), out=b.out[layer], ws=b.ws_attn)
+        for l, o in enumerate(b.out):
+            outs_h[l].copy_(o, non_blocking=True)
+
+    stream = torch.cuda.Stream(device=dev)
+    graphs = {}
+    for s in range(n_steps):
+        e2e_step(s)  # eager warm-up of this step's copies
+    torch.cuda.synchronize()
+    for s in range(n_steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            e2e_step(s)
+        graphs[s] = g
+    for s in range(min(args.warmup, n_steps)):
+        graphs[s].replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(args.steps):
+        graphs[(args.warmup + i) % n_steps].replay()
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * args.steps / (ms / 1e3), 2), "unit": "steps/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": "per-step CUDA graph: H2D of queries + appended cache rows from pinned memory, "
+                   "index + attention calls, D2H of every layer's output"}
+
+
+# ------------------------------------------------------------ other configs
+
+def run_native_other(args, cfg, rank, world, dev, peaks):
+    """Prefill and gist workloads (for the design doc / profiles, not the headline)."""
+    import torch
+    import shared_top_routing_b200 as sa
+    from gen import torch_inputs as TI
+    if isinstance(cfg, R.Gist):
+        inp = TI.gist_inputs(cfg, dev)
+        rows_cap = cfg.rows_cap
+        L = sa.lib()
+        ws_g = torch.empty(max(256, L.sa_gist_route_unfold_workspace(cfg.B, cfg.n_chunks, cfg.d, cfg.k_chunks)),
+                           dtype=torch.uint8, device=dev)
+        ws_a = torch.empty(max(256, L.sa_sparse_attn_decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, rows_cap)),
+                           dtype=torch.uint8, device=dev)
+        out = torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=dev)
+
+        def step(s):
+            rows, cnt = sa.sa_gist_route_unfold(inp["q_route"][s], inp["gist_key"], cfg.chunk_len,
+                                                cfg.k_chunks, inp["partial_len"][s], ws=ws_g)
+            sa.sa_sparse_attn_decode(inp["q"][s], inp["K"], inp["V"], rows, cnt, out=out, ws=ws_a)
+        n_steps, unit, per = cfg.steps, "steps/s", 1
+        nbytes = cfg.B * cfg.n_chunks * cfg.d * 2 + cfg.B * rows_cap * cfg.Hkv * cfg.D * 4
+        launches = 3
+    else:
+        inp = TI.prefill_inputs(cfg, dev)
+        cache = sa.IndexCache(cfg.n_layers, cfg.B, cfg.L, cfg.k, share_every=cfg.share_every, device=dev)
+        L = sa.lib()
+        ws = torch.empty(max(256, L.sa_index_score_topk_workspace(cfg.B, cfg.L, cfg.L, cfg.d, cfg.k)),
+                         dtype=torch.uint8, device=dev)
+        outs = [torch.empty_like(inp["q"][l]) for l in range(cfg.n_layers)]
+
+        def step(s):
+            cache.begin_step()
+            for layer in range(cfg.n_layers):
+                if cache.is_full(layer) == 1:
+                    g = layer // cfg.share_every
+                    cache.update(layer, inp["q_idx"][g], inp["k_idx"][g], ws=ws)
+                idx, cnt, _ = cache.get_tensors(layer)
+                sa.sa_sparse_attn_prefill(inp["q"][layer], inp["K"][layer], inp["V"][layer], idx, cnt,
+                                          out=outs[layer])
+        n_steps, unit, per = 1, "tokens/s", cfg.B * cfg.L
+        nbytes = None
+        launches = None
+    for i in range(max(1, args.warmup)):
+        step(i % n_steps)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(args.steps):
+        step((args.warmup + i) % n_steps)
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    value = world * args.steps * per / (ms / 1e3)
+    line = {"metric": "decode steps/s" if unit == "steps/s" else "prefill tokens/s",
+            "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "timing": "eager launches, CUDA events"}}
+    if nbytes:
+        line["kernels"] = {"step_algorithmic_MiB": round(nbytes / MIB, 2),
+                           "step_hbm_frac": round(nbytes / (ms / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    if launches:
+        line["gpu_launches"] = launches * args.steps
+    return line
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def _decode_oracle_inputs(cfg: R.Decode, step: int, groups=None, layers=None, batches=None):
+    """Host inputs the oracle needs for one decode step (generated untimed):
+    full indexer caches of the groups, the step's queries, and -- after the
+    oracle's own selection -- the selected K/V rows."""
+    import oracle
+    from gen import counter_hash as ch
+    import numpy as np
+    groups = range(cfg.n_groups) if groups is None else groups
+    layers = range(cfg.n_layers) if layers is None else layers
+    batches = range(cfg.B) if batches is None else batches
+    Tk = cfg.N + step + 1
+    inp = {"k_idx": {}, "q_idx": {}, "q": {}, "rows": {}}
+    for g in groups:
+        n = cfg.B * cfg.Tk_max * cfg.d
+        inp["k_idx"][g] = ch.int_bf16(cfg.seed, R.tid(R.KIND_K_IDX, g), count=n).reshape(cfg.B, cfg.Tk_max, cfg.d)
+        inp["q_idx"][g] = R.decode_q_idx_host(cfg, g, step)
+    for l in layers:
+        inp["q"][l] = R.decode_q_host(cfg, l, step)
+    # rows each sequence selects (oracle's own top-k), regenerated per layer
+    sel = {}
+    for g in groups:
+        idx, cnt = oracle.index_topk(inp["q_idx"][g][:, None, :], inp["k_idx"][g], Tk, Tk - 1, cfg.k)
+        sel[g] = (idx[:, 0], cnt[:, 0])
+    for l in layers:
+        g = l // cfg.share_every
+        idx, cnt = sel[g]
+        Kr, Vr = [], []
+        for b in batches:
+            rows = idx[b, : cnt[b]]
+            Kr.append(R.host_rows(cfg.seed, R.tid(R.KIND_K, l), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
+            Vr.append(R.host_rows(cfg.seed, R.tid(R.KIND_V, l), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
+        inp["rows"][l] = (Kr, Vr)
+    return inp, Tk
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_decode_step(cfg: R.Decode, inp, Tk):
+    """One oracle decode step on prepared host inputs: indexer top-k per
+    group (full sort) and fp64 attention of every layer over its group's
+    selected rows."""
+    import oracle
+    for g in inp["k_idx"]:
+        oracle.index_topk(inp["q_idx"][g][:, None, :], inp["k_idx"][g], Tk, Tk - 1, cfg.k)
+    for l, (Kr, Vr) in inp["rows"].items():
+        oracle.sparse_attention_decode(inp["q"][l][: len(Kr)], Kr, Vr)
+
+
+def cpu_baseline_decode(cfg: R.Decode, budget_s: float = 10.0):
+    inp, Tk = _decode_oracle_inputs(cfg, 0)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_decode_step(cfg, inp, Tk)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 100:
+            break
+    return {"value": round(reps / el, 4), "unit": "steps/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"decode step 0 of {cfg.name} (all {cfg.B} sequences, {cfg.n_groups} indexer "
+                      f"group(s), {cfg.n_layers} layers) repeated {reps} times in {el:.1f} s; numpy fp64; "
+                      "host input generation and row regeneration untimed"}
+
+
+def run_reference(args, cfg, rank, world):
+    """The oracle as the reference arm: same metric, unit and config."""
+    if rank != 0:
+        return None
+    if not isinstance(cfg, R.Decode):
+        return {"impl": "reference", "unavailable": "reference arm implemented for decode workloads only"}
+    # each step is one oracle decode step on a bounded sample: sequence 0 only
+    batches = [0]
+    inp, Tk = _decode_oracle_inputs(cfg, 0, batches=batches)
+    sub = {**inp, "q_idx": {g: v[:1] for g, v in inp["q_idx"].items()},
+           "k_idx": {g: v[:1] for g, v in inp["k_idx"].items()}}
+    for _ in range(args.warmup):
+        oracle_decode_step(cfg, sub, Tk)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_decode_step(cfg, sub, Tk)
+    el = time.perf_counter() - t0
+    # a full step covers all B sequences: scale the one-sequence sample
+    value = args.steps / (el * cfg.B)
+    cores = _blas_threads()
+    return {"impl": "reference", "metric": "decode steps/s", "value": round(value, 5), "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el * cfg.B / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.N, "layers": cfg.n_layers,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 5), "unit": "steps/s", "cores": cores, "kind": "oracle",
+                             "sample": f"sequence 0 of {cfg.B} per step (scaled by {cfg.B}); oracle in numpy fp64"},
+            "e2e": {"value": round(value, 5), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="decode_32k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--soak-seconds", type=float, default=1.0,
+                    help="busy time before the timed region so clocks are sampled under load")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        line = run_reference(args, cfg, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_native(args, cfg, rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
