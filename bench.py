@@ -55,6 +55,65 @@ def load_peaks():
                 "source": "fallback"}
 
 
+# ------------------------------------------------------------ CUDA runtime
+
+class Cudart:
+    """The CUDA runtime that torch and libsa.so share, through ctypes: stream
+    capture into CUDA graphs (torch's graph wrapper adds RNG-state fills to
+    every replay) and plain async copies.  One copy per tensor; no batched
+    copy APIs."""
+
+    def __init__(self):
+        import ctypes
+        import torch  # noqa: F401  (loads the runtime first)
+        self.ct = ctypes
+        self.rt = ctypes.CDLL("libcudart.so.12")
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        self.rt.cudaStreamBeginCapture.argtypes = [P, I]
+        self.rt.cudaStreamEndCapture.argtypes = [P, ctypes.POINTER(P)]
+        self.rt.cudaGraphInstantiate.argtypes = [ctypes.POINTER(P), P, ctypes.c_ulonglong]
+        self.rt.cudaGraphLaunch.argtypes = [P, P]
+        self.rt.cudaGraphExecDestroy.argtypes = [P]
+        self.rt.cudaGraphDestroy.argtypes = [P]
+        self.rt.cudaMemcpyAsync.argtypes = [P, P, Z, I, P]
+        self.rt.cudaMemcpy2DAsync.argtypes = [P, Z, P, Z, Z, Z, I, P]
+
+    def check(self, rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what} failed with cudaError {rc}")
+
+    def capture(self, stream, fn):
+        """Records fn()'s work on `stream` into an instantiated graph."""
+        ct = self.ct
+        s = ct.c_void_p(stream.cuda_stream)
+        self.check(self.rt.cudaStreamBeginCapture(s, 1), "cudaStreamBeginCapture")
+        try:
+            fn()
+        finally:
+            g = ct.c_void_p()
+            rc = self.rt.cudaStreamEndCapture(s, ct.byref(g))
+        self.check(rc, "cudaStreamEndCapture")
+        ex = ct.c_void_p()
+        self.check(self.rt.cudaGraphInstantiate(ct.byref(ex), g, 0), "cudaGraphInstantiate")
+        self.rt.cudaGraphDestroy(g)
+        return ex
+
+    def launch(self, ex, stream):
+        self.check(self.rt.cudaGraphLaunch(ex, self.ct.c_void_p(stream.cuda_stream)), "cudaGraphLaunch")
+
+    def h2d(self, dst_ptr, src_ptr, nbytes, stream):
+        self.check(self.rt.cudaMemcpyAsync(dst_ptr, src_ptr, nbytes, 1, self.ct.c_void_p(stream.cuda_stream)),
+                   "cudaMemcpyAsync")
+
+    def d2h(self, dst_ptr, src_ptr, nbytes, stream):
+        self.check(self.rt.cudaMemcpyAsync(dst_ptr, src_ptr, nbytes, 2, self.ct.c_void_p(stream.cuda_stream)),
+                   "cudaMemcpyAsync")
+
+    def h2d_2d(self, dst_ptr, dpitch, src_ptr, spitch, width, height, stream):
+        self.check(self.rt.cudaMemcpy2DAsync(dst_ptr, dpitch, src_ptr, spitch, width, height, 1,
+                                             self.ct.c_void_p(stream.cuda_stream)), "cudaMemcpy2DAsync")
+
+
 # --------------------------------------------------------------- clock sampler
 
 class ClockSampler:
@@ -126,15 +185,16 @@ class DecodeBench:
         c = cfg
         self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
         L = sa.lib()
-        self.ws_idx = torch.empty(L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k),
+        self.ws_idx = torch.zeros(L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k),
                                   dtype=torch.uint8, device=device)
-        self.ws_attn = torch.empty(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
+        self.ws_attn = torch.zeros(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
                                    dtype=torch.uint8, device=device)
         self.out = [torch.empty((c.B, c.Hq, c.D), dtype=torch.bfloat16, device=device)
                     for _ in range(c.n_layers)]
         self.graphs = {}
         self.events = {}
-        self.launches_per_step = c.n_groups * 3 + c.n_layers  # score, collect, finish per group; attention per layer
+        # kernels per indexer run: score + finish, plus collect for rows longer than one CTA scans
+        self.launches_per_step = c.n_groups * (3 if c.Tk_max > (1 << 18) else 2) + c.n_layers
 
     def step(self, s: int, ev=None):
         c, sa = self.cfg, self.sa
@@ -168,16 +228,18 @@ class DecodeBench:
                 ev[("attn", layer, e)] = torch.cuda.Event(enable_timing=True, external=True)
         return ev
 
-    def capture(self, steps):
+    def capture(self, steps, rt):
         torch = self.torch
-        stream = torch.cuda.Stream(device=self.dev)
+        self.rt = rt
+        self.stream = torch.cuda.Stream(device=self.dev)
         for s in steps:
             ev = self._new_events()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                self.step(s, ev)
-            self.graphs[s] = g
+            with torch.cuda.stream(self.stream):
+                self.graphs[s] = rt.capture(self.stream, lambda: self.step(s, ev))
             self.events[s] = ev
+
+    def replay(self, s):
+        self.rt.launch(self.graphs[s], self.stream)
 
     def kernel_times(self, steps):
         """Average per-launch device time (ms) of the index and attention
@@ -210,15 +272,16 @@ def run_native(args, cfg, rank, world):
     if not isinstance(cfg, R.Decode):
         return run_native_other(args, cfg, rank, world, dev, peaks)
     b = DecodeBench(cfg, dev, rank)
+    rt = Cudart()
     n_steps = cfg.steps
     torch.cuda.synchronize()
     # eager warm-up (kernel attributes, first-touch), then graph capture
     for i in range(max(1, args.warmup)):
         b.step(i % n_steps)
     torch.cuda.synchronize()
-    b.capture(range(n_steps))
+    b.capture(range(n_steps), rt)
     for i in range(args.warmup):
-        b.graphs[i % n_steps].replay()
+        b.replay(i % n_steps)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(gpu_uuid(torch, dev)) if rank == 0 else None
@@ -226,7 +289,7 @@ def run_native(args, cfg, rank, world):
     t_end = time.time() + (args.soak_seconds if sampler else 0.0)
     i = 0
     while time.time() < t_end:
-        b.graphs[i % n_steps].replay()
+        b.replay(i % n_steps)
         i += 1
         if i % 64 == 0:
             torch.cuda.synchronize()
@@ -237,10 +300,10 @@ def run_native(args, cfg, rank, world):
     order = [(args.warmup + i) % n_steps for i in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
-    start.record()
+    start.record(b.stream)
     for s in order:
-        b.graphs[s].replay()
-    stop.record()
+        b.replay(s)
+    stop.record(b.stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -294,38 +357,47 @@ def run_native(args, cfg, rank, world):
 
 
 def run_e2e(b, args, dev, world):
+    """Same steps through the public API with host buffers: every step copies
+    its queries and the appended token's cache rows from pinned host memory
+    (one cudaMemcpyAsync / cudaMemcpy2DAsync per tensor), runs the step, and
+    copies every layer's output back to pinned host memory."""
     import torch
     c = b.cfg
+    rt = b.rt
     n_steps = c.steps
-    pin = lambda t: t.cpu().pin_memory()
+    st = b.stream
+    pin = lambda t: t.contiguous().cpu().pin_memory()
     host = {}
     for s in range(n_steps):
         pos = c.N + s
-        h = {"q_idx": {g: pin(b.inp["q_idx"][g][s]) for g in b.inp["q_idx"]},
-             "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
-             "q": {l: pin(b.inp["q"][l][s]) for l in b.inp["q"]},
-             "K_row": {l: pin(b.inp["K"][l][:, pos]) for l in b.inp["K"]},
-             "V_row": {l: pin(b.inp["V"][l][:, pos]) for l in b.inp["V"]}}
-        host[s] = h
+        host[s] = {"q_idx": {g: pin(b.inp["q_idx"][g][s]) for g in b.inp["q_idx"]},
+                   "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
+                   "q": {l: pin(b.inp["q"][l][s]) for l in b.inp["q"]},
+                   "K_row": {l: pin(b.inp["K"][l][:, pos]) for l in b.inp["K"]},
+                   "V_row": {l: pin(b.inp["V"][l][:, pos]) for l in b.inp["V"]}}
     outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in b.out]
-    h2d = 0
-    for v in host[0].values():
-        for t in v.values():
-            h2d += t.numel() * t.element_size()
+    h2d = sum(t.numel() * t.element_size() for v in host[0].values() for t in v.values())
     d2h = sum(o.numel() * o.element_size() for o in outs_h)
     qi_dev = {g: torch.empty_like(b.inp["q_idx"][g][0]) for g in b.inp["q_idx"]}
     q_dev = {l: torch.empty_like(b.inp["q"][l][0]) for l in b.inp["q"]}
+
+    def row_copy(cache, src, pos):
+        # cache [B, Tk_max, ...]: B blocks of one row each, pitch = one sequence
+        row_bytes = src[0].numel() * src.element_size()
+        pitch = cache[0].numel() * cache.element_size()
+        rt.h2d_2d(cache.data_ptr() + pos * row_bytes, pitch, src.data_ptr(), row_bytes, row_bytes,
+                  src.shape[0], st)
 
     def e2e_step(s):
         h = host[s]
         pos = c.N + s
         for g in h["q_idx"]:
-            qi_dev[g].copy_(h["q_idx"][g], non_blocking=True)
-            b.inp["k_idx"][g][:, pos].copy_(h["k_row"][g], non_blocking=True)
+            rt.h2d(qi_dev[g].data_ptr(), h["q_idx"][g].data_ptr(), h["q_idx"][g].numel() * 2, st)
+            row_copy(b.inp["k_idx"][g], h["k_row"][g], pos)
         for l in h["q"]:
-            q_dev[l].copy_(h["q"][l], non_blocking=True)
-            b.inp["K"][l][:, pos].copy_(h["K_row"][l], non_blocking=True)
-            b.inp["V"][l][:, pos].copy_(h["V_row"][l], non_blocking=True)
+            rt.h2d(q_dev[l].data_ptr(), h["q"][l].data_ptr(), h["q"][l].numel() * 2, st)
+            row_copy(b.inp["K"][l], h["K_row"][l], pos)
+            row_copy(b.inp["V"][l], h["V_row"][l], pos)
         Tk = pos + 1
         b.cache.begin_step()
         for layer in range(c.n_layers):
@@ -336,29 +408,27 @@ def run_e2e(b, args, dev, world):
             b.sa.sa_sparse_attn_decode(q_dev[layer], b.inp["K"][layer], b.inp["V"][layer],
                                        idx.view(c.B, c.k), cnt.view(c.B), out=b.out[layer], ws=b.ws_attn)
         for l, o in enumerate(b.out):
-            outs_h[l].copy_(o, non_blocking=True)
+            rt.d2h(outs_h[l].data_ptr(), o.data_ptr(), o.numel() * o.element_size(), st)
 
-    stream = torch.cuda.Stream(device=dev)
-    graphs = {}
-    for s in range(n_steps):
-        e2e_step(s)  # eager warm-up of this step's copies
-    torch.cuda.synchronize()
-    for s in range(n_steps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+    with torch.cuda.stream(st):
+        for s in range(n_steps):
             e2e_step(s)
-        graphs[s] = g
+    torch.cuda.synchronize()
+    graphs = {}
+    with torch.cuda.stream(st):
+        for s in range(n_steps):
+            graphs[s] = rt.capture(st, lambda: e2e_step(s))
     for s in range(min(args.warmup, n_steps)):
-        graphs[s].replay()
+        rt.launch(graphs[s], st)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
-    start.record()
+    start.record(st)
     for i in range(args.steps):
-        graphs[(args.warmup + i) % n_steps].replay()
-    stop.record()
+        rt.launch(graphs[(args.warmup + i) % n_steps], st)
+    stop.record(st)
     torch.cuda.synchronize()
     ms = start.elapsed_time(stop)
     if world > 1:
@@ -382,9 +452,9 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
         inp = TI.gist_inputs(cfg, dev)
         rows_cap = cfg.rows_cap
         L = sa.lib()
-        ws_g = torch.empty(max(256, L.sa_gist_route_unfold_workspace(cfg.B, cfg.n_chunks, cfg.d, cfg.k_chunks)),
+        ws_g = torch.zeros(max(256, L.sa_gist_route_unfold_workspace(cfg.B, cfg.n_chunks, cfg.d, cfg.k_chunks)),
                            dtype=torch.uint8, device=dev)
-        ws_a = torch.empty(max(256, L.sa_sparse_attn_decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, rows_cap)),
+        ws_a = torch.zeros(max(256, L.sa_sparse_attn_decode_workspace(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, rows_cap)),
                            dtype=torch.uint8, device=dev)
         out = torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=dev)
 
@@ -399,7 +469,7 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
         inp = TI.prefill_inputs(cfg, dev)
         cache = sa.IndexCache(cfg.n_layers, cfg.B, cfg.L, cfg.k, share_every=cfg.share_every, device=dev)
         L = sa.lib()
-        ws = torch.empty(max(256, L.sa_index_score_topk_workspace(cfg.B, cfg.L, cfg.L, cfg.d, cfg.k)),
+        ws = torch.zeros(max(256, L.sa_index_score_topk_workspace(cfg.B, cfg.L, cfg.L, cfg.d, cfg.k)),
                          dtype=torch.uint8, device=dev)
         outs = [torch.empty_like(inp["q"][l]) for l in range(cfg.n_layers)]
 
@@ -551,6 +621,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode_32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode only: run fewer layers (small profiling cases; not the headline)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="busy time before the timed region so clocks are sampled under load")
@@ -563,6 +635,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     cfg = CONFIGS[args.config]
+    if args.layers is not None and isinstance(cfg, R.Decode):
+        cfg = R.Decode(**{**cfg.__dict__, "n_layers": args.layers,
+                          "name": f"{cfg.name}_first{args.layers}layers"})
     if args.impl == "reference":
         line = run_reference(args, cfg, rank, world)
         if line is not None:

@@ -23,8 +23,13 @@
  *     any CUDA kernel.
  *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
  *   - No kernel of this library waits on another CTA, kernel or device.
- *   - Calls are not thread-safe with respect to one shared workspace;
- *     calls on different streams need different workspaces.
+ *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned, and
+ *     must be ZERO-FILLED before their first use.  Every call that returns
+ *     SA_OK leaves the parts of its workspace that must start at zero back
+ *     at zero once its kernels complete, so one workspace serves any number
+ *     of calls made one after another on one stream.  Calls that overlap on
+ *     the GPU (different streams) need different workspaces.  After a failed
+ *     or interrupted call, zero the workspace again.
  */
 #ifndef SA_H_
 #define SA_H_
@@ -88,9 +93,8 @@ int sa_version(void);
  *                                      outside are clamped on the device)
  *   idx_out    [B, Tq, k] int32;  count_out [B, Tq] int32
  *   score_out  [B, Tq, k] fp32 or NULL
- *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes,
- *              SA_WS_ALIGN-aligned; contents need no initialisation and are
- *              clobbered.
+ *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes
+ *              (zero-filled before first use; see the conventions above).
  * Supported: d in {64, 128}; 1 <= k <= SA_MAX_K; Tq >= 1; 0 <= Tk <= Tk_max.
  * Scores must be free of NaN (NaN inputs give an unspecified selection).
  * ---------------------------------------------------------------------- */
@@ -121,8 +125,9 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx,
  *   idx      [B, T, k] int32 (each used entry in [0, Tk_max); entries past
  *            count are ignored); count [B, T] int32 (clamped to [0, k])
  *   out      [B, T, Hq, D] bf16;  lse [B, T, Hq] fp32 or NULL
- * Supported: D = 128; Hq % Hkv == 0; 1 <= Hq/Hkv <= 16; k <= SA_MAX_K.
- * Out-of-range used indices are a caller error (the kernel does not check).
+ * Supported: D = 128; Hq % Hkv == 0; 1 <= Hq/Hkv <= 16.
+ * Used indices outside [0, Tk_max) are a caller error; the kernels clamp
+ * them into range (reading a wrong row) rather than fault.
  * ---------------------------------------------------------------------- */
 sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* idx, const int32_t* count,
@@ -141,7 +146,8 @@ sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void*
  *   q        [B, Hq, D] bf16
  *   idx      [B, k] int32 (row stride k); count [B] int32 (clamped to [0, k])
  *   out      [B, Hq, D] bf16;  lse [B, Hq] fp32 or NULL
- *   ws       >= sa_sparse_attn_decode_workspace(...) bytes, SA_WS_ALIGN-aligned
+ *   ws       >= sa_sparse_attn_decode_workspace(...) bytes (zero-filled before
+ *            first use; see the conventions above)
  * Supported: as for prefill.
  * ---------------------------------------------------------------------- */
 size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k);

@@ -72,8 +72,6 @@ sa_status validate_index(const void* q_idx, const void* k_idx, int B, int Tq, in
   return SA_OK;
 }
 
-bool use_candidates(int Tk_max) { return Tk_max > sa::kDirectMaxCand; }
-
 sa_status validate_attn(const void* q, const void* kc, const void* vc, const int32_t* idx,
                         const int32_t* count, int B, int T, int Tk_max, int Hq, int Hkv, int D,
                         int k, const void* out) {
@@ -140,7 +138,11 @@ size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
   (void)d;
   (void)k;
   if (B <= 0 || Tq <= 0 || Tk_max < 0) return 0;
-  if (Tq == 1) return sa::row_workspace_bytes(B, Tk_max, use_candidates(Tk_max));
+  if (Tq == 1) {
+    bool collect = false;
+    sa::finish_mode_for(Tk_max, &collect);
+    return sa::row_workspace_bytes(B, Tk_max, collect);
+  }
   int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
   return sa::row_workspace_bytes(B * rows, Tk_max, false);
 }
@@ -163,19 +165,16 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
   out.score = score_out;
   cudaError_t e;
   if (Tq == 1) {
-    const bool cand = use_candidates(Tk_max);
+    bool collect = false;
+    const int mode = sa::finish_mode_for(Tk_max, &collect);
     sa::RowWorkspace w;
-    sa::carve_row_workspace(ws, B, Tk_max, cand, &w);
-    if (cand) {
-      // histogram and candidate counters start at zero (adjacent in the workspace)
-      size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
-      if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
-    }
-    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, cand, cs)) != cudaSuccess)
+    sa::carve_row_workspace(ws, B, Tk_max, collect, &w);
+    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w,
+                                     mode != sa::kFinishDirect, cs)) != cudaSuccess)
       return cuda_fail(e, "score_decode launch");
-    if (cand && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
+    if (collect && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
       return cuda_fail(e, "collect launch");
-    if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, cand, out, cs)) != cudaSuccess)
+    if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, mode, out, cs)) != cudaSuccess)
       return cuda_fail(e, "finish launch");
     return ok();
   }
@@ -186,7 +185,7 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
     const int nr = (Tq - t0 < rows) ? Tq - t0 : rows;
     if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, w, cs)) != cudaSuccess)
       return cuda_fail(e, "score_prefill launch");
-    if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, false, out, cs)) != cudaSuccess)
+    if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, sa::kFinishDirect, out, cs)) != cudaSuccess)
       return cuda_fail(e, "finish launch");
   }
   return ok();
@@ -239,7 +238,9 @@ size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) 
   (void)d;
   (void)k_chunks;
   if (B <= 0 || n_chunks < 0) return 0;
-  return sa::row_workspace_bytes(B, n_chunks, use_candidates(n_chunks));
+  bool collect = false;
+  sa::finish_mode_for(n_chunks, &collect);
+  return sa::row_workspace_bytes(B, n_chunks, collect);
 }
 
 sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B, int n_chunks,
@@ -261,20 +262,17 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   sa_status st = check_ws(ws, ws_bytes, sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks));
   if (st != SA_OK) return st;
   cudaStream_t cs = as_cuda(stream);
-  const bool cand = use_candidates(n_chunks);
+  bool collect = false;
+  const int mode = sa::finish_mode_for(n_chunks, &collect);
   sa::RowWorkspace w;
-  sa::carve_row_workspace(ws, B, n_chunks, cand, &w);
+  sa::carve_row_workspace(ws, B, n_chunks, collect, &w);
   cudaError_t e;
-  if (cand) {
-    size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
-    if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
-  }
   const int q_pos0 = n_chunks - 1;  // every complete chunk is a candidate
   if ((e = sa::launch_score_decode(static_cast<const uint16_t*>(q_route),
                                    static_cast<const uint16_t*>(gist_key), B, d, n_chunks, n_chunks,
-                                   q_pos0, nullptr, w, cand, cs)) != cudaSuccess)
+                                   q_pos0, nullptr, w, mode != sa::kFinishDirect, cs)) != cudaSuccess)
     return cuda_fail(e, "gist score launch");
-  if (cand && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
+  if (collect && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
     return cuda_fail(e, "gist collect launch");
   sa::FinishOut out;
   out.count = count_out;
@@ -284,7 +282,7 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   out.n_chunks = n_chunks;
   out.partial_len = partial_len;
   out.chunks = chunks_out;
-  if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, cand, out, cs)) != cudaSuccess)
+  if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, mode, out, cs)) != cudaSuccess)
     return cuda_fail(e, "gist finish launch");
   return ok();
 }

@@ -7,19 +7,21 @@
 // one kv head are loaded once for all query heads of its GQA group, and the
 // partial (max, sum, output) triples are merged by the log-sum-exp rule.
 //
-// attn_decode_kernel   grid (splits, Hkv, B), 128 threads.  cp.async gathers
-//                      the split's K rows and V rows into padded shared tiles
-//                      (two commit groups so scores overlap the V transfer),
-//                      CUDA-core fp32 dot products and softmax, and the last
-//                      CTA of each (sequence, kv head) -- found with an atomic
-//                      ticket, never a wait -- merges the partials.
-// attn_prefill_kernel  grid (T, Hkv, B) kv-head-major, 128 threads.  For one
-//                      query token and one kv head, 64-row tiles of gathered
-//                      K/V are double-buffered through shared memory with
-//                      cp.async; each warp owns 16 rows of a tile and runs
-//                      FlashAttention-style online softmax on mma.sync
-//                      m16n8k16 (the G query heads padded to 16 rows); the 4
-//                      warps' partials are merged at the end.
+// Both kernels share one tile loop (attn_tiles): 64 gathered rows per tile,
+// K and V rows of one kv head (256 contiguous bytes each) gathered with
+// 16-byte cp.async into padded shared tiles, two stages so the gather of tile
+// i+1 overlaps the math of tile i.  Each of the 4 warps owns 16 rows of a
+// tile and runs online softmax on mma.sync m16n8k16 (bf16 in, fp32
+// accumulate) with the G query heads of the group as the 16-row M side
+// (zero padded), S = Q K^T then O += P V (V through ldmatrix.trans).
+//
+// attn_prefill_kernel  grid (T, Hkv, B), kv-head-major: one query token x one
+//                      kv head per CTA, all of its selected rows.
+// attn_decode_kernel   grid (splits, Hkv, B): each CTA takes a contiguous
+//                      range of tiles of the sequence's index list and writes
+//                      a partial (m, l, o); the last CTA of each (sequence, kv
+//                      head) -- found with an atomic ticket, never a wait --
+//                      merges them.  With one split it writes the output.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -31,7 +33,8 @@ namespace sa {
 namespace {
 
 constexpr int kD = 128;        // head_dim
-constexpr int kLds = kD + 8;   // padded smem row (elements)
+constexpr int kLds = kD + 8;   // padded smem row (elements): 272 bytes
+constexpr int kTile = 64;      // gathered rows per tile (16 per warp)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -39,249 +42,64 @@ __device__ __forceinline__ int clamp_row(int j, int Tk_max) {
   return j < 0 ? 0 : (j >= Tk_max ? Tk_max - 1 : j);
 }
 
-// ------------------------------------------------------------------ decode
+// Shared memory of one CTA: Q (16 rows), 2 stages of K and V tiles; the
+// stage area is reused for the cross-warp merge.
+constexpr size_t kSmemQ = 16 * kLds * 2;
+constexpr size_t kSmemStage = (size_t)kTile * kLds * 2;
+constexpr size_t kSmemTotal = kSmemQ + 4 * kSmemStage;
 
-template <int G>
-__global__ void __launch_bounds__(128)
-attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
-                   const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
-                   const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k, int R,
-                   int S, float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
-                   unsigned* __restrict__ ticket, uint16_t* __restrict__ out,
-                   float* __restrict__ lse) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  // layout: qs[G][kD] f32 | sc[DS][G][R] f32 | ml[32] f32 | Ks[R][kLds] | Vs[R][kLds]
-  // (every region a multiple of 16 bytes, so the cp.async targets stay aligned)
-  const int DS = 128 / R;  // dim slices for the score phase (R in {32, 64, 128})
-  float* qs = reinterpret_cast<float*>(smem);
-  float* sc = qs + G * kD;
-  float* mls = sc + DS * G * R;
-  uint16_t* Ks = reinterpret_cast<uint16_t*>(mls + 32);
-  uint16_t* Vs = Ks + R * kLds;
-  __shared__ int s_last;
+struct TileAcc {
+  float o[16][4];
+  float m[2], l[2];
+};
 
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int cnt = count[b];
-  cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
-  const int i0 = s * R;
-  const int nrow = max(0, min(R, cnt - i0));
-  const long long part = ((long long)b * Hq + g * G);  // first head of the group
-
-  if (nrow > 0) {
-    // gather: thread -> (row, 16-byte chunk); K group first, then V group
-    const int32_t* irow = idx + (long long)b * k + i0;
-    for (int e = tid; e < R * 16; e += 128) {
-      int r = e >> 4, c = e & 15;
-      bool v = r < nrow;
-      int j = v ? clamp_row(irow[r], Tk_max) : 0;
-      long long off = (((long long)b * Tk_max + j) * Hkv + g) * kD + c * 8;
-      cp_async16(Ks + r * kLds + c * 8, kc + off, v);
-    }
-    cp_async_commit();
-    for (int e = tid; e < R * 16; e += 128) {
-      int r = e >> 4, c = e & 15;
-      bool v = r < nrow;
-      int j = v ? clamp_row(irow[r], Tk_max) : 0;
-      long long off = (((long long)b * Tk_max + j) * Hkv + g) * kD + c * 8;
-      cp_async16(Vs + r * kLds + c * 8, vc + off, v);
-    }
-    cp_async_commit();
-    // q of the group's heads, pre-scaled into the log2 domain
-    for (int e = tid; e < G * kD / 2; e += 128) {
-      int h = e / (kD / 2), c2 = e % (kD / 2);
-      uint32_t v = *reinterpret_cast<const uint32_t*>(q + (part + h) * kD + 2 * c2);
-      qs[h * kD + 2 * c2] = bf_lo(v) * qscale;
-      qs[h * kD + 2 * c2 + 1] = bf_hi(v) * qscale;
-    }
-    cp_async_wait<1>();
-    __syncthreads();
-
-    // scores: thread -> (row within a 32-row band, dim slice)
-    {
-      const int bands = 4 / DS;
-      const int r = (warp % bands) * 32 + lane;
-      const int slice = warp / bands;
-      const int dlen = kD / DS;
-      float acc[G];
+// Gathers tile rows [i0, i0+64) (clipped to `end`) of one kv head into stage.
+__device__ __forceinline__ void gather_tile(uint16_t* sK, uint16_t* sV, const uint16_t* __restrict__ kc,
+                                            const uint16_t* __restrict__ vc, const int32_t* __restrict__ irow,
+                                            int i0, int end, long long head_base, long long row_elems,
+                                            int Tk_max) {
+  const int r = threadIdx.x >> 1, h = threadIdx.x & 1;
+  const int i = i0 + r;
+  const bool v = i < end;
+  const int j = v ? clamp_row(irow[i], Tk_max) : 0;
+  const long long off = head_base + (long long)j * row_elems;
+  uint16_t* dk = sK + r * kLds;
+  uint16_t* dv = sV + r * kLds;
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f;
-      const uint16_t* krow = Ks + r * kLds + slice * dlen;
-      for (int c = 0; c < dlen; c += 8) {
-        uint4 kv = *reinterpret_cast<const uint4*>(krow + c);
-        float kf[8] = {bf_lo(kv.x), bf_hi(kv.x), bf_lo(kv.y), bf_hi(kv.y),
-                       bf_lo(kv.z), bf_hi(kv.z), bf_lo(kv.w), bf_hi(kv.w)};
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float4* qp = reinterpret_cast<const float4*>(qs + h * kD + slice * dlen + c);
-          float4 qa = qp[0], qb = qp[1];
-          float a = acc[h];
-          a = fmaf(kf[0], qa.x, a); a = fmaf(kf[1], qa.y, a);
-          a = fmaf(kf[2], qa.z, a); a = fmaf(kf[3], qa.w, a);
-          a = fmaf(kf[4], qb.x, a); a = fmaf(kf[5], qb.y, a);
-          a = fmaf(kf[6], qb.z, a); a = fmaf(kf[7], qb.w, a);
-          acc[h] = a;
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) sc[(slice * G + h) * R + r] = acc[h];
-    }
-    __syncthreads();
-    // softmax per head (warp per head), p overwrites slice 0
-    for (int h = warp; h < G; h += 4) {
-      float m = -INFINITY;
-      for (int r = lane; r < R; r += 32) {
-        float z = 0.f;
-        for (int sl = 0; sl < DS; ++sl) z += sc[(sl * G + h) * R + r];
-        z = r < nrow ? z : -INFINITY;
-        sc[h * R + r] = z;
-        m = fmaxf(m, z);
-      }
-      m = warp_max(m);
-      float l = 0.f;
-      for (int r = lane; r < R; r += 32) {
-        float p = r < nrow ? exp2f(sc[h * R + r] - m) : 0.f;
-        sc[h * R + r] = p;
-        l += p;
-      }
-      l = warp_sum(l);
-      if (lane == 0) { mls[2 * h] = m; mls[2 * h + 1] = l; }
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    // P V: thread -> dims (2c2, 2c2+1), heads of one parity
-    {
-      const int c2 = tid & 63, hp = tid >> 6;
-      float o0[(G + 1) / 2], o1[(G + 1) / 2];
-#pragma unroll
-      for (int u = 0; u < (G + 1) / 2; ++u) { o0[u] = 0.f; o1[u] = 0.f; }
-      for (int r = 0; r < nrow; ++r) {
-        uint32_t v = *reinterpret_cast<const uint32_t*>(Vs + r * kLds + 2 * c2);
-        float v0 = bf_lo(v), v1 = bf_hi(v);
-#pragma unroll
-        for (int u = 0; u < (G + 1) / 2; ++u) {
-          int h = hp + 2 * u;
-          if (h < G) {
-            float p = sc[h * R + r];
-            o0[u] = fmaf(p, v0, o0[u]);
-            o1[u] = fmaf(p, v1, o1[u]);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < (G + 1) / 2; ++u) {
-        int h = hp + 2 * u;
-        if (h < G) {
-          float2* dst = reinterpret_cast<float2*>(part_o + ((part + h) * S + s) * kD + 2 * c2);
-          *dst = make_float2(o0[u], o1[u]);
-        }
-      }
-    }
-    if (tid < G) {
-      part_ml[((part + tid) * S + s) * 2] = mls[2 * tid];
-      part_ml[((part + tid) * S + s) * 2 + 1] = mls[2 * tid + 1];
-    }
-  } else if (tid < G) {
-    part_ml[((part + tid) * S + s) * 2] = -INFINITY;
-    part_ml[((part + tid) * S + s) * 2 + 1] = 0.f;
+  for (int c = h * 8; c < h * 8 + 8; ++c) {
+    cp_async16(dk + c * 8, kc + off + c * 8, v);
+    cp_async16(dv + c * 8, vc + off + c * 8, v);
   }
-
-  // Last CTA of this (sequence, kv head) merges the S partials.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    unsigned prev = atomicAdd(ticket + (long long)b * Hkv + g, 1u);
-    s_last = (prev == (unsigned)(S - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  {
-    const int c2 = tid & 63, hp = tid >> 6;
-    for (int h = hp; h < G; h += 2) {
-      const float* ml = part_ml + (part + h) * S * 2;
-      float M = -INFINITY;
-      for (int x = 0; x < S; ++x) M = fmaxf(M, __ldcg(ml + 2 * x));
-      float L = 0.f, a0 = 0.f, a1 = 0.f;
-      if (M != -INFINITY) {
-        for (int x = 0; x < S; ++x) {
-          float mx = __ldcg(ml + 2 * x), lx = __ldcg(ml + 2 * x + 1);
-          if (lx == 0.f) continue;
-          float w = exp2f(mx - M);
-          L = fmaf(lx, w, L);
-          float2 o = __ldcg(reinterpret_cast<const float2*>(part_o + ((part + h) * S + x) * kD + 2 * c2));
-          a0 = fmaf(o.x, w, a0);
-          a1 = fmaf(o.y, w, a1);
-        }
-      }
-      float inv = L > 0.f ? 1.f / L : 0.f;
-      *reinterpret_cast<uint32_t*>(out + (part + h) * kD + 2 * c2) = pack_bf2(a0 * inv, a1 * inv);
-      if (c2 == 0 && lse != nullptr)
-        lse[part + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-    }
-  }
-  if (tid == 0) ticket[(long long)b * Hkv + g] = 0u;  // ready for the next call
 }
 
-// ----------------------------------------------------------------- prefill
-
-constexpr int kPTile = 64;  // gathered rows per tile (16 per warp)
-
-template <int G>
-__global__ void __launch_bounds__(128)
-attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
-                    const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
-                    const int32_t* __restrict__ count, int T, int Tk_max, int Hq, int Hkv, int k,
-                    float qscale, uint16_t* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem);          // [16][kLds]
-  uint16_t* sK = sQ + 16 * kLds;                              // [2][kPTile][kLds]
-  uint16_t* sV = sK + 2 * kPTile * kLds;                      // [2][kPTile][kLds]
-
-  const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long tok = (long long)b * T + t;
-  int cnt = count[tok];
-  cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
-  const int32_t* irow = idx + tok * k;
-  const int ntiles = (cnt + kPTile - 1) / kPTile;
-
-  auto load_tile = [&](int it, int stage) {
-    const int r = tid >> 1, h = tid & 1;
-    const int i = it * kPTile + r;
-    const bool v = i < cnt;
-    const int j = v ? clamp_row(irow[i], Tk_max) : 0;
-    const long long off = (((long long)b * Tk_max + j) * Hkv + g) * kD;
-    uint16_t* dk = sK + (stage * kPTile + r) * kLds;
-    uint16_t* dv = sV + (stage * kPTile + r) * kLds;
-#pragma unroll
-    for (int c = h * 8; c < h * 8 + 8; ++c) {
-      cp_async16(dk + c * 8, kc + off + c * 8, v);
-      cp_async16(dv + c * 8, vc + off + c * 8, v);
-    }
-  };
-
-  // Q (G heads, zero padded to 16 rows)
-  for (int e = tid; e < 16 * 16; e += 128) {
-    int h = e >> 4, c = e & 15;
-    bool v = h < G;
-    cp_async16(sQ + h * kLds + c * 8, q + ((tok * Hq) + g * G + (v ? h : 0)) * kD + c * 8, v);
-  }
-  if (ntiles > 0) load_tile(0, 0);
-  cp_async_commit();
-
-  float o[16][4];
+// Online-softmax attention of the 16 (padded) query rows in sQ over the
+// gathered rows [begin, end) of irow.  Leaves per-warp partials in acc
+// (rows gq and gq+8 of the M side for this lane).
+__device__ __forceinline__ void attn_tiles(unsigned char* smem, const uint16_t* __restrict__ kc,
+                                           const uint16_t* __restrict__ vc,
+                                           const int32_t* __restrict__ irow, int begin, int end,
+                                           long long head_base, long long row_elems, int Tk_max,
+                                           float qscale, TileAcc& acc) {
+  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* sK = reinterpret_cast<uint16_t*>(smem + kSmemQ);
+  uint16_t* sV = sK + 2 * kTile * kLds;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tg = lane & 3;
 #pragma unroll
   for (int i = 0; i < 16; ++i)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+    for (int e = 0; e < 4; ++e) acc.o[i][e] = 0.f;
+  acc.m[0] = acc.m[1] = -INFINITY;
+  acc.l[0] = acc.l[1] = 0.f;
+  const int ntiles = end > begin ? (end - begin + kTile - 1) / kTile : 0;
+  if (ntiles > 0) gather_tile(sK, sV, kc, vc, irow, begin, end, head_base, row_elems, Tk_max);
+  cp_async_commit();
   uint32_t qa[8][4];
-  const int gq = lane >> 2, tg = lane & 3;
-
   for (int it = 0; it < ntiles; ++it) {
     const int stage = it & 1;
-    if (it + 1 < ntiles) load_tile(it + 1, stage ^ 1);
+    if (it + 1 < ntiles)
+      gather_tile(sK + (stage ^ 1) * kTile * kLds, sV + (stage ^ 1) * kTile * kLds, kc, vc, irow,
+                  begin + (it + 1) * kTile, end, head_base, row_elems, Tk_max);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
@@ -291,8 +109,8 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
         ldmatrix_x4(qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3],
                     sQ + (lane & 15) * kLds + kk * 16 + (lane >> 4) * 8);
     }
-    const uint16_t* tK = sK + (stage * kPTile + warp * 16) * kLds;
-    const uint16_t* tV = sV + (stage * kPTile + warp * 16) * kLds;
+    const uint16_t* tK = sK + (stage * kTile + warp * 16) * kLds;
+    const uint16_t* tV = sV + (stage * kTile + warp * 16) * kLds;
     float sc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -306,15 +124,14 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
       mma_bf16_16816(sc[0], qa[kk], b0, b1);
       mma_bf16_16816(sc[1], qa[kk], b2, b3);
     }
-    // mask rows past the count, scale into the log2 domain
-    const int rbase = it * kPTile + warp * 16;
+    const int rbase = begin + it * kTile + warp * 16;
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        int row = rbase + nt * 8 + tg * 2 + (e & 1);
-        float z = row < cnt ? sc[nt][e] * qscale : -INFINITY;
+        const int row = rbase + nt * 8 + tg * 2 + (e & 1);
+        const float z = row < end ? sc[nt][e] * qscale : -INFINITY;
         sc[nt][e] = z;
         mx[e >> 1] = fmaxf(mx[e >> 1], z);
       }
@@ -324,10 +141,10 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
       float v = mx[hh];
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-      float mnew = fmaxf(m_r[hh], v);
-      float muse = mnew == -INFINITY ? 0.f : mnew;
-      alpha[hh] = exp2f(m_r[hh] - muse);
-      m_r[hh] = mnew;
+      const float mnew = fmaxf(acc.m[hh], v);
+      const float muse = mnew == -INFINITY ? 0.f : mnew;
+      alpha[hh] = exp2f(acc.m[hh] - muse);
+      acc.m[hh] = mnew;
       mx[hh] = muse;
     }
     float rs[2] = {0.f, 0.f};
@@ -335,21 +152,23 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float p = exp2f(sc[nt][e] - mx[e >> 1]);
-        sc[nt][e] = p;
-        rs[e >> 1] += p;
+        const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+        sc[nt][e] = pv;
+        rs[e >> 1] += pv;
       }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float v = rs[hh];
       v += __shfl_xor_sync(0xffffffffu, v, 1);
       v += __shfl_xor_sync(0xffffffffu, v, 2);
-      l_r[hh] = l_r[hh] * alpha[hh] + v;
+      acc.l[hh] = acc.l[hh] * alpha[hh] + v;
     }
 #pragma unroll
     for (int dt = 0; dt < 16; ++dt) {
-      o[dt][0] *= alpha[0]; o[dt][1] *= alpha[0];
-      o[dt][2] *= alpha[1]; o[dt][3] *= alpha[1];
+      acc.o[dt][0] *= alpha[0];
+      acc.o[dt][1] *= alpha[0];
+      acc.o[dt][2] *= alpha[1];
+      acc.o[dt][3] *= alpha[1];
     }
     uint32_t pa[4];
     pa[0] = pack_bf2(sc[0][0], sc[0][1]);
@@ -361,97 +180,178 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
       const int mtx = lane >> 3;
       uint32_t b0, b1, b2, b3;
       ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * kLds + (dt + (mtx >> 1)) * 8);
-      mma_bf16_16816(o[dt], pa, b0, b1);
-      mma_bf16_16816(o[dt + 1], pa, b2, b3);
+      mma_bf16_16816(acc.o[dt], pa, b0, b1);
+      mma_bf16_16816(acc.o[dt + 1], pa, b2, b3);
     }
     __syncthreads();
   }
   cp_async_wait<0>();
   __syncthreads();
+}
 
-  // Merge the 4 warps: smem reuse of the K/V stages.
-  float* mo = reinterpret_cast<float*>(sK);       // [4][16][kD]
-  float* mm = mo + 4 * 16 * kD;                   // [4][16][2]
+// Loads the G query heads of one token into sQ (rows >= G zero).
+__device__ __forceinline__ void load_q(unsigned char* smem, const uint16_t* __restrict__ qh, int G) {
+  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem);
+  for (int e = threadIdx.x; e < 16 * 16; e += 128) {
+    const int h = e >> 4, c = e & 15;
+    const bool v = h < G;
+    cp_async16(sQ + h * kLds + c * 8, qh + (v ? h : 0) * kD + c * 8, v);
+  }
+}
+
+// Writes the 4 warps' partials to smem: mo[4][16][kD], mm[4][16][2].
+__device__ __forceinline__ void stash_warps(unsigned char* smem, const TileAcc& acc) {
+  float* mo = reinterpret_cast<float*>(smem + kSmemQ);
+  float* mm = mo + 4 * 16 * kD;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tg = lane & 3;
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) {
-    int d0 = dt * 8 + tg * 2;
-    *reinterpret_cast<float2*>(mo + ((warp * 16) + gq) * kD + d0) = make_float2(o[dt][0], o[dt][1]);
-    *reinterpret_cast<float2*>(mo + ((warp * 16) + gq + 8) * kD + d0) = make_float2(o[dt][2], o[dt][3]);
+    const int d0 = dt * 8 + tg * 2;
+    *reinterpret_cast<float2*>(mo + (warp * 16 + gq) * kD + d0) = make_float2(acc.o[dt][0], acc.o[dt][1]);
+    *reinterpret_cast<float2*>(mo + (warp * 16 + gq + 8) * kD + d0) = make_float2(acc.o[dt][2], acc.o[dt][3]);
   }
   if (tg == 0) {
-    mm[((warp * 16) + gq) * 2] = m_r[0];
-    mm[((warp * 16) + gq) * 2 + 1] = l_r[0];
-    mm[((warp * 16) + gq + 8) * 2] = m_r[1];
-    mm[((warp * 16) + gq + 8) * 2 + 1] = l_r[1];
+    mm[(warp * 16 + gq) * 2] = acc.m[0];
+    mm[(warp * 16 + gq) * 2 + 1] = acc.l[0];
+    mm[(warp * 16 + gq + 8) * 2] = acc.m[1];
+    mm[(warp * 16 + gq + 8) * 2 + 1] = acc.l[1];
   }
   __syncthreads();
-  const int d = tid;  // 128 threads <-> 128 dims
+}
+
+// Merge of the 4 warps for head h and dim d (thread = dim): returns the
+// unnormalised sum o, and M, L of the CTA's rows.
+__device__ __forceinline__ void merge_warps(const unsigned char* smem, int h, int d, float& M, float& L,
+                                            float& o) {
+  const float* mo = reinterpret_cast<const float*>(smem + kSmemQ);
+  const float* mm = mo + 4 * 16 * kD;
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[(w * 16 + h) * 2]);
+  L = 0.f;
+  o = 0.f;
+  if (M == -INFINITY) return;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float lw = mm[(w * 16 + h) * 2 + 1];
+    if (lw == 0.f) continue;
+    const float wt = exp2f(mm[(w * 16 + h) * 2] - M);
+    L = fmaf(lw, wt, L);
+    o = fmaf(mo[(w * 16 + h) * kD + d], wt, o);
+  }
+}
+
+// ----------------------------------------------------------------- prefill
+
+__global__ void __launch_bounds__(128)
+attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                    const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
+                    const int32_t* __restrict__ count, int T, int Tk_max, int Hq, int Hkv, int k,
+                    float qscale, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv;
+  const long long tok = (long long)b * T + t;
+  int cnt = count[tok];
+  cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
+  load_q(smem, q + (tok * Hq + (long long)g * G) * kD, G);
+  TileAcc acc;
+  attn_tiles(smem, kc, vc, idx + tok * k, 0, cnt, ((long long)b * Tk_max * Hkv + g) * kD,
+             (long long)Hkv * kD, Tk_max, qscale, acc);
+  stash_warps(smem, acc);
+  const int d = threadIdx.x;
   for (int h = 0; h < G; ++h) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[(w * 16 + h) * 2]);
-    float L = 0.f, a = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        float lw = mm[(w * 16 + h) * 2 + 1];
-        if (lw == 0.f) continue;
-        float wt = exp2f(mm[(w * 16 + h) * 2] - M);
-        L = fmaf(lw, wt, L);
-        a = fmaf(mo[(w * 16 + h) * kD + d], wt, a);
-      }
-    }
-    float v = L > 0.f ? a / L : 0.f;
-    out[(tok * Hq + g * G + h) * kD + d] = f2bf(v);
+    float M, L, o;
+    merge_warps(smem, h, d, M, L, o);
+    out[(tok * Hq + g * G + h) * kD + d] = f2bf(L > 0.f ? o / L : 0.f);
     if (d == 0 && lse != nullptr) lse[tok * Hq + g * G + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
   }
 }
 
-// -------------------------------------------------------------- dispatch
+// ------------------------------------------------------------------ decode
 
-int decode_rows_per_split(int B, int Hkv, int k) {
-  // Enough CTAs to cover 148 SMs about twice, rows a multiple of 32.
-  for (int R : {128, 64}) {
-    long long ctas = (long long)B * Hkv * ((k + R - 1) / R);
-    if (ctas >= 296) return R;
+__global__ void __launch_bounds__(128)
+attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                   const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
+                   const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k,
+                   int tiles_per_split, int S, float qscale, float* __restrict__ part_o,
+                   float* __restrict__ part_ml, unsigned* __restrict__ ticket,
+                   uint16_t* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int s_last;
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv;
+  int cnt = count[b];
+  cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
+  const int begin = min(cnt, s * tiles_per_split * kTile);
+  const int end = min(cnt, (s + 1) * tiles_per_split * kTile);
+  const long long head0 = (long long)b * Hq + (long long)g * G;  // first query head of the group
+  load_q(smem, q + head0 * kD, G);
+  TileAcc acc;
+  attn_tiles(smem, kc, vc, idx + (long long)b * k, begin, end, ((long long)b * Tk_max * Hkv + g) * kD,
+             (long long)Hkv * kD, Tk_max, qscale, acc);
+  stash_warps(smem, acc);
+  const int d = threadIdx.x;
+  if (S == 1) {
+    for (int h = 0; h < G; ++h) {
+      float M, L, o;
+      merge_warps(smem, h, d, M, L, o);
+      out[(head0 + h) * kD + d] = f2bf(L > 0.f ? o / L : 0.f);
+      if (d == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    return;
   }
-  return 32;
+  for (int h = 0; h < G; ++h) {
+    float M, L, o;
+    merge_warps(smem, h, d, M, L, o);
+    part_o[((head0 + h) * S + s) * kD + d] = o;
+    if (d == 0) {
+      part_ml[((head0 + h) * S + s) * 2] = M;
+      part_ml[((head0 + h) * S + s) * 2 + 1] = L;
+    }
+  }
+  // The last CTA of this (sequence, kv head) merges the S partials.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(ticket + (long long)b * Hkv + g, 1u);
+    s_last = prev == (unsigned)(S - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int h = 0; h < G; ++h) {
+    const float* ml = part_ml + (head0 + h) * S * 2;
+    float M = -INFINITY;
+    for (int x = 0; x < S; ++x) M = fmaxf(M, __ldcg(ml + 2 * x));
+    float L = 0.f, a = 0.f;
+    if (M != -INFINITY) {
+      for (int x = 0; x < S; ++x) {
+        const float mx = __ldcg(ml + 2 * x), lx = __ldcg(ml + 2 * x + 1);
+        if (lx == 0.f) continue;
+        const float w = exp2f(mx - M);
+        L = fmaf(lx, w, L);
+        a = fmaf(__ldcg(part_o + ((head0 + h) * S + x) * kD + d), w, a);
+      }
+    }
+    out[(head0 + h) * kD + d] = f2bf(L > 0.f ? a / L : 0.f);
+    if (d == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+  }
+  if (threadIdx.x == 0) ticket[(long long)b * Hkv + g] = 0u;  // ready for the next call
 }
 
-size_t decode_smem(int G, int R) {
-  int DS = 128 / R;
-  size_t f = (size_t)G * kD + (size_t)DS * G * R + 32;
-  return f * 4 + 2 * (size_t)R * kLds * 2;
-}
-
-template <int G>
-cudaError_t launch_decode_g(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
-                            const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,
-                            int Hkv, int k, float qscale, uint16_t* out, float* lse, float* po,
-                            float* pml, unsigned* ticket, int R, int S, cudaStream_t st) {
-  size_t smem = decode_smem(G, R);
-  cudaError_t e = ensure_dynamic_smem((const void*)attn_decode_kernel<G>, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(S, Hkv, B);
-  attn_decode_kernel<G><<<grid, 128, smem, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k, R, S,
-                                                 qscale, po, pml, ticket, out, lse);
-  return cudaGetLastError();
-}
-
-size_t prefill_smem() { return (size_t)(16 + 4 * kPTile) * kLds * 2; }
-
-template <int G>
-cudaError_t launch_prefill_g(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
-                             const int32_t* idx, const int32_t* count, int B, int T, int Tk_max,
-                             int Hq, int Hkv, int k, float qscale, uint16_t* out, float* lse,
-                             cudaStream_t st) {
-  size_t smem = prefill_smem();
-  cudaError_t e = ensure_dynamic_smem((const void*)attn_prefill_kernel<G>, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(T, Hkv, B);
-  attn_prefill_kernel<G><<<grid, 128, smem, st>>>(q, kc, vc, idx, count, T, Tk_max, Hq, Hkv, k,
-                                                  qscale, out, lse);
-  return cudaGetLastError();
+// Splits of the index list: enough CTAs for about 3 per SM, at least one
+// 64-row tile each.
+void decode_split(int B, int Hkv, int k, int* tiles_per_split, int* S) {
+  const int ntiles = (k + kTile - 1) / kTile;
+  const long long pairs = (long long)B * Hkv;
+  long long want = (3 * 148 + pairs - 1) / pairs;
+  if (want < 1) want = 1;
+  if (want > ntiles) want = ntiles;
+  int tps = (int)((ntiles + want - 1) / want);
+  *tiles_per_split = tps;
+  *S = (ntiles + tps - 1) / tps;
 }
 
 }  // namespace
@@ -460,11 +360,11 @@ static size_t align256a(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
   (void)D;
-  int R = decode_rows_per_split(B, Hkv, k);
-  int S = (k + R - 1) / R;
-  size_t po = align256a((size_t)B * Hq * S * kD * 4);
-  size_t pml = align256a((size_t)B * Hq * S * 2 * 4);
-  size_t tk = align256a((size_t)B * Hkv * 4);
+  int tps, S;
+  decode_split(B, Hkv, k, &tps, &S);
+  const size_t tk = align256a((size_t)B * Hkv * 4);
+  const size_t po = align256a((size_t)B * Hq * S * kD * 4);
+  const size_t pml = align256a((size_t)B * Hq * S * 2 * 4);
   return tk + po + pml;
 }
 
@@ -473,27 +373,20 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
                                int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,
                                cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
-  const int R = decode_rows_per_split(B, Hkv, k);
-  const int S = (k + R - 1) / R;
+  int tps, S;
+  decode_split(B, Hkv, k, &tps, &S);
   char* p = static_cast<char*>(ws);
   unsigned* ticket = reinterpret_cast<unsigned*>(p);
   p += align256a((size_t)B * Hkv * 4);
   float* po = reinterpret_cast<float*>(p);
   p += align256a((size_t)B * Hq * S * kD * 4);
   float* pml = reinterpret_cast<float*>(p);
-  cudaError_t e = cudaMemsetAsync(ticket, 0, (size_t)B * Hkv * 4, st);
-  if (e != cudaSuccess) return e;
-  const float qscale = scale * kLog2e;
-  const int G = Hq / Hkv;
-  switch (G) {
-#define SA_DEC_CASE(n) \
-  case n: return launch_decode_g<n>(q, kc, vc, idx, count, B, Tk_max, Hq, Hkv, k, qscale, out, lse, po, pml, ticket, R, S, st);
-    SA_DEC_CASE(1) SA_DEC_CASE(2) SA_DEC_CASE(3) SA_DEC_CASE(4) SA_DEC_CASE(5) SA_DEC_CASE(6)
-    SA_DEC_CASE(7) SA_DEC_CASE(8) SA_DEC_CASE(9) SA_DEC_CASE(10) SA_DEC_CASE(11) SA_DEC_CASE(12)
-    SA_DEC_CASE(13) SA_DEC_CASE(14) SA_DEC_CASE(15) SA_DEC_CASE(16)
-#undef SA_DEC_CASE
-    default: return cudaErrorInvalidValue;
-  }
+  cudaError_t e;
+  if ((e = ensure_dynamic_smem((const void*)attn_decode_kernel, kSmemTotal)) != cudaSuccess) return e;
+  dim3 grid(S, Hkv, B);
+  attn_decode_kernel<<<grid, 128, kSmemTotal, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k, tps, S,
+                                                    scale * kLog2e, po, pml, ticket, out, lse);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
@@ -501,17 +394,12 @@ cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uin
                                 int Hq, int Hkv, int k, float scale, uint16_t* out, float* lse,
                                 cudaStream_t st) {
   if (B <= 0 || T <= 0) return cudaSuccess;
-  const float qscale = scale * kLog2e;
-  const int G = Hq / Hkv;
-  switch (G) {
-#define SA_PRE_CASE(n) \
-  case n: return launch_prefill_g<n>(q, kc, vc, idx, count, B, T, Tk_max, Hq, Hkv, k, qscale, out, lse, st);
-    SA_PRE_CASE(1) SA_PRE_CASE(2) SA_PRE_CASE(3) SA_PRE_CASE(4) SA_PRE_CASE(5) SA_PRE_CASE(6)
-    SA_PRE_CASE(7) SA_PRE_CASE(8) SA_PRE_CASE(9) SA_PRE_CASE(10) SA_PRE_CASE(11) SA_PRE_CASE(12)
-    SA_PRE_CASE(13) SA_PRE_CASE(14) SA_PRE_CASE(15) SA_PRE_CASE(16)
-#undef SA_PRE_CASE
-    default: return cudaErrorInvalidValue;
-  }
+  cudaError_t e = ensure_dynamic_smem((const void*)attn_prefill_kernel, kSmemTotal);
+  if (e != cudaSuccess) return e;
+  dim3 grid(T, Hkv, B);
+  attn_prefill_kernel<<<grid, 128, kSmemTotal, st>>>(q, kc, vc, idx, count, T, Tk_max, Hq, Hkv, k,
+                                                     scale * kLog2e, out, lse);
+  return cudaGetLastError();
 }
 
 }  // namespace sa

@@ -7,24 +7,26 @@
 // position, emitted in ascending position order.
 //
 // Kernels
-//   score_decode_kernel   one query per sequence; streams the indexer-key
-//                         cache with coalesced 16-byte loads (d/8 lanes per
-//                         row), writes order-preserving 32-bit score keys and
-//                         a 4096-bin histogram of each key's top 12 bits.
-//   collect_kernel        finds, from the histogram, the bin holding the
-//                         k-th largest key and appends every key in that bin
-//                         or above to a per-row candidate list (warp-
-//                         aggregated atomics; order of appends is irrelevant).
-//   finish_kernel         one CTA per row: exact radix select (8-bit digits,
-//                         warp-aggregated shared-memory histograms) of the
-//                         k-th key, then of the tie positions, then emission
-//                         in ascending position order (ordered block
-//                         compaction in direct mode, bitonic sort of the <=k
-//                         chosen candidates in candidate mode).  Also expands
-//                         chosen gist chunks into their cache rows.
-//   score_prefill_kernel  causal Q_idx K_idx^T tile product (tensor cores,
-//                         bf16 in, fp32 accumulate) writing score keys of one
-//                         block of query rows into a slab for finish_kernel.
+//   score_decode_kernel  one query per sequence.  The indexer-key cache is
+//       streamed with 16-byte loads straight into mma.sync B fragments: a dot
+//       product is invariant to the order of its terms, so lane (g, t) of a
+//       warp loads whole 16-byte chunks 4j+t of key row g and the query
+//       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
+//       keys (the query is row 0 of the 16-row A side).  Writes the order-
+//       preserving 32-bit score key of every candidate and a 4096-bin
+//       histogram of each key's top 12 bits.
+//   collect_kernel       (rows longer than one CTA can scan) finds, from the
+//       histogram, the bin holding the k-th largest key and appends every key
+//       in that bin or above to a per-row candidate list (one atomic per CTA).
+//   finish_kernel        one CTA per row: gathers the row's candidates into
+//       shared memory (histogram-filtered scan of the row, the collected
+//       list, or the whole row), runs an exact radix select (8-bit digits,
+//       warp-aggregated shared histograms) of the k-th key and of the tie
+//       positions, then emits in ascending position order through a position
+//       bitmap and popcount prefix sums (bitonic sort for rows beyond the
+//       bitmap's reach).  Also expands chosen gist chunks into cache rows and
+//       returns the histogram and counters of its row to zero.
+// The prefill scores come from the tcgen05 kernel in index_tc.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,6 +38,9 @@ namespace {
 
 constexpr int kScoreThreads = 256;
 constexpr int kFinThreads = 1024;
+constexpr int kSmemCand = 8192;          // candidates held in shared memory
+constexpr int kBitmapMax = 1 << 18;      // rows up to this length emit through a bitmap
+constexpr int kBitmapWords = kBitmapMax / 32;
 
 __device__ __forceinline__ int row_len(const int32_t* kv_len, int b, int Tk) {
   if (kv_len == nullptr) return Tk;
@@ -65,9 +70,8 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
                     int Tk, int q_pos0, const int32_t* __restrict__ kv_len,
                     uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist,
                     int chunk) {
-  constexpr int LPR = D / 8;        // lanes per row, 16 bytes each
-  constexpr int RPW = 32 / LPR;     // rows per warp load
-  constexpr int UNROLL = 8;
+  constexpr int J = D / 32;          // 16-byte chunks per lane per key row
+  constexpr int U = 2;               // 8-row tiles per warp iteration
   constexpr int WARPS = kScoreThreads / 32;
   __shared__ uint32_t sh[kHistBins];
 
@@ -77,38 +81,58 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
   if (r0 >= n) return;
   const int r1 = min(r0 + chunk, n);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int sub = lane / LPR, slot = lane % LPR;
+  const int g = lane >> 2, tg = lane & 3;
 
   if (hist != nullptr) {
     for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
     __syncthreads();
   }
-  float qf[8];
-  {
-    uint4 qv = *reinterpret_cast<const uint4*>(q + (long long)b * D + slot * 8);
-    qf[0] = bf_lo(qv.x); qf[1] = bf_hi(qv.x); qf[2] = bf_lo(qv.y); qf[3] = bf_hi(qv.y);
-    qf[4] = bf_lo(qv.z); qf[5] = bf_hi(qv.z); qf[6] = bf_lo(qv.w); qf[7] = bf_hi(qv.w);
+  // A fragments: the query is row 0 of the 16-row A side, so only lanes with
+  // g == 0 hold data.  Chunk 4j+t (dims 8(4j+t) .. +7) feeds two k-steps:
+  // words x, y as (a0, a2) of the first and z, w as (a0, a2) of the second.
+  uint32_t qe[J][2], qo[J][2];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (g == 0) v = *reinterpret_cast<const uint4*>(q + (long long)b * D + (4 * j + tg) * 8);
+    qe[j][0] = v.x; qe[j][1] = v.y;
+    qo[j][0] = v.z; qo[j][1] = v.w;
   }
   const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
   uint32_t* kout = keys + (long long)b * ld;
 
-  for (int base = r0 + warp * RPW * UNROLL; base < r1; base += WARPS * RPW * UNROLL) {
-    uint4 v[UNROLL];
+  for (int base = r0 + warp * 8 * U; base < r1; base += WARPS * 8 * U) {
+    uint4 v[U][J];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      int row = base + u * RPW + sub;
-      v[u] = row < r1 ? __ldg(kb + (long long)row * LPR + slot) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < U; ++u) {
+      const int row = base + u * 8 + g;
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+        v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      float s = dot8(v[u], qf);
+    for (int u = 0; u < U; ++u) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      int row = base + u * RPW + sub;
-      if (slot == 0 && row < r1) {
-        uint32_t key = score_key(s);
-        kout[row] = key;
-        if (hist != nullptr) atomicAdd(&sh[key >> (32 - kHistBits)], 1u);
+      for (int j = 0; j < J; ++j) {
+        const uint32_t a_even[4] = {qe[j][0], 0u, qe[j][1], 0u};
+        const uint32_t a_odd[4] = {qo[j][0], 0u, qo[j][1], 0u};
+        mma_bf16_16816(c, a_even, v[u][j].x, v[u][j].y);
+        mma_bf16_16816(c, a_odd, v[u][j].z, v[u][j].w);
+      }
+      // row 0 of C: lanes 0..3 hold the scores of tile rows 2t and 2t+1
+      if (g == 0) {
+        const int row = base + u * 8 + 2 * tg;
+        const uint32_t k0 = score_key(c[0]), k1 = score_key(c[1]);
+        if (row + 1 < r1) {
+          *reinterpret_cast<uint2*>(kout + row) = make_uint2(k0, k1);
+        } else if (row < r1) {
+          kout[row] = k0;
+        }
+        if (hist != nullptr) {
+          if (row < r1) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
+          if (row + 1 < r1) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
+        }
       }
     }
   }
@@ -116,91 +140,112 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     __syncthreads();
     uint32_t* hg = hist + (long long)b * kHistBins;
     for (int i = tid; i < kHistBins; i += kScoreThreads) {
-      uint32_t c = sh[i];
-      if (c) atomicAdd(hg + i, c);
+      const uint32_t cnt = sh[i];
+      if (cnt) atomicAdd(hg + i, cnt);
     }
   }
 }
 
-// ------------------------------------------------------------------ collect
+// ------------------------------------------------------------ block scans
 
-// Exclusive prefix sum over the 256 threads of a block; returns the total.
-__device__ __forceinline__ uint32_t block_scan_256(uint32_t v, uint32_t* s_warp, uint32_t& excl) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
+// s_warp needs 33 words.  Returns this thread's prefix; `total` the sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   uint32_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) s_warp[warp] = x;
   __syncthreads();
-  uint32_t wsum = 0, total = 0;
+  if (warp == 0) {
+    const uint32_t wv = lane < nw ? s_warp[lane] : 0u;
+    uint32_t y = wv;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    uint32_t c = s_warp[w];
-    if (w < warp) wsum += c;
-    total += c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += z;
+    }
+    if (lane < nw) s_warp[lane] = y - wv;
+    if (lane == 31) s_warp[32] = y;
   }
-  excl = wsum + x - v;
-  return total;
+  __syncthreads();
+  const uint32_t r = s_warp[warp] + x - v;
+  total = s_warp[32];
+  __syncthreads();
+  return r;
 }
+
+// Bin of the K-th largest key in a 4096-bin histogram (bins in key order):
+// s_out[0] = bin, s_out[1] = keys in the bins above it.
+__device__ __forceinline__ void hist_threshold(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
+                                               uint32_t* s_out) {
+  const int per = kHistBins / blockDim.x;  // 16 (256 threads) or 4 (1024 threads)
+  uint32_t loc = 0;
+  for (int j = 0; j < per; ++j) loc += h[kHistBins - 1 - (threadIdx.x * per + j)];
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(loc, s_warp, total);
+  if (excl < K && K <= excl + loc) {
+    uint32_t cum = excl;
+    for (int j = 0; j < per; ++j) {
+      const uint32_t c = h[kHistBins - 1 - (threadIdx.x * per + j)];
+      if (cum + c >= K) {
+        s_out[0] = kHistBins - 1 - (threadIdx.x * per + j);
+        s_out[1] = cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ collect
+
+constexpr int kCollectPer = 16;   // keys per thread of collect_kernel
 
 __global__ void __launch_bounds__(256)
 collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* __restrict__ hist,
                int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int k, int chunk,
                uint32_t* __restrict__ cand_cnt, uint32_t* __restrict__ cand_key,
                uint32_t* __restrict__ cand_pos) {
-  __shared__ uint32_t s_warp[8];
-  __shared__ uint32_t s_bin;
+  __shared__ uint32_t s_warp[33];
+  __shared__ uint32_t s_thr[2];
+  __shared__ uint32_t s_base;
   const int b = blockIdx.y;
   const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
   const int r0 = blockIdx.x * chunk;
   if (r0 >= n) return;
   const int r1 = min(r0 + chunk, n);
   const uint32_t K = (uint32_t)min(k, n);
-  const int tid = threadIdx.x, lane = tid & 31;
-
-  // Bin of the K-th largest key: thread i owns the 16 bins counted from the top.
-  const uint32_t* h = hist + (long long)b * kHistBins;
-  constexpr int PER = kHistBins / 256;
-  uint32_t hv[PER];
-  uint32_t loc = 0;
-#pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    hv[j] = h[kHistBins - 1 - (tid * PER + j)];
-    loc += hv[j];
-  }
-  uint32_t excl;
-  block_scan_256(loc, s_warp, excl);
-  if (excl < K && K <= excl + loc) {
-    uint32_t cum = excl;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      if (cum + hv[j] >= K) { s_bin = kHistBins - 1 - (tid * PER + j); break; }
-      cum += hv[j];
-    }
-  }
-  __syncthreads();
-  const uint32_t bin = s_bin;
+  hist_threshold(hist + (long long)b * kHistBins, K, s_warp, s_thr);
+  const uint32_t bin = s_thr[0];
 
   const uint32_t* row = keys + (long long)b * ld;
+  const int i0 = r0 + threadIdx.x * kCollectPer;
+  uint32_t kv[kCollectPer];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < kCollectPer; ++j) {
+    const int i = i0 + j;
+    kv[j] = i < r1 ? row[i] : 0u;
+    mine += (i < r1 && (kv[j] >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+  }
+  uint32_t total;
+  const uint32_t off = block_excl_scan(mine, s_warp, total);
+  if (threadIdx.x == 0) s_base = total ? atomicAdd(cand_cnt + b, total) : 0u;
+  __syncthreads();
+  uint32_t o = s_base + off;
   uint32_t* ck = cand_key + (long long)b * kCandCap;
   uint32_t* cp = cand_pos + (long long)b * kCandCap;
-  for (int i0 = r0; i0 < r1; i0 += 256) {
-    int i = i0 + tid;
-    uint32_t key = i < r1 ? row[i] : 0u;
-    bool take = i < r1 && (key >> (32 - kHistBits)) >= bin;
-    unsigned m = __ballot_sync(0xffffffffu, take);
-    if (m) {
-      int leader = __ffs(m) - 1;
-      uint32_t base = 0;
-      if (lane == leader) base = atomicAdd(cand_cnt + b, (uint32_t)__popc(m));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (take) {
-        uint32_t s = base + __popc(m & lanemask_lt());
-        if (s < (uint32_t)kCandCap) { ck[s] = key; cp[s] = (uint32_t)i; }
-      }
+#pragma unroll
+  for (int j = 0; j < kCollectPer; ++j) {
+    const int i = i0 + j;
+    if (i < r1 && (kv[j] >> (32 - kHistBits)) >= bin) {
+      if (o < (uint32_t)kCandCap) { ck[o] = kv[j]; cp[o] = (uint32_t)i; }
+      ++o;
     }
   }
 }
@@ -209,40 +254,41 @@ collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* 
 
 struct FinishSmem {
   uint32_t hist[256];
-  uint32_t wcnt[32];
-  uint32_t sel_pos[kMaxK];
-  uint32_t sel_key[kMaxK];
-  uint32_t digit, above, bnd_count, total, nsel;
+  uint32_t swarp[33];
+  uint32_t thr[2];
+  uint32_t digit, above, bnd_count, ncand, total;
+  uint32_t ckey[kSmemCand];
+  uint32_t cpos[kSmemCand];
+  uint32_t bits[kBitmapWords];   // also the sort buffer (positions) for long rows
+  uint32_t wpre[kBitmapWords];   // also the sort buffer (keys) for long rows
 };
 
-// Adds 1 to hist[digit] for every active lane, aggregated over equal digits.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool active) {
-  unsigned act = __ballot_sync(0xffffffffu, active);
+__device__ __forceinline__ void hist_add(uint32_t* h, uint32_t digit, bool active) {
+  const unsigned act = __ballot_sync(0xffffffffu, active);
   if (!active) return;
-  unsigned peers = __match_any_sync(act, digit);
-  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(hist + digit, (uint32_t)__popc(peers));
+  const unsigned peers = __match_any_sync(act, digit);
+  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(h + digit, (uint32_t)__popc(peers));
 }
 
 // Warp 0 locates the digit holding the kk-th element, searching from the
-// top bin down (desc) or the bottom bin up (asc).  Writes digit and the
-// count strictly before it in search order.
+// top bin down (desc) or the bottom bin up (asc).
 __device__ __forceinline__ void find_digit(FinishSmem& s, uint32_t kk, bool desc) {
   if (threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
   uint32_t c[8], loc = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    int bin = desc ? 255 - (lane * 8 + j) : lane * 8 + j;
+    const int bin = desc ? 255 - (lane * 8 + j) : lane * 8 + j;
     c[j] = s.hist[bin];
     loc += c[j];
   }
   uint32_t x = loc;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  uint32_t excl = x - loc;
+  const uint32_t excl = x - loc;
   if (excl < kk && kk <= excl + loc) {
     uint32_t cum = excl;
 #pragma unroll
@@ -258,18 +304,18 @@ __device__ __forceinline__ void find_digit(FinishSmem& s, uint32_t kk, bool desc
   }
 }
 
-// Item accessor: candidate lists (explicit positions) or a whole row of keys.
+// Items: keys with explicit positions, or a row of keys (position = index).
 struct Items {
   const uint32_t* key;
-  const uint32_t* pos;  // null: position = index
+  const uint32_t* pos;
   int n;
   __device__ __forceinline__ uint32_t k(int i) const { return key[i]; }
   __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i] : (uint32_t)i; }
 };
 
-// Exact selection of the K largest keys (ties by lower position) among `it`.
-// Leaves in smem: masked-key threshold (prefix under pmask) and, for the
-// boundary set, the largest selected position (pmax).
+// Exact selection of the K largest keys (ties: lower position) among `it`:
+// on return an item is chosen iff (key & pmask) > prefix, or it equals
+// prefix under pmask and its position is <= pmax.
 __device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uint32_t& prefix,
                                  uint32_t& pmask, uint32_t& pmax) {
   const int tid = threadIdx.x;
@@ -281,9 +327,9 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uin
     for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
     __syncthreads();
     for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-      int i = i0 + tid;
-      uint32_t key = i < it.n ? it.k(i) : 0u;
-      bool act = i < it.n && (key & pmask) == prefix;
+      const int i = i0 + tid;
+      const uint32_t key = i < it.n ? it.k(i) : 0u;
+      const bool act = i < it.n && (key & pmask) == prefix;
       hist_add(s.hist, (key >> shift) & 255u, act);
     }
     __syncthreads();
@@ -294,17 +340,17 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uin
     pmask |= 255u << shift;
     bnd = s.bnd_count;
     __syncthreads();
-    if (bnd == kk) break;  // every item of the boundary prefix is selected
+    if (bnd == kk) break;  // every item of the boundary prefix is chosen
   }
   pmax = 0xFFFFFFFFu;
   if (bnd == kk) return;
-  // Exact key ties: keep the kk lowest positions among key == prefix.
+  // exact key ties: keep the kk lowest positions among key == prefix
   uint32_t pp = 0, pm = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
     __syncthreads();
     for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-      int i = i0 + tid;
+      const int i = i0 + tid;
       bool act = false;
       uint32_t p = 0;
       if (i < it.n && it.k(i) == prefix) {
@@ -319,9 +365,9 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uin
     kk -= s.above;
     pp |= s.digit << shift;
     pm |= 255u << shift;
-    uint32_t c = s.bnd_count;
+    const uint32_t c = s.bnd_count;
     __syncthreads();
-    if (c == kk) {  // take every tie whose position prefix is <= pp
+    if (c == kk) {
       pmax = pp | ~pm;
       return;
     }
@@ -329,123 +375,192 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uin
   pmax = pp;
 }
 
-__device__ __forceinline__ bool is_selected(uint32_t key, uint32_t pos, uint32_t prefix,
-                                            uint32_t pmask, uint32_t pmax) {
-  uint32_t m = key & pmask;
+__device__ __forceinline__ bool is_selected(uint32_t key, uint32_t pos, uint32_t prefix, uint32_t pmask,
+                                            uint32_t pmax) {
+  const uint32_t m = key & pmask;
   return m > prefix || (m == prefix && pos <= pmax);
 }
 
-__global__ void __launch_bounds__(kFinThreads)
-finish_kernel(RowWorkspace w, bool candidates, int rows_per_batch, int t0, int Tq, int Tk,
-              int q_pos0, const int32_t* __restrict__ kv_len, int k, FinishOut out) {
+// Appends item (key, pos) to the shared candidate list (warp-aggregated).
+__device__ __forceinline__ void push_cand(FinishSmem& s, bool take, uint32_t key, uint32_t pos) {
+  const unsigned m = __ballot_sync(0xffffffffu, take);
+  if (!m) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(&s.ncand, (uint32_t)__popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (take) {
+    const uint32_t o = base + __popc(m & lanemask_lt());
+    if (o < (uint32_t)kSmemCand) { s.ckey[o] = key; s.cpos[o] = pos; }
+  }
+}
+
+// Writes the chosen item with rank `slot` (0-based, ascending position).
+__device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int b, uint32_t slot,
+                                     uint32_t pos, uint32_t key) {
+  if (out.rows == nullptr) {
+    out.idx[o_idx + slot] = (int32_t)pos;
+    if (out.score) out.score[o_idx + slot] = key_score(key);
+  } else {
+    const int stride = out.chunk_len + 1;
+    int32_t* rows = out.rows + (long long)b * out.rows_stride + (long long)slot * stride;
+    for (int r = 0; r < stride; ++r) rows[r] = (int32_t)pos * stride + r;
+    if (out.chunks) out.chunks[o_idx + slot] = (int32_t)pos;
+  }
+}
+
+__global__ void __launch_bounds__(kFinThreads, 1)
+finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+              const int32_t* __restrict__ kv_len, int k, FinishOut out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   FinishSmem& s = *reinterpret_cast<FinishSmem*>(smem_raw);
   const int r = blockIdx.x;
   const int b = r / rows_per_batch;
   const int t = t0 + r % rows_per_batch;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
   const uint32_t K = (uint32_t)min(k, n);
+  const uint32_t* row = w.keys + (long long)r * w.ld;
+  if (tid == 0) { s.ncand = 0; s.total = 0; }
+  __syncthreads();
 
+  // ---- gather candidates into shared memory
   Items it;
-  bool direct = true;
-  if (candidates) {
-    uint32_t m = w.cand_cnt[r];
-    if (m <= (uint32_t)kCandCap) {
-      it.key = w.cand_key + (long long)r * kCandCap;
-      it.pos = w.cand_pos + (long long)r * kCandCap;
-      it.n = (int)m;
-      direct = false;
+  it.key = row;
+  it.pos = nullptr;
+  it.n = n;
+  bool in_smem = false;
+  if (K > 0) {
+    if (mode == kFinishHistScan) {
+      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
+      const uint32_t bin = s.thr[0];
+      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
+        const int i = i0 + tid * 4;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i + 3 < n) {
+          v = *reinterpret_cast<const uint4*>(row + i);
+        } else {
+          if (i < n) v.x = row[i];
+          if (i + 1 < n) v.y = row[i + 1];
+          if (i + 2 < n) v.z = row[i + 2];
+        }
+        const uint32_t kk4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool take = i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin;
+          push_cand(s, take, kk4[j], (uint32_t)(i + j));
+        }
+      }
+      __syncthreads();
+      in_smem = s.ncand <= (uint32_t)kSmemCand;
+    } else if (mode == kFinishCandList) {
+      const uint32_t m = w.cand_cnt[r];
+      if (m <= (uint32_t)kSmemCand) {
+        const uint32_t* ck = w.cand_key + (long long)r * kCandCap;
+        const uint32_t* cp = w.cand_pos + (long long)r * kCandCap;
+        for (uint32_t i = tid; i < m; i += kFinThreads) { s.ckey[i] = ck[i]; s.cpos[i] = cp[i]; }
+        if (tid == 0) s.ncand = m;
+        in_smem = true;
+      } else if (m <= (uint32_t)kCandCap) {
+        it.key = w.cand_key + (long long)r * kCandCap;
+        it.pos = w.cand_pos + (long long)r * kCandCap;
+        it.n = (int)m;
+      }
+      __syncthreads();
+    } else {  // kFinishDirect: every candidate of the row
+      if (n <= kSmemCand) {
+        for (int i = tid; i < n; i += kFinThreads) { s.ckey[i] = row[i]; s.cpos[i] = (uint32_t)i; }
+        if (tid == 0) s.ncand = (uint32_t)n;
+        in_smem = true;
+      }
+      __syncthreads();
     }
-  }
-  if (direct) {
-    it.key = w.keys + (long long)r * w.ld;
-    it.pos = nullptr;
-    it.n = n;
+    if (in_smem) {
+      it.key = s.ckey;
+      it.pos = s.cpos;
+      it.n = (int)s.ncand;
+    }
   }
 
   uint32_t prefix = 0, pmask = 0, pmax = 0;
   if (K > 0) select_threshold(s, it, K, prefix, pmask, pmax);
 
-  // Emit the chosen (position, key) pairs into shared memory.
-  if (tid == 0) { s.total = 0; s.nsel = 0; }
-  __syncthreads();
+  const long long o_idx = ((long long)b * Tq + t) * (long long)k;
   if (K > 0) {
-    if (direct) {
-      // Items are in position order: ordered block compaction.
-      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-        int i = i0 + tid;
-        uint32_t key = i < it.n ? it.k(i) : 0u;
-        bool sel = i < it.n && is_selected(key, (uint32_t)i, prefix, pmask, pmax);
-        unsigned m = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) s.wcnt[warp] = __popc(m);
-        __syncthreads();
-        if (warp == 0) {
-          uint32_t c = s.wcnt[lane], x = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-          }
-          s.wcnt[lane] = x - c;
-          if (lane == 31) s.nsel = x;
+    if (n <= kBitmapMax) {
+      // ---- emission through a position bitmap
+      const int W = (n + 31) >> 5;
+      for (int i = tid; i < W; i += kFinThreads) s.bits[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < it.n; i += kFinThreads) {
+        const uint32_t key = it.k(i), pos = it.p(i);
+        if (is_selected(key, pos, prefix, pmask, pmax)) atomicOr(&s.bits[pos >> 5], 1u << (pos & 31));
+      }
+      __syncthreads();
+      const int per = (W + kFinThreads - 1) / kFinThreads;
+      const int w0 = tid * per;
+      uint32_t mine = 0;
+      for (int j = 0; j < per; ++j)
+        if (w0 + j < W) mine += __popc(s.bits[w0 + j]);
+      uint32_t total;
+      uint32_t run = block_excl_scan(mine, s.swarp, total);
+      for (int j = 0; j < per; ++j)
+        if (w0 + j < W) {
+          s.wpre[w0 + j] = run;
+          run += __popc(s.bits[w0 + j]);
         }
-        __syncthreads();
-        if (sel) {
-          uint32_t o = s.total + s.wcnt[warp] + __popc(m & lanemask_lt());
-          if (o < (uint32_t)kMaxK) { s.sel_pos[o] = (uint32_t)i; s.sel_key[o] = key; }
+      __syncthreads();
+      for (int i = tid; i < it.n; i += kFinThreads) {
+        const uint32_t key = it.k(i), pos = it.p(i);
+        if (is_selected(key, pos, prefix, pmask, pmax)) {
+          const uint32_t slot = s.wpre[pos >> 5] + __popc(s.bits[pos >> 5] & ((1u << (pos & 31)) - 1u));
+          emit(out, o_idx, b, slot, pos, key);
         }
-        __syncthreads();
-        if (tid == 0) s.total += s.nsel;
-        __syncthreads();
-        if (s.total >= K) break;
       }
     } else {
-      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-        int i = i0 + tid;
-        bool sel = false;
-        uint32_t key = 0, pos = 0;
-        if (i < it.n) {
-          key = it.k(i);
-          pos = it.p(i);
-          sel = is_selected(key, pos, prefix, pmask, pmax);
-        }
-        if (sel) {
-          uint32_t o = atomicAdd(&s.total, 1u);
-          if (o < (uint32_t)kMaxK) { s.sel_pos[o] = pos; s.sel_key[o] = key; }
+      // ---- long rows: compact the chosen items, bitonic sort by position
+      uint32_t* sp = s.bits;
+      uint32_t* sk = s.wpre;
+      for (int i = tid; i < it.n; i += kFinThreads) {
+        const uint32_t key = it.k(i), pos = it.p(i);
+        if (is_selected(key, pos, prefix, pmask, pmax)) {
+          const uint32_t o = atomicAdd(&s.total, 1u);
+          if (o < (uint32_t)kMaxK) { sp[o] = pos; sk[o] = key; }
         }
       }
       __syncthreads();
-      // Bitonic sort of the K chosen pairs by position.
       int P = 1;
       while (P < (int)K) P <<= 1;
-      for (int i = (int)K + tid; i < P; i += kFinThreads) { s.sel_pos[i] = 0xFFFFFFFFu; s.sel_key[i] = 0; }
+      for (int i = (int)K + tid; i < P; i += kFinThreads) { sp[i] = 0xFFFFFFFFu; sk[i] = 0; }
       __syncthreads();
       for (int size = 2; size <= P; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
           for (int i = tid; i < (P >> 1); i += kFinThreads) {
-            int lo = 2 * i - (i & (stride - 1));
-            int hi = lo + stride;
-            bool asc = (lo & size) == 0;
-            uint32_t a = s.sel_pos[lo], c = s.sel_pos[hi];
+            const int lo = 2 * i - (i & (stride - 1));
+            const int hi = lo + stride;
+            const bool asc = (lo & size) == 0;
+            const uint32_t a = sp[lo], c = sp[hi];
             if ((a > c) == asc) {
-              s.sel_pos[lo] = c; s.sel_pos[hi] = a;
-              uint32_t ka = s.sel_key[lo]; s.sel_key[lo] = s.sel_key[hi]; s.sel_key[hi] = ka;
+              sp[lo] = c;
+              sp[hi] = a;
+              const uint32_t ka = sk[lo];
+              sk[lo] = sk[hi];
+              sk[hi] = ka;
             }
           }
           __syncthreads();
         }
       }
+      for (int i = tid; i < (int)K; i += kFinThreads) emit(out, o_idx, b, (uint32_t)i, sp[i], sk[i]);
     }
   }
-  __syncthreads();
 
+  // ---- padding and counts
   if (out.rows == nullptr) {
-    const long long o = ((long long)b * Tq + t) * k;
-    for (int i = tid; i < k; i += kFinThreads) {
-      bool v = i < (int)K;
-      out.idx[o + i] = v ? (int32_t)s.sel_pos[i] : -1;
-      if (out.score) out.score[o + i] = v ? key_score(s.sel_key[i]) : __int_as_float(0xff800000);
+    for (int i = (int)K + tid; i < k; i += kFinThreads) {
+      out.idx[o_idx + i] = -1;
+      if (out.score) out.score[o_idx + i] = __int_as_float(0xff800000);
     }
     if (tid == 0) out.count[(long long)b * Tq + t] = (int32_t)K;
   } else {
@@ -455,112 +570,19 @@ finish_kernel(RowWorkspace w, bool candidates, int rows_per_batch, int t0, int T
     const int unfolded = (int)K * stride;
     const int total = unfolded + p;
     int32_t* rows = out.rows + (long long)b * out.rows_stride;
-    for (int i = tid; i < out.rows_stride; i += kFinThreads) {
-      int32_t v = -1;
-      if (i < unfolded) v = (int32_t)s.sel_pos[i / stride] * stride + i % stride;
-      else if (i < total) v = out.n_chunks * stride + (i - unfolded);
-      rows[i] = v;
-    }
-    if (out.chunks) {
-      for (int i = tid; i < k; i += kFinThreads)
-        out.chunks[(long long)b * k + i] = i < (int)K ? (int32_t)s.sel_pos[i] : -1;
-    }
+    for (int i = unfolded + tid; i < out.rows_stride; i += kFinThreads)
+      rows[i] = i < total ? out.n_chunks * stride + (i - unfolded) : -1;
+    if (out.chunks)
+      for (int i = (int)K + tid; i < k; i += kFinThreads) out.chunks[o_idx + i] = -1;
     if (tid == 0) out.count[b] = total;
   }
-}
 
-// ------------------------------------------------------------ prefill GEMM
-
-// Causal score tile: 128 query rows x 128 key columns, 8 warps (4 x 2), each
-// warp 32 x 64, mma.sync m16n8k16 bf16 -> fp32.
-template <int D>
-__global__ void __launch_bounds__(256)
-score_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int Tq,
-                     int Tk_max, int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int t0,
-                     int rows, uint32_t* __restrict__ keys, long long ld) {
-  constexpr int LDS = D + 8;  // padded row (elements): 16-byte skew per row
-  extern __shared__ __align__(16) uint16_t sm[];
-  uint16_t* sq = sm;
-  uint16_t* sk = sm + 128 * LDS;
-  const int b = blockIdx.z;
-  const int len = row_len(kv_len, b, Tk);
-  const int tr0 = t0 + blockIdx.y * 128;          // first query row of the tile
-  const int c0 = blockIdx.x * 128;                // first key column
-  const int t_last = min(tr0 + 127, t0 + rows - 1);
-  if (tr0 >= t0 + rows) return;
-  if ((long long)c0 > (long long)q_pos0 + t_last || c0 >= len) return;  // above the diagonal
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  for (int i = tid; i < 128 * CPR; i += 256) {
-    int rr = i / CPR, cc = i % CPR;
-    int tq = tr0 + rr;
-    bool vq = tq < t0 + rows && tq < Tq;
-    cp_async16(sq + rr * LDS + cc * 8, q + (((long long)b * Tq + (vq ? tq : 0)) * D + cc * 8), vq);
-    int j = c0 + rr;
-    bool vk = j < len;
-    cp_async16(sk + rr * LDS + cc * 8, kmat + (((long long)b * Tk_max + (vk ? j : 0)) * D + cc * 8),
-               vk);
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-
-  const int wm = warp >> 1, wn = warp & 1;  // warp tile: rows wm*32, cols wn*64
-  float acc[2][8][4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    uint32_t a[2][4];
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi) {
-      int mrow = wm * 32 + mi * 16 + (lane & 15);
-      int kcol = kk * 16 + (lane >> 4) * 8;
-      ldmatrix_x4(a[mi][0], a[mi][1], a[mi][2], a[mi][3], sq + mrow * LDS + kcol);
-    }
-#pragma unroll
-    for (int nj = 0; nj < 8; nj += 2) {
-      // four 8x8 matrices: (n-tile nj, k lo), (nj, k hi), (nj+1, k lo), (nj+1, k hi)
-      int mtx = lane >> 3;
-      int nrow = wn * 64 + (nj + (mtx >> 1)) * 8 + (lane & 7);
-      int kcol = kk * 16 + (mtx & 1) * 8;
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(b0, b1, b2, b3, sk + nrow * LDS + kcol);
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        mma_bf16_16816(acc[mi][nj], a[mi], b0, b1);
-        mma_bf16_16816(acc[mi][nj + 1], a[mi], b2, b3);
-      }
-    }
-  }
-
-  // Epilogue: keys of causal, in-range entries.
-  const int g = lane >> 2, tg = lane & 3;
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi) {
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      int tq = tr0 + wm * 32 + mi * 16 + g + half * 8;
-      if (tq >= t0 + rows || tq >= Tq) continue;
-      int lim = n_cand(q_pos0, tq, len);  // columns < lim are candidates
-      uint32_t* krow = keys + ((long long)b * rows + (tq - t0)) * ld;
-#pragma unroll
-      for (int nj = 0; nj < 8; ++nj) {
-        int c = c0 + wn * 64 + nj * 8 + tg * 2;
-        float s0 = acc[mi][nj][half * 2 + 0], s1 = acc[mi][nj][half * 2 + 1];
-        if (c + 1 < lim) {
-          *reinterpret_cast<uint2*>(krow + c) = make_uint2(score_key(s0), score_key(s1));
-        } else if (c < lim) {
-          krow[c] = score_key(s0);
-        }
-      }
-    }
+  // ---- leave this row's histogram and counter at zero for the next call
+  if (mode != kFinishDirect) {
+    __syncthreads();
+    uint32_t* h = w.hist + (long long)r * kHistBins;
+    for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
+    if (tid == 0) w.cand_cnt[r] = 0;
   }
 }
 
@@ -569,14 +591,13 @@ score_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
 // ------------------------------------------------------------------ host side
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+static long long row_ld(int Tk_max) { return ((long long)Tk_max + 255) / 256 * 256; }
 
 size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates) {
-  long long ld = ((long long)Tk_max + 63) / 64 * 64;
-  size_t bytes = 0;
-  if (with_candidates) {
-    bytes += align256((size_t)rows * kHistBins * 4);
-    bytes += align256((size_t)rows * 4);
-  }
+  const long long ld = row_ld(Tk_max);
+  size_t bytes = 256;  // error word
+  bytes += align256((size_t)rows * kHistBins * 4);
+  bytes += align256((size_t)rows * 4);
   bytes += align256((size_t)rows * ld * 4);
   if (with_candidates) bytes += 2 * align256((size_t)rows * kCandCap * 4);
   return bytes;
@@ -584,13 +605,13 @@ size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates) {
 
 void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, RowWorkspace* o) {
   char* p = static_cast<char*>(ws);
-  o->ld = ((long long)Tk_max + 63) / 64 * 64;
-  if (with_candidates) {
-    o->hist = reinterpret_cast<uint32_t*>(p);
-    p += align256((size_t)rows * kHistBins * 4);
-    o->cand_cnt = reinterpret_cast<uint32_t*>(p);
-    p += align256((size_t)rows * 4);
-  }
+  o->ld = row_ld(Tk_max);
+  o->err = reinterpret_cast<int*>(p);
+  p += 256;
+  o->hist = reinterpret_cast<uint32_t*>(p);
+  p += align256((size_t)rows * kHistBins * 4);
+  o->cand_cnt = reinterpret_cast<uint32_t*>(p);
+  p += align256((size_t)rows * 4);
   o->keys = reinterpret_cast<uint32_t*>(p);
   p += align256((size_t)rows * o->ld * 4);
   if (with_candidates) {
@@ -604,7 +625,7 @@ cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, 
                                 int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
                                 bool with_hist, cudaStream_t st) {
   if (Tk <= 0 || B <= 0) return cudaSuccess;
-  const int chunk = (256 * 1024) / (d * 2);  // about 256 KB of keys per CTA
+  const int chunk = (128 * 1024) / (d * 2);  // about 128 KB of keys per CTA
   dim3 grid((Tk + chunk - 1) / chunk, B);
   uint32_t* hist = with_hist ? w.hist : nullptr;
   if (d == 128)
@@ -619,56 +640,44 @@ cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, 
 cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
                            const RowWorkspace& w, cudaStream_t st) {
   if (Tk <= 0 || B <= 0) return cudaSuccess;
-  const int chunk = 8192;
+  const int chunk = 256 * kCollectPer;
   dim3 grid((Tk + chunk - 1) / chunk, B);
-  collect_kernel<<<grid, 256, 0, st>>>(w.keys, w.ld, w.hist, Tk, q_pos0, kv_len, k, chunk,
-                                       w.cand_cnt, w.cand_key, w.cand_pos);
+  collect_kernel<<<grid, 256, 0, st>>>(w.keys, w.ld, w.hist, Tk, q_pos0, kv_len, k, chunk, w.cand_cnt,
+                                       w.cand_key, w.cand_pos);
   return cudaGetLastError();
 }
 
 cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
-                          const int32_t* kv_len, int k, const RowWorkspace& w, bool candidates,
+                          const int32_t* kv_len, int k, const RowWorkspace& w, int mode,
                           const FinishOut& out, cudaStream_t st) {
   const int rows = B * rows_per_batch;
   if (rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(FinishSmem);
   cudaError_t e = ensure_dynamic_smem((const void*)finish_kernel, smem);
   if (e != cudaSuccess) return e;
-  finish_kernel<<<rows, kFinThreads, smem, st>>>(w, candidates, rows_per_batch, t0, Tq, Tk, q_pos0,
-                                                 kv_len, k, out);
+  finish_kernel<<<rows, kFinThreads, smem, st>>>(w, mode, rows_per_batch, t0, Tq, Tk, q_pos0, kv_len, k,
+                                                 out);
   return cudaGetLastError();
+}
+
+int finish_mode_for(int Tk_max, bool* need_collect) {
+  // short rows: one CTA reads the whole row; rows one CTA can still scan:
+  // histogram-filtered scan; longer rows: many CTAs collect candidates first
+  *need_collect = false;
+  if (Tk_max <= kDirectMaxCand) return kFinishDirect;
+  if (Tk_max <= kBitmapMax) return kFinishHistScan;
+  *need_collect = true;
+  return kFinishCandList;
 }
 
 int prefill_rows_per_launch(int B, int Tq, int Tk_max) {
   // Key slab of at most 512 MiB: rows * B * ld * 4 bytes.
-  long long ld = ((long long)Tk_max + 63) / 64 * 64;
+  const long long ld = row_ld(Tk_max);
   long long cap = (512ll << 20) / (4ll * ld * (B > 0 ? B : 1));
   cap = cap / 128 * 128;
   if (cap < 128) cap = 128;
   if (cap > Tq) cap = Tq;
   return (int)cap;
-}
-
-cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,
-                                 int Tk_max, int Tk, int q_pos0, const int32_t* kv_len, int t0,
-                                 int rows, const RowWorkspace& w, cudaStream_t st) {
-  if (rows <= 0 || Tk <= 0) return cudaSuccess;
-  long long last = (long long)q_pos0 + t0 + rows;  // columns needed: < min(Tk, last)
-  int ncols = (int)(last < Tk ? (last > 0 ? last : 0) : Tk);
-  if (ncols <= 0) return cudaSuccess;
-  dim3 grid((ncols + 127) / 128, (rows + 127) / 128, B);
-  if (d == 128) {
-    size_t smem = 2 * 128 * (128 + 8) * 2;
-    cudaError_t e = ensure_dynamic_smem((const void*)score_prefill_kernel<128>, smem);
-    if (e != cudaSuccess) return e;
-    score_prefill_kernel<128><<<grid, 256, smem, st>>>(q, kmat, Tq, Tk_max, Tk, q_pos0, kv_len, t0,
-                                                       rows, w.keys, w.ld);
-  } else {
-    size_t smem = 2 * 128 * (64 + 8) * 2;
-    score_prefill_kernel<64><<<grid, 256, smem, st>>>(q, kmat, Tq, Tk_max, Tk, q_pos0, kv_len, t0,
-                                                      rows, w.keys, w.ld);
-  }
-  return cudaGetLastError();
 }
 
 }  // namespace sa

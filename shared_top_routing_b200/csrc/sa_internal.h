@@ -7,11 +7,18 @@
 
 namespace sa {
 
-// Rows of at most this many candidates are selected by one CTA reading the
-// whole row ("direct" mode); longer rows go through histogram + collect.
-constexpr int kDirectMaxCand = 16384;
+// Rows of at most this many candidates are selected by one CTA holding the
+// whole row in shared memory ("direct" mode); longer rows use the key
+// histogram (and, beyond what one CTA can scan, a multi-CTA collect pass).
+constexpr int kDirectMaxCand = 8192;
+
+// finish_kernel candidate sources
+constexpr int kFinishDirect = 0;    // the whole row (no histogram)
+constexpr int kFinishHistScan = 1;  // one CTA scans the row, keeping keys in or above the k-th key's bin
+constexpr int kFinishCandList = 2;  // candidates collected by collect_kernel
 
 struct RowWorkspace {
+  int* err = nullptr;            // first word: kernel error code (0 = none)
   uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys
   long long ld = 0;
   uint32_t* hist = nullptr;      // [rows][kHistBins]
@@ -50,9 +57,12 @@ cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int
 // Exact selection per row.  rows = B * rows_per_batch; row r is query
 // t0 + r % rows_per_batch of batch r / rows_per_batch.
 cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
-                          const int32_t* kv_len, int k, const RowWorkspace& w, bool candidates,
+                          const int32_t* kv_len, int k, const RowWorkspace& w, int mode,
                           const FinishOut& out, cudaStream_t st);
-// Prefill scoring of queries [t0, t0+rows) into the key slab.
+// Candidate source for rows of Tk_max positions; sets *need_collect when the
+// collect pass must run between scoring and finish.
+int finish_mode_for(int Tk_max, bool* need_collect);
+// Prefill scoring of queries [t0, t0+rows) into the key slab (tcgen05, index_tc.cu).
 cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,
                                  int Tk_max, int Tk, int q_pos0, const int32_t* kv_len, int t0,
                                  int rows, const RowWorkspace& w, cudaStream_t st);

@@ -125,7 +125,9 @@ _ws_cache: dict = {}
 
 
 def workspace(nbytes: int, device, key: str = "", stream=None):
-    """A cached device workspace of at least ``nbytes`` (256-byte aligned)."""
+    """A cached, zero-filled device workspace of at least ``nbytes`` (256-byte
+    aligned).  The library returns the parts that must start at zero to zero
+    after each call, so the cache can hand the same buffer to later calls."""
     torch = _torch()
     if nbytes <= 0:
         return None
@@ -133,7 +135,7 @@ def workspace(nbytes: int, device, key: str = "", stream=None):
     k = (str(device), s.cuda_stream, key)
     buf = _ws_cache.get(k)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         _ws_cache[k] = buf
     return buf
 
