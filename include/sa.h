@@ -23,13 +23,14 @@
  *     any CUDA kernel.
  *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
  *   - No kernel of this library waits on another CTA, kernel or device.
- *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned, and
- *     must be ZERO-FILLED before their first use.  Every call that returns
- *     SA_OK leaves the parts of its workspace that must start at zero back
- *     at zero once its kernels complete, so one workspace serves any number
- *     of calls made one after another on one stream.  Calls that overlap on
- *     the GPU (different streams) need different workspaces.  After a failed
- *     or interrupted call, zero the workspace again.
+ *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned.  The
+ *     decode-attention workspace must be ZERO-FILLED before its first use:
+ *     its merge tickets live in a fixed region that every completed call
+ *     returns to zero, so one workspace then serves any number of calls of
+ *     any shape made one after another on one stream (zero it again after a
+ *     failed or interrupted call).  The other workspaces need no
+ *     initialisation.  Calls that overlap on the GPU (different streams)
+ *     need different workspaces.
  */
 #ifndef SA_H_
 #define SA_H_
@@ -58,6 +59,7 @@ typedef enum {
 #define SA_MAX_K 4096           /* largest top-k                                */
 #define SA_HEAD_DIM 128         /* attention head_dim supported                 */
 #define SA_WS_ALIGN 256         /* workspace pointers must be 256-byte aligned  */
+#define SA_DECODE_MAX_PAIRS 16384 /* largest B * Hkv of one decode attention call */
 
 /* Static, never-null description of a status code. */
 const char* sa_status_string(sa_status s);
@@ -93,8 +95,8 @@ int sa_version(void);
  *                                      outside are clamped on the device)
  *   idx_out    [B, Tq, k] int32;  count_out [B, Tq] int32
  *   score_out  [B, Tq, k] fp32 or NULL
- *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes
- *              (zero-filled before first use; see the conventions above).
+ *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes;
+ *              no initialisation needed; contents are clobbered.
  * Supported: d in {64, 128}; 1 <= k <= SA_MAX_K; Tq >= 1; 0 <= Tk <= Tk_max.
  * Scores must be free of NaN (NaN inputs give an unspecified selection).
  * ---------------------------------------------------------------------- */
@@ -148,7 +150,7 @@ sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void*
  *   out      [B, Hq, D] bf16;  lse [B, Hq] fp32 or NULL
  *   ws       >= sa_sparse_attn_decode_workspace(...) bytes (zero-filled before
  *            first use; see the conventions above)
- * Supported: as for prefill.
+ * Supported: as for prefill; B * Hkv <= SA_DECODE_MAX_PAIRS.
  * ---------------------------------------------------------------------- */
 size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k);
 sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -169,8 +169,12 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
     const int mode = sa::finish_mode_for(Tk_max, &collect);
     sa::RowWorkspace w;
     sa::carve_row_workspace(ws, B, Tk_max, collect, &w);
-    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w,
-                                     mode != sa::kFinishDirect, cs)) != cudaSuccess)
+    if (collect) {
+      // the multi-CTA histogram and candidate counters start at zero (adjacent)
+      const size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
+      if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
+    }
+    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, collect, cs)) != cudaSuccess)
       return cuda_fail(e, "score_decode launch");
     if (collect && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
       return cuda_fail(e, "collect launch");
@@ -221,6 +225,8 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
   sa_status st = validate_attn(q, k_cache, v_cache, idx, count, B, 1, Tk_max, Hq, Hkv, D, k, out);
   if (st != SA_OK) return st;
   if (B == 0) return ok();
+  if ((long long)B * Hkv > SA_DECODE_MAX_PAIRS)
+    return fail(SA_ERR_UNSUPPORTED, "B*Hkv=%lld exceeds %d", (long long)B * Hkv, SA_DECODE_MAX_PAIRS);
   if ((st = check_ws(ws, ws_bytes, sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k))) != SA_OK)
     return st;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
@@ -267,10 +273,14 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   sa::RowWorkspace w;
   sa::carve_row_workspace(ws, B, n_chunks, collect, &w);
   cudaError_t e;
+  if (collect) {
+    const size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
+    if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
+  }
   const int q_pos0 = n_chunks - 1;  // every complete chunk is a candidate
   if ((e = sa::launch_score_decode(static_cast<const uint16_t*>(q_route),
                                    static_cast<const uint16_t*>(gist_key), B, d, n_chunks, n_chunks,
-                                   q_pos0, nullptr, w, mode != sa::kFinishDirect, cs)) != cudaSuccess)
+                                   q_pos0, nullptr, w, collect, cs)) != cudaSuccess)
     return cuda_fail(e, "gist score launch");
   if (collect && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
     return cuda_fail(e, "gist collect launch");

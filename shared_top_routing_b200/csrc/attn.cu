@@ -358,11 +358,17 @@ void decode_split(int B, int Hkv, int k, int* tiles_per_split, int* S) {
 
 static size_t align256a(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The merge tickets sit in a fixed region at the start of the workspace
+// (room for kTicketSlots (sequence, kv head) pairs) that holds nothing else,
+// so a zero-filled workspace stays valid across calls of any shape: the last
+// CTA of every pair returns its ticket to zero.
+constexpr int kTicketSlots = 16384;
+
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
   (void)D;
   int tps, S;
   decode_split(B, Hkv, k, &tps, &S);
-  const size_t tk = align256a((size_t)B * Hkv * 4);
+  const size_t tk = (size_t)kTicketSlots * 4;
   const size_t po = align256a((size_t)B * Hq * S * kD * 4);
   const size_t pml = align256a((size_t)B * Hq * S * 2 * 4);
   return tk + po + pml;
@@ -377,7 +383,7 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
   decode_split(B, Hkv, k, &tps, &S);
   char* p = static_cast<char*>(ws);
   unsigned* ticket = reinterpret_cast<unsigned*>(p);
-  p += align256a((size_t)B * Hkv * 4);
+  p += (size_t)kTicketSlots * 4;
   float* po = reinterpret_cast<float*>(p);
   p += align256a((size_t)B * Hq * S * kD * 4);
   float* pml = reinterpret_cast<float*>(p);

@@ -13,8 +13,9 @@
 //       warp loads whole 16-byte chunks 4j+t of key row g and the query
 //       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
 //       keys (the query is row 0 of the 16-row A side).  Writes the order-
-//       preserving 32-bit score key of every candidate and a 4096-bin
-//       histogram of each key's top 12 bits.
+//       preserving 32-bit score key of every candidate and, for rows that
+//       need the multi-CTA collect, a 4096-bin histogram of the keys' top 12
+//       bits.
 //   collect_kernel       (rows longer than one CTA can scan) finds, from the
 //       histogram, the bin holding the k-th largest key and appends every key
 //       in that bin or above to a per-row candidate list (one atomic per CTA).
@@ -24,8 +25,9 @@
 //       warp-aggregated shared histograms) of the k-th key and of the tie
 //       positions, then emits in ascending position order through a position
 //       bitmap and popcount prefix sums (bitonic sort for rows beyond the
-//       bitmap's reach).  Also expands chosen gist chunks into cache rows and
-//       returns the histogram and counters of its row to zero.
+//       bitmap's reach).  Rows a single CTA can scan get their key
+//       histogram built here in shared memory, so no global state needs
+//       clearing between calls.  Also expands chosen gist chunks into rows.
 // The prefill scores come from the tcgen05 kernel in index_tc.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -433,8 +435,29 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   bool in_smem = false;
   if (K > 0) {
     if (mode == kFinishHistScan) {
-      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
+      // pass 1: histogram of the row's top-12-bit key digits in shared memory
+      uint32_t* h = s.bits;
+      for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
+      __syncthreads();
+      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
+        const int i = i0 + tid * 4;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i + 3 < n) {
+          v = *reinterpret_cast<const uint4*>(row + i);
+        } else {
+          if (i < n) v.x = row[i];
+          if (i + 1 < n) v.y = row[i + 1];
+          if (i + 2 < n) v.z = row[i + 2];
+        }
+        hist_add(h, v.x >> (32 - kHistBits), i < n);
+        hist_add(h, v.y >> (32 - kHistBits), i + 1 < n);
+        hist_add(h, v.z >> (32 - kHistBits), i + 2 < n);
+        hist_add(h, v.w >> (32 - kHistBits), i + 3 < n);
+      }
+      __syncthreads();
+      hist_threshold(h, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
+      // pass 2: keep every key in or above the bin of the K-th largest
       for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
         const int i = i0 + tid * 4;
         uint4 v = make_uint4(0, 0, 0, 0);
@@ -575,14 +598,6 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
     if (out.chunks)
       for (int i = (int)K + tid; i < k; i += kFinThreads) out.chunks[o_idx + i] = -1;
     if (tid == 0) out.count[b] = total;
-  }
-
-  // ---- leave this row's histogram and counter at zero for the next call
-  if (mode != kFinishDirect) {
-    __syncthreads();
-    uint32_t* h = w.hist + (long long)r * kHistBins;
-    for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
-    if (tid == 0) w.cand_cnt[r] = 0;
   }
 }
 

@@ -126,8 +126,9 @@ _ws_cache: dict = {}
 
 def workspace(nbytes: int, device, key: str = "", stream=None):
     """A cached, zero-filled device workspace of at least ``nbytes`` (256-byte
-    aligned).  The library returns the parts that must start at zero to zero
-    after each call, so the cache can hand the same buffer to later calls."""
+    aligned).  The decode-attention workspace must start zero-filled; the
+    library returns its ticket region to zero after each call, so the cache
+    can hand the same buffer to later calls of any shape."""
     torch = _torch()
     if nbytes <= 0:
         return None

@@ -318,3 +318,42 @@ def test_device_generator_matches_host_generator():
     gd.fill_int(t, 12, 35, start=5)
     np.testing.assert_array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16),
                                   ch.int_bf16(12, 35, start=5, count=100003))
+
+
+# ------------------------------------------------------- workspace reuse
+
+def test_one_workspace_serves_calls_of_any_shape():
+    """One caller-owned workspace reused by calls whose shapes grow and
+    shrink (index rows in every selection path, including rows longer than
+    the bitmap reach that take the multi-CTA collect path), then decode
+    attention calls of varying B*Hkv on one zero-filled workspace."""
+    L = sa.lib()
+    cases = [(1, 60000, 64, 100), (2, 40000, 64, 3000), (4, 20000, 128, 2048),
+             (1, 300000, 64, 2048), (3, 5000, 128, 7), (2, 270000, 128, 4096)]
+    need = max(L.sa_index_score_topk_workspace(B, 1, n, d, k) for B, n, d, k in cases)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev())
+    ws.fill_(0xAB)   # the index workspace needs no initialisation
+    for i, (B, n, d, k) in enumerate(cases):
+        q = _ints(900 + i, 1, (B, d))
+        kk = _ints(900 + i, 2, (B, n, d))
+        idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, ws=ws)
+        ridx, rcnt = oracle.index_topk(q[:, None, :], kk, n, n - 1, k)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0], err_msg=str((B, n, d, k)))
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0], err_msg=str((B, n, d, k)))
+    acases = [(4, 8, 32, 2048), (1, 4, 28, 2048), (8, 8, 32, 512), (2, 2, 8, 100)]
+    aneed = max(L.sa_sparse_attn_decode_workspace(B, Hq, Hkv, 128, k) for B, Hkv, Hq, k in acases)
+    wsa = torch.zeros(aneed, dtype=torch.uint8, device=dev())
+    rng = np.random.default_rng(77)
+    for i, (B, Hkv, Hq, k) in enumerate(acases):
+        Tk_max = 3000
+        counts = [k - (b % 3) * 5 for b in range(B)]
+        qv = _normals(950 + i, 1, (B, Hq, 128))
+        K = _normals(950 + i, 2, (B, Tk_max, Hkv, 128))
+        V = _normals(950 + i, 3, (B, Tk_max, Hkv, 128))
+        idx = _random_index(rng, B, Tk_max, k, counts)
+        out = sa.sa_sparse_attn_decode(to_dev(qv), to_dev(K), to_dev(V), i32(idx), i32(counts), ws=wsa)
+        ref, _ = oracle.sparse_attention_decode(qv, [K[b, idx[b, :c]] for b, c in enumerate(counts)],
+                                                [V[b, idx[b, :c]] for b, c in enumerate(counts)])
+        torch.cuda.synchronize()
+        assert_close_attn(out.float().cpu().numpy(), ref, f"attention case {i}")
