@@ -23,14 +23,14 @@
  *     any CUDA kernel.
  *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
  *   - No kernel of this library waits on another CTA, kernel or device.
- *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned.  The
- *     decode-attention workspace must be ZERO-FILLED before its first use:
- *     its merge tickets live in a fixed region that every completed call
+ *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned, and
+ *     must be ZERO-FILLED before their first use.  The counters that must
+ *     start at zero (histograms, candidate counts, merge tickets) live in a
+ *     fixed region at the start of each workspace that every completed call
  *     returns to zero, so one workspace then serves any number of calls of
- *     any shape made one after another on one stream (zero it again after a
- *     failed or interrupted call).  The other workspaces need no
- *     initialisation.  Calls that overlap on the GPU (different streams)
- *     need different workspaces.
+ *     any shape made one after another on one stream.  Zero it again after a
+ *     failed or interrupted call.  Calls that overlap on the GPU (different
+ *     streams) need different workspaces.
  */
 #ifndef SA_H_
 #define SA_H_
@@ -95,8 +95,8 @@ int sa_version(void);
  *                                      outside are clamped on the device)
  *   idx_out    [B, Tq, k] int32;  count_out [B, Tq] int32
  *   score_out  [B, Tq, k] fp32 or NULL
- *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes;
- *              no initialisation needed; contents are clobbered.
+ *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes
+ *              (zero-filled before first use; see the conventions above).
  * Supported: d in {64, 128}; 1 <= k <= SA_MAX_K; Tq >= 1; 0 <= Tk <= Tk_max.
  * Scores must be free of NaN (NaN inputs give an unspecified selection).
  * ---------------------------------------------------------------------- */
@@ -182,6 +182,8 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
  *
  *   q_route     [B, d] bf16;   gist_key [B, n_chunks, d] bf16
  *   partial_len [B] int32 (clamped on the device to [0, chunk_len])
+ *   ws          >= sa_gist_route_unfold_workspace(...) bytes (zero-filled
+ *               before first use; see the conventions above)
  *   rows_out    [B, k_chunks*(chunk_len+1) + chunk_len] int32
  *   count_out   [B] int32;    chunks_out [B, k_chunks] int32 or NULL
  * Supported: d in {64, 128}; 1 <= k_chunks <= SA_MAX_K; 1 <= chunk_len <= 256.

@@ -140,11 +140,11 @@ size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
   if (B <= 0 || Tq <= 0 || Tk_max < 0) return 0;
   if (Tq == 1) {
     bool collect = false;
-    sa::finish_mode_for(Tk_max, &collect);
-    return sa::row_workspace_bytes(B, Tk_max, collect);
+    const int mode = sa::finish_mode_for(Tk_max, &collect);
+    return sa::row_workspace_bytes(B, Tk_max, collect, mode != sa::kFinishDirect);
   }
   int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
-  return sa::row_workspace_bytes(B * rows, Tk_max, false);
+  return sa::row_workspace_bytes(B * rows, Tk_max, false, false);
 }
 
 sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int Tq, int Tk,
@@ -168,13 +168,12 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
     bool collect = false;
     const int mode = sa::finish_mode_for(Tk_max, &collect);
     sa::RowWorkspace w;
-    sa::carve_row_workspace(ws, B, Tk_max, collect, &w);
-    if (collect) {
-      // the multi-CTA histogram and candidate counters start at zero (adjacent)
-      const size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
-      if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
-    }
-    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, collect, cs)) != cudaSuccess)
+    sa::carve_row_workspace(ws, B, Tk_max, collect, mode != sa::kFinishDirect, &w);
+    const bool hist = mode != sa::kFinishDirect;
+    if (hist && w.hist_zero_bytes &&
+        (e = cudaMemsetAsync(w.hist, 0, w.hist_zero_bytes, cs)) != cudaSuccess)
+      return cuda_fail(e, "memset");
+    if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, hist, cs)) != cudaSuccess)
       return cuda_fail(e, "score_decode launch");
     if (collect && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
       return cuda_fail(e, "collect launch");
@@ -184,7 +183,7 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
   }
   const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
   sa::RowWorkspace w;
-  sa::carve_row_workspace(ws, B * rows, Tk_max, false, &w);
+  sa::carve_row_workspace(ws, B * rows, Tk_max, false, false, &w);
   for (int t0 = 0; t0 < Tq; t0 += rows) {
     const int nr = (Tq - t0 < rows) ? Tq - t0 : rows;
     if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, w, cs)) != cudaSuccess)
@@ -245,8 +244,8 @@ size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) 
   (void)k_chunks;
   if (B <= 0 || n_chunks < 0) return 0;
   bool collect = false;
-  sa::finish_mode_for(n_chunks, &collect);
-  return sa::row_workspace_bytes(B, n_chunks, collect);
+  const int mode = sa::finish_mode_for(n_chunks, &collect);
+  return sa::row_workspace_bytes(B, n_chunks, collect, mode != sa::kFinishDirect);
 }
 
 sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B, int n_chunks,
@@ -271,16 +270,15 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   bool collect = false;
   const int mode = sa::finish_mode_for(n_chunks, &collect);
   sa::RowWorkspace w;
-  sa::carve_row_workspace(ws, B, n_chunks, collect, &w);
+  sa::carve_row_workspace(ws, B, n_chunks, collect, mode != sa::kFinishDirect, &w);
   cudaError_t e;
-  if (collect) {
-    const size_t zero = reinterpret_cast<char*>(w.keys) - reinterpret_cast<char*>(w.hist);
-    if ((e = cudaMemsetAsync(w.hist, 0, zero, cs)) != cudaSuccess) return cuda_fail(e, "memset");
-  }
+  const bool hist = mode != sa::kFinishDirect;
+  if (hist && w.hist_zero_bytes && (e = cudaMemsetAsync(w.hist, 0, w.hist_zero_bytes, cs)) != cudaSuccess)
+    return cuda_fail(e, "memset");
   const int q_pos0 = n_chunks - 1;  // every complete chunk is a candidate
   if ((e = sa::launch_score_decode(static_cast<const uint16_t*>(q_route),
                                    static_cast<const uint16_t*>(gist_key), B, d, n_chunks, n_chunks,
-                                   q_pos0, nullptr, w, collect, cs)) != cudaSuccess)
+                                   q_pos0, nullptr, w, hist, cs)) != cudaSuccess)
     return cuda_fail(e, "gist score launch");
   if (collect && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
     return cuda_fail(e, "gist collect launch");

@@ -17,11 +17,12 @@
 //
 // attn_prefill_kernel  grid (T, Hkv, B), kv-head-major: one query token x one
 //                      kv head per CTA, all of its selected rows.
-// attn_decode_kernel   grid (splits, Hkv, B): each CTA takes a contiguous
-//                      range of tiles of the sequence's index list and writes
-//                      a partial (m, l, o); the last CTA of each (sequence, kv
-//                      head) -- found with an atomic ticket, never a wait --
-//                      merges them.  With one split it writes the output.
+// attn_decode_kernel   the 16-row tiles of all (sequence, kv head) pairs are
+//                      split evenly over the warps of a resident-sized grid;
+//                      each warp streams its tiles through a private 3-stage
+//                      cp.async ring, writes a partial (m, l, o) where its
+//                      range leaves a pair, and the warp whose atomic ticket
+//                      completes a pair (never a wait) merges its partials.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -53,22 +54,23 @@ struct TileAcc {
   float m[2], l[2];
 };
 
-// Gathers tile rows [i0, i0+64) (clipped to `end`) of one kv head into stage.
+// Gathers tile rows [i0, i0+64) (clipped to `end`) of one kv head into a
+// stage: 16 consecutive threads copy the 16 chunks of one 256-byte row, so
+// every request covers whole 32-byte sectors.
 __device__ __forceinline__ void gather_tile(uint16_t* sK, uint16_t* sV, const uint16_t* __restrict__ kc,
                                             const uint16_t* __restrict__ vc, const int32_t* __restrict__ irow,
                                             int i0, int end, long long head_base, long long row_elems,
                                             int Tk_max) {
-  const int r = threadIdx.x >> 1, h = threadIdx.x & 1;
-  const int i = i0 + r;
-  const bool v = i < end;
-  const int j = v ? clamp_row(irow[i], Tk_max) : 0;
-  const long long off = head_base + (long long)j * row_elems;
-  uint16_t* dk = sK + r * kLds;
-  uint16_t* dv = sV + r * kLds;
+  const int c = threadIdx.x & 15;
 #pragma unroll
-  for (int c = h * 8; c < h * 8 + 8; ++c) {
-    cp_async16(dk + c * 8, kc + off + c * 8, v);
-    cp_async16(dv + c * 8, vc + off + c * 8, v);
+  for (int pass = 0; pass < kTile / 8; ++pass) {
+    const int r = (threadIdx.x >> 4) + 8 * pass;
+    const int i = i0 + r;
+    const bool v = i < end;
+    const int j = v ? clamp_row(irow[i], Tk_max) : 0;
+    const long long off = head_base + (long long)j * row_elems + c * 8;
+    cp_async16(sK + r * kLds + c * 8, kc + off, v);
+    cp_async16(sV + r * kLds + c * 8, vc + off, v);
   }
 }
 
@@ -270,88 +272,295 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 }
 
 // ------------------------------------------------------------------ decode
+//
+// Balanced split of the decode work: the 16-row tiles of every (sequence, kv
+// head) pair form one list of T tiles, cut into equal contiguous ranges, one
+// per warp of a grid sized to the resident warps.  A warp streams its tiles
+// through its own STAGES-deep cp.async ring (no block barrier in the loop)
+// and writes a partial (m, l, o) whenever its range leaves a pair; the warp
+// whose ticket completes a pair merges that pair's partials.
 
-__global__ void __launch_bounds__(128)
-attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
-                   const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
-                   const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k,
-                   int tiles_per_split, int S, float qscale, float* __restrict__ part_o,
-                   float* __restrict__ part_ml, unsigned* __restrict__ ticket,
-                   uint16_t* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int s_last;
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int G = Hq / Hkv;
-  int cnt = count[b];
-  cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
-  const int begin = min(cnt, s * tiles_per_split * kTile);
-  const int end = min(cnt, (s + 1) * tiles_per_split * kTile);
-  const long long head0 = (long long)b * Hq + (long long)g * G;  // first query head of the group
-  load_q(smem, q + head0 * kD, G);
-  TileAcc acc;
-  attn_tiles(smem, kc, vc, idx + (long long)b * k, begin, end, ((long long)b * Tk_max * Hkv + g) * kD,
-             (long long)Hkv * kD, Tk_max, qscale, acc);
-  stash_warps(smem, acc);
-  const int d = threadIdx.x;
-  if (S == 1) {
-    for (int h = 0; h < G; ++h) {
-      float M, L, o;
-      merge_warps(smem, h, d, M, L, o);
-      out[(head0 + h) * kD + d] = f2bf(L > 0.f ? o / L : 0.f);
-      if (d == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-    }
-    return;
-  }
-  for (int h = 0; h < G; ++h) {
-    float M, L, o;
-    merge_warps(smem, h, d, M, L, o);
-    part_o[((head0 + h) * S + s) * kD + d] = o;
-    if (d == 0) {
-      part_ml[((head0 + h) * S + s) * 2] = M;
-      part_ml[((head0 + h) * S + s) * 2 + 1] = L;
-    }
-  }
-  // The last CTA of this (sequence, kv head) merges the S partials.
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(ticket + (long long)b * Hkv + g, 1u);
-    s_last = prev == (unsigned)(S - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int h = 0; h < G; ++h) {
-    const float* ml = part_ml + (head0 + h) * S * 2;
-    float M = -INFINITY;
-    for (int x = 0; x < S; ++x) M = fmaxf(M, __ldcg(ml + 2 * x));
-    float L = 0.f, a = 0.f;
-    if (M != -INFINITY) {
-      for (int x = 0; x < S; ++x) {
-        const float mx = __ldcg(ml + 2 * x), lx = __ldcg(ml + 2 * x + 1);
-        if (lx == 0.f) continue;
-        const float w = exp2f(mx - M);
-        L = fmaf(lx, w, L);
-        a = fmaf(__ldcg(part_o + ((head0 + h) * S + x) * kD + d), w, a);
-      }
-    }
-    out[(head0 + h) * kD + d] = f2bf(L > 0.f ? a / L : 0.f);
-    if (d == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-  }
-  if (threadIdx.x == 0) ticket[(long long)b * Hkv + g] = 0u;  // ready for the next call
+constexpr int kDecWarps = 4;                 // warps per CTA
+constexpr int kDecStages = 3;                // per-warp ring depth
+constexpr int kDecTile = 16;                 // rows per warp tile
+constexpr size_t kDecStageBytes = (size_t)kDecTile * kLds * 2 * 2;   // K + V
+constexpr size_t kDecSmem = (size_t)kDecWarps * kDecStages * kDecStageBytes;
+
+struct DecPlan {
+  int pairs, tpp, cmax;
+  long long T, W;   // tiles, warps
+};
+
+// Warp owning tile t: the largest w with floor(w*T/W) <= t.
+__device__ __forceinline__ long long tile_owner(long long t, long long T, long long W) {
+  return ((t + 1) * W - 1) / T;
 }
 
-// Splits of the index list: enough CTAs for about 3 per SM, at least one
-// 64-row tile each.
-void decode_split(int B, int Hkv, int k, int* tiles_per_split, int* S) {
-  const int ntiles = (k + kTile - 1) / kTile;
-  const long long pairs = (long long)B * Hkv;
-  long long want = (3 * 148 + pairs - 1) / pairs;
-  if (want < 1) want = 1;
-  if (want > ntiles) want = ntiles;
-  int tps = (int)((ntiles + want - 1) / want);
-  *tiles_per_split = tps;
-  *S = (ntiles + tps - 1) / tps;
+__device__ __forceinline__ void dec_gather(uint16_t* st, const uint16_t* __restrict__ kc,
+                                           const uint16_t* __restrict__ vc, int jlane, int i0, int end,
+                                           long long head_base, long long row_elems, int Tk_max, int lane) {
+  const int c = lane & 15;
+  uint16_t* sK = st;
+  uint16_t* sV = st + kDecTile * kLds;
+#pragma unroll
+  for (int pass = 0; pass < kDecTile / 2; ++pass) {
+    const int r = (lane >> 4) + 2 * pass;
+    const int j = __shfl_sync(0xffffffffu, jlane, r);
+    const bool v = i0 + r < end;
+    const long long off = head_base + (long long)(v ? j : 0) * row_elems + c * 8;
+    cp_async16(sK + r * kLds + c * 8, kc + off, v);
+    cp_async16(sV + r * kLds + c * 8, vc + off, v);
+  }
+}
+
+__global__ void __launch_bounds__(kDecWarps * 32)
+attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                   const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
+                   const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k, DecPlan pl,
+                   float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
+                   unsigned* __restrict__ ticket, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tg = lane & 3;
+  const int G = Hq / Hkv;
+  const long long w = (long long)blockIdx.x * kDecWarps + warp;
+  if (w >= pl.W) return;
+  uint16_t* ring = reinterpret_cast<uint16_t*>(smem + (size_t)warp * kDecStages * kDecStageBytes);
+  const long long lo = w * pl.T / pl.W, hi = (w + 1) * pl.T / pl.W;
+
+  for (long long t = lo; t < hi;) {
+    const int p = (int)(t / pl.tpp);
+    const long long seg_end = min(hi, (long long)(p + 1) * pl.tpp);
+    const int b = p / Hkv, g = p % Hkv;
+    int cnt = count[b];
+    cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
+    const int first_tile = (int)(t - (long long)p * pl.tpp);
+    const int ntiles = (int)(seg_end - t);
+    const int32_t* irow = idx + (long long)b * k;
+    const long long head_base = ((long long)b * Tk_max * Hkv + g) * kD;
+    const long long row_elems = (long long)Hkv * kD;
+    const long long head0 = (long long)b * Hq + (long long)g * G;
+
+    // query fragments of the group's heads (rows >= G are zero)
+    uint32_t qa[8][4];
+    {
+      const uint32_t* qr0 = reinterpret_cast<const uint32_t*>(q + (head0 + gq) * kD);
+      const uint32_t* qr1 = reinterpret_cast<const uint32_t*>(q + (head0 + gq + 8) * kD);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int c0 = (kk * 16 + 2 * tg) >> 1, c1 = (kk * 16 + 8 + 2 * tg) >> 1;
+        qa[kk][0] = gq < G ? __ldg(qr0 + c0) : 0u;
+        qa[kk][1] = gq + 8 < G ? __ldg(qr1 + c0) : 0u;
+        qa[kk][2] = gq < G ? __ldg(qr0 + c1) : 0u;
+        qa[kk][3] = gq + 8 < G ? __ldg(qr1 + c1) : 0u;
+      }
+    }
+    float o[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+
+    // pipeline prologue
+#pragma unroll
+    for (int sIdx = 0; sIdx < kDecStages - 1; ++sIdx) {
+      if (sIdx < ntiles) {
+        const int i0 = (first_tile + sIdx) * kDecTile;
+        const int jl = i0 + (lane & 15) < cnt ? clamp_row(irow[i0 + (lane & 15)], Tk_max) : 0;
+        dec_gather(ring + sIdx * (kDecStageBytes / 2), kc, vc, jl, i0, cnt, head_base, row_elems, Tk_max, lane);
+      }
+      cp_async_commit();
+    }
+    for (int it = 0; it < ntiles; ++it) {
+      const int nxt = it + kDecStages - 1;
+      if (nxt < ntiles) {
+        const int i0 = (first_tile + nxt) * kDecTile;
+        const int jl = i0 + (lane & 15) < cnt ? clamp_row(irow[i0 + (lane & 15)], Tk_max) : 0;
+        dec_gather(ring + (nxt % kDecStages) * (kDecStageBytes / 2), kc, vc, jl, i0, cnt, head_base,
+                   row_elems, Tk_max, lane);
+      }
+      cp_async_commit();
+      cp_async_wait<kDecStages - 1>();
+      __syncwarp();
+      const uint16_t* tK = ring + (it % kDecStages) * (kDecStageBytes / 2);
+      const uint16_t* tV = tK + kDecTile * kLds;
+      const int rbase = (first_tile + it) * kDecTile;
+      if (rbase < cnt) {
+        float sc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int mtx = lane >> 3;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(b0, b1, b2, b3, tK + ((mtx >> 1) * 8 + (lane & 7)) * kLds + kk * 16 + (mtx & 1) * 8);
+          mma_bf16_16816(sc[0], qa[kk], b0, b1);
+          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+        }
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = rbase + nt * 8 + tg * 2 + (e & 1);
+            const float z = row < cnt ? sc[nt][e] * qscale : -INFINITY;
+            sc[nt][e] = z;
+            mx[e >> 1] = fmaxf(mx[e >> 1], z);
+          }
+        float alpha[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v = mx[hh];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          const float mnew = fmaxf(m_r[hh], v);
+          const float muse = mnew == -INFINITY ? 0.f : mnew;
+          alpha[hh] = exp2f(m_r[hh] - muse);
+          m_r[hh] = mnew;
+          mx[hh] = muse;
+        }
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+            sc[nt][e] = pv;
+            rs[e >> 1] += pv;
+          }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v = rs[hh];
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          l_r[hh] = l_r[hh] * alpha[hh] + v;
+        }
+#pragma unroll
+        for (int dt = 0; dt < 16; ++dt) {
+          o[dt][0] *= alpha[0];
+          o[dt][1] *= alpha[0];
+          o[dt][2] *= alpha[1];
+          o[dt][3] *= alpha[1];
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf2(sc[0][0], sc[0][1]);
+        pa[1] = pack_bf2(sc[0][2], sc[0][3]);
+        pa[2] = pack_bf2(sc[1][0], sc[1][1]);
+        pa[3] = pack_bf2(sc[1][2], sc[1][3]);
+#pragma unroll
+        for (int dt = 0; dt < 16; dt += 2) {
+          const int mtx = lane >> 3;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * kLds + (dt + (mtx >> 1)) * 8);
+          mma_bf16_16816(o[dt], pa, b0, b1);
+          mma_bf16_16816(o[dt + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+
+    // ---- hand the segment's result on
+    const long long w_first = tile_owner((long long)p * pl.tpp, pl.T, pl.W);
+    const long long w_last = tile_owner((long long)(p + 1) * pl.tpp - 1, pl.T, pl.W);
+    const int ncontrib = (int)(w_last - w_first + 1);
+    if (ncontrib == 1) {
+      // this warp owns the whole pair: normalise and write
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = gq + 8 * hh;
+        if (h < G) {
+          const float inv = l_r[hh] > 0.f ? 1.f / l_r[hh] : 0.f;
+#pragma unroll
+          for (int dt = 0; dt < 16; ++dt)
+            *reinterpret_cast<uint32_t*>(out + (head0 + h) * kD + dt * 8 + 2 * tg) =
+                pack_bf2(o[dt][2 * hh] * inv, o[dt][2 * hh + 1] * inv);
+          if (tg == 0 && lse != nullptr)
+            lse[head0 + h] = l_r[hh] > 0.f ? (m_r[hh] + log2f(l_r[hh])) * kLn2 : -INFINITY;
+        }
+      }
+    } else {
+      const int j = (int)(w - w_first);
+      const long long slot = ((long long)p * pl.cmax + j) * G;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = gq + 8 * hh;
+        if (h < G) {
+#pragma unroll
+          for (int dt = 0; dt < 16; ++dt)
+            *reinterpret_cast<float2*>(part_o + (slot + h) * kD + dt * 8 + 2 * tg) =
+                make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
+          if (tg == 0) {
+            part_ml[(slot + h) * 2] = m_r[hh];
+            part_ml[(slot + h) * 2 + 1] = l_r[hh];
+          }
+        }
+      }
+      __syncwarp();
+      unsigned last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(ticket + p, 1u) == (unsigned)(ncontrib - 1);
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();
+        const long long base = (long long)p * pl.cmax * G;
+        for (int h = 0; h < G; ++h) {
+          float M = -INFINITY;
+          for (int x = 0; x < ncontrib; ++x) M = fmaxf(M, __ldcg(part_ml + (base + (long long)x * G + h) * 2));
+          float L = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+          if (M != -INFINITY) {
+            for (int x = 0; x < ncontrib; ++x) {
+              const long long sl = base + (long long)x * G + h;
+              const float mx = __ldcg(part_ml + sl * 2), lx = __ldcg(part_ml + sl * 2 + 1);
+              if (lx == 0.f) continue;
+              const float wt = exp2f(mx - M);
+              L = fmaf(lx, wt, L);
+              const float4 ov = __ldcg(reinterpret_cast<const float4*>(part_o + sl * kD + lane * 4));
+              a[0] = fmaf(ov.x, wt, a[0]);
+              a[1] = fmaf(ov.y, wt, a[1]);
+              a[2] = fmaf(ov.z, wt, a[2]);
+              a[3] = fmaf(ov.w, wt, a[3]);
+            }
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          *reinterpret_cast<uint2*>(out + (head0 + h) * kD + lane * 4) =
+              make_uint2(pack_bf2(a[0] * inv, a[1] * inv), pack_bf2(a[2] * inv, a[3] * inv));
+          if (lane == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        }
+        if (lane == 0) ticket[p] = 0u;  // ready for the next call
+      }
+    }
+    t = seg_end;
+  }
+}
+
+DecPlan decode_plan(int B, int Hkv, int k) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms = n > 0 ? n : 148;
+  }
+  DecPlan pl;
+  pl.pairs = B * Hkv;
+  pl.tpp = (k + kDecTile - 1) / kDecTile;
+  pl.T = (long long)pl.pairs * pl.tpp;
+  // resident warps (2 CTAs of kDecWarps per SM), but at least 2 tiles per warp
+  long long W = (long long)sms * 2 * kDecWarps;
+  const long long by_tiles = (pl.T + 1) / 2;
+  if (W > by_tiles) W = by_tiles;
+  if (W < 1) W = 1;
+  pl.W = W;
+  // warps meeting one pair's tile range: at most (tpp-1)*W/T + 2
+  pl.cmax = (int)((W + pl.pairs - 1) / pl.pairs) + 2;
+  return pl;
 }
 
 }  // namespace
@@ -360,17 +569,17 @@ static size_t align256a(size_t x) { return (x + 255) & ~size_t(255); }
 
 // The merge tickets sit in a fixed region at the start of the workspace
 // (room for kTicketSlots (sequence, kv head) pairs) that holds nothing else,
-// so a zero-filled workspace stays valid across calls of any shape: the last
-// CTA of every pair returns its ticket to zero.
+// so a zero-filled workspace stays valid across calls of any shape: the warp
+// that merges a pair returns its ticket to zero.
 constexpr int kTicketSlots = 16384;
 
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
   (void)D;
-  int tps, S;
-  decode_split(B, Hkv, k, &tps, &S);
+  const DecPlan pl = decode_plan(B, Hkv, k);
+  const int G = Hq / Hkv;
   const size_t tk = (size_t)kTicketSlots * 4;
-  const size_t po = align256a((size_t)B * Hq * S * kD * 4);
-  const size_t pml = align256a((size_t)B * Hq * S * 2 * 4);
+  const size_t po = align256a((size_t)pl.pairs * pl.cmax * G * kD * 4);
+  const size_t pml = align256a((size_t)pl.pairs * pl.cmax * G * 2 * 4);
   return tk + po + pml;
 }
 
@@ -379,19 +588,19 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
                                int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,
                                cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
-  int tps, S;
-  decode_split(B, Hkv, k, &tps, &S);
+  const DecPlan pl = decode_plan(B, Hkv, k);
+  const int G = Hq / Hkv;
   char* p = static_cast<char*>(ws);
   unsigned* ticket = reinterpret_cast<unsigned*>(p);
   p += (size_t)kTicketSlots * 4;
   float* po = reinterpret_cast<float*>(p);
-  p += align256a((size_t)B * Hq * S * kD * 4);
+  p += align256a((size_t)pl.pairs * pl.cmax * G * kD * 4);
   float* pml = reinterpret_cast<float*>(p);
-  cudaError_t e;
-  if ((e = ensure_dynamic_smem((const void*)attn_decode_kernel, kSmemTotal)) != cudaSuccess) return e;
-  dim3 grid(S, Hkv, B);
-  attn_decode_kernel<<<grid, 128, kSmemTotal, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k, tps, S,
-                                                    scale * kLog2e, po, pml, ticket, out, lse);
+  cudaError_t e = ensure_dynamic_smem((const void*)attn_decode_kernel, kDecSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = (int)((pl.W + kDecWarps - 1) / kDecWarps);
+  attn_decode_kernel<<<grid, kDecWarps * 32, kDecSmem, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k, pl,
+                                                            scale * kLog2e, po, pml, ticket, out, lse);
   return cudaGetLastError();
 }
 

