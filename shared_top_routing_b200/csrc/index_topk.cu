@@ -76,18 +76,21 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
   constexpr int WARPS = kScoreThreads / 32;
   __shared__ uint32_t sh[kHistBins];
 
-  // The B x Tk row space is flattened and split evenly over the grid, so
-  // every CTA streams the same number of key rows.
-  const long long F = (long long)B * Tk;
-  const long long lo = F * blockIdx.x / gridDim.x, hi = F * (blockIdx.x + 1) / gridDim.x;
+  // The B x Tk row space (each batch padded to a multiple of 8 rows) is
+  // flattened and split evenly over the grid at multiples of 8 rows, so every
+  // CTA streams the same number of key rows and 8-row tiles stay aligned.
+  const long long Tp = ((long long)Tk + 7) & ~7ll;
+  const long long F = (long long)B * Tp;
+  const long long lo = (F * blockIdx.x / gridDim.x) & ~7ll;
+  const long long hi = blockIdx.x + 1 == gridDim.x ? F : ((F * (blockIdx.x + 1) / gridDim.x) & ~7ll);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
 
-  for (int b = (int)(lo / Tk); b < B && (long long)b * Tk < hi; ++b) {
-    const long long base_f = (long long)b * Tk;
+  for (int b = (int)(lo / Tp); b < B && (long long)b * Tp < hi; ++b) {
+    const long long base_f = (long long)b * Tp;
     const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
     const int r0 = (int)((lo > base_f ? lo : base_f) - base_f);
-    const int r1 = (int)min((long long)n, (hi < base_f + Tk ? hi : base_f + Tk) - base_f);
+    const int r1 = (int)min((long long)n, (hi < base_f + Tp ? hi : base_f + Tp) - base_f);
     if (r0 >= r1) continue;
     if (hist != nullptr) {
       for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
@@ -129,11 +132,8 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
         if (g == 0) {
           const int row = base + u * 8 + 2 * tg;
           const uint32_t k0 = score_key(c[0]), k1 = score_key(c[1]);
-          if (row + 1 < r1) {
-            *reinterpret_cast<uint2*>(kout + row) = make_uint2(k0, k1);
-          } else if (row < r1) {
-            kout[row] = k0;
-          }
+          if (row < r1) kout[row] = k0;
+          if (row + 1 < r1) kout[row + 1] = k1;
           if (hist != nullptr) {
             if (row < r1) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
             if (row + 1 < r1) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
