@@ -508,30 +508,56 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
       }
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
+        // warp-parallel merge: lane x holds contributor x's (m, l) per head
+        // (at most 32 contributors per pair, see decode_plan)
         __threadfence();
         const long long base = (long long)p * pl.cmax * G;
-        for (int h = 0; h < G; ++h) {
-          float M = -INFINITY;
-          for (int x = 0; x < ncontrib; ++x) M = fmaxf(M, __ldcg(part_ml + (base + (long long)x * G + h) * 2));
-          float L = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
-          if (M != -INFINITY) {
-            for (int x = 0; x < ncontrib; ++x) {
-              const long long sl = base + (long long)x * G + h;
-              const float mx = __ldcg(part_ml + sl * 2), lx = __ldcg(part_ml + sl * 2 + 1);
-              if (lx == 0.f) continue;
-              const float wt = exp2f(mx - M);
-              L = fmaf(lx, wt, L);
-              const float4 ov = __ldcg(reinterpret_cast<const float4*>(part_o + sl * kD + lane * 4));
-              a[0] = fmaf(ov.x, wt, a[0]);
-              a[1] = fmaf(ov.y, wt, a[1]);
-              a[2] = fmaf(ov.z, wt, a[2]);
-              a[3] = fmaf(ov.w, wt, a[3]);
+        float wgt[16], Lh[16], Mh[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          wgt[h] = 0.f;
+          Lh[h] = 0.f;
+          Mh[h] = -INFINITY;
+          if (h < G) {
+            const long long sl = base + (long long)lane * G + h;
+            const float mx = lane < ncontrib ? __ldcg(part_ml + sl * 2) : -INFINITY;
+            const float lx = lane < ncontrib ? __ldcg(part_ml + sl * 2 + 1) : 0.f;
+            const float M = warp_max(mx);
+            const float wv = (lx > 0.f && M != -INFINITY) ? exp2f(mx - M) : 0.f;
+            wgt[h] = wv;
+            Lh[h] = warp_sum(lx * wv);
+            Mh[h] = M;
+          }
+        }
+        float acc[16][4];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+#pragma unroll 2
+        for (int x = 0; x < ncontrib; ++x) {
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            if (h < G) {
+              const float wt = __shfl_sync(0xffffffffu, wgt[h], x);
+              if (wt != 0.f) {
+                const float4 ov =
+                    __ldcg(reinterpret_cast<const float4*>(part_o + (base + (long long)x * G + h) * kD + lane * 4));
+                acc[h][0] = fmaf(ov.x, wt, acc[h][0]);
+                acc[h][1] = fmaf(ov.y, wt, acc[h][1]);
+                acc[h][2] = fmaf(ov.z, wt, acc[h][2]);
+                acc[h][3] = fmaf(ov.w, wt, acc[h][3]);
+              }
             }
           }
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          *reinterpret_cast<uint2*>(out + (head0 + h) * kD + lane * 4) =
-              make_uint2(pack_bf2(a[0] * inv, a[1] * inv), pack_bf2(a[2] * inv, a[3] * inv));
-          if (lane == 0 && lse != nullptr) lse[head0 + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          if (h < G) {
+            const float inv = Lh[h] > 0.f ? 1.f / Lh[h] : 0.f;
+            *reinterpret_cast<uint2*>(out + (head0 + h) * kD + lane * 4) =
+                make_uint2(pack_bf2(acc[h][0] * inv, acc[h][1] * inv), pack_bf2(acc[h][2] * inv, acc[h][3] * inv));
+            if (lane == 0 && lse != nullptr)
+              lse[head0 + h] = Lh[h] > 0.f ? (Mh[h] + log2f(Lh[h])) * kLn2 : -INFINITY;
+          }
         }
         if (lane == 0) ticket[p] = 0u;  // ready for the next call
       }
@@ -552,10 +578,12 @@ DecPlan decode_plan(int B, int Hkv, int k) {
   pl.pairs = B * Hkv;
   pl.tpp = (k + kDecTile - 1) / kDecTile;
   pl.T = (long long)pl.pairs * pl.tpp;
-  // resident warps (2 CTAs of kDecWarps per SM), but at least 2 tiles per warp
+  // resident warps (2 CTAs of kDecWarps per SM), but at least 2 tiles per
+  // warp and at most 30 warps per pair (the merge keeps one contributor per lane)
   long long W = (long long)sms * 2 * kDecWarps;
   const long long by_tiles = (pl.T + 1) / 2;
   if (W > by_tiles) W = by_tiles;
+  if (W > 30ll * pl.pairs) W = 30ll * pl.pairs;
   if (W < 1) W = 1;
   pl.W = W;
   // warps meeting one pair's tile range: at most (tpp-1)*W/T + 2

@@ -442,22 +442,32 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
     if (mode == kFinishHistScan) {
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
-      // keep every key in or above the bin of the K-th largest
-      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4) {
-        const int i = i0 + tid * 4;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (i + 3 < n) {
-          v = *reinterpret_cast<const uint4*>(row + i);
-        } else {
-          if (i < n) v.x = row[i];
-          if (i + 1 < n) v.y = row[i + 1];
-          if (i + 2 < n) v.z = row[i + 2];
-        }
-        const uint32_t kk4[4] = {v.x, v.y, v.z, v.w};
+      // keep every key in or above the bin of the K-th largest; each thread
+      // issues all its 16-byte loads before filtering
+      constexpr int kPer = 8;
+      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4 * kPer) {
+        uint4 v[kPer];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool take = i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin;
-          push_cand(s, take, kk4[j], (uint32_t)(i + j));
+        for (int u = 0; u < kPer; ++u) {
+          const int i = i0 + (u * kFinThreads + tid) * 4;
+          v[u] = make_uint4(0, 0, 0, 0);
+          if (i + 3 < n) {
+            v[u] = *reinterpret_cast<const uint4*>(row + i);
+          } else {
+            if (i < n) v[u].x = row[i];
+            if (i + 1 < n) v[u].y = row[i + 1];
+            if (i + 2 < n) v[u].z = row[i + 2];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int i = i0 + (u * kFinThreads + tid) * 4;
+          const uint32_t kk4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool take = i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin;
+            push_cand(s, take, kk4[j], (uint32_t)(i + j));
+          }
         }
       }
       __syncthreads();
