@@ -362,13 +362,19 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
       for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
     float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
 
-    // pipeline prologue
+    // pipeline prologue; the row indices of the tile gathered next are
+    // loaded one iteration ahead so no gather waits on an index load
+    auto idx_of = [&](int tile) -> int {
+      const int i = (first_tile + tile) * kDecTile + (lane & 15);
+      return (tile < ntiles && i < cnt) ? clamp_row(irow[i], Tk_max) : 0;
+    };
+    int jl_next = idx_of(kDecStages - 1);
 #pragma unroll
     for (int sIdx = 0; sIdx < kDecStages - 1; ++sIdx) {
       if (sIdx < ntiles) {
         const int i0 = (first_tile + sIdx) * kDecTile;
-        const int jl = i0 + (lane & 15) < cnt ? clamp_row(irow[i0 + (lane & 15)], Tk_max) : 0;
-        dec_gather(ring + sIdx * (kDecStageBytes / 2), kc, vc, jl, i0, cnt, head_base, row_elems, Tk_max, lane);
+        dec_gather(ring + sIdx * (kDecStageBytes / 2), kc, vc, idx_of(sIdx), i0, cnt, head_base, row_elems,
+                   Tk_max, lane);
       }
       cp_async_commit();
     }
@@ -376,10 +382,10 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
       const int nxt = it + kDecStages - 1;
       if (nxt < ntiles) {
         const int i0 = (first_tile + nxt) * kDecTile;
-        const int jl = i0 + (lane & 15) < cnt ? clamp_row(irow[i0 + (lane & 15)], Tk_max) : 0;
-        dec_gather(ring + (nxt % kDecStages) * (kDecStageBytes / 2), kc, vc, jl, i0, cnt, head_base,
+        dec_gather(ring + (nxt % kDecStages) * (kDecStageBytes / 2), kc, vc, jl_next, i0, cnt, head_base,
                    row_elems, Tk_max, lane);
       }
+      jl_next = idx_of(nxt + 1);
       cp_async_commit();
       cp_async_wait<kDecStages - 1>();
       __syncwarp();
