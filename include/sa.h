@@ -160,6 +160,32 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
                                 void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Decode attention without a caller workspace.
+ *
+ * No counterpart in the paper: this is an interface for callers that cannot
+ * call cudaMalloc -- for example a host process that may only pass on the
+ * buffers it was handed, or code on a path where allocation is not allowed
+ * -- and so cannot supply the workspace sa_sparse_attn_decode needs.
+ * Arguments, results and limits are those of sa_sparse_attn_decode.  The
+ * scratch is a fixed array of SA_NOALLOC_SCRATCH_BYTES inside the library,
+ * held on every GPU that loads it until the process exits; shapes that need
+ * more scratch (sa_sparse_attn_decode_workspace(...) > SA_NOALLOC_SCRATCH_BYTES)
+ * are rejected with SA_ERR_UNSUPPORTED.  The call allocates nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call clears, on `stream`, the part of the array that must start
+ *     at zero, then leaves its results in the array until the next call.
+ *   - All calls share the one array: calls that overlap on the GPU (e.g. on
+ *     different streams) race and give undefined results.
+ * ---------------------------------------------------------------------- */
+#define SA_NOALLOC_SCRATCH_BYTES (8u << 20)
+sa_status sa_sparse_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* idx, const int32_t* count,
+                                        int B, int Tk_max, int Hq, int Hkv, int D, int k,
+                                        float scale, void* out, float* lse, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Gist-chunk routing with selective unfolding (decode).
  *
  * [SSA] §二/§三 and [GSA] 2.1-2.2: the sequence is cut into chunks of

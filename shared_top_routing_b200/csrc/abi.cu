@@ -94,6 +94,25 @@ sa_status validate_attn(const void* q, const void* kc, const void* vc, const int
 
 namespace sa {
 
+sa_status check_decode_args(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                            const int32_t* count, int B, int Tk_max, int Hq, int Hkv, int D, int k,
+                            const void* out) {
+  sa_status st = validate_attn(q, kc, vc, idx, count, B, 1, Tk_max, Hq, Hkv, D, k, out);
+  if (st != SA_OK) return st;
+  if ((long long)B * Hkv > SA_DECODE_MAX_PAIRS)
+    return fail(SA_ERR_UNSUPPORTED, "B*Hkv=%lld exceeds %d", (long long)B * Hkv, SA_DECODE_MAX_PAIRS);
+  return SA_OK;
+}
+
+void set_last_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
 cudaError_t ensure_dynamic_smem(const void* func, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   static std::mutex mu;

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/sa.h"
+
 namespace sa {
 
 // Rows of at most this many candidates are selected by one CTA holding the
@@ -44,6 +46,14 @@ struct FinishOut {
   const int32_t* partial_len = nullptr;
   int32_t* chunks = nullptr;     // [B, k] or null
 };
+
+// Host-side argument check of sa_sparse_attn_decode (sets the error detail).
+sa_status check_decode_args(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                            const int32_t* count, int B, int Tk_max, int Hq, int Hkv, int D, int k,
+                            const void* out);
+
+// Sets the detail string sa_last_error() returns for this host thread.
+void set_last_error(const char* fmt, ...);
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* func, size_t bytes);

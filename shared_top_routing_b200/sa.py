@@ -40,6 +40,7 @@ SIGNATURES = {
     "sa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
+    "sa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
     "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
@@ -221,6 +222,27 @@ def sa_sparse_attn_decode(q, k_cache, v_cache, idx, count, scale: float = 0.0, o
                                      B, Tk_max, Hq, Hkv, D, k, scale, _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "sa_sparse_attn_decode")
+    return (out, lse) if with_lse else out
+
+
+def sa_sparse_attn_decode_noalloc(q, k_cache, v_cache, idx, count, scale: float = 0.0, out=None,
+                                  with_lse: bool = False, stream=None):
+    """sa_sparse_attn_decode for callers that cannot allocate: no workspace
+    argument; the library's fixed scratch array is used (see sa.h)."""
+    torch = _torch()
+    B, Hq, D = q.shape
+    _, Tk_max, Hkv, _ = k_cache.shape
+    k = idx.shape[-1]
+    for t, n, sz in ((q, "q", 2), (k_cache, "k_cache", 2), (v_cache, "v_cache", 2),
+                     (idx, "idx", 4), (count, "count", 4)):
+        _need(t, n, sz)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    st = lib().sa_sparse_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx),
+                                             _ptr(count), B, Tk_max, Hq, Hkv, D, k, scale, _ptr(out),
+                                             _ptr(lse), _stream(stream))
+    _check(st, "sa_sparse_attn_decode_noalloc")
     return (out, lse) if with_lse else out
 
 
