@@ -393,19 +393,27 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
       const uint16_t* tV = tK + kDecTile * kLds;
       const int rbase = (first_tile + it) * kDecTile;
       if (rbase < cnt) {
-        float sc[2][4];
+        // S = Q K^T over 8 k-steps, in two independent accumulator chains
+        float sc[2][4], sd[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; kk += 2) {
           const int mtx = lane >> 3;
-          uint32_t b0, b1, b2, b3;
+          uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
           ldmatrix_x4(b0, b1, b2, b3, tK + ((mtx >> 1) * 8 + (lane & 7)) * kLds + kk * 16 + (mtx & 1) * 8);
+          ldmatrix_x4(c0, c1, c2, c3, tK + ((mtx >> 1) * 8 + (lane & 7)) * kLds + (kk + 1) * 16 + (mtx & 1) * 8);
           mma_bf16_16816(sc[0], qa[kk], b0, b1);
           mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          mma_bf16_16816(sd[0], qa[kk + 1], c0, c1);
+          mma_bf16_16816(sd[1], qa[kk + 1], c2, c3);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] += sd[nt][e];
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -444,12 +452,14 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
           v += __shfl_xor_sync(0xffffffffu, v, 2);
           l_r[hh] = l_r[hh] * alpha[hh] + v;
         }
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {  // a row max moved
 #pragma unroll
-        for (int dt = 0; dt < 16; ++dt) {
-          o[dt][0] *= alpha[0];
-          o[dt][1] *= alpha[0];
-          o[dt][2] *= alpha[1];
-          o[dt][3] *= alpha[1];
+          for (int dt = 0; dt < 16; ++dt) {
+            o[dt][0] *= alpha[0];
+            o[dt][1] *= alpha[0];
+            o[dt][2] *= alpha[1];
+            o[dt][3] *= alpha[1];
+          }
         }
         uint32_t pa[4];
         pa[0] = pack_bf2(sc[0][0], sc[0][1]);
@@ -535,23 +545,23 @@ attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
             Mh[h] = M;
           }
         }
+        // o: every contributor's partial (zero where it saw no rows) scaled by
+        // its weight; no branch in the loop, so the loads overlap
         float acc[16][4];
 #pragma unroll
         for (int h = 0; h < 16; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
-#pragma unroll 2
+        const float* po_base = part_o + base * kD + lane * 4;
+#pragma unroll 4
         for (int x = 0; x < ncontrib; ++x) {
 #pragma unroll
           for (int h = 0; h < 16; ++h) {
             if (h < G) {
               const float wt = __shfl_sync(0xffffffffu, wgt[h], x);
-              if (wt != 0.f) {
-                const float4 ov =
-                    __ldcg(reinterpret_cast<const float4*>(part_o + (base + (long long)x * G + h) * kD + lane * 4));
-                acc[h][0] = fmaf(ov.x, wt, acc[h][0]);
-                acc[h][1] = fmaf(ov.y, wt, acc[h][1]);
-                acc[h][2] = fmaf(ov.z, wt, acc[h][2]);
-                acc[h][3] = fmaf(ov.w, wt, acc[h][3]);
-              }
+              const float4 ov = __ldcg(reinterpret_cast<const float4*>(po_base + ((long long)x * G + h) * kD));
+              acc[h][0] = fmaf(ov.x, wt, acc[h][0]);
+              acc[h][1] = fmaf(ov.y, wt, acc[h][1]);
+              acc[h][2] = fmaf(ov.z, wt, acc[h][2]);
+              acc[h][3] = fmaf(ov.w, wt, acc[h][3]);
             }
           }
         }
