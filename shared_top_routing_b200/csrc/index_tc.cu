@@ -200,185 +200,6 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
-// ----------------------------------------------------------- decode scoring
-//
-// One query per sequence: the indexer-key cache is streamed through a
-// STAGES-deep ring by TMA (128 keys x d per tile, 128-byte swizzle) and each
-// tile is scored by tcgen05 with the keys as the 128-row M side and the query
-// block as N = 16 (row 0 is this sequence's query; the other rows hold the
-// following queries and are ignored).  Epilogue thread i reads the score of
-// key i from TMEM column 0, writes its 32-bit order-preserving key and counts
-// it in a shared 4096-bin histogram of the top 12 bits, flushed to global
-// memory per sequence.  The B x ceil(Tk/128) tiles are split evenly over one
-// CTA per SM.
-
-constexpr int kDecBM = 128;   // keys per tile (M)
-constexpr int kDecBN = 16;    // query rows (N)
-
-template <int D>
-struct DecTcShape {
-  static constexpr int kAtoms = D / 64;
-  static constexpr int kABytes = kDecBM * D * 2;   // keys
-  static constexpr int kBBytes = kDecBN * D * 2;   // queries
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = D == 64 ? 8 : 4;
-  static constexpr int kSmem = 1024 + kStages * kStageBytes + 4 * kHistBins * 4 + 256;
-};
-
-struct DecTcBars {
-  uint64_t full[8];
-  uint64_t empty[8];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint32_t tmem_base;
-  int abort;
-};
-
-struct DecTcParams {
-  int B, Tk, q_pos0, tpb;       // tiles per batch
-  const int32_t* kv_len;
-  uint32_t* keys;
-  long long ld;
-  uint32_t* hist;
-  int* err;
-};
-
-__device__ __forceinline__ int dec_n(const DecTcParams& p, int b) {
-  return tc_n_cand(p.q_pos0, 0, tc_row_len(p.kv_len, b, p.Tk));
-}
-
-template <int D>
-__global__ void __launch_bounds__(192, 1)
-score_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
-                       DecTcParams p) {
-  using S = DecTcShape<D>;
-  extern __shared__ unsigned char smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  unsigned char* base = smem_raw + ((1024 - (raw & 1023)) & 1023);
-  uint32_t* sh = reinterpret_cast<uint32_t*>(base + S::kStages * S::kStageBytes);
-  DecTcBars& bars = *reinterpret_cast<DecTcBars*>(base + S::kStages * S::kStageBytes + 4 * kHistBins * 4);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long F = (long long)p.B * p.tpb;
-  const long long lo = F * blockIdx.x / gridDim.x, hi = F * (blockIdx.x + 1) / gridDim.x;
-  if (lo >= hi) return;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S::kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&bars.tfull[a], 1); mbar_init(&bars.tempty[a], 4); }
-    bars.abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(&bars.tmem_base, 32);
-    tmem_relinquish();
-  }
-  for (int i = threadIdx.x; i < 4 * kHistBins; i += 192) sh[i] = 0;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = bars.tmem_base;
-  volatile int* abort_flag = &bars.abort;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int i = 0;  // index among valid tiles
-      for (long long f = lo; f < hi; ++f) {
-        const int b = (int)(f / p.tpb), t = (int)(f % p.tpb);
-        if (t * kDecBM >= dec_n(p, b)) continue;
-        const int s = i % S::kStages;
-        const uint32_t ph = (uint32_t)(i / S::kStages) & 1u;
-        if (!mbar_wait(&bars.empty[s], ph ^ 1u, abort_flag, p.err, 11)) break;
-        unsigned char* st = base + s * S::kStageBytes;
-        mbar_arrive_expect_tx(&bars.full[s], S::kStageBytes);
-#pragma unroll
-        for (int a = 0; a < S::kAtoms; ++a) {
-          tma_load_3d(st + a * kDecBM * 128, &tmap_k, &bars.full[s], 64 * a, t * kDecBM, b);
-          tma_load_3d(st + S::kABytes + a * kDecBN * 128, &tmap_q, &bars.full[s], 64 * a, b, 0);
-        }
-        ++i;
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kDecBM, kDecBN);
-      int i = 0;
-      for (long long f = lo; f < hi; ++f) {
-        const int b = (int)(f / p.tpb), t = (int)(f % p.tpb);
-        if (t * kDecBM >= dec_n(p, b)) continue;
-        const int s = i % S::kStages;
-        const uint32_t ph = (uint32_t)(i / S::kStages) & 1u;
-        const int acc = i & 1;
-        const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-        if (!mbar_wait(&bars.tempty[acc], aph ^ 1u, abort_flag, p.err, 12)) break;
-        if (!mbar_wait(&bars.full[s], ph, abort_flag, p.err, 13)) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(base + s * S::kStageBytes);
-        const uint32_t b_addr = a_addr + S::kABytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (uint32_t)((kk & 3) * 32);
-          const uint64_t adesc = sdesc_k_sw128(a_addr + (kk >> 2) * kDecBM * 128 + koff);
-          const uint64_t bdesc = sdesc_k_sw128(b_addr + (kk >> 2) * kDecBN * 128 + koff);
-          umma_bf16(tbase + (uint32_t)(acc * kDecBN), adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars.empty[s]);
-        umma_commit(&bars.tfull[acc]);
-        ++i;
-      }
-    }
-  } else {
-    // epilogue warps 2..5: TMEM lane quarter = warp % 4; thread = key row
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    uint32_t* wh = sh + (warp - 2) * kHistBins;  // this warp's histogram
-    auto flush = [&](int bb) {
-      __syncwarp();
-      uint32_t* hg = p.hist + (long long)bb * kHistBins;
-      for (int j = lane; j < kHistBins; j += 32) {
-        const uint32_t c = wh[j];
-        if (c) { atomicAdd(hg + j, c); wh[j] = 0; }
-      }
-      __syncwarp();
-    };
-    int i = 0;
-    int cur_b = -1;
-    for (long long f = lo; f < hi; ++f) {
-      const int b = (int)(f / p.tpb), t = (int)(f % p.tpb);
-      const int n = dec_n(p, b);
-      if (t * kDecBM >= n) continue;
-      if (b != cur_b) {
-        if (cur_b >= 0 && p.hist != nullptr) flush(cur_b);
-        cur_b = b;
-      }
-      const int acc = i & 1;
-      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-      if (!mbar_wait(&bars.tfull[acc], aph, abort_flag, p.err, 14)) break;
-      tc_fence_after();
-      uint32_t v;
-      asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
-                   : "=r"(v)
-                   : "r"(tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kDecBN)));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.tempty[acc]);
-      const int row = t * kDecBM + r;
-      if (row < n) {
-        const uint32_t key = score_key(__uint_as_float(v));
-        p.keys[(long long)b * p.ld + row] = key;
-        if (p.hist != nullptr) atomicAdd(&wh[key >> (32 - kHistBits)], 1u);
-      }
-      ++i;
-    }
-    if (cur_b >= 0 && p.hist != nullptr) flush(cur_b);
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tbase, 32);
-}
-
 // ------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -412,52 +233,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int d, long long rows, int batche
   return r == CUDA_SUCCESS;
 }
 
-// [rows][d] bf16 (a 2-D tensor of `rows` rows), box = 64 x box_rows, 128-byte swizzle.
-bool make_map_2d(CUtensorMap* m, const void* ptr, int d, long long rows, int box_rows) {
-  return make_map(m, ptr, d, rows, 1, box_rows);
-}
-
 }  // namespace
-
-cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, int d, int Tk_max,
-                                int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
-                                bool with_hist, cudaStream_t st) {
-  if (Tk <= 0 || B <= 0) return cudaSuccess;
-  CUtensorMap mk, mq;
-  if (!make_map(&mk, kmat, d, Tk_max, B, kDecBM) || !make_map_2d(&mq, q, d, B, kDecBN))
-    return cudaErrorInvalidValue;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    sms = n > 0 ? n : 148;
-  }
-  DecTcParams p;
-  p.B = B;
-  p.Tk = Tk;
-  p.q_pos0 = q_pos0;
-  p.tpb = (Tk + kDecBM - 1) / kDecBM;
-  p.kv_len = kv_len;
-  p.keys = w.keys;
-  p.ld = w.ld;
-  p.hist = with_hist ? w.hist : nullptr;
-  p.err = w.err;
-  const long long tiles = (long long)B * p.tpb;
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  if (d == 128) {
-    constexpr int smem = DecTcShape<128>::kSmem;
-    cudaError_t e = ensure_dynamic_smem((const void*)score_decode_tc_kernel<128>, smem);
-    if (e != cudaSuccess) return e;
-    score_decode_tc_kernel<128><<<grid, 192, smem, st>>>(mk, mq, p);
-  } else {
-    constexpr int smem = DecTcShape<64>::kSmem;
-    cudaError_t e = ensure_dynamic_smem((const void*)score_decode_tc_kernel<64>, smem);
-    if (e != cudaSuccess) return e;
-    score_decode_tc_kernel<64><<<grid, 192, smem, st>>>(mk, mq, p);
-  }
-  return cudaGetLastError();
-}
 
 cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,
                                  int Tk_max, int Tk, int q_pos0, const int32_t* kv_len, int t0,

@@ -6,7 +6,18 @@
 // token indices.  Selection rule: largest scores, equal scores by lower
 // position, emitted in ascending position order.
 //
-// Kernels (decode and prefill scoring live in index_tc.cu)
+// Kernels
+//   score_decode_kernel  one query per sequence.  The indexer-key cache is
+//       streamed with 16-byte loads straight into mma.sync B fragments: a dot
+//       product is invariant to the order of its terms, so lane (g, t) of a
+//       warp loads whole 16-byte chunks 4j+t of key row g and the query
+//       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
+//       keys (the query is row 0 of the 16-row A side).  Writes the order-
+//       preserving 32-bit score key of every candidate and a 4096-bin
+//       histogram of the keys' top 12 bits.  The B x Tk key rows are
+//       flattened and split evenly (at multiples of 8 rows) over a grid sized
+//       to the resident CTAs.  (A TMA + tcgen05 variant was measured slower
+//       here: with 128x16 tiles the per-tile TMEM hand-off dominates.)
 //   collect_kernel       (rows longer than one CTA can scan) finds, from the
 //       histogram, the bin holding the k-th largest key and appends every key
 //       in that bin or above to a per-row candidate list (one atomic per CTA).
@@ -27,6 +38,7 @@
 namespace sa {
 namespace {
 
+constexpr int kScoreThreads = 256;
 constexpr int kFinThreads = 1024;
 constexpr int kSmemCand = 8192;          // candidates held in shared memory
 constexpr int kBitmapMax = 1 << 18;      // rows up to this length emit through a bitmap
@@ -53,6 +65,93 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // ------------------------------------------------------------------ scoring
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads)
+score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int B, int Tk_max,
+                    int Tk, int q_pos0, const int32_t* __restrict__ kv_len,
+                    uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist) {
+  constexpr int J = D / 32;          // 16-byte chunks per lane per key row
+  constexpr int U = 4;               // 8-row tiles per warp iteration
+  constexpr int WARPS = kScoreThreads / 32;
+  __shared__ uint32_t sh[kHistBins];
+
+  // The B x Tk row space (each batch padded to a multiple of 8 rows) is
+  // flattened and split evenly over the grid at multiples of 8 rows, so every
+  // CTA streams the same number of key rows and 8-row tiles stay aligned.
+  const long long Tp = ((long long)Tk + 7) & ~7ll;
+  const long long F = (long long)B * Tp;
+  const long long lo = (F * blockIdx.x / gridDim.x) & ~7ll;
+  const long long hi = blockIdx.x + 1 == gridDim.x ? F : ((F * (blockIdx.x + 1) / gridDim.x) & ~7ll);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tg = lane & 3;
+
+  for (int b = (int)(lo / Tp); b < B && (long long)b * Tp < hi; ++b) {
+    const long long base_f = (long long)b * Tp;
+    const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
+    const int r0 = (int)((lo > base_f ? lo : base_f) - base_f);
+    const int r1 = (int)min((long long)n, (hi < base_f + Tp ? hi : base_f + Tp) - base_f);
+    if (r0 >= r1) continue;
+    if (hist != nullptr) {
+      for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
+      __syncthreads();
+    }
+    // A fragments: the query is row 0 of the 16-row A side, so only lanes
+    // with g == 0 hold data.  Chunk 4j+t (dims 8(4j+t) .. +7) feeds two
+    // k-steps: words x, y as (a0, a2) of one and z, w as (a0, a2) of the next.
+    uint32_t qe[J][2], qo[J][2];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (g == 0) v = *reinterpret_cast<const uint4*>(q + (long long)b * D + (4 * j + tg) * 8);
+      qe[j][0] = v.x; qe[j][1] = v.y;
+      qo[j][0] = v.z; qo[j][1] = v.w;
+    }
+    const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
+    uint32_t* kout = keys + (long long)b * ld;
+    for (int base = r0 + warp * 8 * U; base < r1; base += WARPS * 8 * U) {
+      uint4 v[U][J];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int row = base + u * 8 + g;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+          v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          const uint32_t a_even[4] = {qe[j][0], 0u, qe[j][1], 0u};
+          const uint32_t a_odd[4] = {qo[j][0], 0u, qo[j][1], 0u};
+          mma_bf16_16816(c, a_even, v[u][j].x, v[u][j].y);
+          mma_bf16_16816(c, a_odd, v[u][j].z, v[u][j].w);
+        }
+        // row 0 of C: lanes 0..3 hold the scores of tile rows 2t and 2t+1
+        if (g == 0) {
+          const int row = base + u * 8 + 2 * tg;
+          const uint32_t k0 = score_key(c[0]), k1 = score_key(c[1]);
+          if (row < r1) kout[row] = k0;
+          if (row + 1 < r1) kout[row + 1] = k1;
+          if (hist != nullptr) {
+            if (row < r1) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
+            if (row + 1 < r1) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
+          }
+        }
+      }
+    }
+    if (hist != nullptr) {
+      __syncthreads();
+      uint32_t* hg = hist + (long long)b * kHistBins;
+      for (int i = tid; i < kHistBins; i += kScoreThreads) {
+        const uint32_t cnt = sh[i];
+        if (cnt) atomicAdd(hg + i, cnt);
+      }
+      __syncthreads();
+    }
+  }
+}
 
 // ------------------------------------------------------------ block scans
 
@@ -552,6 +651,41 @@ void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, b
     p += align256((size_t)rows * kCandCap * 4);
     o->cand_pos = reinterpret_cast<uint32_t*>(p);
   }
+}
+
+template <int D>
+int score_grid(long long rows) {
+  static int per_sm[2] = {0, 0};
+  static int sms = 0;
+  int& occ = per_sm[D == 128];
+  if (occ == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    int o = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_decode_kernel<D>, kScoreThreads, 0);
+    sms = n > 0 ? n : 148;
+    occ = o > 0 ? o : 1;
+  }
+  long long want = (long long)sms * occ;
+  const long long by_rows = (rows + 255) / 256;  // at least 256 key rows per CTA
+  if (want > by_rows) want = by_rows;
+  return (int)(want < 1 ? 1 : want);
+}
+
+cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, int d, int Tk_max,
+                                int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
+                                bool with_hist, cudaStream_t st) {
+  if (Tk <= 0 || B <= 0) return cudaSuccess;
+  uint32_t* hist = with_hist ? w.hist : nullptr;
+  const long long rows = (long long)B * Tk;
+  if (d == 128)
+    score_decode_kernel<128><<<score_grid<128>(rows), kScoreThreads, 0, st>>>(
+        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
+  else
+    score_decode_kernel<64><<<score_grid<64>(rows), kScoreThreads, 0, st>>>(
+        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
