@@ -193,8 +193,9 @@ class DecodeBench:
                     for _ in range(c.n_layers)]
         self.graphs = {}
         self.events = {}
-        # kernels per indexer run: score + finish, plus collect for rows longer than one CTA scans
-        self.launches_per_step = c.n_groups * (3 if c.Tk_max > (1 << 18) else 2) + c.n_layers
+        # kernels per indexer run: score + finish, plus collect for rows longer
+        # than one CTA scans; per attention call: split + merge
+        self.launches_per_step = c.n_groups * (3 if c.Tk_max > (1 << 18) else 2) + 2 * c.n_layers
 
     def step(self, s: int, ev=None):
         c, sa = self.cfg, self.sa
@@ -323,7 +324,8 @@ def run_native(args, cfg, rank, world):
 
     score_bytes, attn_bytes = b.algorithmic_bytes()
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms else None
-    roof = {"kernel": "attn_decode_kernel", "bound": "hbm", "achieved": round(attn_gbs, 1) if attn_gbs else None,
+    roof = {"kernel": "attn_decode_split_kernel + attn_decode_merge_kernel (one decode attention call)",
+            "bound": "hbm", "achieved": round(attn_gbs, 1) if attn_gbs else None,
             "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(attn_gbs / peaks["hbm_gbs"], 4) if attn_gbs else None,
             "traffic": args.traffic, "peak_source": peaks["source"],
@@ -464,7 +466,7 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
             sa.sa_sparse_attn_decode(inp["q"][s], inp["K"], inp["V"], rows, cnt, out=out, ws=ws_a)
         n_steps, unit, per = cfg.steps, "steps/s", 1
         nbytes = cfg.B * cfg.n_chunks * cfg.d * 2 + cfg.B * rows_cap * cfg.Hkv * cfg.D * 4
-        launches = 3
+        launches = 4   # gist score, finish, attention split, attention merge
     else:
         inp = TI.prefill_inputs(cfg, dev)
         cache = sa.IndexCache(cfg.n_layers, cfg.B, cfg.L, cfg.k, share_every=cfg.share_every, device=dev)

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <string>
@@ -116,15 +117,16 @@ void set_last_error(const char* fmt, ...) {
 cudaError_t ensure_dynamic_smem(const void* func, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   static std::mutex mu;
-  static std::set<std::pair<const void*, int>> done;
+  static std::map<std::pair<const void*, int>, size_t> done;   // largest size set so far
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
   auto key = std::make_pair(func, dev);
-  if (done.count(key)) return cudaSuccess;
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) done.insert(key);
+  if (e == cudaSuccess) done[key] = bytes;
   return e;
 }
 

@@ -29,6 +29,7 @@
 
 #include "sa_common.cuh"
 #include "sa_internal.h"
+#include "tc_common.cuh"
 
 namespace sa {
 namespace {
@@ -273,312 +274,360 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 
 // ------------------------------------------------------------------ decode
 //
-// Balanced split of the decode work: the 16-row tiles of every (sequence, kv
-// head) pair form one list of T tiles, cut into equal contiguous ranges, one
-// per warp of a grid sized to the resident warps.  A warp streams its tiles
-// through its own STAGES-deep cp.async ring (no block barrier in the loop)
-// and writes a partial (m, l, o) whenever its range leaves a pair; the warp
-// whose ticket completes a pair merges that pair's partials.
+// K/V caches are [B, Tk_max, Hkv, D], so the rows of all kv heads at one
+// cache position are one contiguous run of Hkv * 256 bytes.  A work unit is
+// a tile of R selected positions of one sequence for a block of up to 8 kv
+// heads: one bulk copy per position and cache brings the whole run into
+// shared memory (no per-head 256-byte pieces).  The units of all sequences
+// form one list, cut into equal contiguous ranges, one per CTA of a grid of
+// one CTA per SM.
+//
+// CTA: warp 8 is the producer (row indices one unit ahead in registers,
+// bulk copies into a 3-stage ring, completion by mbarrier transaction
+// counts); warps 0..7 are consumers, warp c taking kv head c / wph of the
+// block and rows (c % wph) * 16 .. +16 of the tile (wph = 8 / heads per
+// block, so R = 16 * wph).  Each consumer runs online softmax on mma.sync
+// m16n8k16 with the G query heads of its kv head as the (zero padded) M
+// side and writes a partial (m, l, o) for every (sequence, head block) its
+// range meets.  attn_decode_merge_kernel then folds the partials of each
+// query head with the log-sum-exp rule, one CTA per (sequence, query head).
 
-constexpr int kDecWarps = 4;                 // warps per CTA
-constexpr int kDecStages = 3;                // per-warp ring depth
-constexpr int kDecTile = 16;                 // rows per warp tile
-constexpr size_t kDecStageBytes = (size_t)kDecTile * kLds * 2 * 2;   // K + V
-constexpr size_t kDecSmem = (size_t)kDecWarps * kDecStages * kDecStageBytes;
+constexpr int kDxConsumers = 8;
+constexpr int kDxThreads = (kDxConsumers + 1) * 32;
+constexpr int kDxStages = 3;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeMaxC = 1280;   // contributors of one (sequence, head block)
 
 struct DecPlan {
-  int pairs, tpp, cmax;
-  long long T, W;   // tiles, warps
+  int nh, wph, R, HB;     // heads per block, warps per head, rows per tile, blocks per sequence
+  int pairs, tpp;         // (sequence, block) pairs, tiles per pair
+  int row_bytes;          // padded shared row: nh * 256 + 16
+  int stage_bytes;        // K and V tiles of one stage
+  long long U, W;         // units, CTAs
 };
 
-// Warp owning tile t: the largest w with floor(w*T/W) <= t.
-__device__ __forceinline__ long long tile_owner(long long t, long long T, long long W) {
-  return ((t + 1) * W - 1) / T;
+// CTA owning unit u: the largest c with floor(c*U/W) <= u.
+__device__ __forceinline__ long long unit_owner(long long u, long long U, long long W) {
+  return ((u + 1) * W - 1) / U;
 }
 
-__device__ __forceinline__ void dec_gather(uint16_t* st, const uint16_t* __restrict__ kc,
-                                           const uint16_t* __restrict__ vc, int jlane, int i0, int end,
-                                           long long head_base, long long row_elems, int Tk_max, int lane) {
-  const int c = lane & 15;
-  uint16_t* sK = st;
-  uint16_t* sV = st + kDecTile * kLds;
-#pragma unroll
-  for (int pass = 0; pass < kDecTile / 2; ++pass) {
-    const int r = (lane >> 4) + 2 * pass;
-    const int j = __shfl_sync(0xffffffffu, jlane, r);
-    const bool v = i0 + r < end;
-    const long long off = head_base + (long long)(v ? j : 0) * row_elems + c * 8;
-    cp_async16(sK + r * kLds + c * 8, kc + off, v);
-    cp_async16(sV + r * kLds + c * 8, vc + off, v);
-  }
+__device__ __forceinline__ int clamp_count(const int32_t* __restrict__ count, int b, int k) {
+  const int c = count[b];
+  return c < 0 ? 0 : (c > k ? k : c);
 }
 
-__global__ void __launch_bounds__(kDecWarps * 32)
-attn_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
-                   const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
-                   const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k, DecPlan pl,
-                   float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
-                   unsigned* __restrict__ ticket, uint16_t* __restrict__ out, float* __restrict__ lse) {
+__global__ void __launch_bounds__(kDxThreads, 1)
+attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                         const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
+                         const int32_t* __restrict__ count, int Tk_max, int Hq, int Hkv, int k, DecPlan pl,
+                         float qscale, float* __restrict__ part_o, float* __restrict__ part_ml,
+                         int* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kDxStages * pl.stage_bytes);
+  uint64_t* empty = full + kDxStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDxStages);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gq = lane >> 2, tg = lane & 3;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDxStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kDxConsumers);
+    }
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  tc::pdl_wait();                 // inputs may come from the kernel before
+  tc::pdl_launch_dependents();    // the merge may start launching
+  const long long lo = (long long)blockIdx.x * pl.U / pl.W;
+  const long long hi = (long long)(blockIdx.x + 1) * pl.U / pl.W;
   const int G = Hq / Hkv;
-  const long long w = (long long)blockIdx.x * kDecWarps + warp;
-  if (w >= pl.W) return;
-  uint16_t* ring = reinterpret_cast<uint16_t*>(smem + (size_t)warp * kDecStages * kDecStageBytes);
-  const long long lo = w * pl.T / pl.W, hi = (w + 1) * pl.T / pl.W;
+  const int R = pl.R, rb = pl.row_bytes;
 
-  for (long long t = lo; t < hi;) {
-    const int p = (int)(t / pl.tpp);
-    const long long seg_end = min(hi, (long long)(p + 1) * pl.tpp);
-    const int b = p / Hkv, g = p % Hkv;
-    int cnt = count[b];
-    cnt = cnt < 0 ? 0 : (cnt > k ? k : cnt);
-    const int first_tile = (int)(t - (long long)p * pl.tpp);
-    const int ntiles = (int)(seg_end - t);
-    const int32_t* irow = idx + (long long)b * k;
-    const long long head_base = ((long long)b * Tk_max * Hkv + g) * kD;
-    const long long row_elems = (long long)Hkv * kD;
-    const long long head0 = (long long)b * Hq + (long long)g * G;
+  if (warp == kDxConsumers) {
+    // ------------------------------------------------------------ producer
+    // row indices of the next unit are loaded while the current one is
+    // issued; rows past the count repeat the last selected row so every
+    // byte of the tile is finite (their scores are masked)
+    int jr[4];
+    auto load_rows = [&](long long u, int* out_j) -> bool {
+      if (u >= hi) return false;
+      const int p = (int)(u / pl.tpp), b = p / pl.HB;
+      const int r0 = (int)(u % pl.tpp) * R;
+      const int cnt = clamp_count(count, b, k);
+      if (r0 >= cnt) return false;
+      const int32_t* irow = idx + (long long)b * k;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const int r = lane + 32 * qq;
+        const int i = r0 + min(r, cnt - 1 - r0);
+        out_j[qq] = r < R ? clamp_row(irow[i], Tk_max) : 0;
+      }
+      return true;
+    };
+    bool have = load_rows(lo, jr);
+    uint32_t fill = 0;
+    for (long long u = lo; u < hi; ++u) {
+      int jn[4];
+      const bool have_next = load_rows(u + 1, jn);
+      if (have) {
+        const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
+        const int h0 = hb * pl.nh;
+        const int nh_here = min(pl.nh, Hkv - h0);
+        const uint32_t bytes = (uint32_t)nh_here * 256u;
+        const int s = (int)(fill % kDxStages);
+        const uint32_t use = fill / kDxStages;
+        if (use > 0 && !tc::mbar_wait(&empty[s], (use - 1) & 1u, abort_flag, err, 11)) break;
+        unsigned char* stK = smem + (size_t)s * pl.stage_bytes;
+        unsigned char* stV = stK + (size_t)R * rb;
+        if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)R * bytes);
+        __syncwarp();
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int r = lane + 32 * qq;
+          if (r < R) {
+            const long long off = (((long long)b * Tk_max + jr[qq]) * Hkv + h0) * kD;
+            tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
+            tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
+          }
+        }
+        ++fill;
+      }
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) jr[qq] = jn[qq];
+      have = have_next;
+    }
+    // every copy this CTA issued lands before it exits
+    for (int s = 0; s < kDxStages; ++s) {
+      if ((uint32_t)s < fill) {
+        const uint32_t last_use = (fill - 1 - (uint32_t)s) / kDxStages;
+        tc::mbar_wait(&full[s], last_use & 1u, abort_flag, err, 12);
+      }
+    }
+    return;
+  }
 
-    // query fragments of the group's heads (rows >= G are zero)
-    uint32_t qa[8][4];
-    {
+  // -------------------------------------------------------------- consumers
+  const int gq = lane >> 2, tg = lane & 3;
+  const int hs = warp / pl.wph, rs = warp % pl.wph;
+  const int rs_el = rb / 2;   // shared row stride in elements
+  float o[16][4];
+  float m_r[2], l_r[2];
+  uint32_t qa[8][4];
+  int cur_p = -1;
+  bool active = false;        // this warp's head exists in the current block
+  long long head0 = 0;
+  uint32_t fill = 0;
+
+  auto flush = [&](int p) {
+    if (!active) return;
+    // CTA c's partial of pair p sits in slot p + c: the CTAs meeting pair
+    // p+1 start at or after the last one meeting p, so slots never collide
+    const long long slot = ((long long)p + blockIdx.x) * pl.wph + rs;
+    const long long base = (slot * pl.nh + hs) * G;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = gq + 8 * hh;
+      if (h < G) {
+#pragma unroll
+        for (int dt = 0; dt < 16; ++dt)
+          *reinterpret_cast<float2*>(part_o + (base + h) * kD + dt * 8 + 2 * tg) =
+              make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
+        if (tg == 0) *reinterpret_cast<float2*>(part_ml + (base + h) * 2) = make_float2(m_r[hh], l_r[hh]);
+      }
+    }
+  };
+
+  for (long long u = lo; u < hi; ++u) {
+    const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
+    if (p != cur_p) {
+      if (cur_p >= 0) flush(cur_p);
+      cur_p = p;
+      const int g = hb * pl.nh + hs;
+      active = hs < min(pl.nh, Hkv - hb * pl.nh);
+      head0 = (long long)b * Hq + (long long)(active ? g : 0) * G;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+      m_r[0] = m_r[1] = -INFINITY;
+      l_r[0] = l_r[1] = 0.f;
+      // query fragments of the group's heads (rows >= G are zero)
       const uint32_t* qr0 = reinterpret_cast<const uint32_t*>(q + (head0 + gq) * kD);
       const uint32_t* qr1 = reinterpret_cast<const uint32_t*>(q + (head0 + gq + 8) * kD);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const int c0 = (kk * 16 + 2 * tg) >> 1, c1 = (kk * 16 + 8 + 2 * tg) >> 1;
-        qa[kk][0] = gq < G ? __ldg(qr0 + c0) : 0u;
-        qa[kk][1] = gq + 8 < G ? __ldg(qr1 + c0) : 0u;
-        qa[kk][2] = gq < G ? __ldg(qr0 + c1) : 0u;
-        qa[kk][3] = gq + 8 < G ? __ldg(qr1 + c1) : 0u;
+        qa[kk][0] = active && gq < G ? __ldg(qr0 + c0) : 0u;
+        qa[kk][1] = active && gq + 8 < G ? __ldg(qr1 + c0) : 0u;
+        qa[kk][2] = active && gq < G ? __ldg(qr0 + c1) : 0u;
+        qa[kk][3] = active && gq + 8 < G ? __ldg(qr1 + c1) : 0u;
       }
     }
-    float o[16][4];
+    const int cnt = clamp_count(count, b, k);
+    const int r0 = (int)(u % pl.tpp) * R;
+    if (r0 >= cnt) continue;   // the producer skips this unit too
+    const int s = (int)(fill % kDxStages);
+    if (!tc::mbar_wait(&full[s], (fill / kDxStages) & 1u, abort_flag, err, 13)) break;
+    const int rbase = r0 + rs * 16;
+    if (active && rbase < cnt) {
+      const uint16_t* tK = reinterpret_cast<const uint16_t*>(smem + (size_t)s * pl.stage_bytes) +
+                           (size_t)(rs * 16) * rs_el + hs * kD;
+      const uint16_t* tV = tK + (size_t)R * rs_el;
+      // S = Q K^T over 8 k-steps, in two independent accumulator chains
+      float sc[2][4], sd[2][4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
-    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-
-    // pipeline prologue; the row indices of the tile gathered next are
-    // loaded one iteration ahead so no gather waits on an index load
-    auto idx_of = [&](int tile) -> int {
-      const int i = (first_tile + tile) * kDecTile + (lane & 15);
-      return (tile < ntiles && i < cnt) ? clamp_row(irow[i], Tk_max) : 0;
-    };
-    int jl_next = idx_of(kDecStages - 1);
+        for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
 #pragma unroll
-    for (int sIdx = 0; sIdx < kDecStages - 1; ++sIdx) {
-      if (sIdx < ntiles) {
-        const int i0 = (first_tile + sIdx) * kDecTile;
-        dec_gather(ring + sIdx * (kDecStageBytes / 2), kc, vc, idx_of(sIdx), i0, cnt, head_base, row_elems,
-                   Tk_max, lane);
+      for (int kk = 0; kk < 8; kk += 2) {
+        const int mtx = lane >> 3;
+        const uint16_t* kr = tK + ((mtx >> 1) * 8 + (lane & 7)) * rs_el + (mtx & 1) * 8;
+        uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
+        ldmatrix_x4(b0, b1, b2, b3, kr + kk * 16);
+        ldmatrix_x4(c0, c1, c2, c3, kr + (kk + 1) * 16);
+        mma_bf16_16816(sc[0], qa[kk], b0, b1);
+        mma_bf16_16816(sc[1], qa[kk], b2, b3);
+        mma_bf16_16816(sd[0], qa[kk + 1], c0, c1);
+        mma_bf16_16816(sd[1], qa[kk + 1], c2, c3);
       }
-      cp_async_commit();
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = rbase + nt * 8 + tg * 2 + (e & 1);
+          const float z = row < cnt ? (sc[nt][e] + sd[nt][e]) * qscale : -INFINITY;
+          sc[nt][e] = z;
+          mx[e >> 1] = fmaxf(mx[e >> 1], z);
+        }
+      float alpha[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v = mx[hh];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+        const float mnew = fmaxf(m_r[hh], v);
+        const float muse = mnew == -INFINITY ? 0.f : mnew;
+        alpha[hh] = exp2f(m_r[hh] - muse);
+        m_r[hh] = mnew;
+        mx[hh] = muse;
+      }
+      float rsum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+          sc[nt][e] = pv;
+          rsum[e >> 1] += pv;
+        }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v = rsum[hh];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        l_r[hh] = l_r[hh] * alpha[hh] + v;
+      }
+      if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {   // a row max moved
+#pragma unroll
+        for (int dt = 0; dt < 16; ++dt) {
+          o[dt][0] *= alpha[0];
+          o[dt][1] *= alpha[0];
+          o[dt][2] *= alpha[1];
+          o[dt][3] *= alpha[1];
+        }
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf2(sc[0][0], sc[0][1]);
+      pa[1] = pack_bf2(sc[0][2], sc[0][3]);
+      pa[2] = pack_bf2(sc[1][0], sc[1][1]);
+      pa[3] = pack_bf2(sc[1][2], sc[1][3]);
+#pragma unroll
+      for (int dt = 0; dt < 16; dt += 2) {
+        const int mtx = lane >> 3;
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * rs_el + (dt + (mtx >> 1)) * 8);
+        mma_bf16_16816(o[dt], pa, b0, b1);
+        mma_bf16_16816(o[dt + 1], pa, b2, b3);
+      }
     }
-    for (int it = 0; it < ntiles; ++it) {
-      const int nxt = it + kDecStages - 1;
-      if (nxt < ntiles) {
-        const int i0 = (first_tile + nxt) * kDecTile;
-        dec_gather(ring + (nxt % kDecStages) * (kDecStageBytes / 2), kc, vc, jl_next, i0, cnt, head_base,
-                   row_elems, Tk_max, lane);
-      }
-      jl_next = idx_of(nxt + 1);
-      cp_async_commit();
-      cp_async_wait<kDecStages - 1>();
-      __syncwarp();
-      const uint16_t* tK = ring + (it % kDecStages) * (kDecStageBytes / 2);
-      const uint16_t* tV = tK + kDecTile * kLds;
-      const int rbase = (first_tile + it) * kDecTile;
-      if (rbase < cnt) {
-        // S = Q K^T over 8 k-steps, in two independent accumulator chains
-        float sc[2][4], sd[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 8; kk += 2) {
-          const int mtx = lane >> 3;
-          uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
-          ldmatrix_x4(b0, b1, b2, b3, tK + ((mtx >> 1) * 8 + (lane & 7)) * kLds + kk * 16 + (mtx & 1) * 8);
-          ldmatrix_x4(c0, c1, c2, c3, tK + ((mtx >> 1) * 8 + (lane & 7)) * kLds + (kk + 1) * 16 + (mtx & 1) * 8);
-          mma_bf16_16816(sc[0], qa[kk], b0, b1);
-          mma_bf16_16816(sc[1], qa[kk], b2, b3);
-          mma_bf16_16816(sd[0], qa[kk + 1], c0, c1);
-          mma_bf16_16816(sd[1], qa[kk + 1], c2, c3);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] += sd[nt][e];
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int row = rbase + nt * 8 + tg * 2 + (e & 1);
-            const float z = row < cnt ? sc[nt][e] * qscale : -INFINITY;
-            sc[nt][e] = z;
-            mx[e >> 1] = fmaxf(mx[e >> 1], z);
-          }
-        float alpha[2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float v = mx[hh];
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-          const float mnew = fmaxf(m_r[hh], v);
-          const float muse = mnew == -INFINITY ? 0.f : mnew;
-          alpha[hh] = exp2f(m_r[hh] - muse);
-          m_r[hh] = mnew;
-          mx[hh] = muse;
-        }
-        float rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
-            sc[nt][e] = pv;
-            rs[e >> 1] += pv;
-          }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float v = rs[hh];
-          v += __shfl_xor_sync(0xffffffffu, v, 1);
-          v += __shfl_xor_sync(0xffffffffu, v, 2);
-          l_r[hh] = l_r[hh] * alpha[hh] + v;
-        }
-        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {  // a row max moved
-#pragma unroll
-          for (int dt = 0; dt < 16; ++dt) {
-            o[dt][0] *= alpha[0];
-            o[dt][1] *= alpha[0];
-            o[dt][2] *= alpha[1];
-            o[dt][3] *= alpha[1];
-          }
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf2(sc[0][0], sc[0][1]);
-        pa[1] = pack_bf2(sc[0][2], sc[0][3]);
-        pa[2] = pack_bf2(sc[1][0], sc[1][1]);
-        pa[3] = pack_bf2(sc[1][2], sc[1][3]);
-#pragma unroll
-        for (int dt = 0; dt < 16; dt += 2) {
-          const int mtx = lane >> 3;
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * kLds + (dt + (mtx >> 1)) * 8);
-          mma_bf16_16816(o[dt], pa, b0, b1);
-          mma_bf16_16816(o[dt + 1], pa, b2, b3);
-        }
-      }
-      __syncwarp();
-    }
-    cp_async_wait<0>();
     __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&empty[s]);
+    ++fill;
+  }
+  if (cur_p >= 0 && !*abort_flag) flush(cur_p);
+}
 
-    // ---- hand the segment's result on
-    const long long w_first = tile_owner((long long)p * pl.tpp, pl.T, pl.W);
-    const long long w_last = tile_owner((long long)(p + 1) * pl.tpp - 1, pl.T, pl.W);
-    const int ncontrib = (int)(w_last - w_first + 1);
-    if (ncontrib == 1) {
-      // this warp owns the whole pair: normalise and write
+// Folds the partials of one (sequence, query head): out = sum_x w_x o_x / L,
+// w_x = 2^(m_x - M), L = sum_x w_x l_x, M = max_x m_x (base-2 logits).
+__global__ void __launch_bounds__(kMergeThreads)
+attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, DecPlan pl,
+                         int Hq, int Hkv, const int* __restrict__ err, uint16_t* __restrict__ out,
+                         float* __restrict__ lse) {
+  __shared__ float wts[kMergeMaxC];
+  __shared__ float red[kMergeThreads / 32][kD];
+  __shared__ float rmax[kMergeThreads / 32], rsum[kMergeThreads / 32];
+  tc::pdl_wait();   // the partials come from the split kernel
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = Hq / Hkv;
+  const long long bh = blockIdx.x;
+  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+  const int g = h / G, gq = h % G;
+  const int hb = g / pl.nh, hs = g % pl.nh;
+  const int p = b * pl.HB + hb;
+  if (*err != 0) {   // the split kernel gave up: make the failure visible
+    if (tid < kD) out[bh * kD + tid] = 0x7fc0;
+    if (tid == 0 && lse != nullptr) lse[bh] = __int_as_float(0x7fc00000);
+    return;
+  }
+  const long long first = unit_owner((long long)p * pl.tpp, pl.U, pl.W);
+  const long long last = unit_owner((long long)(p + 1) * pl.tpp - 1, pl.U, pl.W);
+  const int C = (int)(last - first + 1) * pl.wph;
+  const long long sbase = ((long long)p + first) * pl.wph;
+  auto ent = [&](int x) -> long long { return ((sbase + x) * pl.nh + hs) * G + gq; };
+
+  float mloc = -INFINITY;
+  for (int x = tid; x < C; x += kMergeThreads) mloc = fmaxf(mloc, __ldcg(part_ml + ent(x) * 2));
+  mloc = warp_max(mloc);
+  if (lane == 0) rmax[warp] = mloc;
+  __syncthreads();
+  float M = rmax[0];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int h = gq + 8 * hh;
-        if (h < G) {
-          const float inv = l_r[hh] > 0.f ? 1.f / l_r[hh] : 0.f;
+  for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, rmax[w]);
+  float lloc = 0.f;
+  for (int x = tid; x < C; x += kMergeThreads) {
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(part_ml + ent(x) * 2));
+    const float wv = (ml.y > 0.f && M != -INFINITY) ? exp2f(ml.x - M) : 0.f;
+    wts[x] = wv;
+    lloc += ml.y * wv;
+  }
+  lloc = warp_sum(lloc);
+  if (lane == 0) rsum[warp] = lloc;
+  __syncthreads();
+  float L = 0.f;
 #pragma unroll
-          for (int dt = 0; dt < 16; ++dt)
-            *reinterpret_cast<uint32_t*>(out + (head0 + h) * kD + dt * 8 + 2 * tg) =
-                pack_bf2(o[dt][2 * hh] * inv, o[dt][2 * hh + 1] * inv);
-          if (tg == 0 && lse != nullptr)
-            lse[head0 + h] = l_r[hh] > 0.f ? (m_r[hh] + log2f(l_r[hh])) * kLn2 : -INFINITY;
-        }
-      }
-    } else {
-      const int j = (int)(w - w_first);
-      const long long slot = ((long long)p * pl.cmax + j) * G;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int h = gq + 8 * hh;
-        if (h < G) {
-#pragma unroll
-          for (int dt = 0; dt < 16; ++dt)
-            *reinterpret_cast<float2*>(part_o + (slot + h) * kD + dt * 8 + 2 * tg) =
-                make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
-          if (tg == 0) {
-            part_ml[(slot + h) * 2] = m_r[hh];
-            part_ml[(slot + h) * 2 + 1] = l_r[hh];
-          }
-        }
-      }
-      __syncwarp();
-      unsigned last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atomicAdd(ticket + p, 1u) == (unsigned)(ncontrib - 1);
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        // warp-parallel merge: lane x holds contributor x's (m, l) per head
-        // (at most 32 contributors per pair, see decode_plan)
-        __threadfence();
-        const long long base = (long long)p * pl.cmax * G;
-        float wgt[16], Lh[16], Mh[16];
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          wgt[h] = 0.f;
-          Lh[h] = 0.f;
-          Mh[h] = -INFINITY;
-          if (h < G) {
-            const long long sl = base + (long long)lane * G + h;
-            const float mx = lane < ncontrib ? __ldcg(part_ml + sl * 2) : -INFINITY;
-            const float lx = lane < ncontrib ? __ldcg(part_ml + sl * 2 + 1) : 0.f;
-            const float M = warp_max(mx);
-            const float wv = (lx > 0.f && M != -INFINITY) ? exp2f(mx - M) : 0.f;
-            wgt[h] = wv;
-            Lh[h] = warp_sum(lx * wv);
-            Mh[h] = M;
-          }
-        }
-        // o: every contributor's partial (zero where it saw no rows) scaled by
-        // its weight; no branch in the loop, so the loads overlap
-        float acc[16][4];
-#pragma unroll
-        for (int h = 0; h < 16; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
-        const float* po_base = part_o + base * kD + lane * 4;
+  for (int w = 0; w < kMergeThreads / 32; ++w) L += rsum[w];
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-        for (int x = 0; x < ncontrib; ++x) {
+  for (int x = warp; x < C; x += kMergeThreads / 32) {
+    const float wt = wts[x];
+    const float4 ov = __ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane);
+    acc.x = fmaf(ov.x, wt, acc.x);
+    acc.y = fmaf(ov.y, wt, acc.y);
+    acc.z = fmaf(ov.z, wt, acc.z);
+    acc.w = fmaf(ov.w, wt, acc.w);
+  }
+  *reinterpret_cast<float4*>(&red[warp][lane * 4]) = acc;
+  __syncthreads();
+  if (tid < kD) {
+    float v = 0.f;
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            if (h < G) {
-              const float wt = __shfl_sync(0xffffffffu, wgt[h], x);
-              const float4 ov = __ldcg(reinterpret_cast<const float4*>(po_base + ((long long)x * G + h) * kD));
-              acc[h][0] = fmaf(ov.x, wt, acc[h][0]);
-              acc[h][1] = fmaf(ov.y, wt, acc[h][1]);
-              acc[h][2] = fmaf(ov.z, wt, acc[h][2]);
-              acc[h][3] = fmaf(ov.w, wt, acc[h][3]);
-            }
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          if (h < G) {
-            const float inv = Lh[h] > 0.f ? 1.f / Lh[h] : 0.f;
-            *reinterpret_cast<uint2*>(out + (head0 + h) * kD + lane * 4) =
-                make_uint2(pack_bf2(acc[h][0] * inv, acc[h][1] * inv), pack_bf2(acc[h][2] * inv, acc[h][3] * inv));
-            if (lane == 0 && lse != nullptr)
-              lse[head0 + h] = Lh[h] > 0.f ? (Mh[h] + log2f(Lh[h])) * kLn2 : -INFINITY;
-          }
-        }
-        if (lane == 0) ticket[p] = 0u;  // ready for the next call
-      }
-    }
-    t = seg_end;
+    for (int w = 0; w < kMergeThreads / 32; ++w) v += red[w][tid];
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    out[bh * kD + tid] = f2bf(v * inv);
+    if (tid == 0 && lse != nullptr) lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
   }
 }
 
@@ -591,40 +640,42 @@ DecPlan decode_plan(int B, int Hkv, int k) {
     sms = n > 0 ? n : 148;
   }
   DecPlan pl;
-  pl.pairs = B * Hkv;
-  pl.tpp = (k + kDecTile - 1) / kDecTile;
-  pl.T = (long long)pl.pairs * pl.tpp;
-  // resident warps (2 CTAs of kDecWarps per SM), but at least 2 tiles per
-  // warp and at most 30 warps per pair (the merge keeps one contributor per lane)
-  long long W = (long long)sms * 2 * kDecWarps;
-  const long long by_tiles = (pl.T + 1) / 2;
-  if (W > by_tiles) W = by_tiles;
-  if (W > 30ll * pl.pairs) W = 30ll * pl.pairs;
+  pl.nh = Hkv < kDxConsumers ? Hkv : kDxConsumers;
+  pl.wph = kDxConsumers / pl.nh;
+  pl.R = 16 * pl.wph;
+  pl.HB = (Hkv + pl.nh - 1) / pl.nh;
+  pl.pairs = B * pl.HB;
+  pl.tpp = (k + pl.R - 1) / pl.R;
+  pl.row_bytes = pl.nh * kD * 2 + 16;
+  pl.stage_bytes = 2 * pl.R * pl.row_bytes;
+  pl.U = (long long)pl.pairs * pl.tpp;
+  long long W = sms;   // one CTA per SM
+  if (W > kMergeMaxC / pl.wph) W = kMergeMaxC / pl.wph;   // contributors of one pair <= W * wph
+  if (W > pl.U) W = pl.U;
   if (W < 1) W = 1;
   pl.W = W;
-  // warps meeting one pair's tile range: at most (tpp-1)*W/T + 2
-  pl.cmax = (int)((W + pl.pairs - 1) / pl.pairs) + 2;
   return pl;
+}
+
+size_t dec_smem_bytes(const DecPlan& pl) {
+  return (size_t)kDxStages * pl.stage_bytes + 2 * kDxStages * sizeof(uint64_t) + 16;
 }
 
 }  // namespace
 
 static size_t align256a(size_t x) { return (x + 255) & ~size_t(255); }
 
-// The merge tickets sit in a fixed region at the start of the workspace
-// (room for kTicketSlots (sequence, kv head) pairs) that holds nothing else,
-// so a zero-filled workspace stays valid across calls of any shape: the warp
-// that merges a pair returns its ticket to zero.
-constexpr int kTicketSlots = 16384;
+// Decode workspace: a 256-byte head whose first word is the kernel error
+// code (zero when all is well; set if a pipeline wait gave up), then the
+// split partials.  Nothing but the error word needs to start at zero.
+constexpr size_t kDecHead = 256;
 
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
   (void)D;
   const DecPlan pl = decode_plan(B, Hkv, k);
   const int G = Hq / Hkv;
-  const size_t tk = (size_t)kTicketSlots * 4;
-  const size_t po = align256a((size_t)pl.pairs * pl.cmax * G * kD * 4);
-  const size_t pml = align256a((size_t)pl.pairs * pl.cmax * G * 2 * 4);
-  return tk + po + pml;
+  const size_t slots = (size_t)(pl.pairs + pl.W) * pl.wph * pl.nh * G;
+  return kDecHead + align256a(slots * kD * 4) + align256a(slots * 2 * 4);
 }
 
 cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
@@ -634,17 +685,37 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
   if (B <= 0) return cudaSuccess;
   const DecPlan pl = decode_plan(B, Hkv, k);
   const int G = Hq / Hkv;
+  const size_t slots = (size_t)(pl.pairs + pl.W) * pl.wph * pl.nh * G;
   char* p = static_cast<char*>(ws);
-  unsigned* ticket = reinterpret_cast<unsigned*>(p);
-  p += (size_t)kTicketSlots * 4;
+  int* err = reinterpret_cast<int*>(p);
+  p += kDecHead;
   float* po = reinterpret_cast<float*>(p);
-  p += align256a((size_t)pl.pairs * pl.cmax * G * kD * 4);
+  p += align256a(slots * kD * 4);
   float* pml = reinterpret_cast<float*>(p);
-  cudaError_t e = ensure_dynamic_smem((const void*)attn_decode_kernel, kDecSmem);
+  const size_t smem = dec_smem_bytes(pl);
+  cudaError_t e = ensure_dynamic_smem((const void*)attn_decode_split_kernel, smem);
   if (e != cudaSuccess) return e;
-  const int grid = (int)((pl.W + kDecWarps - 1) / kDecWarps);
-  attn_decode_kernel<<<grid, kDecWarps * 32, kDecSmem, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k, pl,
-                                                            scale * kLog2e, po, pml, ticket, out, lse);
+  attn_decode_split_kernel<<<(unsigned)pl.W, kDxThreads, smem, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k,
+                                                                      pl, scale * kLog2e, po, pml, err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the merge is launched with programmatic stream serialization: its CTAs
+  // may be scheduled while the split kernel drains and wait in pdl_wait()
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)B * Hq));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* cpo = po;
+  const float* cpml = pml;
+  const int* cerr = err;
+  e = cudaLaunchKernelEx(&cfg, attn_decode_merge_kernel, cpo, cpml, pl, Hq, Hkv, cerr, out, lse);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

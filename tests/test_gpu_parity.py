@@ -149,7 +149,7 @@ def _random_index(rng, B, Tk_max, k, counts):
     return idx
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (28, 4), (8, 1), (16, 16)])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (28, 4), (8, 1), (16, 16), (24, 12), (15, 3)])
 @pytest.mark.parametrize("k,counts", [(2048, [2048, 1000, 0, 1]), (100, [100, 33, 64, 7]),
                                       (1104, [1104, 1090, 1, 1089])])
 def test_decode_attention_matches_oracle(Hq, Hkv, k, counts):
@@ -170,7 +170,7 @@ def test_decode_attention_matches_oracle(Hq, Hkv, k, counts):
 
 
 def test_decode_attention_scale_and_repeat_calls():
-    """Explicit scale; two calls in a row reuse the workspace (tickets reset)."""
+    """Explicit scale; two calls in a row reuse one workspace."""
     B, Hq, Hkv, D, Tk_max, k = 2, 8, 2, 128, 500, 300
     q = _normals(31, 1, (B, Hq, D))
     K = _normals(31, 2, (B, Tk_max, Hkv, D))
@@ -183,6 +183,26 @@ def test_decode_attention_scale_and_repeat_calls():
                                        scale=0.05)
         torch.cuda.synchronize()
         assert_close_attn(out.float().cpu().numpy(), ref, "decode attention, scale 0.05")
+
+
+def test_decode_attention_many_sequences():
+    """More (sequence, head block) pairs than CTAs: every CTA's range spans
+    several pairs, some pairs are empty, and each pair has one contributor."""
+    rng = np.random.default_rng(77)
+    B, Hq, Hkv, D, Tk_max, k = 300, 8, 2, 128, 200, 64
+    counts = [int(c) for c in rng.integers(0, k + 1, size=B)]
+    counts[0], counts[1], counts[-1] = 0, k, 1
+    q = _normals(41, 1, (B, Hq, D))
+    K = _normals(41, 2, (B, Tk_max, Hkv, D))
+    V = _normals(41, 3, (B, Tk_max, Hkv, D))
+    idx = _random_index(rng, B, Tk_max, k, counts)
+    out, lse = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), i32(idx), i32(counts),
+                                        with_lse=True)
+    ref, rlse = oracle.sparse_attention_decode(q, [K[b, idx[b, :c]] for b, c in enumerate(counts)],
+                                               [V[b, idx[b, :c]] for b, c in enumerate(counts)])
+    torch.cuda.synchronize()
+    assert_close_attn(out.float().cpu().numpy(), ref, "decode attention, 300 sequences")
+    assert_lse_close(lse.cpu().numpy(), rlse, "decode lse, 300 sequences")
 
 
 @pytest.mark.parametrize("Hq,Hkv,k", [(8, 1, 256), (16, 4, 64), (12, 4, 100)])
