@@ -345,32 +345,32 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
 
   if (warp == kDxConsumers) {
     // ------------------------------------------------------------ producer
-    // row indices of the next unit are loaded while the current one is
-    // issued; rows past the count repeat the last selected row so every
-    // byte of the tile is finite (their scores are masked)
-    int jr[4];
-    auto load_rows = [&](long long u, int* out_j) -> bool {
-      if (u >= hi) return false;
-      const int p = (int)(u / pl.tpp), b = p / pl.HB;
+    // The row indices and count of unit u+1 are requested while unit u is
+    // issued, with no branch on the loaded values (idx is [B, k], so every
+    // slot of a tile below k is addressable).  Rows past the count repeat the
+    // tile's first row so every byte of the tile is finite (their scores are
+    // masked).
+    int jr[4], jn[4], cr = 0, cn = 0;
+    auto fetch = [&](long long u, int* out_j, int& out_c) {
+      if (u >= hi) return;
+      const int b = (int)(u / pl.tpp) / pl.HB;
       const int r0 = (int)(u % pl.tpp) * R;
-      const int cnt = clamp_count(count, b, k);
-      if (r0 >= cnt) return false;
-      const int32_t* irow = idx + (long long)b * k;
+      const int32_t* irow = idx + (long long)b * k + r0;
+      out_c = count[b];
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
         const int r = lane + 32 * qq;
-        const int i = r0 + min(r, cnt - 1 - r0);
-        out_j[qq] = r < R ? clamp_row(irow[i], Tk_max) : 0;
+        out_j[qq] = (r < R && r0 + r < k) ? irow[r] : 0;
       }
-      return true;
     };
-    bool have = load_rows(lo, jr);
+    fetch(lo, jr, cr);
     uint32_t fill = 0;
     for (long long u = lo; u < hi; ++u) {
-      int jn[4];
-      const bool have_next = load_rows(u + 1, jn);
-      if (have) {
-        const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
+      fetch(u + 1, jn, cn);
+      const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
+      const int cnt = cr < 0 ? 0 : (cr > k ? k : cr);
+      const int r0 = (int)(u % pl.tpp) * R;
+      if (r0 < cnt) {   // the consumers skip the same units
         const int h0 = hb * pl.nh;
         const int nh_here = min(pl.nh, Hkv - h0);
         const uint32_t bytes = (uint32_t)nh_here * 256u;
@@ -379,13 +379,15 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
         if (use > 0 && !tc::mbar_wait(&empty[s], (use - 1) & 1u, abort_flag, err, 11)) break;
         unsigned char* stK = smem + (size_t)s * pl.stage_bytes;
         unsigned char* stV = stK + (size_t)R * rb;
+        const int j0 = __shfl_sync(0xffffffffu, jr[0], 0);   // row r0 < cnt
         if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)R * bytes);
         __syncwarp();
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int r = lane + 32 * qq;
           if (r < R) {
-            const long long off = (((long long)b * Tk_max + jr[qq]) * Hkv + h0) * kD;
+            const int j = clamp_row(r0 + r < cnt ? jr[qq] : j0, Tk_max);
+            const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
             tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
             tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
           }
@@ -394,7 +396,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
       }
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) jr[qq] = jn[qq];
-      have = have_next;
+      cr = cn;
     }
     // every copy this CTA issued lands before it exits
     for (int s = 0; s < kDxStages; ++s) {
@@ -413,7 +415,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
   float o[16][4];
   float m_r[2], l_r[2];
   uint32_t qa[8][4];
-  int cur_p = -1;
+  int cur_p = -1, cnt = 0;
   bool active = false;        // this warp's head exists in the current block
   long long head0 = 0;
   uint32_t fill = 0;
@@ -442,6 +444,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
     if (p != cur_p) {
       if (cur_p >= 0) flush(cur_p);
       cur_p = p;
+      cnt = clamp_count(count, b, k);
       const int g = hb * pl.nh + hs;
       active = hs < min(pl.nh, Hkv - hb * pl.nh);
       head0 = (long long)b * Hq + (long long)(active ? g : 0) * G;
@@ -463,7 +466,6 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
         qa[kk][3] = active && gq + 8 < G ? __ldg(qr1 + c1) : 0u;
       }
     }
-    const int cnt = clamp_count(count, b, k);
     const int r0 = (int)(u % pl.tpp) * R;
     if (r0 >= cnt) continue;   // the producer skips this unit too
     const int s = (int)(fill % kDxStages);
@@ -560,14 +562,18 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
 }
 
 // Folds the partials of one (sequence, query head): out = sum_x w_x o_x / L,
-// w_x = 2^(m_x - M), L = sum_x w_x l_x, M = max_x m_x (base-2 logits).
+// w_x = 2^(m_x - M), L = sum_x w_x l_x, M = max_x m_x (base-2 logits).  The
+// first loads of every kind are issued together, so the usual case (at most
+// 256 contributors, 4 per warp) costs one memory round trip.
 __global__ void __launch_bounds__(kMergeThreads)
 attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, DecPlan pl,
                          int Hq, int Hkv, const int* __restrict__ err, uint16_t* __restrict__ out,
                          float* __restrict__ lse) {
+  constexpr int kWarps = kMergeThreads / 32;
+  constexpr int kPre = 4;   // o rows prefetched per warp
   __shared__ float wts[kMergeMaxC];
-  __shared__ float red[kMergeThreads / 32][kD];
-  __shared__ float rmax[kMergeThreads / 32], rsum[kMergeThreads / 32];
+  __shared__ float red[kWarps][kD];
+  __shared__ float rmax[kWarps], rsum[kWarps];
   tc::pdl_wait();   // the partials come from the split kernel
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = Hq / Hkv;
@@ -576,29 +582,41 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
   const int g = h / G, gq = h % G;
   const int hb = g / pl.nh, hs = g % pl.nh;
   const int p = b * pl.HB + hb;
-  if (*err != 0) {   // the split kernel gave up: make the failure visible
-    if (tid < kD) out[bh * kD + tid] = 0x7fc0;
-    if (tid == 0 && lse != nullptr) lse[bh] = __int_as_float(0x7fc00000);
-    return;
-  }
   const long long first = unit_owner((long long)p * pl.tpp, pl.U, pl.W);
   const long long last = unit_owner((long long)(p + 1) * pl.tpp - 1, pl.U, pl.W);
   const int C = (int)(last - first + 1) * pl.wph;
   const long long sbase = ((long long)p + first) * pl.wph;
   auto ent = [&](int x) -> long long { return ((sbase + x) * pl.nh + hs) * G + gq; };
 
-  float mloc = -INFINITY;
-  for (int x = tid; x < C; x += kMergeThreads) mloc = fmaxf(mloc, __ldcg(part_ml + ent(x) * 2));
+  const float2 ml0 = tid < C ? __ldcg(reinterpret_cast<const float2*>(part_ml + ent(tid) * 2))
+                             : make_float2(-INFINITY, 0.f);
+  float4 pre[kPre];
+#pragma unroll
+  for (int i = 0; i < kPre; ++i) {
+    const int x = warp + kWarps * i;
+    pre[i] = x < C ? __ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int failed = *err;
+
+  float mloc = ml0.x;
+  for (int x = tid + kMergeThreads; x < C; x += kMergeThreads) mloc = fmaxf(mloc, __ldcg(part_ml + ent(x) * 2));
   mloc = warp_max(mloc);
   if (lane == 0) rmax[warp] = mloc;
   __syncthreads();
   float M = rmax[0];
 #pragma unroll
-  for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, rmax[w]);
+  for (int w = 1; w < kWarps; ++w) M = fmaxf(M, rmax[w]);
+  auto weight = [&](float2 ml) { return (ml.y > 0.f && M != -INFINITY) ? exp2f(ml.x - M) : 0.f; };
   float lloc = 0.f;
-  for (int x = tid; x < C; x += kMergeThreads) {
+  if (tid < C) {
+    const float wv = weight(ml0);
+    wts[tid] = wv;
+    lloc = ml0.y * wv;
+  }
+  for (int x = tid + kMergeThreads; x < C; x += kMergeThreads) {
     const float2 ml = __ldcg(reinterpret_cast<const float2*>(part_ml + ent(x) * 2));
-    const float wv = (ml.y > 0.f && M != -INFINITY) ? exp2f(ml.x - M) : 0.f;
+    const float wv = weight(ml);
     wts[x] = wv;
     lloc += ml.y * wv;
   }
@@ -607,27 +625,34 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
   __syncthreads();
   float L = 0.f;
 #pragma unroll
-  for (int w = 0; w < kMergeThreads / 32; ++w) L += rsum[w];
+  for (int w = 0; w < kWarps; ++w) L += rsum[w];
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int x = warp; x < C; x += kMergeThreads / 32) {
-    const float wt = wts[x];
-    const float4 ov = __ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane);
+  auto fold = [&](float4 ov, float wt) {
     acc.x = fmaf(ov.x, wt, acc.x);
     acc.y = fmaf(ov.y, wt, acc.y);
     acc.z = fmaf(ov.z, wt, acc.z);
     acc.w = fmaf(ov.w, wt, acc.w);
+  };
+#pragma unroll
+  for (int i = 0; i < kPre; ++i) {
+    const int x = warp + kWarps * i;
+    if (x < C) fold(pre[i], wts[x]);
   }
+#pragma unroll 4
+  for (int x = warp + kWarps * kPre; x < C; x += kWarps)
+    fold(__ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane), wts[x]);
   *reinterpret_cast<float4*>(&red[warp][lane * 4]) = acc;
   __syncthreads();
   if (tid < kD) {
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) v += red[w][tid];
+    for (int w = 0; w < kWarps; ++w) v += red[w][tid];
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    out[bh * kD + tid] = f2bf(v * inv);
-    if (tid == 0 && lse != nullptr) lse[bh] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    // a split kernel that gave up leaves NaN, so the failure is visible
+    out[bh * kD + tid] = failed ? (uint16_t)0x7fc0 : f2bf(v * inv);
+    if (tid == 0 && lse != nullptr)
+      lse[bh] = failed ? __int_as_float(0x7fc00000) : (L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY);
   }
 }
 

@@ -58,12 +58,6 @@ __device__ __forceinline__ int n_cand(long long q_pos0, int t, int len) {
   return (int)n;
 }
 
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
 // ------------------------------------------------------------------ scoring
 
 template <int D>
@@ -186,7 +180,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
 }
 
 // Bin of the K-th largest key in a 4096-bin histogram (bins in key order):
-// s_out[0] = bin, s_out[1] = keys in the bins above it.
+// s_out[0] = bin, s_out[1] = keys in the bins above it, s_out[2] = keys in it.
 __device__ __forceinline__ void hist_threshold(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
                                                uint32_t* s_out) {
   const int per = kHistBins / blockDim.x;  // 16 (256 threads) or 4 (1024 threads)
@@ -201,6 +195,7 @@ __device__ __forceinline__ void hist_threshold(const uint32_t* __restrict__ h, u
       if (cum + c >= K) {
         s_out[0] = kHistBins - 1 - (threadIdx.x * per + j);
         s_out[1] = cum;
+        s_out[2] = c;
         break;
       }
       cum += c;
@@ -219,7 +214,7 @@ collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* 
                uint32_t* __restrict__ cand_cnt, uint32_t* __restrict__ cand_key,
                uint32_t* __restrict__ cand_pos) {
   __shared__ uint32_t s_warp[33];
-  __shared__ uint32_t s_thr[2];
+  __shared__ uint32_t s_thr[3];
   __shared__ uint32_t s_base;
   const int b = blockIdx.y;
   const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
@@ -262,12 +257,15 @@ collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* 
 struct FinishSmem {
   uint32_t hist[256];
   uint32_t swarp[33];
-  uint32_t thr[2];
-  uint32_t digit, above, bnd_count, ncand, total;
+  uint32_t thr[3];
+  uint32_t digit, above, bnd_count, ncand;
+  uint32_t kor, kand, por, pand;   // OR / AND of every item's key and position
   uint32_t ckey[kSmemCand];
   uint32_t cpos[kSmemCand];
-  uint32_t bits[kBitmapWords];   // also the sort buffer (positions) for long rows
-  uint32_t wpre[kBitmapWords];   // also the sort buffer (keys) for long rows
+  uint32_t bits[kBitmapWords];   // position bitmap; bucket counts for long rows
+  uint32_t wpre[kBitmapWords];   // word prefix sums; bucket starts for long rows
+  uint32_t opos[kMaxK];          // long rows: chosen items grouped by bucket
+  uint32_t okey[kMaxK];
 };
 
 __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t digit, bool active) {
@@ -320,60 +318,115 @@ struct Items {
   __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i] : (uint32_t)i; }
 };
 
+// Where the search for the K-th key starts: the bits of its key already
+// known (prefix under pmask), how many items still to choose inside that
+// prefix (kk), how many items share it (bnd), and the first digit's shift.
+struct SelStart {
+  uint32_t prefix, pmask, kk, bnd;
+  int shift;
+};
+
 // Exact selection of the K largest keys (ties: lower position) among `it`:
 // on return an item is chosen iff (key & pmask) > prefix, or it equals
-// prefix under pmask and its position is <= pmax.
-__device__ void select_threshold(FinishSmem& s, const Items& it, uint32_t K, uint32_t& prefix,
+// prefix under pmask and its position is <= pmax.  Radix select with 8-bit
+// digits from st.shift down; a digit window on which every item agrees
+// (from the OR / AND of all keys, or of all positions) is settled without
+// a pass -- integer-valued scores leave most low mantissa bits zero, and
+// positions below 2^16 leave the high bits zero.
+__device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, uint32_t& prefix,
                                  uint32_t& pmask, uint32_t& pmax) {
   const int tid = threadIdx.x;
-  prefix = 0;
-  pmask = 0;
-  uint32_t kk = K;
-  uint32_t bnd = (uint32_t)it.n;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-      const int i = i0 + tid;
-      const uint32_t key = i < it.n ? it.k(i) : 0u;
-      const bool act = i < it.n && (key & pmask) == prefix;
-      hist_add(s.hist, (key >> shift) & 255u, act);
+  if (tid == 0) {
+    s.kor = 0u;
+    s.kand = ~0u;
+    s.por = 0u;
+    s.pand = ~0u;
+  }
+  __syncthreads();
+  {
+    uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
+    for (int i = tid; i < it.n; i += kFinThreads) {
+      const uint32_t key = it.k(i), pos = it.p(i);
+      ko |= key;
+      ka &= key;
+      po |= pos;
+      pa &= pos;
     }
-    __syncthreads();
-    find_digit(s, kk, true);
-    __syncthreads();
-    kk -= s.above;
-    prefix |= s.digit << shift;
-    pmask |= 255u << shift;
-    bnd = s.bnd_count;
-    __syncthreads();
-    if (bnd == kk) break;  // every item of the boundary prefix is chosen
+    ko = __reduce_or_sync(0xffffffffu, ko);
+    ka = __reduce_and_sync(0xffffffffu, ka);
+    po = __reduce_or_sync(0xffffffffu, po);
+    pa = __reduce_and_sync(0xffffffffu, pa);
+    if ((tid & 31) == 0) {
+      atomicOr(&s.kor, ko);
+      atomicAnd(&s.kand, ka);
+      atomicOr(&s.por, po);
+      atomicAnd(&s.pand, pa);
+    }
+  }
+  __syncthreads();
+  const uint32_t kvar = s.kor ^ s.kand, kfix = s.kand;
+  const uint32_t pvar = s.por ^ s.pand, pfix = s.pand;
+
+  prefix = st.prefix;
+  pmask = st.pmask;
+  uint32_t kk = st.kk, bnd = st.bnd;
+  for (int shift = st.shift; bnd != kk;) {
+    const uint32_t wmask = (255u << shift) & ~pmask;   // undecided bits of this digit
+    if ((kvar & wmask) == 0u) {
+      prefix |= kfix & wmask;   // every item has these bits: nothing is above
+    } else {
+      for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
+      __syncthreads();
+      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
+        const int i = i0 + tid;
+        const uint32_t key = i < it.n ? it.k(i) : 0u;
+        const bool act = i < it.n && (key & pmask) == prefix;
+        hist_add(s.hist, (key >> shift) & 255u, act);
+      }
+      __syncthreads();
+      find_digit(s, kk, true);
+      __syncthreads();
+      kk -= s.above;
+      prefix |= s.digit << shift;
+      bnd = s.bnd_count;
+      __syncthreads();
+    }
+    pmask |= wmask;
+    if (shift == 0) break;
+    shift = shift >= 8 ? shift - 8 : 0;
   }
   pmax = 0xFFFFFFFFu;
   if (bnd == kk) return;
   // exact key ties: keep the kk lowest positions among key == prefix
   uint32_t pp = 0, pm = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
-      const int i = i0 + tid;
-      bool act = false;
-      uint32_t p = 0;
-      if (i < it.n && it.k(i) == prefix) {
-        p = it.p(i);
-        act = (p & pm) == pp;
+    const uint32_t wmask = 255u << shift;
+    uint32_t c = bnd;
+    if ((pvar & wmask) == 0u) {
+      pp |= pfix & wmask;
+    } else {
+      for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
+      __syncthreads();
+      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
+        const int i = i0 + tid;
+        bool act = false;
+        uint32_t p = 0;
+        if (i < it.n && it.k(i) == prefix) {
+          p = it.p(i);
+          act = (p & pm) == pp;
+        }
+        hist_add(s.hist, (p >> shift) & 255u, act);
       }
-      hist_add(s.hist, (p >> shift) & 255u, act);
+      __syncthreads();
+      find_digit(s, kk, false);
+      __syncthreads();
+      kk -= s.above;
+      pp |= s.digit << shift;
+      c = s.bnd_count;
+      __syncthreads();
     }
-    __syncthreads();
-    find_digit(s, kk, false);
-    __syncthreads();
-    kk -= s.above;
-    pp |= s.digit << shift;
-    pm |= 255u << shift;
-    const uint32_t c = s.bnd_count;
-    __syncthreads();
+    pm |= wmask;
+    bnd = c;
     if (c == kk) {
       pmax = pp | ~pm;
       return;
@@ -386,21 +439,6 @@ __device__ __forceinline__ bool is_selected(uint32_t key, uint32_t pos, uint32_t
                                             uint32_t pmax) {
   const uint32_t m = key & pmask;
   return m > prefix || (m == prefix && pos <= pmax);
-}
-
-// Appends item (key, pos) to the shared candidate list (warp-aggregated).
-__device__ __forceinline__ void push_cand(FinishSmem& s, bool take, uint32_t key, uint32_t pos) {
-  const unsigned m = __ballot_sync(0xffffffffu, take);
-  if (!m) return;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(&s.ncand, (uint32_t)__popc(m));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  if (take) {
-    const uint32_t o = base + __popc(m & lanemask_lt());
-    if (o < (uint32_t)kSmemCand) { s.ckey[o] = key; s.cpos[o] = pos; }
-  }
 }
 
 // Writes the chosen item with rank `slot` (0-based, ascending position).
@@ -429,7 +467,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
   const uint32_t K = (uint32_t)min(k, n);
   const uint32_t* row = w.keys + (long long)r * w.ld;
-  if (tid == 0) { s.ncand = 0; s.total = 0; }
+  if (tid == 0) s.ncand = 0;
   __syncthreads();
 
   // ---- gather candidates into shared memory
@@ -442,9 +480,11 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
     if (mode == kFinishHistScan) {
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
-      // keep every key in or above the bin of the K-th largest; each thread
-      // issues all its 16-byte loads before filtering
-      constexpr int kPer = 8;
+      // keep every key in or above the bin of the K-th largest: each thread
+      // issues all its 16-byte loads, counts its takes, and one block scan
+      // places them (no shared atomics)
+      constexpr int kPer = 4;   // 8 spills at 64 registers
+      uint32_t base = 0;
       for (int i0 = 0; i0 < n; i0 += kFinThreads * 4 * kPer) {
         uint4 v[kPer];
 #pragma unroll
@@ -459,20 +499,39 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
             if (i + 2 < n) v[u].z = row[i + 2];
           }
         }
+        uint32_t mine = 0;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int i = i0 + (u * kFinThreads + tid) * 4;
+          mine += (i < n && (v[u].x >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 1 < n && (v[u].y >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 2 < n && (v[u].z >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 3 < n && (v[u].w >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+        }
+        uint32_t total;
+        uint32_t o = base + block_excl_scan(mine, s.swarp, total);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
           const int i = i0 + (u * kFinThreads + tid) * 4;
           const uint32_t kk4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const bool take = i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin;
-            push_cand(s, take, kk4[j], (uint32_t)(i + j));
+            if (i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin) {
+              if (o < (uint32_t)kSmemCand) {
+                s.ckey[o] = kk4[j];
+                s.cpos[o] = (uint32_t)(i + j);
+              }
+              ++o;
+            }
           }
         }
+        base += total;
       }
+      if (tid == 0) s.ncand = base;
       __syncthreads();
       in_smem = s.ncand <= (uint32_t)kSmemCand;
     } else if (mode == kFinishCandList) {
+      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t m = w.cand_cnt[r];
       if (m <= (uint32_t)kSmemCand) {
         const uint32_t* ck = w.cand_key + (long long)r * kCandCap;
@@ -502,7 +561,18 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   }
 
   uint32_t prefix = 0, pmask = 0, pmax = 0;
-  if (K > 0) select_threshold(s, it, K, prefix, pmask, pmax);
+  if (K > 0) {
+    SelStart st;
+    if (mode == kFinishDirect) {
+      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24};
+    } else {
+      // the histogram already fixes the top 12 bits: every item above the
+      // bin is chosen, K - above of the bin's items remain to pick
+      st = SelStart{s.thr[0] << (32 - kHistBits), ~0u << (32 - kHistBits), K - s.thr[1], s.thr[2],
+                    32 - kHistBits - 8};
+    }
+    select_threshold(s, it, st, prefix, pmask, pmax);
+  }
 
   const long long o_idx = ((long long)b * Tq + t) * (long long)k;
   if (K > 0) {
@@ -537,40 +607,55 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
         }
       }
     } else {
-      // ---- long rows: compact the chosen items, bitonic sort by position
-      uint32_t* sp = s.bits;
-      uint32_t* sk = s.wpre;
+      // ---- long rows: the chosen items are counted into kBitmapWords
+      // equal position ranges, placed range by range, and ranked inside
+      // their range (ranges hold about K / kBitmapWords items each)
+      int bsh = 0;
+      while (((n - 1) >> bsh) >= kBitmapWords) ++bsh;
+      uint32_t* cnt = s.bits;
+      uint32_t* start = s.wpre;
+      for (int i = tid; i < kBitmapWords; i += kFinThreads) cnt[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < it.n; i += kFinThreads) {
+        const uint32_t key = it.k(i), pos = it.p(i);
+        if (is_selected(key, pos, prefix, pmask, pmax)) atomicAdd(&cnt[pos >> bsh], 1u);
+      }
+      __syncthreads();
+      constexpr int per = kBitmapWords / kFinThreads;
+      uint32_t c[per], mine = 0;
+#pragma unroll
+      for (int j = 0; j < per; ++j) {
+        c[j] = cnt[tid * per + j];
+        mine += c[j];
+      }
+      uint32_t total;
+      uint32_t run = block_excl_scan(mine, s.swarp, total);
+#pragma unroll
+      for (int j = 0; j < per; ++j) {
+        start[tid * per + j] = run;
+        run += c[j];
+        cnt[tid * per + j] = 0;   // becomes the fill counter
+      }
+      __syncthreads();
       for (int i = tid; i < it.n; i += kFinThreads) {
         const uint32_t key = it.k(i), pos = it.p(i);
         if (is_selected(key, pos, prefix, pmask, pmax)) {
-          const uint32_t o = atomicAdd(&s.total, 1u);
-          if (o < (uint32_t)kMaxK) { sp[o] = pos; sk[o] = key; }
-        }
-      }
-      __syncthreads();
-      int P = 1;
-      while (P < (int)K) P <<= 1;
-      for (int i = (int)K + tid; i < P; i += kFinThreads) { sp[i] = 0xFFFFFFFFu; sk[i] = 0; }
-      __syncthreads();
-      for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int i = tid; i < (P >> 1); i += kFinThreads) {
-            const int lo = 2 * i - (i & (stride - 1));
-            const int hi = lo + stride;
-            const bool asc = (lo & size) == 0;
-            const uint32_t a = sp[lo], c = sp[hi];
-            if ((a > c) == asc) {
-              sp[lo] = c;
-              sp[hi] = a;
-              const uint32_t ka = sk[lo];
-              sk[lo] = sk[hi];
-              sk[hi] = ka;
-            }
+          const uint32_t bk = pos >> bsh;
+          const uint32_t o = start[bk] + atomicAdd(&cnt[bk], 1u);
+          if (o < (uint32_t)kMaxK) {
+            s.opos[o] = pos;
+            s.okey[o] = key;
           }
-          __syncthreads();
         }
       }
-      for (int i = tid; i < (int)K; i += kFinThreads) emit(out, o_idx, b, (uint32_t)i, sp[i], sk[i]);
+      __syncthreads();
+      for (int i = tid; i < (int)K; i += kFinThreads) {
+        const uint32_t pos = s.opos[i], bk = pos >> bsh;
+        const uint32_t b0 = start[bk], b1 = b0 + cnt[bk];
+        uint32_t rank = b0;
+        for (uint32_t j = b0; j < b1; ++j) rank += s.opos[j] < pos ? 1u : 0u;
+        emit(out, o_idx, b, rank, pos, s.okey[i]);
+      }
     }
   }
 
