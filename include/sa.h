@@ -23,6 +23,9 @@
  *     any CUDA kernel.
  *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
  *   - No kernel of this library waits on another CTA, kernel or device.
+ *     Waits inside a kernel (its own pipeline barriers) are bounded; decode
+ *     attention records a wait that gave up as a nonzero error word at the
+ *     start of its workspace and writes NaN to the outputs.
  *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned, and
  *     must be ZERO-FILLED before their first use.  The counters that must
  *     start at zero (histograms, candidate counts, merge tickets) live in a
@@ -51,7 +54,7 @@ typedef enum {
   SA_ERR_UNSUPPORTED = 2,   /* valid but outside this build's shape support  */
   SA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned    */
   SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed          */
-  SA_ERR_TIMEOUT = 5,       /* reserved: no kernel in this library waits     */
+  SA_ERR_TIMEOUT = 5,       /* reserved (kernel waits report in the workspace) */
   SA_ERR_STALE_INDEX = 6    /* shared layer read before its full layer ran   */
 } sa_status;
 
@@ -140,16 +143,18 @@ sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void*
  * Gathered sparse attention, decode (one query token per sequence).
  *
  * Same arithmetic as the prefill call.  The selected rows are split across
- * CTAs; each CTA loads every selected K/V row of its kv head once for all
- * Hq/Hkv query heads of that group, and the partial results are merged with
- * the log-sum-exp rule ([SSA] §六: split-K partial attention over a compact
- * index list, KV shared by a GQA group loaded once, then a log-sum-exp merge).
+ * CTAs; each CTA loads every selected K/V row once for all Hq/Hkv query
+ * heads of each kv head, and the partial results are merged with the
+ * log-sum-exp rule ([SSA] §六: split-K partial attention over a compact
+ * index list, KV shared by a GQA group loaded once, then a log-sum-exp
+ * merge).
  *
  *   q        [B, Hq, D] bf16
  *   idx      [B, k] int32 (row stride k); count [B] int32 (clamped to [0, k])
  *   out      [B, Hq, D] bf16;  lse [B, Hq] fp32 or NULL
  *   ws       >= sa_sparse_attn_decode_workspace(...) bytes (zero-filled before
- *            first use; see the conventions above)
+ *            first use; see the conventions above).  Its first int32 is the
+ *            kernel error word: 0 after a good call.
  * Supported: as for prefill; B * Hkv <= SA_DECODE_MAX_PAIRS.
  * ---------------------------------------------------------------------- */
 size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k);

@@ -27,6 +27,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "../../include/sa.h"
 #include "sa_common.cuh"
 #include "sa_internal.h"
 #include "tc_common.cuh"
@@ -282,19 +283,23 @@ attn_prefill_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 // form one list, cut into equal contiguous ranges, one per CTA of a grid of
 // one CTA per SM.
 //
-// CTA: warp 8 is the producer (row indices one unit ahead in registers,
-// bulk copies into a 3-stage ring, completion by mbarrier transaction
-// counts); warps 0..7 are consumers, warp c taking kv head c / wph of the
-// block and rows (c % wph) * 16 .. +16 of the tile (wph = 8 / heads per
-// block, so R = 16 * wph).  Each consumer runs online softmax on mma.sync
-// m16n8k16 with the G query heads of its kv head as the (zero padded) M
-// side and writes a partial (m, l, o) for every (sequence, head block) its
-// range meets.  attn_decode_merge_kernel then folds the partials of each
-// query head with the log-sum-exp rule, one CTA per (sequence, query head).
+// CTA: warp 8 is the producer (the range's row indices staged in shared
+// memory, bulk copies into a 3-stage ring, completion by mbarrier
+// transaction counts); warps 0..7 are consumers, warp c taking kv head
+// c / wph of the block and rows (c % wph) * 16 .. +16 of the tile (wph = 8 /
+// heads per block, so R = 16 * wph).  Each consumer runs online softmax on
+// mma.sync m16n8k16 with the G query heads of its kv head as the (zero
+// padded) M side and writes a partial (m, l, o) for every (sequence, head
+// block) pair its range meets.  attn_decode_merge_kernel, launched with
+// programmatic stream serialization, then folds the partials of each query
+// head with the log-sum-exp rule, one CTA per (sequence, query head).
 
 constexpr int kDxConsumers = 8;
 constexpr int kDxThreads = (kDxConsumers + 1) * 32;
 constexpr int kDxStages = 3;
+constexpr int kIdxChunk = 2048;   // staged row indices per chunk (two chunks)
+constexpr int kCntChunk = kIdxChunk / 16;   // staged counts per chunk (units of >= 16 rows)
+constexpr int kDxBarBytes = 64;   // mbarriers + abort word
 constexpr int kMergeThreads = 256;
 constexpr int kMergeMaxC = 1280;   // contributors of one (sequence, head block)
 
@@ -303,7 +308,7 @@ struct DecPlan {
   int pairs, tpp;         // (sequence, block) pairs, tiles per pair
   int row_bytes;          // padded shared row: nh * 256 + 16
   int stage_bytes;        // K and V tiles of one stage
-  long long U, W;         // units, CTAs
+  int U, W;               // units (< 2^31: pairs <= 2^14, tiles per pair <= 2^16), CTAs
 };
 
 // CTA owning unit u: the largest c with floor(c*U/W) <= u.
@@ -326,6 +331,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kDxStages * pl.stage_bytes);
   uint64_t* empty = full + kDxStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDxStages);
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + (size_t)kDxStages * pl.stage_bytes + kDxBarBytes);
+  int32_t* scnt = sidx + 2 * kIdxChunk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDxStages; ++s) {
@@ -338,66 +345,78 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
   __syncthreads();
   tc::pdl_wait();                 // inputs may come from the kernel before
   tc::pdl_launch_dependents();    // the merge may start launching
-  const long long lo = (long long)blockIdx.x * pl.U / pl.W;
-  const long long hi = (long long)(blockIdx.x + 1) * pl.U / pl.W;
+  const int lo = (int)((long long)blockIdx.x * pl.U / pl.W);
+  const int hi = (int)((long long)(blockIdx.x + 1) * pl.U / pl.W);
   const int G = Hq / Hkv;
   const int R = pl.R, rb = pl.row_bytes;
 
   if (warp == kDxConsumers) {
     // ------------------------------------------------------------ producer
-    // The row indices and count of unit u+1 are requested while unit u is
-    // issued, with no branch on the loaded values (idx is [B, k], so every
-    // slot of a tile below k is addressable).  Rows past the count repeat the
-    // tile's first row so every byte of the tile is finite (their scores are
-    // masked).
-    int jr[4], jn[4], cr = 0, cn = 0;
-    auto fetch = [&](long long u, int* out_j, int& out_c) {
-      if (u >= hi) return;
-      const int b = (int)(u / pl.tpp) / pl.HB;
-      const int r0 = (int)(u % pl.tpp) * R;
-      const int32_t* irow = idx + (long long)b * k + r0;
-      out_c = count[b];
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const int r = lane + 32 * qq;
-        out_j[qq] = (r < R && r0 + r < k) ? irow[r] : 0;
+    // The row indices and counts of the CTA's units are staged in shared
+    // memory with cp.async, kIdxChunk rows at a time and one chunk ahead, so
+    // issuing a tile never waits on an index load (under full DRAM load a
+    // dependent load per tile would pace the ring).  Rows past the count
+    // repeat the tile's first row so every byte of the tile is finite (their
+    // scores are masked).
+    const int CU = kIdxChunk / R;   // units per chunk
+    auto stage_chunk = [&](int c0, int buf) {
+      const int c1 = min(c0 + CU, hi);
+      int32_t* si = sidx + buf * kIdxChunk;
+      for (int e = lane; e < (c1 - c0) * R; e += 32) {
+        const int u = c0 + e / R;
+        const int r = e % R;
+        const int b = u / pl.tpp / pl.HB;
+        const int row = u % pl.tpp * R + r;
+        const bool v = row < k;
+        cp_async4(si + e, idx + (long long)b * k + (v ? row : 0), v);
       }
+      for (int e = lane; e < c1 - c0; e += 32)
+        cp_async4(scnt + buf * kCntChunk + e, count + (c0 + e) / pl.tpp / pl.HB, true);
+      cp_async_commit();
     };
-    fetch(lo, jr, cr);
+    int chunk_lo = lo;
+    int buf = 0;
+    stage_chunk(lo, 0);
+    if (lo + CU < hi) stage_chunk(lo + CU, 1);
+    else cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
     uint32_t fill = 0;
-    for (long long u = lo; u < hi; ++u) {
-      fetch(u + 1, jn, cn);
-      const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
-      const int cnt = cr < 0 ? 0 : (cr > k ? k : cr);
-      const int r0 = (int)(u % pl.tpp) * R;
-      if (r0 < cnt) {   // the consumers skip the same units
-        const int h0 = hb * pl.nh;
-        const int nh_here = min(pl.nh, Hkv - h0);
-        const uint32_t bytes = (uint32_t)nh_here * 256u;
-        const int s = (int)(fill % kDxStages);
-        const uint32_t use = fill / kDxStages;
-        if (use > 0 && !tc::mbar_wait(&empty[s], (use - 1) & 1u, abort_flag, err, 11)) break;
-        unsigned char* stK = smem + (size_t)s * pl.stage_bytes;
-        unsigned char* stV = stK + (size_t)R * rb;
-        const int j0 = __shfl_sync(0xffffffffu, jr[0], 0);   // row r0 < cnt
-        if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)R * bytes);
+    for (int u = lo; u < hi; ++u) {
+      if (u == chunk_lo + CU) {   // next chunk (staged one chunk ago)
+        chunk_lo += CU;
+        buf ^= 1;
+        cp_async_wait<0>();
         __syncwarp();
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int r = lane + 32 * qq;
-          if (r < R) {
-            const int j = clamp_row(r0 + r < cnt ? jr[qq] : j0, Tk_max);
-            const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
-            tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
-            tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
-          }
-        }
-        ++fill;
+        if (chunk_lo + CU < hi) stage_chunk(chunk_lo + CU, buf ^ 1);
       }
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) jr[qq] = jn[qq];
-      cr = cn;
+      const int ul = u - chunk_lo;
+      const int p = u / pl.tpp, b = p / pl.HB, hb = p % pl.HB;
+      const int cr = scnt[buf * kCntChunk + ul];
+      const int cnt = cr < 0 ? 0 : (cr > k ? k : cr);
+      const int r0 = u % pl.tpp * R;
+      if (r0 >= cnt) continue;   // the consumers skip the same units
+      const int32_t* si = sidx + buf * kIdxChunk + ul * R;
+      const int h0 = hb * pl.nh;
+      const int nh_here = min(pl.nh, Hkv - h0);
+      const uint32_t bytes = (uint32_t)nh_here * 256u;
+      const int s = (int)(fill % kDxStages);
+      const uint32_t use = fill / kDxStages;
+      if (use > 0 && !tc::mbar_wait(&empty[s], (use - 1) & 1u, abort_flag, err, 11)) break;
+      unsigned char* stK = smem + (size_t)s * pl.stage_bytes;
+      unsigned char* stV = stK + (size_t)R * rb;
+      const int j0 = si[0];   // row r0 < cnt
+      if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)R * bytes);
+      __syncwarp();
+      for (int r = lane; r < R; r += 32) {
+        const int j = clamp_row(r0 + r < cnt ? si[r] : j0, Tk_max);
+        const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
+        tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
+        tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
+      }
+      ++fill;
     }
+    cp_async_wait<0>();
     // every copy this CTA issued lands before it exits
     for (int s = 0; s < kDxStages; ++s) {
       if ((uint32_t)s < fill) {
@@ -439,8 +458,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
     }
   };
 
-  for (long long u = lo; u < hi; ++u) {
-    const int p = (int)(u / pl.tpp), b = p / pl.HB, hb = p % pl.HB;
+  for (int u = lo; u < hi; ++u) {
+    const int p = u / pl.tpp, b = p / pl.HB, hb = p % pl.HB;
     if (p != cur_p) {
       if (cur_p >= 0) flush(cur_p);
       cur_p = p;
@@ -466,7 +485,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
         qa[kk][3] = active && gq + 8 < G ? __ldg(qr1 + c1) : 0u;
       }
     }
-    const int r0 = (int)(u % pl.tpp) * R;
+    const int r0 = u % pl.tpp * R;
     if (r0 >= cnt) continue;   // the producer skips this unit too
     const int s = (int)(fill % kDxStages);
     if (!tc::mbar_wait(&full[s], (fill / kDxStages) & 1u, abort_flag, err, 13)) break;
@@ -673,8 +692,8 @@ DecPlan decode_plan(int B, int Hkv, int k) {
   pl.tpp = (k + pl.R - 1) / pl.R;
   pl.row_bytes = pl.nh * kD * 2 + 16;
   pl.stage_bytes = 2 * pl.R * pl.row_bytes;
-  pl.U = (long long)pl.pairs * pl.tpp;
-  long long W = sms;   // one CTA per SM
+  pl.U = pl.pairs * pl.tpp;
+  int W = sms;   // one CTA per SM
   if (W > kMergeMaxC / pl.wph) W = kMergeMaxC / pl.wph;   // contributors of one pair <= W * wph
   if (W > pl.U) W = pl.U;
   if (W < 1) W = 1;
@@ -683,7 +702,7 @@ DecPlan decode_plan(int B, int Hkv, int k) {
 }
 
 size_t dec_smem_bytes(const DecPlan& pl) {
-  return (size_t)kDxStages * pl.stage_bytes + 2 * kDxStages * sizeof(uint64_t) + 16;
+  return (size_t)kDxStages * pl.stage_bytes + kDxBarBytes + (2 * kIdxChunk + 2 * kCntChunk) * sizeof(int32_t);
 }
 
 }  // namespace
@@ -694,6 +713,11 @@ static size_t align256a(size_t x) { return (x + 255) & ~size_t(255); }
 // code (zero when all is well; set if a pipeline wait gave up), then the
 // split partials.  Nothing but the error word needs to start at zero.
 constexpr size_t kDecHead = 256;
+
+size_t decode_attn_zero_bytes(int B, int Hkv, int k) {
+  (void)B, (void)Hkv, (void)k;
+  return kDecHead;
+}
 
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
   (void)D;

@@ -85,6 +85,9 @@ int prefill_rows_per_launch(int B, int Tq, int Tk_max);
 
 // Attention.
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
+// Leading bytes of the decode workspace that must be zero when a call starts
+// (error word and the pair counters this shape uses).
+size_t decode_attn_zero_bytes(int B, int Hkv, int k);
 cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,
                                int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,

@@ -178,11 +178,15 @@ def test_decode_attention_scale_and_repeat_calls():
     idx = _random_index(np.random.default_rng(5), B, Tk_max, k, [300, 250])
     ref, _ = oracle.sparse_attention_decode(q, [K[0, idx[0]], K[1, idx[1, :250]]],
                                             [V[0, idx[0]], V[1, idx[1, :250]]], scale=0.05)
+    L = sa.lib()
+    ws = torch.zeros(L.sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k), dtype=torch.uint8, device="cuda")
     for _ in range(2):
         out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), i32(idx), i32([300, 250]),
-                                       scale=0.05)
+                                       scale=0.05, ws=ws)
         torch.cuda.synchronize()
         assert_close_attn(out.float().cpu().numpy(), ref, "decode attention, scale 0.05")
+        # the kernel error word is zero after a good call
+        assert not ws[:4].cpu().numpy().any(), "decode workspace error word set"
 
 
 def test_decode_attention_many_sequences():

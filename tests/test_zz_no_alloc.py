@@ -5,9 +5,9 @@ buffers it was handed, or code on a path where allocation is not allowed), so
 they cannot provide the workspace sa_sparse_attn_decode needs.
 sa_sparse_attn_decode_noalloc serves them from a fixed scratch array inside
 the library.  This test calls it through the C ABI twice in a row (two
-shapes; the second needs more merge tickets than the first) and checks each
-result against sa_sparse_attn_decode given a caller workspace, within the
-attention tolerance the other tests use.  It is collected last so that a run
+shapes, the second with more sequences and heads than the first) and checks
+each result against sa_sparse_attn_decode given a caller workspace, within
+the attention tolerance the other tests use.  It is collected last so that a run
 stopping at its first failure has run every other test already, and it
 passes both alone in a fresh process and after the other tests."""
 import ctypes
