@@ -343,8 +343,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
     tc::fence_barrier_init();
   }
   __syncthreads();
-  tc::pdl_wait();                 // inputs may come from the kernel before
-  tc::pdl_launch_dependents();    // the merge may start launching
+  pdl_wait();                 // inputs may come from the kernel before
+  pdl_launch_dependents();    // the merge may start launching
   const int lo = (int)((long long)blockIdx.x * pl.U / pl.W);
   const int hi = (int)((long long)(blockIdx.x + 1) * pl.U / pl.W);
   const int G = Hq / Hkv;
@@ -583,7 +583,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
 // Folds the partials of one (sequence, query head): out = sum_x w_x o_x / L,
 // w_x = 2^(m_x - M), L = sum_x w_x l_x, M = max_x m_x (base-2 logits).  The
 // first loads of every kind are issued together, so the usual case (at most
-// 256 contributors, 4 per warp) costs one memory round trip.
+// 256 contributors, 4 per warp) costs one memory round trip.  All index
+// arithmetic happens before the wait for the split kernel.
 __global__ void __launch_bounds__(kMergeThreads)
 attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, DecPlan pl,
                          int Hq, int Hkv, const int* __restrict__ err, uint16_t* __restrict__ out,
@@ -593,33 +594,36 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
   __shared__ float wts[kMergeMaxC];
   __shared__ float red[kWarps][kD];
   __shared__ float rmax[kWarps], rsum[kWarps];
-  tc::pdl_wait();   // the partials come from the split kernel
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = Hq / Hkv;
-  const long long bh = blockIdx.x;
-  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+  const int bh = blockIdx.x;
+  const int b = bh / Hq, h = bh % Hq;
   const int g = h / G, gq = h % G;
   const int hb = g / pl.nh, hs = g % pl.nh;
   const int p = b * pl.HB + hb;
   const long long first = unit_owner((long long)p * pl.tpp, pl.U, pl.W);
   const long long last = unit_owner((long long)(p + 1) * pl.tpp - 1, pl.U, pl.W);
   const int C = (int)(last - first + 1) * pl.wph;
-  const long long sbase = ((long long)p + first) * pl.wph;
-  auto ent = [&](int x) -> long long { return ((sbase + x) * pl.nh + hs) * G + gq; };
+  const float* pml = part_ml + ((((long long)p + first) * pl.wph * pl.nh + hs) * G + gq) * 2;
+  const float* po = part_o + ((((long long)p + first) * pl.wph * pl.nh + hs) * G + gq) * kD;
+  const int xstride = pl.nh * G;   // entries between consecutive contributors
+  pdl_wait();   // the partials come from the split kernel
+  pdl_launch_dependents();
 
-  const float2 ml0 = tid < C ? __ldcg(reinterpret_cast<const float2*>(part_ml + ent(tid) * 2))
+  const float2 ml0 = tid < C ? __ldcg(reinterpret_cast<const float2*>(pml + (long long)tid * xstride * 2))
                              : make_float2(-INFINITY, 0.f);
   float4 pre[kPre];
 #pragma unroll
   for (int i = 0; i < kPre; ++i) {
     const int x = warp + kWarps * i;
-    pre[i] = x < C ? __ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane)
+    pre[i] = x < C ? __ldcg(reinterpret_cast<const float4*>(po + (long long)x * xstride * kD) + lane)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const int failed = *err;
 
   float mloc = ml0.x;
-  for (int x = tid + kMergeThreads; x < C; x += kMergeThreads) mloc = fmaxf(mloc, __ldcg(part_ml + ent(x) * 2));
+  for (int x = tid + kMergeThreads; x < C; x += kMergeThreads)
+    mloc = fmaxf(mloc, __ldcg(pml + (long long)x * xstride * 2));
   mloc = warp_max(mloc);
   if (lane == 0) rmax[warp] = mloc;
   __syncthreads();
@@ -634,7 +638,7 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
     lloc = ml0.y * wv;
   }
   for (int x = tid + kMergeThreads; x < C; x += kMergeThreads) {
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(part_ml + ent(x) * 2));
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(pml + (long long)x * xstride * 2));
     const float wv = weight(ml);
     wts[x] = wv;
     lloc += ml.y * wv;
@@ -660,7 +664,7 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
   }
 #pragma unroll 4
   for (int x = warp + kWarps * kPre; x < C; x += kWarps)
-    fold(__ldcg(reinterpret_cast<const float4*>(part_o + ent(x) * kD) + lane), wts[x]);
+    fold(__ldcg(reinterpret_cast<const float4*>(po + (long long)x * xstride * kD) + lane), wts[x]);
   *reinterpret_cast<float4*>(&red[warp][lane * 4]) = acc;
   __syncthreads();
   if (tid < kD) {
@@ -669,7 +673,7 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
     for (int w = 0; w < kWarps; ++w) v += red[w][tid];
     const float inv = L > 0.f ? 1.f / L : 0.f;
     // a split kernel that gave up leaves NaN, so the failure is visible
-    out[bh * kD + tid] = failed ? (uint16_t)0x7fc0 : f2bf(v * inv);
+    out[(long long)bh * kD + tid] = failed ? (uint16_t)0x7fc0 : f2bf(v * inv);
     if (tid == 0 && lse != nullptr)
       lse[bh] = failed ? __int_as_float(0x7fc00000) : (L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY);
   }
@@ -744,26 +748,13 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
   const size_t smem = dec_smem_bytes(pl);
   cudaError_t e = ensure_dynamic_smem((const void*)attn_decode_split_kernel, smem);
   if (e != cudaSuccess) return e;
-  attn_decode_split_kernel<<<(unsigned)pl.W, kDxThreads, smem, st>>>(q, kc, vc, idx, count, Tk_max, Hq, Hkv, k,
-                                                                      pl, scale * kLog2e, po, pml, err);
-  e = cudaGetLastError();
+  // both kernels are launched with programmatic stream serialization: each
+  // may be scheduled while the kernel before it drains and waits in pdl_wait()
+  e = launch_pdl(attn_decode_split_kernel, dim3((unsigned)pl.W), dim3(kDxThreads), smem, st, q, kc, vc, idx, count,
+                 Tk_max, Hq, Hkv, k, pl, scale * kLog2e, po, pml, err);
   if (e != cudaSuccess) return e;
-  // the merge is launched with programmatic stream serialization: its CTAs
-  // may be scheduled while the split kernel drains and wait in pdl_wait()
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long long)B * Hq));
-  cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const float* cpo = po;
-  const float* cpml = pml;
-  const int* cerr = err;
-  e = cudaLaunchKernelEx(&cfg, attn_decode_merge_kernel, cpo, cpml, pl, Hq, Hkv, cerr, out, lse);
+  e = launch_pdl(attn_decode_merge_kernel, dim3((unsigned)((long long)B * Hq)), dim3(kMergeThreads), 0, st, po, pml,
+                 pl, Hq, Hkv, err, out, lse);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

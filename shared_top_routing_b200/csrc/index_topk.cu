@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kScoreThreads)
 score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int B, int Tk_max,
                     int Tk, int q_pos0, const int32_t* __restrict__ kv_len,
                     uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int J = D / 32;          // 16-byte chunks per lane per key row
   constexpr int U = 4;               // 8-row tiles per warp iteration
   constexpr int WARPS = kScoreThreads / 32;
@@ -213,6 +215,8 @@ collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* 
                int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int k, int chunk,
                uint32_t* __restrict__ cand_cnt, uint32_t* __restrict__ cand_key,
                uint32_t* __restrict__ cand_pos) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ uint32_t s_warp[33];
   __shared__ uint32_t s_thr[3];
   __shared__ uint32_t s_base;
@@ -458,6 +462,8 @@ __device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int 
 __global__ void __launch_bounds__(kFinThreads, 1)
 finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
               const int32_t* __restrict__ kv_len, int k, FinishOut out) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   FinishSmem& s = *reinterpret_cast<FinishSmem*>(smem_raw);
   const int r = blockIdx.x;
@@ -764,13 +770,14 @@ cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, 
   if (Tk <= 0 || B <= 0) return cudaSuccess;
   uint32_t* hist = with_hist ? w.hist : nullptr;
   const long long rows = (long long)B * Tk;
+  cudaError_t e;
   if (d == 128)
-    score_decode_kernel<128><<<score_grid<128>(rows), kScoreThreads, 0, st>>>(
-        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
+    e = launch_pdl(score_decode_kernel<128>, dim3(score_grid<128>(rows)), dim3(kScoreThreads), 0, st, q, kmat, B,
+                   Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
   else
-    score_decode_kernel<64><<<score_grid<64>(rows), kScoreThreads, 0, st>>>(
-        q, kmat, B, Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
-  return cudaGetLastError();
+    e = launch_pdl(score_decode_kernel<64>, dim3(score_grid<64>(rows)), dim3(kScoreThreads), 0, st, q, kmat, B,
+                   Tk_max, Tk, q_pos0, kv_len, w.keys, w.ld, hist);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
@@ -778,9 +785,9 @@ cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int
   if (Tk <= 0 || B <= 0) return cudaSuccess;
   const int chunk = 256 * kCollectPer;
   dim3 grid((Tk + chunk - 1) / chunk, B);
-  collect_kernel<<<grid, 256, 0, st>>>(w.keys, w.ld, w.hist, Tk, q_pos0, kv_len, k, chunk, w.cand_cnt,
-                                       w.cand_key, w.cand_pos);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(collect_kernel, grid, dim3(256), 0, st, w.keys, w.ld, w.hist, Tk, q_pos0,
+                                   kv_len, k, chunk, w.cand_cnt, w.cand_key, w.cand_pos);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
@@ -791,9 +798,9 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
   const size_t smem = sizeof(FinishSmem);
   cudaError_t e = ensure_dynamic_smem((const void*)finish_kernel, smem);
   if (e != cudaSuccess) return e;
-  finish_kernel<<<rows, kFinThreads, smem, st>>>(w, mode, rows_per_batch, t0, Tq, Tk, q_pos0, kv_len, k,
-                                                 out);
-  return cudaGetLastError();
+  e = launch_pdl(finish_kernel, dim3(rows), dim3(kFinThreads), smem, st, w, mode, rows_per_batch, t0, Tq, Tk,
+                 q_pos0, kv_len, k, out);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 int finish_mode_for(int Tk_max, bool* need_collect) {

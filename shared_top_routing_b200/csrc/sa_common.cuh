@@ -70,6 +70,16 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
 }
 // 4-byte variant (cp.async.ca; .cg takes 16 bytes only).
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it drains; it waits in
+// pdl_wait() (a no-op for an ordinary launch) until that kernel has completed
+// and its writes are visible, so pdl_wait() comes before any global memory
+// access.  pdl_launch_dependents() lets the next such kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid) {
   uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
   int n = valid ? 4 : 0;

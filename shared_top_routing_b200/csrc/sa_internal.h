@@ -52,6 +52,25 @@ sa_status check_decode_args(const void* q, const void* kc, const void* vc, const
                             const int32_t* count, int B, int Tk_max, int Hq, int Hkv, int D, int k,
                             const void* out);
 
+// Launches `kernel` with programmatic stream serialization, so it may start
+// while the kernel before it on `st` drains (the kernel calls pdl_wait()
+// before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Sets the detail string sa_last_error() returns for this host thread.
 void set_last_error(const char* fmt, ...);
 
