@@ -275,6 +275,12 @@ class DecodeBench:
         return score, attn_one
 
 
+# DRAM bytes (read + write) per decode attention call, split + merge kernels,
+# from the ncu capture summarised in profiles/attn_decode_b8_32k.md.  Must be
+# re-measured (or removed) whenever either kernel changes.
+MEASURED_TRAFFIC = {"decode_b8_32k_4layers": 67_303_936 + 1_043_200 + 2_549_760}
+
+
 def run_native(args, cfg, rank, world):
     import torch
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -340,7 +346,8 @@ def run_native(args, cfg, rank, world):
             "bound": "hbm", "achieved": round(attn_gbs, 1) if attn_gbs else None,
             "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(attn_gbs / peaks["hbm_gbs"], 4) if attn_gbs else None,
-            "traffic": args.traffic, "peak_source": peaks["source"],
+            "traffic": args.traffic if args.traffic is not None else MEASURED_TRAFFIC.get(cfg.name),
+            "peak_source": peaks["source"],
             "algorithmic_bytes_per_launch": attn_bytes}
     idx_gbs = score_bytes / cfg.n_groups / (idx_ms * 1e-3) / 1e9 if idx_ms else None
     step_bytes = score_bytes + cfg.n_layers * attn_bytes
