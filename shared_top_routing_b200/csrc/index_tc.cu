@@ -98,8 +98,12 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   const int t_last = min(tr0 + kBM - 1, min(p.t0 + p.rows, p.Tq) - 1);
   long long nc = (long long)p.q_pos0 + t_last + 1;
   if (nc > len) nc = len;
-  const int ntiles = nc > 0 ? (int)((nc + kBN - 1) / kBN) : 0;
-  if (ntiles == 0 || t_last < tr0) return;
+  const int ntiles_all = nc > 0 ? (int)((nc + kBN - 1) / kBN) : 0;
+  // key tiles [i_lo, i_lo + ntiles) of the row block: the block's causal
+  // tiles are split evenly over gridDim.z CTAs (each score is written once)
+  const int i_lo = (int)((long long)blockIdx.z * ntiles_all / gridDim.z);
+  const int ntiles = (int)((long long)(blockIdx.z + 1) * ntiles_all / gridDim.z) - i_lo;
+  if (ntiles <= 0 || t_last < tr0) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
@@ -131,7 +135,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         mbar_arrive_expect_tx(&bars.full[s], S::kBBytes);
 #pragma unroll
         for (int a = 0; a < S::kAtoms; ++a)
-          tma_load_3d(sB + s * S::kBBytes + a * kBN * 128, &tmap_k, &bars.full[s], 64 * a, i * kBN, b);
+          tma_load_3d(sB + s * S::kBBytes + a * kBN * 128, &tmap_k, &bars.full[s], 64 * a, (i_lo + i) * kBN, b);
       }
     }
   } else if (warp == 1) {
@@ -179,7 +183,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         uint32_t v[32];
         tmem_ld32(tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + ch * 32), v);
         tmem_ld_wait();
-        const int c = i * kBN + ch * 32;
+        const int c = (i_lo + i) * kBN + ch * 32;
         if (c < lim) {
           uint4* dst = reinterpret_cast<uint4*>(krow + c);
 #pragma unroll
@@ -253,7 +257,21 @@ cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B,
   p.keys = w.keys;
   p.ld = w.ld;
   p.err = w.err;
-  dim3 grid(p.nblk, B);
+  // key tiles of a row block are split over enough CTAs to fill the GPU
+  // (one CTA per SM: 512 TMEM columns and ~150 KB of shared memory each)
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    sms = n > 0 ? n : 148;
+  }
+  const long long max_tiles = ((long long)q_pos0 + t0 + rows + kBN - 1) / kBN;   // of the last row block
+  long long ks = (2LL * sms + (long long)p.nblk * B - 1) / ((long long)p.nblk * B);
+  if (ks > max_tiles) ks = max_tiles;
+  if (ks > 64) ks = 64;
+  if (ks < 1) ks = 1;
+  dim3 grid(p.nblk, B, (unsigned)ks);
   if (d == 128) {
     constexpr int smem = TcShape<128>::kSmem;
     cudaError_t e = ensure_dynamic_smem((const void*)score_prefill_tc_kernel<128>, smem);
