@@ -7,22 +7,18 @@
 // one kv head are loaded once for all query heads of its GQA group, and the
 // partial (max, sum, output) triples are merged by the log-sum-exp rule.
 //
-// Both kernels share one tile loop (attn_tiles): 64 gathered rows per tile,
-// K and V rows of one kv head (256 contiguous bytes each) gathered with
-// 16-byte cp.async into padded shared tiles, two stages so the gather of tile
-// i+1 overlaps the math of tile i.  Each of the 4 warps owns 16 rows of a
-// tile and runs online softmax on mma.sync m16n8k16 (bf16 in, fp32
-// accumulate) with the G query heads of the group as the 16-row M side
-// (zero padded), S = Q K^T then O += P V (V through ldmatrix.trans).
+// Both paths run online softmax on mma.sync m16n8k16 (bf16 in, fp32
+// accumulate) with the G query heads of a kv head as the 16-row M side (zero
+// padded): S = Q K^T, then O += P V with V through ldmatrix.trans.
 //
-// attn_prefill_kernel  grid (T, Hkv, B), kv-head-major: one query token x one
-//                      kv head per CTA, all of its selected rows.
-// attn_decode_kernel   the 16-row tiles of all (sequence, kv head) pairs are
-//                      split evenly over the warps of a resident-sized grid;
-//                      each warp streams its tiles through a private 3-stage
-//                      cp.async ring, writes a partial (m, l, o) where its
-//                      range leaves a pair, and the warp whose atomic ticket
-//                      completes a pair (never a wait) merges its partials.
+// attn_decode_split_kernel / attn_decode_merge_kernel  one query per
+//     sequence: the tiles of all (sequence, head block) pairs are cut evenly
+//     over one CTA per SM (bulk copies per row run), partials are folded by
+//     the merge kernel.
+// attn_prefill_kernel  one query token x one kv head per CTA, grid (T, Hkv,
+//     B): the token's selected rows of that head (256 bytes each) in 64-row
+//     tiles gathered with 16-byte cp.async by all four warps, two stages, the
+//     four warps' partials merged in shared memory at the end.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -321,6 +317,126 @@ __device__ __forceinline__ int clamp_count(const int32_t* __restrict__ count, in
   return c < 0 ? 0 : (c > k ? k : c);
 }
 
+// One online-softmax step over a 16-row slice of a gathered tile ([YOIO]
+// §1.1 softmax(QK^T/sqrt(d))V, evaluated incrementally): S = Q K^T with the
+// query fragments qa as the M side (G heads, zero padded to 16 rows), rows at
+// or past cnt masked, running max / sum / output rescaled, O += P V.  tK and
+// tV point at the slice's first row for this kv head; rs_el is the shared
+// row stride in elements; rbase is the slice's first row index.
+struct Online {
+  float o[16][4];
+  float m[2], l[2];
+};
+
+__device__ __forceinline__ void online_init(Online& st) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) st.o[i][e] = 0.f;
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.f;
+}
+
+__device__ __forceinline__ void online_tile(Online& st, const uint32_t (&qa)[8][4], const uint16_t* tK,
+                                            const uint16_t* tV, int rs_el, int rbase, int cnt, float qscale) {
+  const int lane = threadIdx.x & 31, tg = lane & 3;
+  // S = Q K^T over 8 k-steps, in two independent accumulator chains
+  float sc[2][4], sd[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 2) {
+    const int mtx = lane >> 3;
+    const uint16_t* kr = tK + ((mtx >> 1) * 8 + (lane & 7)) * rs_el + (mtx & 1) * 8;
+    uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
+    ldmatrix_x4(b0, b1, b2, b3, kr + kk * 16);
+    ldmatrix_x4(c0, c1, c2, c3, kr + (kk + 1) * 16);
+    mma_bf16_16816(sc[0], qa[kk], b0, b1);
+    mma_bf16_16816(sc[1], qa[kk], b2, b3);
+    mma_bf16_16816(sd[0], qa[kk + 1], c0, c1);
+    mma_bf16_16816(sd[1], qa[kk + 1], c2, c3);
+  }
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int row = rbase + nt * 8 + tg * 2 + (e & 1);
+      const float z = row < cnt ? (sc[nt][e] + sd[nt][e]) * qscale : -INFINITY;
+      sc[nt][e] = z;
+      mx[e >> 1] = fmaxf(mx[e >> 1], z);
+    }
+  float alpha[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float v = mx[hh];
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+    const float mnew = fmaxf(st.m[hh], v);
+    const float muse = mnew == -INFINITY ? 0.f : mnew;
+    alpha[hh] = exp2f(st.m[hh] - muse);
+    st.m[hh] = mnew;
+    mx[hh] = muse;
+  }
+  float rsum[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+      sc[nt][e] = pv;
+      rsum[e >> 1] += pv;
+    }
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float v = rsum[hh];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    st.l[hh] = st.l[hh] * alpha[hh] + v;
+  }
+  if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {   // a row max moved
+#pragma unroll
+    for (int dt = 0; dt < 16; ++dt) {
+      st.o[dt][0] *= alpha[0];
+      st.o[dt][1] *= alpha[0];
+      st.o[dt][2] *= alpha[1];
+      st.o[dt][3] *= alpha[1];
+    }
+  }
+  uint32_t pa[4];
+  pa[0] = pack_bf2(sc[0][0], sc[0][1]);
+  pa[1] = pack_bf2(sc[0][2], sc[0][3]);
+  pa[2] = pack_bf2(sc[1][0], sc[1][1]);
+  pa[3] = pack_bf2(sc[1][2], sc[1][3]);
+#pragma unroll
+  for (int dt = 0; dt < 16; dt += 2) {
+    const int mtx = lane >> 3;
+    uint32_t b0, b1, b2, b3;
+    ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * rs_el + (dt + (mtx >> 1)) * 8);
+    mma_bf16_16816(st.o[dt], pa, b0, b1);
+    mma_bf16_16816(st.o[dt + 1], pa, b2, b3);
+  }
+}
+
+// Query fragments of the G heads starting at row head0 of q (rows >= G, or
+// all rows when !active, are zero).
+__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[8][4], const uint16_t* __restrict__ q, long long head0,
+                                             int G, bool active) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tg = lane & 3;
+  const uint32_t* qr0 = reinterpret_cast<const uint32_t*>(q + (head0 + gq) * kD);
+  const uint32_t* qr1 = reinterpret_cast<const uint32_t*>(q + (head0 + gq + 8) * kD);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const int c0 = (kk * 16 + 2 * tg) >> 1, c1 = (kk * 16 + 8 + 2 * tg) >> 1;
+    qa[kk][0] = active && gq < G ? __ldg(qr0 + c0) : 0u;
+    qa[kk][1] = active && gq + 8 < G ? __ldg(qr1 + c0) : 0u;
+    qa[kk][2] = active && gq < G ? __ldg(qr0 + c1) : 0u;
+    qa[kk][3] = active && gq + 8 < G ? __ldg(qr1 + c1) : 0u;
+  }
+}
+
 __global__ void __launch_bounds__(kDxThreads, 1)
 attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
                          const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
@@ -431,8 +547,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
   const int gq = lane >> 2, tg = lane & 3;
   const int hs = warp / pl.wph, rs = warp % pl.wph;
   const int rs_el = rb / 2;   // shared row stride in elements
-  float o[16][4];
-  float m_r[2], l_r[2];
+  Online st;
   uint32_t qa[8][4];
   int cur_p = -1, cnt = 0;
   bool active = false;        // this warp's head exists in the current block
@@ -452,8 +567,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
 #pragma unroll
         for (int dt = 0; dt < 16; ++dt)
           *reinterpret_cast<float2*>(part_o + (base + h) * kD + dt * 8 + 2 * tg) =
-              make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
-        if (tg == 0) *reinterpret_cast<float2*>(part_ml + (base + h) * 2) = make_float2(m_r[hh], l_r[hh]);
+              make_float2(st.o[dt][2 * hh], st.o[dt][2 * hh + 1]);
+        if (tg == 0) *reinterpret_cast<float2*>(part_ml + (base + h) * 2) = make_float2(st.m[hh], st.l[hh]);
       }
     }
   };
@@ -467,23 +582,8 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
       const int g = hb * pl.nh + hs;
       active = hs < min(pl.nh, Hkv - hb * pl.nh);
       head0 = (long long)b * Hq + (long long)(active ? g : 0) * G;
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
-      m_r[0] = m_r[1] = -INFINITY;
-      l_r[0] = l_r[1] = 0.f;
-      // query fragments of the group's heads (rows >= G are zero)
-      const uint32_t* qr0 = reinterpret_cast<const uint32_t*>(q + (head0 + gq) * kD);
-      const uint32_t* qr1 = reinterpret_cast<const uint32_t*>(q + (head0 + gq + 8) * kD);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int c0 = (kk * 16 + 2 * tg) >> 1, c1 = (kk * 16 + 8 + 2 * tg) >> 1;
-        qa[kk][0] = active && gq < G ? __ldg(qr0 + c0) : 0u;
-        qa[kk][1] = active && gq + 8 < G ? __ldg(qr1 + c0) : 0u;
-        qa[kk][2] = active && gq < G ? __ldg(qr0 + c1) : 0u;
-        qa[kk][3] = active && gq + 8 < G ? __ldg(qr1 + c1) : 0u;
-      }
+      online_init(st);
+      load_q_frags(qa, q, head0, G, active);
     }
     const int r0 = u % pl.tpp * R;
     if (r0 >= cnt) continue;   // the producer skips this unit too
@@ -494,84 +594,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
       const uint16_t* tK = reinterpret_cast<const uint16_t*>(smem + (size_t)s * pl.stage_bytes) +
                            (size_t)(rs * 16) * rs_el + hs * kD;
       const uint16_t* tV = tK + (size_t)R * rs_el;
-      // S = Q K^T over 8 k-steps, in two independent accumulator chains
-      float sc[2][4], sd[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] = sd[nt][e] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; kk += 2) {
-        const int mtx = lane >> 3;
-        const uint16_t* kr = tK + ((mtx >> 1) * 8 + (lane & 7)) * rs_el + (mtx & 1) * 8;
-        uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
-        ldmatrix_x4(b0, b1, b2, b3, kr + kk * 16);
-        ldmatrix_x4(c0, c1, c2, c3, kr + (kk + 1) * 16);
-        mma_bf16_16816(sc[0], qa[kk], b0, b1);
-        mma_bf16_16816(sc[1], qa[kk], b2, b3);
-        mma_bf16_16816(sd[0], qa[kk + 1], c0, c1);
-        mma_bf16_16816(sd[1], qa[kk + 1], c2, c3);
-      }
-      float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = rbase + nt * 8 + tg * 2 + (e & 1);
-          const float z = row < cnt ? (sc[nt][e] + sd[nt][e]) * qscale : -INFINITY;
-          sc[nt][e] = z;
-          mx[e >> 1] = fmaxf(mx[e >> 1], z);
-        }
-      float alpha[2];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v = mx[hh];
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-        const float mnew = fmaxf(m_r[hh], v);
-        const float muse = mnew == -INFINITY ? 0.f : mnew;
-        alpha[hh] = exp2f(m_r[hh] - muse);
-        m_r[hh] = mnew;
-        mx[hh] = muse;
-      }
-      float rsum[2] = {0.f, 0.f};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
-          sc[nt][e] = pv;
-          rsum[e >> 1] += pv;
-        }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v = rsum[hh];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        l_r[hh] = l_r[hh] * alpha[hh] + v;
-      }
-      if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {   // a row max moved
-#pragma unroll
-        for (int dt = 0; dt < 16; ++dt) {
-          o[dt][0] *= alpha[0];
-          o[dt][1] *= alpha[0];
-          o[dt][2] *= alpha[1];
-          o[dt][3] *= alpha[1];
-        }
-      }
-      uint32_t pa[4];
-      pa[0] = pack_bf2(sc[0][0], sc[0][1]);
-      pa[1] = pack_bf2(sc[0][2], sc[0][3]);
-      pa[2] = pack_bf2(sc[1][0], sc[1][1]);
-      pa[3] = pack_bf2(sc[1][2], sc[1][3]);
-#pragma unroll
-      for (int dt = 0; dt < 16; dt += 2) {
-        const int mtx = lane >> 3;
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(b0, b1, b2, b3, tV + ((mtx & 1) * 8 + (lane & 7)) * rs_el + (dt + (mtx >> 1)) * 8);
-        mma_bf16_16816(o[dt], pa, b0, b1);
-        mma_bf16_16816(o[dt + 1], pa, b2, b3);
-      }
+      online_tile(st, qa, tK, tV, rs_el, rbase, cnt, qscale);
     }
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(&empty[s]);
