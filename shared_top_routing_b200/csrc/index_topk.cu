@@ -30,10 +30,12 @@
 //       bitmap's reach).  Also expands chosen gist chunks into cache rows, and
 //       returns the row's histogram and candidate counter to zero.
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "sa_common.cuh"
 #include "sa_internal.h"
+#include "tc_common.cuh"
 
 namespace sa {
 namespace {
@@ -264,13 +266,23 @@ struct FinishSmem {
   uint32_t thr[3];
   uint32_t digit, above, bnd_count, ncand;
   uint32_t kor, kand, por, pand;   // OR / AND of every item's key and position
-  uint32_t ckey[kSmemCand];
-  uint32_t cpos[kSmemCand];
-  uint32_t bits[kBitmapWords];   // position bitmap; bucket counts for long rows
+  uint64_t stage_bar[2];           // bulk copies of the row into the staging chunks
+  int abort;
+  alignas(16) uint32_t ckey[kSmemCand];
+  alignas(16) uint32_t cpos[kSmemCand];
+  // bits .. okey are contiguous: before emission they hold the two staging
+  // chunks of the filtered row scan (2 x kStageKeys keys)
+  alignas(16) uint32_t bits[kBitmapWords];   // position bitmap; bucket counts for long rows
   uint32_t wpre[kBitmapWords];   // word prefix sums; bucket starts for long rows
   uint32_t opos[kMaxK];          // long rows: chosen items grouped by bucket
   uint32_t okey[kMaxK];
 };
+constexpr int kStageKeys = 12288;   // keys per staging chunk (48 KB)
+// bulk copies and 16-byte shared loads need 16-byte aligned chunks
+static_assert(offsetof(FinishSmem, bits) % 16 == 0, "staging area must be 16-byte aligned");
+static_assert((kStageKeys * 4) % 16 == 0, "staging chunks must be 16-byte multiples");
+static_assert(offsetof(FinishSmem, stage_bar) % 8 == 0, "mbarriers must be 8-byte aligned");
+static_assert(2 * kStageKeys <= 2 * kBitmapWords + 2 * kMaxK, "staging chunks exceed their area");
 
 __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t digit, bool active) {
   const unsigned act = __ballot_sync(0xffffffffu, active);
@@ -484,56 +496,85 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   bool in_smem = false;
   if (K > 0) {
     if (mode == kFinishHistScan) {
+      // The row streams into shared memory in chunks of kStageKeys keys with
+      // bulk copies, two in flight, the first issued before the histogram
+      // is read; every key in or above the bin of the K-th largest is kept,
+      // each thread counting its takes and one block scan placing them.
+      uint32_t* stage = s.bits;
+      const int nchunks = (n + kStageKeys - 1) / kStageKeys;
+      if (tid == 0) {
+        tc::mbar_init(&s.stage_bar[0], 1);
+        tc::mbar_init(&s.stage_bar[1], 1);
+        s.abort = 0;
+        tc::fence_barrier_init();
+      }
+      __syncthreads();
+      auto issue = [&](int c) {   // thread 0
+        const int c0 = c * kStageKeys, len = min(kStageKeys, n - c0);
+        const uint32_t bytes = (uint32_t)((len + 3) & ~3) * 4u;   // rows are padded to 256 keys
+        tc::mbar_arrive_expect_tx(&s.stage_bar[c & 1], bytes);
+        tc::bulk_load(stage + (c & 1) * kStageKeys, row + c0, bytes, &s.stage_bar[c & 1]);
+      };
+      int issued = 0;   // thread 0: chunks whose copies were issued
+      if (tid == 0) {
+        issue(0);
+        if (nchunks > 1) issue(1);
+        issued = min(nchunks, 2);
+      }
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
-      // keep every key in or above the bin of the K-th largest: each thread
-      // issues all its 16-byte loads, counts its takes, and one block scan
-      // places them (no shared atomics)
-      constexpr int kPer = 4;   // 8 spills at 64 registers
       uint32_t base = 0;
-      for (int i0 = 0; i0 < n; i0 += kFinThreads * 4 * kPer) {
+      for (int c = 0; c < nchunks; ++c) {
+        const bool ok = tc::mbar_wait(&s.stage_bar[c & 1], (uint32_t)(c >> 1) & 1u, &s.abort, w.err, 31);
+        const uint32_t* ck = stage + (c & 1) * kStageKeys;
+        const int c0 = c * kStageKeys, len = ok ? min(kStageKeys, n - c0) : 0;
+        constexpr int kPer = kStageKeys / (4 * kFinThreads);   // uint4 per thread
         uint4 v[kPer];
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int i = i0 + (u * kFinThreads + tid) * 4;
-          v[u] = make_uint4(0, 0, 0, 0);
-          if (i + 3 < n) {
-            v[u] = *reinterpret_cast<const uint4*>(row + i);
-          } else {
-            if (i < n) v[u].x = row[i];
-            if (i + 1 < n) v[u].y = row[i + 1];
-            if (i + 2 < n) v[u].z = row[i + 2];
-          }
-        }
         uint32_t mine = 0;
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
-          const int i = i0 + (u * kFinThreads + tid) * 4;
-          mine += (i < n && (v[u].x >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 1 < n && (v[u].y >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 2 < n && (v[u].z >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 3 < n && (v[u].w >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          const int i = (u * kFinThreads + tid) * 4;
+          v[u] = i < len ? *reinterpret_cast<const uint4*>(ck + i) : make_uint4(0, 0, 0, 0);
+          mine += (i < len && (v[u].x >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 1 < len && (v[u].y >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 2 < len && (v[u].z >> (32 - kHistBits)) >= bin) ? 1u : 0u;
+          mine += (i + 3 < len && (v[u].w >> (32 - kHistBits)) >= bin) ? 1u : 0u;
         }
         uint32_t total;
         uint32_t o = base + block_excl_scan(mine, s.swarp, total);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
-          const int i = i0 + (u * kFinThreads + tid) * 4;
+          const int i = (u * kFinThreads + tid) * 4;
           const uint32_t kk4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            if (i + j < n && (kk4[j] >> (32 - kHistBits)) >= bin) {
+            if (i + j < len && (kk4[j] >> (32 - kHistBits)) >= bin) {
               if (o < (uint32_t)kSmemCand) {
                 s.ckey[o] = kk4[j];
-                s.cpos[o] = (uint32_t)(i + j);
+                s.cpos[o] = (uint32_t)(c0 + i + j);
               }
               ++o;
             }
           }
         }
         base += total;
+        __syncthreads();   // every read of this chunk is done before it is refilled
+        if (tid == 0 && c + 2 < nchunks && !s.abort) {
+          tc::fence_proxy_async();
+          issue(c + 2);
+          issued = c + 3;
+        }
       }
-      if (tid == 0) s.ncand = base;
+      if (tid == 0) {
+        s.ncand = base;
+        // after a wait that gave up, copies may still be in flight: let the
+        // last issued ones land (bounded) before the area is reused
+        if (s.abort) {
+          volatile int keep_waiting = 0;
+          for (int c = max(0, issued - 2); c < issued; ++c)
+            tc::mbar_wait(&s.stage_bar[c & 1], (uint32_t)(c >> 1) & 1u, &keep_waiting, nullptr, 0);
+        }
+      }
       __syncthreads();
       in_smem = s.ncand <= (uint32_t)kSmemCand;
     } else if (mode == kFinishCandList) {
