@@ -494,12 +494,15 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   it.pos = nullptr;
   it.n = n;
   bool in_smem = false;
+  bool from_hist = mode != kFinishDirect;   // the top 12 bits of the K-th key are known
   if (K > 0) {
-    if (mode == kFinishHistScan) {
+    if (mode == kFinishHistScan || (mode == kFinishDirect && n > kSmemCand)) {
       // The row streams into shared memory in chunks of kStageKeys keys with
-      // bulk copies, two in flight, the first issued before the histogram
-      // is read; every key in or above the bin of the K-th largest is kept,
-      // each thread counting its takes and one block scan placing them.
+      // bulk copies, two in flight.  Without the scorer's histogram (long
+      // direct rows) a first pass builds the row's 4096-bin histogram of the
+      // keys' top 12 bits in shared memory.  The filter pass keeps every key
+      // in or above the bin of the K-th largest, each thread counting its
+      // takes and one block scan per chunk placing them.
       uint32_t* stage = s.bits;
       const int nchunks = (n + kStageKeys - 1) / kStageKeys;
       if (tid == 0) {
@@ -509,26 +512,64 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
         tc::fence_barrier_init();
       }
       __syncthreads();
-      auto issue = [&](int c) {   // thread 0
+      int seq = 0;          // chunks streamed so far over all passes (buffer seq & 1)
+      int issued = 0;       // thread 0: chunks issued so far over all passes
+      auto issue = [&](int g, int c) {   // thread 0: chunk c of the pass as stream chunk g
         const int c0 = c * kStageKeys, len = min(kStageKeys, n - c0);
         const uint32_t bytes = (uint32_t)((len + 3) & ~3) * 4u;   // rows are padded to 256 keys
-        tc::mbar_arrive_expect_tx(&s.stage_bar[c & 1], bytes);
-        tc::bulk_load(stage + (c & 1) * kStageKeys, row + c0, bytes, &s.stage_bar[c & 1]);
+        tc::mbar_arrive_expect_tx(&s.stage_bar[g & 1], bytes);
+        tc::bulk_load(stage + (g & 1) * kStageKeys, row + c0, bytes, &s.stage_bar[g & 1]);
+        issued = g + 1;
       };
-      int issued = 0;   // thread 0: chunks whose copies were issued
-      if (tid == 0) {
-        issue(0);
-        if (nchunks > 1) issue(1);
-        issued = min(nchunks, 2);
+      auto prime = [&]() {   // the first two chunks of the next pass
+        if (tid == 0) {
+          tc::fence_proxy_async();
+          issue(seq, 0);
+          if (nchunks > 1) issue(seq + 1, 1);
+        }
+      };
+      auto stream = [&](auto&& visit) {
+        for (int c = 0; c < nchunks; ++c) {
+          const int g = seq + c;
+          const bool ok = tc::mbar_wait(&s.stage_bar[g & 1], (uint32_t)(g >> 1) & 1u, &s.abort, w.err, 31);
+          const int c0 = c * kStageKeys;
+          visit(stage + (g & 1) * kStageKeys, c0, ok ? min(kStageKeys, n - c0) : 0);
+          __syncthreads();   // every read of this chunk is done before it is refilled
+          if (tid == 0 && c + 2 < nchunks && !s.abort) {
+            tc::fence_proxy_async();
+            issue(g + 2, c + 2);
+          }
+        }
+        seq += nchunks;
+      };
+      constexpr int kPer = kStageKeys / (4 * kFinThreads);   // uint4 per thread and chunk
+      if (mode == kFinishHistScan) {
+        prime();
+        hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
+      } else {
+        uint32_t* h = s.ckey;   // the histogram, until the filter pass fills the candidates
+        prime();
+        for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
+        __syncthreads();
+        stream([&](const uint32_t* ck, int, int len) {
+#pragma unroll
+          for (int u = 0; u < kPer; ++u) {
+            const int i = (u * kFinThreads + tid) * 4;
+            if (i < len) {
+              const uint4 v = *reinterpret_cast<const uint4*>(ck + i);
+              atomicAdd(&h[v.x >> (32 - kHistBits)], 1u);
+              if (i + 1 < len) atomicAdd(&h[v.y >> (32 - kHistBits)], 1u);
+              if (i + 2 < len) atomicAdd(&h[v.z >> (32 - kHistBits)], 1u);
+              if (i + 3 < len) atomicAdd(&h[v.w >> (32 - kHistBits)], 1u);
+            }
+          }
+        });
+        prime();
+        hist_threshold(h, K, s.swarp, s.thr);
       }
-      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t bin = s.thr[0];
       uint32_t base = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const bool ok = tc::mbar_wait(&s.stage_bar[c & 1], (uint32_t)(c >> 1) & 1u, &s.abort, w.err, 31);
-        const uint32_t* ck = stage + (c & 1) * kStageKeys;
-        const int c0 = c * kStageKeys, len = ok ? min(kStageKeys, n - c0) : 0;
-        constexpr int kPer = kStageKeys / (4 * kFinThreads);   // uint4 per thread
+      stream([&](const uint32_t* ck, int c0, int len) {
         uint4 v[kPer];
         uint32_t mine = 0;
 #pragma unroll
@@ -558,25 +599,20 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
           }
         }
         base += total;
-        __syncthreads();   // every read of this chunk is done before it is refilled
-        if (tid == 0 && c + 2 < nchunks && !s.abort) {
-          tc::fence_proxy_async();
-          issue(c + 2);
-          issued = c + 3;
-        }
-      }
+      });
       if (tid == 0) {
         s.ncand = base;
         // after a wait that gave up, copies may still be in flight: let the
         // last issued ones land (bounded) before the area is reused
         if (s.abort) {
           volatile int keep_waiting = 0;
-          for (int c = max(0, issued - 2); c < issued; ++c)
-            tc::mbar_wait(&s.stage_bar[c & 1], (uint32_t)(c >> 1) & 1u, &keep_waiting, nullptr, 0);
+          for (int g = max(0, issued - 2); g < issued; ++g)
+            tc::mbar_wait(&s.stage_bar[g & 1], (uint32_t)(g >> 1) & 1u, &keep_waiting, nullptr, 0);
         }
       }
       __syncthreads();
       in_smem = s.ncand <= (uint32_t)kSmemCand;
+      from_hist = true;
     } else if (mode == kFinishCandList) {
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t m = w.cand_cnt[r];
@@ -610,7 +646,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   uint32_t prefix = 0, pmask = 0, pmax = 0;
   if (K > 0) {
     SelStart st;
-    if (mode == kFinishDirect) {
+    if (!from_hist) {
       st = SelStart{0u, 0u, K, (uint32_t)it.n, 24};
     } else {
       // the histogram already fixes the top 12 bits: every item above the

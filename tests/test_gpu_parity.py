@@ -107,6 +107,8 @@ def test_decode_topk_q_pos0_limits_candidates():
     (1, 300, 64, 300, 0),
     (1, 1000, 256, 1000, 0),
     (2, 130, 40, 530, 400),     # chunked prefill: queries are the last 130 of 530 tokens
+    (1, 64, 2048, 20000, 19936),  # rows longer than the in-smem limit: streamed row scan, 2 chunks
+    (1, 16, 300, 40000, 39984),   # 4 chunks, small k
 ])
 def test_prefill_topk_matches_oracle(d, B, L, k, Tk, q_pos0):
     seed = 2000 + L + d
