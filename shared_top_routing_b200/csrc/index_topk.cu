@@ -188,6 +188,11 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
 __device__ __forceinline__ void hist_threshold(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
                                                uint32_t* s_out) {
   const int per = kHistBins / blockDim.x;  // 16 (256 threads) or 4 (1024 threads)
+  if (threadIdx.x == 0) {   // a histogram holding fewer than K keys leaves bin 0 (keep everything)
+    s_out[0] = 0u;
+    s_out[1] = 0u;
+    s_out[2] = 0u;
+  }
   uint32_t loc = 0;
   for (int j = 0; j < per; ++j) loc += h[kHistBins - 1 - (threadIdx.x * per + j)];
   uint32_t total;
@@ -686,7 +691,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
         const uint32_t key = it.k(i), pos = it.p(i);
         if (is_selected(key, pos, prefix, pmask, pmax)) {
           const uint32_t slot = s.wpre[pos >> 5] + __popc(s.bits[pos >> 5] & ((1u << (pos & 31)) - 1u));
-          emit(out, o_idx, b, slot, pos, key);
+          if (slot < K) emit(out, o_idx, b, slot, pos, key);   // exactly K are chosen
         }
       }
     } else {
@@ -732,12 +737,17 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
         }
       }
       __syncthreads();
-      for (int i = tid; i < (int)K; i += kFinThreads) {
+      // exactly K items are chosen; the bounds below only keep a broken
+      // input (e.g. a histogram that does not match the keys) from reading
+      // or writing out of range
+      const uint32_t placed = min(min(total, K), (uint32_t)kMaxK);
+      for (int i = tid; i < (int)placed; i += kFinThreads) {
         const uint32_t pos = s.opos[i], bk = pos >> bsh;
-        const uint32_t b0 = start[bk], b1 = b0 + cnt[bk];
+        if (bk >= (uint32_t)kBitmapWords) continue;
+        const uint32_t b0 = start[bk], b1 = min(b0 + cnt[bk], placed);
         uint32_t rank = b0;
         for (uint32_t j = b0; j < b1; ++j) rank += s.opos[j] < pos ? 1u : 0u;
-        emit(out, o_idx, b, rank, pos, s.okey[i]);
+        if (rank < K) emit(out, o_idx, b, rank, pos, s.okey[i]);
       }
     }
   }
