@@ -606,14 +606,14 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
 // Folds the partials of one (sequence, query head): out = sum_x w_x o_x / L,
 // w_x = 2^(m_x - M), L = sum_x w_x l_x, M = max_x m_x (base-2 logits).  The
 // first loads of every kind are issued together, so the usual case (at most
-// 256 contributors, 4 per warp) costs one memory round trip.  All index
+// 128 contributors, 16 per warp) costs one memory round trip.  All index
 // arithmetic happens before the wait for the split kernel.
 __global__ void __launch_bounds__(kMergeThreads)
 attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, DecPlan pl,
                          int Hq, int Hkv, const int* __restrict__ err, uint16_t* __restrict__ out,
                          float* __restrict__ lse) {
   constexpr int kWarps = kMergeThreads / 32;
-  constexpr int kPre = 4;   // o rows prefetched per warp
+  constexpr int kPre = 16;  // o rows prefetched per warp: up to 128 contributors in one round
   __shared__ float wts[kMergeMaxC];
   __shared__ float red[kWarps][kD];
   __shared__ float rmax[kWarps], rsum[kWarps];
