@@ -345,6 +345,7 @@ struct Items {
 struct SelStart {
   uint32_t prefix, pmask, kk, bnd;
   int shift;
+  bool bits_known;   // s.kor / kand / por / pand already hold the items' OR / AND
 };
 
 // Exact selection of the K largest keys (ties: lower position) among `it`:
@@ -357,14 +358,14 @@ struct SelStart {
 __device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, uint32_t& prefix,
                                  uint32_t& pmask, uint32_t& pmax) {
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    s.kor = 0u;
-    s.kand = ~0u;
-    s.por = 0u;
-    s.pand = ~0u;
-  }
-  __syncthreads();
-  {
+  if (!st.bits_known) {
+    if (tid == 0) {
+      s.kor = 0u;
+      s.kand = ~0u;
+      s.por = 0u;
+      s.pand = ~0u;
+    }
+    __syncthreads();
     uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
     for (int i = tid; i < it.n; i += kFinThreads) {
       const uint32_t key = it.k(i), pos = it.p(i);
@@ -383,8 +384,8 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, ui
       atomicOr(&s.por, po);
       atomicAnd(&s.pand, pa);
     }
+    __syncthreads();
   }
-  __syncthreads();
   const uint32_t kvar = s.kor ^ s.kand, kfix = s.kand;
   const uint32_t pvar = s.por ^ s.pand, pfix = s.pand;
 
@@ -500,6 +501,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   it.n = n;
   bool in_smem = false;
   bool from_hist = mode != kFinishDirect;   // the top 12 bits of the K-th key are known
+  bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
     if (mode == kFinishHistScan || (mode == kFinishDirect && n > kSmemCand)) {
       // The row streams into shared memory in chunks of kStageKeys keys with
@@ -573,7 +575,14 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
         hist_threshold(h, K, s.swarp, s.thr);
       }
       const uint32_t bin = s.thr[0];
+      if (tid == 0) {   // OR / AND of the kept keys and positions, for the select
+        s.kor = 0u;
+        s.kand = ~0u;
+        s.por = 0u;
+        s.pand = ~0u;
+      }
       uint32_t base = 0;
+      uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
       stream([&](const uint32_t* ck, int c0, int len) {
         uint4 v[kPer];
         uint32_t mine = 0;
@@ -595,16 +604,31 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (i + j < len && (kk4[j] >> (32 - kHistBits)) >= bin) {
+              const uint32_t pos = (uint32_t)(c0 + i + j);
               if (o < (uint32_t)kSmemCand) {
                 s.ckey[o] = kk4[j];
-                s.cpos[o] = (uint32_t)(c0 + i + j);
+                s.cpos[o] = pos;
               }
               ++o;
+              ko |= kk4[j];
+              ka &= kk4[j];
+              po |= pos;
+              pa &= pos;
             }
           }
         }
         base += total;
       });
+      ko = __reduce_or_sync(0xffffffffu, ko);
+      ka = __reduce_and_sync(0xffffffffu, ka);
+      po = __reduce_or_sync(0xffffffffu, po);
+      pa = __reduce_and_sync(0xffffffffu, pa);
+      if ((tid & 31) == 0) {
+        atomicOr(&s.kor, ko);
+        atomicAnd(&s.kand, ka);
+        atomicOr(&s.por, po);
+        atomicAnd(&s.pand, pa);
+      }
       if (tid == 0) {
         s.ncand = base;
         // after a wait that gave up, copies may still be in flight: let the
@@ -618,6 +642,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
       __syncthreads();
       in_smem = s.ncand <= (uint32_t)kSmemCand;
       from_hist = true;
+      bits_known = in_smem;   // the OR / AND covers exactly the kept candidates
     } else if (mode == kFinishCandList) {
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t m = w.cand_cnt[r];
@@ -652,12 +677,12 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   if (K > 0) {
     SelStart st;
     if (!from_hist) {
-      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24};
+      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24, false};
     } else {
       // the histogram already fixes the top 12 bits: every item above the
       // bin is chosen, K - above of the bin's items remain to pick
       st = SelStart{s.thr[0] << (32 - kHistBits), ~0u << (32 - kHistBits), K - s.thr[1], s.thr[2],
-                    32 - kHistBits - 8};
+                    32 - kHistBits - 8, bits_known};
     }
     select_threshold(s, it, st, prefix, pmask, pmax);
   }
