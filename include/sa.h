@@ -191,6 +191,23 @@ sa_status sa_sparse_attn_decode_noalloc(const void* q, const void* k_cache, cons
                                         float scale, void* out, float* lse, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Self-test of the bounded waits (no counterpart in the pages).
+ *
+ * Every pipeline kernel of the library waits on mbarrier phases with a poll
+ * limit: a wait that runs out sets the kernel's abort flag and records its
+ * code in an error word instead of hanging the GPU.  This call launches a
+ * one-thread probe that (1) waits on a phase nothing completes, with
+ * `poll_limit` polls, and (2) waits on a phase that does complete.
+ *   err  device int32[5], zero-filled by the caller.  After the stream
+ *        reaches the call: err[0] = 77 (the timed-out wait's code),
+ *        err[1] = 0, err[2] = 0 (the first wait returned false),
+ *        err[3] = 1 (its abort flag was set), err[4] = 1 (the second wait
+ *        returned true).
+ * Faults nothing; returns SA_ERR_INVALID_ARG for a null err or a zero limit.
+ * ---------------------------------------------------------------------- */
+sa_status sa_self_test_bounded_wait(int32_t* err, uint32_t poll_limit, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Gist-chunk routing with selective unfolding (decode).
  *
  * [SSA] §二/§三 and [GSA] 2.1-2.2: the sequence is cut into chunks of

@@ -56,8 +56,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // *flag (shared abort word) and `err_code` in the global error word, and
 // returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* gerr, int err_code) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+                                          int* gerr, int err_code, uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
   }

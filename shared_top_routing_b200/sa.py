@@ -41,6 +41,7 @@ SIGNATURES = {
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "sa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "sa_self_test_bounded_wait": (_I, [_P, ctypes.c_uint32, _P]),
     "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
     "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
@@ -244,6 +245,17 @@ def sa_sparse_attn_decode_noalloc(q, k_cache, v_cache, idx, count, scale: float 
                                              _ptr(lse), _stream(stream))
     _check(st, "sa_sparse_attn_decode_noalloc")
     return (out, lse) if with_lse else out
+
+
+def sa_self_test_bounded_wait(poll_limit: int = 4096, stream=None):
+    """Runs the library's bounded-wait probe on the GPU and returns its five
+    result words (see sa.h): a wait nothing completes must give up with code
+    77 and set its abort flag; a wait that completes must succeed."""
+    import torch
+    err = torch.zeros(5, dtype=torch.int32, device="cuda")
+    st = lib().sa_self_test_bounded_wait(_ptr(err), poll_limit, _stream(stream))
+    _check(st, "sa_self_test_bounded_wait")
+    return err
 
 
 def sa_gist_route_unfold(q_route, gist_key, chunk_len: int, k_chunks: int, partial_len,
