@@ -30,6 +30,8 @@
 //       bitmap's reach).  Also expands chosen gist chunks into cache rows, and
 //       returns the row's histogram and candidate counter to zero.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -265,7 +267,11 @@ collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* 
 
 // ------------------------------------------------------------------- finish
 
-struct FinishSmem {
+// Shared memory of the finish kernel for rows of up to CAND candidates held
+// in shared memory, a position bitmap of BMW words and MAXK staged outputs.
+template <int CAND, int BMW, int MAXK>
+struct FinishSmemT {
+  static constexpr int kCand = CAND, kBmw = BMW, kOut = MAXK;
   uint32_t hist[256];
   uint32_t swarp[33];
   uint32_t thr[3];
@@ -273,15 +279,20 @@ struct FinishSmem {
   uint32_t kor, kand, por, pand;   // OR / AND of every item's key and position
   uint64_t stage_bar[2];           // bulk copies of the row into the staging chunks
   int abort;
-  alignas(16) uint32_t ckey[kSmemCand];
-  alignas(16) uint32_t cpos[kSmemCand];
+  alignas(16) uint32_t ckey[CAND];
+  alignas(16) uint32_t cpos[CAND];
   // bits .. okey are contiguous: before emission they hold the two staging
   // chunks of the filtered row scan (2 x kStageKeys keys)
-  alignas(16) uint32_t bits[kBitmapWords];   // position bitmap; bucket counts for long rows
-  uint32_t wpre[kBitmapWords];   // word prefix sums; bucket starts for long rows
-  uint32_t opos[kMaxK];          // long rows: chosen items grouped by bucket
-  uint32_t okey[kMaxK];
+  alignas(16) uint32_t bits[BMW];   // position bitmap; bucket counts for long rows
+  uint32_t wpre[BMW];               // word prefix sums; bucket starts for long rows
+  uint32_t opos[MAXK];              // long rows: chosen items grouped by bucket
+  uint32_t okey[MAXK];
 };
+// rows of any length (streamed scans, bucketed emission), 1024 threads
+using FinishSmem = FinishSmemT<kSmemCand, kBitmapWords, kMaxK>;
+// rows of at most 2048 candidates, 256 threads: several rows per SM
+using FinishSmemSmall = FinishSmemT<2048, 64, 1>;
+constexpr int kFinThreadsSmall = 256;
 constexpr int kStageKeys = 12288;   // keys per staging chunk (48 KB)
 // bulk copies and 16-byte shared loads need 16-byte aligned chunks
 static_assert(offsetof(FinishSmem, bits) % 16 == 0, "staging area must be 16-byte aligned");
@@ -298,7 +309,8 @@ __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t digit, bool activ
 
 // Warp 0 locates the digit holding the kk-th element, searching from the
 // top bin down (desc) or the bottom bin up (asc).
-__device__ __forceinline__ void find_digit(FinishSmem& s, uint32_t kk, bool desc) {
+template <class Sm>
+__device__ __forceinline__ void find_digit(Sm& s, uint32_t kk, bool desc) {
   if (threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
   uint32_t c[8], loc = 0;
@@ -355,8 +367,9 @@ struct SelStart {
 // (from the OR / AND of all keys, or of all positions) is settled without
 // a pass -- integer-valued scores leave most low mantissa bits zero, and
 // positions below 2^16 leave the high bits zero.
-__device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, uint32_t& prefix,
-                                 uint32_t& pmask, uint32_t& pmax) {
+template <class Sm, int THREADS>
+__device__ void select_threshold(Sm& s, const Items& it, SelStart st, uint32_t& prefix, uint32_t& pmask,
+                                 uint32_t& pmax) {
   const int tid = threadIdx.x;
   if (!st.bits_known) {
     if (tid == 0) {
@@ -367,7 +380,7 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, ui
     }
     __syncthreads();
     uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
-    for (int i = tid; i < it.n; i += kFinThreads) {
+    for (int i = tid; i < it.n; i += THREADS) {
       const uint32_t key = it.k(i), pos = it.p(i);
       ko |= key;
       ka &= key;
@@ -397,9 +410,9 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, ui
     if ((kvar & wmask) == 0u) {
       prefix |= kfix & wmask;   // every item has these bits: nothing is above
     } else {
-      for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
+      for (int i = tid; i < 256; i += THREADS) s.hist[i] = 0;
       __syncthreads();
-      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
+      for (int i0 = 0; i0 < it.n; i0 += THREADS) {
         const int i = i0 + tid;
         const uint32_t key = i < it.n ? it.k(i) : 0u;
         const bool act = i < it.n && (key & pmask) == prefix;
@@ -427,9 +440,9 @@ __device__ void select_threshold(FinishSmem& s, const Items& it, SelStart st, ui
     if ((pvar & wmask) == 0u) {
       pp |= pfix & wmask;
     } else {
-      for (int i = tid; i < 256; i += kFinThreads) s.hist[i] = 0;
+      for (int i = tid; i < 256; i += THREADS) s.hist[i] = 0;
       __syncthreads();
-      for (int i0 = 0; i0 < it.n; i0 += kFinThreads) {
+      for (int i0 = 0; i0 < it.n; i0 += THREADS) {
         const int i = i0 + tid;
         bool act = false;
         uint32_t p = 0;
@@ -477,13 +490,19 @@ __device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int 
   }
 }
 
-__global__ void __launch_bounds__(kFinThreads, 1)
+template <class Sm, int THREADS>
+__global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 4)
 finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
               const int32_t* __restrict__ kv_len, int k, FinishOut out) {
   pdl_wait();
   pdl_launch_dependents();
+  constexpr int kFinThreads = THREADS;
+  constexpr int kSmemCand = Sm::kCand;
+  constexpr int kBitmapWords = Sm::kBmw;
+  constexpr int kMaxK = Sm::kOut;
+  constexpr bool kLong = Sm::kCand == ::sa::kSmemCand;   // the layout that serves rows of any length
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  FinishSmem& s = *reinterpret_cast<FinishSmem*>(smem_raw);
+  Sm& s = *reinterpret_cast<Sm*>(smem_raw);
   const int r = blockIdx.x;
   const int b = r / rows_per_batch;
   const int t = t0 + r % rows_per_batch;
@@ -503,6 +522,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   bool from_hist = mode != kFinishDirect;   // the top 12 bits of the K-th key are known
   bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
+    if constexpr (kLong) {
     if (mode == kFinishHistScan || (mode == kFinishDirect && n > kSmemCand)) {
       // The row streams into shared memory in chunks of kStageKeys keys with
       // bulk copies, two in flight.  Without the scorer's histogram (long
@@ -666,6 +686,13 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
       }
       __syncthreads();
     }
+    } else {
+      // the small layout serves direct rows of at most kSmemCand candidates
+      for (int i = tid; i < n; i += kFinThreads) { s.ckey[i] = row[i]; s.cpos[i] = (uint32_t)i; }
+      if (tid == 0) s.ncand = (uint32_t)n;
+      in_smem = true;
+      __syncthreads();
+    }
     if (in_smem) {
       it.key = s.ckey;
       it.pos = s.cpos;
@@ -684,7 +711,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
       st = SelStart{s.thr[0] << (32 - kHistBits), ~0u << (32 - kHistBits), K - s.thr[1], s.thr[2],
                     32 - kHistBits - 8, bits_known};
     }
-    select_threshold(s, it, st, prefix, pmask, pmax);
+    select_threshold<Sm, THREADS>(s, it, st, prefix, pmask, pmax);
   }
 
   const long long o_idx = ((long long)b * Tq + t) * (long long)k;
@@ -719,7 +746,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
           if (slot < K) emit(out, o_idx, b, slot, pos, key);   // exactly K are chosen
         }
       }
-    } else {
+    } else if constexpr (kLong) {
       // ---- long rows: the chosen items are counted into kBitmapWords
       // equal position ranges, placed range by range, and ranked inside
       // their range (ranges hold about K / kBitmapWords items each)
@@ -907,11 +934,23 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
                           const FinishOut& out, cudaStream_t st) {
   const int rows = B * rows_per_batch;
   if (rows <= 0) return cudaSuccess;
-  const size_t smem = sizeof(FinishSmem);
-  cudaError_t e = ensure_dynamic_smem((const void*)finish_kernel, smem);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(finish_kernel, dim3(rows), dim3(kFinThreads), smem, st, w, mode, rows_per_batch, t0, Tq, Tk,
-                 q_pos0, kv_len, k, out);
+  // the longest row of the launch decides the layout: direct rows of at most
+  // 2048 candidates take the small one (256 threads, several rows per SM)
+  const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + t0 + rows_per_batch);
+  cudaError_t e;
+  if (mode == kFinishDirect && n_max <= FinishSmemSmall::kCand) {
+    const size_t smem = sizeof(FinishSmemSmall);
+    auto kern = finish_kernel<FinishSmemSmall, kFinThreadsSmall>;
+    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3(rows), dim3(kFinThreadsSmall), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
+                   kv_len, k, out);
+  } else {
+    const size_t smem = sizeof(FinishSmem);
+    auto kern = finish_kernel<FinishSmem, kFinThreads>;
+    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3(rows), dim3(kFinThreads), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
+                   kv_len, k, out);
+  }
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
