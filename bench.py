@@ -211,13 +211,16 @@ class DecodeBench:
                 if ev is not None:
                     ev[("idx", layer, 1)].record()
             idx, cnt, _ = self.cache.get_tensors(layer)
-            if ev is not None:
-                ev[("attn", layer, 0)].record()
+            g = layer // c.share_every
+            first = layer % c.share_every == 0
+            last = layer % c.share_every == c.share_every - 1 or layer == c.n_layers - 1
+            if ev is not None and first:
+                ev[("attn", g, 0)].record()
             sa.sa_sparse_attn_decode(self.inp["q"][layer][s], self.inp["K"][layer], self.inp["V"][layer],
                                      idx.view(c.B, c.k), cnt.view(c.B), out=self.out[layer],
                                      ws=self.ws_attn)
-            if ev is not None:
-                ev[("attn", layer, 1)].record()
+            if ev is not None and last:
+                ev[("attn", g, 1)].record()
 
     def _new_events(self):
         torch, c = self.torch, self.cfg
@@ -226,13 +229,14 @@ class DecodeBench:
             for e in (0, 1):
                 if layer % c.share_every == 0:
                     ev[("idx", layer, e)] = torch.cuda.Event(enable_timing=True, external=True)
-                ev[("attn", layer, e)] = torch.cuda.Event(enable_timing=True, external=True)
+                    ev[("attn", layer // c.share_every, e)] = torch.cuda.Event(enable_timing=True, external=True)
         return ev
 
     def capture(self, steps, rt):
         """Two graphs per step: the timed one holds only the step's kernels
         (event nodes between them would break the programmatic launch chain);
-        the other brackets every call with events for per-kernel times."""
+        the other brackets each indexer run, and each group's run of
+        consecutive attention calls, with events."""
         torch = self.torch
         self.rt = rt
         self.stream = torch.cuda.Stream(device=self.dev)
@@ -253,16 +257,24 @@ class DecodeBench:
         self.torch.cuda.synchronize()
 
     def kernel_times(self, steps):
-        """Average per-launch device time (ms) of the index and attention
-        parts, from the events captured inside the graphs."""
+        """Average device time (ms) of one indexer run and of one attention
+        call, from the events captured inside the graphs.  An attention call
+        is timed as its group's run of consecutive calls (chained by
+        programmatic launch, as in the timed graphs) divided by the calls in
+        the run."""
+        c = self.cfg
         idx_t, attn_t = [], []
         for s in set(steps):
             ev = self.events[s]
-            for (kind, layer, e), a in ev.items():
+            for (kind, i, e), a in ev.items():
                 if e != 0:
                     continue
-                dt = a.elapsed_time(ev[(kind, layer, 1)])
-                (idx_t if kind == "idx" else attn_t).append(dt)
+                dt = a.elapsed_time(ev[(kind, i, 1)])
+                if kind == "idx":
+                    idx_t.append(dt)
+                else:
+                    calls = min(c.share_every, c.n_layers - i * c.share_every)
+                    attn_t.append(dt / calls)
         return (statistics.mean(idx_t) if idx_t else None, statistics.mean(attn_t) if attn_t else None)
 
     def algorithmic_bytes(self):
@@ -362,7 +374,8 @@ def run_native(args, cfg, rank, world):
                    "parallelism": f"replicas{world}",
                    "l2": "no flush; per-step working set 320 MiB and caches 4.3 GB exceed the 126 MB L2",
                    "timing": "CUDA graphs per step, CUDA events on the launch stream, max over ranks; "
-                             "per-call kernel times from separate event-bracketed graphs"},
+                             "per-call kernel times from separate graphs whose events bracket each "
+                             "indexer run and each group's run of attention calls (time / calls)"},
         "roofline": roof,
         "kernels": {"index_topk_ms": round(idx_ms, 5) if idx_ms else None,
                     "index_topk_scoring_GBps": round(idx_gbs, 1) if idx_gbs else None,

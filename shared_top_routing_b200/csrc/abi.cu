@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <set>
@@ -164,8 +165,8 @@ size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
     const int mode = sa::finish_mode_for(Tk_max, &collect);
     return sa::row_workspace_bytes(B, Tk_max, collect, mode != sa::kFinishDirect);
   }
-  int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
-  return sa::row_workspace_bytes(B * rows, Tk_max, false, false);
+  const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
+  return sa::prefill_workspace_bytes(B * rows, Tk_max, k);
 }
 
 sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int Tq, int Tk,
@@ -202,15 +203,34 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
       return cuda_fail(e, "finish launch");
     return ok();
   }
-  const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max);
+  const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
   sa::RowWorkspace w;
-  sa::carve_row_workspace(ws, B * rows, Tk_max, false, false, &w);
+  sa::carve_prefill_workspace(ws, B * rows, Tk_max, k, &w);
   for (int t0 = 0; t0 < Tq; t0 += rows) {
     const int nr = (Tq - t0 < rows) ? Tq - t0 : rows;
-    if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, w, cs)) != cudaSuccess)
-      return cuda_fail(e, "score_prefill launch");
-    if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, sa::kFinishDirect, out, cs)) != cudaSuccess)
-      return cuda_fail(e, "finish launch");
+    const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + t0 + nr);
+    if (n_max <= sa::kBoundedMinCand) {
+      // short rows: every score's key, then one CTA per row selects
+      if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, k, sa::kScoreKeys, w,
+                                        cs)) != cudaSuccess)
+        return cuda_fail(e, "score_prefill launch");
+      if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, sa::kFinishDirect, out, cs)) != cudaSuccess)
+        return cuda_fail(e, "finish launch");
+    } else {
+      // long rows: group maxima, the per-row bound, the keys at or above it,
+      // then the exact selection among those
+      if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, k, sa::kScoreGroupMax,
+                                        w, cs)) != cudaSuccess)
+        return cuda_fail(e, "score_prefill launch");
+      if ((e = sa::launch_prefill_threshold(B, nr, t0, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
+        return cuda_fail(e, "threshold launch");
+      if ((e = sa::launch_score_prefill(q, km, B, Tq, d, Tk_max, Tk, q_pos0, kv_len, t0, nr, k, sa::kScoreCand, w,
+                                        cs)) != cudaSuccess)
+        return cuda_fail(e, "score_prefill launch");
+      if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, sa::kFinishCandRows, out, cs)) !=
+          cudaSuccess)
+        return cuda_fail(e, "finish launch");
+    }
   }
   return ok();
 }

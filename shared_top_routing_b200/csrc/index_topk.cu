@@ -21,9 +21,13 @@
 //   collect_kernel       (rows longer than one CTA can scan) finds, from the
 //       histogram, the bin holding the k-th largest key and appends every key
 //       in that bin or above to a per-row candidate list (one atomic per CTA).
+//   prefill_threshold_kernel  (long prefill rows) the k-th largest of the
+//       row's 16-bit group maxima, by a two-digit radix select: the bound the
+//       second scoring pass keeps keys against.
 //   finish_kernel        one CTA per row: gathers the row's candidates into
 //       shared memory (histogram-filtered scan of the row, the collected
-//       list, or the whole row), runs an exact radix select (8-bit digits,
+//       list, the bounded pass's list, or the whole row), runs an exact
+//       radix select (8-bit digits,
 //       warp-aggregated shared histograms) of the k-th key and of the tie
 //       positions, then emits in ascending position order through a position
 //       bitmap and popcount prefix sums (bitonic sort for rows beyond the
@@ -293,6 +297,9 @@ using FinishSmem = FinishSmemT<kSmemCand, kBitmapWords, kMaxK>;
 // rows of at most 2048 candidates, 256 threads: several rows per SM
 using FinishSmemSmall = FinishSmemT<2048, 64, 1>;
 constexpr int kFinThreadsSmall = 256;
+// candidate lists of rows up to 65536 positions (4096 held in shared
+// memory, more read in place), 256 threads: several rows per SM
+using FinishSmemMed = FinishSmemT<4096, 2048, 1>;
 constexpr int kStageKeys = 12288;   // keys per staging chunk (48 KB)
 // bulk copies and 16-byte shared loads need 16-byte aligned chunks
 static_assert(offsetof(FinishSmem, bits) % 16 == 0, "staging area must be 16-byte aligned");
@@ -343,12 +350,14 @@ __device__ __forceinline__ void find_digit(Sm& s, uint32_t kk, bool desc) {
 }
 
 // Items: keys with explicit positions, or a row of keys (position = index).
+// (stride 2: keys and positions interleaved as (key, position) pairs)
 struct Items {
   const uint32_t* key;
   const uint32_t* pos;
   int n;
-  __device__ __forceinline__ uint32_t k(int i) const { return key[i]; }
-  __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i] : (uint32_t)i; }
+  int stride = 1;
+  __device__ __forceinline__ uint32_t k(int i) const { return key[(long long)i * stride]; }
+  __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[(long long)i * stride] : (uint32_t)i; }
 };
 
 // Where the search for the K-th key starts: the bits of its key already
@@ -490,6 +499,153 @@ __device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int 
   }
 }
 
+// ---------------------------------------------------------------- threshold
+
+constexpr int kThrBins = 4096;     // window of the counting select
+constexpr int kThrThreads = 512;
+constexpr int kThrVec = 4;         // 16-byte loads (8 maxima each) per thread
+constexpr int kThrRegMax = kThrThreads * kThrVec * 8;   // maxima held in registers
+
+struct ThrSmem {
+  uint32_t hist[kThrBins];
+  uint32_t swarp[33];
+  uint32_t lo, hi;
+  uint32_t digit, above, bnd_count;
+};
+
+// One CTA per row: the k-th largest of the row's m group maxima (16-bit
+// keys).  Up to kThrRegMax maxima are loaded once, 16 bytes at a time, and
+// kept in registers.  One counting pass over the kThrBins values ending at
+// their maximum finds the k-th when at least k maxima fall in that window
+// (the usual case: the upper maxima of large groups sit in a narrow band);
+// otherwise a two-digit radix select (high byte, then low byte) does,
+// reading the row again.
+__global__ void __launch_bounds__(kThrThreads)
+prefill_threshold_kernel(const uint16_t* __restrict__ gmax, long long ld2, int rows_per_batch, int t0, int Tk,
+                         int q_pos0, const int32_t* __restrict__ kv_len, int k, uint32_t* __restrict__ theta) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ ThrSmem s;
+  const int r = blockIdx.x;
+  const int b = r / rows_per_batch;
+  const int t = t0 + r % rows_per_batch;
+  const int tid = threadIdx.x;
+  const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
+  const int g = prefill_group_size(n, k);
+  if (g == 0) {   // every candidate is chosen
+    if (tid == 0) theta[r] = 0u;
+    return;
+  }
+  const int m = (n + g - 1) / g;   // > k
+  const uint16_t* row = gmax + (long long)r * ld2;
+  const bool in_regs = m <= kThrRegMax;
+  uint4 v[kThrVec];
+  uint32_t vmax = 0u;
+  if (in_regs) {
+#pragma unroll
+    for (int q = 0; q < kThrVec; ++q) {
+      const int i = (q * kThrThreads + tid) * 8;
+      v[q] = i < m ? *reinterpret_cast<const uint4*>(row + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < kThrVec; ++q) {
+      const int i = (q * kThrThreads + tid) * 8;
+      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (i + e < m) vmax = max(vmax, (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
+      }
+    }
+  } else {
+    for (int i = tid; i < m; i += kThrThreads) vmax = max(vmax, (uint32_t)row[i]);
+  }
+  vmax = __reduce_max_sync(0xffffffffu, vmax);
+  if (tid == 0) s.hi = 0u;
+  for (int i = tid; i < kThrBins; i += kThrThreads) s.hist[i] = 0u;
+  __syncthreads();
+  if ((tid & 31) == 0) atomicMax(&s.hi, vmax);
+  __syncthreads();
+  const uint32_t lo = s.hi >= (uint32_t)(kThrBins - 1) ? s.hi - (uint32_t)(kThrBins - 1) : 0u;
+  {
+    uint32_t below = 0;   // maxima under the window
+    if (in_regs) {
+#pragma unroll
+      for (int q = 0; q < kThrVec; ++q) {
+        const int i = (q * kThrThreads + tid) * 8;
+        const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t x = (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+          if (i + e < m) {
+            if (x >= lo) atomicAdd(&s.hist[x - lo], 1u);
+            else ++below;
+          }
+        }
+      }
+    } else {
+      for (int i = tid; i < m; i += kThrThreads) {
+        const uint32_t x = row[i];
+        if (x >= lo) atomicAdd(&s.hist[x - lo], 1u);
+        else ++below;
+      }
+    }
+    below = __reduce_add_sync(0xffffffffu, below);
+    if (tid == 0) s.lo = 0u;
+    __syncthreads();
+    if ((tid & 31) == 0) atomicAdd(&s.lo, below);
+    __syncthreads();
+  }
+  if ((uint32_t)m - s.lo >= (uint32_t)k) {   // the k-th largest lies in the window
+    // thread tid holds bins [kThrBins - per (tid + 1), kThrBins - per tid), counted from the top
+    constexpr int per = kThrBins / kThrThreads;
+    uint32_t c[per], loc = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      c[j] = s.hist[kThrBins - 1 - (tid * per + j)];
+      loc += c[j];
+    }
+    uint32_t total;
+    const uint32_t above = block_excl_scan(loc, s.swarp, total);
+    if (above < (uint32_t)k && (uint32_t)k <= above + loc) {
+      uint32_t cum = above;
+#pragma unroll
+      for (int j = 0; j < per; ++j) {
+        cum += c[j];
+        if (cum >= (uint32_t)k) {
+          theta[r] = lo + (uint32_t)(kThrBins - 1 - (tid * per + j));
+          break;
+        }
+      }
+    }
+    return;
+  }
+  // wide span: high byte, then low byte among the values sharing it
+  if (tid < 256) s.hist[tid] = 0u;
+  __syncthreads();
+  for (int i0 = 0; i0 < m; i0 += kThrThreads) {
+    const int i = i0 + tid;
+    const uint32_t x = i < m ? row[i] : 0u;
+    hist_add(s.hist, x >> 8, i < m);
+  }
+  __syncthreads();
+  find_digit(s, (uint32_t)k, true);
+  __syncthreads();
+  const uint32_t hi = s.digit;
+  const uint32_t kk = (uint32_t)k - s.above;
+  __syncthreads();
+  if (tid < 256) s.hist[tid] = 0u;
+  __syncthreads();
+  for (int i0 = 0; i0 < m; i0 += kThrThreads) {
+    const int i = i0 + tid;
+    const uint32_t x = i < m ? row[i] : 0u;
+    hist_add(s.hist, x & 255u, i < m && (x >> 8) == hi);
+  }
+  __syncthreads();
+  find_digit(s, kk, true);
+  __syncthreads();
+  if (tid == 0) theta[r] = hi << 8 | s.digit;
+}
+
 template <class Sm, int THREADS>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 4)
 finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
@@ -519,10 +675,100 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   it.pos = nullptr;
   it.n = n;
   bool in_smem = false;
-  bool from_hist = mode != kFinishDirect;   // the top 12 bits of the K-th key are known
+  // the top 12 bits of the K-th key are known from the scorer's histogram
+  bool from_hist = mode == kFinishHistScan || mode == kFinishCandList;
   bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
-    if constexpr (kLong) {
+    if (mode == kFinishCandRows) {
+      // the bounded pass's takes, (score bits, position) pairs: each scoring
+      // CTA left its run of this row at the run's first column, the run's
+      // count in that tile's slot (0 in the run's other slots).  Counts are
+      // clamped to the columns left, so every read stays in the row.  Slots
+      // are taken kFinThreads at a time; each warp copies its lanes' runs
+      // with all 32 lanes.
+      uint2* cr = reinterpret_cast<uint2*>(w.keys) + (long long)r * w.ld;
+      const uint32_t* tcnt = w.tile_cnt + (long long)r * (w.ld / 256);
+      const int nslot = (n + 255) / 256;
+      auto slot_count = [&](int sl) { return sl < nslot ? min(tcnt[sl], (uint32_t)(n - sl * 256)) : 0u; };
+      uint32_t total = 0;
+      for (int s0 = 0; s0 < nslot; s0 += kFinThreads) {
+        uint32_t part;
+        block_excl_scan(slot_count(s0 + tid), s.swarp, part);
+        total += part;
+      }
+      if (total <= (uint32_t)kSmemCand) {
+        uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
+        uint32_t base = 0;
+        for (int s0 = 0; s0 < nslot; s0 += kFinThreads) {
+          const int sl = s0 + tid;
+          const uint32_t c = slot_count(sl);
+          uint32_t part;
+          const uint32_t o = base + block_excl_scan(c, s.swarp, part);
+          base += part;
+          unsigned todo = __ballot_sync(0xffffffffu, c != 0u);
+          while (todo) {
+            const int L = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const uint32_t cL = __shfl_sync(0xffffffffu, c, L);
+            const uint32_t oL = __shfl_sync(0xffffffffu, o, L);
+            const long long from = (long long)__shfl_sync(0xffffffffu, sl, L) * 256;
+            for (uint32_t j = (uint32_t)(tid & 31); j < cL; j += 32) {
+              const uint2 e = cr[from + j];
+              const uint32_t key = score_key(__uint_as_float(e.x));
+              s.ckey[oL + j] = key;
+              s.cpos[oL + j] = e.y;
+              ko |= key;
+              ka &= key;
+              po |= e.y;
+              pa &= e.y;
+            }
+          }
+        }
+        if (tid == 0) {
+          s.kor = 0u;
+          s.kand = ~0u;
+          s.por = 0u;
+          s.pand = ~0u;
+          s.ncand = total;
+        }
+        __syncthreads();
+        ko = __reduce_or_sync(0xffffffffu, ko);
+        ka = __reduce_and_sync(0xffffffffu, ka);
+        po = __reduce_or_sync(0xffffffffu, po);
+        pa = __reduce_and_sync(0xffffffffu, pa);
+        if ((tid & 31) == 0) {
+          atomicOr(&s.kor, ko);
+          atomicAnd(&s.kand, ka);
+          atomicOr(&s.por, po);
+          atomicAnd(&s.pand, pa);
+        }
+        in_smem = true;
+        bits_known = true;
+      } else {
+        // more takes than shared memory holds (heavy ties): close the gaps
+        // between runs in place, kFinThreads pairs per round (a round's
+        // writes land at or before its reads, which are all done), turning
+        // scores into keys on the way
+        uint32_t dst = 0;
+        for (int sl = 0; sl < nslot; ++sl) {
+          const uint32_t c = slot_count(sl);
+          for (uint32_t j0 = 0; j0 < c; j0 += kFinThreads) {
+            const uint32_t j = j0 + tid;
+            uint2 e = make_uint2(0u, 0u);
+            if (j < c) e = cr[(long long)sl * 256 + j];
+            __syncthreads();
+            if (j < c) cr[dst + j] = make_uint2(score_key(__uint_as_float(e.x)), e.y);
+            __syncthreads();
+          }
+          dst += c;
+        }
+        it.key = reinterpret_cast<const uint32_t*>(cr);
+        it.pos = reinterpret_cast<const uint32_t*>(cr) + 1;
+        it.stride = 2;
+        it.n = (int)total;
+      }
+      __syncthreads();
+    } else if constexpr (kLong) {
     if (mode == kFinishHistScan || (mode == kFinishDirect && n > kSmemCand)) {
       // The row streams into shared memory in chunks of kStageKeys keys with
       // bulk copies, two in flight.  Without the scorer's histogram (long
@@ -716,7 +962,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
 
   const long long o_idx = ((long long)b * Tq + t) * (long long)k;
   if (K > 0) {
-    if (n <= kBitmapMax) {
+    if (n <= kBitmapWords * 32) {
       // ---- emission through a position bitmap
       const int W = (n + 31) >> 5;
       for (int i = tid; i < W; i += kFinThreads) s.bits[i] = 0;
@@ -826,7 +1072,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   }
 
   // ---- return this row's histogram and candidate counter to zero
-  if (mode != kFinishDirect) {
+  if (mode == kFinishHistScan || mode == kFinishCandList) {
     __syncthreads();
     uint32_t* h = w.hist + (long long)r * kHistBins;
     for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
@@ -944,6 +1190,12 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
     if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
     e = launch_pdl(kern, dim3(rows), dim3(kFinThreadsSmall), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
                    kv_len, k, out);
+  } else if (mode == kFinishCandRows && n_max <= FinishSmemMed::kBmw * 32) {
+    const size_t smem = sizeof(FinishSmemMed);
+    auto kern = finish_kernel<FinishSmemMed, kFinThreadsSmall>;
+    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3(rows), dim3(kFinThreadsSmall), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
+                   kv_len, k, out);
   } else {
     const size_t smem = sizeof(FinishSmem);
     auto kern = finish_kernel<FinishSmem, kFinThreads>;
@@ -964,14 +1216,53 @@ int finish_mode_for(int Tk_max, bool* need_collect) {
   return kFinishCandList;
 }
 
-int prefill_rows_per_launch(int B, int Tq, int Tk_max) {
-  // Key slab of at most 512 MiB: rows * B * ld * 4 bytes.
+// Prefill layout: [error word][keys: rows x ld][second slab: rows x ld]
+// [group maxima: rows x ld2 (16-bit)][bound: rows][run counts: rows x
+// ld/256].  Short batches use only the key slab; long ones use both slabs as
+// one [rows][ld] array of (score bits, position) pairs for the bounded
+// pass's takes (each scoring CTA's run of a row at the run's first column).
+size_t prefill_workspace_bytes(int rows, int Tk_max, int k) {
   const long long ld = row_ld(Tk_max);
-  long long cap = (512ll << 20) / (4ll * ld * (B > 0 ? B : 1));
+  const long long ld2 = prefill_groups_ld(Tk_max, k);
+  return 256 + 2 * align256((size_t)rows * ld * 4) + align256((size_t)rows * ld2 * 2) +
+         align256((size_t)rows * 4) + align256((size_t)rows * (ld / 256) * 4);
+}
+
+void carve_prefill_workspace(void* ws, int rows, int Tk_max, int k, RowWorkspace* o) {
+  char* p = static_cast<char*>(ws);
+  o->ld = row_ld(Tk_max);
+  o->ld2 = prefill_groups_ld(Tk_max, k);
+  o->err = reinterpret_cast<int*>(p);
+  p += 256;
+  o->keys = reinterpret_cast<uint32_t*>(p);
+  p += align256((size_t)rows * o->ld * 4);
+  o->cand_pos = reinterpret_cast<uint32_t*>(p);
+  p += align256((size_t)rows * o->ld * 4);
+  o->gmax = reinterpret_cast<uint16_t*>(p);
+  p += align256((size_t)rows * o->ld2 * 2);
+  o->theta = reinterpret_cast<uint32_t*>(p);
+  p += align256((size_t)rows * 4);
+  o->tile_cnt = reinterpret_cast<uint32_t*>(p);
+}
+
+int prefill_rows_per_launch(int B, int Tq, int Tk_max, int k) {
+  // the two [rows][ld] slabs (keys, candidate positions) take at most 1 GiB;
+  // the group maxima and per-row words come on top
+  (void)k;
+  long long cap = (1ll << 30) / (8ll * row_ld(Tk_max) * (B > 0 ? B : 1));
   cap = cap / 128 * 128;
   if (cap < 128) cap = 128;
   if (cap > Tq) cap = Tq;
   return (int)cap;
+}
+
+cudaError_t launch_prefill_threshold(int B, int rows_per_batch, int t0, int Tk, int q_pos0,
+                                     const int32_t* kv_len, int k, const RowWorkspace& w, cudaStream_t st) {
+  const int rows = B * rows_per_batch;
+  if (rows <= 0) return cudaSuccess;
+  const cudaError_t e = launch_pdl(prefill_threshold_kernel, dim3(rows), dim3(kThrThreads), 0, st, w.gmax, w.ld2,
+                                   rows_per_batch, t0, Tk, q_pos0, kv_len, k, w.theta);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sa

@@ -11,6 +11,33 @@ constexpr int kHistBits = 12;        // first radix digit of a score key
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kCandCap = 32768;      // candidate slots per row before the full-row fallback
 
+// Long prefill rows are selected in two scoring passes.  The first keeps,
+// per row, only the maximum score of each group of g consecutive positions
+// (g a power of two <= kGroupMax, the largest with n >= 2 k g, so a row has
+// between k+1 and 4k groups while g < kGroupMax).  At least k keys are >= the
+// k-th largest group maximum, so it bounds the k-th largest key from below;
+// the second pass keeps only the keys at or above that bound.
+constexpr int kGroupMax = 64;
+
+// Group size of a row of n candidates for top-k (0: n <= k, every candidate
+// is chosen and no bound is needed).
+__host__ __device__ __forceinline__ int prefill_group_size(int n, int k) {
+  if (n <= k) return 0;
+  int g = 1;
+  while (g * 2 <= kGroupMax && (long long)n >= 4LL * k * g) g *= 2;
+  return g;
+}
+
+// Group maxima kept per row for rows of at most n_max candidates (plus one
+// 32-column chunk of slack: a chunk past the row end is written whole),
+// rounded to 8 entries so rows stay 16-byte aligned.
+__host__ __device__ __forceinline__ long long prefill_groups_ld(long long n_max, int k) {
+  long long m = 4LL * k;
+  const long long m_cap = (n_max + kGroupMax - 1) / kGroupMax;
+  if (m_cap > m) m = m_cap;
+  return (m + 32 + 7) / 8 * 8;
+}
+
 // Order-preserving 32-bit key of an fp32 score: a larger key is a larger
 // score.  -0.0 is mapped to +0.0 first so that the two compare equal.
 __device__ __forceinline__ uint32_t score_key(float s) {

@@ -18,6 +18,12 @@ constexpr int kDirectMaxCand = 8192;
 constexpr int kFinishDirect = 0;    // the whole row (no histogram)
 constexpr int kFinishHistScan = 1;  // one CTA scans the row, keeping keys in or above the k-th key's bin
 constexpr int kFinishCandList = 2;  // candidates collected by collect_kernel
+constexpr int kFinishCandRows = 3;  // prefill: candidates appended by the bounded scoring pass
+
+// Prefill scoring passes (launch_score_prefill `epi`)
+constexpr int kScoreKeys = 0;       // every score's key into the row slab
+constexpr int kScoreGroupMax = 1;   // per-row group maxima (16-bit keys)
+constexpr int kScoreCand = 2;       // keys at or above the row's bound, appended with positions
 
 // Rows whose histograms live in the fixed, self-cleaning workspace region.
 constexpr int kHistRowsFixed = 64;
@@ -25,12 +31,16 @@ constexpr int kHistRowsFixed = 64;
 struct RowWorkspace {
   int* err = nullptr;            // first word: kernel error code (0 = none)
   size_t hist_zero_bytes = 0;    // > 0: histograms + counters must be zeroed per call
-  uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys
+  uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys (prefill candidate rows: their keys)
   long long ld = 0;
   uint32_t* hist = nullptr;      // [rows][kHistBins]
   uint32_t* cand_cnt = nullptr;  // [rows]
   uint32_t* cand_key = nullptr;  // [rows][kCandCap]
-  uint32_t* cand_pos = nullptr;  // [rows][kCandCap]
+  uint32_t* cand_pos = nullptr;  // [rows][kCandCap]; prefill candidate rows: [rows][ld]
+  uint16_t* gmax = nullptr;      // prefill: [rows][ld2] group maxima
+  long long ld2 = 0;
+  uint32_t* theta = nullptr;     // prefill: [rows] 16-bit bound per row
+  uint32_t* tile_cnt = nullptr;  // prefill: [rows][ld / 256] takes of the run starting at each key tile
 };
 
 // Finish-kernel output description.
@@ -96,11 +106,22 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
 // Candidate source for rows of Tk_max positions; sets *need_collect when the
 // collect pass must run between scoring and finish.
 int finish_mode_for(int Tk_max, bool* need_collect);
-// Prefill scoring of queries [t0, t0+rows) into the key slab (tcgen05, index_tc.cu).
+// Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`
+// picks what is kept per score (kScoreKeys / kScoreGroupMax / kScoreCand).
 cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,
                                  int Tk_max, int Tk, int q_pos0, const int32_t* kv_len, int t0,
-                                 int rows, const RowWorkspace& w, cudaStream_t st);
-int prefill_rows_per_launch(int B, int Tq, int Tk_max);
+                                 int rows, int k, int epi, const RowWorkspace& w, cudaStream_t st);
+// Per-row bound of the bounded pass: the k-th largest group maximum (rows of
+// at most k candidates: 0).
+cudaError_t launch_prefill_threshold(int B, int rows_per_batch, int t0, int Tk, int q_pos0,
+                                     const int32_t* kv_len, int k, const RowWorkspace& w, cudaStream_t st);
+// Prefill rows per launch and workspace: the key slab, candidate positions,
+// group maxima and per-row bound and counter for B * rows rows.
+int prefill_rows_per_launch(int B, int Tq, int Tk_max, int k);
+size_t prefill_workspace_bytes(int rows, int Tk_max, int k);
+void carve_prefill_workspace(void* ws, int rows, int Tk_max, int k, RowWorkspace* out);
+// Rows whose candidates exceed this many use the two bounded passes.
+constexpr int kBoundedMinCand = 8192;
 
 // Attention.
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k);

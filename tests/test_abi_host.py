@@ -81,8 +81,10 @@ def test_workspace_sizes():
     assert 0 < small < big
     assert big % 256 == 0
     assert L.sa_index_score_topk_workspace(0, 1, 100, 64, 8) == 0
-    # prefill: a key slab of at most 512 MiB plus the fixed 1 MiB counter region
-    assert L.sa_index_score_topk_workspace(1, 65536, 65536, 64, 2048) <= (512 << 20) + (2 << 20)
+    # prefill: key and candidate-position slabs of at most 1 GiB, plus group
+    # maxima (2048 rows x 8224 16-bit entries) and per-row words
+    ws = L.sa_index_score_topk_workspace(1, 65536, 65536, 64, 2048)
+    assert (1 << 30) < ws <= (1 << 30) + (40 << 20)
     assert L.sa_sparse_attn_decode_workspace(8, 32, 8, 128, 2048) > 0
     assert L.sa_gist_route_unfold_workspace(4, 8192, 128, 64) > 0
 

@@ -121,6 +121,79 @@ def test_prefill_topk_matches_oracle(d, B, L, k, Tk, q_pos0):
     np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
 
 
+# Rows of more than 8192 candidates take two scoring passes: the first keeps
+# each group's maximum (groups of g = 1..128 positions, chosen per row), the
+# k-th largest group maximum bounds the k-th key from below, the second keeps
+# only the keys at or above the bound.
+
+@pytest.mark.parametrize("k", [4096, 2048, 1024, 512, 256, 128, 64, 32, 7])
+def test_prefill_topk_bounded_every_group_size(k):
+    """~9000-candidate rows: k from 4096 down to 7 gives groups of 1 to 128
+    positions; 200 rows span two row blocks with a ragged tail."""
+    B, L, d = 1, 200, 64
+    q_pos0 = 9000
+    Tk = q_pos0 + L
+    seed = 3100 + k
+    q = _ints(seed, 1, (B, L, d))
+    kk = _ints(seed, 2, (B, Tk, d))
+    idx, cnt, score = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0, with_scores=True)
+    ridx, rcnt = oracle.index_topk(q, kk, Tk, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    s = oracle.index_scores(q[0], kk[0])
+    got = score.cpu().numpy()[0]
+    for t in (0, 77, L - 1):
+        np.testing.assert_array_equal(got[t, :k], s[t, ridx[0, t]].astype(np.float32))
+
+
+def test_prefill_topk_bounded_mixed_row_lengths():
+    """One launch whose rows hold 3601..8200 candidates with k = 4096: rows
+    of at most k candidates take every one, the rest are bounded."""
+    B, L, d, k = 1, 4600, 64, 4096
+    q_pos0 = 3600
+    Tk = q_pos0 + L
+    q = _ints(3201, 1, (B, L, d))
+    kk = _ints(3201, 2, (B, Tk, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0)
+    ridx, rcnt = oracle.index_topk(q, kk, Tk, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
+@pytest.mark.parametrize("lo,hi", [(0, 0), (-1, 1)])
+def test_prefill_topk_bounded_ties(lo, hi):
+    """All-equal scores make every key a candidate (lists longer than shared
+    memory, read in place); scores in [-64, 64] tie heavily at the bound."""
+    B, L, d, k = 1, 130, 64, 2048
+    q_pos0 = 12000
+    Tk = q_pos0 + L
+    q = _ints(3301 + hi, 1, (B, L, d), lo, hi)
+    kk = _ints(3301 + hi, 2, (B, Tk, d), lo, hi)
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0)
+    ridx, rcnt = oracle.index_topk(q, kk, Tk, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
+def test_prefill_topk_bounded_per_sequence_lengths():
+    """Two sequences with cache lengths 20000 and 11000 in a 20480-row cache:
+    the second sequence's rows are capped by its length."""
+    B, L, d, k = 2, 150, 128, 1000
+    Tk_max, Tk, q_pos0 = 20480, 20000, 19850
+    q = _ints(3401, 1, (B, L, d))
+    kk = _ints(3401, 2, (B, Tk_max, d))
+    lens = np.array([20000, 11000], np.int32)
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0,
+                                      kv_len=torch.from_numpy(lens).to(dev()))
+    ridx, rcnt = oracle.index_topk(q, kk, lens, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
 def test_prefill_topk_real_valued_scores():
     """Non-integer bf16 inputs: the GPU's fp32 tile sums may differ from the
     fp64 oracle in the last bits, so compare sets via the oracle's scores:
