@@ -507,16 +507,28 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
         ws = torch.zeros(max(256, L.sa_index_score_topk_workspace(cfg.B, cfg.L, cfg.L, cfg.d, cfg.k)),
                          dtype=torch.uint8, device=dev)
         outs = [torch.empty_like(inp["q"][l]) for l in range(cfg.n_layers)]
+        part_ev = []   # (kind, start, stop) of the last step, when recording
 
-        def step(s):
+        def ev():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            return e
+
+        def step(s, record=False):
             cache.begin_step()
             for layer in range(cfg.n_layers):
                 if cache.is_full(layer) == 1:
                     g = layer // cfg.share_every
+                    a = ev() if record else None
                     cache.update(layer, inp["q_idx"][g], inp["k_idx"][g], ws=ws)
+                    if record:
+                        part_ev.append(("index", a, ev()))
                 idx, cnt, _ = cache.get_tensors(layer)
+                a = ev() if record else None
                 sa.sa_sparse_attn_prefill(inp["q"][layer], inp["K"][layer], inp["V"][layer], idx, cnt,
                                           out=outs[layer])
+                if record:
+                    part_ev.append(("attn", a, ev()))
         n_steps, unit, per = 1, "tokens/s", cfg.B * cfg.L
         nbytes = None
         launches = None
@@ -542,6 +554,32 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
                            "step_hbm_frac": round(nbytes / (ms / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     if launches:
         line["gpu_launches"] = launches * args.steps
+    if isinstance(cfg, R.Prefill):
+        # one more step with events around the indexer runs and the attention
+        # calls (after the timed region)
+        step(0, record=True)
+        torch.cuda.synchronize()
+        idx_ms = sum(a.elapsed_time(b) for kind, a, b in part_ev if kind == "index")
+        attn_ms = [a.elapsed_time(b) for kind, a, b in part_ev if kind == "attn"]
+        # causal (query, key) pairs per sequence, selected rows per sequence
+        pairs = cfg.L * (cfg.L + 1) // 2
+        sel = sum(min(cfg.k, t + 1) for t in range(cfg.L))
+        idx_flops = cfg.n_groups * cfg.B * pairs * 2 * cfg.d            # one scoring of every causal pair
+        attn_bytes = cfg.B * sel * cfg.Hkv * cfg.D * 2 * 2              # gathered K and V rows per layer
+        attn_gbs = attn_bytes / (statistics.mean(attn_ms) * 1e-3) / 1e9
+        idx_tf = idx_flops / (idx_ms * 1e-3) / 1e12
+        line["roofline"] = {"kernel": "attn_prefill_kernel (one layer's attention)", "bound": "hbm",
+                            "achieved": round(attn_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                            "peak_source": peaks["source"], "algorithmic_bytes_per_launch": attn_bytes,
+                            "note": "gathered rows are mostly L2 hits (one layer's K/V is about the L2 size)"}
+        line["indexer"] = {"ms_per_step": round(idx_ms, 4), "runs_per_step": cfg.n_groups,
+                           "algorithmic_gflop_per_step": round(idx_flops / 1e9, 2),
+                           "achieved_tflops": round(idx_tf, 1), "peak_tflops": peaks["bf16_tflops"],
+                           "frac_of_tensor_peak": round(idx_tf * 1e12 / (peaks["bf16_tflops"] * 1e12), 4),
+                           "what": "every causal pair scored once (2 d flops each) over the whole indexer "
+                                   "run: scoring passes, bound, selection and emission"}
+        line["attention_ms_per_layer"] = round(statistics.mean(attn_ms), 4)
     return line
 
 
