@@ -33,8 +33,10 @@
 //                 column of the row's pair array (a shared per-row counter
 //                 hands out the places), and the run's count goes to the
 //                 run's first tile slot.  A 32-bit mask per 32 columns finds
-//                 the takes; a chunk with any is stashed in shared memory so
-//                 the takes can be picked by index.
+//                 the takes (the sign of bound' - score, bound' the float
+//                 just below the bound, so one add decides "not below"); a
+//                 chunk with any is stashed in shared memory so the takes
+//                 can be picked by index.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -54,9 +56,11 @@ using namespace tc;
 constexpr int kBM = 128;   // query rows per block (TMEM lanes)
 constexpr int kBN = 256;   // key columns per MMA tile
 constexpr int kTmemCols = 512;
+// pipeline waits poll at most this many times, each poll sleeping up to kWaitNs
+constexpr uint32_t kWaitPolls = 1u << 20, kWaitNs = 2000;
 
 constexpr int kEpiKeys = 0, kEpiGroupMax = 1, kEpiCand = 2;
-constexpr int kStashFloats = 32;   // per thread: one 32-column chunk, 16-byte pieces XOR-swizzled by lane
+constexpr int kStashFloats = 36;   // per thread: one 32-column chunk (rows padded to 36 floats)
 
 template <int D, int EPI>
 struct TcShape {
@@ -106,11 +110,27 @@ struct TcParams {
   int* err;
 };
 
-// 0xFFFFFFFF when !(a < b) (a >= b, or either is NaN), else 0.
-__device__ __forceinline__ uint32_t set_geu(float a, float b) {
-  uint32_t r;
-  asm("set.geu.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+// Maximum of three (a NaN operand is ignored, as by fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Maximum of N consecutive values, as a chain of three-input maxima
+// (ceil((N - 1) / 2) instructions).
+template <int N>
+__device__ __forceinline__ float chain_max(const float* x) {
+  if constexpr (N == 1) {
+    return x[0];
+  } else {
+    float a = N == 2 ? fmaxf(x[0], x[1]) : fmax3(x[0], x[1], x[2]);
+    int i = N == 2 ? 2 : 3;
+#pragma unroll
+    for (; i + 1 < N; i += 2) a = fmax3(a, x[i], x[i + 1]);
+    if (i < N) a = fmaxf(a, x[i]);
+    return a;
+  }
 }
 
 // Order-preserving key for the group-maximum bound.  Unlike score_key it
@@ -229,7 +249,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           ++blk;
           const int ab = blk % S::kABuf;
           if (blk >= S::kABuf &&
-              !mbar_wait(&bars.aempty[ab], (uint32_t)((blk - S::kABuf) / S::kABuf) & 1u, abort_flag, p.err, 6))
+              !mbar_wait(&bars.aempty[ab], (uint32_t)((blk - S::kABuf) / S::kABuf) & 1u, abort_flag, p.err, 6, kWaitPolls, kWaitNs))
             break;
           mbar_arrive_expect_tx(&bars.afull[ab], S::kABytes);
 #pragma unroll
@@ -240,7 +260,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int i = (int)(u - lo);
         const int s = i % S::kStages;
         const uint32_t ph = (uint32_t)(i / S::kStages) & 1u;
-        if (!mbar_wait(&bars.empty[s], ph ^ 1u, abort_flag, p.err, 1)) break;
+        if (!mbar_wait(&bars.empty[s], ph ^ 1u, abort_flag, p.err, 1, kWaitPolls, kWaitNs)) break;
         mbar_arrive_expect_tx(&bars.full[s], S::kBBytes);
 #pragma unroll
         for (int a = 0; a < S::kAtoms; ++a)
@@ -258,7 +278,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       for (long long u = lo; u < hi; ++u, cur.next(p)) {
         if (u == lo || cur.tile == 0) {
           ++blk;
-          if (!mbar_wait(&bars.afull[blk % S::kABuf], (uint32_t)(blk / S::kABuf) & 1u, abort_flag, p.err, 2)) break;
+          if (!mbar_wait(&bars.afull[blk % S::kABuf], (uint32_t)(blk / S::kABuf) & 1u, abort_flag, p.err, 2, kWaitPolls, kWaitNs)) break;
           a_addr = smem_u32(sA + (blk % S::kABuf) * S::kABytes);
         }
         const int i = (int)(u - lo);
@@ -266,8 +286,8 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const uint32_t ph = (uint32_t)(i / S::kStages) & 1u;
         const int acc = i & 1;
         const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-        if (!mbar_wait(&bars.tempty[acc], aph ^ 1u, abort_flag, p.err, 3)) break;
-        if (!mbar_wait(&bars.full[s], ph, abort_flag, p.err, 4)) break;
+        if (!mbar_wait(&bars.tempty[acc], aph ^ 1u, abort_flag, p.err, 3, kWaitPolls, kWaitNs)) break;
+        if (!mbar_wait(&bars.full[s], ph, abort_flag, p.err, 4, kWaitPolls, kWaitNs)) break;
         tc_fence_after();
         const uint32_t b_addr = smem_u32(sB + s * S::kBBytes);
         const uint32_t d_tmem = tbase + (uint32_t)(acc * kBN);
@@ -307,13 +327,18 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         g = prefill_group_size(n, p.k);
         run_tile = cur.tile;   // the candidate run of this block starts at this tile
         ++run_idx;
-        // bound 0 (rows of at most k candidates) gives a NaN threshold: every key passes
-        if constexpr (EPI == kEpiCand) xth = n > 0 ? key_score(p.theta[rloc] << 16) : 0.f;
+        // xth: the float just below the bound, so a score s is kept when
+        // xth - s < 0 (sign bit set); bound 0 (rows of at most k candidates)
+        // keeps every finite score
+        if constexpr (EPI == kEpiCand) {
+          const uint32_t th = n > 0 ? p.theta[rloc] : 0u;
+          xth = th == 0u ? -INFINITY : nextafterf(key_score(th << 16), -INFINITY);
+        }
       }
       const int i = (int)(u - lo);
       const int acc = i & 1;
       const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-      if (!mbar_wait(&bars.tfull[acc], aph, abort_flag, p.err, 5)) break;
+      if (!mbar_wait(&bars.tfull[acc], aph, abort_flag, p.err, 5, kWaitPolls, kWaitNs)) break;
       tc_fence_after();
       const int cb = cur.tile * kBN + part * S::kPartCols;   // first column of this thread's part
       const uint32_t tcol = tbase + tlane + (uint32_t)(acc * kBN + part * S::kPartCols);
@@ -362,46 +387,42 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                   pack_key16(x[8 * q + 4], x[8 * q + 5]), pack_key16(x[8 * q + 6], x[8 * q + 7]));
             continue;
           }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = fmaxf(x[2 * j], x[2 * j + 1]);   // groups of 2
           if (g == 2) {
+            float y[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = fmaxf(x[2 * j], x[2 * j + 1]);
             uint4* dst = reinterpret_cast<uint4*>(gm + c / 2);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack_key16(x[8 * q + 0], x[8 * q + 1]), pack_key16(x[8 * q + 2], x[8 * q + 3]),
-                                  pack_key16(x[8 * q + 4], x[8 * q + 5]), pack_key16(x[8 * q + 6], x[8 * q + 7]));
-            continue;
-          }
+              dst[q] = make_uint4(pack_key16(y[8 * q + 0], y[8 * q + 1]), pack_key16(y[8 * q + 2], y[8 * q + 3]),
+                                  pack_key16(y[8 * q + 4], y[8 * q + 5]), pack_key16(y[8 * q + 6], y[8 * q + 7]));
+          } else if (g == 4) {
+            float y[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) x[j] = fmaxf(x[2 * j], x[2 * j + 1]);   // 4
-          if (g == 4) {
+            for (int j = 0; j < 16; ++j) y[j] = chain_max<4>(x + 4 * j);
             uint4* dst = reinterpret_cast<uint4*>(gm + c / 4);
 #pragma unroll
             for (int q = 0; q < 2; ++q)
-              dst[q] = make_uint4(pack_key16(x[8 * q + 0], x[8 * q + 1]), pack_key16(x[8 * q + 2], x[8 * q + 3]),
-                                  pack_key16(x[8 * q + 4], x[8 * q + 5]), pack_key16(x[8 * q + 6], x[8 * q + 7]));
-            continue;
-          }
+              dst[q] = make_uint4(pack_key16(y[8 * q + 0], y[8 * q + 1]), pack_key16(y[8 * q + 2], y[8 * q + 3]),
+                                  pack_key16(y[8 * q + 4], y[8 * q + 5]), pack_key16(y[8 * q + 6], y[8 * q + 7]));
+          } else if (g == 8) {
+            float y[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) x[j] = fmaxf(x[2 * j], x[2 * j + 1]);   // 8
-          if (g == 8) {
+            for (int j = 0; j < 8; ++j) y[j] = chain_max<8>(x + 8 * j);
             *reinterpret_cast<uint4*>(gm + c / 8) =
-                make_uint4(pack_key16(x[0], x[1]), pack_key16(x[2], x[3]), pack_key16(x[4], x[5]), pack_key16(x[6], x[7]));
-            continue;
-          }
+                make_uint4(pack_key16(y[0], y[1]), pack_key16(y[2], y[3]), pack_key16(y[4], y[5]), pack_key16(y[6], y[7]));
+          } else {
+            float y[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) x[j] = fmaxf(x[2 * j], x[2 * j + 1]);   // 16
-          if (g == 16) {
-            *reinterpret_cast<uint2*>(gm + c / 16) = make_uint2(pack_key16(x[0], x[1]), pack_key16(x[2], x[3]));
-            continue;
+            for (int j = 0; j < 4; ++j) y[j] = chain_max<16>(x + 16 * j);
+            if (g == 16) {
+              *reinterpret_cast<uint2*>(gm + c / 16) = make_uint2(pack_key16(y[0], y[1]), pack_key16(y[2], y[3]));
+            } else if (g == 32) {
+              *reinterpret_cast<uint32_t*>(gm + c / 32) = pack_key16(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+            } else {   // 64
+              gm[c / 64] = (uint16_t)(bound_key(fmax3(y[0], y[1], fmaxf(y[2], y[3]))) >> 16);
+            }
           }
-          x[0] = fmaxf(x[0], x[1]);   // 32
-          x[1] = fmaxf(x[2], x[3]);
-          if (g == 32) {
-            *reinterpret_cast<uint32_t*>(gm + c / 32) = pack_key16(x[0], x[1]);
-            continue;
-          }
-          gm[c / 64] = (uint16_t)(bound_key(fmaxf(x[0], x[1])) >> 16);   // 64
         }
       } else {
         uint2* run = reinterpret_cast<uint2*>(p.keys) + rloc * p.ld + (long long)run_tile * kBN;
@@ -409,7 +430,6 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         float* stash = reinterpret_cast<float*>(base + S::kABuf * S::kABytes + S::kStages * S::kBBytes +
                                                 S::kBarBytes + S::kCntBytes) +
                        ((warp - 2) * 32 + lane) * kStashFloats;
-        const int sw = lane & 7;   // 16-byte piece q of this thread's stash sits at q ^ sw
 #pragma unroll 1
         for (int cc = 0; cc < S::kPartCols; cc += 64) {
           const int c0 = cb + cc;
@@ -421,22 +441,27 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int c = c0 + 32 * h;
-            // bit (31 - j) of m marks column c + j as a take
-            uint32_t m = 0u;
+            // bit (31 - j) of m marks column c + j as a take: the sign bit of
+            // xth - score (four independent 8-column chains, joined)
+            uint32_t mq[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) m = __funnelshift_l(set_geu(__uint_as_float(v[32 * h + j]), xth), m, 1);
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                mq[q] = __funnelshift_l(__float_as_uint(xth - __uint_as_float(v[32 * h + 8 * q + j])), mq[q], 1);
+            uint32_t m = mq[0] << 24 | mq[1] << 16 | mq[2] << 8 | mq[3];
             const int valid = n - c;
             m = valid >= 32 ? m : (valid > 0 ? m & (~0u << (32 - valid)) : 0u);
             if (m) {
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4)
-                *reinterpret_cast<uint4*>(stash + 4 * (q4 ^ sw)) =
+                *reinterpret_cast<uint4*>(stash + 4 * q4) =
                     make_uint4(v[32 * h + 4 * q4], v[32 * h + 4 * q4 + 1], v[32 * h + 4 * q4 + 2], v[32 * h + 4 * q4 + 3]);
               uint2* dst = run + atomicAdd(cnt, (uint32_t)__popc(m));
               while (m) {
                 const int j = __clz(m);
                 m &= ~(0x80000000u >> j);
-                *dst++ = make_uint2(__float_as_uint(stash[4 * ((j >> 2) ^ sw) + (j & 3)]), (uint32_t)(c + j));
+                *dst++ = make_uint2(__float_as_uint(stash[j]), (uint32_t)(c + j));
               }
             }
           }

@@ -950,7 +950,7 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   if (K > 0) {
     SelStart st;
     if (!from_hist) {
-      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24, false};
+      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24, bits_known};
     } else {
       // the histogram already fixes the top 12 bits: every item above the
       // bin is chosen, K - above of the bin's items remain to pick

@@ -52,13 +52,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete may sleep up
+// to about `hint_ns` nanoseconds (it wakes when the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete.  On timeout sets
 // *flag (shared abort word) and `err_code` in the global error word, and
-// returns false.
+// returns false.  With sleep_ns > 0 each poll may sleep that long, so a
+// waiting warp leaves its scheduler's issue slots to the others.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* gerr, int err_code, uint32_t limit = kSpinLimit) {
+                                          int* gerr, int err_code, uint32_t limit = kSpinLimit,
+                                          uint32_t sleep_ns = 0) {
   for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (sleep_ns ? mbar_try_wait_hint(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
   }
   *abort_flag = 1;
