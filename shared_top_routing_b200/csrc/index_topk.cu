@@ -76,7 +76,7 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
   pdl_wait();
   pdl_launch_dependents();
   constexpr int J = D / 32;          // 16-byte chunks per lane per key row
-  constexpr int U = 4;               // 8-row tiles per warp iteration
+  constexpr int U = 2;               // 8-row tiles per register buffer (two buffers)
   constexpr int WARPS = kScoreThreads / 32;
   __shared__ uint32_t sh[kHistBins];
 
@@ -113,8 +113,10 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     }
     const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
     uint32_t* kout = keys + (long long)b * ld;
-    for (int base = r0 + warp * 8 * U; base < r1; base += WARPS * 8 * U) {
-      uint4 v[U][J];
+    // Two register buffers of U 8-row tiles: the next buffer's loads are in
+    // flight while the current one is scored, so each warp keeps memory busy
+    // instead of alternating a burst of loads with compute.
+    auto load = [&](uint4 (&v)[U][J], int base) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int row = base + u * 8 + g;
@@ -122,6 +124,8 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
         for (int j = 0; j < J; ++j)
           v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
       }
+    };
+    auto score = [&](const uint4 (&v)[U][J], int base) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -144,6 +148,17 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
           }
         }
       }
+    };
+    constexpr int kStep = WARPS * 8 * U;
+    uint4 va[U][J], vb[U][J];
+    int base = r0 + warp * 8 * U;
+    if (base < r1) load(va, base);
+    for (; base < r1; base += 2 * kStep) {
+      if (base + kStep < r1) load(vb, base + kStep);
+      score(va, base);
+      if (base + kStep >= r1) break;
+      if (base + 2 * kStep < r1) load(va, base + 2 * kStep);
+      score(vb, base + kStep);
     }
     if (hist != nullptr) {
       __syncthreads();
@@ -350,14 +365,12 @@ __device__ __forceinline__ void find_digit(Sm& s, uint32_t kk, bool desc) {
 }
 
 // Items: keys with explicit positions, or a row of keys (position = index).
-// (stride 2: keys and positions interleaved as (key, position) pairs)
 struct Items {
   const uint32_t* key;
   const uint32_t* pos;
   int n;
-  int stride = 1;
-  __device__ __forceinline__ uint32_t k(int i) const { return key[(long long)i * stride]; }
-  __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[(long long)i * stride] : (uint32_t)i; }
+  __device__ __forceinline__ uint32_t k(int i) const { return key[i]; }
+  __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i] : (uint32_t)i; }
 };
 
 // Where the search for the K-th key starts: the bits of its key already
@@ -680,13 +693,15 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
   bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
     if (mode == kFinishCandRows) {
-      // the bounded pass's takes, (score bits, position) pairs: each scoring
-      // CTA left its run of this row at the run's first column, the run's
-      // count in that tile's slot (0 in the run's other slots).  Counts are
-      // clamped to the columns left, so every read stays in the row.  Slots
-      // are taken kFinThreads at a time; each warp copies its lanes' runs
-      // with all 32 lanes.
-      uint2* cr = reinterpret_cast<uint2*>(w.keys) + (long long)r * w.ld;
+      // the bounded pass's takes: score bits in the first half of the row's
+      // 2 * ld words, positions in the second.  Each scoring CTA left its run
+      // of this row at the run's first column, the run's count in that
+      // tile's slot (0 in the run's other slots).  Counts are clamped to the
+      // columns left, so every read stays in the row.  Slots are taken
+      // kFinThreads at a time; each warp copies its lanes' runs with all 32
+      // lanes.
+      uint32_t* ck = w.keys + (long long)r * 2 * w.ld;
+      uint32_t* cp = ck + w.ld;
       const uint32_t* tcnt = w.tile_cnt + (long long)r * (w.ld / 256);
       const int nslot = (n + 255) / 256;
       auto slot_count = [&](int sl) { return sl < nslot ? min(tcnt[sl], (uint32_t)(n - sl * 256)) : 0u; };
@@ -713,14 +728,13 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
             const uint32_t oL = __shfl_sync(0xffffffffu, o, L);
             const long long from = (long long)__shfl_sync(0xffffffffu, sl, L) * 256;
             for (uint32_t j = (uint32_t)(tid & 31); j < cL; j += 32) {
-              const uint2 e = cr[from + j];
-              const uint32_t key = score_key(__uint_as_float(e.x));
+              const uint32_t key = score_key(__uint_as_float(ck[from + j])), pos = cp[from + j];
               s.ckey[oL + j] = key;
-              s.cpos[oL + j] = e.y;
+              s.cpos[oL + j] = pos;
               ko |= key;
               ka &= key;
-              po |= e.y;
-              pa &= e.y;
+              po |= pos;
+              pa &= pos;
             }
           }
         }
@@ -754,17 +768,22 @@ finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int 
           const uint32_t c = slot_count(sl);
           for (uint32_t j0 = 0; j0 < c; j0 += kFinThreads) {
             const uint32_t j = j0 + tid;
-            uint2 e = make_uint2(0u, 0u);
-            if (j < c) e = cr[(long long)sl * 256 + j];
+            uint32_t key = 0u, pos = 0u;
+            if (j < c) {
+              key = ck[(long long)sl * 256 + j];
+              pos = cp[(long long)sl * 256 + j];
+            }
             __syncthreads();
-            if (j < c) cr[dst + j] = make_uint2(score_key(__uint_as_float(e.x)), e.y);
+            if (j < c) {
+              ck[dst + j] = score_key(__uint_as_float(key));
+              cp[dst + j] = pos;
+            }
             __syncthreads();
           }
           dst += c;
         }
-        it.key = reinterpret_cast<const uint32_t*>(cr);
-        it.pos = reinterpret_cast<const uint32_t*>(cr) + 1;
-        it.stride = 2;
+        it.key = ck;
+        it.pos = cp;
         it.n = (int)total;
       }
       __syncthreads();
@@ -1219,8 +1238,9 @@ int finish_mode_for(int Tk_max, bool* need_collect) {
 // Prefill layout: [error word][keys: rows x ld][second slab: rows x ld]
 // [group maxima: rows x ld2 (16-bit)][bound: rows][run counts: rows x
 // ld/256].  Short batches use only the key slab; long ones use both slabs as
-// one [rows][ld] array of (score bits, position) pairs for the bounded
-// pass's takes (each scoring CTA's run of a row at the run's first column).
+// [rows][2 ld] words for the bounded pass's takes: score bits in the first
+// ld, positions in the second (each scoring CTA's run of a row at the run's
+// first column).
 size_t prefill_workspace_bytes(int rows, int Tk_max, int k) {
   const long long ld = row_ld(Tk_max);
   const long long ld2 = prefill_groups_ld(Tk_max, k);
