@@ -659,12 +659,15 @@ prefill_threshold_kernel(const uint16_t* __restrict__ gmax, long long ld2, int r
   if (tid == 0) theta[r] = hi << 8 | s.digit;
 }
 
-template <class Sm, int THREADS>
+// One instance per (layout, candidate source): each holds only its own
+// path, which keeps the instruction footprint of the hot instances small.
+template <class Sm, int THREADS, int MODE>
 __global__ void __launch_bounds__(THREADS, THREADS >= 1024 ? 1 : 4)
-finish_kernel(RowWorkspace w, int mode, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
               const int32_t* __restrict__ kv_len, int k, FinishOut out) {
   pdl_wait();
   pdl_launch_dependents();
+  constexpr int mode = MODE;
   constexpr int kFinThreads = THREADS;
   constexpr int kSmemCand = Sm::kCand;
   constexpr int kBitmapWords = Sm::kBmw;
@@ -1202,26 +1205,25 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
   // the longest row of the launch decides the layout: direct rows of at most
   // 2048 candidates take the small one (256 threads, several rows per SM)
   const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + t0 + rows_per_batch);
+  auto go = [&](auto kern, size_t smem, int threads) {
+    cudaError_t e = ensure_dynamic_smem((const void*)kern, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(rows), dim3(threads), smem, st, w, rows_per_batch, t0, Tq, Tk, q_pos0, kv_len, k,
+                      out);
+  };
   cudaError_t e;
-  if (mode == kFinishDirect && n_max <= FinishSmemSmall::kCand) {
-    const size_t smem = sizeof(FinishSmemSmall);
-    auto kern = finish_kernel<FinishSmemSmall, kFinThreadsSmall>;
-    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(rows), dim3(kFinThreadsSmall), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
-                   kv_len, k, out);
-  } else if (mode == kFinishCandRows && n_max <= FinishSmemMed::kBmw * 32) {
-    const size_t smem = sizeof(FinishSmemMed);
-    auto kern = finish_kernel<FinishSmemMed, kFinThreadsSmall>;
-    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(rows), dim3(kFinThreadsSmall), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
-                   kv_len, k, out);
-  } else {
-    const size_t smem = sizeof(FinishSmem);
-    auto kern = finish_kernel<FinishSmem, kFinThreads>;
-    if ((e = ensure_dynamic_smem((const void*)kern, smem)) != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(rows), dim3(kFinThreads), smem, st, w, mode, rows_per_batch, t0, Tq, Tk, q_pos0,
-                   kv_len, k, out);
-  }
+  if (mode == kFinishDirect && n_max <= FinishSmemSmall::kCand)
+    e = go(finish_kernel<FinishSmemSmall, kFinThreadsSmall, kFinishDirect>, sizeof(FinishSmemSmall), kFinThreadsSmall);
+  else if (mode == kFinishCandRows && n_max <= FinishSmemMed::kBmw * 32)
+    e = go(finish_kernel<FinishSmemMed, kFinThreadsSmall, kFinishCandRows>, sizeof(FinishSmemMed), kFinThreadsSmall);
+  else if (mode == kFinishDirect)
+    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishDirect>, sizeof(FinishSmem), kFinThreads);
+  else if (mode == kFinishHistScan)
+    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishHistScan>, sizeof(FinishSmem), kFinThreads);
+  else if (mode == kFinishCandList)
+    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishCandList>, sizeof(FinishSmem), kFinThreads);
+  else
+    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishCandRows>, sizeof(FinishSmem), kFinThreads);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
