@@ -290,7 +290,7 @@ class DecodeBench:
 # DRAM bytes (read + write) per decode attention call, split + merge kernels,
 # from the ncu capture summarised in profiles/attn_decode_b8_32k.md.  Must be
 # re-measured (or removed) whenever either kernel changes.
-MEASURED_TRAFFIC = {"decode_b8_32k_4layers": 67_306_752 + 1_240_064 + 2_549_760}
+MEASURED_TRAFFIC = {"decode_b8_32k_4layers": 67_303_680 + 1_033_984 + 2_554_880}
 
 
 def run_native(args, cfg, rank, world):
