@@ -183,14 +183,22 @@ class DecodeBench:
         seed_cfg = R.Decode(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
         self.inp = TI.decode_inputs(seed_cfg, device)
         c = cfg
+        # all layers' K and V caches as slices of one [layers, 2, B, Tk_max, Hkv, D]
+        # array, so a step's appended rows of every layer are one strided copy
+        self.kv_all = torch.empty((c.n_layers, 2, c.B, c.Tk_max, c.Hkv, c.D), dtype=torch.bfloat16, device=device)
+        for l in range(c.n_layers):
+            self.kv_all[l, 0].copy_(self.inp["K"][l])
+            self.kv_all[l, 1].copy_(self.inp["V"][l])
+            self.inp["K"][l], self.inp["V"][l] = self.kv_all[l, 0], self.kv_all[l, 1]
+        torch.cuda.empty_cache()
         self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
         L = sa.lib()
         self.ws_idx = torch.zeros(L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k),
                                   dtype=torch.uint8, device=device)
         self.ws_attn = torch.zeros(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
                                    dtype=torch.uint8, device=device)
-        self.out = [torch.empty((c.B, c.Hq, c.D), dtype=torch.bfloat16, device=device)
-                    for _ in range(c.n_layers)]
+        self.out_all = torch.empty((c.n_layers, c.B, c.Hq, c.D), dtype=torch.bfloat16, device=device)
+        self.out = [self.out_all[l] for l in range(c.n_layers)]
         self.graphs = {}
         self.events = {}
         # kernels per indexer run: score + finish, plus collect for rows longer
@@ -394,45 +402,48 @@ def run_native(args, cfg, rank, world):
 def run_e2e(b, args, dev, world):
     """Same steps through the public API with host buffers: every step copies
     its queries and the appended token's cache rows from pinned host memory
-    (one cudaMemcpyAsync / cudaMemcpy2DAsync per tensor), runs the step, and
-    copies every layer's output back to pinned host memory."""
+    and every layer's output back to pinned host memory.  The caches, queries
+    and outputs of all layers are slices of one array each, so a step takes
+    one copy for all layers' queries, one strided copy for all layers'
+    appended K/V rows, one per indexer group for its query and key row, and
+    one for all outputs."""
     import torch
     c = b.cfg
     rt = b.rt
     n_steps = c.steps
     st = b.stream
     pin = lambda t: t.contiguous().cpu().pin_memory()
+    L, B = c.n_layers, c.B
     host = {}
     for s in range(n_steps):
         pos = c.N + s
         host[s] = {"q_idx": {g: pin(b.inp["q_idx"][g][s]) for g in b.inp["q_idx"]},
                    "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
-                   "q": {l: pin(b.inp["q"][l][s]) for l in b.inp["q"]},
-                   "K_row": {l: pin(b.inp["K"][l][:, pos]) for l in b.inp["K"]},
-                   "V_row": {l: pin(b.inp["V"][l][:, pos]) for l in b.inp["V"]}}
-    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in b.out]
-    h2d = sum(t.numel() * t.element_size() for v in host[0].values() for t in v.values())
-    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+                   "q": pin(torch.stack([b.inp["q"][l][s] for l in range(L)])),
+                   # rows (layer, K/V, sequence) in the order of b.kv_all
+                   "kv_row": pin(b.kv_all[:, :, :, pos].reshape(L * 2 * B, -1))}
+    out_h = torch.empty(b.out_all.shape, dtype=b.out_all.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host[0]["q_idx"].values()) + \
+        sum(t.numel() * t.element_size() for t in host[0]["k_row"].values()) + \
+        host[0]["q"].numel() * 2 + host[0]["kv_row"].numel() * 2
+    d2h = out_h.numel() * out_h.element_size()
     qi_dev = {g: torch.empty_like(b.inp["q_idx"][g][0]) for g in b.inp["q_idx"]}
-    q_dev = {l: torch.empty_like(b.inp["q"][l][0]) for l in b.inp["q"]}
+    q_all = torch.empty((L,) + tuple(b.inp["q"][0][0].shape), dtype=torch.bfloat16, device=dev)
 
-    def row_copy(cache, src, pos):
-        # cache [B, Tk_max, ...]: B blocks of one row each, pitch = one sequence
+    def row_copy(cache, src, pos, rows):
+        # rows of one cache position, one per block of `pitch` bytes
         row_bytes = src[0].numel() * src.element_size()
-        pitch = cache[0].numel() * cache.element_size()
-        rt.h2d_2d(cache.data_ptr() + pos * row_bytes, pitch, src.data_ptr(), row_bytes, row_bytes,
-                  src.shape[0], st)
+        pitch = cache.shape[-3] * row_bytes if cache.dim() > 3 else cache[0].numel() * cache.element_size()
+        rt.h2d_2d(cache.data_ptr() + pos * row_bytes, pitch, src.data_ptr(), row_bytes, row_bytes, rows, st)
 
     def e2e_step(s):
         h = host[s]
         pos = c.N + s
         for g in h["q_idx"]:
             rt.h2d(qi_dev[g].data_ptr(), h["q_idx"][g].data_ptr(), h["q_idx"][g].numel() * 2, st)
-            row_copy(b.inp["k_idx"][g], h["k_row"][g], pos)
-        for l in h["q"]:
-            rt.h2d(q_dev[l].data_ptr(), h["q"][l].data_ptr(), h["q"][l].numel() * 2, st)
-            row_copy(b.inp["K"][l], h["K_row"][l], pos)
-            row_copy(b.inp["V"][l], h["V_row"][l], pos)
+            row_copy(b.inp["k_idx"][g], h["k_row"][g], pos, B)
+        rt.h2d(q_all.data_ptr(), h["q"].data_ptr(), h["q"].numel() * 2, st)
+        row_copy(b.kv_all, h["kv_row"], pos, L * 2 * B)
         Tk = pos + 1
         b.cache.begin_step()
         for layer in range(c.n_layers):
@@ -440,10 +451,9 @@ def run_e2e(b, args, dev, world):
                 g = layer // c.share_every
                 b.cache.update(layer, qi_dev[g], b.inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=b.ws_idx)
             idx, cnt, _ = b.cache.get_tensors(layer)
-            b.sa.sa_sparse_attn_decode(q_dev[layer], b.inp["K"][layer], b.inp["V"][layer],
+            b.sa.sa_sparse_attn_decode(q_all[layer], b.inp["K"][layer], b.inp["V"][layer],
                                        idx.view(c.B, c.k), cnt.view(c.B), out=b.out[layer], ws=b.ws_attn)
-        for l, o in enumerate(b.out):
-            rt.d2h(outs_h[l].data_ptr(), o.data_ptr(), o.numel() * o.element_size(), st)
+        rt.d2h(out_h.data_ptr(), b.out_all.data_ptr(), out_h.numel() * out_h.element_size(), st)
 
     with torch.cuda.stream(st):
         for s in range(n_steps):
@@ -472,8 +482,9 @@ def run_e2e(b, args, dev, world):
         ms = float(t.item())
     return {"value": round(world * args.steps / (ms / 1e3), 2), "unit": "steps/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "how": "per-step CUDA graph: H2D of queries + appended cache rows from pinned memory, "
-                   "index + attention calls, D2H of every layer's output"}
+            "how": "per-step CUDA graph: H2D of queries + appended cache rows from pinned memory "
+                   "(all layers' queries in one copy, all layers' K/V rows in one strided copy), "
+                   "index + attention calls, D2H of every layer's output (one copy)"}
 
 
 # ------------------------------------------------------------ other configs
