@@ -27,13 +27,12 @@
 //                 16-bit truncated key (the top half of the 32-bit key,
 //                 which never exceeds the group's largest key).
 //   kEpiCand      as kEpiGroupMax; per row, every score at or above the
-//                 row's bound (from the group maxima) is kept: its score
-//                 bits in the first half of the row's 2 * ld words, its
-//                 position at the same place in the second half.  A CTA's
-//                 tiles of one row block form a run; its takes of a row are
-//                 appended at the run's first column (a shared per-row
-//                 counter hands out the places), and the run's count goes to
-//                 the run's first tile slot.  A 32-bit mask per 32 columns finds
+//                 row's bound (from the group maxima) is kept as a (score
+//                 bits, position) pair.  A CTA's tiles of one row block form
+//                 a run; its takes of a row are appended at the run's first
+//                 column of the row's pair array (a shared per-row counter
+//                 hands out the places, one 8-byte store per take), and the
+//                 run's count goes to the run's first tile slot.  A 32-bit mask per 32 columns finds
 //                 the takes (the sign of bound' - score, bound' the float
 //                 just below the bound, so one add decides "not below"); a
 //                 chunk with any is stashed in shared memory so the takes
@@ -102,7 +101,7 @@ struct TcParams {
   const int32_t* kv_len;
   int t0, rows, nblk, B;
   long long tiles_per_seq;   // key tiles of all row blocks of one sequence
-  uint32_t* keys;          // kEpiKeys: [rows][ld] slab; kEpiCand: [rows][2 ld] score bits, then positions
+  uint32_t* keys;          // kEpiKeys: [rows][ld] slab; kEpiCand: [rows][ld] (score bits, position) pairs
   long long ld;
   uint32_t* tile_cnt;      // kEpiCand: [rows][ld / kBN] takes of the run starting at each tile
   const uint32_t* theta;   // kEpiCand: [rows] 16-bit bound of each row
@@ -426,7 +425,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           }
         }
       } else {
-        uint32_t* run = p.keys + rloc * 2 * p.ld + (long long)run_tile * kBN;   // scores; positions at + ld
+        uint2* run = reinterpret_cast<uint2*>(p.keys) + rloc * p.ld + (long long)run_tile * kBN;
         uint32_t* cnt = s_cnt + (run_idx & 1) * kBM + r;
         float* stash = reinterpret_cast<float*>(base + S::kABuf * S::kABytes + S::kStages * S::kBBytes +
                                                 S::kBarBytes + S::kCntBytes) +
@@ -458,13 +457,11 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
               for (int q4 = 0; q4 < 8; ++q4)
                 *reinterpret_cast<uint4*>(stash + 4 * q4) =
                     make_uint4(v[32 * h + 4 * q4], v[32 * h + 4 * q4 + 1], v[32 * h + 4 * q4 + 2], v[32 * h + 4 * q4 + 3]);
-              uint32_t* dst = run + atomicAdd(cnt, (uint32_t)__popc(m));
+              uint2* dst = run + atomicAdd(cnt, (uint32_t)__popc(m));
               while (m) {
                 const int j = __clz(m);
                 m &= ~(0x80000000u >> j);
-                dst[0] = __float_as_uint(stash[j]);
-                dst[p.ld] = (uint32_t)(c + j);
-                ++dst;
+                *dst++ = make_uint2(__float_as_uint(stash[j]), (uint32_t)(c + j));
               }
             }
           }

@@ -36,6 +36,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -373,6 +374,17 @@ struct Items {
   __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i] : (uint32_t)i; }
 };
 
+// The same, for sources that may also hand over (key, position) pairs in
+// global memory (shift 1: element i at word 2 i).
+struct PairItems {
+  const uint32_t* key;
+  const uint32_t* pos;
+  int n;
+  int shift = 0;
+  __device__ __forceinline__ uint32_t k(int i) const { return key[i << shift]; }
+  __device__ __forceinline__ uint32_t p(int i) const { return pos ? pos[i << shift] : (uint32_t)i; }
+};
+
 // Where the search for the K-th key starts: the bits of its key already
 // known (prefix under pmask), how many items still to choose inside that
 // prefix (kk), how many items share it (bnd), and the first digit's shift.
@@ -389,8 +401,8 @@ struct SelStart {
 // (from the OR / AND of all keys, or of all positions) is settled without
 // a pass -- integer-valued scores leave most low mantissa bits zero, and
 // positions below 2^16 leave the high bits zero.
-template <class Sm, int THREADS>
-__device__ void select_threshold(Sm& s, const Items& it, SelStart st, uint32_t& prefix, uint32_t& pmask,
+template <class Sm, int THREADS, class It>
+__device__ void select_threshold(Sm& s, const It& it, SelStart st, uint32_t& prefix, uint32_t& pmask,
                                  uint32_t& pmax) {
   const int tid = threadIdx.x;
   if (!st.bits_known) {
@@ -686,7 +698,7 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
   __syncthreads();
 
   // ---- gather candidates into shared memory
-  Items it;
+  std::conditional_t<MODE == kFinishCandRows, PairItems, Items> it;
   it.key = row;
   it.pos = nullptr;
   it.n = n;
@@ -696,15 +708,13 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
   bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
     if (mode == kFinishCandRows) {
-      // the bounded pass's takes: score bits in the first half of the row's
-      // 2 * ld words, positions in the second.  Each scoring CTA left its run
-      // of this row at the run's first column, the run's count in that
-      // tile's slot (0 in the run's other slots).  Counts are clamped to the
-      // columns left, so every read stays in the row.  Slots are taken
-      // kFinThreads at a time; each warp copies its lanes' runs with all 32
-      // lanes.
-      uint32_t* ck = w.keys + (long long)r * 2 * w.ld;
-      uint32_t* cp = ck + w.ld;
+      // the bounded pass's takes, (score bits, position) pairs: each scoring
+      // CTA left its run of this row at the run's first column, the run's
+      // count in that tile's slot (0 in the run's other slots).  Counts are
+      // clamped to the columns left, so every read stays in the row.  Slots
+      // are taken kFinThreads at a time; each warp copies its lanes' runs
+      // with all 32 lanes.
+      uint2* cr = reinterpret_cast<uint2*>(w.keys) + (long long)r * w.ld;
       const uint32_t* tcnt = w.tile_cnt + (long long)r * (w.ld / 256);
       const int nslot = (n + 255) / 256;
       auto slot_count = [&](int sl) { return sl < nslot ? min(tcnt[sl], (uint32_t)(n - sl * 256)) : 0u; };
@@ -731,13 +741,14 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
             const uint32_t oL = __shfl_sync(0xffffffffu, o, L);
             const long long from = (long long)__shfl_sync(0xffffffffu, sl, L) * 256;
             for (uint32_t j = (uint32_t)(tid & 31); j < cL; j += 32) {
-              const uint32_t key = score_key(__uint_as_float(ck[from + j])), pos = cp[from + j];
+              const uint2 e = cr[from + j];
+              const uint32_t key = score_key(__uint_as_float(e.x));
               s.ckey[oL + j] = key;
-              s.cpos[oL + j] = pos;
+              s.cpos[oL + j] = e.y;
               ko |= key;
               ka &= key;
-              po |= pos;
-              pa &= pos;
+              po |= e.y;
+              pa &= e.y;
             }
           }
         }
@@ -771,22 +782,19 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
           const uint32_t c = slot_count(sl);
           for (uint32_t j0 = 0; j0 < c; j0 += kFinThreads) {
             const uint32_t j = j0 + tid;
-            uint32_t key = 0u, pos = 0u;
-            if (j < c) {
-              key = ck[(long long)sl * 256 + j];
-              pos = cp[(long long)sl * 256 + j];
-            }
+            uint2 e = make_uint2(0u, 0u);
+            if (j < c) e = cr[(long long)sl * 256 + j];
             __syncthreads();
-            if (j < c) {
-              ck[dst + j] = score_key(__uint_as_float(key));
-              cp[dst + j] = pos;
-            }
+            if (j < c) cr[dst + j] = make_uint2(score_key(__uint_as_float(e.x)), e.y);
             __syncthreads();
           }
           dst += c;
         }
-        it.key = ck;
-        it.pos = cp;
+        if constexpr (MODE == kFinishCandRows) {
+          it.key = reinterpret_cast<const uint32_t*>(cr);
+          it.pos = reinterpret_cast<const uint32_t*>(cr) + 1;
+          it.shift = 1;
+        }
         it.n = (int)total;
       }
       __syncthreads();
@@ -1240,9 +1248,8 @@ int finish_mode_for(int Tk_max, bool* need_collect) {
 // Prefill layout: [error word][keys: rows x ld][second slab: rows x ld]
 // [group maxima: rows x ld2 (16-bit)][bound: rows][run counts: rows x
 // ld/256].  Short batches use only the key slab; long ones use both slabs as
-// [rows][2 ld] words for the bounded pass's takes: score bits in the first
-// ld, positions in the second (each scoring CTA's run of a row at the run's
-// first column).
+// one [rows][ld] array of (score bits, position) pairs for the bounded
+// pass's takes (each scoring CTA's run of a row at the run's first column).
 size_t prefill_workspace_bytes(int rows, int Tk_max, int k) {
   const long long ld = row_ld(Tk_max);
   const long long ld2 = prefill_groups_ld(Tk_max, k);
