@@ -466,7 +466,34 @@ __device__ void select_threshold(Sm& s, const It& it, SelStart st, uint32_t& pre
   }
   pmax = 0xFFFFFFFFu;
   if (bnd == kk) return;
-  // exact key ties: keep the kk lowest positions among key == prefix
+  // exact key ties: keep the kk lowest positions among the bnd items with
+  // key == prefix.  A small tie group is gathered once and the kk-th lowest
+  // position found by counting, for each, the tied positions below it
+  // (positions are distinct); larger groups take radix passes over positions.
+  constexpr uint32_t kTieList = Sm::kBmw < 256 ? Sm::kBmw : 256;
+  if (bnd <= kTieList) {
+    uint32_t* list = s.bits;   // free until the emission
+    if (tid == 0) s.hist[0] = 0u;
+    __syncthreads();
+    for (int i = tid; i < it.n; i += THREADS) {
+      if (it.k(i) == prefix) {
+        const uint32_t slot = atomicAdd(&s.hist[0], 1u);
+        if (slot < kTieList) list[slot] = it.p(i);
+      }
+    }
+    __syncthreads();
+    const uint32_t m = min(s.hist[0], kTieList);   // == bnd
+    for (uint32_t i = tid; i < m; i += THREADS) {
+      const uint32_t p = list[i];
+      uint32_t below = 0;
+      for (uint32_t j = 0; j < m; ++j) below += list[j] < p ? 1u : 0u;
+      if (below == kk - 1) s.hist[1] = p;
+    }
+    __syncthreads();
+    pmax = s.hist[1];
+    __syncthreads();
+    return;
+  }
   uint32_t pp = 0, pm = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
     const uint32_t wmask = 255u << shift;
