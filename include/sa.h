@@ -93,7 +93,9 @@ int sa_version(void);
  * fp32 score in the same slots (NaN-free padding value: -inf).
  *
  *   q_idx      [B, Tq, d]      bf16
- *   k_idx      [B, Tk_max, d]  bf16   (rows >= len_b are never read)
+ *   k_idx      [B, Tk_max, d]  bf16   (rows >= len_b never affect the result;
+ *                                      prefill may read them, within Tk_max,
+ *                                      as parts of whole 256-row tiles)
  *   kv_len     [B] int32 or NULL      (each 0 <= kv_len[b] <= Tk; values
  *                                      outside are clamped on the device)
  *   idx_out    [B, Tq, k] int32;  count_out [B, Tq] int32
