@@ -18,6 +18,7 @@ are generated on the device before timing.  The per-step working set
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -31,6 +32,28 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from gen import recipes as R  # noqa: E402
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's inputs: every rank decodes its own sequences."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of a per-rank value over the process group (a job's time
+    is its slowest rank's); the value itself when world == 1."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time."""
+    return world * units_per_rank / (ms / 1e3)
 
 CONFIGS = {
     "decode_32k": R.DECODE_32K,
@@ -180,7 +203,7 @@ class DecodeBench:
         import shared_top_routing_b200 as sa
         from gen import torch_inputs as TI
         self.torch, self.sa, self.cfg, self.dev = torch, sa, cfg, device
-        seed_cfg = R.Decode(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+        seed_cfg = R.Decode(**{**cfg.__dict__, "seed": rank_seed(cfg.seed, rank)})
         self.inp = TI.decode_inputs(seed_cfg, device)
         c = cfg
         # all layers' K and V caches as slices of one [layers, 2, B, Tk_max, Hkv, D]
@@ -346,15 +369,12 @@ def run_native(args, cfg, rank, world):
         torch.distributed.barrier()
     ms = start.elapsed_time(stop)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     # per-call times from the event-bracketed graphs, replayed after the timed region
     b.replay_with_events(sorted(set(order)))
     idx_ms, attn_ms = b.kernel_times(order)
     ms_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = job_rate(world, args.steps, ms)
 
     # end to end: per step H2D of the new token's rows and queries from pinned
     # host memory, the step, D2H of all layers' outputs; through the same API
@@ -475,12 +495,8 @@ def run_e2e(b, args, dev, world):
         rt.launch(graphs[(args.warmup + i) % n_steps], st)
     stop.record(st)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * args.steps / (ms / 1e3), 2), "unit": "steps/s",
+    ms = max_over_ranks(start.elapsed_time(stop), world, dev)
+    return {"value": round(job_rate(world, args.steps, ms), 2), "unit": "steps/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "how": "per-step CUDA graph: H2D of queries + appended cache rows from pinned memory "
                    "(all layers' queries in one copy, all layers' K/V rows in one strided copy), "
@@ -495,7 +511,7 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
     import shared_top_routing_b200 as sa
     from gen import torch_inputs as TI
     if isinstance(cfg, R.Gist):
-        inp = TI.gist_inputs(cfg, dev)
+        inp = TI.gist_inputs(dataclasses.replace(cfg, seed=rank_seed(cfg.seed, rank)), dev)
         rows_cap = cfg.rows_cap
         L = sa.lib()
         ws_g = torch.zeros(max(256, L.sa_gist_route_unfold_workspace(cfg.B, cfg.n_chunks, cfg.d, cfg.k_chunks)),
@@ -512,7 +528,7 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
         nbytes = cfg.B * cfg.n_chunks * cfg.d * 2 + cfg.B * rows_cap * cfg.Hkv * cfg.D * 4
         launches = 4   # gist score, finish, attention split, attention merge
     else:
-        inp = TI.prefill_inputs(cfg, dev)
+        inp = TI.prefill_inputs(dataclasses.replace(cfg, seed=rank_seed(cfg.seed, rank)), dev)
         cache = sa.IndexCache(cfg.n_layers, cfg.B, cfg.L, cfg.k, share_every=cfg.share_every, device=dev)
         L = sa.lib()
         ws = torch.zeros(max(256, L.sa_index_score_topk_workspace(cfg.B, cfg.L, cfg.L, cfg.d, cfg.k)),
@@ -546,6 +562,9 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
     for i in range(max(1, args.warmup)):
         step(i % n_steps)
     torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     start.record()
@@ -553,8 +572,10 @@ def run_native_other(args, cfg, rank, world, dev, peaks):
         step((args.warmup + i) % n_steps)
     stop.record()
     torch.cuda.synchronize()
-    ms = start.elapsed_time(stop)
-    value = world * args.steps * per / (ms / 1e3)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = max_over_ranks(start.elapsed_time(stop), world, dev)
+    value = job_rate(world, args.steps * per, ms)
     line = {"metric": "decode steps/s" if unit == "steps/s" else "prefill tokens/s",
             "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
