@@ -12,27 +12,32 @@
 //       product is invariant to the order of its terms, so lane (g, t) of a
 //       warp loads whole 16-byte chunks 4j+t of key row g and the query
 //       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
-//       keys (the query is row 0 of the 16-row A side).  Writes the order-
-//       preserving 32-bit score key of every candidate and a 4096-bin
-//       histogram of the keys' top 12 bits.  The B x Tk key rows are
-//       flattened and split evenly (at multiples of 8 rows) over a grid sized
-//       to the resident CTAs.  (A TMA + tcgen05 variant was measured slower
-//       here: with 128x16 tiles the per-tile TMEM hand-off dominates.)
+//       keys (the query is row 0 of the 16-row A side).  Each warp keeps two
+//       register buffers of key tiles, the next in flight while the current
+//       is scored.  Writes the order-preserving 32-bit score key of every
+//       candidate and a 4096-bin histogram of the keys' top 12 bits.  The
+//       B x Tk key rows are flattened and split evenly (at multiples of 8
+//       rows) over a grid sized to the resident CTAs.  (A TMA + tcgen05
+//       variant was measured slower here: with 128x16 tiles the per-tile
+//       TMEM hand-off dominates.)
 //   collect_kernel       (rows longer than one CTA can scan) finds, from the
 //       histogram, the bin holding the k-th largest key and appends every key
 //       in that bin or above to a per-row candidate list (one atomic per CTA).
 //   prefill_threshold_kernel  (long prefill rows) the k-th largest of the
-//       row's 16-bit group maxima, by a two-digit radix select: the bound the
-//       second scoring pass keeps keys against.
-//   finish_kernel        one CTA per row: gathers the row's candidates into
-//       shared memory (histogram-filtered scan of the row, the collected
-//       list, the bounded pass's list, or the whole row), runs an exact
-//       radix select (8-bit digits,
-//       warp-aggregated shared histograms) of the k-th key and of the tie
-//       positions, then emits in ascending position order through a position
-//       bitmap and popcount prefix sums (bitonic sort for rows beyond the
-//       bitmap's reach).  Also expands chosen gist chunks into cache rows, and
-//       returns the row's histogram and candidate counter to zero.
+//       row's 16-bit group maxima -- a counting pass over a window below
+//       their maximum, or a two-digit radix select -- the bound the second
+//       scoring pass keeps keys against.
+//   finish_kernel        one CTA per row, one instance per candidate source:
+//       gathers the row's candidates into shared memory (histogram-filtered
+//       scan of the row, the collected list, the bounded pass's runs, or the
+//       whole row), runs an exact radix select (8-bit digits, warp-aggregated
+//       shared histograms) of the k-th key, resolves ties at that key by
+//       position (counting within a small tie group, radix passes
+//       otherwise), then emits in ascending position order through a
+//       position bitmap and popcount prefix sums (rows beyond the bitmap's
+//       reach: counts per position range, ranked inside each range).  Also
+//       expands chosen gist chunks into cache rows, and returns the row's
+//       histogram and candidate counter to zero.
 #include <cuda_runtime.h>
 
 #include <algorithm>
