@@ -319,7 +319,7 @@ class DecodeBench:
 
 
 # DRAM bytes (read + write) per decode attention call, split + merge kernels,
-# from the ncu capture summarised in profiles/attn_decode_b8_32k.md.  Must be
+# from an ncu capture of one call (split and merge kernels, DRAM read + write).
 # re-measured (or removed) whenever either kernel changes.
 MEASURED_TRAFFIC = {"decode_b8_32k_4layers": 67_303_680 + 1_033_984 + 2_554_880}
 
@@ -506,7 +506,7 @@ def run_e2e(b, args, dev, world):
 # ------------------------------------------------------------ other configs
 
 def run_native_other(args, cfg, rank, world, dev, peaks):
-    """Prefill and gist workloads (for the design doc / profiles, not the headline)."""
+    """Prefill and gist workloads (reported beside the headline, not as it)."""
     import torch
     import shared_top_routing_b200 as sa
     from gen import torch_inputs as TI
