@@ -319,8 +319,8 @@ class DecodeBench:
 
 
 # DRAM bytes (read + write) per decode attention call, split + merge kernels,
-# from an ncu capture of one call (split and merge kernels, DRAM read + write).
-# re-measured (or removed) whenever either kernel changes.
+# from an ncu capture of one call.  Must be re-measured (or removed) whenever
+# either kernel changes.
 MEASURED_TRAFFIC = {"decode_b8_32k_4layers": 67_303_680 + 1_033_984 + 2_554_880}
 
 
