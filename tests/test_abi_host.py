@@ -189,3 +189,27 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(S, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         S.lib()
+
+
+def _prefill_ws_parts(B, Tq, Tk_max, k):
+    """Bytes the prefill layout needs for `rows` rows per sequence: two
+    [rows, ld] u32 slabs, group maxima [rows, ld2] u16, a u32 bound per row
+    and run counts [rows, ld / 256] u32 (each part 256-byte aligned)."""
+    ld = (Tk_max + 255) // 256 * 256
+    rows = min(Tq, max(128, (1 << 30) // (8 * ld * B) // 128 * 128))
+    m = max(4 * k, (Tk_max + 63) // 64)
+    ld2 = (m + 32 + 7) // 8 * 8
+    R = B * rows
+    a = lambda x: (x + 255) // 256 * 256
+    return 256 + 2 * a(R * ld * 4) + a(R * ld2 * 2) + a(R * 4) + a(R * (ld // 256) * 4)
+
+
+@pytest.mark.parametrize("B,Tq,Tk_max,k", [(1, 2048, 2048, 256), (1, 65536, 65536, 2048), (2, 300, 20480, 1000),
+                                           (3, 100000, 131072, 4096), (1, 4600, 8200, 4096)])
+def test_prefill_workspace_layout(B, Tq, Tk_max, k):
+    """The prefill workspace holds exactly the bounded-pass layout (batches of
+    rows sized so the two slabs take at most 1 GiB, at least 128 rows)."""
+    L = S.lib()
+    got = L.sa_index_score_topk_workspace(B, Tq, Tk_max, 64, k)
+    assert got == _prefill_ws_parts(B, Tq, Tk_max, k)
+    assert got % 256 == 0
