@@ -194,6 +194,23 @@ def test_prefill_topk_bounded_per_sequence_lengths():
     np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
 
 
+def test_prefill_topk_bounded_several_batches():
+    """A 2^20-row key buffer makes a batch 128 rows, so 300 queries over
+    ~10000 live keys take three bounded batches (the later ones start past
+    row 0 of the queries)."""
+    B, L, d, k = 1, 300, 64, 512
+    Tk_max, Tk = 1 << 20, 10000
+    q_pos0 = Tk - L
+    q = _ints(3501, 1, (B, L, d))
+    kk = np.zeros((B, Tk_max, d), dtype=np.uint16)
+    kk[:, :Tk] = _ints(3501, 2, (B, Tk, d))
+    idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, Tk=Tk, q_pos0=q_pos0)
+    ridx, rcnt = oracle.index_topk(q, kk[:, :Tk], Tk, q_pos0, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
 def test_prefill_topk_real_valued_scores():
     """Non-integer bf16 inputs: the GPU's fp32 tile sums may differ from the
     fp64 oracle in the last bits, so compare sets via the oracle's scores:
