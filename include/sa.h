@@ -23,9 +23,11 @@
  *     any CUDA kernel.
  *   - Selected positions are int32 absolute cache rows; unused slots hold -1.
  *   - No kernel of this library waits on another CTA, kernel or device.
- *     Waits inside a kernel (its own pipeline barriers) are bounded; decode
- *     attention records a wait that gave up as a nonzero error word at the
- *     start of its workspace and writes NaN to the outputs.
+ *     Waits inside a kernel (its own pipeline barriers) are bounded.  A wait
+ *     that gave up is recorded as a nonzero error word at the start of the
+ *     call's workspace, and the outputs show it: decode attention writes
+ *     NaN, indexer top-k and gist routing write the failure sentinel
+ *     (count 0, every index -1).
  *   - Workspaces are caller-owned device memory, SA_WS_ALIGN-aligned, and
  *     must be ZERO-FILLED before their first use.  The counters that must
  *     start at zero (histograms, candidate counts, merge tickets) live in a
@@ -102,6 +104,11 @@ int sa_version(void);
  *   score_out  [B, Tq, k] fp32 or NULL
  *   ws         device workspace of >= sa_index_score_topk_workspace(...) bytes
  *              (zero-filled before first use; see the conventions above).
+ *              Its first int32 is the kernel error word: 0 after a good call.
+ *              If a pipeline wait of the call's kernels gave up, the word is
+ *              nonzero and every row gets count 0 and idx -1 (score -inf);
+ *              a workspace whose word is nonzero keeps giving that sentinel
+ *              until the caller zero-fills it again.
  * Supported: d in {64, 128}; 1 <= k <= SA_MAX_K; Tq >= 1; 0 <= Tk <= Tk_max.
  * Scores must be free of NaN (NaN inputs give an unspecified selection).
  * ---------------------------------------------------------------------- */
@@ -233,7 +240,9 @@ sa_status sa_self_test_bounded_wait(int32_t* err, uint32_t poll_limit, sa_stream
  *   q_route     [B, d] bf16;   gist_key [B, n_chunks, d] bf16
  *   partial_len [B] int32 (clamped on the device to [0, chunk_len])
  *   ws          >= sa_gist_route_unfold_workspace(...) bytes (zero-filled
- *               before first use; see the conventions above)
+ *               before first use; see the conventions above).  Its first
+ *               int32 is the kernel error word, as for sa_index_score_topk;
+ *               when it is nonzero every row gets count 0 and rows -1.
  *   rows_out    [B, k_chunks*(chunk_len+1) + chunk_len] int32
  *   count_out   [B] int32;    chunks_out [B, k_chunks] int32 or NULL
  * Supported: d in {64, 128}; 1 <= k_chunks <= SA_MAX_K; 1 <= chunk_len <= 256.

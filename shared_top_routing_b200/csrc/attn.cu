@@ -703,13 +703,7 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
 }
 
 DecPlan decode_plan(int B, int Hkv, int k) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    sms = n > 0 ? n : 148;
-  }
+  const int sms = device_sm_count();
   DecPlan pl;
   pl.nh = Hkv < kDxConsumers ? Hkv : kDxConsumers;
   pl.wph = kDxConsumers / pl.nh;

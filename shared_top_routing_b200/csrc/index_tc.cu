@@ -579,13 +579,7 @@ cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B,
   if (per_seq <= 0) return cudaSuccess;
   p.tiles_per_seq = per_seq;
   // one persistent CTA per SM (512 TMEM columns and most of shared memory each)
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    sms = n > 0 ? n : 148;
-  }
+  const int sms = device_sm_count();
   const long long total = per_seq * B;
   dim3 grid((unsigned)(total < sms ? total : sms));
   if (d == 128) {

@@ -724,7 +724,12 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
   const int t = t0 + r % rows_per_batch;
   const int tid = threadIdx.x;
   const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
-  const uint32_t K = (uint32_t)min(k, n);
+  // A wait in an earlier kernel of this call (the tensor-core scorer) that
+  // gave up left a nonzero error word: the scores are incomplete, so the row
+  // gets the failure sentinel (count 0, every slot -1) instead of a
+  // plausible but wrong selection.
+  bool failed = w.err != nullptr && *reinterpret_cast<volatile const int*>(w.err) != 0;
+  uint32_t K = failed ? 0u : (uint32_t)min(k, n);
   const uint32_t* row = w.keys + (long long)r * w.ld;
   if (tid == 0) s.ncand = 0;
   __syncthreads();
@@ -971,6 +976,10 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
       in_smem = s.ncand <= (uint32_t)kSmemCand;
       from_hist = true;
       bits_known = in_smem;   // the OR / AND covers exactly the kept candidates
+      if (s.abort) {          // a stage wait gave up: the sentinel, as above
+        failed = true;
+        K = 0u;
+      }
     } else if (mode == kFinishCandList) {
       hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
       const uint32_t m = w.cand_cnt[r];
@@ -1123,6 +1132,7 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
     const int stride = out.chunk_len + 1;
     int p = out.partial_len ? out.partial_len[b] : 0;
     p = p < 0 ? 0 : (p > out.chunk_len ? out.chunk_len : p);
+    if (failed) p = 0;   // failure sentinel: no rows at all
     const int unfolded = (int)K * stride;
     const int total = unfolded + p;
     int32_t* rows = out.rows + (long long)b * out.rows_stride;
@@ -1193,18 +1203,8 @@ void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, b
 
 template <int D>
 int score_grid(long long rows) {
-  static int per_sm[2] = {0, 0};
-  static int sms = 0;
-  int& occ = per_sm[D == 128];
-  if (occ == 0) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    int o = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_decode_kernel<D>, kScoreThreads, 0);
-    sms = n > 0 ? n : 148;
-    occ = o > 0 ? o : 1;
-  }
+  const int sms = device_sm_count();
+  const int occ = device_occupancy((const void*)score_decode_kernel<D>, kScoreThreads, 0);
   long long want = (long long)sms * occ;
   const long long by_rows = (rows + 255) / 256;  // at least 256 key rows per CTA
   if (want > by_rows) want = by_rows;

@@ -24,8 +24,8 @@ namespace {
 constexpr size_t kScratchBytes = SA_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// The scratch: the kernel error word and the pair counters (which must start
-// at zero) and the split partials.
+// The scratch: the kernel error word (which must start at zero) and the
+// split partials.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_mu;
@@ -81,8 +81,8 @@ extern "C" sa_status sa_sparse_attn_decode_noalloc(const void* q, const void* k_
   if (B > 0) {
     st = scratch_address(&scratch);
     if (st != SA_OK) return st;
-    // The error word and the pair counters this call uses must start at
-    // zero; clear them on the call's stream (no allocation involved).
+    // The error word must start at zero; clear it on the call's stream (no
+    // allocation involved).
     cudaError_t e = cudaMemsetAsync(scratch, 0, sa::decode_attn_zero_bytes(B, Hkv, k),
                                     reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {

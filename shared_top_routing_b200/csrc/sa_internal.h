@@ -87,6 +87,13 @@ void set_last_error(const char* fmt, ...);
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* func, size_t bytes);
 
+// Number of SMs of the current device, looked up once per device (safe to
+// call from several host threads).
+int device_sm_count();
+// Resident CTAs per SM of `func` at `threads` threads and `smem` dynamic
+// shared bytes on the current device, looked up once per (func, device).
+int device_occupancy(const void* func, int threads, size_t smem);
+
 size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates, bool with_hist);
 void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, bool with_hist,
                          RowWorkspace* out);
@@ -126,7 +133,7 @@ constexpr int kBoundedMinCand = 8192;
 // Attention.
 size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
 // Leading bytes of the decode workspace that must be zero when a call starts
-// (error word and the pair counters this shape uses).
+// (the kernel error word).
 size_t decode_attn_zero_bytes(int B, int Hkv, int k);
 cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,

@@ -423,6 +423,45 @@ def test_index_cache_layers_share_one_index():
     cache.close()
 
 
+def test_index_cache_non_uniform_pattern_fssfsf():
+    """[IC] §三: the full/shared pattern need not be uniform (a searched
+    pattern keeps some indexers and drops others).  Pattern "FSSFSF" over 6
+    layers with 3 indexers (layers 0, 3, 5, each with its own indexer query
+    and keys): every layer attends over exactly its owner's index, and each
+    owner's index matches the oracle."""
+    B, T, d, k, Hq, Hkv, D = 2, 4000, 64, 256, 8, 2, 128
+    pattern = "FSSFSF"
+    owners = oracle.layer_owners(len(pattern), pattern)
+    cache = sa.IndexCache(len(pattern), B, 1, k, pattern=pattern, device=dev())
+    q_idx = {f: _ints(80 + f, 1, (B, d)) for f in set(owners)}
+    k_idx = {f: _ints(80 + f, 2, (B, T, d)) for f in set(owners)}
+    ref = {f: oracle.index_topk(q_idx[f][:, None, :], k_idx[f], T, T - 1, k) for f in set(owners)}
+    cache.begin_step()
+    versions = {}
+    for layer, c in enumerate(pattern):
+        assert cache.is_full(layer) == (1 if c == "F" else 0)
+        assert cache.owner(layer) == owners[layer]
+        if c == "F":
+            cache.update(layer, to_dev(q_idx[layer]), to_dev(k_idx[layer]), Tk=T, q_pos0=T - 1)
+        idx, cnt, ver = cache.get_tensors(layer)
+        versions.setdefault(owners[layer], set()).add(ver)
+        q = _normals(90 + layer, 1, (B, Hq, D))
+        K = _normals(90 + layer, 2, (B, T, Hkv, D))
+        V = _normals(90 + layer, 3, (B, T, Hkv, D))
+        out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), idx.view(B, k), cnt.view(B))
+        torch.cuda.synchronize()
+        ridx, rcnt = ref[owners[layer]]
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+        want, _ = oracle.sparse_attention_decode(q, [K[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)],
+                                                 [V[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)])
+        assert_close_attn(out.float().cpu().numpy(), want, f"pattern {pattern} layer {layer}")
+    # one version per full layer, a new one at each full layer
+    assert all(len(v) == 1 for v in versions.values())
+    assert len({next(iter(v)) for v in versions.values()}) == 3
+    cache.close()
+
+
 # ------------------------------------------------------------- device inputs
 
 def test_device_generator_matches_host_generator():

@@ -126,13 +126,19 @@ def test_prefill_2k_full_parity():
 
 
 def test_prefill_64k_needles_sampled_rows():
+    """Indices bit-exact on the first and last row of every 2048-row batch
+    the indexer runs (the bounded passes work batch by batch), on every
+    needle row and on random rows; every needle retrieved; attention checked
+    on sampled rows of all four layers (different rows per layer)."""
     cfg = R.PREFILL_64K
     idx, cnt, outs = _prefill_run(cfg)
     host = R.prefill_host_inputs(cfg, with_attention=False)
     qi, ki = host["q_idx"][0][0], host["k_idx"][0][0]
     pairs = R.needle_pairs(cfg)
     rng = np.random.default_rng(0)
-    rows = sorted(set([0, 1, 255, 2047, 2048, cfg.L - 1] + [t for _, t in pairs]
+    batch = 2048
+    edges = [r for b0 in range(0, cfg.L, batch) for r in (b0, b0 + 1, b0 + batch - 1)]
+    rows = sorted(set([255, 256, 8191, 8192, 8193] + edges + [t for _, t in pairs]
                       + list(rng.integers(0, cfg.L, 40))))
     s = oracle.index_scores(qi[rows], ki)
     for n_i, t in enumerate(rows):
@@ -142,10 +148,10 @@ def test_prefill_64k_needles_sampled_rows():
         assert np.all(idx[0, t, sel.size:] == -1)
     for p, t in pairs:                       # every needle retrieved
         assert p in set(idx[0, t, : cnt[0, t]].tolist())
-    # attention on sampled rows of the first and last layer of the group
-    att_rows = rows[::3][:16]
-    for layer in (0, cfg.n_layers - 1):
+    # attention: 10 rows per layer, together spanning the batches
+    for layer in range(cfg.n_layers):
         o = outs[layer].float().cpu().numpy()
+        att_rows = rows[layer::max(1, len(rows) // 10)][:10]
         for t in att_rows:
             sel = idx[0, t, : cnt[0, t]]
             q = R.host_rows(cfg.seed, R.tid(R.KIND_Q, layer), (cfg.Hq, cfg.D), np.array([t]), True, 0, cfg.L)[0]

@@ -12,6 +12,7 @@ import os
 import numpy as np
 import pytest
 import torch
+from scipy.special import logsumexp as scipy_logsumexp
 
 import oracle
 from gen import counter_hash as ch
@@ -235,6 +236,81 @@ def test_sparse_attention_with_k_at_least_context_is_dense_causal():
     np.testing.assert_allclose(out[0], ref, rtol=1e-12, atol=1e-12)
 
 
+def _sdpa_over_rows(q, K_rows, V_rows):
+    """torch's scaled_dot_product_attention (float64, no mask) of one query
+    token's heads over its own selected rows, each kv head repeated for its
+    query heads."""
+    Hq, D = q.shape
+    Hkv = K_rows.shape[1]
+    G = Hq // Hkv
+    qt = torch.from_numpy(np.ascontiguousarray(q))[:, None, :]                          # [Hq, 1, D]
+    kt = torch.from_numpy(np.repeat(K_rows, G, axis=1)).permute(1, 0, 2)               # [Hq, n, D]
+    vt = torch.from_numpy(np.repeat(V_rows, G, axis=1)).permute(1, 0, 2)
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[:, 0].numpy()  # [Hq, D]
+
+
+def test_sparse_attention_decode_each_sequence_attends_over_its_own_rows():
+    """[YOIO] §1.1 and §2.3 per decode sequence: sequence b's query heads
+    attend over sequence b's selected rows only.  Four sequences with
+    different row counts (one empty, between two full ones) against torch's
+    SDPA on each sequence alone; an output computed from another sequence's
+    query or rows, or a batch broadcast, differs."""
+    rng = _rng(21)
+    Hq, Hkv, D = 8, 2, 16
+    counts = [5, 0, 37, 12]
+    B = len(counts)
+    q = rng.standard_normal((B, Hq, D)) * 2
+    Kr = [rng.standard_normal((n, Hkv, D)) for n in counts]
+    Vr = [rng.standard_normal((n, Hkv, D)) for n in counts]
+    out, lse = oracle.sparse_attention_decode(q, Kr, Vr)
+    assert out.shape == (B, Hq, D) and lse.shape == (B, Hq)
+    scale = 1.0 / math.sqrt(D)
+    for b, n in enumerate(counts):
+        if n == 0:
+            assert np.all(out[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        np.testing.assert_allclose(out[b], _sdpa_over_rows(q[b], Kr[b], Vr[b]), rtol=1e-12, atol=1e-12)
+        G = Hq // Hkv
+        for h in range(Hq):
+            z = Kr[b][:, h // G] @ q[b, h] * scale
+            assert abs(lse[b, h] - scipy_logsumexp(z)) < 1e-12
+    # each sequence alone gives the same result as inside the batch
+    for b in (0, 2, 3):
+        o1, l1 = oracle.sparse_attention_decode(q[b:b + 1], Kr[b:b + 1], Vr[b:b + 1])
+        np.testing.assert_array_equal(o1[0], out[b])
+        np.testing.assert_array_equal(l1[0], lse[b])
+
+
+def test_sparse_attention_batched_with_per_sequence_indices():
+    """Prefill sparse attention at B = 2 with different indices per sequence
+    and row: each (b, t) against torch's SDPA with a boolean mask holding
+    exactly row t's selected positions of sequence b's cache."""
+    rng = _rng(22)
+    B, T, Hq, Hkv, D, k = 2, 12, 4, 2, 16, 5
+    q = rng.standard_normal((B, T, Hq, D))
+    K = rng.standard_normal((B, T, Hkv, D))
+    V = rng.standard_normal((B, T, Hkv, D))
+    idx = np.full((B, T, k), -1, np.int32)
+    count = np.zeros((B, T), np.int32)
+    for b in range(B):
+        for t in range(T):
+            n = min(k, t + 1) - (b * t) % 2      # sequences differ in counts as well as positions
+            sel = np.sort(rng.choice(t + 1, size=max(n, 1), replace=False))
+            idx[b, t, : sel.size] = sel
+            count[b, t] = sel.size
+    out, _ = oracle.sparse_attention(q, K, V, idx, count)
+    G = Hq // Hkv
+    for b in range(B):
+        mask = np.zeros((T, T), dtype=bool)
+        for t in range(T):
+            mask[t, idx[b, t, : count[b, t]]] = True
+        qt = torch.from_numpy(q[b]).permute(1, 0, 2)
+        kt = torch.from_numpy(np.repeat(K[b], G, axis=1)).permute(1, 0, 2)
+        vt = torch.from_numpy(np.repeat(V[b], G, axis=1)).permute(1, 0, 2)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(mask))
+        np.testing.assert_allclose(out[b], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
 def test_attention_output_is_convex_combination_of_selected_rows():
     rng = _rng(8)
     Hq, Hkv, D, n = 8, 2, 16, 33
@@ -349,3 +425,42 @@ def test_layer_owners_pattern():
     for bad in ("SFF", "FX", "FF"):
         with pytest.raises(ValueError):
             oracle.layer_owners(3, pattern=bad)
+
+
+# ------------------------------------------------------- the pins catch slips
+#
+# Plausible slips planted in the oracle (on the CPU, through monkeypatch)
+# must make the batch pins above fail.
+
+def _mutant_decode_swapped(q, Kr, Vr, scale=None):
+    B = len(Kr)
+    return _ORIG_DECODE(q, [Kr[(b + 1) % B] for b in range(B)], [Vr[(b + 1) % B] for b in range(B)], scale)
+
+
+def _mutant_decode_first_query(q, Kr, Vr, scale=None):
+    q = np.asarray(q)
+    return _ORIG_DECODE(np.broadcast_to(q[:1], q.shape).copy(), Kr, Vr, scale)
+
+
+def _mutant_prefill_first_cache(q, K, V, idx, count, scale=None):
+    K = np.asarray(K)
+    V = np.asarray(V)
+    return _ORIG_PREFILL(q, np.broadcast_to(K[:1], K.shape).copy(), np.broadcast_to(V[:1], V.shape).copy(),
+                         idx, count, scale)
+
+
+_ORIG_DECODE = oracle.sparse_attention_decode
+_ORIG_PREFILL = oracle.sparse_attention
+
+
+@pytest.mark.parametrize("mutant", [_mutant_decode_swapped, _mutant_decode_first_query])
+def test_decode_pin_catches_batch_slips(monkeypatch, mutant):
+    monkeypatch.setattr(oracle, "sparse_attention_decode", mutant)
+    with pytest.raises(AssertionError):
+        test_sparse_attention_decode_each_sequence_attends_over_its_own_rows()
+
+
+def test_prefill_batch_pin_catches_a_shared_cache(monkeypatch):
+    monkeypatch.setattr(oracle, "sparse_attention", _mutant_prefill_first_cache)
+    with pytest.raises(AssertionError):
+        test_sparse_attention_batched_with_per_sequence_indices()
