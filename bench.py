@@ -283,6 +283,21 @@ class Ctx:
         import torch
         return ClockSampler(gpu_uuid(torch, self.dev)) if self.rank == 0 else None
 
+    def soak(self, replay, order, stream, seconds: float, flush: bool = False):
+        """Replays steps for about `seconds` (untimed), so clock samples taken
+        during the timed region that follows see the GPU under load."""
+        import torch
+        t_end = time.time() + seconds
+        i = 0
+        while time.time() < t_end:
+            if flush:
+                self.flush_l2(stream)
+            replay(order[i % len(order)])
+            i += 1
+            if i % 16 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+
     def timed(self, replay, order, stream, flush: bool):
         """Device time (ms, max over ranks) of replay(s) for s in `order`.
         Without flush: one event pair around all steps.  With flush: an event
@@ -554,15 +569,9 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
     torch.cuda.synchronize()
 
     sampler = ctx.sampler()
-    # keep the GPU busy ~1 s before the timed region so clocks are sampled under load
-    t_end = time.time() + (args.soak_seconds if sampler and headline else 0.0)
-    i = 0
-    while time.time() < t_end:
-        b.replay(i % n_steps)
-        i += 1
-        if i % 64 == 0:
-            torch.cuda.synchronize()
     order = [(warmup + i) % n_steps for i in range(steps)]
+    # keep the GPU busy before the timed region so clocks are sampled under load
+    ctx.soak(b.replay, order, b.stream, args.soak_seconds if headline else args.soak_seconds / 2)
     ms = ctx.timed(b.replay, order, b.stream, flush=False)
     clocks = sampler.stop() if sampler else None
     launches = sum(b.kernels_per_step(s) for s in order)
@@ -751,6 +760,7 @@ def measure_prefill(ctx: Ctx, cfg: R.Prefill, steps: int, warmup: int):
     for _ in range(warmup):
         pb.replay()
     sampler = ctx.sampler()
+    ctx.soak(pb.replay, [0], pb.stream, args.soak_seconds / 2, flush)
     ms = ctx.timed(pb.replay, range(steps), pb.stream, flush=flush)
     clocks = sampler.stop() if sampler else None
     idx_ms, attn_ms = pb.part_times(max(1, min(3, steps)), ctx, flush)
@@ -948,6 +958,7 @@ def measure_gist(ctx: Ctx, cfg: R.Gist, steps: int, warmup: int):
         gb.replay(i % cfg.steps)
     order = [(warmup + i) % cfg.steps for i in range(steps)]
     sampler = ctx.sampler()
+    ctx.soak(gb.replay, order, gb.stream, args.soak_seconds / 2, True)
     ms = ctx.timed(gb.replay, order, gb.stream, flush=True)
     clocks = sampler.stop() if sampler else None
     route_ms, attn_ms = gb.part_times(ctx)

@@ -5,6 +5,12 @@ in ``csrc/``).  ``shared_top_routing_b200.sa`` is its Python binding; it only
 marshals arguments.  Build with ``python -m shared_top_routing_b200.build``.
 """
 from .sa import (  # noqa: F401
+    SA_ERR_CUDA,
+    SA_ERR_INVALID_ARG,
+    SA_ERR_STALE_INDEX,
+    SA_ERR_UNSUPPORTED,
+    SA_ERR_WORKSPACE,
+    SA_OK,
     IndexCache,
     SAError,
     lib,
@@ -15,6 +21,12 @@ from .sa import (  # noqa: F401
 )
 
 __all__ = [
+    "SA_ERR_CUDA",
+    "SA_ERR_INVALID_ARG",
+    "SA_ERR_STALE_INDEX",
+    "SA_ERR_UNSUPPORTED",
+    "SA_ERR_WORKSPACE",
+    "SA_OK",
     "IndexCache",
     "SAError",
     "lib",

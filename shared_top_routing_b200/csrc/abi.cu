@@ -198,9 +198,8 @@ size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
   (void)k;
   if (B <= 0 || Tq <= 0 || Tk_max < 0) return 0;
   if (Tq == 1) {
-    bool collect = false;
-    const int mode = sa::finish_mode_for(Tk_max, &collect);
-    return sa::row_workspace_bytes(B, Tk_max, collect, mode != sa::kFinishDirect);
+    const int mode = sa::finish_mode_for(Tk_max);
+    return sa::row_workspace_bytes(B, Tk_max, mode == sa::kFinishSplit, mode != sa::kFinishDirect);
   }
   const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
   return sa::prefill_workspace_bytes(B * rows, Tk_max, k);
@@ -224,20 +223,21 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
   out.score = score_out;
   cudaError_t e;
   if (Tq == 1) {
-    bool collect = false;
-    const int mode = sa::finish_mode_for(Tk_max, &collect);
+    const int mode = sa::finish_mode_for(Tk_max);
     sa::RowWorkspace w;
-    sa::carve_row_workspace(ws, B, Tk_max, collect, mode != sa::kFinishDirect, &w);
+    sa::carve_row_workspace(ws, B, Tk_max, mode == sa::kFinishSplit, mode != sa::kFinishDirect, &w);
     const bool hist = mode != sa::kFinishDirect;
     if (hist && w.hist_zero_bytes &&
         (e = cudaMemsetAsync(w.hist, 0, w.hist_zero_bytes, cs)) != cudaSuccess)
       return cuda_fail(e, "memset");
     if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, hist, cs)) != cudaSuccess)
       return cuda_fail(e, "score_decode launch");
-    if (collect && (e = sa::launch_collect(B, Tk, q_pos0, kv_len, k, w, cs)) != cudaSuccess)
-      return cuda_fail(e, "collect launch");
-    if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, mode, out, cs)) != cudaSuccess)
+    if (mode == sa::kFinishSplit) {
+      if ((e = sa::launch_split_topk(B, Tk, q_pos0, kv_len, k, w, out, cs)) != cudaSuccess)
+        return cuda_fail(e, "split top-k launch");
+    } else if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, mode, out, cs)) != cudaSuccess) {
       return cuda_fail(e, "finish launch");
+    }
     return ok();
   }
   const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
@@ -321,9 +321,8 @@ size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) 
   (void)d;
   (void)k_chunks;
   if (B <= 0 || n_chunks < 0) return 0;
-  bool collect = false;
-  const int mode = sa::finish_mode_for(n_chunks, &collect);
-  return sa::row_workspace_bytes(B, n_chunks, collect, mode != sa::kFinishDirect);
+  const int mode = sa::finish_mode_for(n_chunks);
+  return sa::row_workspace_bytes(B, n_chunks, mode == sa::kFinishSplit, mode != sa::kFinishDirect);
 }
 
 sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B, int n_chunks,
@@ -345,10 +344,9 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   sa_status st = check_ws(ws, ws_bytes, sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks));
   if (st != SA_OK) return st;
   cudaStream_t cs = as_cuda(stream);
-  bool collect = false;
-  const int mode = sa::finish_mode_for(n_chunks, &collect);
+  const int mode = sa::finish_mode_for(n_chunks);
   sa::RowWorkspace w;
-  sa::carve_row_workspace(ws, B, n_chunks, collect, mode != sa::kFinishDirect, &w);
+  sa::carve_row_workspace(ws, B, n_chunks, mode == sa::kFinishSplit, mode != sa::kFinishDirect, &w);
   cudaError_t e;
   const bool hist = mode != sa::kFinishDirect;
   if (hist && w.hist_zero_bytes && (e = cudaMemsetAsync(w.hist, 0, w.hist_zero_bytes, cs)) != cudaSuccess)
@@ -358,8 +356,6 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
                                    static_cast<const uint16_t*>(gist_key), B, d, n_chunks, n_chunks,
                                    q_pos0, nullptr, w, hist, cs)) != cudaSuccess)
     return cuda_fail(e, "gist score launch");
-  if (collect && (e = sa::launch_collect(B, n_chunks, q_pos0, nullptr, k_chunks, w, cs)) != cudaSuccess)
-    return cuda_fail(e, "gist collect launch");
   sa::FinishOut out;
   out.count = count_out;
   out.rows = rows_out;
@@ -368,8 +364,13 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   out.n_chunks = n_chunks;
   out.partial_len = partial_len;
   out.chunks = chunks_out;
-  if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, mode, out, cs)) != cudaSuccess)
+  if (mode == sa::kFinishSplit) {
+    if ((e = sa::launch_split_topk(B, n_chunks, q_pos0, nullptr, k_chunks, w, out, cs)) != cudaSuccess)
+      return cuda_fail(e, "gist split top-k launch");
+  } else if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, mode, out, cs)) !=
+             cudaSuccess) {
     return cuda_fail(e, "gist finish launch");
+  }
   return ok();
 }
 

@@ -20,24 +20,25 @@
 //       rows) over a grid sized to the resident CTAs.  (A TMA + tcgen05
 //       variant was measured slower here: with 128x16 tiles the per-tile
 //       TMEM hand-off dominates.)
-//   collect_kernel       (rows longer than one CTA can scan) finds, from the
-//       histogram, the bin holding the k-th largest key and appends every key
-//       in that bin or above to a per-row candidate list (one atomic per CTA).
 //   prefill_threshold_kernel  (long prefill rows) the k-th largest of the
 //       row's 16-bit group maxima -- a counting pass over a window below
 //       their maximum, or a two-digit radix select -- the bound the second
 //       scoring pass keeps keys against.
-//   finish_kernel        one CTA per row, one instance per candidate source:
-//       gathers the row's candidates into shared memory (histogram-filtered
-//       scan of the row, the collected list, the bounded pass's runs, or the
-//       whole row), runs an exact radix select (8-bit digits, warp-aggregated
+//   finish_kernel        one CTA per row, one instance per candidate source
+//       (the whole row of a short prefill or decode row, or the bounded
+//       prefill pass's runs): gathers the row's candidates into shared
+//       memory, runs an exact radix select (8-bit digits, warp-aggregated
 //       shared histograms) of the k-th key, resolves ties at that key by
 //       position (counting within a small tie group, radix passes
 //       otherwise), then emits in ascending position order through a
 //       position bitmap and popcount prefix sums (rows beyond the bitmap's
 //       reach: counts per position range, ranked inside each range).  Also
-//       expands chosen gist chunks into cache rows, and returns the row's
-//       histogram and candidate counter to zero.
+//       expands chosen gist chunks into cache rows.
+//   split_topk_kernel    one-query rows longer than a CTA's share: many CTAs
+//       per row filter slices against the scorer histogram's threshold bin
+//       and build a second-level histogram; the row's last CTA (ticket, no
+//       waiting) finds the exact threshold and writes the chosen positions
+//       in order with one packed block scan (see the section below).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -168,7 +169,7 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     }
     if (hist != nullptr) {
       __syncthreads();
-      uint32_t* hg = hist + (long long)b * kHistBins;
+      uint32_t* hg = hist + (long long)b * kHistStride;
       for (int i = tid; i < kHistBins; i += kScoreThreads) {
         const uint32_t cnt = sh[i];
         if (cnt) atomicAdd(hg + i, cnt);
@@ -210,86 +211,6 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return r;
 }
 
-// Bin of the K-th largest key in a 4096-bin histogram (bins in key order):
-// s_out[0] = bin, s_out[1] = keys in the bins above it, s_out[2] = keys in it.
-__device__ __forceinline__ void hist_threshold(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
-                                               uint32_t* s_out) {
-  const int per = kHistBins / blockDim.x;  // 16 (256 threads) or 4 (1024 threads)
-  if (threadIdx.x == 0) {   // a histogram holding fewer than K keys leaves bin 0 (keep everything)
-    s_out[0] = 0u;
-    s_out[1] = 0u;
-    s_out[2] = 0u;
-  }
-  uint32_t loc = 0;
-  for (int j = 0; j < per; ++j) loc += h[kHistBins - 1 - (threadIdx.x * per + j)];
-  uint32_t total;
-  const uint32_t excl = block_excl_scan(loc, s_warp, total);
-  if (excl < K && K <= excl + loc) {
-    uint32_t cum = excl;
-    for (int j = 0; j < per; ++j) {
-      const uint32_t c = h[kHistBins - 1 - (threadIdx.x * per + j)];
-      if (cum + c >= K) {
-        s_out[0] = kHistBins - 1 - (threadIdx.x * per + j);
-        s_out[1] = cum;
-        s_out[2] = c;
-        break;
-      }
-      cum += c;
-    }
-  }
-  __syncthreads();
-}
-
-// ------------------------------------------------------------------ collect
-
-constexpr int kCollectPer = 16;   // keys per thread of collect_kernel
-
-__global__ void __launch_bounds__(256)
-collect_kernel(const uint32_t* __restrict__ keys, long long ld, const uint32_t* __restrict__ hist,
-               int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int k, int chunk,
-               uint32_t* __restrict__ cand_cnt, uint32_t* __restrict__ cand_key,
-               uint32_t* __restrict__ cand_pos) {
-  pdl_wait();
-  pdl_launch_dependents();
-  __shared__ uint32_t s_warp[33];
-  __shared__ uint32_t s_thr[3];
-  __shared__ uint32_t s_base;
-  const int b = blockIdx.y;
-  const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
-  const int r0 = blockIdx.x * chunk;
-  if (r0 >= n) return;
-  const int r1 = min(r0 + chunk, n);
-  const uint32_t K = (uint32_t)min(k, n);
-  hist_threshold(hist + (long long)b * kHistBins, K, s_warp, s_thr);
-  const uint32_t bin = s_thr[0];
-
-  const uint32_t* row = keys + (long long)b * ld;
-  const int i0 = r0 + threadIdx.x * kCollectPer;
-  uint32_t kv[kCollectPer];
-  uint32_t mine = 0;
-#pragma unroll
-  for (int j = 0; j < kCollectPer; ++j) {
-    const int i = i0 + j;
-    kv[j] = i < r1 ? row[i] : 0u;
-    mine += (i < r1 && (kv[j] >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-  }
-  uint32_t total;
-  const uint32_t off = block_excl_scan(mine, s_warp, total);
-  if (threadIdx.x == 0) s_base = total ? atomicAdd(cand_cnt + b, total) : 0u;
-  __syncthreads();
-  uint32_t o = s_base + off;
-  uint32_t* ck = cand_key + (long long)b * kCandCap;
-  uint32_t* cp = cand_pos + (long long)b * kCandCap;
-#pragma unroll
-  for (int j = 0; j < kCollectPer; ++j) {
-    const int i = i0 + j;
-    if (i < r1 && (kv[j] >> (32 - kHistBits)) >= bin) {
-      if (o < (uint32_t)kCandCap) { ck[o] = kv[j]; cp[o] = (uint32_t)i; }
-      ++o;
-    }
-  }
-}
-
 // ------------------------------------------------------------------- finish
 
 // Shared memory of the finish kernel for rows of up to CAND candidates held
@@ -302,12 +223,8 @@ struct FinishSmemT {
   uint32_t thr[3];
   uint32_t digit, above, bnd_count, ncand;
   uint32_t kor, kand, por, pand;   // OR / AND of every item's key and position
-  uint64_t stage_bar[2];           // bulk copies of the row into the staging chunks
-  int abort;
   alignas(16) uint32_t ckey[CAND];
   alignas(16) uint32_t cpos[CAND];
-  // bits .. okey are contiguous: before emission they hold the two staging
-  // chunks of the filtered row scan (2 x kStageKeys keys)
   alignas(16) uint32_t bits[BMW];   // position bitmap; bucket counts for long rows
   uint32_t wpre[BMW];               // word prefix sums; bucket starts for long rows
   uint32_t opos[MAXK];              // long rows: chosen items grouped by bucket
@@ -321,12 +238,6 @@ constexpr int kFinThreadsSmall = 256;
 // candidate lists of rows up to 65536 positions (4096 held in shared
 // memory, more read in place), 256 threads: several rows per SM
 using FinishSmemMed = FinishSmemT<4096, 2048, 1>;
-constexpr int kStageKeys = 12288;   // keys per staging chunk (48 KB)
-// bulk copies and 16-byte shared loads need 16-byte aligned chunks
-static_assert(offsetof(FinishSmem, bits) % 16 == 0, "staging area must be 16-byte aligned");
-static_assert((kStageKeys * 4) % 16 == 0, "staging chunks must be 16-byte multiples");
-static_assert(offsetof(FinishSmem, stage_bar) % 8 == 0, "mbarriers must be 8-byte aligned");
-static_assert(2 * kStageKeys <= 2 * kBitmapWords + 2 * kMaxK, "staging chunks exceed their area");
 
 __device__ __forceinline__ void hist_add(uint32_t* h, uint32_t digit, bool active) {
   const unsigned act = __ballot_sync(0xffffffffu, active);
@@ -556,6 +467,35 @@ __device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int 
   }
 }
 
+// Writes a row's padding (slots K..k-1 = -1, scores -inf) and count, or, for
+// gist routing, the partial chunk's rows after the unfolded ones, the row
+// padding and the row count.  A failed row (an upstream wait gave up) gets
+// count 0 and no rows at all.
+__device__ __forceinline__ void finish_tail(const FinishOut& out, int b, int t, int Tq, int k, uint32_t K,
+                                            bool failed, int tid, int nthreads) {
+  const long long o_idx = ((long long)b * Tq + t) * (long long)k;
+  if (out.rows == nullptr) {
+    for (int i = (int)K + tid; i < k; i += nthreads) {
+      out.idx[o_idx + i] = -1;
+      if (out.score) out.score[o_idx + i] = __int_as_float(0xff800000);
+    }
+    if (tid == 0) out.count[(long long)b * Tq + t] = (int32_t)K;
+  } else {
+    const int stride = out.chunk_len + 1;
+    int p = out.partial_len ? out.partial_len[b] : 0;
+    p = p < 0 ? 0 : (p > out.chunk_len ? out.chunk_len : p);
+    if (failed) p = 0;
+    const int unfolded = (int)K * stride;
+    const int total = unfolded + p;
+    int32_t* rows = out.rows + (long long)b * out.rows_stride;
+    for (int i = unfolded + tid; i < out.rows_stride; i += nthreads)
+      rows[i] = i < total ? out.n_chunks * stride + (i - unfolded) : -1;
+    if (out.chunks)
+      for (int i = (int)K + tid; i < k; i += nthreads) out.chunks[o_idx + i] = -1;
+    if (tid == 0) out.count[b] = total;
+  }
+}
+
 // ---------------------------------------------------------------- threshold
 
 constexpr int kThrBins = 4096;     // window of the counting select
@@ -740,8 +680,6 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
   it.pos = nullptr;
   it.n = n;
   bool in_smem = false;
-  // the top 12 bits of the K-th key are known from the scorer's histogram
-  bool from_hist = mode == kFinishHistScan || mode == kFinishCandList;
   bool bits_known = false;                   // the candidates' OR / AND is already in s
   if (K > 0) {
     if (mode == kFinishCandRows) {
@@ -835,176 +773,9 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
         it.n = (int)total;
       }
       __syncthreads();
-    } else if constexpr (kLong) {
-    if (mode == kFinishHistScan || (mode == kFinishDirect && n > kSmemCand)) {
-      // The row streams into shared memory in chunks of kStageKeys keys with
-      // bulk copies, two in flight.  Without the scorer's histogram (long
-      // direct rows) a first pass builds the row's 4096-bin histogram of the
-      // keys' top 12 bits in shared memory.  The filter pass keeps every key
-      // in or above the bin of the K-th largest, each thread counting its
-      // takes and one block scan per chunk placing them.
-      uint32_t* stage = s.bits;
-      const int nchunks = (n + kStageKeys - 1) / kStageKeys;
-      if (tid == 0) {
-        tc::mbar_init(&s.stage_bar[0], 1);
-        tc::mbar_init(&s.stage_bar[1], 1);
-        s.abort = 0;
-        tc::fence_barrier_init();
-      }
-      __syncthreads();
-      int seq = 0;          // chunks streamed so far over all passes (buffer seq & 1)
-      int issued = 0;       // thread 0: chunks issued so far over all passes
-      auto issue = [&](int g, int c) {   // thread 0: chunk c of the pass as stream chunk g
-        const int c0 = c * kStageKeys, len = min(kStageKeys, n - c0);
-        const uint32_t bytes = (uint32_t)((len + 3) & ~3) * 4u;   // rows are padded to 256 keys
-        tc::mbar_arrive_expect_tx(&s.stage_bar[g & 1], bytes);
-        tc::bulk_load(stage + (g & 1) * kStageKeys, row + c0, bytes, &s.stage_bar[g & 1]);
-        issued = g + 1;
-      };
-      auto prime = [&]() {   // the first two chunks of the next pass
-        if (tid == 0) {
-          tc::fence_proxy_async();
-          issue(seq, 0);
-          if (nchunks > 1) issue(seq + 1, 1);
-        }
-      };
-      auto stream = [&](auto&& visit) {
-        for (int c = 0; c < nchunks; ++c) {
-          const int g = seq + c;
-          const bool ok = tc::mbar_wait(&s.stage_bar[g & 1], (uint32_t)(g >> 1) & 1u, &s.abort, w.err, 31);
-          const int c0 = c * kStageKeys;
-          visit(stage + (g & 1) * kStageKeys, c0, ok ? min(kStageKeys, n - c0) : 0);
-          __syncthreads();   // every read of this chunk is done before it is refilled
-          if (tid == 0 && c + 2 < nchunks && !s.abort) {
-            tc::fence_proxy_async();
-            issue(g + 2, c + 2);
-          }
-        }
-        seq += nchunks;
-      };
-      constexpr int kPer = kStageKeys / (4 * kFinThreads);   // uint4 per thread and chunk
-      if (mode == kFinishHistScan) {
-        prime();
-        hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
-      } else {
-        uint32_t* h = s.ckey;   // the histogram, until the filter pass fills the candidates
-        prime();
-        for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
-        __syncthreads();
-        stream([&](const uint32_t* ck, int, int len) {
-#pragma unroll
-          for (int u = 0; u < kPer; ++u) {
-            const int i = (u * kFinThreads + tid) * 4;
-            if (i < len) {
-              const uint4 v = *reinterpret_cast<const uint4*>(ck + i);
-              atomicAdd(&h[v.x >> (32 - kHistBits)], 1u);
-              if (i + 1 < len) atomicAdd(&h[v.y >> (32 - kHistBits)], 1u);
-              if (i + 2 < len) atomicAdd(&h[v.z >> (32 - kHistBits)], 1u);
-              if (i + 3 < len) atomicAdd(&h[v.w >> (32 - kHistBits)], 1u);
-            }
-          }
-        });
-        prime();
-        hist_threshold(h, K, s.swarp, s.thr);
-      }
-      const uint32_t bin = s.thr[0];
-      if (tid == 0) {   // OR / AND of the kept keys and positions, for the select
-        s.kor = 0u;
-        s.kand = ~0u;
-        s.por = 0u;
-        s.pand = ~0u;
-      }
-      uint32_t base = 0;
-      uint32_t ko = 0u, ka = ~0u, po = 0u, pa = ~0u;
-      stream([&](const uint32_t* ck, int c0, int len) {
-        uint4 v[kPer];
-        uint32_t mine = 0;
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int i = (u * kFinThreads + tid) * 4;
-          v[u] = i < len ? *reinterpret_cast<const uint4*>(ck + i) : make_uint4(0, 0, 0, 0);
-          mine += (i < len && (v[u].x >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 1 < len && (v[u].y >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 2 < len && (v[u].z >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-          mine += (i + 3 < len && (v[u].w >> (32 - kHistBits)) >= bin) ? 1u : 0u;
-        }
-        uint32_t total;
-        uint32_t o = base + block_excl_scan(mine, s.swarp, total);
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int i = (u * kFinThreads + tid) * 4;
-          const uint32_t kk4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (i + j < len && (kk4[j] >> (32 - kHistBits)) >= bin) {
-              const uint32_t pos = (uint32_t)(c0 + i + j);
-              if (o < (uint32_t)kSmemCand) {
-                s.ckey[o] = kk4[j];
-                s.cpos[o] = pos;
-              }
-              ++o;
-              ko |= kk4[j];
-              ka &= kk4[j];
-              po |= pos;
-              pa &= pos;
-            }
-          }
-        }
-        base += total;
-      });
-      ko = __reduce_or_sync(0xffffffffu, ko);
-      ka = __reduce_and_sync(0xffffffffu, ka);
-      po = __reduce_or_sync(0xffffffffu, po);
-      pa = __reduce_and_sync(0xffffffffu, pa);
-      if ((tid & 31) == 0) {
-        atomicOr(&s.kor, ko);
-        atomicAnd(&s.kand, ka);
-        atomicOr(&s.por, po);
-        atomicAnd(&s.pand, pa);
-      }
-      if (tid == 0) {
-        s.ncand = base;
-        // after a wait that gave up, copies may still be in flight: let the
-        // last issued ones land (bounded) before the area is reused
-        if (s.abort) {
-          volatile int keep_waiting = 0;
-          for (int g = max(0, issued - 2); g < issued; ++g)
-            tc::mbar_wait(&s.stage_bar[g & 1], (uint32_t)(g >> 1) & 1u, &keep_waiting, nullptr, 0);
-        }
-      }
-      __syncthreads();
-      in_smem = s.ncand <= (uint32_t)kSmemCand;
-      from_hist = true;
-      bits_known = in_smem;   // the OR / AND covers exactly the kept candidates
-      if (s.abort) {          // a stage wait gave up: the sentinel, as above
-        failed = true;
-        K = 0u;
-      }
-    } else if (mode == kFinishCandList) {
-      hist_threshold(w.hist + (long long)r * kHistBins, K, s.swarp, s.thr);
-      const uint32_t m = w.cand_cnt[r];
-      if (m <= (uint32_t)kSmemCand) {
-        const uint32_t* ck = w.cand_key + (long long)r * kCandCap;
-        const uint32_t* cp = w.cand_pos + (long long)r * kCandCap;
-        for (uint32_t i = tid; i < m; i += kFinThreads) { s.ckey[i] = ck[i]; s.cpos[i] = cp[i]; }
-        if (tid == 0) s.ncand = m;
-        in_smem = true;
-      } else if (m <= (uint32_t)kCandCap) {
-        it.key = w.cand_key + (long long)r * kCandCap;
-        it.pos = w.cand_pos + (long long)r * kCandCap;
-        it.n = (int)m;
-      }
-      __syncthreads();
-    } else {  // kFinishDirect: every candidate of the row
-      if (n <= kSmemCand) {
-        for (int i = tid; i < n; i += kFinThreads) { s.ckey[i] = row[i]; s.cpos[i] = (uint32_t)i; }
-        if (tid == 0) s.ncand = (uint32_t)n;
-        in_smem = true;
-      }
-      __syncthreads();
-    }
     } else {
-      // the small layout serves direct rows of at most kSmemCand candidates
+      // kFinishDirect: every candidate of the row (direct launches hold rows
+      // of at most kSmemCand candidates)
       for (int i = tid; i < n; i += kFinThreads) { s.ckey[i] = row[i]; s.cpos[i] = (uint32_t)i; }
       if (tid == 0) s.ncand = (uint32_t)n;
       in_smem = true;
@@ -1019,15 +790,7 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
 
   uint32_t prefix = 0, pmask = 0, pmax = 0;
   if (K > 0) {
-    SelStart st;
-    if (!from_hist) {
-      st = SelStart{0u, 0u, K, (uint32_t)it.n, 24, bits_known};
-    } else {
-      // the histogram already fixes the top 12 bits: every item above the
-      // bin is chosen, K - above of the bin's items remain to pick
-      st = SelStart{s.thr[0] << (32 - kHistBits), ~0u << (32 - kHistBits), K - s.thr[1], s.thr[2],
-                    32 - kHistBits - 8, bits_known};
-    }
+    const SelStart st{0u, 0u, K, (uint32_t)it.n, 24, bits_known};
     select_threshold<Sm, THREADS>(s, it, st, prefix, pmask, pmax);
   }
 
@@ -1122,34 +885,344 @@ finish_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_
   }
 
   // ---- padding and counts
-  if (out.rows == nullptr) {
-    for (int i = (int)K + tid; i < k; i += kFinThreads) {
-      out.idx[o_idx + i] = -1;
-      if (out.score) out.score[o_idx + i] = __int_as_float(0xff800000);
-    }
-    if (tid == 0) out.count[(long long)b * Tq + t] = (int32_t)K;
-  } else {
-    const int stride = out.chunk_len + 1;
-    int p = out.partial_len ? out.partial_len[b] : 0;
-    p = p < 0 ? 0 : (p > out.chunk_len ? out.chunk_len : p);
-    if (failed) p = 0;   // failure sentinel: no rows at all
-    const int unfolded = (int)K * stride;
-    const int total = unfolded + p;
-    int32_t* rows = out.rows + (long long)b * out.rows_stride;
-    for (int i = unfolded + tid; i < out.rows_stride; i += kFinThreads)
-      rows[i] = i < total ? out.n_chunks * stride + (i - unfolded) : -1;
-    if (out.chunks)
-      for (int i = (int)K + tid; i < k; i += kFinThreads) out.chunks[o_idx + i] = -1;
-    if (tid == 0) out.count[b] = total;
-  }
+  finish_tail(out, b, t, Tq, k, K, failed, tid, kFinThreads);
+}
 
-  // ---- return this row's histogram and candidate counter to zero
-  if (mode == kFinishHistScan || mode == kFinishCandList) {
-    __syncthreads();
-    uint32_t* h = w.hist + (long long)r * kHistBins;
-    for (int i = tid; i < kHistBins; i += kFinThreads) h[i] = 0;
-    if (tid == 0) w.cand_cnt[r] = 0;
+// ------------------------------------------------------------- split rows
+//
+// Rows that carry the scorer's histogram (one query per sequence: decode
+// scoring and gist routing over more than kDirectMaxCand candidates) are
+// selected by many CTAs per row, with no CTA waiting for another.
+//   1. Every CTA finds, from the scorer's histogram of the keys' top 12 bits,
+//      the bin of the row's K-th largest key.  CTA c then filters positions
+//      [c * chunk, (c + 1) * chunk): each key in or above that bin goes, with
+//      its position and in position order (one block scan), into the slice's
+//      part of the row's candidate array; keys inside the bin also count in a
+//      second histogram of their next 12 bits.  The slice's candidate count
+//      goes to its slot, and the CTA takes a ticket on the row's counter
+//      (threadfence, then atomicAdd).
+//   2. The row's last CTA gathers every slice's candidates (already in
+//      ascending position order) and finds, from the second histogram, the
+//      24-bit prefix T of the K-th key and how many of the keys with prefix T
+//      are still to take (kk).  When those keys are all equal (integer-valued
+//      scores make every key a multiple of 256), the first kk of them in
+//      position order are the chosen ones, so one block scan of packed
+//      (above-T, equal-to-T) counts gives every item both its choice and its
+//      output slot.  Otherwise an exact radix select over the low 8 bits and
+//      the positions decides, followed by an ordered compaction.
+//   3. The last CTA returns the row's histograms and counter to zero.
+
+constexpr int kSplitThreads = 512;
+constexpr int kSplitCand = 8192;         // candidates the finishing CTA holds in shared memory
+constexpr int kSplitSlice = kSplitThreads * 4;   // positions per slice unit (one uint4 per thread)
+constexpr int kSplitPer = 8;             // candidates per thread and pass of the finishing CTA
+
+struct SplitSmem {
+  static constexpr int kBmw = 256;       // bounds the select's tie list
+  uint32_t hist[256];
+  uint32_t swarp[33];
+  uint32_t thr[3];                       // first-level bin of the K-th key, keys above it, keys in it
+  uint32_t thr2[3];                      // the same for the next 12 bits inside that bin
+  uint32_t digit, above, bnd_count, ncand;
+  uint32_t kor, kand, por, pand;
+  int last;
+  uint32_t bits[256];                    // tie list of the general select
+  uint32_t pre[kSplitMaxSlices];         // first gathered index of each slice
+  alignas(16) uint32_t ckey[kSplitCand];
+  alignas(16) uint32_t cpos[kSplitCand];
+};
+static_assert(offsetof(SplitSmem, ckey) % 16 == 0 && offsetof(SplitSmem, cpos) % 16 == 0,
+              "candidate arrays are read as 16-byte vectors");
+
+// Bin of the K-th largest key of a 4096-bin histogram (bins in key order),
+// read once with 16-byte loads through L2 and kept in registers: s_out[0] =
+// bin, s_out[1] = keys in the bins above it, s_out[2] = keys in it (0, 0, 0
+// when the histogram holds fewer than K keys).
+template <int THREADS>
+__device__ __forceinline__ void hist_threshold_v(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
+                                                 uint32_t* s_out) {
+  constexpr int per = kHistBins / THREADS;
+  static_assert(per % 4 == 0, "16-byte loads of whole bins");
+  const int base = kHistBins - per * ((int)threadIdx.x + 1);   // thread 0 holds the top bins
+  uint32_t c[per];
+#pragma unroll
+  for (int v = 0; v < per / 4; ++v) {
+    const uint4 x = __ldcg(reinterpret_cast<const uint4*>(h + base) + v);
+    c[4 * v] = x.x;
+    c[4 * v + 1] = x.y;
+    c[4 * v + 2] = x.z;
+    c[4 * v + 3] = x.w;
   }
+  if (threadIdx.x == 0) {
+    s_out[0] = 0u;
+    s_out[1] = 0u;
+    s_out[2] = 0u;
+  }
+  uint32_t loc = 0;
+#pragma unroll
+  for (int j = 0; j < per; ++j) loc += c[j];
+  uint32_t total;
+  const uint32_t excl = block_excl_scan(loc, s_warp, total);   // keys in the bins above this thread's
+  if (excl < K && K <= excl + loc) {
+    uint32_t cum = excl;
+#pragma unroll
+    for (int j = per - 1; j >= 0; --j) {
+      if (cum < K && cum + c[j] >= K) {
+        s_out[0] = (uint32_t)(base + j);
+        s_out[1] = cum;
+        s_out[2] = c[j];
+      }
+      cum += c[j];
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSplitThreads)
+split_topk_kernel(RowWorkspace w, int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int k, int chunk,
+                  FinishOut out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SplitSmem& s = *reinterpret_cast<SplitSmem*>(smem_raw);
+  const int c = blockIdx.x, F = gridDim.x, r = blockIdx.y;
+  const int b = r;
+  const int tid = threadIdx.x;
+  const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
+  // a wait in an earlier kernel of this call that gave up: failure sentinel
+  const bool failed = w.err != nullptr && *reinterpret_cast<volatile const int*>(w.err) != 0;
+  const uint32_t K = failed ? 0u : (uint32_t)min(k, n);
+  const uint32_t* row = w.keys + (long long)r * w.ld;
+  uint32_t* hist1 = w.hist + (long long)r * kHistStride;
+  uint32_t* hist2 = hist1 + kHistBins;
+  uint2* cand = w.cand + (long long)r * w.ld;
+  uint32_t* slot = w.slot_cnt + (long long)r * kSplitMaxSlices;
+  const int c0 = c * chunk;
+  constexpr int kLo = 32 - kHistBits;        // shift of the first-level bin
+  constexpr int kLo2 = 32 - 2 * kHistBits;   // shift of the second-level bin
+
+  // ---- 1. filter this slice (in position order)
+  uint32_t taken = 0;
+  if (K > 0) {
+    hist_threshold_v<kSplitThreads>(hist1, K, s.swarp, s.thr);
+    const uint32_t bin = s.thr[0];
+    for (int u0 = 0; u0 < chunk; u0 += kSplitSlice) {
+      const int i = c0 + u0 + tid * 4;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i < n) v = *reinterpret_cast<const uint4*>(row + i);   // rows are padded to 256 keys
+      const uint32_t kv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t mine = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mine += (i + e < n && (kv[e] >> kLo) >= bin) ? 1u : 0u;
+      uint32_t tot;
+      uint32_t o = (uint32_t)c0 + taken + block_excl_scan(mine, s.swarp, tot);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e < n && (kv[e] >> kLo) >= bin) {
+          cand[o++] = make_uint2(kv[e], (uint32_t)(i + e));
+          if ((kv[e] >> kLo) == bin) atomicAdd(hist2 + ((kv[e] >> kLo2) & (kHistBins - 1)), 1u);
+        }
+      taken += tot;
+      if (c0 + u0 + kSplitSlice >= n) break;
+    }
+  }
+  if (tid == 0) slot[c] = taken;
+
+  // ---- ticket: the row's last CTA finishes the row
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s.last = atomicAdd(&w.cand_cnt[r], 1u) == (uint32_t)F - 1u;
+  }
+  __syncthreads();
+  if (!s.last) return;
+  __threadfence();
+
+  // ---- 2. the finishing CTA
+  uint32_t total = 0;
+  for (int s0 = 0; s0 < F; s0 += kSplitThreads) {
+    const int sl = s0 + tid;
+    const uint32_t v = sl < F ? __ldcg(slot + sl) : 0u;
+    uint32_t part;
+    const uint32_t o = total + block_excl_scan(v, s.swarp, part);
+    if (sl < F) s.pre[sl] = o;
+    total += part;
+  }
+  __syncthreads();
+  const bool in_smem = total <= (uint32_t)kSplitCand;
+  const long long o_idx = (long long)b * k;
+  if (K > 0) {
+    // gathered candidate i belongs to the last slice whose first index is <= i
+    auto fetch = [&](uint32_t i) {
+      int lo = 0, hi = F - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.pre[mid] <= i) lo = mid;
+        else hi = mid - 1;
+      }
+      return __ldcg(cand + (long long)lo * chunk + (i - s.pre[lo]));
+    };
+    // the first pass's loads are issued before the second histogram is read,
+    // so both are in flight together
+    uint2 e[kSplitPer];
+    uint32_t i0 = 0;
+    if (in_smem) {
+#pragma unroll
+      for (int u = 0; u < kSplitPer; ++u) {
+        const uint32_t i = (uint32_t)tid * kSplitPer + u;
+        e[u] = i < total ? fetch(i) : make_uint2(0u, 0u);
+      }
+    }
+    hist_threshold_v<kSplitThreads>(hist2, K - s.thr[1], s.swarp, s.thr2);
+    const uint32_t T = s.thr[0] << kHistBits | s.thr2[0];   // 24-bit prefix of the K-th key
+    const uint32_t kk = K - s.thr[1] - s.thr2[1];           // keys with prefix T still to take
+    PairItems it;
+    it.n = (int)total;
+    bool uniform = false;   // every key with prefix T is the same key
+    if (in_smem) {
+      if (tid == 0) {
+        s.kor = 0u;
+        s.kand = ~0u;
+      }
+      uint32_t ko = 0u, ka = ~0u;
+      for (i0 = 0; i0 < total; i0 += kSplitThreads * kSplitPer) {
+        if (i0 > 0) {
+#pragma unroll
+          for (int u = 0; u < kSplitPer; ++u) {
+            const uint32_t i = i0 + (uint32_t)tid * kSplitPer + u;
+            e[u] = i < total ? fetch(i) : make_uint2(0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kSplitPer; ++u) {
+          const uint32_t i = i0 + (uint32_t)tid * kSplitPer + u;
+          if (i < total) {
+            s.ckey[i] = e[u].x;
+            s.cpos[i] = e[u].y;
+            if ((e[u].x >> 8) == T) {
+              ko |= e[u].x;
+              ka &= e[u].x;
+            }
+          }
+        }
+      }
+      __syncthreads();
+      ko = __reduce_or_sync(0xffffffffu, ko);
+      ka = __reduce_and_sync(0xffffffffu, ka);
+      if ((tid & 31) == 0) {
+        atomicOr(&s.kor, ko);
+        atomicAnd(&s.kand, ka);
+      }
+      __syncthreads();
+      uniform = s.kor == s.kand;   // (no key with prefix T at all cannot happen: kk >= 1)
+      it.key = s.ckey;
+      it.pos = s.cpos;
+      it.shift = 0;
+    } else {
+      // more candidates than shared memory holds (heavy ties): close the gaps
+      // between slices in place, kSplitThreads pairs per round (a round's
+      // writes land at or before its reads, which are all done)
+      for (int sl = 0; sl < F; ++sl) {
+        const uint32_t cnt = __ldcg(slot + sl);
+        const uint32_t dst = s.pre[sl];
+        for (uint32_t j0 = 0; j0 < cnt; j0 += kSplitThreads) {
+          const uint32_t j = j0 + tid;
+          uint2 v = make_uint2(0u, 0u);
+          if (j < cnt) v = __ldcg(cand + (long long)sl * chunk + j);
+          __syncthreads();
+          if (j < cnt) cand[dst + j] = v;
+          __syncthreads();
+        }
+      }
+      it.key = reinterpret_cast<const uint32_t*>(cand);
+      it.pos = reinterpret_cast<const uint32_t*>(cand) + 1;
+      it.shift = 1;
+    }
+
+    if (uniform) {
+      // ---- 2a. the first kk keys equal to the K-th key, in position order,
+      // are chosen: slot = (chosen keys above T before it) + min(keys equal
+      // to T before it, kk); counts packed as (equal << 16 | above)
+      uint32_t base = 0;
+      for (i0 = 0; i0 < total; i0 += kSplitThreads * kSplitPer) {
+        const uint32_t i = i0 + (uint32_t)tid * kSplitPer;
+        uint32_t kk8[kSplitPer], pp8[kSplitPer], mine = 0;
+#pragma unroll
+        for (int u = 0; u < kSplitPer; u += 4) {
+          uint4 kv = make_uint4(0u, 0u, 0u, 0u), pv = make_uint4(0u, 0u, 0u, 0u);
+          if (i + u + 3 < total) {
+            kv = *reinterpret_cast<const uint4*>(s.ckey + i + u);
+            pv = *reinterpret_cast<const uint4*>(s.cpos + i + u);
+          } else {
+            if (i + u < total) { kv.x = s.ckey[i + u]; pv.x = s.cpos[i + u]; }
+            if (i + u + 1 < total) { kv.y = s.ckey[i + u + 1]; pv.y = s.cpos[i + u + 1]; }
+            if (i + u + 2 < total) { kv.z = s.ckey[i + u + 2]; pv.z = s.cpos[i + u + 2]; }
+          }
+          kk8[u] = kv.x; kk8[u + 1] = kv.y; kk8[u + 2] = kv.z; kk8[u + 3] = kv.w;
+          pp8[u] = pv.x; pp8[u + 1] = pv.y; pp8[u + 2] = pv.z; pp8[u + 3] = pv.w;
+        }
+#pragma unroll
+        for (int u = 0; u < kSplitPer; ++u) {
+          const bool v = i + u < total;
+          const uint32_t p24 = kk8[u] >> 8;
+          mine += v && p24 > T ? 1u : (v && p24 == T ? 0x10000u : 0u);
+        }
+        uint32_t tot;
+        uint32_t run = base + block_excl_scan(mine, s.swarp, tot);
+#pragma unroll
+        for (int u = 0; u < kSplitPer; ++u) {
+          if (i + u < total) {
+            const uint32_t p24 = kk8[u] >> 8;
+            const uint32_t above = run & 0xFFFFu, equal = run >> 16;
+            if (p24 > T) {
+              emit(out, o_idx, b, above + min(equal, kk), pp8[u], kk8[u]);
+              run += 1u;
+            } else if (p24 == T) {
+              if (equal < kk) emit(out, o_idx, b, above + equal, pp8[u], kk8[u]);
+              run += 0x10000u;
+            }
+          }
+        }
+        base += tot;
+      }
+    } else {
+      // ---- 2b. exact select below the 24-bit prefix (low 8 bits, then
+      // positions), then an ordered compaction of the chosen items
+      uint32_t prefix = 0u, pmask = 0u, pmax = 0xFFFFFFFFu;
+      const SelStart st{T << 8, 0xFFFFFF00u, kk, s.thr2[2], 0, false};
+      select_threshold<SplitSmem, kSplitThreads>(s, it, st, prefix, pmask, pmax);
+      uint32_t base = 0;
+      for (i0 = 0; i0 < total; i0 += kSplitThreads * 4) {
+        const uint32_t i = i0 + (uint32_t)tid * 4;
+        uint32_t kk4[4], pp4[4];
+        bool sel[4];
+        uint32_t mine = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          kk4[u] = i + u < total ? it.k((int)(i + u)) : 0u;
+          pp4[u] = i + u < total ? it.p((int)(i + u)) : 0u;
+          sel[u] = i + u < total && is_selected(kk4[u], pp4[u], prefix, pmask, pmax);
+          mine += sel[u] ? 1u : 0u;
+        }
+        uint32_t tot;
+        uint32_t o = base + block_excl_scan(mine, s.swarp, tot);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (sel[u]) {
+            if (o < K) emit(out, o_idx, b, o, pp4[u], kk4[u]);   // exactly K are chosen
+            ++o;
+          }
+        base += tot;
+      }
+    }
+  }
+  finish_tail(out, b, 0, 1, k, K, failed, tid, kSplitThreads);
+
+  // ---- 3. every CTA of the row has used the histograms: return them and
+  // the ticket to zero for the next call
+  for (int i = tid * 4; i < kHistStride; i += kSplitThreads * 4)
+    *reinterpret_cast<uint4*>(hist1 + i) = make_uint4(0u, 0u, 0u, 0u);
+  if (tid == 0) w.cand_cnt[r] = 0u;
 }
 
 }  // namespace
@@ -1160,44 +1233,44 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 static long long row_ld(int Tk_max) { return ((long long)Tk_max + 255) / 256 * 256; }
 
 // Layout: [error word][fixed histograms + counters for kHistRowsFixed rows]
-// [histograms + counters for larger row counts][keys][candidate lists].  The
-// fixed region holds nothing else, so once zero-filled it stays valid across
-// calls of any shape (the finish kernel returns each row it used to zero).
-size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates, bool with_hist) {
+// [histograms + counters for larger row counts][keys][split rows: candidate
+// pairs, slice counts].  The fixed region holds nothing else, so once
+// zero-filled it stays valid across calls of any shape (the selection
+// returns each row it used to zero).
+size_t row_workspace_bytes(int rows, int Tk_max, bool split, bool with_hist) {
   const long long ld = row_ld(Tk_max);
   size_t bytes = 256;
-  bytes += align256((size_t)kHistRowsFixed * kHistBins * 4) + align256((size_t)kHistRowsFixed * 4);
+  bytes += align256((size_t)kHistRowsFixed * kHistStride * 4) + align256((size_t)kHistRowsFixed * 4);
   if (with_hist && rows > kHistRowsFixed)
-    bytes += align256((size_t)rows * kHistBins * 4) + align256((size_t)rows * 4);
+    bytes += align256((size_t)rows * kHistStride * 4) + align256((size_t)rows * 4);
   bytes += align256((size_t)rows * ld * 4);
-  if (with_candidates) bytes += 2 * align256((size_t)rows * kCandCap * 4);
+  if (split) bytes += align256((size_t)rows * ld * 8) + align256((size_t)rows * kSplitMaxSlices * 4);
   return bytes;
 }
 
-void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, bool with_hist,
-                         RowWorkspace* o) {
+void carve_row_workspace(void* ws, int rows, int Tk_max, bool split, bool with_hist, RowWorkspace* o) {
   char* p = static_cast<char*>(ws);
   o->ld = row_ld(Tk_max);
   o->err = reinterpret_cast<int*>(p);
   p += 256;
   o->hist = reinterpret_cast<uint32_t*>(p);
-  p += align256((size_t)kHistRowsFixed * kHistBins * 4);
+  p += align256((size_t)kHistRowsFixed * kHistStride * 4);
   o->cand_cnt = reinterpret_cast<uint32_t*>(p);
   p += align256((size_t)kHistRowsFixed * 4);
   o->hist_zero_bytes = 0;
   if (with_hist && rows > kHistRowsFixed) {
     o->hist = reinterpret_cast<uint32_t*>(p);
-    p += align256((size_t)rows * kHistBins * 4);
+    p += align256((size_t)rows * kHistStride * 4);
     o->cand_cnt = reinterpret_cast<uint32_t*>(p);
     p += align256((size_t)rows * 4);
     o->hist_zero_bytes = (size_t)(p - reinterpret_cast<char*>(o->hist));
   }
   o->keys = reinterpret_cast<uint32_t*>(p);
   p += align256((size_t)rows * o->ld * 4);
-  if (with_candidates) {
-    o->cand_key = reinterpret_cast<uint32_t*>(p);
-    p += align256((size_t)rows * kCandCap * 4);
-    o->cand_pos = reinterpret_cast<uint32_t*>(p);
+  if (split) {
+    o->cand = reinterpret_cast<uint2*>(p);
+    p += align256((size_t)rows * o->ld * 8);
+    o->slot_cnt = reinterpret_cast<uint32_t*>(p);
   }
 }
 
@@ -1227,16 +1300,6 @@ cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, 
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
-                           const RowWorkspace& w, cudaStream_t st) {
-  if (Tk <= 0 || B <= 0) return cudaSuccess;
-  const int chunk = 256 * kCollectPer;
-  dim3 grid((Tk + chunk - 1) / chunk, B);
-  const cudaError_t e = launch_pdl(collect_kernel, grid, dim3(256), 0, st, w.keys, w.ld, w.hist, Tk, q_pos0,
-                                   kv_len, k, chunk, w.cand_cnt, w.cand_key, w.cand_pos);
-  return e != cudaSuccess ? e : cudaGetLastError();
-}
-
 cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
                           const int32_t* kv_len, int k, const RowWorkspace& w, int mode,
                           const FinishOut& out, cudaStream_t st) {
@@ -1258,34 +1321,54 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
     e = go(finish_kernel<FinishSmemMed, kFinThreadsSmall, kFinishCandRows>, sizeof(FinishSmemMed), kFinThreadsSmall);
   else if (mode == kFinishDirect)
     e = go(finish_kernel<FinishSmem, kFinThreads, kFinishDirect>, sizeof(FinishSmem), kFinThreads);
-  else if (mode == kFinishHistScan)
-    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishHistScan>, sizeof(FinishSmem), kFinThreads);
-  else if (mode == kFinishCandList)
-    e = go(finish_kernel<FinishSmem, kFinThreads, kFinishCandList>, sizeof(FinishSmem), kFinThreads);
   else
     e = go(finish_kernel<FinishSmem, kFinThreads, kFinishCandRows>, sizeof(FinishSmem), kFinThreads);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-int finish_mode_for(int Tk_max, bool* need_collect) {
-  // short rows: one CTA holds the whole row; rows one CTA can still scan:
-  // histogram-filtered scan; longer rows: many CTAs collect candidates first
-  *need_collect = false;
-  if (Tk_max <= kDirectMaxCand) return kFinishDirect;
-  if (Tk_max <= kBitmapMax) return kFinishHistScan;
-  *need_collect = true;
-  return kFinishCandList;
+int finish_mode_for(int Tk_max) {
+  // short rows: one CTA holds the whole row; longer rows: slices over many
+  // CTAs, the row's last CTA selects
+  return Tk_max <= kDirectMaxCand ? kFinishDirect : kFinishSplit;
 }
 
-// Prefill layout: [error word][keys: rows x ld][second slab: rows x ld]
-// [group maxima: rows x ld2 (16-bit)][bound: rows][run counts: rows x
-// ld/256].  Short batches use only the key slab; long ones use both slabs as
-// one [rows][ld] array of (score bits, position) pairs for the bounded
-// pass's takes (each scoring CTA's run of a row at the run's first column).
+cudaError_t launch_split_topk(int B, int Tk, int q_pos0, const int32_t* kv_len, int k, const RowWorkspace& w,
+                              const FinishOut& out, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  // slices of a multiple of kSplitSlice positions: about two CTAs per SM over
+  // all rows, at most kSplitMaxSlices per row
+  const long long n_max = std::max<long long>(1, std::min<long long>(Tk, (long long)q_pos0 + 1));
+  const long long target = std::max<long long>(1, 2LL * device_sm_count() / B);
+  long long chunk = (n_max + target - 1) / target;
+  const long long floor_chunk = (n_max + kSplitMaxSlices - 1) / kSplitMaxSlices;
+  chunk = std::max(chunk, floor_chunk);
+  chunk = (chunk + kSplitSlice - 1) / kSplitSlice * kSplitSlice;
+  const int F = (int)((n_max + chunk - 1) / chunk);
+  const size_t smem = sizeof(SplitSmem);
+  cudaError_t e = ensure_dynamic_smem((const void*)split_topk_kernel, smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(split_topk_kernel, dim3((unsigned)F, (unsigned)B), dim3(kSplitThreads), smem, st, w, Tk, q_pos0,
+                 kv_len, k, (int)chunk, out);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Bytes of the fixed, self-cleaning region of one-query workspaces (the
+// histograms and tickets of kHistRowsFixed rows) after the error word.
+static size_t fixed_region_bytes() {
+  return align256((size_t)kHistRowsFixed * kHistStride * 4) + align256((size_t)kHistRowsFixed * 4);
+}
+
+// Prefill layout: [error word][the one-query fixed region, left untouched so
+// that a workspace can alternate between prefill and decode calls][keys:
+// rows x ld][second slab: rows x ld][group maxima: rows x ld2 (16-bit)]
+// [bound: rows][run counts: rows x ld/256].  Short batches use only the key
+// slab; long ones use both slabs as one [rows][ld] array of (score bits,
+// position) pairs for the bounded pass's takes (each scoring CTA's run of a
+// row at the run's first column).
 size_t prefill_workspace_bytes(int rows, int Tk_max, int k) {
   const long long ld = row_ld(Tk_max);
   const long long ld2 = prefill_groups_ld(Tk_max, k);
-  return 256 + 2 * align256((size_t)rows * ld * 4) + align256((size_t)rows * ld2 * 2) +
+  return 256 + fixed_region_bytes() + 2 * align256((size_t)rows * ld * 4) + align256((size_t)rows * ld2 * 2) +
          align256((size_t)rows * 4) + align256((size_t)rows * (ld / 256) * 4);
 }
 
@@ -1294,7 +1377,7 @@ void carve_prefill_workspace(void* ws, int rows, int Tk_max, int k, RowWorkspace
   o->ld = row_ld(Tk_max);
   o->ld2 = prefill_groups_ld(Tk_max, k);
   o->err = reinterpret_cast<int*>(p);
-  p += 256;
+  p += 256 + fixed_region_bytes();
   o->keys = reinterpret_cast<uint32_t*>(p);
   p += align256((size_t)rows * o->ld * 4);
   o->cand_pos = reinterpret_cast<uint32_t*>(p);

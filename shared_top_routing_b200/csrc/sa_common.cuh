@@ -9,7 +9,10 @@ namespace sa {
 constexpr int kMaxK = 4096;          // SA_MAX_K
 constexpr int kHistBits = 12;        // first radix digit of a score key
 constexpr int kHistBins = 1 << kHistBits;
-constexpr int kCandCap = 32768;      // candidate slots per row before the full-row fallback
+// Words per row of the one-query histograms: the scorer's histogram of the
+// keys' top 12 bits, then the split selection's histogram of the next 12
+// bits of the keys in the K-th key's first bin.
+constexpr int kHistStride = 2 * kHistBins;
 
 // Long prefill rows are selected in two scoring passes.  The first keeps,
 // per row, only the maximum score of each group of g consecutive positions

@@ -9,16 +9,19 @@
 
 namespace sa {
 
-// Rows of at most this many candidates are selected by one CTA holding the
-// whole row in shared memory ("direct" mode); longer rows use the key
-// histogram (and, beyond what one CTA can scan, a multi-CTA collect pass).
-constexpr int kDirectMaxCand = 8192;
+// One-query rows (decode, gist routing) of at most this many candidates are
+// selected by one CTA holding the whole row in shared memory ("direct"
+// mode); longer rows carry the scorer's key histogram and are selected by
+// slices over many CTAs (kFinishSplit).
+constexpr int kDirectMaxCand = 4096;
 
 // finish_kernel candidate sources
 constexpr int kFinishDirect = 0;    // the whole row (no histogram)
-constexpr int kFinishHistScan = 1;  // one CTA scans the row, keeping keys in or above the k-th key's bin
-constexpr int kFinishCandList = 2;  // candidates collected by collect_kernel
 constexpr int kFinishCandRows = 3;  // prefill: candidates appended by the bounded scoring pass
+constexpr int kFinishSplit = 4;     // many CTAs per row filter slices, the row's last CTA selects
+
+// Slices (CTAs) per row of the split selection, at most.
+constexpr int kSplitMaxSlices = 1024;
 
 // Prefill scoring passes (launch_score_prefill `epi`)
 constexpr int kScoreKeys = 0;       // every score's key into the row slab
@@ -34,13 +37,14 @@ struct RowWorkspace {
   uint32_t* keys = nullptr;      // [rows][ld] order-preserving score keys (prefill candidate rows: their keys)
   long long ld = 0;
   uint32_t* hist = nullptr;      // [rows][kHistBins]
-  uint32_t* cand_cnt = nullptr;  // [rows]
-  uint32_t* cand_key = nullptr;  // [rows][kCandCap]
-  uint32_t* cand_pos = nullptr;  // [rows][kCandCap]; prefill candidate rows: [rows][ld]
+  uint32_t* cand_cnt = nullptr;  // [rows] split rows: the row's ticket counter
+  uint32_t* cand_pos = nullptr;  // prefill: [rows][ld] second slab
   uint16_t* gmax = nullptr;      // prefill: [rows][ld2] group maxima
   long long ld2 = 0;
   uint32_t* theta = nullptr;     // prefill: [rows] 16-bit bound per row
   uint32_t* tile_cnt = nullptr;  // prefill: [rows][ld / 256] takes of the run starting at each key tile
+  uint2* cand = nullptr;         // split rows: [rows][ld] (key, position) candidates, slice c at c * chunk
+  uint32_t* slot_cnt = nullptr;  // split rows: [rows][kSplitMaxSlices] candidates of each slice
 };
 
 // Finish-kernel output description.
@@ -94,25 +98,27 @@ int device_sm_count();
 // shared bytes on the current device, looked up once per (func, device).
 int device_occupancy(const void* func, int threads, size_t smem);
 
-size_t row_workspace_bytes(int rows, int Tk_max, bool with_candidates, bool with_hist);
-void carve_row_workspace(void* ws, int rows, int Tk_max, bool with_candidates, bool with_hist,
-                         RowWorkspace* out);
+// Workspace of one-query rows: error word, histograms and counters, the key
+// rows, and for split rows the candidate pairs and slice counts.
+size_t row_workspace_bytes(int rows, int Tk_max, bool split, bool with_hist);
+void carve_row_workspace(void* ws, int rows, int Tk_max, bool split, bool with_hist, RowWorkspace* out);
 
 // One query per batch row (decode / gist): keys[b][j] = key(q[b].k[b][j]) for
 // j < n_b = clamp(min(q_pos0+1, len_b), 0), plus the first-digit histogram.
 cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, int d, int Tk_max,
                                 int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w,
                                 bool with_hist, cudaStream_t st);
-cudaError_t launch_collect(int B, int Tk, int q_pos0, const int32_t* kv_len, int k,
-                           const RowWorkspace& w, cudaStream_t st);
 // Exact selection per row.  rows = B * rows_per_batch; row r is query
 // t0 + r % rows_per_batch of batch r / rows_per_batch.
 cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
                           const int32_t* kv_len, int k, const RowWorkspace& w, int mode,
                           const FinishOut& out, cudaStream_t st);
-// Candidate source for rows of Tk_max positions; sets *need_collect when the
-// collect pass must run between scoring and finish.
-int finish_mode_for(int Tk_max, bool* need_collect);
+// Selection of one-query rows of Tk_max positions: kFinishDirect or kFinishSplit.
+int finish_mode_for(int Tk_max);
+// Exact selection of one-query rows by slices: many CTAs per row filter, the
+// row's last CTA selects (the rows' histograms must come from the scorer).
+cudaError_t launch_split_topk(int B, int Tk, int q_pos0, const int32_t* kv_len, int k, const RowWorkspace& w,
+                              const FinishOut& out, cudaStream_t st);
 // Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`
 // picks what is kept per score (kScoreKeys / kScoreGroupMax / kScoreCand).
 cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,

@@ -281,6 +281,32 @@ def test_decode_attention_scale_and_repeat_calls():
         assert not ws[:4].cpu().numpy().any(), "decode workspace error word set"
 
 
+@pytest.mark.parametrize("Hq,Hkv,k", [(32, 8, 2048), (28, 4, 2048), (16, 4, 100)])
+def test_decode_attention_chained_after_an_index_run(Hq, Hkv, k):
+    """A full layer's index run, then three layers attending over its index,
+    launched back to back (each kernel may start while the one before it
+    drains).  The newest key is forced into some sequences' selection.
+    Every layer matches the oracle, and the index is unchanged."""
+    B, T, d, D = 3, 9000, 128, 128
+    qi = _ints(51, 1, (B, d))
+    ki = _ints(51, 2, (B, T, d))
+    for b in (0, 1):   # the newest key of sequences 0 and 1 is 8 x their query: selected
+        ki[b, T - 1] = ch.f32_to_bf16_bits(8.0 * ch.bf16_bits_to_f64(qi[b]))
+    ridx, rcnt = oracle.index_topk(qi[:, None, :], ki, T, T - 1, k)
+    assert T - 1 in set(ridx[0, 0].tolist()) and T - 1 in set(ridx[1, 0].tolist())
+    dev_in = [(_normals(52 + layer, 1, (B, Hq, D)), _normals(52 + layer, 2, (B, T, Hkv, D)),
+               _normals(52 + layer, 3, (B, T, Hkv, D))) for layer in range(3)]
+    dev_t = [tuple(to_dev(x) for x in trio) for trio in dev_in]
+    idx_d, cnt_d = sa.sa_index_score_topk(to_dev(qi), to_dev(ki), k, Tk=T, q_pos0=T - 1)
+    outs = [sa.sa_sparse_attn_decode(q, K, V, idx_d, cnt_d) for q, K, V in dev_t]
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx_d.cpu().numpy(), ridx[:, 0])
+    for layer, ((q, K, V), out) in enumerate(zip(dev_in, outs)):
+        ref, _ = oracle.sparse_attention_decode(q, [K[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)],
+                                                [V[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)])
+        assert_close_attn(out.float().cpu().numpy(), ref, f"layer {layer}")
+
+
 def test_decode_attention_many_sequences():
     """More (sequence, head block) pairs than CTAs: every CTA's range spans
     several pairs, some pairs are empty, and each pair has one contributor."""
@@ -479,22 +505,27 @@ def test_device_generator_matches_host_generator():
 
 def test_one_workspace_serves_calls_of_any_shape():
     """One caller-owned workspace reused by calls whose shapes grow and
-    shrink (index rows in every selection path, including rows longer than
-    the bitmap reach that take the multi-CTA collect path), then decode
+    shrink: one-query rows in every selection path (one CTA per row, slices
+    over many CTAs, 1/4-million-key rows, more rows than the fixed
+    histogram region holds) with prefill calls between them, then decode
     attention calls of varying B*Hkv on one zero-filled workspace."""
     L = sa.lib()
-    cases = [(1, 60000, 64, 100), (2, 40000, 64, 3000), (4, 20000, 128, 2048),
-             (1, 300000, 64, 2048), (3, 5000, 128, 7), (2, 270000, 128, 4096)]
-    need = max(L.sa_index_score_topk_workspace(B, 1, n, d, k) for B, n, d, k in cases)
+    # (B, rows per sequence, key rows, d, k): one-query rows of every
+    # selection path, with prefill calls (short and bounded rows) between
+    # them on the same workspace
+    cases = [(1, 1, 60000, 64, 100), (2, 1, 40000, 64, 3000), (1, 300, 300, 64, 64),
+             (4, 1, 20000, 128, 2048), (1, 1, 300000, 64, 2048), (1, 200, 9000, 64, 512),
+             (3, 1, 5000, 128, 7), (2, 1, 270000, 128, 4096), (65, 1, 6000, 64, 100)]
+    need = max(L.sa_index_score_topk_workspace(B, Tq, n, d, k) for B, Tq, n, d, k in cases)
     ws = torch.zeros(need, dtype=torch.uint8, device=dev())
-    for i, (B, n, d, k) in enumerate(cases):
-        q = _ints(900 + i, 1, (B, d))
+    for i, (B, Tq, n, d, k) in enumerate(cases):
+        q = _ints(900 + i, 1, (B, Tq, d))
         kk = _ints(900 + i, 2, (B, n, d))
         idx, cnt = sa.sa_index_score_topk(to_dev(q), to_dev(kk), k, ws=ws)
-        ridx, rcnt = oracle.index_topk(q[:, None, :], kk, n, n - 1, k)
+        ridx, rcnt = oracle.index_topk(q, kk, n, n - Tq, k)
         torch.cuda.synchronize()
-        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0], err_msg=str((B, n, d, k)))
-        np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0], err_msg=str((B, n, d, k)))
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt, err_msg=str((B, Tq, n, d, k)))
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=str((B, Tq, n, d, k)))
     acases = [(4, 8, 32, 2048), (1, 4, 28, 2048), (8, 8, 32, 512), (2, 2, 8, 100)]
     aneed = max(L.sa_sparse_attn_decode_workspace(B, Hq, Hkv, 128, k) for B, Hkv, Hq, k in acases)
     wsa = torch.zeros(aneed, dtype=torch.uint8, device=dev())
