@@ -15,6 +15,7 @@ from .reference import (  # noqa: F401
     bf16_bits_to_f64,
     n_candidates,
     index_scores,
+    index_scores_multihead,
     topk_select,
     index_topk,
     attention_over_rows,

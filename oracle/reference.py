@@ -33,6 +33,10 @@ Readings where the pages are silent (each also stated where it is used):
    unfolds each chosen chunk's raw tokens plus its own gist, then appends
    the current partial chunk; unchosen gists are left out ([SSA] §三 and §八,
    [GSA] 2.2 and the ablation in 4).
+7. The multi-head indexer (an extension beyond the pages' light indexer,
+   after DeepSeek's published lightning indexer): H indexer heads, each
+   with its own query vector and a per-query weight, score one shared key
+   per token as sum_h w_h * ReLU(q_h . k).  Selection is unchanged.
 """
 from __future__ import annotations
 
@@ -74,6 +78,21 @@ def index_scores(q_idx, k_idx) -> np.ndarray:
     return q @ k.T
 
 
+def index_scores_multihead(q_idx, w, k_idx) -> np.ndarray:
+    """Multi-head weighted indexer scores (reading 7):
+    s[t, j] = sum_h w[t, h] * max(0, q_idx[t, h] . k_idx[j]).
+
+    q_idx: [Tq, H, d]; w: [Tq, H] (per query and indexer head); k_idx:
+    [Tk, d], one key per cached token shared by every indexer head.  Returns
+    [Tq, Tk] float64 (exact integers for integer-valued inputs).
+    """
+    q = _f64(q_idx)
+    k = _f64(k_idx)
+    wt = np.asarray(w, dtype=np.float64)
+    dots = np.einsum("thd,jd->thj", q, k)
+    return np.einsum("th,thj->tj", wt, np.maximum(dots, 0.0))
+
+
 def topk_select(scores, k: int) -> np.ndarray:
     """Top-k of one query's candidate scores ([LC] "DSA 与 IndexShare": each
     query keeps only its top-k tokens; [YOIO] §1.3 token-level top-k).
@@ -91,17 +110,18 @@ def topk_select(scores, k: int) -> np.ndarray:
     return np.sort(order[: min(k, n)])
 
 
-def index_topk(q_idx, k_idx, kv_len, q_pos0: int, k: int):
+def index_topk(q_idx, k_idx, kv_len, q_pos0: int, k: int, w=None):
     """Indexer scoring plus per-query top-k for a batch.
 
-    q_idx: [B, Tq, d]; k_idx: [B, Tk_max, d]; kv_len: int or [B] cache
-    lengths; query t of batch b has n_candidates(t, q_pos0, kv_len[b])
-    candidates.  Returns (idx int32 [B, Tq, k] padded with -1,
-    count int32 [B, Tq]).
+    q_idx: [B, Tq, d] (one indexer head), or [B, Tq, H, d] with weights w
+    [B, Tq, H] (the multi-head indexer of index_scores_multihead); k_idx:
+    [B, Tk_max, d]; kv_len: int or [B] cache lengths; query t of batch b has
+    n_candidates(t, q_pos0, kv_len[b]) candidates.  Returns (idx int32
+    [B, Tq, k] padded with -1, count int32 [B, Tq]).
     """
     q_idx = np.asarray(q_idx)
     k_idx = np.asarray(k_idx)
-    B, Tq, _ = q_idx.shape
+    B, Tq = q_idx.shape[:2]
     lens = np.broadcast_to(np.asarray(kv_len, dtype=np.int64), (B,))
     idx = np.full((B, Tq, k), -1, dtype=np.int32)
     count = np.zeros((B, Tq), dtype=np.int32)
@@ -109,7 +129,10 @@ def index_topk(q_idx, k_idx, kv_len, q_pos0: int, k: int):
         n_max = n_candidates(Tq - 1, q_pos0, int(lens[b]))
         if n_max == 0:
             continue
-        s = index_scores(q_idx[b], k_idx[b, :n_max])
+        if w is None:
+            s = index_scores(q_idx[b], k_idx[b, :n_max])
+        else:
+            s = index_scores_multihead(q_idx[b], np.asarray(w)[b], k_idx[b, :n_max])
         for t in range(Tq):
             n = n_candidates(t, q_pos0, int(lens[b]))
             sel = topk_select(s[t, :n], k)

@@ -464,3 +464,101 @@ def test_prefill_batch_pin_catches_a_shared_cache(monkeypatch):
     monkeypatch.setattr(oracle, "sparse_attention", _mutant_prefill_first_cache)
     with pytest.raises(AssertionError):
         test_sparse_attention_batched_with_per_sequence_indices()
+
+
+# ------------------------------------------------------- multi-head indexer
+
+def _mh_brute(q, w, k):
+    """sum_h w[t,h] * max(0, q[t,h] . k[j]) in Python integers."""
+    Tq, H, d = q.shape
+    out = [[0] * k.shape[0] for _ in range(Tq)]
+    for t in range(Tq):
+        for j in range(k.shape[0]):
+            tot = 0
+            for h in range(H):
+                dot = sum(int(q[t, h, c]) * int(k[j, c]) for c in range(d))
+                tot += int(w[t, h]) * max(0, dot)
+            out[t][j] = tot
+    return np.array(out, dtype=np.float64)
+
+
+def test_multihead_scores_match_python_integers():
+    """The multi-head indexer (an extension of the pages' light indexer,
+    [LC] "DSA 与 IndexShare") on integer inputs equals the sum over heads
+    of weight x ReLU(dot) evaluated in Python integers."""
+    rng = _rng(31)
+    Tq, H, d, Tk = 3, 5, 7, 11
+    q = rng.integers(-4, 5, size=(Tq, H, d))
+    w = rng.integers(-3, 4, size=(Tq, H))
+    k = rng.integers(-4, 5, size=(Tk, d))
+    got = oracle.index_scores_multihead(_bf16(q), w.astype(np.float32), _bf16(k))
+    np.testing.assert_array_equal(got, _mh_brute(q, w, k))
+
+
+def test_multihead_special_cases():
+    rng = _rng(32)
+    Tq, d, Tk = 4, 16, 30
+    q1 = rng.integers(-4, 5, size=(Tq, 1, d))
+    k = rng.integers(-4, 5, size=(Tk, d))
+    plain = oracle.index_scores(_bf16(q1[:, 0]), _bf16(k))
+    # one head with weight 1 is the plain dot product clipped at zero
+    one = oracle.index_scores_multihead(_bf16(q1), np.ones((Tq, 1)), _bf16(k))
+    np.testing.assert_array_equal(one, np.maximum(plain, 0))
+    # linear in the weights; invariant to the order of the heads
+    H = 6
+    q = rng.integers(-4, 5, size=(Tq, H, d))
+    w1 = rng.integers(-3, 4, size=(Tq, H)).astype(np.float64)
+    w2 = rng.integers(-3, 4, size=(Tq, H)).astype(np.float64)
+    s = lambda ww, qq=q: oracle.index_scores_multihead(_bf16(qq), ww, _bf16(k))
+    np.testing.assert_array_equal(s(w1 + w2), s(w1) + s(w2))
+    perm = rng.permutation(H)
+    np.testing.assert_array_equal(s(w1[:, perm], q[:, perm]), s(w1))
+    # heads whose dot is negative everywhere contribute nothing
+    qn = q.copy()
+    qn[:, 0] = -1                             # head 0: q = -1 everywhere ...
+    kp = np.abs(k) + 1                        # ... against all-positive keys
+    a = oracle.index_scores_multihead(_bf16(qn), w1, _bf16(kp))
+    b = oracle.index_scores_multihead(_bf16(qn[:, 1:]), w1[:, 1:], _bf16(kp))
+    np.testing.assert_array_equal(a, b)
+
+
+def test_multihead_topk_uses_the_weighted_scores():
+    """index_topk with weights selects by the multi-head score, with the
+    same tie rule, and one head of weight 1 over non-negative dots selects
+    as the single-head indexer does."""
+    rng = _rng(33)
+    B, Tq, H, d, Tk, kk = 2, 5, 4, 8, 40, 7
+    q = rng.integers(-4, 5, size=(B, Tq, H, d))
+    w = rng.integers(0, 4, size=(B, Tq, H)).astype(np.float32)
+    k = rng.integers(-4, 5, size=(B, Tk, d))
+    idx, cnt = oracle.index_topk(_bf16(q), _bf16(k), Tk, Tk - Tq, kk, w=w)
+    for b in range(B):
+        sc = _mh_brute(q[b], w[b], k[b])
+        for t in range(Tq):
+            n = Tk - Tq + t + 1
+            order = sorted(range(n), key=lambda j: (-sc[t, j], j))[:kk]
+            np.testing.assert_array_equal(idx[b, t, :cnt[b, t]], sorted(order))
+    qa = np.abs(rng.integers(0, 5, size=(1, Tq, 1, d)))
+    ka = np.abs(rng.integers(0, 5, size=(1, Tk, d)))
+    i1, _ = oracle.index_topk(_bf16(qa), _bf16(ka), Tk, Tk - Tq, kk, w=np.ones((1, Tq, 1)))
+    i2, _ = oracle.index_topk(_bf16(qa[:, :, 0]), _bf16(ka), Tk, Tk - Tq, kk)
+    np.testing.assert_array_equal(i1, i2)
+
+
+def _mutant_mh_no_relu(q_idx, w, k_idx):
+    q = oracle.bf16_bits_to_f64(q_idx)
+    k = oracle.bf16_bits_to_f64(k_idx)
+    return np.einsum("th,thj->tj", np.asarray(w, np.float64), np.einsum("thd,jd->thj", q, k))
+
+
+def _mutant_mh_relu_after_sum(q_idx, w, k_idx):
+    q = oracle.bf16_bits_to_f64(q_idx)
+    k = oracle.bf16_bits_to_f64(k_idx)
+    return np.maximum(np.einsum("th,thj->tj", np.asarray(w, np.float64), np.einsum("thd,jd->thj", q, k)), 0)
+
+
+@pytest.mark.parametrize("mutant", [_mutant_mh_no_relu, _mutant_mh_relu_after_sum])
+def test_multihead_pin_catches_slips(monkeypatch, mutant):
+    monkeypatch.setattr(oracle, "index_scores_multihead", mutant)
+    with pytest.raises(AssertionError):
+        test_multihead_scores_match_python_integers()
