@@ -70,13 +70,14 @@ def job_rate(world: int, units_per_rank: float, ms: float) -> float:
 
 CONFIGS = {
     "decode_32k": R.DECODE_32K,
+    "decode_32k_mh": R.DECODE_32K_MH16,
     "decode_1m": R.DECODE_1M,
     "gist": R.GIST_128K,
     "prefill_2k": R.PREFILL_2K,
     "prefill_64k": R.PREFILL_64K,
 }
 # workloads reported under "workloads" beside the headline, in run order
-SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "decode_1m")
+SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "decode_1m", "decode_32k_mh")
 
 
 def load_peaks():
@@ -372,8 +373,9 @@ class DecodeBench:
             self.inp["q"][l] = TI.dev_normal((c.steps, c.B, c.Hq, c.D), seed, R.tid(R.KIND_Q, l), device)
         self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
         L = sa.lib()
-        self.ws_idx = torch.zeros(L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k),
-                                  dtype=torch.uint8, device=device)
+        ws_idx = (L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k) if c.H_idx == 1 else
+                  L.sa_index_score_topk_mh_workspace(c.B, 1, c.Tk_max, c.H_idx, c.d, c.k))
+        self.ws_idx = torch.zeros(ws_idx, dtype=torch.uint8, device=device)
         self.ws_attn = torch.zeros(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
                                    dtype=torch.uint8, device=device)
         self.out_all = torch.empty((c.n_layers, c.B, c.Hq, c.D), dtype=torch.bfloat16, device=device)
@@ -382,7 +384,7 @@ class DecodeBench:
         self.graphs_ev = {}
         self.events = {}
 
-    def step(self, s: int, ev=None, q_all=None, q_idx=None):
+    def step(self, s: int, ev=None, q_all=None, q_idx=None, w_idx=None):
         c, sa = self.cfg, self.sa
         Tk = c.N + s + 1
         self.cache.begin_step()
@@ -392,7 +394,15 @@ class DecodeBench:
                 if ev is not None:
                     ev[("idx", layer, 0)].record()
                 qi = q_idx[g] if q_idx is not None else self.inp["q_idx"][g][s]
-                self.cache.update(layer, qi, self.inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=self.ws_idx)
+                if c.H_idx == 1:
+                    self.cache.update(layer, qi, self.inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=self.ws_idx)
+                else:
+                    # the multi-head indexer writes the group's buffers itself
+                    wi = w_idx[g] if w_idx is not None else self.inp["w_idx"][g][s]
+                    sa.sa_index_score_topk_mh(qi, wi, self.inp["k_idx"][g], c.k, Tk=Tk, q_pos0=Tk - 1,
+                                              idx_out=self.cache.idx_buf, count_out=self.cache.count_buf,
+                                              ws=self.ws_idx)
+                    self.cache.mark_written(layer)
                 if ev is not None:
                     ev[("idx", layer, 1)].record()
             idx, cnt, _ = self.cache.get_tensors(layer)
@@ -468,7 +478,7 @@ class DecodeBench:
         kept rows, queries, outputs and indices)."""
         c = self.cfg
         Tk = c.N + 1
-        score_run = c.B * Tk * c.d * 2
+        score_run = c.B * Tk * c.d * 2 + c.B * c.H_idx * c.d * 2
         attn_one = c.B * c.k * c.Hkv * c.D * 2 * 2 + c.B * c.Hq * c.D * 2 * 2 + c.B * c.k * 4
         return score_run, attn_one
 
@@ -501,16 +511,19 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
     for s in range(n_steps):
         pos = c.N + s
         host[s] = {"q_idx": {g: pin(b.inp["q_idx"][g][s]) for g in b.inp["q_idx"]},
+                   "w_idx": {g: pin(b.inp["w_idx"][g][s]) for g in b.inp.get("w_idx", {})},
                    "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
                    "q": pin(torch.stack([b.inp["q"][l][s] for l in range(L)])),
                    # rows (layer, K/V, sequence) in the order of b.kv_all
                    "kv_row": pin(b.kv_all[:, :, :, pos].reshape(L * 2 * B, -1))}
     out_h = torch.empty(b.out_all.shape, dtype=b.out_all.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host[0]["q_idx"].values()) + \
+        sum(t.numel() * t.element_size() for t in host[0]["w_idx"].values()) + \
         sum(t.numel() * t.element_size() for t in host[0]["k_row"].values()) + \
         host[0]["q"].numel() * 2 + host[0]["kv_row"].numel() * 2
     d2h = out_h.numel() * out_h.element_size()
     qi_dev = {g: torch.empty_like(b.inp["q_idx"][g][0]) for g in b.inp["q_idx"]}
+    wi_dev = {g: torch.empty_like(b.inp["w_idx"][g][0]) for g in b.inp.get("w_idx", {})}
     q_all = torch.empty((L,) + tuple(b.inp["q"][0][0].shape), dtype=torch.bfloat16, device=ctx.dev)
 
     def row_copy(cache, src, pos, rows):
@@ -525,10 +538,12 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
         pos = c.N + s
         for g in h["q_idx"]:
             rt.h2d(qi_dev[g].data_ptr(), h["q_idx"][g].data_ptr(), h["q_idx"][g].numel() * 2, st)
+            if g in wi_dev:
+                rt.h2d(wi_dev[g].data_ptr(), h["w_idx"][g].data_ptr(), h["w_idx"][g].numel() * 4, st)
             row_copy(b.inp["k_idx"][g], h["k_row"][g], pos, B)
         rt.h2d(q_all.data_ptr(), h["q"].data_ptr(), h["q"].numel() * 2, st)
         row_copy(b.kv_all, h["kv_row"], pos, L * 2 * B)
-        b.step(s, q_all=q_all, q_idx=qi_dev)
+        b.step(s, q_all=q_all, q_idx=qi_dev, w_idx=wi_dev if wi_dev else None)
         rt.d2h(out_h.data_ptr(), b.out_all.data_ptr(), d2h, st)
 
     with torch.cuda.stream(st):
@@ -608,7 +623,7 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter-hash generator; integer indexer inputs, Irwin-Hall normal K/V/q)",
         "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.N, "layers": cfg.n_layers,
-                   "share_every": cfg.share_every, "d_idx": cfg.d, "q_heads": cfg.Hq,
+                   "share_every": cfg.share_every, "d_idx": cfg.d, "indexer_heads": cfg.H_idx, "q_heads": cfg.Hq,
                    "kv_heads": cfg.Hkv, "head_dim": cfg.D, "top_k": cfg.k,
                    "parallelism": f"replicas{ctx.world}",
                    "l2": _l2_note(step_bytes, resident, False),
@@ -1053,18 +1068,22 @@ class OracleDecode:
         from gen import counter_hash as ch
         self.cfg = cfg
         self.Tk = Tk = cfg.N + step + 1
-        self.k_idx, self.q_idx, self.q, self.rows = {}, {}, {}, {}
+        self.k_idx, self.q_idx, self.w_idx, self.q, self.rows = {}, {}, {}, {}, {}
         bl = list(batches)
         for g in groups:
             if bench is not None:
                 self.k_idx[g] = _bits(bench.inp["k_idx"][g][bl])
                 self.q_idx[g] = _bits(bench.inp["q_idx"][g][step][bl])
+                if cfg.H_idx > 1:
+                    self.w_idx[g] = bench.inp["w_idx"][g][step][bl].cpu().numpy()
             else:
                 n = cfg.B * cfg.Tk_max * cfg.d
                 self.k_idx[g] = ch.int_bf16(cfg.seed, R.tid(R.KIND_K_IDX, g), count=n) \
                     .reshape(cfg.B, cfg.Tk_max, cfg.d)[bl]
                 self.q_idx[g] = R.decode_q_idx_host(cfg, g, step)[bl]
-        sel = {g: oracle.index_topk(self.q_idx[g][:, None, :], self.k_idx[g], Tk, Tk - 1, cfg.k) for g in groups}
+                if cfg.H_idx > 1:
+                    self.w_idx[g] = R.decode_w_idx_host(cfg, g, step)[bl]
+        sel = {g: self._topk(g) for g in groups}
         for l in layers:
             g = l // cfg.share_every
             idx, cnt = sel[g]
@@ -1082,10 +1101,15 @@ class OracleDecode:
             self.q[l] = _bits(bench.inp["q"][l][step][bl]) if bench is not None else R.decode_q_host(cfg, l, step)[bl]
             self.rows[l] = (Kr, Vr)
 
+    def _topk(self, g):
+        import oracle
+        w = self.w_idx[g][:, None] if g in self.w_idx else None
+        return oracle.index_topk(self.q_idx[g][:, None], self.k_idx[g], self.Tk, self.Tk - 1, self.cfg.k, w=w)
+
     def run(self):
         import oracle
         for g in self.k_idx:
-            oracle.index_topk(self.q_idx[g][:, None, :], self.k_idx[g], self.Tk, self.Tk - 1, self.cfg.k)
+            self._topk(g)
         for l, (Kr, Vr) in self.rows.items():
             oracle.sparse_attention_decode(self.q[l], Kr, Vr)
 

@@ -34,6 +34,7 @@ KIND_Q_ROUTE = 6
 KIND_GIST_KEY = 7
 KIND_NEEDLE_T = 8
 KIND_NEEDLE_P = 9
+KIND_W_IDX = 10
 
 
 def tid(kind: int, index: int = 0) -> int:
@@ -74,6 +75,7 @@ class Decode:
     n_layers: int
     share_every: int
     steps: int
+    H_idx: int = 1          # indexer heads (> 1: the multi-head weighted indexer)
 
     @property
     def Tk_max(self) -> int:
@@ -118,6 +120,12 @@ GIST_128K = Gist("gist_decode_b4_128k", seed=4, B=4, n_chunks=8192, chunk_len=16
                  k_chunks=64, Hq=32, Hkv=8, D=128, steps=16)
 DECODE_1M = Decode("decode_1m_28layers", seed=5, B=1, N=1 << 20, d=64, Hq=28, Hkv=4, D=128,
                    k=2048, n_layers=28, share_every=4, steps=16)
+
+# The batch-8 decode step with a 16-head weighted indexer (sum over heads of
+# weight x ReLU(q_h . k), integer weights in [-3, 3]) in place of the one-head
+# dot product.
+DECODE_32K_MH16 = Decode("decode_b8_32k_4layers_idx16heads", seed=6, B=8, N=32768, d=128, Hq=32, Hkv=8,
+                         D=128, k=2048, n_layers=4, share_every=4, steps=64, H_idx=16)
 
 ALL = [PREFILL_2K, DECODE_32K, PREFILL_64K, GIST_128K, DECODE_1M]
 
@@ -210,8 +218,17 @@ def prefill_host_inputs(cfg: Prefill, with_attention: bool = True) -> dict:
 
 
 def decode_q_idx_host(cfg: Decode, g: int, step: int) -> np.ndarray:
-    n = cfg.B * cfg.d
-    return _ints(cfg.seed, tid(KIND_Q_IDX, g), n, start=step * n).reshape(cfg.B, cfg.d)
+    """[B, d], or [B, H_idx, d] for a multi-head indexer."""
+    n = cfg.B * cfg.H_idx * cfg.d
+    q = _ints(cfg.seed, tid(KIND_Q_IDX, g), n, start=step * n)
+    return q.reshape(cfg.B, cfg.d) if cfg.H_idx == 1 else q.reshape(cfg.B, cfg.H_idx, cfg.d)
+
+
+def decode_w_idx_host(cfg: Decode, g: int, step: int) -> np.ndarray:
+    """Multi-head indexer weights [B, H_idx] (float32 integers in [-3, 3])."""
+    n = cfg.B * cfg.H_idx
+    bits = ch.int_bf16(cfg.seed, tid(KIND_W_IDX, g), start=step * n, count=n, lo=-3, hi=3)
+    return ch.bf16_bits_to_f64(bits).astype(np.float32).reshape(cfg.B, cfg.H_idx)
 
 
 def decode_q_host(cfg: Decode, layer: int, step: int) -> np.ndarray:

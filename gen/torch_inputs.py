@@ -38,9 +38,17 @@ def decode_inputs(cfg: R.Decode, device, layers=None, groups=None):
     groups = range(cfg.n_groups) if groups is None else groups
     s = cfg.seed
     out = {"k_idx": {}, "q_idx": {}, "K": {}, "V": {}, "q": {}}
+    if cfg.H_idx > 1:
+        out["w_idx"] = {}
     for g in groups:
         out["k_idx"][g] = dev_int((cfg.B, cfg.Tk_max, cfg.d), s, R.tid(R.KIND_K_IDX, g), device)
-        out["q_idx"][g] = dev_int((cfg.steps, cfg.B, cfg.d), s, R.tid(R.KIND_Q_IDX, g), device)
+        if cfg.H_idx == 1:
+            out["q_idx"][g] = dev_int((cfg.steps, cfg.B, cfg.d), s, R.tid(R.KIND_Q_IDX, g), device)
+        else:
+            out["q_idx"][g] = dev_int((cfg.steps, cfg.B, cfg.H_idx, cfg.d), s, R.tid(R.KIND_Q_IDX, g), device)
+            wb = torch.empty((cfg.steps, cfg.B, cfg.H_idx), dtype=torch.bfloat16, device=device)
+            gd.fill_int(wb, s, R.tid(R.KIND_W_IDX, g), 0, lo=-3, hi=3)
+            out["w_idx"][g] = wb.float()
     for l in layers:
         out["K"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_K, l), device)
         out["V"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_V, l), device)

@@ -120,6 +120,31 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx,
                               void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Multi-head weighted indexer scoring + per-query top-k.
+ *
+ * A wider score function for the same selection ([LC] "DSA 与 IndexShare"
+ * names only a light indexer; this is the multi-head form of DeepSeek's
+ * published lightning indexer): H indexer heads, each with its own query
+ * vector and weight, score one shared key per cached token as
+ *     s = sum_h w[b,t,h] * max(0, q_idx[b,t,h,:] . k_idx[b,j,:]),
+ * accumulated in fp32 (exact for integer-valued inputs with every partial
+ * sum below 2^24).  Candidates, tie rule, output order, kv_len, q_pos0,
+ * score_out and the error word are exactly as for sa_index_score_topk.
+ *
+ *   q_idx  [B, Tq, H, d] bf16;   w [B, Tq, H] fp32;   k_idx [B, Tk_max, d] bf16
+ *   ws     >= sa_index_score_topk_mh_workspace(...) bytes (zero-filled
+ *          before first use; see the conventions above)
+ * Supported: d in {64, 128}; 1 <= H <= 64 (d = 64) or 32 (d = 128);
+ * 1 <= k <= SA_MAX_K.
+ * ---------------------------------------------------------------------- */
+size_t sa_index_score_topk_mh_workspace(int B, int Tq, int Tk_max, int H, int d, int k);
+sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* k_idx,
+                                 int B, int Tq, int H, int Tk, int Tk_max, int d, int k,
+                                 int q_pos0, const int32_t* kv_len,
+                                 int32_t* idx_out, int32_t* count_out, float* score_out,
+                                 void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Gathered sparse attention, prefill (one call per layer).
  *
  * [YOIO] §1.1: Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V; §2.3: each

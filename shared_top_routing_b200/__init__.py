@@ -16,6 +16,7 @@ from .sa import (  # noqa: F401
     lib,
     sa_gist_route_unfold,
     sa_index_score_topk,
+    sa_index_score_topk_mh,
     sa_sparse_attn_decode,
     sa_sparse_attn_prefill,
 )
@@ -32,6 +33,7 @@ __all__ = [
     "lib",
     "sa_gist_route_unfold",
     "sa_index_score_topk",
+    "sa_index_score_topk_mh",
     "sa_sparse_attn_decode",
     "sa_sparse_attn_prefill",
 ]

@@ -233,7 +233,7 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
     if ((e = sa::launch_score_decode(q, km, B, d, Tk_max, Tk, q_pos0, kv_len, w, hist, cs)) != cudaSuccess)
       return cuda_fail(e, "score_decode launch");
     if (mode == sa::kFinishSplit) {
-      if ((e = sa::launch_split_topk(B, Tk, q_pos0, kv_len, k, w, out, cs)) != cudaSuccess)
+      if ((e = sa::launch_split_topk(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, out, cs)) != cudaSuccess)
         return cuda_fail(e, "split top-k launch");
     } else if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, mode, out, cs)) != cudaSuccess) {
       return cuda_fail(e, "finish launch");
@@ -267,6 +267,61 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
       if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, w, sa::kFinishCandRows, out, cs)) !=
           cudaSuccess)
         return cuda_fail(e, "finish launch");
+    }
+  }
+  return ok();
+}
+
+// --------------------------------------------------- multi-head indexer
+
+size_t sa_index_score_topk_mh_workspace(int B, int Tq, int Tk_max, int H, int d, int k) {
+  (void)d;
+  (void)k;
+  if (B <= 0 || Tq <= 0 || Tk_max < 0 || H < 1) return 0;
+  const int rows = sa::mh_rows_per_launch(B, Tq, Tk_max);
+  return sa::row_workspace_bytes(B * rows, Tk_max, true, true);
+}
+
+sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* k_idx, int B, int Tq, int H,
+                                 int Tk, int Tk_max, int d, int k, int q_pos0, const int32_t* kv_len,
+                                 int32_t* idx_out, int32_t* count_out, float* score_out, void* ws,
+                                 size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = validate_index(q_idx, k_idx, B, Tq, Tk, Tk_max, d, k, idx_out, count_out);
+  if (st != SA_OK) return st;
+  if (H < 1) return fail(SA_ERR_INVALID_ARG, "H=%d must be >= 1", H);
+  if (H > sa::mh_max_heads(d))
+    return fail(SA_ERR_UNSUPPORTED, "H=%d indexer heads exceed %d for d=%d", H, sa::mh_max_heads(d), d);
+  if (B == 0) return ok();
+  if (w == nullptr) return fail(SA_ERR_INVALID_ARG, "NULL weight pointer");
+  if (!aligned(w, 4)) return fail(SA_ERR_INVALID_ARG, "w must be 4-byte aligned");
+  const size_t need = sa_index_score_topk_mh_workspace(B, Tq, Tk_max, H, d, k);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
+  cudaStream_t cs = as_cuda(stream);
+  const int rows = sa::mh_rows_per_launch(B, Tq, Tk_max);
+  sa::RowWorkspace wsp;
+  sa::carve_row_workspace(ws, B * rows, Tk_max, true, true, &wsp);
+  cudaError_t e;
+  if (wsp.hist_zero_bytes && (e = cudaMemsetAsync(wsp.hist, 0, wsp.hist_zero_bytes, cs)) != cudaSuccess)
+    return cuda_fail(e, "memset");
+  sa::FinishOut out;
+  out.idx = idx_out;
+  out.count = count_out;
+  out.score = score_out;
+  const uint16_t* q = static_cast<const uint16_t*>(q_idx);
+  const uint16_t* km = static_cast<const uint16_t*>(k_idx);
+  for (int t0 = 0; t0 < Tq; t0 += rows) {
+    const int nr = (Tq - t0 < rows) ? Tq - t0 : rows;
+    const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + t0 + nr);
+    const bool split = n_max > sa::kDirectMaxCand;   // short rows: one CTA holds the whole row
+    if ((e = sa::launch_score_mh(q, w, km, B, H, d, nr, t0, Tq, Tk_max, Tk, q_pos0, kv_len, wsp, split, cs)) !=
+        cudaSuccess)
+      return cuda_fail(e, "multi-head score launch");
+    if (split) {
+      if ((e = sa::launch_split_topk(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, wsp, out, cs)) != cudaSuccess)
+        return cuda_fail(e, "split top-k launch");
+    } else if ((e = sa::launch_finish(B, nr, t0, Tq, Tk, q_pos0, kv_len, k, wsp, sa::kFinishDirect, out, cs)) !=
+               cudaSuccess) {
+      return cuda_fail(e, "finish launch");
     }
   }
   return ok();
@@ -365,7 +420,7 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   out.partial_len = partial_len;
   out.chunks = chunks_out;
   if (mode == sa::kFinishSplit) {
-    if ((e = sa::launch_split_topk(B, n_chunks, q_pos0, nullptr, k_chunks, w, out, cs)) != cudaSuccess)
+    if ((e = sa::launch_split_topk(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, out, cs)) != cudaSuccess)
       return cuda_fail(e, "gist split top-k launch");
   } else if ((e = sa::launch_finish(B, 1, 0, 1, n_chunks, q_pos0, nullptr, k_chunks, w, mode, out, cs)) !=
              cudaSuccess) {

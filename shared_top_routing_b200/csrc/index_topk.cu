@@ -179,6 +179,134 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
   }
 }
 
+// -------------------------------------------------------- multi-head scoring
+//
+// score_mh_kernel: the multi-head weighted indexer, s = sum_h w_h *
+// ReLU(q_h . k), for rows that each carry their own H query vectors and
+// weights (one row per decode sequence, or per prefill query) against the
+// key cache of their sequence.  The key cache is streamed as in
+// score_decode_kernel (16-byte loads straight into mma.sync B fragments,
+// two register buffers of 8-row tiles); the 16-row A side holds 16 indexer
+// heads (rows g and g+8 of a lane's fragment are heads 16 hg + g and 16 hg
+// + g + 8 of head group hg), so one m16n8k16 per 16 dimensions scores every
+// head of a group at once.  The epilogue takes weight x ReLU per head and
+// sums over heads with three shuffles; integer-valued inputs keep every
+// partial sum an exact fp32 integer.  Grid: (key chunks, rows); each CTA
+// scores one chunk of one row, writes the keys and adds its 4096-bin
+// histogram of their top 12 bits to the row's.
+
+template <int D, int HG>
+__global__ void __launch_bounds__(kScoreThreads)
+score_mh_kernel(const uint16_t* __restrict__ q, const float* __restrict__ wts, const uint16_t* __restrict__ kmat,
+                int H, int rows_per_batch, int t0, int Tq, int Tk_max, int Tk, int q_pos0,
+                const int32_t* __restrict__ kv_len, int chunk, uint32_t* __restrict__ keys, long long ld,
+                uint32_t* __restrict__ hist) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int J = D / 32;          // 16-byte chunks per lane per key row
+  constexpr int U = 2;               // 8-row tiles per register buffer (two buffers)
+  constexpr int WARPS = kScoreThreads / 32;
+  __shared__ uint32_t sh[kHistBins];
+  const int r = blockIdx.y;
+  const int b = r / rows_per_batch, t = t0 + r % rows_per_batch;
+  const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
+  const int r0 = blockIdx.x * chunk;
+  if (r0 >= n) return;
+  const int r1 = min(n, r0 + chunk);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tg = lane & 3;
+  if (hist != nullptr) {
+    for (int i = tid; i < kHistBins; i += kScoreThreads) sh[i] = 0;
+    __syncthreads();
+  }
+
+  // query fragments: for k-step pair j, lane (g, tg) holds dims of chunk
+  // 4j + tg of heads 16hg + g (A rows g) and 16hg + g + 8 (A rows g + 8)
+  const long long qrow = (long long)b * Tq + t;
+  const uint16_t* qr = q + qrow * H * D;
+  uint32_t qe[HG][J][4], qo[HG][J][4];
+  float w0[HG], w1[HG];
+#pragma unroll
+  for (int hg = 0; hg < HG; ++hg) {
+    const int h0 = 16 * hg + g, h1 = h0 + 8;
+    w0[hg] = h0 < H ? wts[qrow * H + h0] : 0.f;
+    w1[hg] = h1 < H ? wts[qrow * H + h1] : 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+      if (h0 < H) v0 = *reinterpret_cast<const uint4*>(qr + (long long)h0 * D + (4 * j + tg) * 8);
+      if (h1 < H) v1 = *reinterpret_cast<const uint4*>(qr + (long long)h1 * D + (4 * j + tg) * 8);
+      qe[hg][j][0] = v0.x; qe[hg][j][1] = v1.x; qe[hg][j][2] = v0.y; qe[hg][j][3] = v1.y;
+      qo[hg][j][0] = v0.z; qo[hg][j][1] = v1.z; qo[hg][j][2] = v0.w; qo[hg][j][3] = v1.w;
+    }
+  }
+  const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
+  uint32_t* kout = keys + (long long)r * ld;
+  auto load = [&](uint4 (&v)[U][J], int base) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int row = base + u * 8 + g;
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+        v[u][j] = row < r1 ? __ldg(kb + (long long)row * (D / 8) + 4 * j + tg) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto score = [&](const uint4 (&v)[U][J], int base) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float s0 = 0.f, s1 = 0.f;   // keys 2tg and 2tg+1 of the tile: this lane's heads
+#pragma unroll
+      for (int hg = 0; hg < HG; ++hg) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          mma_bf16_16816(c, qe[hg][j], v[u][j].x, v[u][j].y);
+          mma_bf16_16816(c, qo[hg][j], v[u][j].z, v[u][j].w);
+        }
+        s0 = fmaf(w0[hg], fmaxf(c[0], 0.f), s0);
+        s0 = fmaf(w1[hg], fmaxf(c[2], 0.f), s0);
+        s1 = fmaf(w0[hg], fmaxf(c[1], 0.f), s1);
+        s1 = fmaf(w1[hg], fmaxf(c[3], 0.f), s1);
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {   // sum over g: the lanes sharing tg
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      }
+      if (g == 0) {
+        const int row = base + u * 8 + 2 * tg;
+        const uint32_t k0 = score_key(s0), k1 = score_key(s1);
+        if (row < r1) {
+          kout[row] = k0;
+          if (hist != nullptr) atomicAdd(&sh[k0 >> (32 - kHistBits)], 1u);
+        }
+        if (row + 1 < r1) {
+          kout[row + 1] = k1;
+          if (hist != nullptr) atomicAdd(&sh[k1 >> (32 - kHistBits)], 1u);
+        }
+      }
+    }
+  };
+  constexpr int kStep = WARPS * 8 * U;
+  uint4 va[U][J], vb[U][J];
+  int base = r0 + warp * 8 * U;
+  if (base < r1) load(va, base);
+  for (; base < r1; base += 2 * kStep) {
+    if (base + kStep < r1) load(vb, base + kStep);
+    score(va, base);
+    if (base + kStep >= r1) break;
+    if (base + 2 * kStep < r1) load(va, base + 2 * kStep);
+    score(vb, base + kStep);
+  }
+  if (hist == nullptr) return;
+  __syncthreads();
+  uint32_t* hg_row = hist + (long long)r * kHistStride;
+  for (int i = tid; i < kHistBins; i += kScoreThreads) {
+    const uint32_t cnt = sh[i];
+    if (cnt) atomicAdd(hg_row + i, cnt);
+  }
+}
+
 // ------------------------------------------------------------ block scans
 
 // Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
@@ -979,16 +1107,17 @@ __device__ __forceinline__ void hist_threshold_v(const uint32_t* __restrict__ h,
 }
 
 __global__ void __launch_bounds__(kSplitThreads)
-split_topk_kernel(RowWorkspace w, int Tk, int q_pos0, const int32_t* __restrict__ kv_len, int k, int chunk,
-                  FinishOut out) {
+split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+                  const int32_t* __restrict__ kv_len, int k, int chunk, FinishOut out) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SplitSmem& s = *reinterpret_cast<SplitSmem*>(smem_raw);
   const int c = blockIdx.x, F = gridDim.x, r = blockIdx.y;
-  const int b = r;
+  const int b = r / rows_per_batch;
+  const int t = t0 + r % rows_per_batch;
   const int tid = threadIdx.x;
-  const int n = n_cand(q_pos0, 0, row_len(kv_len, b, Tk));
+  const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
   // a wait in an earlier kernel of this call that gave up: failure sentinel
   const bool failed = w.err != nullptr && *reinterpret_cast<volatile const int*>(w.err) != 0;
   const uint32_t K = failed ? 0u : (uint32_t)min(k, n);
@@ -1050,7 +1179,7 @@ split_topk_kernel(RowWorkspace w, int Tk, int q_pos0, const int32_t* __restrict_
   }
   __syncthreads();
   const bool in_smem = total <= (uint32_t)kSplitCand;
-  const long long o_idx = (long long)b * k;
+  const long long o_idx = ((long long)b * Tq + t) * (long long)k;
   if (K > 0) {
     // gathered candidate i belongs to the last slice whose first index is <= i
     auto fetch = [&](uint32_t i) {
@@ -1216,7 +1345,7 @@ split_topk_kernel(RowWorkspace w, int Tk, int q_pos0, const int32_t* __restrict_
       }
     }
   }
-  finish_tail(out, b, 0, 1, k, K, failed, tid, kSplitThreads);
+  finish_tail(out, b, t, Tq, k, K, failed, tid, kSplitThreads);
 
   // ---- 3. every CTA of the row has used the histograms: return them and
   // the ticket to zero for the next call
@@ -1332,13 +1461,16 @@ int finish_mode_for(int Tk_max) {
   return Tk_max <= kDirectMaxCand ? kFinishDirect : kFinishSplit;
 }
 
-cudaError_t launch_split_topk(int B, int Tk, int q_pos0, const int32_t* kv_len, int k, const RowWorkspace& w,
-                              const FinishOut& out, cudaStream_t st) {
-  if (B <= 0) return cudaSuccess;
+cudaError_t launch_split_topk(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+                              const int32_t* kv_len, int k, const RowWorkspace& w, const FinishOut& out,
+                              cudaStream_t st) {
+  const int rows = B * rows_per_batch;
+  if (rows <= 0) return cudaSuccess;
   // slices of a multiple of kSplitSlice positions: about two CTAs per SM over
   // all rows, at most kSplitMaxSlices per row
-  const long long n_max = std::max<long long>(1, std::min<long long>(Tk, (long long)q_pos0 + 1));
-  const long long target = std::max<long long>(1, 2LL * device_sm_count() / B);
+  const long long n_max =
+      std::max<long long>(1, std::min<long long>(Tk, (long long)q_pos0 + t0 + rows_per_batch));
+  const long long target = std::max<long long>(1, 2LL * device_sm_count() / rows);
   long long chunk = (n_max + target - 1) / target;
   const long long floor_chunk = (n_max + kSplitMaxSlices - 1) / kSplitMaxSlices;
   chunk = std::max(chunk, floor_chunk);
@@ -1347,8 +1479,50 @@ cudaError_t launch_split_topk(int B, int Tk, int q_pos0, const int32_t* kv_len, 
   const size_t smem = sizeof(SplitSmem);
   cudaError_t e = ensure_dynamic_smem((const void*)split_topk_kernel, smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(split_topk_kernel, dim3((unsigned)F, (unsigned)B), dim3(kSplitThreads), smem, st, w, Tk, q_pos0,
-                 kv_len, k, (int)chunk, out);
+  e = launch_pdl(split_topk_kernel, dim3((unsigned)F, (unsigned)rows), dim3(kSplitThreads), smem, st, w,
+                 rows_per_batch, t0, Tq, Tk, q_pos0, kv_len, k, (int)chunk, out);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+int mh_rows_per_launch(int B, int Tq, int Tk_max) {
+  // keys (4 B) and candidate pairs (8 B) per position of every row: at most
+  // about 1 GiB per launch
+  long long cap = (1ll << 30) / (12ll * row_ld(Tk_max) * (B > 0 ? B : 1));
+  if (cap > 64) cap = cap / 64 * 64;
+  if (cap < 1) cap = 1;
+  if (cap > Tq) cap = Tq;
+  return (int)cap;
+}
+
+cudaError_t launch_score_mh(const uint16_t* q, const float* wts, const uint16_t* kmat, int B, int H, int d,
+                            int rows_per_batch, int t0, int Tq, int Tk_max, int Tk, int q_pos0,
+                            const int32_t* kv_len, const RowWorkspace& w, bool with_hist, cudaStream_t st) {
+  uint32_t* hist = with_hist ? w.hist : nullptr;
+  const int rows = B * rows_per_batch;
+  if (rows <= 0 || Tk <= 0) return cudaSuccess;
+  const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + t0 + rows_per_batch);
+  if (n_max <= 0) return cudaSuccess;
+  // chunks of a multiple of 256 keys: about two CTAs per SM over all rows
+  const long long target = std::max<long long>(1, 2LL * device_sm_count() / rows);
+  long long chunk = (n_max + target - 1) / target;
+  chunk = std::max<long long>(256, (chunk + 255) / 256 * 256);
+  const unsigned gx = (unsigned)((n_max + chunk - 1) / chunk);
+  const dim3 grid(gx, (unsigned)rows);
+  const int hg = (H + 15) / 16;
+  cudaError_t e;
+#define SA_MH_LAUNCH(DD, GG)                                                                                  \
+  e = launch_pdl(score_mh_kernel<DD, GG>, grid, dim3(kScoreThreads), 0, st, q, wts, kmat, H, rows_per_batch, t0, \
+                 Tq, Tk_max, Tk, q_pos0, kv_len, (int)chunk, w.keys, w.ld, hist)
+  if (d == 128) {
+    if (hg == 1) SA_MH_LAUNCH(128, 1);
+    else SA_MH_LAUNCH(128, 2);
+  } else {
+    if (hg == 1) SA_MH_LAUNCH(64, 1);
+    else if (hg == 2) SA_MH_LAUNCH(64, 2);
+    else if (hg == 3) SA_MH_LAUNCH(64, 3);
+    else SA_MH_LAUNCH(64, 4);
+  }
+#undef SA_MH_LAUNCH
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -117,8 +117,18 @@ cudaError_t launch_finish(int B, int rows_per_batch, int t0, int Tq, int Tk, int
 int finish_mode_for(int Tk_max);
 // Exact selection of one-query rows by slices: many CTAs per row filter, the
 // row's last CTA selects (the rows' histograms must come from the scorer).
-cudaError_t launch_split_topk(int B, int Tk, int q_pos0, const int32_t* kv_len, int k, const RowWorkspace& w,
-                              const FinishOut& out, cudaStream_t st);
+cudaError_t launch_split_topk(int B, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
+                              const int32_t* kv_len, int k, const RowWorkspace& w, const FinishOut& out,
+                              cudaStream_t st);
+// Multi-head weighted indexer: rows per launch (B * rows rows at once) and
+// the scoring of queries [t0, t0 + rows_per_batch) of every sequence into
+// the keys and histograms of a split-row workspace.
+int mh_rows_per_launch(int B, int Tq, int Tk_max);
+cudaError_t launch_score_mh(const uint16_t* q, const float* wts, const uint16_t* kmat, int B, int H, int d,
+                            int rows_per_batch, int t0, int Tq, int Tk_max, int Tk, int q_pos0,
+                            const int32_t* kv_len, const RowWorkspace& w, bool with_hist, cudaStream_t st);
+// Largest number of indexer heads of the multi-head indexer for key width d.
+constexpr int mh_max_heads(int d) { return d == 64 ? 64 : 32; }
 // Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`
 // picks what is kept per score (kScoreKeys / kScoreGroupMax / kScoreCand).
 cudaError_t launch_score_prefill(const uint16_t* q, const uint16_t* kmat, int B, int Tq, int d,

@@ -37,6 +37,8 @@ SIGNATURES = {
     "sa_version": (_I, []),
     "sa_index_score_topk_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_index_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "sa_index_score_topk_mh_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sa_index_score_topk_mh": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
@@ -177,6 +179,45 @@ def sa_index_score_topk(q_idx, k_idx, k: int, Tk: int | None = None, q_pos0: int
                                    _ptr(kv_len), _ptr(idx_out), _ptr(count_out), _ptr(score),
                                    _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "sa_index_score_topk")
+    if decode_shape:
+        idx_v, cnt_v = idx_out.view(B, k), count_out.view(B)
+        return (idx_v, cnt_v, score.view(B, k)) if with_scores else (idx_v, cnt_v)
+    return (idx_out, count_out, score) if with_scores else (idx_out, count_out)
+
+
+def sa_index_score_topk_mh(q_idx, w, k_idx, k: int, Tk: int | None = None, q_pos0: int | None = None,
+                           kv_len=None, idx_out=None, count_out=None, with_scores: bool = False,
+                           ws=None, stream=None):
+    """Multi-head weighted indexer scores + per-query top-k (see sa.h).
+
+    q_idx [B, Tq, H, d] or [B, H, d] (decode) bf16; w [B, Tq, H] or [B, H]
+    fp32; k_idx [B, Tk_max, d] bf16.  Defaults and results as for
+    sa_index_score_topk.
+    """
+    torch = _torch()
+    decode_shape = q_idx.dim() == 3
+    q4 = q_idx.unsqueeze(1) if decode_shape else q_idx
+    w3 = w.unsqueeze(1) if decode_shape else w
+    B, Tq, H, d = q4.shape
+    Tk_max = k_idx.shape[1]
+    Tk = Tk_max if Tk is None else Tk
+    q_pos0 = Tk - Tq if q_pos0 is None else q_pos0
+    _need(q4, "q_idx", 2)
+    _need(w3, "w", 4)
+    _need(k_idx, "k_idx", 2)
+    dev = q4.device
+    if idx_out is None:
+        idx_out = torch.empty((B, Tq, k), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((B, Tq), dtype=torch.int32, device=dev)
+    score = torch.empty((B, Tq, k), dtype=torch.float32, device=dev) if with_scores else None
+    need = lib().sa_index_score_topk_mh_workspace(B, Tq, Tk_max, H, d, k)
+    if ws is None:
+        ws = workspace(need, dev, "index_mh", stream)
+    st = lib().sa_index_score_topk_mh(_ptr(q4), _ptr(w3), _ptr(k_idx), B, Tq, H, Tk, Tk_max, d, k, q_pos0,
+                                      _ptr(kv_len), _ptr(idx_out), _ptr(count_out), _ptr(score),
+                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "sa_index_score_topk_mh")
     if decode_shape:
         idx_v, cnt_v = idx_out.view(B, k), count_out.view(B)
         return (idx_v, cnt_v, score.view(B, k)) if with_scores else (idx_v, cnt_v)

@@ -5,6 +5,8 @@ every fp32 score exact); attention outputs must be within max-abs 2e-2 and
 mean-abs 2e-3 of the fp64 oracle.  Sizes span several tiles and ragged
 tails; edge cases cover empty rows, k >= candidates, all-equal and signed-zero
 scores, heavy ties and the candidate-overflow fallback."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -233,6 +235,77 @@ def test_prefill_topk_real_valued_scores():
 
 
 # ----------------------------------------------------------------- attention
+
+# ------------------------------------------------------ multi-head indexer
+
+def _weights(seed, shape, lo=-3, hi=3):
+    rng = np.random.default_rng(seed)
+    return rng.integers(lo, hi + 1, size=shape).astype(np.float32)
+
+
+@pytest.mark.parametrize("d,H", [(64, 1), (64, 4), (64, 16), (64, 33), (64, 64), (128, 8), (128, 32)])
+@pytest.mark.parametrize("lens,Tk_max,k", [([3000, 1700], 3000, 256), ([40000, 9000, 20000], 40000, 2048)])
+def test_decode_multihead_topk_matches_oracle(d, H, lens, Tk_max, k):
+    """Multi-head weighted indexer (sum over heads of weight x ReLU(q_h . k)),
+    one query per sequence: indices and counts bit-exact against the oracle
+    (integer inputs and weights keep every fp32 partial sum exact), with
+    per-sequence lengths, head counts that fill one to four 16-head groups
+    and negative weights."""
+    B = len(lens)
+    seed = 700 + d + H
+    q = _ints(seed, 1, (B, H, d))
+    w = _weights(seed, (B, H))
+    kk = _ints(seed, 2, (B, Tk_max, d))
+    idx, cnt, sc = sa.sa_index_score_topk_mh(to_dev(q), torch.from_numpy(w).to(dev()), to_dev(kk), k, Tk=Tk_max,
+                                             q_pos0=Tk_max - 1, kv_len=i32(lens), with_scores=True)
+    ridx, rcnt = oracle.index_topk(q[:, None], kk, np.array(lens), Tk_max - 1, k, w=w[:, None])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0])
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
+    # the reported scores are the oracle's scores of the chosen positions
+    sc = sc.cpu().numpy()
+    for b, n in enumerate(lens):
+        ref = oracle.index_scores_multihead(q[b][None], w[b][None], kk[b, :n])[0]
+        c = rcnt[b, 0]
+        np.testing.assert_array_equal(sc[b, :c], ref[ridx[b, 0, :c]])
+
+
+@pytest.mark.parametrize("d,H,B,L,k", [(64, 16, 2, 300, 64), (128, 8, 1, 2500, 256), (64, 3, 1, 5000, 512)])
+def test_prefill_multihead_topk_matches_oracle(d, H, B, L, k):
+    """Causal prefill rows with the multi-head indexer: short rows (one CTA
+    per row) and rows over 4096 candidates (slices over many CTAs)."""
+    seed = 800 + d + H + L
+    q = _ints(seed, 1, (B, L, H, d))
+    w = _weights(seed, (B, L, H))
+    kk = _ints(seed, 2, (B, L, d))
+    idx, cnt = sa.sa_index_score_topk_mh(to_dev(q), torch.from_numpy(w).to(dev()), to_dev(kk), k)
+    ridx, rcnt = oracle.index_topk(q, kk, L, 0, k, w=w)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
+def test_multihead_topk_ties_and_bad_arguments():
+    """Zero weights make every score 0: the lowest positions win.  Head
+    counts beyond the supported maximum and a missing weight pointer are
+    refused on the host."""
+    B, H, d, T, k = 2, 5, 64, 9000, 1000
+    q = _ints(77, 1, (B, H, d))
+    kk = _ints(77, 2, (B, T, d))
+    w = torch.zeros((B, H), dtype=torch.float32, device=dev())
+    idx, cnt = sa.sa_index_score_topk_mh(to_dev(q), w, to_dev(kk), k, Tk=T, q_pos0=T - 1)
+    torch.cuda.synchronize()
+    assert (cnt.cpu().numpy() == k).all()
+    np.testing.assert_array_equal(idx.cpu().numpy(), np.tile(np.arange(k, dtype=np.int32), (B, 1)))
+    L = sa.lib()
+    fake = ctypes.c_void_p(0x100000)
+    assert L.sa_index_score_topk_mh(fake, fake, fake, 1, 1, 65, 10, 10, 64, 4, 9, None, fake, fake, None,
+                                    fake, 1 << 30, None) == sa.SA_ERR_UNSUPPORTED
+    assert L.sa_index_score_topk_mh(fake, fake, fake, 1, 1, 33, 10, 10, 128, 4, 9, None, fake, fake, None,
+                                    fake, 1 << 30, None) == sa.SA_ERR_UNSUPPORTED
+    assert L.sa_index_score_topk_mh(fake, None, fake, 1, 1, 4, 10, 10, 64, 4, 9, None, fake, fake, None,
+                                    fake, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
+
 
 def _random_index(rng, B, Tk_max, k, counts):
     idx = np.full((B, k), -1, np.int32)

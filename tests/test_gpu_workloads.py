@@ -30,8 +30,10 @@ def _check_decode(cfg, steps, check_groups, check_layers):
     d = dev()
     inp = TI.decode_inputs(cfg, d)
     cache = sa.IndexCache(cfg.n_layers, cfg.B, 1, cfg.k, share_every=cfg.share_every, device=d)
-    ws_idx = torch.zeros(sa.lib().sa_index_score_topk_workspace(cfg.B, 1, cfg.Tk_max, cfg.d, cfg.k),
-                         dtype=torch.uint8, device=d)
+    L = sa.lib()
+    ws_bytes = (L.sa_index_score_topk_workspace(cfg.B, 1, cfg.Tk_max, cfg.d, cfg.k) if cfg.H_idx == 1 else
+                L.sa_index_score_topk_mh_workspace(cfg.B, 1, cfg.Tk_max, cfg.H_idx, cfg.d, cfg.k))
+    ws_idx = torch.zeros(ws_bytes, dtype=torch.uint8, device=d)
     outs = [torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=d) for _ in range(cfg.n_layers)]
     host_k = {g: ch.int_bf16(cfg.seed, R.tid(R.KIND_K_IDX, g), count=cfg.B * cfg.Tk_max * cfg.d)
               .reshape(cfg.B, cfg.Tk_max, cfg.d) for g in check_groups}
@@ -44,7 +46,13 @@ def _check_decode(cfg, steps, check_groups, check_layers):
         for layer in range(cfg.n_layers):
             g = layer // cfg.share_every
             if cache.is_full(layer) == 1:
-                cache.update(layer, inp["q_idx"][g][s], inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=ws_idx)
+                if cfg.H_idx == 1:
+                    cache.update(layer, inp["q_idx"][g][s], inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=ws_idx)
+                else:
+                    sa.sa_index_score_topk_mh(inp["q_idx"][g][s], inp["w_idx"][g][s], inp["k_idx"][g], cfg.k,
+                                              Tk=Tk, q_pos0=Tk - 1, idx_out=cache.idx_buf,
+                                              count_out=cache.count_buf, ws=ws_idx)
+                    cache.mark_written(layer)
                 versions[g] = None
             idx, cnt, ver = cache.get_tensors(layer)
             versions[g] = ver if versions[g] is None else versions[g]
@@ -58,7 +66,8 @@ def _check_decode(cfg, steps, check_groups, check_layers):
         torch.cuda.synchronize()
         for g in check_groups:
             qi = R.decode_q_idx_host(cfg, g, s)
-            ridx, rcnt = oracle.index_topk(qi[:, None, :], host_k[g], Tk, Tk - 1, cfg.k)
+            wi = R.decode_w_idx_host(cfg, g, s)[:, None] if cfg.H_idx > 1 else None
+            ridx, rcnt = oracle.index_topk(qi[:, None], host_k[g], Tk, Tk - 1, cfg.k, w=wi)
             gi, gc = got_idx[g]
             np.testing.assert_array_equal(gc.cpu().numpy(), rcnt[:, 0])
             np.testing.assert_array_equal(gi.cpu().numpy(), ridx[:, 0])
@@ -86,6 +95,12 @@ def test_decode_32k_batch8_four_layers_share_one_index():
 
 def test_decode_1m_28_layers_seven_groups():
     _check_decode(R.DECODE_1M, steps=[0, 15], check_groups=[0, 6], check_layers=[0, 27])
+
+
+def test_decode_32k_batch8_sixteen_head_indexer():
+    """The batch-8 decode step with the 16-head weighted indexer (the bench's
+    multi-head workload): indices bit-exact, two layers' attention checked."""
+    _check_decode(R.DECODE_32K_MH16, steps=[0, 63], check_groups=[0], check_layers=[0, 3])
 
 
 # ---------------------------------------------------------------- prefill
