@@ -71,13 +71,14 @@ def job_rate(world: int, units_per_rank: float, ms: float) -> float:
 CONFIGS = {
     "decode_32k": R.DECODE_32K,
     "decode_32k_mh": R.DECODE_32K_MH16,
+    "yoco_32k": R.YOCO_32K,
     "decode_1m": R.DECODE_1M,
     "gist": R.GIST_128K,
     "prefill_2k": R.PREFILL_2K,
     "prefill_64k": R.PREFILL_64K,
 }
 # workloads reported under "workloads" beside the headline, in run order
-SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "decode_1m", "decode_32k_mh")
+SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "decode_1m", "decode_32k_mh", "yoco_32k")
 
 
 def load_peaks():
@@ -365,12 +366,20 @@ class DecodeBench:
         self.inp = TI.decode_inputs(R.Decode(**{**cfg.__dict__, "seed": seed}), device, layers=[])
         # all layers' K and V caches as slices of one [layers, 2, B, Tk_max, Hkv, D]
         # array, so a step's appended rows of every layer are one strided copy
-        self.kv_all = torch.empty((c.n_layers, 2, c.B, c.Tk_max, c.Hkv, c.D), dtype=torch.bfloat16, device=device)
-        for l in range(c.n_layers):
+        # (one cache for every layer when the layers share it)
+        n_kv = 1 if c.shared_kv else c.n_layers
+        self.kv_all = torch.empty((n_kv, 2, c.B, c.Tk_max, c.Hkv, c.D), dtype=torch.bfloat16, device=device)
+        for l in range(n_kv):
             gd.fill_normal(self.kv_all[l, 0], seed, R.tid(R.KIND_K, l))
             gd.fill_normal(self.kv_all[l, 1], seed, R.tid(R.KIND_V, l))
-            self.inp["K"][l], self.inp["V"][l] = self.kv_all[l, 0], self.kv_all[l, 1]
+        for l in range(c.n_layers):
+            lk = 0 if c.shared_kv else l
+            self.inp["K"][l], self.inp["V"][l] = self.kv_all[lk, 0], self.kv_all[lk, 1]
             self.inp["q"][l] = TI.dev_normal((c.steps, c.B, c.Hq, c.D), seed, R.tid(R.KIND_Q, l), device)
+        self.gather_once = c.shared_kv
+        if c.shared_kv:
+            self.k_rows = torch.empty((c.B, c.k, c.Hkv * c.D + 8), dtype=torch.bfloat16, device=device)
+            self.v_rows = torch.empty_like(self.k_rows)
         self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
         L = sa.lib()
         ws_idx = (L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k) if c.H_idx == 1 else
@@ -411,8 +420,17 @@ class DecodeBench:
             if ev is not None and first:
                 ev[("attn", g, 0)].record()
             q = q_all[layer] if q_all is not None else self.inp["q"][layer][s]
-            sa.sa_sparse_attn_decode(q, self.inp["K"][layer], self.inp["V"][layer],
-                                     idx.view(c.B, c.k), cnt.view(c.B), out=self.out[layer], ws=self.ws_attn)
+            if self.gather_once:
+                # one cache and one index for the group: gather the rows at its
+                # first layer, every layer attends over the compact rows
+                if first:
+                    sa.sa_gather_rows(self.inp["K"][layer], self.inp["V"][layer], idx.view(c.B, c.k),
+                                      cnt.view(c.B), k_rows=self.k_rows, v_rows=self.v_rows)
+                sa.sa_sparse_attn_decode_rows(q, self.k_rows, self.v_rows, cnt.view(c.B), out=self.out[layer],
+                                              ws=self.ws_attn)
+            else:
+                sa.sa_sparse_attn_decode(q, self.inp["K"][layer], self.inp["V"][layer],
+                                         idx.view(c.B, c.k), cnt.view(c.B), out=self.out[layer], ws=self.ws_attn)
             if ev is not None and last:
                 ev[("attn", g, 1)].record()
 
@@ -507,6 +525,7 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
     st = b.stream
     pin = lambda t: t.contiguous().cpu().pin_memory()
     L, B = c.n_layers, c.B
+    nkv = b.kv_all.shape[0]   # caches: one per layer, or one shared by every layer
     host = {}
     for s in range(n_steps):
         pos = c.N + s
@@ -515,7 +534,7 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
                    "k_row": {g: pin(b.inp["k_idx"][g][:, pos]) for g in b.inp["k_idx"]},
                    "q": pin(torch.stack([b.inp["q"][l][s] for l in range(L)])),
                    # rows (layer, K/V, sequence) in the order of b.kv_all
-                   "kv_row": pin(b.kv_all[:, :, :, pos].reshape(L * 2 * B, -1))}
+                   "kv_row": pin(b.kv_all[:, :, :, pos].reshape(nkv * 2 * B, -1))}
     out_h = torch.empty(b.out_all.shape, dtype=b.out_all.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host[0]["q_idx"].values()) + \
         sum(t.numel() * t.element_size() for t in host[0]["w_idx"].values()) + \
@@ -542,7 +561,7 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
                 rt.h2d(wi_dev[g].data_ptr(), h["w_idx"][g].data_ptr(), h["w_idx"][g].numel() * 4, st)
             row_copy(b.inp["k_idx"][g], h["k_row"][g], pos, B)
         rt.h2d(q_all.data_ptr(), h["q"].data_ptr(), h["q"].numel() * 2, st)
-        row_copy(b.kv_all, h["kv_row"], pos, L * 2 * B)
+        row_copy(b.kv_all, h["kv_row"], pos, nkv * 2 * B)
         b.step(s, q_all=q_all, q_idx=qi_dev, w_idx=wi_dev if wi_dev else None)
         rt.d2h(out_h.data_ptr(), b.out_all.data_ptr(), d2h, st)
 
@@ -597,9 +616,32 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
     value = job_rate(ctx.world, steps, ms)
 
     e2e = None if args.no_e2e else decode_e2e(b, ctx, steps, warmup)
+    compare = None
+    if cfg.shared_kv:
+        # the same steps with the rows gathered again by every layer
+        b.gather_once = False
+        graphs = {}
+        with torch.cuda.stream(b.stream):
+            for s in range(n_steps):
+                graphs[s] = rt.capture(b.stream, lambda: b.step(s))
+        for i in range(warmup):
+            rt.launch(graphs[i % n_steps], b.stream)
+        ms2 = ctx.timed(lambda s: rt.launch(graphs[s], b.stream), order, b.stream, flush=False)
+        for g in graphs.values():
+            rt.destroy(g)
+        b.gather_once = True
+        compare = {"gather_per_layer_ms_per_step": round(ms2 / steps, 5),
+                   "gather_once_ms_per_step": round(ms_step, 5),
+                   "speedup": round(ms2 / ms, 4),
+                   "what": "the same steps with every layer gathering its rows from the shared cache "
+                           "(sa_sparse_attn_decode) instead of one gather per step and attention over the "
+                           "compact rows (sa_gather_rows + sa_sparse_attn_decode_rows)"}
 
     score_run, attn_bytes = b.algorithmic_bytes()
     step_bytes = cfg.n_groups * score_run + cfg.n_layers * attn_bytes
+    if cfg.shared_kv:   # the selected rows cross HBM once per step; each layer reads q/out/indices
+        step_bytes = cfg.n_groups * score_run + attn_bytes + (cfg.n_layers - 1) * (attn_bytes - cfg.B * cfg.k *
+                                                                                   cfg.Hkv * cfg.D * 4)
     attn_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9 if attn_ms else None
     idx_gbs = score_run / (idx_ms * 1e-3) / 1e9 if idx_ms else None
     attn_total = cfg.n_layers * attn_ms if attn_ms else 0.0
@@ -642,6 +684,11 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if compare is not None:
+        line["compare"] = compare
+        line["config"]["shared_kv"] = True
+        roof["note"] = ("attention over the compact rows, which one gather per step brought in; "
+                        "the bytes are those of one gathered attention call")
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_decode(cfg, args.cpu_seconds, b)
     b.close()
@@ -1096,8 +1143,9 @@ class OracleDecode:
                     Kr.append(_bits(bench.inp["K"][l][b][r]))
                     Vr.append(_bits(bench.inp["V"][l][b][r]))
                 else:
-                    Kr.append(R.host_rows(cfg.seed, R.tid(R.KIND_K, l), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
-                    Vr.append(R.host_rows(cfg.seed, R.tid(R.KIND_V, l), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
+                    lk = 0 if cfg.shared_kv else l
+                    Kr.append(R.host_rows(cfg.seed, R.tid(R.KIND_K, lk), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
+                    Vr.append(R.host_rows(cfg.seed, R.tid(R.KIND_V, lk), (cfg.Hkv, cfg.D), rows, True, b, cfg.Tk_max))
             self.q[l] = _bits(bench.inp["q"][l][step][bl]) if bench is not None else R.decode_q_host(cfg, l, step)[bl]
             self.rows[l] = (Kr, Vr)
 

@@ -76,6 +76,7 @@ class Decode:
     share_every: int
     steps: int
     H_idx: int = 1          # indexer heads (> 1: the multi-head weighted indexer)
+    shared_kv: bool = False  # one K/V cache for every layer (YOCO); the rows are gathered once per step
 
     @property
     def Tk_max(self) -> int:
@@ -126,6 +127,12 @@ DECODE_1M = Decode("decode_1m_28layers", seed=5, B=1, N=1 << 20, d=64, Hq=28, Hk
 # dot product.
 DECODE_32K_MH16 = Decode("decode_b8_32k_4layers_idx16heads", seed=6, B=8, N=32768, d=128, Hq=32, Hkv=8,
                          D=128, k=2048, n_layers=4, share_every=4, steps=64, H_idx=16)
+
+# The batch-8 decode step with one K/V cache shared by all 4 layers (YOCO) and
+# one index (CLSA): the selected rows are gathered once per step and every
+# layer attends over the compact rows with its own queries.
+YOCO_32K = Decode("yoco_decode_b8_32k_4layers_one_cache", seed=7, B=8, N=32768, d=128, Hq=32, Hkv=8, D=128,
+                  k=2048, n_layers=4, share_every=4, steps=64, shared_kv=True)
 
 ALL = [PREFILL_2K, DECODE_32K, PREFILL_64K, GIST_128K, DECODE_1M]
 

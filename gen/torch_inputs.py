@@ -50,8 +50,12 @@ def decode_inputs(cfg: R.Decode, device, layers=None, groups=None):
             gd.fill_int(wb, s, R.tid(R.KIND_W_IDX, g), 0, lo=-3, hi=3)
             out["w_idx"][g] = wb.float()
     for l in layers:
-        out["K"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_K, l), device)
-        out["V"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_V, l), device)
+        if cfg.shared_kv and l > 0 and 0 in out["K"]:   # one cache for every layer
+            out["K"][l], out["V"][l] = out["K"][0], out["V"][0]
+        else:
+            lk = 0 if cfg.shared_kv else l
+            out["K"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_K, lk), device)
+            out["V"][l] = dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_V, lk), device)
         out["q"][l] = dev_normal((cfg.steps, cfg.B, cfg.Hq, cfg.D), s, R.tid(R.KIND_Q, l), device)
     return out
 

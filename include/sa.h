@@ -199,6 +199,40 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
                                 void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Gather once, attend many (one KV cache shared by every layer).
+ *
+ * [YOIO] §2.1-§2.2: YOCO keeps one KV cache for all layers, and the shared
+ * routing adds one index for all layers, so each decode step needs the
+ * selected K/V rows only once.  sa_gather_rows copies them into compact
+ * buffers; each layer then runs sa_sparse_attn_decode_rows over those rows
+ * with its own queries.
+ *
+ * sa_gather_rows:
+ *   k_cache, v_cache  [B, Tk_max, Hkv, D] bf16;  idx [B, k] int32 (entries
+ *                     below count[b] in [0, Tk_max); others are not read);
+ *                     count [B] int32 (clamped to [0, k])
+ *   k_rows, v_rows    [B, k, Hkv * D + 8] bf16: row i of sequence b holds the
+ *                     Hkv * D values of cache row idx[b, i] for i < count[b],
+ *                     zeros after it; the last 8 values (16 bytes) of every
+ *                     row are a zero pad (the layout the attention stages a
+ *                     tile in, so one copy moves a whole tile).
+ * sa_sparse_attn_decode_rows: the attention of sa_sparse_attn_decode over
+ *   the first count[b] rows of k_rows / v_rows (laid out as above, pad
+ *   included; rows from count[b] to k must hold finite values, as the
+ *   gather's zeros do).
+ *   q [B, Hq, D]; out [B, Hq, D]; lse [B, Hq] or NULL;
+ *   ws >= sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k) bytes (same
+ *   conventions).  Supported: D = 128, Hkv <= 8, Hq % Hkv == 0, Hq/Hkv <= 16.
+ * ---------------------------------------------------------------------- */
+sa_status sa_gather_rows(const void* k_cache, const void* v_cache, const int32_t* idx,
+                         const int32_t* count, int B, int Tk_max, int Hkv, int D, int k,
+                         void* k_rows, void* v_rows, sa_stream_t stream);
+sa_status sa_sparse_attn_decode_rows(const void* q, const void* k_rows, const void* v_rows,
+                                     const int32_t* count, int B, int Hq, int Hkv, int D, int k,
+                                     float scale, void* out, float* lse,
+                                     void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Decode attention without a caller workspace.
  *
  * No counterpart in the paper: this is an interface for callers that cannot

@@ -14,10 +14,12 @@ from .sa import (  # noqa: F401
     IndexCache,
     SAError,
     lib,
+    sa_gather_rows,
     sa_gist_route_unfold,
     sa_index_score_topk,
     sa_index_score_topk_mh,
     sa_sparse_attn_decode,
+    sa_sparse_attn_decode_rows,
     sa_sparse_attn_prefill,
 )
 
@@ -31,9 +33,11 @@ __all__ = [
     "IndexCache",
     "SAError",
     "lib",
+    "sa_gather_rows",
     "sa_gist_route_unfold",
     "sa_index_score_topk",
     "sa_index_score_topk_mh",
     "sa_sparse_attn_decode",
+    "sa_sparse_attn_decode_rows",
     "sa_sparse_attn_prefill",
 ]

@@ -370,6 +370,48 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
   return ok();
 }
 
+// ------------------------------------------------------- gather once
+
+sa_status sa_gather_rows(const void* k_cache, const void* v_cache, const int32_t* idx, const int32_t* count,
+                         int B, int Tk_max, int Hkv, int D, int k, void* k_rows, void* v_rows,
+                         sa_stream_t stream) {
+  if (B < 0 || Tk_max < 1 || Hkv < 1 || k < 1)
+    return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d Tk_max=%d Hkv=%d k=%d", B, Tk_max, Hkv, k);
+  if (D != SA_HEAD_DIM) return fail(SA_ERR_UNSUPPORTED, "D=%d unsupported (only %d)", D, SA_HEAD_DIM);
+  if (k > (1 << 20)) return fail(SA_ERR_UNSUPPORTED, "k=%d too large", k);
+  if (B == 0) return ok();
+  if (!k_cache || !v_cache || !idx || !count || !k_rows || !v_rows) return fail(SA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_rows, 16) || !aligned(v_rows, 16))
+    return fail(SA_ERR_INVALID_ARG, "caches and row buffers must be 16-byte aligned");
+  if (!aligned(idx, 4) || !aligned(count, 4)) return fail(SA_ERR_INVALID_ARG, "idx/count misaligned");
+  const cudaError_t e = sa::launch_gather_rows(
+      static_cast<const uint16_t*>(k_cache), static_cast<const uint16_t*>(v_cache), idx, count, B, Tk_max, Hkv, k,
+      static_cast<uint16_t*>(k_rows), static_cast<uint16_t*>(v_rows), as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather_rows launch");
+  return ok();
+}
+
+sa_status sa_sparse_attn_decode_rows(const void* q, const void* k_rows, const void* v_rows, const int32_t* count,
+                                     int B, int Hq, int Hkv, int D, int k, float scale, void* out, float* lse,
+                                     void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || k < 1)
+    return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d Hq=%d Hkv=%d k=%d", B, Hq, Hkv, k);
+  if (Hkv > 8) return fail(SA_ERR_UNSUPPORTED, "Hkv=%d > 8 unsupported for compact rows", Hkv);
+  // idx is not read for compact rows; any aligned non-null pointer passes validation
+  sa_status st = validate_attn(q, k_rows, v_rows, count, count, B, 1, k, Hq, Hkv, D, k, out);
+  if (st != SA_OK) return st;
+  if (B == 0) return ok();
+  if ((long long)B * Hkv > SA_DECODE_MAX_PAIRS)
+    return fail(SA_ERR_UNSUPPORTED, "B*Hkv=%lld exceeds %d", (long long)B * Hkv, SA_DECODE_MAX_PAIRS);
+  if ((st = check_ws(ws, ws_bytes, sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k))) != SA_OK) return st;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+  const cudaError_t e = sa::launch_attn_decode(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k_rows), static_cast<const uint16_t*>(v_rows),
+      nullptr, count, B, k, Hq, Hkv, k, sc, static_cast<uint16_t*>(out), lse, ws, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_rows launch");
+  return ok();
+}
+
 // ---------------------------------------------------------------- gist
 
 size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) {

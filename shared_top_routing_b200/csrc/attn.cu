@@ -302,7 +302,8 @@ constexpr int kMergeMaxC = 1280;   // contributors of one (sequence, head block)
 struct DecPlan {
   int nh, wph, R, HB;     // heads per block, warps per head, rows per tile, blocks per sequence
   int pairs, tpp;         // (sequence, block) pairs, tiles per pair
-  int row_bytes;          // padded shared row: nh * 256 + 16
+  int dense;              // rows are the first count[b] rows of compact buffers (one copy per tile)
+  int row_bytes;          // shared row: nh * 256, padded by 16 when rows are gathered one by one
   int stage_bytes;        // K and V tiles of one stage
   int U, W;               // units (< 2^31: pairs <= 2^14, tiles per pair <= 2^16), CTAs
 };
@@ -478,7 +479,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
     auto stage_chunk = [&](int c0, int buf) {
       const int c1 = min(c0 + CU, hi);
       int32_t* si = sidx + buf * kIdxChunk;
-      for (int e = lane; e < (c1 - c0) * R; e += 32) {
+      for (int e = lane; e < (pl.dense ? 0 : (c1 - c0) * R); e += 32) {
         const int u = c0 + e / R;
         const int r = e % R;
         const int b = u / pl.tpp / pl.HB;
@@ -521,14 +522,34 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
       if (use > 0 && !tc::mbar_wait(&empty[s], (use - 1) & 1u, abort_flag, err, 11)) break;
       unsigned char* stK = smem + (size_t)s * pl.stage_bytes;
       unsigned char* stV = stK + (size_t)R * rb;
-      const int j0 = si[0];   // row r0 < cnt
-      if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)R * bytes);
+      // bytes this tile's copies bring (compact rows copy their pads too)
+      const int rows_in = pl.dense ? min(R, k - r0) : 0;
+      const uint32_t tile_bytes = pl.dense ? (uint32_t)(rows_in * rb) + (uint32_t)(R - rows_in) * bytes
+                                           : (uint32_t)R * bytes;
+      if (lane == 0) tc::mbar_arrive_expect_tx(&full[s], 2u * tile_bytes);
       __syncwarp();
-      for (int r = lane; r < R; r += 32) {
-        const int j = clamp_row(r0 + r < cnt ? si[r] : j0, Tk_max);
-        const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
-        tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
-        tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
+      if (pl.dense) {
+        // compact rows (one head block), each Hkv * 256 bytes plus the same
+        // 16-byte pad as a shared row: the tile's rows are contiguous, so one
+        // bulk copy per cache brings them all in the padded layout; rows past
+        // the buffer's end repeat the tile's first row (finite, masked)
+        const long long off = ((long long)b * k + r0) * (rb / 2);
+        if (lane == 0) {
+          tc::bulk_load(stK, kc + off, (uint32_t)(rows_in * rb), &full[s]);
+          tc::bulk_load(stV, vc + off, (uint32_t)(rows_in * rb), &full[s]);
+        }
+        for (int r = rows_in + lane; r < R; r += 32) {
+          tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
+          tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
+        }
+      } else {
+        const int j0 = si[0];   // row r0 < cnt
+        for (int r = lane; r < R; r += 32) {
+          const int j = clamp_row(r0 + r < cnt ? si[r] : j0, Tk_max);
+          const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
+          tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
+          tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
+        }
       }
       ++fill;
     }
@@ -702,7 +723,48 @@ attn_decode_merge_kernel(const float* __restrict__ part_o, const float* __restri
   }
 }
 
-DecPlan decode_plan(int B, int Hkv, int k) {
+// Gathers the selected rows of each sequence (all kv heads of a position,
+// Hkv * 256 contiguous bytes per cache) into compact buffers of rows of
+// Hkv * 256 bytes plus a 16-byte zero pad ([B][k][Hkv * D + 8] elements),
+// the layout of a shared-memory row of the decode split kernel, so that a
+// tile of rows is one contiguous copy; rows from count[b] to k are written
+// as zeros.  One warp per row, 16-byte loads and stores.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc,
+                   const int32_t* __restrict__ idx, const int32_t* __restrict__ count, int Tk_max, int Hkv,
+                   int k, uint16_t* __restrict__ ko, uint16_t* __restrict__ vo) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= k) return;
+  const int cnt = clamp_count(count, b, k);
+  const int chunks = Hkv * kD / 8;   // 16-byte chunks per row (then one chunk of pad)
+  uint4* dk = reinterpret_cast<uint4*>(ko + ((long long)b * k + r) * (Hkv * kD + 8));
+  uint4* dv = reinterpret_cast<uint4*>(vo + ((long long)b * k + r) * (Hkv * kD + 8));
+  if (lane == 0) {
+    dk[chunks] = make_uint4(0u, 0u, 0u, 0u);
+    dv[chunks] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (r < cnt) {
+    const int j = clamp_row(idx[(long long)b * k + r], Tk_max);
+    const uint4* sk = reinterpret_cast<const uint4*>(kc + ((long long)b * Tk_max + j) * Hkv * kD);
+    const uint4* sv = reinterpret_cast<const uint4*>(vc + ((long long)b * Tk_max + j) * Hkv * kD);
+    for (int c = lane; c < chunks; c += 32) {
+      const uint4 a = __ldg(sk + c), v = __ldg(sv + c);
+      dk[c] = a;
+      dv[c] = v;
+    }
+  } else {
+    for (int c = lane; c < chunks; c += 32) {
+      dk[c] = make_uint4(0u, 0u, 0u, 0u);
+      dv[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+DecPlan decode_plan(int B, int Hkv, int k, bool dense = false) {
   const int sms = device_sm_count();
   DecPlan pl;
   pl.nh = Hkv < kDxConsumers ? Hkv : kDxConsumers;
@@ -711,7 +773,8 @@ DecPlan decode_plan(int B, int Hkv, int k) {
   pl.HB = (Hkv + pl.nh - 1) / pl.nh;
   pl.pairs = B * pl.HB;
   pl.tpp = (k + pl.R - 1) / pl.R;
-  pl.row_bytes = pl.nh * kD * 2 + 16;
+  pl.dense = dense ? 1 : 0;
+  pl.row_bytes = pl.nh * kD * 2 + 16;   // the pad keeps the consumers' ldmatrix free of bank conflicts
   pl.stage_bytes = 2 * pl.R * pl.row_bytes;
   pl.U = pl.pairs * pl.tpp;
   int W = sms;   // one CTA per SM
@@ -753,7 +816,8 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
                                int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,
                                cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
-  const DecPlan pl = decode_plan(B, Hkv, k);
+  const bool dense = idx == nullptr;   // compact rows [B][k][Hkv][D] (Hkv <= 8, Tk_max == k)
+  const DecPlan pl = decode_plan(B, Hkv, k, dense);
   const int G = Hq / Hkv;
   const size_t slots = (size_t)(pl.pairs + pl.W) * pl.wph * pl.nh * G;
   char* p = static_cast<char*>(ws);
@@ -774,6 +838,14 @@ cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint
                  pl, Hq, Hkv, err, out, lse);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t* kc, const uint16_t* vc, const int32_t* idx, const int32_t* count,
+                               int B, int Tk_max, int Hkv, int k, uint16_t* ko, uint16_t* vo, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  const cudaError_t e = launch_pdl(gather_rows_kernel, dim3((unsigned)((k + 7) / 8), (unsigned)B), dim3(256), 0, st,
+                                   kc, vc, idx, count, Tk_max, Hkv, k, ko, vo);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,

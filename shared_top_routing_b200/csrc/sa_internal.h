@@ -151,10 +151,15 @@ size_t decode_attn_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
 // Leading bytes of the decode workspace that must be zero when a call starts
 // (the kernel error word).
 size_t decode_attn_zero_bytes(int B, int Hkv, int k);
+// idx == nullptr: kc / vc are compact rows [B][k][Hkv][D] (Hkv <= 8, Tk_max ==
+// k) and each sequence attends over its first count[b] rows.
 cudaError_t launch_attn_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                const int32_t* idx, const int32_t* count, int B, int Tk_max, int Hq,
                                int Hkv, int k, float scale, uint16_t* out, float* lse, void* ws,
                                cudaStream_t st);
+// Compact copies of the selected rows (rows past count zero-filled).
+cudaError_t launch_gather_rows(const uint16_t* kc, const uint16_t* vc, const int32_t* idx, const int32_t* count,
+                               int B, int Tk_max, int Hkv, int k, uint16_t* ko, uint16_t* vo, cudaStream_t st);
 cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                 const int32_t* idx, const int32_t* count, int B, int T, int Tk_max,
                                 int Hq, int Hkv, int k, float scale, uint16_t* out, float* lse,

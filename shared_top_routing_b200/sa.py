@@ -43,6 +43,8 @@ SIGNATURES = {
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "sa_sparse_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "sa_gather_rows": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_sparse_attn_decode_rows": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
     "sa_self_test_bounded_wait": (_I, [_P, ctypes.c_uint32, _P]),
     "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
     "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
@@ -264,6 +266,47 @@ def sa_sparse_attn_decode(q, k_cache, v_cache, idx, count, scale: float = 0.0, o
                                      B, Tk_max, Hq, Hkv, D, k, scale, _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "sa_sparse_attn_decode")
+    return (out, lse) if with_lse else out
+
+
+def sa_gather_rows(k_cache, v_cache, idx, count, k_rows=None, v_rows=None, stream=None):
+    """Compact copies [B, k, Hkv * D + 8] of the selected rows (zeros past
+    count; the last 8 values of each row are a zero pad, see sa.h)."""
+    torch = _torch()
+    B, Tk_max, Hkv, D = k_cache.shape
+    k = idx.shape[-1]
+    for t, n, sz in ((k_cache, "k_cache", 2), (v_cache, "v_cache", 2), (idx, "idx", 4), (count, "count", 4)):
+        _need(t, n, sz)
+    if k_rows is None:
+        k_rows = torch.empty((B, k, Hkv * D + 8), dtype=k_cache.dtype, device=k_cache.device)
+    if v_rows is None:
+        v_rows = torch.empty((B, k, Hkv * D + 8), dtype=v_cache.dtype, device=v_cache.device)
+    st = lib().sa_gather_rows(_ptr(k_cache), _ptr(v_cache), _ptr(idx), _ptr(count), B, Tk_max, Hkv, D, k,
+                              _ptr(k_rows), _ptr(v_rows), _stream(stream))
+    _check(st, "sa_gather_rows")
+    return k_rows, v_rows
+
+
+def sa_sparse_attn_decode_rows(q, k_rows, v_rows, count, scale: float = 0.0, out=None, with_lse: bool = False,
+                               ws=None, stream=None):
+    """q [B, Hq, D]; k_rows / v_rows [B, k, Hkv * D + 8] compact rows (from
+    sa_gather_rows); count [B]."""
+    torch = _torch()
+    B, Hq, D = q.shape
+    _, k, row = k_rows.shape
+    Hkv = (row - 8) // D
+    for t, n, sz in ((q, "q", 2), (k_rows, "k_rows", 2), (v_rows, "v_rows", 2), (count, "count", 4)):
+        _need(t, n, sz)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if with_lse else None
+    need = lib().sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k)
+    if ws is None:
+        ws = workspace(need, q.device, "attn_decode", stream)
+    st = lib().sa_sparse_attn_decode_rows(_ptr(q), _ptr(k_rows), _ptr(v_rows), _ptr(count), B, Hq, Hkv, D, k,
+                                          scale, _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
+                                          _stream(stream))
+    _check(st, "sa_sparse_attn_decode_rows")
     return (out, lse) if with_lse else out
 
 

@@ -14,7 +14,7 @@ import torch
 import oracle
 import shared_top_routing_b200 as sa
 from gen import counter_hash as ch
-from tests.gpu_util import assert_close_attn, assert_lse_close, dev, i32, to_dev
+from tests.gpu_util import assert_close_attn, assert_lse_close, bits_of, dev, i32, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -378,6 +378,77 @@ def test_decode_attention_chained_after_an_index_run(Hq, Hkv, k):
         ref, _ = oracle.sparse_attention_decode(q, [K[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)],
                                                 [V[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)])
         assert_close_attn(out.float().cpu().numpy(), ref, f"layer {layer}")
+
+
+# ------------------------------------------------- gather once, attend many
+
+@pytest.mark.parametrize("Hkv,k,counts", [(8, 2048, [2048, 1000, 0]), (4, 100, [100, 37, 64]),
+                                          (2, 1104, [1104, 1090, 5]), (1, 300, [1, 299, 300])])
+def test_gather_rows_copies_the_selected_rows(Hkv, k, counts):
+    """[YOIO] §2.1-§2.2: the selected rows of the shared cache, once, in
+    selection order; zeros past each count."""
+    rng = np.random.default_rng(k + Hkv)
+    B, Tk_max = len(counts), 3000
+    K = _normals(61, 2, (B, Tk_max, Hkv, 128))
+    V = _normals(61, 3, (B, Tk_max, Hkv, 128))
+    idx = _random_index(rng, B, Tk_max, k, counts)
+    kr, vr = sa.sa_gather_rows(to_dev(K), to_dev(V), i32(idx), i32(counts))
+    torch.cuda.synchronize()
+    kr, vr = bits_of(kr), bits_of(vr)
+    assert kr.shape == (B, k, Hkv * 128 + 8)
+    assert not kr[:, :, Hkv * 128:].any() and not vr[:, :, Hkv * 128:].any()   # the row pads
+    kr = kr[:, :, : Hkv * 128].reshape(B, k, Hkv, 128)
+    vr = vr[:, :, : Hkv * 128].reshape(B, k, Hkv, 128)
+    for b, c in enumerate(counts):
+        np.testing.assert_array_equal(kr[b, :c], K[b, idx[b, :c]])
+        np.testing.assert_array_equal(vr[b, :c], V[b, idx[b, :c]])
+        assert not kr[b, c:].any() and not vr[b, c:].any()
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (28, 4), (8, 2), (8, 1), (15, 3)])
+@pytest.mark.parametrize("k,counts", [(2048, [2048, 1000, 0, 1]), (100, [100, 33, 64, 7]), (1104, [1104, 1090, 1, 17])])
+def test_decode_attention_over_compact_rows_matches_oracle(Hq, Hkv, k, counts):
+    rng = np.random.default_rng(Hq * 100 + k)
+    B, Tk_max, D = len(counts), 3000, 128
+    q = _normals(4000 + Hq, 1, (B, Hq, D))
+    K = _normals(4000 + Hq, 2, (B, Tk_max, Hkv, D))
+    V = _normals(4000 + Hq, 3, (B, Tk_max, Hkv, D))
+    idx = _random_index(rng, B, Tk_max, k, counts)
+    kr, vr = sa.sa_gather_rows(to_dev(K), to_dev(V), i32(idx), i32(counts))
+    out, lse = sa.sa_sparse_attn_decode_rows(to_dev(q), kr, vr, i32(counts), with_lse=True)
+    ref, rlse = oracle.sparse_attention_decode(q, [K[b, idx[b, :c]] for b, c in enumerate(counts)],
+                                               [V[b, idx[b, :c]] for b, c in enumerate(counts)])
+    torch.cuda.synchronize()
+    assert_close_attn(out.float().cpu().numpy(), ref, "attention over compact rows")
+    assert_lse_close(lse.cpu().numpy(), rlse, "lse over compact rows")
+
+
+def test_one_cache_one_index_gather_once_attend_many():
+    """YOCO + CLSA ([YOIO] §2.1-§2.2): four layers share one KV cache and one
+    index; the rows are gathered once and each layer attends over them with
+    its own queries.  Every layer matches the oracle and the per-layer
+    gathered path."""
+    B, T, d, k, Hq, Hkv = 3, 9000, 128, 2048, 32, 8
+    qi = _ints(62, 1, (B, d))
+    ki = _ints(62, 2, (B, T, d))
+    K = _normals(62, 3, (B, T, Hkv, 128))
+    V = _normals(62, 4, (B, T, Hkv, 128))
+    Kd, Vd = to_dev(K), to_dev(V)
+    idx, cnt = sa.sa_index_score_topk(to_dev(qi), to_dev(ki), k, Tk=T, q_pos0=T - 1)
+    kr, vr = sa.sa_gather_rows(Kd, Vd, idx, cnt)
+    ridx, rcnt = oracle.index_topk(qi[:, None, :], ki, T, T - 1, k)
+    Kr = [K[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)]
+    Vr = [V[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)]
+    for layer in range(4):
+        q = _normals(63 + layer, 1, (B, Hq, 128))
+        qd = to_dev(q)
+        once = sa.sa_sparse_attn_decode_rows(qd, kr, vr, cnt)
+        each = sa.sa_sparse_attn_decode(qd, Kd, Vd, idx, cnt)
+        torch.cuda.synchronize()
+        ref, _ = oracle.sparse_attention_decode(q, Kr, Vr)
+        assert_close_attn(once.float().cpu().numpy(), ref, f"layer {layer}, gathered once")
+        assert_close_attn(each.float().cpu().numpy(), ref, f"layer {layer}, gathered per layer")
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
 
 
 def test_decode_attention_many_sequences():

@@ -57,8 +57,14 @@ def _check_decode(cfg, steps, check_groups, check_layers):
             idx, cnt, ver = cache.get_tensors(layer)
             versions[g] = ver if versions[g] is None else versions[g]
             assert ver == versions[g]          # every layer of the group reads the same write
-            sa.sa_sparse_attn_decode(inp["q"][layer][s], inp["K"][layer], inp["V"][layer],
-                                     idx.view(cfg.B, cfg.k), cnt.view(cfg.B), out=outs[layer])
+            if cfg.shared_kv:                  # one cache: gather once, every layer over the compact rows
+                if layer % cfg.share_every == 0:
+                    kr, vr = sa.sa_gather_rows(inp["K"][layer], inp["V"][layer], idx.view(cfg.B, cfg.k),
+                                               cnt.view(cfg.B))
+                sa.sa_sparse_attn_decode_rows(inp["q"][layer][s], kr, vr, cnt.view(cfg.B), out=outs[layer])
+            else:
+                sa.sa_sparse_attn_decode(inp["q"][layer][s], inp["K"][layer], inp["V"][layer],
+                                         idx.view(cfg.B, cfg.k), cnt.view(cfg.B), out=outs[layer])
             if g in check_groups and layer % cfg.share_every == 0:
                 got_idx[g] = (idx.view(cfg.B, cfg.k).clone(), cnt.view(cfg.B).clone())
             if layer in check_layers:
@@ -76,9 +82,10 @@ def _check_decode(cfg, steps, check_groups, check_layers):
             gi = got_idx[g][0].cpu().numpy() if g in got_idx else None
             assert gi is not None
             q = R.decode_q_host(cfg, layer, s)
-            Kr = [R.host_rows(cfg.seed, R.tid(R.KIND_K, layer), (cfg.Hkv, cfg.D), gi[b], True, b, cfg.Tk_max)
+            lk = 0 if cfg.shared_kv else layer
+            Kr = [R.host_rows(cfg.seed, R.tid(R.KIND_K, lk), (cfg.Hkv, cfg.D), gi[b], True, b, cfg.Tk_max)
                   for b in range(cfg.B)]
-            Vr = [R.host_rows(cfg.seed, R.tid(R.KIND_V, layer), (cfg.Hkv, cfg.D), gi[b], True, b, cfg.Tk_max)
+            Vr = [R.host_rows(cfg.seed, R.tid(R.KIND_V, lk), (cfg.Hkv, cfg.D), gi[b], True, b, cfg.Tk_max)
                   for b in range(cfg.B)]
             ref, _ = oracle.sparse_attention_decode(q, Kr, Vr)
             assert_close_attn(outs[layer].float().cpu().numpy(), ref, f"{cfg.name} step {s} layer {layer}")
@@ -95,6 +102,12 @@ def test_decode_32k_batch8_four_layers_share_one_index():
 
 def test_decode_1m_28_layers_seven_groups():
     _check_decode(R.DECODE_1M, steps=[0, 15], check_groups=[0, 6], check_layers=[0, 27])
+
+
+def test_decode_32k_one_cache_gathered_once():
+    """The bench's one-cache workload (YOCO + CLSA): one gather per step, four
+    layers over the compact rows, checked at full size."""
+    _check_decode(R.YOCO_32K, steps=[0, 63], check_groups=[0], check_layers=[0, 3])
 
 
 def test_decode_32k_batch8_sixteen_head_indexer():
