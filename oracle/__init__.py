@@ -22,6 +22,7 @@ from .reference import (  # noqa: F401
     sparse_attention,
     sparse_attention_decode,
     gist_route_unfold,
+    hier_gist_route_unfold,
     layer_owners,
     kv_cache_gib,
     pair_counts,

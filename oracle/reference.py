@@ -37,6 +37,11 @@ Readings where the pages are silent (each also stated where it is used):
    after DeepSeek's published lightning indexer): H indexer heads, each
    with its own query vector and a per-query weight, score one shared key
    per token as sum_h w_h * ReLU(q_h . k).  Selection is unchanged.
+8. Two-level gist routing: meta-gist keys are routing keys only (their
+   rows are not attended), one per complete group of chunks; the chunks
+   after the last complete group have no meta-gist yet and are always
+   second-stage candidates; the unfolded rows are those of single-level
+   routing for the chunks chosen in the second stage.
 """
 from __future__ import annotations
 
@@ -236,6 +241,40 @@ def gist_route_unfold(q_route, gist_key, chunk_len: int, k_chunks: int, partial_
     parts.append(n_chunks * stride + np.arange(partial_len))
     rows = np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
     return rows.astype(np.int64), chunks.astype(np.int64)
+
+
+def hier_gist_route_unfold(q_route, meta_key, gist_key, group_size: int, chunk_len: int, k_groups: int,
+                           k_chunks: int, partial_len: int):
+    """Two-level (coarse-to-fine) gist routing for one decode query ([SSA]
+    §五 H-SSA, [GSA] 2.4 H-GSA; reading 8).
+
+    Every complete group of group_size consecutive chunks has one meta-gist
+    routing key.  The query is scored against every meta key and the top
+    k_groups groups are kept (equal scores: lower group first).  The
+    candidate chunks are those of the kept groups plus the chunks after the
+    last complete group (no meta-gist yet); the query is scored against
+    their gist keys and the top k_chunks candidates are kept (equal scores:
+    lower chunk first).  They are unfolded exactly as gist_route_unfold does.
+
+    meta_key: [n_chunks // group_size, d]; gist_key: [n_chunks, d].
+    Returns (rows int64 ascending, chunks int64 ascending, groups int64
+    ascending).
+    """
+    gk = _f64(gist_key)
+    mk = _f64(meta_key)
+    q = _f64(q_route)
+    n_chunks = gk.shape[0]
+    n_groups = n_chunks // group_size
+    groups = topk_select(mk[:n_groups] @ q, k_groups) if n_groups else np.zeros(0, dtype=np.int64)
+    parts = [g * group_size + np.arange(group_size) for g in groups]
+    parts.append(np.arange(n_groups * group_size, n_chunks))
+    cand = np.concatenate(parts).astype(np.int64)
+    chunks = cand[topk_select(gk[cand] @ q, k_chunks)] if cand.size else cand
+    stride = chunk_len + 1
+    rparts = [c * stride + np.arange(stride) for c in chunks]
+    rparts.append(n_chunks * stride + np.arange(partial_len))
+    rows = np.concatenate(rparts)
+    return rows.astype(np.int64), chunks.astype(np.int64), np.asarray(groups, dtype=np.int64)
 
 
 # ----------------------------------------------------------------- sharing

@@ -562,3 +562,48 @@ def test_multihead_pin_catches_slips(monkeypatch, mutant):
     monkeypatch.setattr(oracle, "index_scores_multihead", mutant)
     with pytest.raises(AssertionError):
         test_multihead_scores_match_python_integers()
+
+
+# ------------------------------------------------------ two-level gist routing
+
+def test_hier_gist_with_every_group_kept_is_single_level_routing():
+    """[SSA] §五 / [GSA] 2.4: when the coarse stage keeps every group, the
+    two-level routing is the single-level selective unfolding ([SSA] §三)."""
+    rng = _rng(41)
+    n_chunks, M, d = 50, 8, 16
+    q = _bf16(rng.integers(-4, 5, size=d))
+    gk = _bf16(rng.integers(-4, 5, size=(n_chunks, d)))
+    mk = _bf16(rng.integers(-4, 5, size=(n_chunks // M, d)))
+    for kc in (1, 5, 40, 60):
+        rows, chunks, groups = oracle.hier_gist_route_unfold(q, mk, gk, M, 4, n_chunks // M, kc, 3)
+        r1, c1 = oracle.gist_route_unfold(q, gk, 4, kc, 3)
+        np.testing.assert_array_equal(chunks, c1)
+        np.testing.assert_array_equal(rows, r1)
+        np.testing.assert_array_equal(groups, np.arange(n_chunks // M))
+
+
+def test_hier_gist_hand_worked_example():
+    """Four groups of two chunks plus one trailing chunk (9 chunks, group
+    size 2), d = 2, query (1, 0): the meta scores are the meta keys' first
+    entries (3, 1, 4, 1): k_groups = 2 keeps groups 0 and 2 (chunks 0, 1, 4,
+    5) and chunk 8 (no meta-gist yet) is a candidate too.  Gist scores of
+    chunks 0..8 are (0, 2, 9, 9, 5, 1, 7, 7, 3): among the candidates the top
+    3 are chunks 4 (5), 8 (3), 1 (2) -- chunks 2, 3, 6, 7 score higher but
+    sit in groups the coarse stage dropped."""
+    q = _bf16([1, 0])
+    gk = _bf16([[0, 1], [2, 0], [9, 0], [9, 0], [5, 0], [1, 0], [7, 0], [7, 0], [3, 0]])
+    mk = _bf16([[3, 0], [1, 0], [4, 0], [1, 0]])
+    rows, chunks, groups = oracle.hier_gist_route_unfold(q, mk, gk, 2, 1, 2, 3, 1)
+    np.testing.assert_array_equal(groups, [0, 2])
+    np.testing.assert_array_equal(chunks, [1, 4, 8])
+    # chunk_len 1: chunk c occupies rows 2c (raw) and 2c + 1 (gist); the partial chunk starts at 18
+    np.testing.assert_array_equal(rows, [2, 3, 8, 9, 16, 17, 18])
+
+
+def test_hier_gist_ties_take_lower_groups_and_chunks():
+    q = _bf16([0, 0])
+    gk = _bf16(np.ones((12, 2)))
+    mk = _bf16(np.ones((3, 2)))
+    _, chunks, groups = oracle.hier_gist_route_unfold(q, mk, gk, 4, 2, 2, 5, 0)
+    np.testing.assert_array_equal(groups, [0, 1])
+    np.testing.assert_array_equal(chunks, [0, 1, 2, 3, 4])
