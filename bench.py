@@ -72,13 +72,14 @@ CONFIGS = {
     "decode_32k": R.DECODE_32K,
     "decode_32k_mh": R.DECODE_32K_MH16,
     "yoco_32k": R.YOCO_32K,
+    "hgist": R.HGIST_128K,
     "decode_1m": R.DECODE_1M,
     "gist": R.GIST_128K,
     "prefill_2k": R.PREFILL_2K,
     "prefill_64k": R.PREFILL_64K,
 }
 # workloads reported under "workloads" beside the headline, in run order
-SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "decode_1m", "decode_32k_mh", "yoco_32k")
+SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "hgist", "decode_1m", "decode_32k_mh", "yoco_32k")
 
 
 def load_peaks():
@@ -652,7 +653,8 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
                 "frac": _frac(attn_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": attn_bytes,
                 "launch_ms": _r(attn_ms, 5)}
     else:
-        roof = {"kernel": "score_decode_kernel + collect_kernel + finish_kernel (one indexer run)",
+        roof = {"kernel": ("score_mh_kernel" if cfg.H_idx > 1 else "score_decode_kernel")
+                          + " + split_topk_kernel (one indexer run)",
                 "bound": "hbm", "achieved": _r(idx_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": _frac(idx_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": score_run,
                 "launch_ms": _r(idx_ms, 5)}
@@ -910,14 +912,18 @@ class GistBench:
         self.out = torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=device)
         self.graphs, self.graphs_ev, self.ev = {}, {}, {}
 
-    def step(self, s, ev=None, q_route=None, q=None, partial=None):
+    def step(self, s, ev=None, q_route=None, q=None, partial=None, single_level=False):
         c, sa = self.cfg, self.sa
         if ev is not None:
             ev[0].record()
-        sa.sa_gist_route_unfold(q_route if q_route is not None else self.inp["q_route"][s], self.inp["gist_key"],
-                                c.chunk_len, c.k_chunks,
-                                partial if partial is not None else self.inp["partial_len"][s],
-                                rows_out=self.rows, count_out=self.cnt, ws=self.ws_g)
+        qr = q_route if q_route is not None else self.inp["q_route"][s]
+        pl = partial if partial is not None else self.inp["partial_len"][s]
+        if c.group_size and not single_level:
+            sa.sa_hier_gist_route_unfold(qr, self.inp["meta_key"], self.inp["gist_key"], c.chunk_len, c.group_size,
+                                         c.k_groups, c.k_chunks, pl, rows_out=self.rows, count_out=self.cnt)
+        else:
+            sa.sa_gist_route_unfold(qr, self.inp["gist_key"], c.chunk_len, c.k_chunks, pl, rows_out=self.rows,
+                                    count_out=self.cnt, ws=self.ws_g)
         if ev is not None:
             ev[1].record()
         sa.sa_sparse_attn_decode(q if q is not None else self.inp["q"][s], self.inp["K"], self.inp["V"],
@@ -1027,6 +1033,23 @@ def measure_gist(ctx: Ctx, cfg: R.Gist, steps: int, warmup: int):
     launches = sum(ctx.rt.kernel_nodes[gb.graphs[s].value] for s in order)
     value = job_rate(ctx.world, steps, ms)
     route_bytes = cfg.B * cfg.n_chunks * cfg.d * 2
+    compare = None
+    if cfg.group_size:
+        # bytes the two-level routing reads: every meta key, the kept groups' and trailing chunks' gist keys
+        n_groups = cfg.n_chunks // cfg.group_size
+        cand = min(cfg.k_groups, n_groups) * cfg.group_size + cfg.n_chunks - n_groups * cfg.group_size
+        route_bytes = cfg.B * (n_groups + cand) * cfg.d * 2
+        graphs = {}
+        with torch.cuda.stream(gb.stream):
+            for s in range(cfg.steps):
+                graphs[s] = ctx.rt.capture(gb.stream, lambda: gb.step(s, single_level=True))
+        ms1 = ctx.timed(lambda s: ctx.rt.launch(graphs[s], gb.stream), order, gb.stream, flush=True)
+        for g in graphs.values():
+            ctx.rt.destroy(g)
+        compare = {"single_level_ms_per_step": round(ms1 / steps, 5), "two_level_ms_per_step": round(ms / steps, 5),
+                   "what": "the same steps routed over every gist key (sa_gist_route_unfold) instead of meta "
+                           "keys then the kept groups' gist keys (sa_hier_gist_route_unfold); the chosen chunks "
+                           "differ, so this compares cost only"}
     mean_rows = cfg.k_chunks * (cfg.chunk_len + 1) + statistics.mean(s % cfg.steps + 1 for s in order)
     attn_bytes = int(cfg.B * mean_rows * cfg.Hkv * cfg.D * 2 * 2 + cfg.B * cfg.Hq * cfg.D * 2 * 2
                      + cfg.B * mean_rows * 4)
@@ -1038,7 +1061,8 @@ def measure_gist(ctx: Ctx, cfg: R.Gist, steps: int, warmup: int):
                 "achieved": round(attn_gbs, 1), "algorithmic_bytes_per_launch": attn_bytes,
                 "launch_ms": round(attn_ms, 5)}
     else:
-        roof = {"kernel": "score_decode_kernel + finish_kernel (the routing call)",
+        roof = {"kernel": ("hier_gist_kernel (the two-level routing call)" if cfg.group_size else
+                           "score_decode_kernel + split_topk_kernel (the routing call)"),
                 "achieved": round(route_gbs, 1), "algorithmic_bytes_per_launch": route_bytes,
                 "launch_ms": round(route_ms, 5)}
     roof.update({"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -1065,6 +1089,10 @@ def measure_gist(ctx: Ctx, cfg: R.Gist, steps: int, warmup: int):
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if compare is not None:
+        line["compare"] = compare
+        line["config"].update({"group_size": cfg.group_size, "meta_gists": cfg.n_chunks // cfg.group_size,
+                               "top_k_groups": cfg.k_groups})
     line["e2e"] = None if args.no_e2e else gist_e2e(gb, ctx, steps, warmup)
     if ctx.rank == 0 and ctx.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_gist(cfg, args.cpu_seconds, gb)
@@ -1252,18 +1280,24 @@ class OracleGist:
         import oracle
         from gen import counter_hash as ch
         self.cfg, self.step = cfg, step
+        self.mk = None
         if bench is not None:
             self.gk = _bits(bench.inp["gist_key"])
             self.qr = _bits(bench.inp["q_route"][step])
             self.q = _bits(bench.inp["q"][step])
+            if cfg.group_size:
+                self.mk = _bits(bench.inp["meta_key"])
         else:
             self.gk = ch.int_bf16(cfg.seed, R.tid(R.KIND_GIST_KEY), count=cfg.B * cfg.n_chunks * cfg.d) \
                 .reshape(cfg.B, cfg.n_chunks, cfg.d)
             self.qr = R.gist_q_route_host(cfg, step)
             self.q = R.gist_q_host(cfg, step)
+            if cfg.group_size:
+                ng = cfg.n_chunks // cfg.group_size
+                self.mk = ch.int_bf16(cfg.seed, R.tid(R.KIND_META_KEY), count=cfg.B * ng * cfg.d).reshape(cfg.B, ng, cfg.d)
         self.rows = []
         for b in range(cfg.B):
-            rr, _ = oracle.gist_route_unfold(self.qr[b], self.gk[b], cfg.chunk_len, cfg.k_chunks, step + 1)
+            rr = self._route(b)
             if bench is not None:
                 import torch
                 r = torch.as_tensor(np.asarray(rr, dtype=np.int64), device=bench.dev)
@@ -1272,11 +1306,19 @@ class OracleGist:
                 self.rows.append((R.host_rows(cfg.seed, R.tid(R.KIND_K, 0), (cfg.Hkv, cfg.D), rr, True, b, cfg.Tk_max),
                                   R.host_rows(cfg.seed, R.tid(R.KIND_V, 0), (cfg.Hkv, cfg.D), rr, True, b, cfg.Tk_max)))
 
+    def _route(self, b):
+        import oracle
+        c = self.cfg
+        if c.group_size:
+            return oracle.hier_gist_route_unfold(self.qr[b], self.mk[b], self.gk[b], c.group_size, c.chunk_len,
+                                                 c.k_groups, c.k_chunks, self.step + 1)[0]
+        return oracle.gist_route_unfold(self.qr[b], self.gk[b], c.chunk_len, c.k_chunks, self.step + 1)[0]
+
     def run(self):
         import oracle
         c = self.cfg
         for b in range(c.B):
-            oracle.gist_route_unfold(self.qr[b], self.gk[b], c.chunk_len, c.k_chunks, self.step + 1)
+            self._route(b)
         oracle.sparse_attention_decode(self.q, [r[0] for r in self.rows], [r[1] for r in self.rows])
 
 

@@ -35,6 +35,7 @@ KIND_GIST_KEY = 7
 KIND_NEEDLE_T = 8
 KIND_NEEDLE_P = 9
 KIND_W_IDX = 10
+KIND_META_KEY = 11
 
 
 def tid(kind: int, index: int = 0) -> int:
@@ -100,6 +101,8 @@ class Gist:
     Hkv: int
     D: int
     steps: int
+    group_size: int = 0     # > 0: two-level routing, one meta-gist per group of chunks
+    k_groups: int = 0
 
     @property
     def Tk_max(self) -> int:
@@ -133,6 +136,11 @@ DECODE_32K_MH16 = Decode("decode_b8_32k_4layers_idx16heads", seed=6, B=8, N=3276
 # layer attends over the compact rows with its own queries.
 YOCO_32K = Decode("yoco_decode_b8_32k_4layers_one_cache", seed=7, B=8, N=32768, d=128, Hq=32, Hkv=8, D=128,
                   k=2048, n_layers=4, share_every=4, steps=64, shared_kv=True)
+
+# The gist decode step with two-level routing: one meta-gist per 16 chunks
+# (512 meta keys), the top 8 groups' 128 chunks compete for the 64 unfolded.
+HGIST_128K = Gist("hgist_decode_b4_128k_meta16", seed=8, B=4, n_chunks=8192, chunk_len=16, d=128, k_chunks=64,
+                  Hq=32, Hkv=8, D=128, steps=16, group_size=16, k_groups=8)
 
 ALL = [PREFILL_2K, DECODE_32K, PREFILL_64K, GIST_128K, DECODE_1M]
 

@@ -86,7 +86,11 @@ def gist_inputs(cfg: R.Gist, device):
     """gist_key [B, n_chunks, d]; K, V [B, Tk_max, Hkv, D] (interleaved cache);
     q_route [steps, B, d]; q [steps, B, Hq, D]; partial_len[s] = s + 1."""
     s = cfg.seed
+    extra = {}
+    if cfg.group_size:
+        extra["meta_key"] = dev_int((cfg.B, cfg.n_chunks // cfg.group_size, cfg.d), s, R.tid(R.KIND_META_KEY), device)
     return {
+        **extra,
         "gist_key": dev_int((cfg.B, cfg.n_chunks, cfg.d), s, R.tid(R.KIND_GIST_KEY), device),
         "K": dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_K, 0), device),
         "V": dev_normal((cfg.B, cfg.Tk_max, cfg.Hkv, cfg.D), s, R.tid(R.KIND_V, 0), device),

@@ -314,6 +314,34 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key,
                                void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Two-level (coarse-to-fine) gist routing with selective unfolding.
+ *
+ * [SSA] §五 (H-SSA) and [GSA] 2.4 (H-GSA): gists of gists.  Every complete
+ * group of group_size consecutive chunks has one meta-gist routing key.  The
+ * query is scored against every meta key and the top k_groups groups are
+ * kept (equal scores: lower group first); the candidate chunks are those of
+ * the kept groups plus the chunks after the last complete group (which has
+ * no meta-gist yet); the query is scored against their gist keys and the top
+ * k_chunks candidates are kept (equal scores: lower chunk first) and
+ * unfolded exactly as by sa_gist_route_unfold.  Meta-gists are routing keys
+ * only: their rows are not part of the attended context.
+ *
+ *   q_route   [B, d] bf16;  meta_key [B, n_chunks / group_size, d] bf16;
+ *   gist_key  [B, n_chunks, d] bf16;  partial_len [B] int32 or NULL
+ *   rows_out  [B, k_chunks*(chunk_len+1) + chunk_len] int32;  count_out [B]
+ *   chunks_out [B, k_chunks] int32 or NULL;  groups_out [B, k_groups] int32
+ *   or NULL (kept groups ascending, -1 padded)
+ * No workspace.  Supported: d in {64, 128}; 1 <= chunk_len <= 256;
+ * n_chunks / group_size <= 8192 and min(k_groups, n_chunks / group_size) *
+ * group_size + (n_chunks % group_size) <= 8192; 1 <= k_chunks <= SA_MAX_K.
+ * ---------------------------------------------------------------------- */
+sa_status sa_hier_gist_route_unfold(const void* q_route, const void* meta_key, const void* gist_key,
+                                    int B, int n_chunks, int chunk_len, int group_size, int d,
+                                    int k_groups, int k_chunks, const int32_t* partial_len,
+                                    int32_t* rows_out, int32_t* count_out, int32_t* chunks_out,
+                                    int32_t* groups_out, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Shared index cache (host object; its device buffers are caller-owned).
  *
  * [IC] §二 and §六: layers are "full" (run their own indexer and store the

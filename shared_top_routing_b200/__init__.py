@@ -16,6 +16,7 @@ from .sa import (  # noqa: F401
     lib,
     sa_gather_rows,
     sa_gist_route_unfold,
+    sa_hier_gist_route_unfold,
     sa_index_score_topk,
     sa_index_score_topk_mh,
     sa_sparse_attn_decode,
@@ -35,6 +36,7 @@ __all__ = [
     "lib",
     "sa_gather_rows",
     "sa_gist_route_unfold",
+    "sa_hier_gist_route_unfold",
     "sa_index_score_topk",
     "sa_index_score_topk_mh",
     "sa_sparse_attn_decode",

@@ -471,6 +471,43 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   return ok();
 }
 
+sa_status sa_hier_gist_route_unfold(const void* q_route, const void* meta_key, const void* gist_key, int B,
+                                    int n_chunks, int chunk_len, int group_size, int d, int k_groups, int k_chunks,
+                                    const int32_t* partial_len, int32_t* rows_out, int32_t* count_out,
+                                    int32_t* chunks_out, int32_t* groups_out, sa_stream_t stream) {
+  if (B < 0 || n_chunks < 0) return fail(SA_ERR_INVALID_ARG, "bad sizes: B=%d n_chunks=%d", B, n_chunks);
+  if (group_size < 1) return fail(SA_ERR_INVALID_ARG, "group_size=%d must be >= 1", group_size);
+  if (chunk_len < 1 || chunk_len > 256)
+    return fail(SA_ERR_UNSUPPORTED, "chunk_len=%d unsupported (1..256)", chunk_len);
+  if (k_groups < 1 || k_chunks < 1) return fail(SA_ERR_INVALID_ARG, "k_groups and k_chunks must be >= 1");
+  if (k_chunks > SA_MAX_K) return fail(SA_ERR_UNSUPPORTED, "k_chunks=%d exceeds SA_MAX_K", k_chunks);
+  if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "d=%d unsupported (64 or 128)", d);
+  const long long n_groups = n_chunks / group_size;
+  const long long cand = std::min<long long>(k_groups, n_groups) * group_size + (n_chunks - n_groups * group_size);
+  if (n_groups > sa::kHierMax || cand > sa::kHierMax)
+    return fail(SA_ERR_UNSUPPORTED, "%lld groups / %lld candidate chunks exceed %d", n_groups, cand, sa::kHierMax);
+  if ((long long)(n_chunks + 1) * (chunk_len + 1) > 0x7FFFFFFFll) return fail(SA_ERR_UNSUPPORTED, "row ids overflow int32");
+  if (B == 0) return ok();
+  if (!q_route || !gist_key || !rows_out || !count_out || (n_groups > 0 && !meta_key))
+    return fail(SA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned(q_route, 16) || !aligned(gist_key, 16) || (meta_key && !aligned(meta_key, 16)))
+    return fail(SA_ERR_INVALID_ARG, "q_route, meta_key and gist_key must be 16-byte aligned");
+  sa::FinishOut out;
+  out.count = count_out;
+  out.rows = rows_out;
+  out.rows_stride = k_chunks * (chunk_len + 1) + chunk_len;
+  out.chunk_len = chunk_len;
+  out.n_chunks = n_chunks;
+  out.partial_len = partial_len;
+  out.chunks = chunks_out;
+  const cudaError_t e = sa::launch_hier_gist(
+      static_cast<const uint16_t*>(q_route), static_cast<const uint16_t*>(meta_key),
+      static_cast<const uint16_t*>(gist_key), B, d, n_chunks, group_size, k_groups, k_chunks, out, groups_out,
+      as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hier gist launch");
+  return ok();
+}
+
 }  // extern "C"
 
 // ========================================================= index cache

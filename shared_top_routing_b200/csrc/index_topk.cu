@@ -1354,6 +1354,129 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
   if (tid == 0) w.cand_cnt[r] = 0u;
 }
 
+// ------------------------------------------------------ two-level gist routing
+//
+// hier_gist_kernel: one CTA per sequence routes one decode query coarse to
+// fine ([SSA] §五 H-SSA, [GSA] 2.4): (1) the query is scored against the
+// meta-gist key of every complete group of group_size chunks and the top
+// k_groups groups are kept; (2) the candidate chunks -- those of the kept
+// groups, in ascending order, then the chunks after the last complete group
+// (no meta-gist yet) -- are scored against their gist keys and the top
+// k_chunks are kept; (3) they are unfolded like single-level routing.  Both
+// selections are the exact radix select of the other paths (equal scores:
+// lower group / chunk first); the chosen items are placed in ascending
+// order by block scans.  Scores are fp32 sums of bf16 products (exact for
+// integer-valued inputs).
+
+constexpr int kHgThreads = 256;
+constexpr int kHgMax = 8192;   // meta keys, and candidate chunks, held in shared memory
+
+struct HGistSmem {
+  static constexpr int kBmw = 256;   // bounds the select's tie list
+  uint32_t hist[256];
+  uint32_t swarp[33];
+  uint32_t digit, above, bnd_count;
+  uint32_t kor, kand, por, pand;
+  uint32_t bits[256];
+  alignas(16) float q[128];
+  alignas(16) uint32_t key[kHgMax];
+  uint32_t list[kHgMax];           // kept groups in ascending order
+};
+
+template <int D>
+__device__ __forceinline__ float hg_dot(const uint16_t* __restrict__ krow, const float* qs) {
+  const uint4* kv = reinterpret_cast<const uint4*>(krow);
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) s += dot8(__ldg(kv + c), qs + 8 * c);
+  return s;
+}
+
+// Ascending list of the chosen items among n (one block scan per pass of
+// kHgThreads items): out[slot] = index.  Returns the number placed.
+__device__ __forceinline__ uint32_t hg_place(HGistSmem& s, const uint32_t* key, int n, uint32_t prefix,
+                                             uint32_t pmask, uint32_t pmax, uint32_t* out, uint32_t cap) {
+  uint32_t base = 0;
+  for (int i0 = 0; i0 < n; i0 += kHgThreads) {
+    const int i = i0 + threadIdx.x;
+    const bool sel = i < n && is_selected(key[i], (uint32_t)i, prefix, pmask, pmax);
+    uint32_t tot;
+    const uint32_t o = base + block_excl_scan(sel ? 1u : 0u, s.swarp, tot);
+    if (sel && o < cap) out[o] = (uint32_t)i;
+    base += tot;
+  }
+  __syncthreads();
+  return base < cap ? base : cap;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kHgThreads)
+hier_gist_kernel(const uint16_t* __restrict__ q_route, const uint16_t* __restrict__ meta_key,
+                 const uint16_t* __restrict__ gist_key, int n_chunks, int group_size, int k_groups, int k,
+                 FinishOut out, int32_t* __restrict__ groups_out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  HGistSmem& s = *reinterpret_cast<HGistSmem*>(smem_raw);
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int n_groups = n_chunks / group_size;
+  for (int i = tid; i < D; i += kHgThreads) {
+    const uint16_t v = q_route[(long long)b * D + i];
+    s.q[i] = __uint_as_float((uint32_t)v << 16);
+  }
+  __syncthreads();
+
+  // ---- 1. coarse: meta keys of the complete groups
+  const uint16_t* mk = meta_key + (long long)b * n_groups * D;
+  for (int g = tid; g < n_groups; g += kHgThreads) s.key[g] = score_key(hg_dot<D>(mk + (long long)g * D, s.q));
+  __syncthreads();
+  const uint32_t KG = (uint32_t)min(k_groups, n_groups);
+  uint32_t prefix = 0u, pmask = 0u, pmax = 0xFFFFFFFFu;   // every item chosen
+  if (KG > 0 && KG < (uint32_t)n_groups) {
+    const Items it{s.key, nullptr, n_groups};
+    select_threshold<HGistSmem, kHgThreads>(s, it, SelStart{0u, 0u, KG, (uint32_t)n_groups, 24, false}, prefix,
+                                            pmask, pmax);
+  }
+  const uint32_t n_sel = KG > 0 ? hg_place(s, s.key, n_groups, prefix, pmask, pmax, s.list, KG) : 0u;
+  if (groups_out != nullptr)
+    for (int i = tid; i < k_groups; i += kHgThreads)
+      groups_out[(long long)b * k_groups + i] = i < (int)n_sel ? (int32_t)s.list[i] : -1;
+
+  // ---- 2. fine: gist keys of the candidate chunks (ascending chunk order)
+  const int trail0 = n_groups * group_size;
+  const int n_cand = (int)n_sel * group_size + (n_chunks - trail0);
+  auto cand_chunk = [&](int j) {
+    return j < (int)n_sel * group_size ? (int)s.list[j / group_size] * group_size + j % group_size
+                                       : trail0 + (j - (int)n_sel * group_size);
+  };
+  const uint16_t* gk = gist_key + (long long)b * n_chunks * D;
+  for (int j = tid; j < n_cand; j += kHgThreads)
+    s.key[j] = score_key(hg_dot<D>(gk + (long long)cand_chunk(j) * D, s.q));
+  __syncthreads();
+  const uint32_t K = (uint32_t)min(k, n_cand);
+  prefix = 0u;
+  pmask = 0u;
+  pmax = 0xFFFFFFFFu;
+  if (K > 0 && K < (uint32_t)n_cand) {
+    const Items it{s.key, nullptr, n_cand};
+    select_threshold<HGistSmem, kHgThreads>(s, it, SelStart{0u, 0u, K, (uint32_t)n_cand, 24, false}, prefix, pmask,
+                                            pmax);
+  }
+
+  // ---- 3. unfold the chosen chunks in ascending order
+  const long long o_idx = (long long)b * k;
+  uint32_t base = 0;
+  for (int i0 = 0; i0 < n_cand; i0 += kHgThreads) {
+    const int j = i0 + tid;
+    const bool sel = K > 0 && j < n_cand && is_selected(s.key[j], (uint32_t)j, prefix, pmask, pmax);
+    uint32_t tot;
+    const uint32_t o = base + block_excl_scan(sel ? 1u : 0u, s.swarp, tot);
+    if (sel && o < K) emit(out, o_idx, b, o, (uint32_t)cand_chunk(j), 0u);
+    base += tot;
+  }
+  finish_tail(out, b, 0, 1, k, K, false, tid, kHgThreads);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ host side
@@ -1481,6 +1604,24 @@ cudaError_t launch_split_topk(int B, int rows_per_batch, int t0, int Tq, int Tk,
   if (e != cudaSuccess) return e;
   e = launch_pdl(split_topk_kernel, dim3((unsigned)F, (unsigned)rows), dim3(kSplitThreads), smem, st, w,
                  rows_per_batch, t0, Tq, Tk, q_pos0, kv_len, k, (int)chunk, out);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_hier_gist(const uint16_t* q_route, const uint16_t* meta_key, const uint16_t* gist_key, int B,
+                             int d, int n_chunks, int group_size, int k_groups, int k, const FinishOut& out,
+                             int32_t* groups_out, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  const size_t smem = sizeof(HGistSmem);
+  cudaError_t e;
+  if (d == 128) {
+    if ((e = ensure_dynamic_smem((const void*)hier_gist_kernel<128>, smem)) != cudaSuccess) return e;
+    e = launch_pdl(hier_gist_kernel<128>, dim3((unsigned)B), dim3(kHgThreads), smem, st, q_route, meta_key,
+                   gist_key, n_chunks, group_size, k_groups, k, out, groups_out);
+  } else {
+    if ((e = ensure_dynamic_smem((const void*)hier_gist_kernel<64>, smem)) != cudaSuccess) return e;
+    e = launch_pdl(hier_gist_kernel<64>, dim3((unsigned)B), dim3(kHgThreads), smem, st, q_route, meta_key,
+                   gist_key, n_chunks, group_size, k_groups, k, out, groups_out);
+  }
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -127,6 +127,12 @@ int mh_rows_per_launch(int B, int Tq, int Tk_max);
 cudaError_t launch_score_mh(const uint16_t* q, const float* wts, const uint16_t* kmat, int B, int H, int d,
                             int rows_per_batch, int t0, int Tq, int Tk_max, int Tk, int q_pos0,
                             const int32_t* kv_len, const RowWorkspace& w, bool with_hist, cudaStream_t st);
+// Two-level gist routing, one CTA per sequence (shared memory holds up to
+// kHierMax meta keys and kHierMax candidate chunks).
+constexpr int kHierMax = 8192;
+cudaError_t launch_hier_gist(const uint16_t* q_route, const uint16_t* meta_key, const uint16_t* gist_key, int B,
+                             int d, int n_chunks, int group_size, int k_groups, int k, const FinishOut& out,
+                             int32_t* groups_out, cudaStream_t st);
 // Largest number of indexer heads of the multi-head indexer for key width d.
 constexpr int mh_max_heads(int d) { return d == 64 ? 64 : 32; }
 // Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`

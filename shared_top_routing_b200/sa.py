@@ -48,6 +48,7 @@ SIGNATURES = {
     "sa_self_test_bounded_wait": (_I, [_P, ctypes.c_uint32, _P]),
     "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
     "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "sa_hier_gist_route_unfold": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
     "sa_index_cache_destroy": (None, [_P]),
     "sa_index_cache_is_full": (_I, [_P, _I]),
@@ -369,6 +370,40 @@ def sa_gist_route_unfold(q_route, gist_key, chunk_len: int, k_chunks: int, parti
                                     _stream(stream))
     _check(st, "sa_gist_route_unfold")
     return (rows_out, count_out, chunks) if with_chunks else (rows_out, count_out)
+
+
+def sa_hier_gist_route_unfold(q_route, meta_key, gist_key, chunk_len: int, group_size: int, k_groups: int,
+                              k_chunks: int, partial_len=None, rows_out=None, count_out=None,
+                              with_chunks: bool = False, with_groups: bool = False, stream=None):
+    """Two-level gist routing (see sa.h).  q_route [B, d]; meta_key
+    [B, n_chunks // group_size, d]; gist_key [B, n_chunks, d].
+    Returns (rows, count[, chunks][, groups])."""
+    torch = _torch()
+    B, d = q_route.shape
+    n_chunks = gist_key.shape[1]
+    _need(q_route, "q_route", 2)
+    _need(meta_key, "meta_key", 2)
+    _need(gist_key, "gist_key", 2)
+    if partial_len is not None:
+        _need(partial_len, "partial_len", 4)
+    dev = q_route.device
+    stride = k_chunks * (chunk_len + 1) + chunk_len
+    if rows_out is None:
+        rows_out = torch.empty((B, stride), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    chunks = torch.empty((B, k_chunks), dtype=torch.int32, device=dev) if with_chunks else None
+    groups = torch.empty((B, k_groups), dtype=torch.int32, device=dev) if with_groups else None
+    st = lib().sa_hier_gist_route_unfold(_ptr(q_route), _ptr(meta_key), _ptr(gist_key), B, n_chunks, chunk_len,
+                                         group_size, d, k_groups, k_chunks, _ptr(partial_len), _ptr(rows_out),
+                                         _ptr(count_out), _ptr(chunks), _ptr(groups), _stream(stream))
+    _check(st, "sa_hier_gist_route_unfold")
+    res = [rows_out, count_out]
+    if with_chunks:
+        res.append(chunks)
+    if with_groups:
+        res.append(groups)
+    return tuple(res)
 
 
 class IndexCache:

@@ -552,6 +552,56 @@ def test_gist_route_unfold_matches_oracle(n_chunks, k_chunks, chunk_len, partial
         assert np.all(chunks[b, rc.size:] == -1)
 
 
+@pytest.mark.parametrize("n_chunks,M,k_groups,k_chunks,chunk_len,partial,d", [
+    (8192, 16, 8, 64, 16, 5, 128), (8192, 16, 8, 128, 16, 16, 128), (1000, 7, 12, 40, 4, 0, 64),
+    (40, 8, 10, 20, 16, 3, 128), (300, 32, 2, 100, 8, 8, 64), (5, 8, 3, 4, 16, 2, 128)])
+def test_hier_gist_route_unfold_matches_oracle(n_chunks, M, k_groups, k_chunks, chunk_len, partial, d):
+    """[SSA] §五 / [GSA] 2.4: coarse meta-gist selection, fine gist selection
+    among the kept groups' chunks plus the trailing chunks, unfolding.  Cases:
+    the bench's shape, every candidate kept, a ragged trailing group, every
+    group kept, fewer candidates than k, and no complete group at all."""
+    B = 3
+    seed = n_chunks + M
+    qr = _ints(seed, 1, (B, d))
+    gk = _ints(seed, 2, (B, n_chunks, d))
+    mk = _ints(seed, 3, (B, n_chunks // M, d))
+    part = i32([partial, 0, chunk_len][:B])
+    rows, cnt, chunks, groups = sa.sa_hier_gist_route_unfold(to_dev(qr), to_dev(mk), to_dev(gk), chunk_len, M,
+                                                             k_groups, k_chunks, part, with_chunks=True,
+                                                             with_groups=True)
+    torch.cuda.synchronize()
+    rows, cnt, chunks, groups = (x.cpu().numpy() for x in (rows, cnt, chunks, groups))
+    for b, p in enumerate([partial, 0, chunk_len][:B]):
+        rr, rc, rg = oracle.hier_gist_route_unfold(qr[b], mk[b], gk[b], M, chunk_len, k_groups, k_chunks, p)
+        np.testing.assert_array_equal(groups[b, : rg.size], rg)
+        assert (groups[b, rg.size:] == -1).all()
+        np.testing.assert_array_equal(chunks[b, : rc.size], rc)
+        assert (chunks[b, rc.size:] == -1).all()
+        assert cnt[b] == rr.size
+        np.testing.assert_array_equal(rows[b, : rr.size], rr)
+        assert (rows[b, rr.size:] == -1).all()
+
+
+def test_hier_gist_ties_and_limits():
+    B, n_chunks, M, d = 2, 4096, 16, 64
+    qr = np.zeros((B, d), np.uint16)                 # every score 0: lowest groups and chunks win
+    gk = _ints(5, 2, (B, n_chunks, d))
+    mk = _ints(5, 3, (B, n_chunks // M, d))
+    rows, cnt, chunks, groups = sa.sa_hier_gist_route_unfold(to_dev(qr), to_dev(mk), to_dev(gk), 16, M, 4, 10,
+                                                             None, with_chunks=True, with_groups=True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(groups.cpu().numpy(), np.tile(np.arange(4), (B, 1)))
+    np.testing.assert_array_equal(chunks.cpu().numpy(), np.tile(np.arange(10), (B, 1)))
+    assert (cnt.cpu().numpy() == 10 * 17).all()
+    fake = ctypes.c_void_p(0x100000)
+    L = sa.lib()
+    # too many meta keys / candidates for one CTA's shared memory: refused on the host
+    assert L.sa_hier_gist_route_unfold(fake, fake, fake, 1, 8193 * 2, 16, 1, 64, 4, 4, None, fake, fake, None, None,
+                                       None) == sa.SA_ERR_UNSUPPORTED
+    assert L.sa_hier_gist_route_unfold(fake, fake, fake, 1, 100000, 16, 16, 64, 600, 4, None, fake, fake, None,
+                                       None, None) == sa.SA_ERR_UNSUPPORTED
+
+
 def test_gist_equal_scores_take_first_chunks():
     B, n_chunks, d = 2, 300, 64
     qr = np.zeros((B, d), np.uint16)

@@ -191,15 +191,22 @@ def test_prefill_64k_needles_sampled_rows():
 
 # -------------------------------------------------------------------- gist
 
-def test_gist_decode_128k():
-    cfg = R.GIST_128K
+def _check_gist(cfg):
     d = dev()
     inp = TI.gist_inputs(cfg, d)
     host_gk = ch.int_bf16(cfg.seed, R.tid(R.KIND_GIST_KEY), count=cfg.B * cfg.n_chunks * cfg.d) \
         .reshape(cfg.B, cfg.n_chunks, cfg.d)
+    ng = cfg.n_chunks // cfg.group_size if cfg.group_size else 0
+    host_mk = ch.int_bf16(cfg.seed, R.tid(R.KIND_META_KEY), count=cfg.B * ng * cfg.d).reshape(cfg.B, ng, cfg.d) \
+        if cfg.group_size else None
     for s in (0, cfg.steps - 1):
-        rows, cnt = sa.sa_gist_route_unfold(inp["q_route"][s], inp["gist_key"], cfg.chunk_len,
-                                            cfg.k_chunks, inp["partial_len"][s])
+        if cfg.group_size:
+            rows, cnt = sa.sa_hier_gist_route_unfold(inp["q_route"][s], inp["meta_key"], inp["gist_key"],
+                                                     cfg.chunk_len, cfg.group_size, cfg.k_groups, cfg.k_chunks,
+                                                     inp["partial_len"][s])
+        else:
+            rows, cnt = sa.sa_gist_route_unfold(inp["q_route"][s], inp["gist_key"], cfg.chunk_len,
+                                                cfg.k_chunks, inp["partial_len"][s])
         out = sa.sa_sparse_attn_decode(inp["q"][s], inp["K"], inp["V"], rows, cnt)
         torch.cuda.synchronize()
         rows, cnt, out = rows.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy()
@@ -207,12 +214,26 @@ def test_gist_decode_128k():
         q = R.gist_q_host(cfg, s)
         Kr, Vr = [], []
         for b in range(cfg.B):
-            rr, _ = oracle.gist_route_unfold(qr[b], host_gk[b], cfg.chunk_len, cfg.k_chunks, s + 1)
+            if cfg.group_size:
+                rr = oracle.hier_gist_route_unfold(qr[b], host_mk[b], host_gk[b], cfg.group_size, cfg.chunk_len,
+                                                   cfg.k_groups, cfg.k_chunks, s + 1)[0]
+            else:
+                rr, _ = oracle.gist_route_unfold(qr[b], host_gk[b], cfg.chunk_len, cfg.k_chunks, s + 1)
             assert cnt[b] == rr.size == cfg.k_chunks * 17 + s + 1
             np.testing.assert_array_equal(rows[b, : rr.size], rr)
             Kr.append(R.host_rows(cfg.seed, R.tid(R.KIND_K, 0), (cfg.Hkv, cfg.D), rr, True, b, cfg.Tk_max))
             Vr.append(R.host_rows(cfg.seed, R.tid(R.KIND_V, 0), (cfg.Hkv, cfg.D), rr, True, b, cfg.Tk_max))
         ref, _ = oracle.sparse_attention_decode(q, Kr, Vr)
-        assert_close_attn(out, ref, f"gist step {s}")
+        assert_close_attn(out, ref, f"{cfg.name} step {s}")
     inp.clear()
     _free()
+
+
+def test_gist_decode_128k():
+    _check_gist(R.GIST_128K)
+
+
+def test_hier_gist_decode_128k_meta16():
+    """The bench's two-level gist workload: 512 meta keys, 8 groups kept,
+    64 of their 128 chunks unfolded, then attention."""
+    _check_gist(R.HGIST_128K)
