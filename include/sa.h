@@ -342,6 +342,32 @@ sa_status sa_hier_gist_route_unfold(const void* q_route, const void* meta_key, c
                                     int32_t* groups_out, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Index overlap between layers, and a training-free layer-role search.
+ *
+ * [IC] §一: the top-k sets of adjacent layers' indexers overlap by 70-100%,
+ * which is why a shared layer can reuse a full layer's index.
+ * sa_index_overlap counts, per row, the positions two selections share:
+ *   idx_a, idx_b   [rows, k] int32, each row ascending (as every selection
+ *                  of this library is) within its count; count_a, count_b
+ *                  [rows] int32 (clamped to [0, k]); inter_out [rows] int32.
+ *
+ * [IC] §三: starting with every layer full, the indexer whose removal hurts
+ * least is removed, repeatedly.  sa_index_pattern_greedy runs that search on
+ * the host with the retained overlap as the measure (the pages measure a
+ * model's loss on calibration data, which needs a trained model):
+ *   overlap        [n_layers, n_layers] row-major: overlap[l, j] = mean
+ *                  fraction of layer l's own selection contained in layer
+ *                  j's (j <= l is what a shared layer reads)
+ *   pattern_out    n_layers + 1 chars: 'F'/'S' per layer and a NUL.  Layer 0
+ *                  stays full; n_full layers stay full; ties remove the
+ *                  lower layer first.  The pattern feeds sa_index_cache_create.
+ * ---------------------------------------------------------------------- */
+sa_status sa_index_overlap(const int32_t* idx_a, const int32_t* count_a, const int32_t* idx_b,
+                           const int32_t* count_b, int rows, int k, int32_t* inter_out,
+                           sa_stream_t stream);
+sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_full, char* pattern_out);
+
+/* ------------------------------------------------------------------------
  * Shared index cache (host object; its device buffers are caller-owned).
  *
  * [IC] §二 and §六: layers are "full" (run their own indexer and store the

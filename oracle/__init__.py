@@ -24,6 +24,8 @@ from .reference import (  # noqa: F401
     gist_route_unfold,
     hier_gist_route_unfold,
     layer_owners,
+    index_overlap,
+    greedy_pattern,
     kv_cache_gib,
     pair_counts,
 )

@@ -42,6 +42,10 @@ Readings where the pages are silent (each also stated where it is used):
    after the last complete group have no meta-gist yet and are always
    second-stage candidates; the unfolded rows are those of single-level
    routing for the chunks chosen in the second stage.
+9. The layer-role search of IndexCache needs a trained model and a
+   calibration loss; here the loss of sharing is stood in for by the index
+   overlap itself (1 - overlap of a layer's own selection with the one it
+   would reuse), the greedy removal order being the page's.
 """
 from __future__ import annotations
 
@@ -302,7 +306,54 @@ def layer_owners(n_layers: int, pattern: str | None = None, share_every: int | N
     return owners
 
 
-# -------------------------------------------------------------- accounting
+def index_overlap(idx_a, count_a, idx_b, count_b) -> np.ndarray:
+    """Per row, how many positions two selections share ([IC] §一: adjacent
+    layers' indexers pick 70-100% of the same tokens).  idx_*: [rows, k]
+    (entries past count_* ignored).  Returns int64 [rows]."""
+    ia = np.asarray(idx_a)
+    ib = np.asarray(idx_b)
+    ca = np.asarray(count_a).reshape(-1)
+    cb = np.asarray(count_b).reshape(-1)
+    ia = ia.reshape(ca.size, -1)
+    ib = ib.reshape(cb.size, -1)
+    return np.array([np.intersect1d(ia[r, : ca[r]], ib[r, : cb[r]]).size for r in range(ca.size)], dtype=np.int64)
+
+
+def greedy_pattern(overlap, n_full: int) -> str:
+    """Training-free layer-role search ([IC] §三, reading 9): start with every
+    layer full; repeatedly make shared the one full layer (never layer 0)
+    whose removal keeps the largest total retained overlap, until n_full
+    full layers remain.  A shared layer reads its nearest preceding full
+    layer's index, and retains overlap[l, owner] of its own selection
+    (overlap[l, j]: mean fraction of layer l's own top-k that layer j's top-k
+    contains).  Equal totals: the lower layer is made shared first."""
+    ov = np.asarray(overlap, dtype=np.float64)
+    L = ov.shape[0]
+    full = [True] * L
+
+    def total(fl):
+        owner, t = 0, 0.0
+        for l in range(L):
+            if fl[l]:
+                owner = l
+            t += ov[l, owner]
+        return t
+
+    while sum(full) > max(1, n_full):
+        best, best_t = None, None
+        for l in range(1, L):
+            if not full[l]:
+                continue
+            trial = list(full)
+            trial[l] = False
+            t = total(trial)
+            if best_t is None or t > best_t:
+                best, best_t = l, t
+        full[best] = False
+    return "".join("F" if f else "S" for f in full)
+
+
+# -------------------------------------------------------------- accounting# -------------------------------------------------------------- accounting
 
 def kv_cache_gib(n_layers: int, kv_heads: int, head_dim: int, n_tok: int, bytes_per: int = 2) -> float:
     """KV-cache size in GiB: layers x kv heads x head dim x 2 (K and V) x

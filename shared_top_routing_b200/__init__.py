@@ -17,6 +17,8 @@ from .sa import (  # noqa: F401
     sa_gather_rows,
     sa_gist_route_unfold,
     sa_hier_gist_route_unfold,
+    sa_index_overlap,
+    sa_index_pattern_greedy,
     sa_index_score_topk,
     sa_index_score_topk_mh,
     sa_sparse_attn_decode,
@@ -37,6 +39,8 @@ __all__ = [
     "sa_gather_rows",
     "sa_gist_route_unfold",
     "sa_hier_gist_route_unfold",
+    "sa_index_overlap",
+    "sa_index_pattern_greedy",
     "sa_index_score_topk",
     "sa_index_score_topk_mh",
     "sa_sparse_attn_decode",

@@ -508,6 +508,57 @@ sa_status sa_hier_gist_route_unfold(const void* q_route, const void* meta_key, c
   return ok();
 }
 
+sa_status sa_index_overlap(const int32_t* idx_a, const int32_t* count_a, const int32_t* idx_b,
+                           const int32_t* count_b, int rows, int k, int32_t* inter_out, sa_stream_t stream) {
+  if (rows < 0 || k < 1) return fail(SA_ERR_INVALID_ARG, "bad sizes: rows=%d k=%d", rows, k);
+  if (rows == 0) return ok();
+  if (!idx_a || !count_a || !idx_b || !count_b || !inter_out) return fail(SA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(idx_a, 4) || !aligned(idx_b, 4) || !aligned(count_a, 4) || !aligned(count_b, 4) ||
+      !aligned(inter_out, 4))
+    return fail(SA_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  const cudaError_t e = sa::launch_index_overlap(idx_a, count_a, idx_b, count_b, rows, k, inter_out,
+                                                 as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "index_overlap launch");
+  return ok();
+}
+
+sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_full, char* pattern_out) {
+  if (!overlap || !pattern_out) return fail(SA_ERR_INVALID_ARG, "NULL pointer");
+  if (n_layers < 1 || n_full < 1) return fail(SA_ERR_INVALID_ARG, "n_layers=%d and n_full=%d must be >= 1",
+                                              n_layers, n_full);
+  std::vector<char> full(n_layers, 1);
+  auto total = [&](const std::vector<char>& f) {
+    int owner = 0;
+    double t = 0.0;
+    for (int l = 0; l < n_layers; ++l) {
+      if (f[l]) owner = l;
+      t += overlap[(size_t)l * n_layers + owner];
+    }
+    return t;
+  };
+  int n = n_layers;
+  while (n > n_full) {
+    int best = -1;
+    double best_t = 0.0;
+    for (int l = 1; l < n_layers; ++l) {
+      if (!full[l]) continue;
+      full[l] = 0;
+      const double t = total(full);
+      full[l] = 1;
+      if (best < 0 || t > best_t) {
+        best = l;
+        best_t = t;
+      }
+    }
+    if (best < 0) break;   // only layer 0 is left
+    full[best] = 0;
+    --n;
+  }
+  for (int l = 0; l < n_layers; ++l) pattern_out[l] = full[l] ? 'F' : 'S';
+  pattern_out[n_layers] = '\0';
+  return ok();
+}
+
 }  // extern "C"
 
 // ========================================================= index cache

@@ -1477,6 +1477,39 @@ hier_gist_kernel(const uint16_t* __restrict__ q_route, const uint16_t* __restric
   finish_tail(out, b, 0, 1, k, K, false, tid, kHgThreads);
 }
 
+// ------------------------------------------------------------ index overlap
+//
+// index_overlap_kernel: per row, the number of positions two ascending
+// selections share ([IC] §一 measures 70-100% between adjacent layers).  One
+// warp per row: each lane binary-searches its share of A's positions in B.
+
+__global__ void __launch_bounds__(256)
+index_overlap_kernel(const int32_t* __restrict__ a, const int32_t* __restrict__ ca, const int32_t* __restrict__ b,
+                     const int32_t* __restrict__ cb, int rows, int k, int32_t* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;
+  const int na = min(max(ca[r], 0), k), nb = min(max(cb[r], 0), k);
+  const int32_t* A = a + (long long)r * k;
+  const int32_t* Bv = b + (long long)r * k;
+  int hits = 0;
+  for (int i = lane; i < na; i += 32) {
+    const int32_t x = A[i];
+    int lo = 0, hi = nb;   // first position in B not below x
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (Bv[mid] < x) lo = mid + 1;
+      else hi = mid;
+    }
+    hits += (lo < nb && Bv[lo] == x) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) hits += __shfl_xor_sync(0xffffffffu, hits, o);
+  if (lane == 0) out[r] = hits;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ host side
@@ -1622,6 +1655,14 @@ cudaError_t launch_hier_gist(const uint16_t* q_route, const uint16_t* meta_key, 
     e = launch_pdl(hier_gist_kernel<64>, dim3((unsigned)B), dim3(kHgThreads), smem, st, q_route, meta_key,
                    gist_key, n_chunks, group_size, k_groups, k, out, groups_out);
   }
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_index_overlap(const int32_t* a, const int32_t* ca, const int32_t* b, const int32_t* cb, int rows,
+                                 int k, int32_t* out, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const cudaError_t e =
+      launch_pdl(index_overlap_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, a, ca, b, cb, rows, k, out);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

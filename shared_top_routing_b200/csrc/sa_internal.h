@@ -133,6 +133,9 @@ constexpr int kHierMax = 8192;
 cudaError_t launch_hier_gist(const uint16_t* q_route, const uint16_t* meta_key, const uint16_t* gist_key, int B,
                              int d, int n_chunks, int group_size, int k_groups, int k, const FinishOut& out,
                              int32_t* groups_out, cudaStream_t st);
+// Per-row shared positions of two ascending selections.
+cudaError_t launch_index_overlap(const int32_t* a, const int32_t* ca, const int32_t* b, const int32_t* cb, int rows,
+                                 int k, int32_t* out, cudaStream_t st);
 // Largest number of indexer heads of the multi-head indexer for key width d.
 constexpr int mh_max_heads(int d) { return d == 64 ? 64 : 32; }
 // Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`

@@ -49,6 +49,8 @@ SIGNATURES = {
     "sa_gist_route_unfold_workspace": (_Z, [_I, _I, _I, _I]),
     "sa_gist_route_unfold": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_hier_gist_route_unfold": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "sa_index_overlap": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
+    "sa_index_pattern_greedy": (_I, [_P, _I, _I, ctypes.c_char_p]),
     "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
     "sa_index_cache_destroy": (None, [_P]),
     "sa_index_cache_is_full": (_I, [_P, _I]),
@@ -404,6 +406,33 @@ def sa_hier_gist_route_unfold(q_route, meta_key, gist_key, chunk_len: int, group
     if with_groups:
         res.append(groups)
     return tuple(res)
+
+
+def sa_index_overlap(idx_a, count_a, idx_b, count_b, out=None, stream=None):
+    """Per-row count of the positions two selections share.  idx_* [..., k]
+    int32 (ascending rows); count_* [...] int32.  Returns int32 [rows]."""
+    torch = _torch()
+    k = idx_a.shape[-1]
+    rows = idx_a.numel() // k
+    for t, n in ((idx_a, "idx_a"), (idx_b, "idx_b"), (count_a, "count_a"), (count_b, "count_b")):
+        _need(t, n, 4)
+    if out is None:
+        out = torch.empty((rows,), dtype=torch.int32, device=idx_a.device)
+    st = lib().sa_index_overlap(_ptr(idx_a), _ptr(count_a), _ptr(idx_b), _ptr(count_b), rows, k, _ptr(out),
+                                _stream(stream))
+    _check(st, "sa_index_overlap")
+    return out
+
+
+def sa_index_pattern_greedy(overlap, n_full: int) -> str:
+    """Greedy layer-role search on an [L, L] overlap matrix (host; see sa.h)."""
+    import numpy as np
+    ov = np.ascontiguousarray(np.asarray(overlap, dtype=np.float64))
+    L = ov.shape[0]
+    buf = ctypes.create_string_buffer(L + 1)
+    st = lib().sa_index_pattern_greedy(ov.ctypes.data_as(ctypes.c_void_p), L, n_full, buf)
+    _check(st, "sa_index_pattern_greedy")
+    return buf.value.decode()
 
 
 class IndexCache:

@@ -223,3 +223,23 @@ def test_prefill_workspace_grows_with_the_shape_while_one_batch_holds_every_row(
         assert sizes == sorted(sizes)
     sizes = [L.sa_index_score_topk_workspace(b, 300, 8192, 64, 256) for b in (1, 2, 3, 4)]
     assert sizes == sorted(sizes)
+
+
+def test_greedy_pattern_search_matches_the_oracle():
+    """The library's host-side layer-role search ([IC] §三, with the index
+    overlap as the measure) picks the oracle's pattern on random and block
+    structured overlap matrices."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(5)
+    for L, n_full in ((6, 2), (12, 3), (28, 7), (47, 12), (4, 4), (5, 1)):
+        ov = rng.uniform(0.2, 1.0, (L, L))
+        np.fill_diagonal(ov, 1.0)
+        assert S.sa_index_pattern_greedy(ov, n_full) == oracle.greedy_pattern(ov, n_full)
+    blocks = np.full((8, 8), 0.1)   # two blocks of layers: {0, 1, 2} and {3, ..., 7}
+    blocks[:3, :3] = blocks[3:, 3:] = 0.95
+    np.fill_diagonal(blocks, 1.0)
+    assert S.sa_index_pattern_greedy(blocks, 2) == "FSSFSSSS"
+    buf = ctypes.create_string_buffer(9)
+    assert S.lib().sa_index_pattern_greedy(None, 8, 2, buf) == S.SA_ERR_INVALID_ARG
+    assert S.lib().sa_index_overlap(None, None, None, None, 3, 16, None, None) == S.SA_ERR_INVALID_ARG

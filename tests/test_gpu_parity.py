@@ -682,6 +682,55 @@ def test_index_cache_non_uniform_pattern_fssfsf():
     cache.close()
 
 
+def test_index_overlap_and_a_searched_pattern_end_to_end():
+    """[IC] §一-§三 on synthetic layers: six layers in two blocks whose
+    indexer queries differ little inside a block; each layer's own top-k,
+    the adjacent-layer overlaps (kernel against the oracle), the greedy
+    search keeping two indexers (library against the oracle), then a decode
+    step through an index cache with the searched pattern, every layer's
+    attention against the oracle."""
+    rng = np.random.default_rng(91)
+    B, T, d, k, Hq, Hkv, L = 2, 6000, 64, 512, 8, 2, 6
+    ki = _ints(92, 2, (B, T, d))
+    base = [rng.integers(-4, 5, size=(B, d)) for _ in range(2)]
+    qs = []
+    for l in range(L):
+        q = base[l // 3].copy()
+        q[:, rng.choice(d, 3, replace=False)] = rng.integers(-4, 5, size=(B, 3))   # a small per-layer change
+        qs.append(ch.f32_to_bf16_bits(q.astype(np.float64)))
+    own = [sa.sa_index_score_topk(to_dev(qs[l]), to_dev(ki), k, Tk=T, q_pos0=T - 1) for l in range(L)]
+    ref = [oracle.index_topk(qs[l][:, None, :], ki, T, T - 1, k) for l in range(L)]
+    ov = np.zeros((L, L))
+    for a in range(L):
+        for b in range(L):
+            got = sa.sa_index_overlap(own[a][0], own[a][1], own[b][0], own[b][1])
+            want = oracle.index_overlap(ref[a][0][:, 0], ref[a][1][:, 0], ref[b][0][:, 0], ref[b][1][:, 0])
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(got.cpu().numpy(), want)
+            ov[a, b] = (want / ref[a][1][:, 0]).mean()
+    assert ov[1, 0] > 0.5 and ov[3, 2] < 0.5          # similar inside a block, not across
+    pattern = sa.sa_index_pattern_greedy(ov, 2)
+    assert pattern == oracle.greedy_pattern(ov, 2)
+    owners = oracle.layer_owners(L, pattern)
+    cache = sa.IndexCache(L, B, 1, k, pattern=pattern, device=dev())
+    cache.begin_step()
+    for layer in range(L):
+        if cache.is_full(layer) == 1:
+            cache.update(layer, to_dev(qs[layer]), to_dev(ki), Tk=T, q_pos0=T - 1)
+        idx, cnt, _ = cache.get_tensors(layer)
+        q = _normals(93 + layer, 1, (B, Hq, 128))
+        K = _normals(93 + layer, 2, (B, T, Hkv, 128))
+        V = _normals(93 + layer, 3, (B, T, Hkv, 128))
+        out = sa.sa_sparse_attn_decode(to_dev(q), to_dev(K), to_dev(V), idx.view(B, k), cnt.view(B))
+        torch.cuda.synchronize()
+        ridx, rcnt = ref[owners[layer]]
+        np.testing.assert_array_equal(idx.view(B, k).cpu().numpy(), ridx[:, 0])
+        want, _ = oracle.sparse_attention_decode(q, [K[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)],
+                                                 [V[b, ridx[b, 0, : rcnt[b, 0]]] for b in range(B)])
+        assert_close_attn(out.float().cpu().numpy(), want, f"pattern {pattern} layer {layer}")
+    cache.close()
+
+
 # ------------------------------------------------------------- device inputs
 
 def test_device_generator_matches_host_generator():

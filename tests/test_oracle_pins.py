@@ -607,3 +607,55 @@ def test_hier_gist_ties_take_lower_groups_and_chunks():
     _, chunks, groups = oracle.hier_gist_route_unfold(q, mk, gk, 4, 2, 2, 5, 0)
     np.testing.assert_array_equal(groups, [0, 1])
     np.testing.assert_array_equal(chunks, [0, 1, 2, 3, 4])
+
+
+# ------------------------------------------------- index overlap, layer roles
+
+def test_index_overlap_counts_shared_positions():
+    """[IC] §一: the overlap of two selections, against Python sets."""
+    rng = _rng(51)
+    rows, k = 20, 30
+    a = np.full((rows, k), -1, np.int32)
+    b = np.full((rows, k), -1, np.int32)
+    ca, cb = rng.integers(0, k + 1, rows), rng.integers(0, k + 1, rows)
+    for r in range(rows):
+        a[r, : ca[r]] = np.sort(rng.choice(60, ca[r], replace=False))
+        b[r, : cb[r]] = np.sort(rng.choice(60, cb[r], replace=False))
+    got = oracle.index_overlap(a, ca, b, cb)
+    for r in range(rows):
+        assert got[r] == len(set(a[r, : ca[r]].tolist()) & set(b[r, : cb[r]].tolist()))
+    np.testing.assert_array_equal(oracle.index_overlap(a, ca, a, ca), ca)   # a selection overlaps itself fully
+
+
+def test_greedy_pattern_hand_worked():
+    """[IC] §三: greedy removal of the indexer whose loss is smallest.  Six
+    layers in two blocks {0, 1, 2} and {3, 4, 5}: within a block the overlap
+    is 0.9, across blocks 0.2.  Keeping two indexers, the search keeps the
+    first layer of each block: "FSSFSS"."""
+    L = 6
+    ov = np.full((L, L), 0.2)
+    for blk in ((0, 1, 2), (3, 4, 5)):
+        for i in blk:
+            for j in blk:
+                ov[i, j] = 0.9
+    np.fill_diagonal(ov, 1.0)
+    assert oracle.greedy_pattern(ov, 2) == "FSSFSS"
+    assert oracle.greedy_pattern(ov, 6) == "FFFFFF"
+    assert oracle.greedy_pattern(ov, 1) == "FSSSSS"
+    # equal losses everywhere: the lower layers go first
+    assert oracle.greedy_pattern(np.ones((5, 5)), 3) == "FSSFF"
+
+
+def test_greedy_pattern_is_exhaustive_optimum_when_one_indexer_is_removed():
+    """Removing one indexer, the greedy step is the exhaustive best single
+    removal (checked against every choice)."""
+    rng = _rng(52)
+    L = 7
+    ov = rng.uniform(0.3, 1.0, (L, L))
+    np.fill_diagonal(ov, 1.0)
+    pat = oracle.greedy_pattern(ov, L - 1)
+    owners = oracle.layer_owners(L, pat)
+    got = sum(ov[l, owners[l]] for l in range(L))
+    best = max(sum(ov[l, oracle.layer_owners(L, "".join("S" if i == r else "F" for i in range(L)))[l]]
+                   for l in range(L)) for r in range(1, L))
+    assert abs(got - best) < 1e-12
