@@ -368,6 +368,33 @@ sa_status sa_index_overlap(const int32_t* idx_a, const int32_t* count_a, const i
 sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_full, char* pattern_out);
 
 /* ------------------------------------------------------------------------
+ * Debug builds (libsa_debug.so, compiled with SA_DEBUG; no counterpart in the
+ * pages).
+ *
+ * The debug build checks, on the device, every gathered row index a call
+ * uses (those below its count) against [0, Tk_max), and puts a 256-byte
+ * canary after the bytes each workspace call may use (the *_workspace
+ * functions count it; every call writes it and checks it after its
+ * kernels).  A violation is recorded -- never trapped -- and the access is
+ * clamped exactly as in the release build, so results match it.
+ *   sa_debug_enabled(): 1 in a debug build, 0 otherwise.
+ *   sa_debug_read(record, reset): host int32[4] = {code of the first
+ *     violation (0 none, 1 prefill attention index, 2 decode attention index,
+ *     3 gathered-rows index, 4 workspace canary), its first detail (the index;
+ *     for a canary the call: 1 index top-k, 2 multi-head top-k, 3 decode
+ *     attention, 4 gist routing), its second detail (Tk_max; for a canary the
+ *     first changed byte), number of violations}; reset != 0 clears it.
+ *     Synchronous; the release build reports zeros.
+ * ---------------------------------------------------------------------- */
+int sa_debug_enabled(void);
+sa_status sa_debug_read(int32_t* record, int reset);
+/* The canary check every workspace call runs after its kernels, on its own:
+ * the 256 bytes at ws + offset must all be 0xA5, else code 4 is recorded with
+ * `site` and the first changed byte.  Asynchronous on `stream`; a no-op in
+ * the release build. */
+sa_status sa_debug_check_canary(const void* ws, size_t offset, int site, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Shared index cache (host object; its device buffers are caller-owned).
  *
  * [IC] §二 and §六: layers are "full" (run their own indexer and store the

@@ -1,9 +1,11 @@
-"""Builds libsa.so (the C ABI in include/sa.h) in-tree with nvcc for sm_100a.
+"""Builds libsa.so (the C ABI in include/sa.h) in-tree with nvcc for sm_100a,
+and its debug variant libsa_debug.so (compiled with SA_DEBUG: gathered row
+indices and workspace canaries checked on the device, see sa.h).
 
-    python -m shared_top_routing_b200.build [--verbose]
+    python -m shared_top_routing_b200.build [--verbose] [--debug]
 
-Objects go to ``_build/`` at the repository root; the shared library is
-written next to this file, where the Python binding loads it.
+Objects go to ``_build/`` (``_build/debug/``) at the repository root; the
+shared libraries are written next to this file, where the binding loads them.
 """
 from __future__ import annotations
 
@@ -16,6 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
+LIB_DEBUG = os.path.join(PKG, "libsa_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
@@ -29,13 +32,14 @@ def _run(cmd, verbose):
     return subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
 
 
-def build(verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
-    extra = list(extra_flags or [])
+def build(verbose: bool = False, extra_flags: list[str] | None = None, debug: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    os.makedirs(out_dir, exist_ok=True)
+    extra = list(extra_flags or []) + (["-DSA_DEBUG"] if debug else [])
     procs = []
     objs = []
     for src in SOURCES:
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        obj = os.path.join(out_dir, src.replace(".cu", ".o"))
         objs.append(obj)
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         procs.append((src, _run(cmd, verbose)))
@@ -49,13 +53,14 @@ def build(verbose: bool = False, extra_flags: list[str] | None = None) -> str:
     if failed:
         msg = "\n".join(f"--- {s}\n{o}" for s, o in failed)
         raise RuntimeError(f"nvcc failed:\n{msg}")
-    cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
+    lib = LIB_DEBUG if debug else LIB
+    cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs, "-lcudart"]
     p = _run(cmd, verbose)
     out, _ = p.communicate()
     if p.returncode != 0:
         raise RuntimeError(f"link failed:\n{out}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

@@ -199,10 +199,10 @@ size_t sa_index_score_topk_workspace(int B, int Tq, int Tk_max, int d, int k) {
   if (B <= 0 || Tq <= 0 || Tk_max < 0) return 0;
   if (Tq == 1) {
     const int mode = sa::finish_mode_for(Tk_max);
-    return sa::row_workspace_bytes(B, Tk_max, mode == sa::kFinishSplit, mode != sa::kFinishDirect);
+    return sa::row_workspace_bytes(B, Tk_max, mode == sa::kFinishSplit, mode != sa::kFinishDirect) + sa::kWsCanary;
   }
   const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
-  return sa::prefill_workspace_bytes(B * rows, Tk_max, k);
+  return sa::prefill_workspace_bytes(B * rows, Tk_max, k) + sa::kWsCanary;
 }
 
 sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int Tq, int Tk,
@@ -215,13 +215,14 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
   const size_t need = sa_index_score_topk_workspace(B, Tq, Tk_max, d, k);
   if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
   cudaStream_t cs = as_cuda(stream);
+  cudaError_t e;
+  if ((e = sa::dbg_arm(ws, need - sa::kWsCanary, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   const uint16_t* q = static_cast<const uint16_t*>(q_idx);
   const uint16_t* km = static_cast<const uint16_t*>(k_idx);
   sa::FinishOut out;
   out.idx = idx_out;
   out.count = count_out;
   out.score = score_out;
-  cudaError_t e;
   if (Tq == 1) {
     const int mode = sa::finish_mode_for(Tk_max);
     sa::RowWorkspace w;
@@ -238,6 +239,7 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
     } else if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, w, mode, out, cs)) != cudaSuccess) {
       return cuda_fail(e, "finish launch");
     }
+    if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 1, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
     return ok();
   }
   const int rows = sa::prefill_rows_per_launch(B, Tq, Tk_max, k);
@@ -269,6 +271,7 @@ sa_status sa_index_score_topk(const void* q_idx, const void* k_idx, int B, int T
         return cuda_fail(e, "finish launch");
     }
   }
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 1, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   return ok();
 }
 
@@ -279,7 +282,7 @@ size_t sa_index_score_topk_mh_workspace(int B, int Tq, int Tk_max, int H, int d,
   (void)k;
   if (B <= 0 || Tq <= 0 || Tk_max < 0 || H < 1) return 0;
   const int rows = sa::mh_rows_per_launch(B, Tq, Tk_max);
-  return sa::row_workspace_bytes(B * rows, Tk_max, true, true);
+  return sa::row_workspace_bytes(B * rows, Tk_max, true, true) + sa::kWsCanary;
 }
 
 sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* k_idx, int B, int Tq, int H,
@@ -301,6 +304,7 @@ sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* 
   sa::RowWorkspace wsp;
   sa::carve_row_workspace(ws, B * rows, Tk_max, true, true, &wsp);
   cudaError_t e;
+  if ((e = sa::dbg_arm(ws, need - sa::kWsCanary, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   if (wsp.hist_zero_bytes && (e = cudaMemsetAsync(wsp.hist, 0, wsp.hist_zero_bytes, cs)) != cudaSuccess)
     return cuda_fail(e, "memset");
   sa::FinishOut out;
@@ -324,6 +328,7 @@ sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* 
       return cuda_fail(e, "finish launch");
     }
   }
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 2, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   return ok();
 }
 
@@ -347,7 +352,7 @@ sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void*
 
 size_t sa_sparse_attn_decode_workspace(int B, int Hq, int Hkv, int D, int k) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || k <= 0) return 0;
-  return sa::decode_attn_workspace_bytes(B, Hq, Hkv, D, k);
+  return sa::decode_attn_workspace_bytes(B, Hq, Hkv, D, k) + sa::kWsCanary;
 }
 
 sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -359,14 +364,18 @@ sa_status sa_sparse_attn_decode(const void* q, const void* k_cache, const void* 
   if (B == 0) return ok();
   if ((long long)B * Hkv > SA_DECODE_MAX_PAIRS)
     return fail(SA_ERR_UNSUPPORTED, "B*Hkv=%lld exceeds %d", (long long)B * Hkv, SA_DECODE_MAX_PAIRS);
-  if ((st = check_ws(ws, ws_bytes, sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k))) != SA_OK)
-    return st;
+  const size_t need = sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
-  cudaError_t e = sa::launch_attn_decode(
+  cudaError_t e = sa::dbg_arm(ws, need - sa::kWsCanary, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "debug canary");
+  e = sa::launch_attn_decode(
       static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k_cache),
       static_cast<const uint16_t*>(v_cache), idx, count, B, Tk_max, Hq, Hkv, k, sc,
       static_cast<uint16_t*>(out), lse, ws, as_cuda(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode launch");
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 3, as_cuda(stream))) != cudaSuccess)
+    return cuda_fail(e, "debug canary");
   return ok();
 }
 
@@ -403,12 +412,17 @@ sa_status sa_sparse_attn_decode_rows(const void* q, const void* k_rows, const vo
   if (B == 0) return ok();
   if ((long long)B * Hkv > SA_DECODE_MAX_PAIRS)
     return fail(SA_ERR_UNSUPPORTED, "B*Hkv=%lld exceeds %d", (long long)B * Hkv, SA_DECODE_MAX_PAIRS);
-  if ((st = check_ws(ws, ws_bytes, sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k))) != SA_OK) return st;
+  const size_t need = sa_sparse_attn_decode_workspace(B, Hq, Hkv, D, k);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
-  const cudaError_t e = sa::launch_attn_decode(
+  cudaError_t e = sa::dbg_arm(ws, need - sa::kWsCanary, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "debug canary");
+  e = sa::launch_attn_decode(
       static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k_rows), static_cast<const uint16_t*>(v_rows),
       nullptr, count, B, k, Hq, Hkv, k, sc, static_cast<uint16_t*>(out), lse, ws, as_cuda(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_rows launch");
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 3, as_cuda(stream))) != cudaSuccess)
+    return cuda_fail(e, "debug canary");
   return ok();
 }
 
@@ -419,7 +433,7 @@ size_t sa_gist_route_unfold_workspace(int B, int n_chunks, int d, int k_chunks) 
   (void)k_chunks;
   if (B <= 0 || n_chunks < 0) return 0;
   const int mode = sa::finish_mode_for(n_chunks);
-  return sa::row_workspace_bytes(B, n_chunks, mode == sa::kFinishSplit, mode != sa::kFinishDirect);
+  return sa::row_workspace_bytes(B, n_chunks, mode == sa::kFinishSplit, mode != sa::kFinishDirect) + sa::kWsCanary;
 }
 
 sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B, int n_chunks,
@@ -438,13 +452,15 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
   if (!q_route || !gist_key || !rows_out || !count_out) return fail(SA_ERR_INVALID_ARG, "NULL tensor pointer");
   if (!aligned(q_route, 16) || !aligned(gist_key, 16))
     return fail(SA_ERR_INVALID_ARG, "q_route and gist_key must be 16-byte aligned");
-  sa_status st = check_ws(ws, ws_bytes, sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks));
+  const size_t need = sa_gist_route_unfold_workspace(B, n_chunks, d, k_chunks);
+  sa_status st = check_ws(ws, ws_bytes, need);
   if (st != SA_OK) return st;
   cudaStream_t cs = as_cuda(stream);
   const int mode = sa::finish_mode_for(n_chunks);
   sa::RowWorkspace w;
   sa::carve_row_workspace(ws, B, n_chunks, mode == sa::kFinishSplit, mode != sa::kFinishDirect, &w);
   cudaError_t e;
+  if ((e = sa::dbg_arm(ws, need - sa::kWsCanary, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   const bool hist = mode != sa::kFinishDirect;
   if (hist && w.hist_zero_bytes && (e = cudaMemsetAsync(w.hist, 0, w.hist_zero_bytes, cs)) != cudaSuccess)
     return cuda_fail(e, "memset");
@@ -468,6 +484,7 @@ sa_status sa_gist_route_unfold(const void* q_route, const void* gist_key, int B,
              cudaSuccess) {
     return cuda_fail(e, "gist finish launch");
   }
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 4, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
   return ok();
 }
 
@@ -556,6 +573,28 @@ sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_ful
   }
   for (int l = 0; l < n_layers; ++l) pattern_out[l] = full[l] ? 'F' : 'S';
   pattern_out[n_layers] = '\0';
+  return ok();
+}
+
+int sa_debug_enabled(void) {
+#ifdef SA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+sa_status sa_debug_check_canary(const void* ws, size_t offset, int site, sa_stream_t stream) {
+  if (ws == nullptr) return fail(SA_ERR_INVALID_ARG, "ws is NULL");
+  const cudaError_t e = sa::dbg_check(ws, offset, site, as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "debug canary check");
+  return ok();
+}
+
+sa_status sa_debug_read(int32_t* record, int reset) {
+  if (record == nullptr) return fail(SA_ERR_INVALID_ARG, "record is NULL");
+  const cudaError_t e = sa::dbg_read(record, reset != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "debug record read");
   return ok();
 }
 

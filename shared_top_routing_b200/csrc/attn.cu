@@ -41,6 +41,30 @@ __device__ __forceinline__ int clamp_row(int j, int Tk_max) {
   return j < 0 ? 0 : (j >= Tk_max ? Tk_max - 1 : j);
 }
 
+#ifdef SA_DEBUG
+// Debug builds record the first violation (code, two details) and count
+// them all; nothing traps, and the access is clamped as in release builds.
+__device__ int g_dbg[4];
+__device__ __noinline__ void dbg_note(int code, int a, int b) {
+  if (atomicCAS(&g_dbg[0], 0, code) == 0) {
+    g_dbg[1] = a;
+    g_dbg[2] = b;
+  }
+  atomicAdd(&g_dbg[3], 1);
+}
+#endif
+
+// A gathered row index: checked against [0, Tk_max) in debug builds (site =
+// the debug record code), clamped into range in every build.
+__device__ __forceinline__ int checked_row(int j, int Tk_max, int site) {
+#ifdef SA_DEBUG
+  if (j < 0 || j >= Tk_max) dbg_note(site, j, Tk_max);
+#else
+  (void)site;
+#endif
+  return clamp_row(j, Tk_max);
+}
+
 // Shared memory of one CTA: Q (16 rows), 2 stages of K and V tiles; the
 // stage area is reused for the cross-warp merge.
 constexpr size_t kSmemQ = 16 * kLds * 2;
@@ -65,7 +89,7 @@ __device__ __forceinline__ void gather_tile(uint16_t* sK, uint16_t* sV, const ui
     const int r = (threadIdx.x >> 4) + 8 * pass;
     const int i = i0 + r;
     const bool v = i < end;
-    const int j = v ? clamp_row(irow[i], Tk_max) : 0;
+    const int j = v ? checked_row(irow[i], Tk_max, kDbgPrefillIndex) : 0;
     const long long off = head_base + (long long)j * row_elems + c * 8;
     cp_async16(sK + r * kLds + c * 8, kc + off, v);
     cp_async16(sV + r * kLds + c * 8, vc + off, v);
@@ -545,7 +569,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
       } else {
         const int j0 = si[0];   // row r0 < cnt
         for (int r = lane; r < R; r += 32) {
-          const int j = clamp_row(r0 + r < cnt ? si[r] : j0, Tk_max);
+          const int j = checked_row(r0 + r < cnt ? si[r] : j0, Tk_max, kDbgDecodeIndex);
           const long long off = (((long long)b * Tk_max + j) * Hkv + h0) * kD;
           tc::bulk_load(stK + (size_t)r * rb, kc + off, bytes, &full[s]);
           tc::bulk_load(stV + (size_t)r * rb, vc + off, bytes, &full[s]);
@@ -748,7 +772,7 @@ gather_rows_kernel(const uint16_t* __restrict__ kc, const uint16_t* __restrict__
     dv[chunks] = make_uint4(0u, 0u, 0u, 0u);
   }
   if (r < cnt) {
-    const int j = clamp_row(idx[(long long)b * k + r], Tk_max);
+    const int j = checked_row(idx[(long long)b * k + r], Tk_max, kDbgGatherIndex);
     const uint4* sk = reinterpret_cast<const uint4*>(kc + ((long long)b * Tk_max + j) * Hkv * kD);
     const uint4* sv = reinterpret_cast<const uint4*>(vc + ((long long)b * Tk_max + j) * Hkv * kD);
     for (int c = lane; c < chunks; c += 32) {
@@ -846,6 +870,50 @@ cudaError_t launch_gather_rows(const uint16_t* kc, const uint16_t* vc, const int
   const cudaError_t e = launch_pdl(gather_rows_kernel, dim3((unsigned)((k + 7) / 8), (unsigned)B), dim3(256), 0, st,
                                    kc, vc, idx, count, Tk_max, Hkv, k, ko, vo);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+#ifdef SA_DEBUG
+namespace {
+__global__ void dbg_canary_kernel(const unsigned char* __restrict__ c, int site) {
+  if (c[threadIdx.x] != kDbgCanaryByte) dbg_note(kDbgCanary, site, (int)threadIdx.x);
+}
+}  // namespace
+#endif
+
+cudaError_t dbg_arm(void* ws, size_t off, cudaStream_t st) {
+#ifdef SA_DEBUG
+  if (ws == nullptr) return cudaSuccess;
+  return cudaMemsetAsync(static_cast<unsigned char*>(ws) + off, kDbgCanaryByte, kDbgCanaryBytes, st);
+#else
+  (void)ws, (void)off, (void)st;
+  return cudaSuccess;
+#endif
+}
+
+cudaError_t dbg_check(const void* ws, size_t off, int site, cudaStream_t st) {
+#ifdef SA_DEBUG
+  if (ws == nullptr) return cudaSuccess;
+  dbg_canary_kernel<<<1, kDbgCanaryBytes, 0, st>>>(static_cast<const unsigned char*>(ws) + off, site);
+  return cudaGetLastError();
+#else
+  (void)ws, (void)off, (void)site, (void)st;
+  return cudaSuccess;
+#endif
+}
+
+cudaError_t dbg_read(int* host4, bool reset) {
+#ifdef SA_DEBUG
+  cudaError_t e = cudaMemcpyFromSymbol(host4, g_dbg, 4 * sizeof(int));
+  if (e == cudaSuccess && reset) {
+    const int zero[4] = {0, 0, 0, 0};
+    e = cudaMemcpyToSymbol(g_dbg, zero, sizeof(zero));
+  }
+  return e;
+#else
+  (void)reset;
+  for (int i = 0; i < 4; ++i) host4[i] = 0;
+  return cudaSuccess;
+#endif
 }
 
 cudaError_t launch_attn_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,

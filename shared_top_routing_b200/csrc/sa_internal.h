@@ -28,6 +28,26 @@ constexpr int kScoreKeys = 0;       // every score's key into the row slab
 constexpr int kScoreGroupMax = 1;   // per-row group maxima (16-bit keys)
 constexpr int kScoreCand = 2;       // keys at or above the row's bound, appended with positions
 
+// Debug builds (SA_DEBUG): codes of the device debug record, and the canary
+// after every workspace's used bytes.
+constexpr int kDbgPrefillIndex = 1;
+constexpr int kDbgDecodeIndex = 2;
+constexpr int kDbgGatherIndex = 3;
+constexpr int kDbgCanary = 4;
+constexpr int kDbgCanaryBytes = 256;
+constexpr unsigned char kDbgCanaryByte = 0xA5;
+#ifdef SA_DEBUG
+constexpr size_t kWsCanary = kDbgCanaryBytes;
+#else
+constexpr size_t kWsCanary = 0;
+#endif
+// Writes the canary at ws + off / checks it after a call's kernels (site:
+// which call) / copies (and optionally clears) the record.  No-ops (zeros)
+// in release builds.
+cudaError_t dbg_arm(void* ws, size_t off, cudaStream_t st);
+cudaError_t dbg_check(const void* ws, size_t off, int site, cudaStream_t st);
+cudaError_t dbg_read(int* host4, bool reset);
+
 // Rows whose histograms live in the fixed, self-cleaning workspace region.
 constexpr int kHistRowsFixed = 64;
 

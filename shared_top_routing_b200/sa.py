@@ -14,6 +14,7 @@ import threading
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsa.so")
+LIB_DEBUG_PATH = os.path.join(_HERE, "libsa_debug.so")
 
 SA_OK = 0
 SA_ERR_INVALID_ARG = 1
@@ -51,6 +52,9 @@ SIGNATURES = {
     "sa_hier_gist_route_unfold": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "sa_index_overlap": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
     "sa_index_pattern_greedy": (_I, [_P, _I, _I, ctypes.c_char_p]),
+    "sa_debug_enabled": (_I, []),
+    "sa_debug_read": (_I, [_P, _I]),
+    "sa_debug_check_canary": (_I, [_P, _Z, _I, _P]),
     "sa_index_cache_create": (_I, [_I, ctypes.c_char_p, _I, _I, _I, _I, _P, _P, ctypes.POINTER(_P)]),
     "sa_index_cache_destroy": (None, [_P]),
     "sa_index_cache_is_full": (_I, [_P, _I]),
@@ -89,6 +93,36 @@ def lib():
                     f.argtypes = args
                 _lib = L
     return _lib
+
+
+_lib_debug = None
+
+
+def lib_debug():
+    """The debug build libsa_debug.so (same ABI; see sa.h), loaded on its own."""
+    global _lib_debug
+    if _lib_debug is None:
+        with _lock:
+            if _lib_debug is None:
+                if not os.path.exists(LIB_DEBUG_PATH):
+                    raise RuntimeError(f"libsa_debug.so not found at {LIB_DEBUG_PATH}; build it with "
+                                       "`python -m shared_top_routing_b200.build --debug`")
+                L = ctypes.CDLL(LIB_DEBUG_PATH)
+                for name, (res, args) in SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib_debug = L
+    return _lib_debug
+
+
+def debug_read(L=None, reset: bool = True):
+    """The debug record {code, detail, detail, count} of a library (see sa.h)."""
+    rec = (ctypes.c_int32 * 4)()
+    st = (L or lib_debug()).sa_debug_read(ctypes.cast(rec, ctypes.c_void_p), 1 if reset else 0)
+    if st != SA_OK:
+        raise SAError(st, "sa_debug_read", last_error())
+    return list(rec)
 
 
 def status_string(s: int) -> str:

@@ -243,3 +243,16 @@ def test_greedy_pattern_search_matches_the_oracle():
     buf = ctypes.create_string_buffer(9)
     assert S.lib().sa_index_pattern_greedy(None, 8, 2, buf) == S.SA_ERR_INVALID_ARG
     assert S.lib().sa_index_overlap(None, None, None, None, 3, 16, None, None) == S.SA_ERR_INVALID_ARG
+
+
+def test_debug_library_loads_and_reports_itself():
+    """libsa_debug.so exports the same ABI; it says it is a debug build, the
+    release library says it is not, and both refuse a NULL record."""
+    LD = S.lib_debug()
+    assert LD.sa_debug_enabled() == 1
+    assert S.lib().sa_debug_enabled() == 0
+    assert LD.sa_debug_read(None, 0) == S.SA_ERR_INVALID_ARG
+    assert S.lib().sa_debug_check_canary(None, 0, 1, None) == S.SA_ERR_INVALID_ARG
+    # the debug workspaces carry the 256-byte canary
+    assert LD.sa_sparse_attn_decode_workspace(8, 32, 8, 128, 2048) == \
+        S.lib().sa_sparse_attn_decode_workspace(8, 32, 8, 128, 2048) + 256
