@@ -65,32 +65,46 @@ __device__ __forceinline__ int checked_row(int j, int Tk_max, int site) {
   return clamp_row(j, Tk_max);
 }
 
-// Shared memory of one CTA: Q (16 rows), 2 stages of K and V tiles; the
-// stage area is reused for the cross-warp merge.
+// Shared memory of one CTA: Q (16 rows), kPfStages stages of K and V tiles;
+// the stage area is reused for the cross-warp merge.
+constexpr int kPfStages = 2;
+constexpr int kRowsPerThread = kTile / 8;   // gathered rows per thread and tile
 constexpr size_t kSmemQ = 16 * kLds * 2;
 constexpr size_t kSmemStage = (size_t)kTile * kLds * 2;
-constexpr size_t kSmemTotal = kSmemQ + 4 * kSmemStage;
+constexpr size_t kSmemTotal = kSmemQ + 2 * kPfStages * kSmemStage;
 
 struct TileAcc {
   float o[16][4];
   float m[2], l[2];
 };
 
+// Thread t gathers rows (t >> 4) + 8 p, p < kRowsPerThread, of a tile: the
+// row indices of tile rows [i0, i0+64) (clipped to `end`) it copies.  They
+// are loaded one tile ahead of the copies, so the copies never wait on an
+// index load.
+__device__ __forceinline__ void load_tile_rows(int (&j)[kRowsPerThread], const int32_t* __restrict__ irow, int i0,
+                                               int end) {
+#pragma unroll
+  for (int p = 0; p < kRowsPerThread; ++p) {
+    const int i = i0 + (threadIdx.x >> 4) + 8 * p;
+    j[p] = i < end ? __ldg(irow + i) : 0;
+  }
+}
+
 // Gathers tile rows [i0, i0+64) (clipped to `end`) of one kv head into a
 // stage: 16 consecutive threads copy the 16 chunks of one 256-byte row, so
 // every request covers whole 32-byte sectors.
 __device__ __forceinline__ void gather_tile(uint16_t* sK, uint16_t* sV, const uint16_t* __restrict__ kc,
-                                            const uint16_t* __restrict__ vc, const int32_t* __restrict__ irow,
+                                            const uint16_t* __restrict__ vc, const int (&j)[kRowsPerThread],
                                             int i0, int end, long long head_base, long long row_elems,
                                             int Tk_max) {
   const int c = threadIdx.x & 15;
 #pragma unroll
-  for (int pass = 0; pass < kTile / 8; ++pass) {
-    const int r = (threadIdx.x >> 4) + 8 * pass;
-    const int i = i0 + r;
-    const bool v = i < end;
-    const int j = v ? checked_row(irow[i], Tk_max, kDbgPrefillIndex) : 0;
-    const long long off = head_base + (long long)j * row_elems + c * 8;
+  for (int p = 0; p < kRowsPerThread; ++p) {
+    const int r = (threadIdx.x >> 4) + 8 * p;
+    const bool v = i0 + r < end;
+    const int row = v ? checked_row(j[p], Tk_max, kDbgPrefillIndex) : 0;
+    const long long off = head_base + (long long)row * row_elems + c * 8;
     cp_async16(sK + r * kLds + c * 8, kc + off, v);
     cp_async16(sV + r * kLds + c * 8, vc + off, v);
   }
@@ -106,7 +120,7 @@ __device__ __forceinline__ void attn_tiles(unsigned char* smem, const uint16_t* 
                                            float qscale, TileAcc& acc) {
   uint16_t* sQ = reinterpret_cast<uint16_t*>(smem);
   uint16_t* sK = reinterpret_cast<uint16_t*>(smem + kSmemQ);
-  uint16_t* sV = sK + 2 * kTile * kLds;
+  uint16_t* sV = sK + kPfStages * kTile * kLds;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tg = lane & 3;
 #pragma unroll
@@ -116,16 +130,32 @@ __device__ __forceinline__ void attn_tiles(unsigned char* smem, const uint16_t* 
   acc.m[0] = acc.m[1] = -INFINITY;
   acc.l[0] = acc.l[1] = 0.f;
   const int ntiles = end > begin ? (end - begin + kTile - 1) / kTile : 0;
-  if (ntiles > 0) gather_tile(sK, sV, kc, vc, irow, begin, end, head_base, row_elems, Tk_max);
-  cp_async_commit();
+  // ring of kPfStages stages: tiles it+1 .. it+kPfStages-1 are in flight
+  // while tile it is consumed, and the indices of the tile after them sit in
+  // registers
+  int jn[kRowsPerThread];
+#pragma unroll
+  for (int s = 0; s < kPfStages - 1; ++s) {
+    if (s < ntiles) {
+      load_tile_rows(jn, irow, begin + s * kTile, end);
+      gather_tile(sK + s * kTile * kLds, sV + s * kTile * kLds, kc, vc, jn, begin + s * kTile, end, head_base,
+                  row_elems, Tk_max);
+    }
+    cp_async_commit();
+  }
+  if (kPfStages - 1 < ntiles) load_tile_rows(jn, irow, begin + (kPfStages - 1) * kTile, end);
   uint32_t qa[8][4];
   for (int it = 0; it < ntiles; ++it) {
-    const int stage = it & 1;
-    if (it + 1 < ntiles)
-      gather_tile(sK + (stage ^ 1) * kTile * kLds, sV + (stage ^ 1) * kTile * kLds, kc, vc, irow,
-                  begin + (it + 1) * kTile, end, head_base, row_elems, Tk_max);
+    const int stage = it % kPfStages;
+    const int nxt = it + kPfStages - 1;
+    if (nxt < ntiles) {
+      const int ns = nxt % kPfStages;
+      gather_tile(sK + ns * kTile * kLds, sV + ns * kTile * kLds, kc, vc, jn, begin + nxt * kTile, end, head_base,
+                  row_elems, Tk_max);
+    }
     cp_async_commit();
-    cp_async_wait<1>();
+    if (nxt + 1 < ntiles) load_tile_rows(jn, irow, begin + (nxt + 1) * kTile, end);
+    cp_async_wait<kPfStages - 1>();
     __syncthreads();
     if (it == 0) {
 #pragma unroll
@@ -582,7 +612,7 @@ attn_decode_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restr
     for (int s = 0; s < kDxStages; ++s) {
       if ((uint32_t)s < fill) {
         const uint32_t last_use = (fill - 1 - (uint32_t)s) / kDxStages;
-        tc::mbar_wait(&full[s], last_use & 1u, abort_flag, err, 12);
+        if (!tc::mbar_wait_drain(&full[s], last_use & 1u) && err) atomicCAS(err, 0, 12);
       }
     }
     return;

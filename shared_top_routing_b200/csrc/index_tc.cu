@@ -243,6 +243,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       TileCursor cur;
       cur.start(p, lo);
       int blk = -1;
+      int nA = 0, nB = 0;   // query blocks and key tiles whose loads were issued
       for (long long u = lo; u < hi; ++u, cur.next(p)) {
         if (u == lo || cur.tile == 0) {
           // block blk goes to buffer blk % kABuf, once the MMAs of block blk - kABuf are done
@@ -256,6 +257,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           for (int a = 0; a < S::kAtoms; ++a)
             tma_load_3d(sA + ab * S::kABytes + a * kBM * 128, &tmap_q, &bars.afull[ab], 64 * a,
                         p.t0 + cur.rb * kBM, cur.b);
+          nA = blk + 1;
         }
         const int i = (int)(u - lo);
         const int s = i % S::kStages;
@@ -265,7 +267,16 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
         for (int a = 0; a < S::kAtoms; ++a)
           tma_load_3d(sB + s * S::kBBytes + a * kBN * 128, &tmap_k, &bars.full[s], 64 * a, cur.tile * kBN, cur.b);
+        nB = i + 1;
       }
+      // every load this CTA issued lands before it exits (also after a wait
+      // gave up): bounded waits on the last phase of each buffer
+      for (int s = 0; s < S::kStages; ++s)
+        if (s < nB && !mbar_wait_drain(&bars.full[s], (uint32_t)((nB - 1 - s) / S::kStages) & 1u) && p.err)
+          atomicCAS(p.err, 0, 7);
+      for (int a = 0; a < S::kABuf; ++a)
+        if (a < nA && !mbar_wait_drain(&bars.afull[a], (uint32_t)((nA - 1 - a) / S::kABuf) & 1u) && p.err)
+          atomicCAS(p.err, 0, 7);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -274,6 +285,7 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       TileCursor cur;
       cur.start(p, lo);
       int blk = -1;
+      int last = -1;   // the last tile whose MMAs were committed
       uint32_t a_addr = 0;
       for (long long u = lo; u < hi; ++u, cur.next(p)) {
         if (u == lo || cur.tile == 0) {
@@ -301,7 +313,12 @@ score_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         umma_commit(&bars.empty[s]);
         umma_commit(&bars.tfull[acc]);
         if (cur.tile == cur.nt - 1 || u == hi - 1) umma_commit(&bars.aempty[blk % S::kABuf]);   // its query block is free
+        last = i;
       }
+      // every MMA issued completes before the accumulator is freed (a commit
+      // covers all earlier MMAs of this thread)
+      if (last >= 0 && !mbar_wait_drain(&bars.tfull[last & 1], (uint32_t)(last >> 1) & 1u) && p.err)
+        atomicCAS(p.err, 0, 8);
     }
   } else {
     // epilogue: warp w reads TMEM lanes of quarter w % 4, columns part *

@@ -12,14 +12,15 @@
 //       product is invariant to the order of its terms, so lane (g, t) of a
 //       warp loads whole 16-byte chunks 4j+t of key row g and the query
 //       fragment is permuted to match.  One m16n8k16 per 16 dims scores 8
-//       keys (the query is row 0 of the 16-row A side).  Each warp keeps two
-//       register buffers of key tiles, the next in flight while the current
-//       is scored.  Writes the order-preserving 32-bit score key of every
-//       candidate and a 4096-bin histogram of the keys' top 12 bits.  The
-//       B x Tk key rows are flattened and split evenly (at multiples of 8
-//       rows) over a grid sized to the resident CTAs.  (A TMA + tcgen05
-//       variant was measured slower here: with 128x16 tiles the per-tile
-//       TMEM hand-off dominates.)
+//       keys (the query is row 0 of the 16-row A side).  Each warp loads one
+//       register buffer of key tiles and scores it; four CTAs per SM keep 32
+//       warps of loads in flight.  Writes the order-preserving 32-bit score
+//       key of every candidate and a 4096-bin histogram of the keys' top 12
+//       bits.  The B x Tk key rows are flattened and split evenly (at
+//       multiples of 8 rows) over a grid sized to the resident CTAs.  (Two
+//       other designs measured no faster: TMA + tcgen05, where with 128x16
+//       tiles the per-tile TMEM hand-off dominates, and a TMA bulk-copy ring
+//       into shared memory feeding mma.sync warps.)
 //   prefill_threshold_kernel  (long prefill rows) the k-th largest of the
 //       row's 16-bit group maxima -- a counting pass over a window below
 //       their maximum, or a two-digit radix select -- the bound the second
@@ -76,7 +77,7 @@ __device__ __forceinline__ int n_cand(long long q_pos0, int t, int len) {
 // ------------------------------------------------------------------ scoring
 
 template <int D>
-__global__ void __launch_bounds__(kScoreThreads)
+__global__ void __launch_bounds__(kScoreThreads, 4)
 score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kmat, int B, int Tk_max,
                     int Tk, int q_pos0, const int32_t* __restrict__ kv_len,
                     uint32_t* __restrict__ keys, long long ld, uint32_t* __restrict__ hist) {
@@ -120,9 +121,11 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
     }
     const uint4* kb = reinterpret_cast<const uint4*>(kmat + (long long)b * Tk_max * D);
     uint32_t* kout = keys + (long long)b * ld;
-    // Two register buffers of U 8-row tiles: the next buffer's loads are in
-    // flight while the current one is scored, so each warp keeps memory busy
-    // instead of alternating a burst of loads with compute.
+    // One register buffer of U 8-row tiles per warp, loaded then scored: at
+    // 64 registers four CTAs (32 warps) fit on an SM, and it is that many
+    // warps with loads in flight, not a second buffer per warp, that keeps
+    // HBM streaming (with two buffers, two CTAs fit and the read rate drops
+    // by a third).
     auto load = [&](uint4 (&v)[U][J], int base) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -157,15 +160,10 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
       }
     };
     constexpr int kStep = WARPS * 8 * U;
-    uint4 va[U][J], vb[U][J];
-    int base = r0 + warp * 8 * U;
-    if (base < r1) load(va, base);
-    for (; base < r1; base += 2 * kStep) {
-      if (base + kStep < r1) load(vb, base + kStep);
+    for (int base = r0 + warp * 8 * U; base < r1; base += kStep) {
+      uint4 va[U][J];
+      load(va, base);
       score(va, base);
-      if (base + kStep >= r1) break;
-      if (base + 2 * kStep < r1) load(va, base + 2 * kStep);
-      score(vb, base + kStep);
     }
     if (hist != nullptr) {
       __syncthreads();
@@ -185,8 +183,8 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 // ReLU(q_h . k), for rows that each carry their own H query vectors and
 // weights (one row per decode sequence, or per prefill query) against the
 // key cache of their sequence.  The key cache is streamed as in
-// score_decode_kernel (16-byte loads straight into mma.sync B fragments,
-// two register buffers of 8-row tiles); the 16-row A side holds 16 indexer
+// score_decode_kernel (16-byte loads straight into mma.sync B fragments;
+// here two register buffers of 8-row tiles per warp); the 16-row A side holds 16 indexer
 // heads (rows g and g+8 of a lane's fragment are heads 16 hg + g and 16 hg
 // + g + 8 of head group hg), so one m16n8k16 per 16 dimensions scores every
 // head of a group at once.  The epilogue takes weight x ReLU per head and
@@ -1062,25 +1060,39 @@ struct SplitSmem {
 static_assert(offsetof(SplitSmem, ckey) % 16 == 0 && offsetof(SplitSmem, cpos) % 16 == 0,
               "candidate arrays are read as 16-byte vectors");
 
-// Bin of the K-th largest key of a 4096-bin histogram (bins in key order),
-// read once with 16-byte loads through L2 and kept in registers: s_out[0] =
-// bin, s_out[1] = keys in the bins above it, s_out[2] = keys in it (0, 0, 0
-// when the histogram holds fewer than K keys).
+// A 4096-bin histogram (bins in key order) read with 16-byte loads through
+// L2 into registers, thread 0 holding the top bins.  The loads are issued
+// here and consumed by hist_pick, so other loads can share their round trip.
 template <int THREADS>
-__device__ __forceinline__ void hist_threshold_v(const uint32_t* __restrict__ h, uint32_t K, uint32_t* s_warp,
-                                                 uint32_t* s_out) {
-  constexpr int per = kHistBins / THREADS;
+struct HistRegs {
+  static constexpr int per = kHistBins / THREADS;
   static_assert(per % 4 == 0, "16-byte loads of whole bins");
-  const int base = kHistBins - per * ((int)threadIdx.x + 1);   // thread 0 holds the top bins
   uint32_t c[per];
+};
+
+template <int THREADS>
+__device__ __forceinline__ void hist_load(const uint32_t* __restrict__ h, HistRegs<THREADS>& r) {
+  constexpr int per = HistRegs<THREADS>::per;
+  const int base = kHistBins - per * ((int)threadIdx.x + 1);
 #pragma unroll
   for (int v = 0; v < per / 4; ++v) {
     const uint4 x = __ldcg(reinterpret_cast<const uint4*>(h + base) + v);
-    c[4 * v] = x.x;
-    c[4 * v + 1] = x.y;
-    c[4 * v + 2] = x.z;
-    c[4 * v + 3] = x.w;
+    r.c[4 * v] = x.x;
+    r.c[4 * v + 1] = x.y;
+    r.c[4 * v + 2] = x.z;
+    r.c[4 * v + 3] = x.w;
   }
+}
+
+// Bin of the K-th largest key of the histogram in r: s_out[0] = bin,
+// s_out[1] = keys in the bins above it, s_out[2] = keys in it (0, 0, 0 when
+// the histogram holds fewer than K keys).  Every thread of the block calls it.
+template <int THREADS>
+__device__ __forceinline__ void hist_pick(const HistRegs<THREADS> r, uint32_t K, uint32_t* s_warp,
+                                          uint32_t* s_out) {
+  constexpr int per = HistRegs<THREADS>::per;
+  const int base = kHistBins - per * ((int)threadIdx.x + 1);
+  const uint32_t* c = r.c;
   if (threadIdx.x == 0) {
     s_out[0] = 0u;
     s_out[1] = 0u;
@@ -1106,7 +1118,7 @@ __device__ __forceinline__ void hist_threshold_v(const uint32_t* __restrict__ h,
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSplitThreads)
+__global__ void __launch_bounds__(kSplitThreads, 2)
 split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, int q_pos0,
                   const int32_t* __restrict__ kv_len, int k, int chunk, FinishOut out) {
   pdl_wait();
@@ -1118,12 +1130,15 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
   const int t = t0 + r % rows_per_batch;
   const int tid = threadIdx.x;
   const int n = n_cand(q_pos0, t, row_len(kv_len, b, Tk));
+  uint32_t* hist1 = w.hist + (long long)r * kHistStride;
+  uint32_t* hist2 = hist1 + kHistBins;
+  // the first histogram's loads share their round trip with the error word's
+  HistRegs<kSplitThreads> h1;
+  hist_load(hist1, h1);
   // a wait in an earlier kernel of this call that gave up: failure sentinel
   const bool failed = w.err != nullptr && *reinterpret_cast<volatile const int*>(w.err) != 0;
   const uint32_t K = failed ? 0u : (uint32_t)min(k, n);
   const uint32_t* row = w.keys + (long long)r * w.ld;
-  uint32_t* hist1 = w.hist + (long long)r * kHistStride;
-  uint32_t* hist2 = hist1 + kHistBins;
   uint2* cand = w.cand + (long long)r * w.ld;
   uint32_t* slot = w.slot_cnt + (long long)r * kSplitMaxSlices;
   const int c0 = c * chunk;
@@ -1133,7 +1148,7 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
   // ---- 1. filter this slice (in position order)
   uint32_t taken = 0;
   if (K > 0) {
-    hist_threshold_v<kSplitThreads>(hist1, K, s.swarp, s.thr);
+    hist_pick(h1, K, s.swarp, s.thr);
     const uint32_t bin = s.thr[0];
     for (int u0 = 0; u0 < chunk; u0 += kSplitSlice) {
       const int i = c0 + u0 + tid * 4;
@@ -1167,7 +1182,10 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
   if (!s.last) return;
   __threadfence();
 
-  // ---- 2. the finishing CTA
+  // ---- 2. the finishing CTA (the second histogram's loads share their
+  // round trip with the slice counts')
+  HistRegs<kSplitThreads> h2;
+  hist_load(hist2, h2);
   uint32_t total = 0;
   for (int s0 = 0; s0 < F; s0 += kSplitThreads) {
     const int sl = s0 + tid;
@@ -1202,7 +1220,7 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
         e[u] = i < total ? fetch(i) : make_uint2(0u, 0u);
       }
     }
-    hist_threshold_v<kSplitThreads>(hist2, K - s.thr[1], s.swarp, s.thr2);
+    hist_pick(h2, K - s.thr[1], s.swarp, s.thr2);
     const uint32_t T = s.thr[0] << kHistBits | s.thr2[0];   // 24-bit prefix of the K-th key
     const uint32_t kk = K - s.thr[1] - s.thr2[1];           // keys with prefix T still to take
     PairItems it;
@@ -1564,7 +1582,7 @@ int score_grid(long long rows) {
   const int sms = device_sm_count();
   const int occ = device_occupancy((const void*)score_decode_kernel<D>, kScoreThreads, 0);
   long long want = (long long)sms * occ;
-  const long long by_rows = (rows + 255) / 256;  // at least 256 key rows per CTA
+  const long long by_rows = (rows + 255) / 256;
   if (want > by_rows) want = by_rows;
   return (int)(want < 1 ? 1 : want);
 }
@@ -1574,7 +1592,7 @@ cudaError_t launch_score_decode(const uint16_t* q, const uint16_t* kmat, int B, 
                                 bool with_hist, cudaStream_t st) {
   if (Tk <= 0 || B <= 0) return cudaSuccess;
   uint32_t* hist = with_hist ? w.hist : nullptr;
-  const long long rows = (long long)B * Tk;
+  const long long rows = (long long)B * (((long long)Tk + 7) & ~7ll);
   cudaError_t e;
   if (d == 128)
     e = launch_pdl(score_decode_kernel<128>, dim3(score_grid<128>(rows)), dim3(kScoreThreads), 0, st, q, kmat, B,
