@@ -593,6 +593,26 @@ __device__ __forceinline__ void emit(const FinishOut& out, long long o_idx, int 
   }
 }
 
+// Writes the K chosen items staged in shared memory (spos / skey indexed by
+// output slot) like emit, with consecutive threads on consecutive slots (or
+// unfolded rows), so the stores coalesce.
+__device__ __forceinline__ void emit_staged(const FinishOut& out, long long o_idx, int b, const uint32_t* spos,
+                                            const uint32_t* skey, uint32_t K, int tid, int nthreads) {
+  if (out.rows == nullptr) {
+    for (uint32_t i = (uint32_t)tid; i < K; i += (uint32_t)nthreads) {
+      out.idx[o_idx + i] = (int32_t)spos[i];
+      if (out.score) out.score[o_idx + i] = key_score(skey[i]);
+    }
+  } else {
+    const uint32_t stride = (uint32_t)out.chunk_len + 1u;
+    int32_t* rows = out.rows + (long long)b * out.rows_stride;
+    for (uint32_t e = (uint32_t)tid; e < K * stride; e += (uint32_t)nthreads)
+      rows[e] = (int32_t)(spos[e / stride] * stride + e % stride);
+    if (out.chunks)
+      for (uint32_t i = (uint32_t)tid; i < K; i += (uint32_t)nthreads) out.chunks[o_idx + i] = (int32_t)spos[i];
+  }
+}
+
 // Writes a row's padding (slots K..k-1 = -1, scores -inf) and count, or, for
 // gist routing, the partial chunk's rows after the unfolded ones, the row
 // padding and the row count.  A failed row (an upstream wait gave up) gets
@@ -1199,27 +1219,29 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
   const bool in_smem = total <= (uint32_t)kSplitCand;
   const long long o_idx = ((long long)b * Tq + t) * (long long)k;
   if (K > 0) {
-    // gathered candidate i belongs to the last slice whose first index is <= i
-    auto fetch = [&](uint32_t i) {
+    // Gathered candidate i belongs to the last slice whose first index is
+    // <= i.  A thread's kSplitPer candidates of a pass are consecutive, so one
+    // binary search places the first and the slice only moves forward.
+    auto fetch = [&](uint32_t i0, uint2 (&e)[kSplitPer]) {
+      const uint32_t ib = i0 + (uint32_t)tid * kSplitPer;
       int lo = 0, hi = F - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (s.pre[mid] <= i) lo = mid;
+        if (s.pre[mid] <= ib) lo = mid;
         else hi = mid - 1;
       }
-      return __ldcg(cand + (long long)lo * chunk + (i - s.pre[lo]));
+#pragma unroll
+      for (int u = 0; u < kSplitPer; ++u) {
+        const uint32_t i = ib + u;
+        while (lo + 1 < F && s.pre[lo + 1] <= i) ++lo;
+        e[u] = i < total ? __ldcg(cand + (long long)lo * chunk + (i - s.pre[lo])) : make_uint2(0u, 0u);
+      }
     };
     // the first pass's loads are issued before the second histogram is read,
     // so both are in flight together
     uint2 e[kSplitPer];
     uint32_t i0 = 0;
-    if (in_smem) {
-#pragma unroll
-      for (int u = 0; u < kSplitPer; ++u) {
-        const uint32_t i = (uint32_t)tid * kSplitPer + u;
-        e[u] = i < total ? fetch(i) : make_uint2(0u, 0u);
-      }
-    }
+    if (in_smem) fetch(0u, e);
     hist_pick(h2, K - s.thr[1], s.swarp, s.thr2);
     const uint32_t T = s.thr[0] << kHistBits | s.thr2[0];   // 24-bit prefix of the K-th key
     const uint32_t kk = K - s.thr[1] - s.thr2[1];           // keys with prefix T still to take
@@ -1232,26 +1254,31 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
         s.kand = ~0u;
       }
       uint32_t ko = 0u, ka = ~0u;
+      static_assert(kSplitPer == 8, "two 16-byte stores per array and thread");
       for (i0 = 0; i0 < total; i0 += kSplitThreads * kSplitPer) {
-        if (i0 > 0) {
+        if (i0 > 0) fetch(i0, e);
+        const uint32_t ib = i0 + (uint32_t)tid * kSplitPer;
+        if (ib + kSplitPer <= total) {   // 16-byte stores: two-way bank conflicts at most
+          uint4* dk = reinterpret_cast<uint4*>(s.ckey + ib);
+          uint4* dp = reinterpret_cast<uint4*>(s.cpos + ib);
+          dk[0] = make_uint4(e[0].x, e[1].x, e[2].x, e[3].x);
+          dk[1] = make_uint4(e[4].x, e[5].x, e[6].x, e[7].x);
+          dp[0] = make_uint4(e[0].y, e[1].y, e[2].y, e[3].y);
+          dp[1] = make_uint4(e[4].y, e[5].y, e[6].y, e[7].y);
+        } else {
 #pragma unroll
-          for (int u = 0; u < kSplitPer; ++u) {
-            const uint32_t i = i0 + (uint32_t)tid * kSplitPer + u;
-            e[u] = i < total ? fetch(i) : make_uint2(0u, 0u);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kSplitPer; ++u) {
-          const uint32_t i = i0 + (uint32_t)tid * kSplitPer + u;
-          if (i < total) {
-            s.ckey[i] = e[u].x;
-            s.cpos[i] = e[u].y;
-            if ((e[u].x >> 8) == T) {
-              ko |= e[u].x;
-              ka &= e[u].x;
+          for (int u = 0; u < kSplitPer; ++u)
+            if (ib + u < total) {
+              s.ckey[ib + u] = e[u].x;
+              s.cpos[ib + u] = e[u].y;
             }
-          }
         }
+#pragma unroll
+        for (int u = 0; u < kSplitPer; ++u)
+          if (ib + u < total && (e[u].x >> 8) == T) {
+            ko |= e[u].x;
+            ka &= e[u].x;
+          }
       }
       __syncthreads();
       ko = __reduce_or_sync(0xffffffffu, ko);
@@ -1321,11 +1348,20 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
           if (i + u < total) {
             const uint32_t p24 = kk8[u] >> 8;
             const uint32_t above = run & 0xFFFFu, equal = run >> 16;
+            // staged by output slot (a slot never exceeds its item's index, and
+            // this pass's reads are done), written out coalesced below
             if (p24 > T) {
-              emit(out, o_idx, b, above + min(equal, kk), pp8[u], kk8[u]);
+              const uint32_t sl = above + min(equal, kk);
+              if (sl < K) {
+                s.cpos[sl] = pp8[u];
+                s.ckey[sl] = kk8[u];
+              }
               run += 1u;
             } else if (p24 == T) {
-              if (equal < kk) emit(out, o_idx, b, above + equal, pp8[u], kk8[u]);
+              if (equal < kk && above + equal < K) {
+                s.cpos[above + equal] = pp8[u];
+                s.ckey[above + equal] = kk8[u];
+              }
               run += 0x10000u;
             }
           }
@@ -1356,12 +1392,17 @@ split_topk_kernel(RowWorkspace w, int rows_per_batch, int t0, int Tq, int Tk, in
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           if (sel[u]) {
-            if (o < K) emit(out, o_idx, b, o, pp4[u], kk4[u]);   // exactly K are chosen
+            if (o < K) {   // exactly K are chosen; staged by slot as in 2a
+              s.cpos[o] = pp4[u];
+              s.ckey[o] = kk4[u];
+            }
             ++o;
           }
         base += tot;
       }
     }
+    __syncthreads();
+    emit_staged(out, o_idx, b, s.cpos, s.ckey, K, tid, kSplitThreads);
   }
   finish_tail(out, b, t, Tq, k, K, failed, tid, kSplitThreads);
 
