@@ -98,8 +98,13 @@ def load_peaks():
 # ------------------------------------------------------------ ncu traffic
 #
 # DRAM bytes (read + write) per launch of a workload's roofline kernel(s),
-# from one ncu capture.  Each entry holds the hash of the library sources it
-# was taken on; when any source has changed since, the bench reports null.
+# from one `ncu --set full --clock-control none` capture on one B200: "attn"
+# one decode attention call (split + merge) or one prefill attention layer,
+# "index" one indexer run (scorer + split top-k), "route" one gist routing
+# call.  The decode captures ran the workload with one layer (--layers 1:
+# the per-call shapes are the workload's); prefill took the first attention
+# launch.  NCU_SOURCES is the hash of the library sources they were taken
+# on: once any source changes, the bench reports null.
 
 CSRC = os.path.join(ROOT, "shared_top_routing_b200", "csrc")
 
@@ -113,14 +118,26 @@ def sources_sha16() -> str:
     return h.hexdigest()[:16]
 
 
-NCU_TRAFFIC: dict = {}
+NCU_SOURCES = "67b889b323250e48"
+NCU_TRAFFIC: dict = {
+    "decode_b8_32k_4layers": {"attn": 70990080, "index": 69245440},
+    "decode_1m_28layers": {"attn": 6152704, "index": 143977472},
+    "decode_b8_32k_4layers_idx16heads": {"attn": 71118592, "index": 68971008},
+    "yoco_decode_b8_32k_4layers_one_cache": {"attn": 71278080},
+    "gist_decode_b4_128k": {"attn": 20435200, "route": 8747520},
+    "hgist_decode_b4_128k_meta16": {"attn": 20434944, "route": 727040},
+    "prefill_64k_4layers_needles": {"attn": 2805648904},
+    "prefill_2k_1layer": {"attn": 7254272},
+}
 
 
-def traffic_for(workload: str):
+def traffic_for(workload: str, kind: str):
+    """DRAM bytes per launch of the workload's roofline kernel(s) of `kind`,
+    or None when the library sources changed since the capture."""
     e = NCU_TRAFFIC.get(workload)
-    if e is None or e["sources_sha16"] != sources_sha16():
+    if e is None or kind not in e or NCU_SOURCES != sources_sha16():
         return None
-    return e["bytes"]
+    return e[kind]
 
 
 # ------------------------------------------------------------ CUDA runtime
@@ -658,7 +675,8 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
                 "bound": "hbm", "achieved": _r(idx_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": _frac(idx_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": score_run,
                 "launch_ms": _r(idx_ms, 5)}
-    roof["traffic"] = args.traffic if (args.traffic is not None and headline) else traffic_for(cfg.name)
+    kind = "attn" if attn_total >= idx_total else "index"
+    roof["traffic"] = args.traffic if (args.traffic is not None and headline) else traffic_for(cfg.name, kind)
     roof["peak_source"] = peaks["source"]
     resident = b.kv_all.numel() * 2 + sum(t.numel() * 2 for t in b.inp["k_idx"].values())
     line = {
@@ -869,7 +887,7 @@ def measure_prefill(ctx: Ctx, cfg: R.Prefill, steps: int, warmup: int):
                      "tensor": {"achieved_TFLOPs": round(attn_tf, 2), "peak": peaks["bf16_tflops"],
                                 "frac": _frac(attn_tf, peaks["bf16_tflops"]), "flops_per_launch": attn_flops},
                      "algorithmic_bytes_per_launch": gathered, "launch_ms": round(attn_ms, 4),
-                     "traffic": traffic_for(cfg.name), "peak_source": peaks["source"]},
+                     "traffic": traffic_for(cfg.name, "attn"), "peak_source": peaks["source"]},
         "indexer": {"kernel": "score_prefill_tc_kernel passes + prefill_threshold_kernel + finish_kernel "
                               "(one indexer run)",
                     "bound": "tensor", "ms_per_run": round(idx_ms, 4), "runs_per_step": cfg.n_groups,
@@ -1066,7 +1084,8 @@ def measure_gist(ctx: Ctx, cfg: R.Gist, steps: int, warmup: int):
                 "achieved": round(route_gbs, 1), "algorithmic_bytes_per_launch": route_bytes,
                 "launch_ms": round(route_ms, 5)}
     roof.update({"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                 "frac": _frac(roof["achieved"], peaks["hbm_gbs"]), "traffic": traffic_for(cfg.name),
+                 "frac": _frac(roof["achieved"], peaks["hbm_gbs"]),
+                 "traffic": traffic_for(cfg.name, "attn" if attn_ms >= route_ms else "route"),
                  "peak_source": peaks["source"]})
     resident = sum(gb.inp[x].numel() * 2 for x in ("K", "V", "gist_key"))
     line = {
