@@ -71,6 +71,7 @@ def job_rate(world: int, units_per_rank: float, ms: float) -> float:
 CONFIGS = {
     "decode_32k": R.DECODE_32K,
     "decode_32k_mh": R.DECODE_32K_MH16,
+    "decode_32k_mh_fp8": R.DECODE_32K_MH16_FP8,
     "yoco_32k": R.YOCO_32K,
     "hgist": R.HGIST_128K,
     "decode_1m": R.DECODE_1M,
@@ -79,7 +80,8 @@ CONFIGS = {
     "prefill_64k": R.PREFILL_64K,
 }
 # workloads reported under "workloads" beside the headline, in run order
-SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "hgist", "decode_1m", "decode_32k_mh", "yoco_32k")
+SUB_WORKLOADS = ("prefill_2k", "prefill_64k", "gist", "hgist", "decode_1m", "decode_32k_mh", "decode_32k_mh_fp8",
+                 "yoco_32k")
 
 
 def load_peaks():
@@ -103,22 +105,30 @@ def load_peaks():
 # "index" one indexer run (scorer + split top-k), "route" one gist routing
 # call.  The decode captures ran the workload with one layer (--layers 1:
 # the per-call shapes are the workload's); prefill took the first attention
-# launch.  NCU_SOURCES is the hash of the library sources they were taken
-# on: once any source changes, the bench reports null.
+# launch.  NCU_SOURCES holds, per kind, the hash of the source files its
+# kernels are built from at the capture: once one of them changes, the bench
+# reports null.
 
 CSRC = os.path.join(ROOT, "shared_top_routing_b200", "csrc")
+KIND_SOURCES = {
+    "attn": ("attn.cu", "sa_common.cuh", "tc_common.cuh"),
+    "index": ("index_topk.cu", "sa_common.cuh", "tc_common.cuh"),
+    "route": ("index_topk.cu", "sa_common.cuh", "tc_common.cuh"),
+}
 
 
-def sources_sha16() -> str:
+def sources_sha16(files=None) -> str:
+    """Hash of the named library source files (all of them by default)."""
+    if files is None:
+        files = [n for n in os.listdir(CSRC) if n.endswith((".cu", ".cuh", ".h"))]
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(files):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-NCU_SOURCES = "67b889b323250e48"
+NCU_SOURCES = {"attn": "b1422ee3c289212e", "index": "6e816b3d3471a6e3", "route": "6e816b3d3471a6e3"}
 NCU_TRAFFIC: dict = {
     "decode_b8_32k_4layers": {"attn": 70990080, "index": 69245440},
     "decode_1m_28layers": {"attn": 6152704, "index": 143977472},
@@ -135,7 +145,7 @@ def traffic_for(workload: str, kind: str):
     """DRAM bytes per launch of the workload's roofline kernel(s) of `kind`,
     or None when the library sources changed since the capture."""
     e = NCU_TRAFFIC.get(workload)
-    if e is None or kind not in e or NCU_SOURCES != sources_sha16():
+    if e is None or kind not in e or NCU_SOURCES[kind] != sources_sha16(KIND_SOURCES[kind]):
         return None
     return e[kind]
 
@@ -400,8 +410,12 @@ class DecodeBench:
             self.v_rows = torch.empty_like(self.k_rows)
         self.cache = sa.IndexCache(c.n_layers, c.B, 1, c.k, share_every=c.share_every, device=device)
         L = sa.lib()
-        ws_idx = (L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k) if c.H_idx == 1 else
-                  L.sa_index_score_topk_mh_workspace(c.B, 1, c.Tk_max, c.H_idx, c.d, c.k))
+        if c.fp8_idx:
+            ws_idx = L.sa_index_score_topk_fp8_workspace(c.B, c.Tk_max, c.H_idx, c.d, c.k)
+        elif c.H_idx == 1:
+            ws_idx = L.sa_index_score_topk_workspace(c.B, 1, c.Tk_max, c.d, c.k)
+        else:
+            ws_idx = L.sa_index_score_topk_mh_workspace(c.B, 1, c.Tk_max, c.H_idx, c.d, c.k)
         self.ws_idx = torch.zeros(ws_idx, dtype=torch.uint8, device=device)
         self.ws_attn = torch.zeros(max(256, L.sa_sparse_attn_decode_workspace(c.B, c.Hq, c.Hkv, c.D, c.k)),
                                    dtype=torch.uint8, device=device)
@@ -421,7 +435,16 @@ class DecodeBench:
                 if ev is not None:
                     ev[("idx", layer, 0)].record()
                 qi = q_idx[g] if q_idx is not None else self.inp["q_idx"][g][s]
-                if c.H_idx == 1:
+                if c.fp8_idx:
+                    # the fp8 indexer writes the group's buffers itself
+                    wi = None
+                    if c.H_idx > 1:
+                        wi = w_idx[g] if w_idx is not None else self.inp["w_idx"][g][s]
+                    sa.sa_index_score_topk_fp8(qi, self.inp["k_idx"][g], c.k, w=wi, Tk=Tk, q_pos0=Tk - 1,
+                                               idx_out=self.cache.idx_buf.view(c.B, c.k),
+                                               count_out=self.cache.count_buf.view(c.B), ws=self.ws_idx)
+                    self.cache.mark_written(layer)
+                elif c.H_idx == 1:
                     self.cache.update(layer, qi, self.inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=self.ws_idx)
                 else:
                     # the multi-head indexer writes the group's buffers itself
@@ -514,7 +537,8 @@ class DecodeBench:
         kept rows, queries, outputs and indices)."""
         c = self.cfg
         Tk = c.N + 1
-        score_run = c.B * Tk * c.d * 2 + c.B * c.H_idx * c.d * 2
+        eb = 1 if c.fp8_idx else 2   # bytes per indexer element
+        score_run = c.B * Tk * c.d * eb + c.B * c.H_idx * c.d * eb
         attn_one = c.B * c.k * c.Hkv * c.D * 2 * 2 + c.B * c.Hq * c.D * 2 * 2 + c.B * c.k * 4
         return score_run, attn_one
 
@@ -574,7 +598,8 @@ def decode_e2e(b: DecodeBench, ctx: Ctx, steps: int, warmup: int):
         h = host[s]
         pos = c.N + s
         for g in h["q_idx"]:
-            rt.h2d(qi_dev[g].data_ptr(), h["q_idx"][g].data_ptr(), h["q_idx"][g].numel() * 2, st)
+            rt.h2d(qi_dev[g].data_ptr(), h["q_idx"][g].data_ptr(),
+                   h["q_idx"][g].numel() * h["q_idx"][g].element_size(), st)
             if g in wi_dev:
                 rt.h2d(wi_dev[g].data_ptr(), h["w_idx"][g].data_ptr(), h["w_idx"][g].numel() * 4, st)
             row_copy(b.inp["k_idx"][g], h["k_row"][g], pos, B)
@@ -670,7 +695,8 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
                 "frac": _frac(attn_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": attn_bytes,
                 "launch_ms": _r(attn_ms, 5)}
     else:
-        roof = {"kernel": ("score_mh_kernel" if cfg.H_idx > 1 else "score_decode_kernel")
+        roof = {"kernel": ("score_fp8_kernel" if cfg.fp8_idx else
+                           "score_mh_kernel" if cfg.H_idx > 1 else "score_decode_kernel")
                           + " + split_topk_kernel (one indexer run)",
                 "bound": "hbm", "achieved": _r(idx_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": _frac(idx_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": score_run,
@@ -678,14 +704,16 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
     kind = "attn" if attn_total >= idx_total else "index"
     roof["traffic"] = args.traffic if (args.traffic is not None and headline) else traffic_for(cfg.name, kind)
     roof["peak_source"] = peaks["source"]
-    resident = b.kv_all.numel() * 2 + sum(t.numel() * 2 for t in b.inp["k_idx"].values())
+    resident = b.kv_all.numel() * 2 + sum(t.numel() * t.element_size() for t in b.inp["k_idx"].values())
     line = {
         "metric": "decode steps/s", "value": round(value, 2), "unit": "steps/s", "n_gpus": ctx.world,
         "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (indexer e4m3)" if cfg.fp8_idx else "bf16",
         "data": "synthetic (seeded counter-hash generator; integer indexer inputs, Irwin-Hall normal K/V/q)",
         "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.N, "layers": cfg.n_layers,
-                   "share_every": cfg.share_every, "d_idx": cfg.d, "indexer_heads": cfg.H_idx, "q_heads": cfg.Hq,
+                   "share_every": cfg.share_every, "d_idx": cfg.d, "indexer_heads": cfg.H_idx,
+                   "indexer_dtype": "e4m3" if cfg.fp8_idx else "bf16", "q_heads": cfg.Hq,
                    "kv_heads": cfg.Hkv, "head_dim": cfg.D, "top_k": cfg.k,
                    "parallelism": f"replicas{ctx.world}",
                    "l2": _l2_note(step_bytes, resident, False),
@@ -1166,8 +1194,10 @@ class OracleDecode:
         bl = list(batches)
         for g in groups:
             if bench is not None:
-                self.k_idx[g] = _bits(bench.inp["k_idx"][g][bl])
-                self.q_idx[g] = _bits(bench.inp["q_idx"][g][step][bl])
+                # bf16 bit patterns, or E4M3 codes (uint8) for an fp8 indexer
+                raw = (lambda t: t.contiguous().cpu().numpy()) if cfg.fp8_idx else _bits
+                self.k_idx[g] = raw(bench.inp["k_idx"][g][bl])
+                self.q_idx[g] = raw(bench.inp["q_idx"][g][step][bl])
                 if cfg.H_idx > 1:
                     self.w_idx[g] = bench.inp["w_idx"][g][step][bl].cpu().numpy()
             else:
@@ -1175,6 +1205,9 @@ class OracleDecode:
                 self.k_idx[g] = ch.int_bf16(cfg.seed, R.tid(R.KIND_K_IDX, g), count=n) \
                     .reshape(cfg.B, cfg.Tk_max, cfg.d)[bl]
                 self.q_idx[g] = R.decode_q_idx_host(cfg, g, step)[bl]
+                if cfg.fp8_idx:
+                    to8 = lambda bits: ch.e4m3_codes(ch.bf16_bits_to_f64(bits))
+                    self.k_idx[g], self.q_idx[g] = to8(self.k_idx[g]), to8(self.q_idx[g])
                 if cfg.H_idx > 1:
                     self.w_idx[g] = R.decode_w_idx_host(cfg, g, step)[bl]
         sel = {g: self._topk(g) for g in groups}

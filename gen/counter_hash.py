@@ -97,6 +97,34 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """Values exactly representable in OCP FP8 E4M3 -> their codes (uint8):
+    sign bit, 4-bit exponent field with bias 7 (0 for subnormals, steps of
+    2^-9), 3-bit mantissa.  Zero is +0.  Raises for values E4M3 cannot hold
+    exactly."""
+    v = np.asarray(x, dtype=np.float64)
+    a = np.abs(v)
+    out = np.zeros(v.shape, dtype=np.uint8)
+    nz = a > 0
+    e = np.floor(np.log2(np.where(nz, a, 1.0))).astype(np.int64)
+    normal = nz & (e >= -6)
+    m_norm = (a / np.exp2(e.astype(np.float64)) - 1.0) * 8.0
+    m_sub = a / 2.0 ** -9
+    m = np.where(normal, m_norm, m_sub)
+    ok = ~nz | ((m == np.round(m)) & np.where(normal, (e <= 8) & (m <= 7) & ~((e == 8) & (m == 7)), m <= 7))
+    if not ok.all():
+        raise ValueError("values not exactly representable in E4M3")
+    field = np.where(normal, e + 7, 0)
+    code = (np.where(v < 0, 0x80, 0) | (field << 3) | np.round(m).astype(np.int64)).astype(np.uint8)
+    return np.where(nz, code, 0).astype(np.uint8)
+
+
+def int_e4m3(seed: int, tid: int, start: int = 0, count: int | None = None,
+             index: np.ndarray | None = None, lo: int = -4, hi: int = 4) -> np.ndarray:
+    """The integer values of int_bf16 (same stream), as E4M3 codes."""
+    return e4m3_codes(int_values(seed, tid, start, count, index, lo, hi))
+
+
 def int_bf16(seed: int, tid: int, start: int = 0, count: int | None = None,
              index: np.ndarray | None = None, lo: int = -4, hi: int = 4) -> np.ndarray:
     """Integer values stored as bfloat16 bits (exact for |v| <= 256)."""

@@ -78,6 +78,7 @@ class Decode:
     steps: int
     H_idx: int = 1          # indexer heads (> 1: the multi-head weighted indexer)
     shared_kv: bool = False  # one K/V cache for every layer (YOCO); the rows are gathered once per step
+    fp8_idx: bool = False   # indexer queries and keys stored as E4M3 codes (the same integer values)
 
     @property
     def Tk_max(self) -> int:
@@ -141,6 +142,11 @@ YOCO_32K = Decode("yoco_decode_b8_32k_4layers_one_cache", seed=7, B=8, N=32768, 
 # (512 meta keys), the top 8 groups' 128 chunks compete for the 64 unfolded.
 HGIST_128K = Gist("hgist_decode_b4_128k_meta16", seed=8, B=4, n_chunks=8192, chunk_len=16, d=128, k_chunks=64,
                   Hq=32, Hkv=8, D=128, steps=16, group_size=16, k_groups=8)
+
+# The 16-head decode step with the indexer's queries and keys stored as fp8
+# (E4M3): the integer values of the bf16 workload in half the bytes.
+DECODE_32K_MH16_FP8 = Decode("decode_b8_32k_4layers_idx16heads_fp8", seed=9, B=8, N=32768, d=128, Hq=32, Hkv=8,
+                             D=128, k=2048, n_layers=4, share_every=4, steps=64, H_idx=16, fp8_idx=True)
 
 ALL = [PREFILL_2K, DECODE_32K, PREFILL_64K, GIST_128K, DECODE_1M]
 

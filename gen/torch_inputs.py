@@ -23,6 +23,11 @@ def dev_normal(shape, seed: int, tid: int, device, start: int = 0):
     return gd.fill_normal(t, seed, tid, start)
 
 
+def to_e4m3(t):
+    """A bfloat16 tensor of values exact in E4M3 -> their E4M3 codes (uint8)."""
+    return t.float().to(torch.float8_e4m3fn).view(torch.uint8)
+
+
 def from_host_bits(bits: np.ndarray, device):
     """Host bf16 bit patterns -> device bfloat16 tensor."""
     a = np.ascontiguousarray(bits).view(np.int16)
@@ -49,6 +54,11 @@ def decode_inputs(cfg: R.Decode, device, layers=None, groups=None):
             wb = torch.empty((cfg.steps, cfg.B, cfg.H_idx), dtype=torch.bfloat16, device=device)
             gd.fill_int(wb, s, R.tid(R.KIND_W_IDX, g), 0, lo=-3, hi=3)
             out["w_idx"][g] = wb.float()
+    if cfg.fp8_idx:
+        # the same integer values as E4M3 codes (exact: |v| <= 4)
+        for name in ("k_idx", "q_idx"):
+            for g in out[name]:
+                out[name][g] = to_e4m3(out[name][g])
     for l in layers:
         if cfg.shared_kv and l > 0 and 0 in out["K"]:   # one cache for every layer
             out["K"][l], out["V"][l] = out["K"][0], out["V"][0]

@@ -145,6 +145,37 @@ sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* 
                                  void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fp8 indexer, decode (one query per sequence; no counterpart in the pages,
+ * which name only a light indexer: an extension for an indexer cache stored
+ * in 8 bits, half the bytes the decode scorer streams).
+ *
+ * q_idx and k_idx hold OCP FP8 E4M3 bytes (1 sign, 4 exponent bits with bias
+ * 7, 3 mantissa bits; no infinities; S.1111.111 is NaN).  Products are exact
+ * and accumulate in fp32, so integer-valued inputs give exact scores.
+ *   w == NULL (then H must be 1): s = q_idx[b,0,:] . k_idx[b,j,:], the
+ *     one-head score of sa_index_score_topk;
+ *   w != NULL: s = sum_h w[b,h] * max(0, q_idx[b,h,:] . k_idx[b,j,:]), the
+ *     multi-head score of sa_index_score_topk_mh.
+ * The query of sequence b sits at position q_pos0; its candidates are
+ * j <= q_pos0, j < kv_len[b].  Selection, tie rule, output order, score_out
+ * and the error word are exactly as for sa_index_score_topk with Tq = 1.
+ *
+ *   q_idx  [B, H, d] e4m3 bytes (16-byte aligned);  w [B, H] fp32 or NULL
+ *   k_idx  [B, Tk_max, d] e4m3 bytes (16-byte aligned)
+ *   kv_len [B] int32 or NULL;  idx_out [B, k] int32;  count_out [B] int32
+ *   score_out [B, k] fp32 or NULL
+ *   ws     >= sa_index_score_topk_fp8_workspace(...) bytes (zero-filled
+ *          before first use; see the conventions above)
+ * Supported: d in {64, 128}; 1 <= H <= 32; 1 <= k <= SA_MAX_K.
+ * ---------------------------------------------------------------------- */
+size_t sa_index_score_topk_fp8_workspace(int B, int Tk_max, int H, int d, int k);
+sa_status sa_index_score_topk_fp8(const void* q_idx, const float* w, const void* k_idx,
+                                  int B, int H, int Tk, int Tk_max, int d, int k,
+                                  int q_pos0, const int32_t* kv_len,
+                                  int32_t* idx_out, int32_t* count_out, float* score_out,
+                                  void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Gathered sparse attention, prefill (one call per layer).
  *
  * [YOIO] §1.1: Attention(Q,K,V) = softmax(QK^T/sqrt(d_k))V; §2.3: each
@@ -382,7 +413,7 @@ sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_ful
  *     violation (0 none, 1 prefill attention index, 2 decode attention index,
  *     3 gathered-rows index, 4 workspace canary), its first detail (the index;
  *     for a canary the call: 1 index top-k, 2 multi-head top-k, 3 decode
- *     attention, 4 gist routing), its second detail (Tk_max; for a canary the
+ *     attention, 4 gist routing, 5 fp8 top-k), its second detail (Tk_max; for a canary the
  *     first changed byte), number of violations}; reset != 0 clears it.
  *     Synchronous; the release build reports zeros.
  * ---------------------------------------------------------------------- */

@@ -13,6 +13,7 @@ than itself live in ``tests/test_oracle_pins.py``.
 """
 from .reference import (  # noqa: F401
     bf16_bits_to_f64,
+    e4m3_bits_to_f64,
     n_candidates,
     index_scores,
     index_scores_multihead,

@@ -46,6 +46,11 @@ Readings where the pages are silent (each also stated where it is used):
    calibration loss; here the loss of sharing is stood in for by the index
    overlap itself (1 - overlap of a layer's own selection with the one it
    would reuse), the greedy removal order being the page's.
+10. fp8 indexer inputs (an extension: the pages do not give the indexer's
+    number format) are OCP FP8 E4M3 codes: 1 sign bit, 4 exponent bits with
+    bias 7, 3 mantissa bits, subnormals at exponent field 0, no infinities,
+    S.1111.111 is NaN.  A score is the exact dot product of the decoded
+    values, as for bf16 inputs.
 """
 from __future__ import annotations
 
@@ -60,10 +65,28 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def e4m3_bits_to_f64(codes) -> np.ndarray:
+    """OCP FP8 E4M3 codes (uint8) -> float64, exactly (reading 10):
+    exponent field e and mantissa field m give (-1)^s (1 + m/8) 2^(e-7) for
+    e > 0, (-1)^s (m/8) 2^-6 for e = 0, and NaN for e = 15, m = 7."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0)
+    subnormal = (m / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, subnormal, normal)
+    return np.where((e == 15) & ((c & 0x7) == 7), np.nan, v)
+
+
 def _f64(x) -> np.ndarray:
+    """Inputs as float64: uint16 arrays are bf16 bit patterns, uint8 arrays
+    E4M3 codes, anything else is taken as values."""
     x = np.asarray(x)
     if x.dtype == np.uint16:
         return bf16_bits_to_f64(x)
+    if x.dtype == np.uint8:
+        return e4m3_bits_to_f64(x)
     return x.astype(np.float64)
 
 

@@ -23,7 +23,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
-SOURCES = ["abi.cu", "attn.cu", "index_topk.cu", "index_tc.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["abi.cu", "attn.cu", "index_topk.cu", "index_tc.cu", "index_fp8.cu", "noalloc.cu", "selftest.cu"]
 
 
 def _run(cmd, verbose):

@@ -332,6 +332,50 @@ sa_status sa_index_score_topk_mh(const void* q_idx, const float* w, const void* 
   return ok();
 }
 
+size_t sa_index_score_topk_fp8_workspace(int B, int Tk_max, int H, int d, int k) {
+  (void)H;
+  return sa_index_score_topk_workspace(B, 1, Tk_max, d, k);
+}
+
+sa_status sa_index_score_topk_fp8(const void* q_idx, const float* w, const void* k_idx, int B, int H, int Tk,
+                                  int Tk_max, int d, int k, int q_pos0, const int32_t* kv_len, int32_t* idx_out,
+                                  int32_t* count_out, float* score_out, void* ws, size_t ws_bytes,
+                                  sa_stream_t stream) {
+  sa_status st = validate_index(q_idx, k_idx, B, 1, Tk, Tk_max, d, k, idx_out, count_out);
+  if (st != SA_OK) return st;
+  if (H < 1) return fail(SA_ERR_INVALID_ARG, "H=%d must be >= 1", H);
+  if (w == nullptr && H != 1) return fail(SA_ERR_INVALID_ARG, "H=%d heads need weights (w is NULL)", H);
+  if (H > sa::kFp8MaxHeads) return fail(SA_ERR_UNSUPPORTED, "H=%d indexer heads exceed %d", H, sa::kFp8MaxHeads);
+  if (B == 0) return ok();
+  if (w != nullptr && !aligned(w, 4)) return fail(SA_ERR_INVALID_ARG, "w must be 4-byte aligned");
+  const size_t need = sa_index_score_topk_fp8_workspace(B, Tk_max, H, d, k);
+  if ((st = check_ws(ws, ws_bytes, need)) != SA_OK) return st;
+  cudaStream_t cs = as_cuda(stream);
+  cudaError_t e;
+  if ((e = sa::dbg_arm(ws, need - sa::kWsCanary, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
+  const int mode = sa::finish_mode_for(Tk_max);
+  sa::RowWorkspace wsp;
+  sa::carve_row_workspace(ws, B, Tk_max, mode == sa::kFinishSplit, mode != sa::kFinishDirect, &wsp);
+  const bool hist = mode != sa::kFinishDirect;
+  if (hist && wsp.hist_zero_bytes && (e = cudaMemsetAsync(wsp.hist, 0, wsp.hist_zero_bytes, cs)) != cudaSuccess)
+    return cuda_fail(e, "memset");
+  if ((e = sa::launch_score_fp8(static_cast<const uint8_t*>(q_idx), w, static_cast<const uint8_t*>(k_idx), B, H, d,
+                                Tk_max, Tk, q_pos0, kv_len, wsp, hist, cs)) != cudaSuccess)
+    return cuda_fail(e, "fp8 score launch");
+  sa::FinishOut out;
+  out.idx = idx_out;
+  out.count = count_out;
+  out.score = score_out;
+  if (mode == sa::kFinishSplit) {
+    if ((e = sa::launch_split_topk(B, 1, 0, 1, Tk, q_pos0, kv_len, k, wsp, out, cs)) != cudaSuccess)
+      return cuda_fail(e, "split top-k launch");
+  } else if ((e = sa::launch_finish(B, 1, 0, 1, Tk, q_pos0, kv_len, k, wsp, mode, out, cs)) != cudaSuccess) {
+    return cuda_fail(e, "finish launch");
+  }
+  if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 5, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
+  return ok();
+}
+
 // ----------------------------------------------------------- attention
 
 sa_status sa_sparse_attn_prefill(const void* q, const void* k_cache, const void* v_cache,

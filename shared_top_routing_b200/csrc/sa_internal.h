@@ -156,6 +156,14 @@ cudaError_t launch_hier_gist(const uint16_t* q_route, const uint16_t* meta_key, 
 // Per-row shared positions of two ascending selections.
 cudaError_t launch_index_overlap(const int32_t* a, const int32_t* ca, const int32_t* b, const int32_t* cb, int rows,
                                  int k, int32_t* out, cudaStream_t st);
+// fp8 (e4m3) indexer scoring of one-query rows (index_fp8.cu): wts == null
+// is the one-head dot product (H == 1), otherwise sum_h w_h * ReLU(q_h . k)
+// over H <= kFp8MaxHeads heads.  Keys and the first-digit histogram go to the
+// row workspace as for launch_score_decode.
+constexpr int kFp8MaxHeads = 32;
+cudaError_t launch_score_fp8(const uint8_t* q, const float* wts, const uint8_t* kmat, int B, int H, int d, int Tk_max,
+                             int Tk, int q_pos0, const int32_t* kv_len, const RowWorkspace& w, bool with_hist,
+                             cudaStream_t st);
 // Largest number of indexer heads of the multi-head indexer for key width d.
 constexpr int mh_max_heads(int d) { return d == 64 ? 64 : 32; }
 // Prefill scoring of queries [t0, t0+rows) (tcgen05, index_tc.cu); `epi`

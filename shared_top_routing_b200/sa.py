@@ -40,6 +40,8 @@ SIGNATURES = {
     "sa_index_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_index_score_topk_mh_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_index_score_topk_mh": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "sa_index_score_topk_fp8_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "sa_index_score_topk_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "sa_sparse_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _Z, _P]),
@@ -260,6 +262,46 @@ def sa_index_score_topk_mh(q_idx, w, k_idx, k: int, Tk: int | None = None, q_pos
     if decode_shape:
         idx_v, cnt_v = idx_out.view(B, k), count_out.view(B)
         return (idx_v, cnt_v, score.view(B, k)) if with_scores else (idx_v, cnt_v)
+    return (idx_out, count_out, score) if with_scores else (idx_out, count_out)
+
+
+def sa_index_score_topk_fp8(q_idx, k_idx, k: int, w=None, Tk: int | None = None, q_pos0: int | None = None,
+                            kv_len=None, idx_out=None, count_out=None, with_scores: bool = False,
+                            ws=None, stream=None):
+    """fp8 (E4M3) indexer scores + top-k of one decode query per sequence
+    (see sa.h).
+
+    q_idx [B, d] (one head) or [B, H, d]; k_idx [B, Tk_max, d]: E4M3 codes as
+    uint8 (or torch.float8_e4m3fn) tensors.  w [B, H] fp32 selects the
+    multi-head score; without it H must be 1.  Tk defaults to Tk_max, q_pos0
+    to Tk - 1.  Returns (idx [B, k] int32, count [B] int32[, score [B, k]]).
+    """
+    torch = _torch()
+    as_bytes = lambda t: t.view(torch.uint8) if t.dtype != torch.uint8 else t
+    q3 = as_bytes(q_idx)
+    q3 = q3.unsqueeze(1) if q3.dim() == 2 else q3
+    kb = as_bytes(k_idx)
+    B, H, d = q3.shape
+    Tk_max = kb.shape[1]
+    Tk = Tk_max if Tk is None else Tk
+    q_pos0 = Tk - 1 if q_pos0 is None else q_pos0
+    _need(q3, "q_idx", 1)
+    _need(kb, "k_idx", 1)
+    if w is not None:
+        _need(w, "w", 4)
+    dev = q3.device
+    if idx_out is None:
+        idx_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((B,), dtype=torch.int32, device=dev)
+    score = torch.empty((B, k), dtype=torch.float32, device=dev) if with_scores else None
+    need = lib().sa_index_score_topk_fp8_workspace(B, Tk_max, H, d, k)
+    if ws is None:
+        ws = workspace(need, dev, "index", stream)
+    st = lib().sa_index_score_topk_fp8(_ptr(q3), _ptr(w), _ptr(kb), B, H, Tk, Tk_max, d, k, q_pos0, _ptr(kv_len),
+                                       _ptr(idx_out), _ptr(count_out), _ptr(score), _ptr(ws),
+                                       0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "sa_index_score_topk_fp8")
     return (idx_out, count_out, score) if with_scores else (idx_out, count_out)
 
 

@@ -74,6 +74,33 @@ def test_index_topk_validation():
     assert _topk(B=0) == S.SA_OK                                # nothing to do, no launch
 
 
+def _fp8(**kw):
+    a = dict(q=FAKE, w=None, k=FAKE, B=1, H=1, Tk=10, Tk_max=10, d=64, kk=4, q_pos0=9, kv_len=None, idx=FAKE,
+             cnt=FAKE, score=None, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return S.lib().sa_index_score_topk_fp8(a["q"], a["w"], a["k"], a["B"], a["H"], a["Tk"], a["Tk_max"], a["d"],
+                                           a["kk"], a["q_pos0"], a["kv_len"], a["idx"], a["cnt"], a["score"],
+                                           a["ws"], a["ws_bytes"], None)
+
+
+def test_fp8_index_topk_validation():
+    """The fp8 indexer checks its arguments on the host, before any launch."""
+    assert _fp8(H=2) == S.SA_ERR_INVALID_ARG                    # several heads need weights
+    assert "weights" in S.last_error()
+    assert _fp8(H=0) == S.SA_ERR_INVALID_ARG
+    assert _fp8(H=33, w=FAKE) == S.SA_ERR_UNSUPPORTED
+    assert _fp8(d=96) == S.SA_ERR_UNSUPPORTED
+    assert _fp8(Tk=11) == S.SA_ERR_INVALID_ARG
+    assert _fp8(kk=S.SA_MAX_K + 1) == S.SA_ERR_UNSUPPORTED
+    assert _fp8(k=ctypes.c_void_p(0x100008)) == S.SA_ERR_INVALID_ARG   # misaligned keys
+    assert _fp8(H=4, w=ctypes.c_void_p(0x100002)) == S.SA_ERR_INVALID_ARG   # misaligned weights
+    assert _fp8(ws=FAKE, ws_bytes=16) == S.SA_ERR_WORKSPACE
+    assert _fp8(B=0) == S.SA_OK
+    L = S.lib()
+    assert L.sa_index_score_topk_fp8_workspace(8, 32832, 16, 128, 2048) == \
+        L.sa_index_score_topk_workspace(8, 1, 32832, 128, 2048)
+
+
 def test_workspace_sizes():
     L = S.lib()
     small = L.sa_index_score_topk_workspace(8, 1, 4096, 128, 2048)

@@ -1,6 +1,7 @@
 """Host generator checks (CPU): published SplitMix64 outputs, distributions,
 random access, recipes."""
 import numpy as np
+import pytest
 
 from gen import counter_hash as ch
 from gen import recipes
@@ -61,3 +62,17 @@ def test_recipe_sizes():
     assert kv_bytes / 2 ** 30 == 56.0
     assert recipes.GIST_128K.rows_cap == 64 * 17 + 16
     assert recipes.GIST_128K.Tk_max == 8192 * 17 + 16
+
+
+def test_e4m3_codes_of_integers_and_rejections():
+    """Integers in [-4, 4] have the E4M3 codes the format gives them (sign
+    bit, exponent field e + 7, mantissa of |v| / 2^e - 1 in eighths); values
+    E4M3 cannot hold exactly are rejected; the integer stream in E4M3 is the
+    bf16 stream's values."""
+    codes = ch.e4m3_codes(np.arange(-4, 5))
+    assert [int(c) for c in codes] == [0xC8, 0xC4, 0xC0, 0xB8, 0x00, 0x38, 0x40, 0x44, 0x48]
+    for bad in (4.25, 1000.0, 2.0 ** -10, 1.0625):
+        with pytest.raises(ValueError):
+            ch.e4m3_codes(np.array([bad]))
+    ints = ch.int_values(5, 77, count=4096)
+    np.testing.assert_array_equal(ch.int_e4m3(5, 77, count=4096), ch.e4m3_codes(ints))

@@ -307,6 +307,96 @@ def test_multihead_topk_ties_and_bad_arguments():
                                     fake, 1 << 30, None) == sa.SA_ERR_INVALID_ARG
 
 
+# ------------------------------------------------------------- fp8 indexer
+
+def _e4m3(seed, tid, shape, lo=-4, hi=4):
+    return ch.int_e4m3(seed, tid, count=int(np.prod(shape)), lo=lo, hi=hi).reshape(shape)
+
+
+def _u8(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).to(dev())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,k,lens,Tk_max", [
+    (1, 256, [3000, 1, 0, 257], 3000),          # direct selection, ragged, empty row
+    (1, 2048, [16385, 30000, 2047, 40000], 40000),   # split selection
+    (1, 7, [9999, 5000, 7, 6], 10007),          # n <= k rows
+    (4, 512, [9000, 4096, 4097, 1], 9000),      # multi-head, both sides of the split threshold
+    (16, 2048, [33000, 20000], 33000),          # the 16-head workload's shape
+    (32, 100, [5000, 3000, 4100], 5000),        # two head groups
+])
+def test_fp8_decode_topk_matches_oracle(d, H, k, lens, Tk_max):
+    """fp8 (E4M3) queries and keys: indices, counts and scores bit-exact
+    against the oracle on the same codes, and equal to the bf16 path's
+    selection of the same integers."""
+    B = len(lens)
+    seed = 5000 + d + 7 * H + k
+    q8 = _e4m3(seed, 1, (B, H, d))
+    k8 = _e4m3(seed, 2, (B, Tk_max, d))
+    w = _ints(seed, 3, (B, H), lo=-3, hi=3) if H > 1 else None
+    wf = oracle.bf16_bits_to_f64(w).astype(np.float32) if w is not None else None
+    wt = torch.from_numpy(wf).to(dev()) if w is not None else None
+    idx, cnt, sc = sa.sa_index_score_topk_fp8(_u8(q8), _u8(k8), k, w=wt, Tk=max(lens), q_pos0=10 ** 9,
+                                              kv_len=i32(lens), with_scores=True)
+    if H == 1:
+        ridx, rcnt = oracle.index_topk(q8[:, :, :].reshape(B, 1, d), k8, np.array(lens), 10 ** 9, k)
+    else:
+        ridx, rcnt = oracle.index_topk(q8[:, None], k8, np.array(lens), 10 ** 9, k, w=wf[:, None])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0])
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
+    sc = sc.cpu().numpy()
+    for b in range(B):
+        n = rcnt[b, 0]
+        if n:
+            rows = k8[b, ridx[b, 0, :n]]
+            if H == 1:
+                full = oracle.index_scores(q8[b, :1], rows)[0]
+            else:
+                full = oracle.index_scores_multihead(q8[b][None], wf[b][None], rows)[0]
+            np.testing.assert_array_equal(sc[b, :n], full)
+        assert np.all(np.isneginf(sc[b, n:]))
+    # the same integers through the bf16 indexer choose the same positions
+    qb = oracle.e4m3_bits_to_f64(q8)
+    kb = ch.f32_to_bf16_bits(oracle.e4m3_bits_to_f64(k8))
+    if H == 1:
+        bidx, bcnt = sa.sa_index_score_topk(to_dev(ch.f32_to_bf16_bits(qb[:, 0])), to_dev(kb), k, Tk=max(lens),
+                                            q_pos0=10 ** 9, kv_len=i32(lens))
+    else:
+        bidx, bcnt = sa.sa_index_score_topk_mh(to_dev(ch.f32_to_bf16_bits(qb)), wt, to_dev(kb), k, Tk=max(lens),
+                                               q_pos0=10 ** 9, kv_len=i32(lens))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bidx.cpu().numpy(), idx.cpu().numpy())
+    np.testing.assert_array_equal(bcnt.cpu().numpy(), cnt.cpu().numpy())
+
+
+def test_fp8_decode_topk_heavy_ties_and_float8_tensors():
+    """A one-hot query gives 9 distinct scores, so the boundary is a huge tie
+    group decided by position; torch.float8_e4m3fn tensors are accepted as
+    they are."""
+    d, n, k = 128, 40000, 3000
+    q = np.zeros((2, d))
+    q[0, 5] = 1.0
+    q[1, 100] = -2.0
+    k8 = _e4m3(91, 2, (2, n, d))
+    q8 = ch.e4m3_codes(q)
+    idx, cnt = sa.sa_index_score_topk_fp8(_u8(q8).view(torch.float8_e4m3fn), _u8(k8).view(torch.float8_e4m3fn), k)
+    ridx, rcnt = oracle.index_topk(q8[:, None, :], k8, n, n - 1, k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt[:, 0])
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx[:, 0])
+
+
+def test_fp8_device_codes_match_the_host_generator():
+    """The device inputs of the fp8 workload (the bf16 integer tensors
+    converted on the device) are the host generator's E4M3 codes."""
+    from gen import torch_inputs as TI
+    t = TI.dev_int((4, 1000, 64), 13, 7, dev())
+    got = TI.to_e4m3(t).cpu().numpy()
+    np.testing.assert_array_equal(got, _e4m3(13, 7, (4, 1000, 64)))
+
+
 def _random_index(rng, B, Tk_max, k, counts):
     idx = np.full((B, k), -1, np.int32)
     for b, c in enumerate(counts):

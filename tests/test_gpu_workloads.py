@@ -31,11 +31,16 @@ def _check_decode(cfg, steps, check_groups, check_layers):
     inp = TI.decode_inputs(cfg, d)
     cache = sa.IndexCache(cfg.n_layers, cfg.B, 1, cfg.k, share_every=cfg.share_every, device=d)
     L = sa.lib()
-    ws_bytes = (L.sa_index_score_topk_workspace(cfg.B, 1, cfg.Tk_max, cfg.d, cfg.k) if cfg.H_idx == 1 else
-                L.sa_index_score_topk_mh_workspace(cfg.B, 1, cfg.Tk_max, cfg.H_idx, cfg.d, cfg.k))
+    if cfg.fp8_idx:
+        ws_bytes = L.sa_index_score_topk_fp8_workspace(cfg.B, cfg.Tk_max, cfg.H_idx, cfg.d, cfg.k)
+    elif cfg.H_idx == 1:
+        ws_bytes = L.sa_index_score_topk_workspace(cfg.B, 1, cfg.Tk_max, cfg.d, cfg.k)
+    else:
+        ws_bytes = L.sa_index_score_topk_mh_workspace(cfg.B, 1, cfg.Tk_max, cfg.H_idx, cfg.d, cfg.k)
     ws_idx = torch.zeros(ws_bytes, dtype=torch.uint8, device=d)
     outs = [torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device=d) for _ in range(cfg.n_layers)]
-    host_k = {g: ch.int_bf16(cfg.seed, R.tid(R.KIND_K_IDX, g), count=cfg.B * cfg.Tk_max * cfg.d)
+    host_int = ch.int_e4m3 if cfg.fp8_idx else ch.int_bf16   # E4M3 codes or bf16 bits of the same integers
+    host_k = {g: host_int(cfg.seed, R.tid(R.KIND_K_IDX, g), count=cfg.B * cfg.Tk_max * cfg.d)
               .reshape(cfg.B, cfg.Tk_max, cfg.d) for g in check_groups}
     for s in steps:
         # run the whole step, snapshotting each group's index right after its layers
@@ -46,7 +51,13 @@ def _check_decode(cfg, steps, check_groups, check_layers):
         for layer in range(cfg.n_layers):
             g = layer // cfg.share_every
             if cache.is_full(layer) == 1:
-                if cfg.H_idx == 1:
+                if cfg.fp8_idx:
+                    wi = inp["w_idx"][g][s] if cfg.H_idx > 1 else None
+                    sa.sa_index_score_topk_fp8(inp["q_idx"][g][s], inp["k_idx"][g], cfg.k, w=wi, Tk=Tk, q_pos0=Tk - 1,
+                                               idx_out=cache.idx_buf.view(cfg.B, cfg.k),
+                                               count_out=cache.count_buf.view(cfg.B), ws=ws_idx)
+                    cache.mark_written(layer)
+                elif cfg.H_idx == 1:
                     cache.update(layer, inp["q_idx"][g][s], inp["k_idx"][g], Tk=Tk, q_pos0=Tk - 1, ws=ws_idx)
                 else:
                     sa.sa_index_score_topk_mh(inp["q_idx"][g][s], inp["w_idx"][g][s], inp["k_idx"][g], cfg.k,
@@ -72,6 +83,8 @@ def _check_decode(cfg, steps, check_groups, check_layers):
         torch.cuda.synchronize()
         for g in check_groups:
             qi = R.decode_q_idx_host(cfg, g, s)
+            if cfg.fp8_idx:
+                qi = ch.e4m3_codes(ch.bf16_bits_to_f64(qi))
             wi = R.decode_w_idx_host(cfg, g, s)[:, None] if cfg.H_idx > 1 else None
             ridx, rcnt = oracle.index_topk(qi[:, None], host_k[g], Tk, Tk - 1, cfg.k, w=wi)
             gi, gc = got_idx[g]
@@ -114,6 +127,13 @@ def test_decode_32k_batch8_sixteen_head_indexer():
     """The batch-8 decode step with the 16-head weighted indexer (the bench's
     multi-head workload): indices bit-exact, two layers' attention checked."""
     _check_decode(R.DECODE_32K_MH16, steps=[0, 63], check_groups=[0], check_layers=[0, 3])
+
+
+def test_decode_32k_batch8_sixteen_head_fp8_indexer():
+    """The 16-head decode step with the indexer's queries and keys in E4M3
+    (the bench's fp8 workload): indices bit-exact against the oracle on the
+    same codes, one layer's attention checked."""
+    _check_decode(R.DECODE_32K_MH16_FP8, steps=[0, 63], check_groups=[0], check_layers=[0])
 
 
 # ---------------------------------------------------------------- prefill

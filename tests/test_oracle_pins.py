@@ -659,3 +659,65 @@ def test_greedy_pattern_is_exhaustive_optimum_when_one_indexer_is_removed():
     best = max(sum(ov[l, oracle.layer_owners(L, "".join("S" if i == r else "F" for i in range(L)))[l]]
                    for l in range(L)) for r in range(1, L))
     assert abs(got - best) < 1e-12
+
+
+# ------------------------------------------------------------ fp8 (E4M3) inputs
+
+def test_e4m3_decoder_format_values():
+    """The E4M3 decoder (reading 10) against values the OCP FP8 format fixes:
+    1.0 is exponent field 7 with a zero mantissa, the largest finite value is
+    448 (field 15, mantissa 6), the smallest normal 2^-6, the smallest
+    subnormal 2^-9, S.1111.111 is NaN, and there are no infinities."""
+    dec = lambda c: float(oracle.e4m3_bits_to_f64(np.array([c], dtype=np.uint8))[0])
+    assert dec(0x00) == 0.0 and dec(0x80) == 0.0 and math.copysign(1.0, dec(0x80)) == -1.0
+    for code, value in [(0x38, 1.0), (0xB8, -1.0), (0x40, 2.0), (0x44, 3.0), (0x48, 4.0), (0xC8, -4.0),
+                        (0x3C, 1.5), (0x7E, 448.0), (0xFE, -448.0), (0x08, 2.0 ** -6), (0x01, 2.0 ** -9),
+                        (0x07, 7 * 2.0 ** -9), (0x0F, 1.875 * 2.0 ** -6), (0x77, 240.0), (0x78, 256.0)]:
+        assert dec(code) == value, hex(code)
+    assert math.isnan(dec(0x7F)) and math.isnan(dec(0xFF))
+    vals = oracle.e4m3_bits_to_f64(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(vals) > 0), "positive codes must decode in increasing order"
+    assert not np.isinf(oracle.e4m3_bits_to_f64(np.arange(256, dtype=np.uint8))).any()
+    neg = oracle.e4m3_bits_to_f64(np.arange(0x80, 0xFF, dtype=np.uint8))
+    np.testing.assert_array_equal(neg, -vals)
+
+
+def test_e4m3_pin_catches_slips(monkeypatch):
+    """A decoder with the exponent bias off by one, or subnormals scaled as
+    normals, fails the format pin."""
+    real = oracle.e4m3_bits_to_f64
+
+    def bias8(codes):
+        return real(codes) / 2.0
+
+    def no_subnormal(codes):
+        c = np.asarray(codes, dtype=np.uint8)
+        v = real(c)
+        sub = ((c >> 3) & 0xF) == 0
+        return np.where(sub, np.where(c & 0x80, -1.0, 1.0) * (1 + (c & 7) / 8.0) * 2.0 ** -6 * (c & 7 > 0), v)
+
+    for mutant in (bias8, no_subnormal):
+        monkeypatch.setattr(oracle, "e4m3_bits_to_f64", mutant)
+        with pytest.raises(AssertionError):
+            test_e4m3_decoder_format_values()
+    monkeypatch.setattr(oracle, "e4m3_bits_to_f64", real)
+
+
+def test_fp8_inputs_select_as_the_same_integers_in_bf16():
+    """Integer values in [-4, 4] are exact in E4M3, so the top-k of their
+    E4M3 codes equals the top-k of their bf16 bits, one head and several."""
+    rng = _rng(41)
+    B, Tk, d, k = 3, 70, 64, 9
+    q = rng.integers(-4, 5, size=(B, 1, d))
+    kk = rng.integers(-4, 5, size=(B, Tk, d))
+    lens = np.array([70, 33, 5])
+    a = oracle.index_topk(ch.e4m3_codes(q), ch.e4m3_codes(kk), lens, Tk - 1, k)
+    b = oracle.index_topk(_bf16(q), _bf16(kk), lens, Tk - 1, k)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    H = 6
+    qh = rng.integers(-4, 5, size=(B, 1, H, d))
+    w = rng.integers(-3, 4, size=(B, 1, H)).astype(np.float32)
+    a = oracle.index_topk(ch.e4m3_codes(qh), ch.e4m3_codes(kk), Tk, Tk - 1, k, w=w)
+    b = oracle.index_topk(_bf16(qh), _bf16(kk), Tk, Tk - 1, k, w=w)
+    np.testing.assert_array_equal(a[0], b[0])
