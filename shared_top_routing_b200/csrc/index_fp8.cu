@@ -185,27 +185,25 @@ cudaError_t launch_score_fp8(const uint8_t* q, const float* wts, const uint8_t* 
   if (B <= 0 || Tk <= 0) return cudaSuccess;
   const long long n_max = std::min<long long>(Tk, (long long)q_pos0 + 1);
   if (n_max <= 0) return cudaSuccess;
-  // chunks of a multiple of 256 keys: about four CTAs per SM over all rows
-  const long long target = std::max<long long>(1, 4LL * device_sm_count() / B);
-  long long chunk = (n_max + target - 1) / target;
-  chunk = std::max<long long>(256, (chunk + 255) / 256 * 256);
-  const dim3 grid((unsigned)((n_max + chunk - 1) / chunk), (unsigned)B);
+  using Kern = void (*)(const uint8_t*, const float*, const uint8_t*, int, int, int, int, const int32_t*, int,
+                        uint32_t*, long long, uint32_t*);
   const bool weighted = wts != nullptr;
   const int hg = (H + 15) / 16;
-  cudaError_t e;
-#define SA_F8_LAUNCH(DD, GG, WW)                                                                              \
-  e = launch_pdl(score_fp8_kernel<DD, GG, WW>, grid, dim3(kF8Threads), 0, st, q, wts, kmat, H, Tk_max, Tk, q_pos0, \
-                 kv_len, (int)chunk, w.keys, w.ld, hist)
-  if (d == 128) {
-    if (!weighted) SA_F8_LAUNCH(128, 1, false);
-    else if (hg == 1) SA_F8_LAUNCH(128, 1, true);
-    else SA_F8_LAUNCH(128, 2, true);
-  } else {
-    if (!weighted) SA_F8_LAUNCH(64, 1, false);
-    else if (hg == 1) SA_F8_LAUNCH(64, 1, true);
-    else SA_F8_LAUNCH(64, 2, true);
-  }
-#undef SA_F8_LAUNCH
+  Kern kern;
+  if (d == 128)
+    kern = !weighted ? score_fp8_kernel<128, 1, false>
+                     : (hg == 1 ? score_fp8_kernel<128, 1, true> : score_fp8_kernel<128, 2, true>);
+  else
+    kern = !weighted ? score_fp8_kernel<64, 1, false>
+                     : (hg == 1 ? score_fp8_kernel<64, 1, true> : score_fp8_kernel<64, 2, true>);
+  // one wave of resident CTAs over all rows, each CTA's chunk a whole number
+  // of 128-row steps of its eight warps
+  const long long slots = (long long)device_sm_count() * std::max(1, device_occupancy((const void*)kern, kF8Threads, 0));
+  long long chunk = (n_max * B + slots - 1) / slots;
+  chunk = std::max<long long>(128, (chunk + 127) / 128 * 128);
+  const dim3 grid((unsigned)((n_max + chunk - 1) / chunk), (unsigned)B);
+  const cudaError_t e = launch_pdl(kern, grid, dim3(kF8Threads), 0, st, q, wts, kmat, H, Tk_max, Tk, q_pos0, kv_len,
+                                   (int)chunk, w.keys, w.ld, hist);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
