@@ -114,6 +114,7 @@ KIND_SOURCES = {
     "attn": ("attn.cu", "sa_common.cuh", "tc_common.cuh"),
     "index": ("index_topk.cu", "sa_common.cuh", "tc_common.cuh"),
     "route": ("index_topk.cu", "sa_common.cuh", "tc_common.cuh"),
+    "index_fp8": ("index_fp8.cu", "index_topk.cu", "sa_common.cuh", "tc_common.cuh"),
 }
 
 
@@ -128,7 +129,8 @@ def sources_sha16(files=None) -> str:
     return h.hexdigest()[:16]
 
 
-NCU_SOURCES = {"attn": "b1422ee3c289212e", "index": "6e816b3d3471a6e3", "route": "6e816b3d3471a6e3"}
+NCU_SOURCES = {"attn": "b1422ee3c289212e", "index": "6e816b3d3471a6e3", "route": "6e816b3d3471a6e3",
+               "index_fp8": "25a53375bc345ef4"}
 NCU_TRAFFIC: dict = {
     "decode_b8_32k_4layers": {"attn": 70990080, "index": 69245440},
     "decode_1m_28layers": {"attn": 6152704, "index": 143977472},
@@ -138,6 +140,7 @@ NCU_TRAFFIC: dict = {
     "hgist_decode_b4_128k_meta16": {"attn": 20434944, "route": 727040},
     "prefill_64k_4layers_needles": {"attn": 2805648904},
     "prefill_2k_1layer": {"attn": 7254272},
+    "decode_b8_32k_4layers_idx16heads_fp8": {"attn": 71000832, "index_fp8": 34981888},
 }
 
 
@@ -701,7 +704,7 @@ def measure_decode(ctx: Ctx, cfg: R.Decode, steps: int, warmup: int, headline: b
                 "bound": "hbm", "achieved": _r(idx_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": _frac(idx_gbs, peaks["hbm_gbs"]), "algorithmic_bytes_per_launch": score_run,
                 "launch_ms": _r(idx_ms, 5)}
-    kind = "attn" if attn_total >= idx_total else "index"
+    kind = "attn" if attn_total >= idx_total else ("index_fp8" if cfg.fp8_idx else "index")
     roof["traffic"] = args.traffic if (args.traffic is not None and headline) else traffic_for(cfg.name, kind)
     roof["peak_source"] = peaks["source"]
     resident = b.kv_all.numel() * 2 + sum(t.numel() * t.element_size() for t in b.inp["k_idx"].values())
