@@ -129,18 +129,18 @@ def sources_sha16(files=None) -> str:
     return h.hexdigest()[:16]
 
 
-NCU_SOURCES = {"attn": "b1422ee3c289212e", "index": "6e816b3d3471a6e3", "route": "6e816b3d3471a6e3",
-               "index_fp8": "25a53375bc345ef4"}
+NCU_SOURCES = {"attn": "b1422ee3c289212e", "index": "220203bc23977917", "route": "220203bc23977917",
+               "index_fp8": "2e72ef0fb2a9d60f"}
 NCU_TRAFFIC: dict = {
-    "decode_b8_32k_4layers": {"attn": 70990080, "index": 69245440},
-    "decode_1m_28layers": {"attn": 6152704, "index": 143977472},
-    "decode_b8_32k_4layers_idx16heads": {"attn": 71118592, "index": 68971008},
+    "decode_b8_32k_4layers": {"attn": 70906624, "index": 69190656},
+    "decode_1m_28layers": {"attn": 6152704, "index": 144029952},
+    "decode_b8_32k_4layers_idx16heads": {"attn": 70926592, "index": 68858880},
     "yoco_decode_b8_32k_4layers_one_cache": {"attn": 71278080},
-    "gist_decode_b4_128k": {"attn": 20435200, "route": 8747520},
-    "hgist_decode_b4_128k_meta16": {"attn": 20434944, "route": 727040},
+    "gist_decode_b4_128k": {"attn": 20434944, "route": 8747264},
+    "hgist_decode_b4_128k_meta16": {"attn": 20435200, "route": 727296},
     "prefill_64k_4layers_needles": {"attn": 2805648904},
     "prefill_2k_1layer": {"attn": 7254272},
-    "decode_b8_32k_4layers_idx16heads_fp8": {"attn": 71000832, "index_fp8": 34981888},
+    "decode_b8_32k_4layers_idx16heads_fp8": {"attn": 70881024, "index_fp8": 34980864},
 }
 
 

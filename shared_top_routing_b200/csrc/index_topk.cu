@@ -84,7 +84,7 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
   pdl_wait();
   pdl_launch_dependents();
   constexpr int J = D / 32;          // 16-byte chunks per lane per key row
-  constexpr int U = 2;               // 8-row tiles per register buffer (two buffers)
+  constexpr int U = 2;               // 8-row tiles per warp and load
   constexpr int WARPS = kScoreThreads / 32;
   __shared__ uint32_t sh[kHistBins];
 
@@ -184,14 +184,14 @@ score_decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__
 // weights (one row per decode sequence, or per prefill query) against the
 // key cache of their sequence.  The key cache is streamed as in
 // score_decode_kernel (16-byte loads straight into mma.sync B fragments;
-// here two register buffers of 8-row tiles per warp); the 16-row A side holds 16 indexer
-// heads (rows g and g+8 of a lane's fragment are heads 16 hg + g and 16 hg
-// + g + 8 of head group hg), so one m16n8k16 per 16 dimensions scores every
-// head of a group at once.  The epilogue takes weight x ReLU per head and
-// sums over heads with three shuffles; integer-valued inputs keep every
-// partial sum an exact fp32 integer.  Grid: (key chunks, rows); each CTA
-// scores one chunk of one row, writes the keys and adds its 4096-bin
-// histogram of their top 12 bits to the row's.
+// here two register buffers of 8-row tiles per warp); the 16-row A side
+// holds 16 indexer heads (rows g and g+8 of a lane's fragment are heads
+// 16 hg + g and 16 hg + g + 8 of head group hg), so one m16n8k16 per 16
+// dimensions scores every head of a group at once.  The epilogue takes
+// weight x ReLU per head and sums over heads with three shuffles;
+// integer-valued inputs keep every partial sum an exact fp32 integer.
+// Grid: (key chunks, rows); each CTA scores one chunk of one row, writes the
+// keys and adds its 4096-bin histogram of their top 12 bits to the row's.
 
 template <int D, int HG>
 __global__ void __launch_bounds__(kScoreThreads)
