@@ -8,17 +8,22 @@ the group plus the gathered sparse attention of all 4 layers for one new
 token of every sequence.  Metric: decode steps/s (whole job; weak scaling
 over GPUs, each rank runs its own 8 sequences).
 
-The same JSON line carries, under "workloads", the four other workloads of
-the path, each timed as CUDA-graph steps with its own roofline, CPU-oracle
-baseline and end-to-end figure:
-  prefill_2k_1layer            prefill tokens/s (L2 flushed between steps)
-  prefill_64k_4layers_needles  prefill tokens/s
-  gist_decode_b4_128k          decode steps/s (L2 flushed between steps)
-  decode_1m_28layers           decode steps/s
+The same JSON line carries, under "workloads", the other workloads of the
+path, each timed as CUDA-graph steps with its own roofline, clocks,
+CPU-oracle baseline and end-to-end figure:
+  prefill_2k_1layer                      prefill tokens/s (L2 flushed between steps)
+  prefill_64k_4layers_needles            prefill tokens/s
+  gist_decode_b4_128k                    decode steps/s (L2 flushed between steps)
+  hgist_decode_b4_128k_meta16            decode steps/s, two-level gist routing
+  decode_1m_28layers                     decode steps/s
+  decode_b8_32k_4layers_idx16heads       decode steps/s, 16-head weighted indexer
+  decode_b8_32k_4layers_idx16heads_fp8   the same with E4M3 indexer queries and keys
+  yoco_decode_b8_32k_4layers_one_cache   decode steps/s, one K/V cache gathered once
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--config decode_32k|decode_1m|gist|prefill_2k|prefill_64k]
-                    [--no-workloads]
+                    [--config decode_32k|decode_32k_mh|decode_32k_mh_fp8|yoco_32k|
+                              decode_1m|gist|hgist|prefill_2k|prefill_64k]
+                    [--no-workloads] [--layers L]
 
 Prints one JSON line (rank 0).  Inputs are synthetic and seeded (gen/); they
 are generated on the device before timing.
