@@ -1486,7 +1486,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode_32k")
     ap.add_argument("--no-workloads", action="store_true",
-                    help="headline only (skip the four other workloads)")
+                    help="headline only (skip the other workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only: run fewer layers (small profiling cases; not the headline)")
