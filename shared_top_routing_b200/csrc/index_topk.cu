@@ -356,7 +356,8 @@ struct FinishSmemT {
   uint32_t opos[MAXK];              // long rows: chosen items grouped by bucket
   uint32_t okey[MAXK];
 };
-// rows of any length (streamed scans, bucketed emission), 1024 threads
+// direct rows of more than 2048 candidates and candidate lists of rows over
+// 65536 positions (bucketed emission for long rows), 1024 threads
 using FinishSmem = FinishSmemT<kSmemCand, kBitmapWords, kMaxK>;
 // rows of at most 2048 candidates, 256 threads: several rows per SM
 using FinishSmemSmall = FinishSmemT<2048, 64, 1>;

@@ -45,3 +45,16 @@ def test_reference_arm_prints_the_contract_line():
     assert line["config"]["workload"] == "prefill_2k_1layer"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    a = "int f(int x) {  // doubles\n  return 2 * x; /* plain */\n}\n"
+    b = "int f(int x) {\n  // a longer, reflowed\n  // comment\n  return 2 * x;\n}\n"
+    c = "int f(int x) {  // doubles\n  return 3 * x;\n}\n"
+    for name, text in (("a.cu", a), ("b.cu", b), ("c.cu", c)):
+        (tmp_path / name).write_text(text)
+    monkeypatch.setattr(bench, "CSRC", str(tmp_path))
+    ha, hb, hc = (bench.sources_sha16([n]) for n in ("a.cu", "b.cu", "c.cu"))
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert ha != hc
