@@ -56,7 +56,7 @@ typedef enum {
   SA_ERR_UNSUPPORTED = 2,   /* valid but outside this build's shape support  */
   SA_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned    */
   SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed          */
-  SA_ERR_TIMEOUT = 5,       /* reserved (kernel waits report in the workspace) */
+  SA_ERR_TIMEOUT = 5,       /* a kernel wait gave up (read by sa_workspace_status) */
   SA_ERR_STALE_INDEX = 6    /* shared layer read before its full layer ran   */
 } sa_status;
 
@@ -397,6 +397,20 @@ sa_status sa_index_overlap(const int32_t* idx_a, const int32_t* count_a, const i
                            const int32_t* count_b, int rows, int k, int32_t* inter_out,
                            sa_stream_t stream);
 sa_status sa_index_pattern_greedy(const double* overlap, int n_layers, int n_full, char* pattern_out);
+
+/* ------------------------------------------------------------------------
+ * The error word of a workspace, read on the host.
+ *
+ * Waits for the work queued on `stream` so far (synchronizes it), then reads
+ * the kernel error word at the start of `ws`, the workspace of any call above
+ * that takes one (indexer top-k of every form, gist routing, decode
+ * attention).  Returns SA_OK when the word is zero and SA_ERR_TIMEOUT when a
+ * pipeline wait of a call that used the workspace gave up; sa_last_error()
+ * then names the wait's code.  The word is left as it is (zero-fill the
+ * workspace to use it again).  SA_ERR_INVALID_ARG for a NULL ws,
+ * SA_ERR_CUDA if the copy fails.
+ * ---------------------------------------------------------------------- */
+sa_status sa_workspace_status(const void* ws, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Debug builds (libsa_debug.so, compiled with SA_DEBUG; no counterpart in the

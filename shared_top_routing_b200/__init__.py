@@ -22,6 +22,7 @@ from .sa import (  # noqa: F401
     sa_index_score_topk,
     sa_index_score_topk_mh,
     sa_index_score_topk_fp8,
+    sa_workspace_status,
     sa_sparse_attn_decode,
     sa_sparse_attn_decode_rows,
     sa_sparse_attn_prefill,
@@ -45,6 +46,7 @@ __all__ = [
     "sa_index_score_topk",
     "sa_index_score_topk_mh",
     "sa_index_score_topk_fp8",
+    "sa_workspace_status",
     "sa_sparse_attn_decode",
     "sa_sparse_attn_decode_rows",
     "sa_sparse_attn_prefill",

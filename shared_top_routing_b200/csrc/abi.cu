@@ -181,7 +181,7 @@ const char* sa_status_string(sa_status s) {
     case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED: shape not supported by this build";
     case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case SA_ERR_CUDA: return "SA_ERR_CUDA: CUDA runtime or launch failure";
-    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT: reserved";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT: a kernel wait gave up";
     case SA_ERR_STALE_INDEX: return "SA_ERR_STALE_INDEX: shared layer read before its full layer wrote";
   }
   return "unknown sa_status";
@@ -373,6 +373,17 @@ sa_status sa_index_score_topk_fp8(const void* q_idx, const float* w, const void*
     return cuda_fail(e, "finish launch");
   }
   if ((e = sa::dbg_check(ws, need - sa::kWsCanary, 5, cs)) != cudaSuccess) return cuda_fail(e, "debug canary");
+  return ok();
+}
+
+sa_status sa_workspace_status(const void* ws, sa_stream_t stream) {
+  if (ws == nullptr) return fail(SA_ERR_INVALID_ARG, "NULL workspace");
+  cudaStream_t cs = as_cuda(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (word != 0) return fail(SA_ERR_TIMEOUT, "a pipeline wait gave up (wait code %d)", word);
   return ok();
 }
 

@@ -41,6 +41,7 @@ SIGNATURES = {
     "sa_index_score_topk_mh_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sa_index_score_topk_mh": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_index_score_topk_fp8_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "sa_workspace_status": (_I, [_P, _P]),
     "sa_index_score_topk_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "sa_sparse_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "sa_sparse_attn_decode_workspace": (_Z, [_I, _I, _I, _I, _I]),
@@ -303,6 +304,13 @@ def sa_index_score_topk_fp8(q_idx, k_idx, k: int, w=None, Tk: int | None = None,
                                        0 if ws is None else ws.numel(), _stream(stream))
     _check(st, "sa_index_score_topk_fp8")
     return (idx_out, count_out, score) if with_scores else (idx_out, count_out)
+
+
+def sa_workspace_status(ws, stream=None) -> int:
+    """The status the error word at the start of a workspace reports (see
+    sa.h): SA_OK, or SA_ERR_TIMEOUT when a kernel wait of a call that used it
+    gave up.  Synchronizes `stream`."""
+    return lib().sa_workspace_status(_ptr(ws), _stream(stream))
 
 
 def sa_sparse_attn_prefill(q, k_cache, v_cache, idx, count, scale: float = 0.0, out=None,

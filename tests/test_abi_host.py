@@ -101,6 +101,14 @@ def test_fp8_index_topk_validation():
         L.sa_index_score_topk_workspace(8, 1, 32832, 128, 2048)
 
 
+def test_workspace_status_validation():
+    """A NULL workspace is refused on the host; the timeout status has its
+    own string."""
+    assert S.lib().sa_workspace_status(None, None) == S.SA_ERR_INVALID_ARG
+    assert "workspace" in S.last_error()
+    assert "wait" in S.status_string(S.SA_ERR_TIMEOUT)
+
+
 def test_workspace_sizes():
     L = S.lib()
     small = L.sa_index_score_topk_workspace(8, 1, 4096, 128, 2048)

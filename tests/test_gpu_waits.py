@@ -67,11 +67,15 @@ def test_indexer_error_word_gives_the_sentinel(B, Tq, T, d, k):
         if code == 0:
             np.testing.assert_array_equal(cnt.cpu().numpy(), ref_cnt)
             np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+            assert sa.sa_workspace_status(ws) == sa.SA_OK
         else:
             assert (cnt.cpu().numpy() == 0).all()
             assert (idx.cpu().numpy() == -1).all()
             assert np.isneginf(sc.cpu().numpy()).all()
             assert ws[:4].view(torch.int32)[0].item() == code   # the word is left for the caller
+            # ... and the host reads it as a timed-out wait, naming the code
+            assert sa.sa_workspace_status(ws) == sa.SA_ERR_TIMEOUT
+            assert str(code) in sa.last_error()
 
 
 def test_gist_error_word_gives_the_sentinel():
@@ -92,3 +96,4 @@ def test_gist_error_word_gives_the_sentinel():
                 np.testing.assert_array_equal(rows[b, : rr.size], rr)
             else:
                 assert cnt[b] == 0 and (rows[b] == -1).all()
+        assert sa.sa_workspace_status(ws) == (sa.SA_OK if code == 0 else sa.SA_ERR_TIMEOUT)
