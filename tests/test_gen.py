@@ -76,3 +76,14 @@ def test_e4m3_codes_of_integers_and_rejections():
             ch.e4m3_codes(np.array([bad]))
     ints = ch.int_values(5, 77, count=4096)
     np.testing.assert_array_equal(ch.int_e4m3(5, 77, count=4096), ch.e4m3_codes(ints))
+
+
+def test_device_e4m3_conversion_matches_the_host_codes_on_cpu_tensors():
+    """The conversion the fp8 workload's device inputs take (torch's E4M3
+    cast of the integer bf16 tensor) gives the host generator's codes; the
+    same check runs on the GPU in the parity tests."""
+    import torch
+    from gen import torch_inputs as TI
+    bits = ch.int_bf16(13, 9, count=5000)
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    np.testing.assert_array_equal(TI.to_e4m3(t).numpy(), ch.int_e4m3(13, 9, count=5000))
